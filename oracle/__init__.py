@@ -1,0 +1,303 @@
+"""CPU oracle for the NVFP4 block-numerics hot path (TEST INFRASTRUCTURE).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  It wraps the plain C99 library built from
+the ``*.c`` files beside this file (FP64, exact comparisons) and shares nothing
+with the CUDA library: no code, headers, tables or constants, and it never
+imports the product package.
+
+Rows (or Hessian blocks) are fanned out over a thread pool; the C calls release
+the GIL, so the threads run in parallel.  Each function's definition and source
+page is documented in the C file that implements it.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+import subprocess
+import threading
+from concurrent.futures import ThreadPoolExecutor
+
+import numpy as np
+
+_DIR = os.path.dirname(os.path.abspath(__file__))
+_SOURCES = ["formats.c", "act.c", "hessian.c", "sweep.c", "cast.c"]
+_LIB_PATH = os.path.join(_DIR, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+BF16, F32 = 0, 2
+FLAG_NONFINITE, FLAG_E8M0_NAN, FLAG_OVERFLOW = 1, 2, 4
+
+
+def build(force: bool = False) -> str:
+    """Compile liboracle.so with gcc (no FMA contraction, no fast-math)."""
+    srcs = [os.path.join(_DIR, s) for s in _SOURCES]
+    hdr = os.path.join(_DIR, "nv4_oracle.h")
+    if not force and os.path.exists(_LIB_PATH):
+        newest = max(os.path.getmtime(p) for p in srcs + [hdr])
+        if os.path.getmtime(_LIB_PATH) >= newest:
+            return _LIB_PATH
+    tmp = _LIB_PATH + f".tmp{os.getpid()}"
+    cmd = ["gcc", "-O2", "-std=c11", "-Wall", "-Wextra", "-fPIC", "-shared",
+           "-ffp-contract=off", "-fno-fast-math", *srcs, "-lm", "-o", tmp]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _L():
+    global _lib
+    with _lock:
+        if _lib is None:
+            build()
+            lib = C.CDLL(_LIB_PATH)
+            vp, i64, u32p = C.c_void_p, C.c_int64, C.POINTER(C.c_uint32)
+            sig = {
+                "orc_e2m1_value": (C.c_double, [C.c_uint]),
+                "orc_e4m3_value": (C.c_double, [C.c_uint]),
+                "orc_e8m0_value": (C.c_double, [C.c_uint]),
+                "orc_e4m3_encode": (C.c_uint, [C.c_double, C.c_double]),
+                "orc_e2m1_encode": (C.c_uint, [C.c_double, C.c_double]),
+                "orc_s2_from_amax": (C.c_float, [C.c_float]),
+                "orc_bf16_value": (C.c_double, [C.c_uint16]),
+                "orc_f32_to_bf16": (C.c_uint16, [C.c_float]),
+                "orc_f32_to_f16": (C.c_uint16, [C.c_float]),
+                "orc_tensor_amax": (C.c_float, [vp, C.c_int, i64, u32p]),
+                "orc_act_quant": (C.c_float, [vp, i64, i64, i64, C.c_float, i64, i64, vp, vp, u32p]),
+                "orc_dequant": (None, [vp, vp, C.c_float, i64, i64, C.c_int, i64, i64, vp]),
+                "orc_hessian_accum": (None, [vp, i64, i64, i64, i64, i64, vp]),
+                "orc_scale_sweep": (None, [vp, C.c_int, i64, i64, i64, vp, C.c_float, i64, i64,
+                                           vp, vp, vp, vp, u32p]),
+                "orc_mx_kmax": (C.c_int, [vp, i64, u32p]),
+                "orc_mxfp4_to_nvfp4": (None, [vp, vp, i64, i64, C.c_int, i64, i64, vp, vp, vp]),
+                "orc_mx_global": (None, [C.c_int, C.POINTER(C.c_float), C.POINTER(C.c_float), u32p]),
+            }
+            for name, (res, args) in sig.items():
+                fn = getattr(lib, name)
+                fn.restype, fn.argtypes = res, args
+            _lib = lib
+    return _lib
+
+
+def default_threads() -> int:
+    return len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else (os.cpu_count() or 1)
+
+
+def _p(a: np.ndarray | None):
+    return None if a is None else a.ctypes.data_as(C.c_void_p)
+
+
+def _chunks(n: int, parts: int):
+    parts = max(1, min(parts, n))
+    step = -(-n // parts)
+    return [(i, min(n, i + step)) for i in range(0, n, step)]
+
+
+def _fanout(fn, n: int, threads: int | None):
+    threads = threads or default_threads()
+    ranges = _chunks(n, threads * 4)
+    if threads == 1 or len(ranges) == 1:
+        for r in ranges:
+            fn(*r)
+        return
+    with ThreadPoolExecutor(threads) as ex:
+        list(ex.map(lambda r: fn(*r), ranges))
+
+
+# ---------------------------------------------------------------- formats
+def e2m1_value(code: int) -> float:
+    return _L().orc_e2m1_value(code)
+
+
+def e4m3_value(code: int) -> float:
+    return _L().orc_e4m3_value(code)
+
+
+def e8m0_value(code: int) -> float:
+    return _L().orc_e8m0_value(code)
+
+
+def e4m3_encode(num: float, den: float) -> int:
+    return _L().orc_e4m3_encode(num, den)
+
+
+def e2m1_encode(x: float, S: float) -> int:
+    return _L().orc_e2m1_encode(x, S)
+
+
+def s2_from_amax(amax: float) -> float:
+    return _L().orc_s2_from_amax(amax)
+
+
+def f32_to_bf16(f: float) -> int:
+    return _L().orc_f32_to_bf16(f)
+
+
+def f32_to_f16(f: float) -> int:
+    return _L().orc_f32_to_f16(f)
+
+
+# ---------------------------------------------------------------- amax
+def tensor_amax(x: np.ndarray, threads: int | None = None):
+    """x: uint16 (bf16 bits) or float32, any shape (contiguous).  Returns (amax, flags)."""
+    x = np.ascontiguousarray(x)
+    dtype = F32 if x.dtype == np.float32 else BF16
+    assert x.dtype in (np.float32, np.uint16)
+    flat = x.reshape(-1)
+    n = flat.size
+    ranges = _chunks(n, (threads or default_threads()) * 4) if n else []
+    res = [None] * len(ranges)
+
+    def run(k):
+        lo, hi = ranges[k]
+        f = C.c_uint32(0)
+        a = _L().orc_tensor_amax(_p(flat[lo:hi]), dtype, hi - lo, C.byref(f))
+        res[k] = (a, f.value)
+
+    if len(ranges) > 1 and (threads or default_threads()) > 1:
+        with ThreadPoolExecutor(threads or default_threads()) as ex:
+            list(ex.map(run, range(len(ranges))))
+    else:
+        for k in range(len(ranges)):
+            run(k)
+    amax = max([r[0] for r in res], default=0.0)
+    flags = 0
+    for r in res:
+        flags |= r[1]
+    return float(np.float32(amax)), flags
+
+
+# ---------------------------------------------------------------- act quant / dequant
+def act_quant(x: np.ndarray, amax: float, cols: int | None = None, threads: int | None = None):
+    """x: uint16 bf16 bits [rows, ld].  Returns (q [rows, cols/2], scales [rows, cols/16], s2, flags)."""
+    assert x.dtype == np.uint16 and x.ndim == 2 and x.flags.c_contiguous
+    rows, ld = x.shape
+    cols = ld if cols is None else cols
+    assert cols % 16 == 0
+    q = np.zeros((rows, cols // 2), np.uint8)
+    sc = np.zeros((rows, cols // 16), np.uint8)
+    flags = [0]
+    s2 = [0.0]
+    lk = threading.Lock()
+
+    def run(r0, r1):
+        f = C.c_uint32(0)
+        s = _L().orc_act_quant(_p(x), rows, cols, ld, amax, r0, r1, _p(q), _p(sc), C.byref(f))
+        with lk:
+            flags[0] |= f.value
+            s2[0] = s
+
+    if rows == 0:
+        f = C.c_uint32(0)
+        s2[0] = _L().orc_act_quant(_p(x), 0, cols, ld, amax, 0, 0, _p(q), _p(sc), C.byref(f))
+    else:
+        _fanout(run, rows, threads)
+    return q, sc, float(np.float32(s2[0])), flags[0]
+
+
+def dequant(q: np.ndarray, scales: np.ndarray, s2: float, out_dtype: str = "bf16",
+            threads: int | None = None) -> np.ndarray:
+    """Returns uint16 bits (bf16/fp16) or float32 [rows, cols]."""
+    rows = q.shape[0]
+    cols = q.shape[1] * 2
+    code = {"bf16": 0, "fp16": 1, "fp32": 2}[out_dtype]
+    out = np.zeros((rows, cols), np.float32 if code == 2 else np.uint16)
+    q = np.ascontiguousarray(q)
+    scales = np.ascontiguousarray(scales)
+    _fanout(lambda r0, r1: _L().orc_dequant(_p(q), _p(scales), s2, rows, cols, code, r0, r1, _p(out)),
+            rows, threads)
+    return out
+
+
+# ---------------------------------------------------------------- Hessian
+def hessian_accum(x: np.ndarray, H: np.ndarray | None = None, cols: int | None = None,
+                  threads: int | None = None) -> np.ndarray:
+    """x: uint16 bf16 bits [tokens, ld]; returns H (float64 [cols/16, 16, 16]) += X_b^T X_b."""
+    assert x.dtype == np.uint16 and x.ndim == 2 and x.flags.c_contiguous
+    tokens, ld = x.shape
+    cols = ld if cols is None else cols
+    nblk = cols // 16
+    if H is None:
+        H = np.zeros((nblk, 16, 16), np.float64)
+    assert H.dtype == np.float64 and H.flags.c_contiguous and H.shape == (nblk, 16, 16)
+    _fanout(lambda b0, b1: _L().orc_hessian_accum(_p(x), tokens, cols, ld, b0, b1, _p(H)), nblk, threads)
+    return H
+
+
+# ---------------------------------------------------------------- sweep
+def scale_sweep(w: np.ndarray, H: np.ndarray, amax_w: float, rows=None, cols: int | None = None,
+                threads: int | None = None):
+    """w: float32 or uint16 (bf16 bits) [N, ld]; H: float64 [cols/16, 16, 16].
+
+    ``rows``: None for all rows, or an iterable of row indices (a sample); outputs
+    then hold the sampled rows in the given order.  Returns a dict with codes, q,
+    cost1, cost2 and flags.
+    """
+    assert w.ndim == 2 and w.flags.c_contiguous
+    dtype = F32 if w.dtype == np.float32 else BF16
+    assert w.dtype in (np.float32, np.uint16)
+    N, ld = w.shape
+    cols = ld if cols is None else cols
+    nblk = cols // 16
+    H = np.ascontiguousarray(H, dtype=np.float64)
+    assert H.shape == (nblk, 16, 16)
+    idx = np.arange(N) if rows is None else np.asarray(list(rows), dtype=np.int64)
+    n = len(idx)
+    codes = np.zeros((n, nblk), np.uint8)
+    q = np.zeros((n, cols // 2), np.uint8)
+    c1 = np.zeros((n, nblk), np.float64)
+    c2 = np.zeros((n, nblk), np.float64)
+    flags = [0]
+    lk = threading.Lock()
+    es = w.itemsize
+
+    def run(k0, k1):
+        f = C.c_uint32(0)
+        for k in range(k0, k1):
+            r = int(idx[k])
+            wp = C.c_void_p(w.ctypes.data + r * ld * es)
+            _L().orc_scale_sweep(wp, dtype, 1, cols, ld, _p(H), amax_w, 0, 1,
+                                 _p(codes[k]), _p(q[k]), _p(c1[k]), _p(c2[k]), C.byref(f))
+        with lk:
+            flags[0] |= f.value
+
+    if n:
+        _fanout(run, n, threads)
+    return {"codes": codes, "q": q, "cost1": c1, "cost2": c2, "flags": flags[0], "rows": idx}
+
+
+# ---------------------------------------------------------------- MXFP4 -> NVFP4
+def mxfp4_to_nvfp4(mx_q: np.ndarray, e8m0: np.ndarray, threads: int | None = None):
+    """One matrix: mx_q uint8 [rows, cols/2], e8m0 uint8 [rows, cols/32].
+
+    Raises ValueError on an E8M0 NaN code.  Returns a dict with nv_q, nv_scales, s2,
+    global_amax, k_max, counts (in-window, fallback, lossless 16-blocks) and flags.
+    """
+    mx_q = np.ascontiguousarray(mx_q)
+    e8m0 = np.ascontiguousarray(e8m0)
+    rows, half = mx_q.shape
+    cols = 2 * half
+    assert cols % 32 == 0 and e8m0.shape == (rows, cols // 32)
+    f = C.c_uint32(0)
+    kmax = _L().orc_mx_kmax(_p(e8m0), e8m0.size, C.byref(f))
+    if f.value & FLAG_E8M0_NAN:
+        raise ValueError("E8M0 NaN code 0xFF in the input")
+    s2 = C.c_float(0)
+    ga = C.c_float(0)
+    _L().orc_mx_global(kmax, C.byref(s2), C.byref(ga), C.byref(f))
+    nv_q = np.zeros_like(mx_q)
+    nv_s = np.zeros((rows, cols // 16), np.uint8)
+    parts = []
+    lk = threading.Lock()
+
+    def run(r0, r1):
+        cnt = np.zeros(3, np.int64)
+        _L().orc_mxfp4_to_nvfp4(_p(mx_q), _p(e8m0), rows, cols, kmax, r0, r1, _p(nv_q), _p(nv_s), _p(cnt))
+        with lk:
+            parts.append(cnt)
+
+    _fanout(run, rows, threads)
+    counts = np.sum(parts, axis=0) if parts else np.zeros(3, np.int64)
+    return {"nv_q": nv_q, "nv_scales": nv_s, "s2": s2.value, "global_amax": ga.value,
+            "k_max": kmax, "counts": counts, "flags": f.value}

@@ -1,0 +1,247 @@
+/*
+ * nv4.h -- C ABI of libnv4.so, a B200 (sm_100a) NVFP4 block-numerics engine.
+ *
+ * NVFP4 stores 16-element blocks of E2M1 (FP4) values, each block with one E4M3
+ * scale, plus one FP32 second-level scale per tensor.  The library implements
+ * the data-parallel hot path of Hessian-weighted NVFP4 post-training
+ * quantization as described on these pages (cited by title and section):
+ *
+ *  [CAL]    "Coder390 NVFP4 calibration method", section 2: max calibration, local
+ *           Hessian H = sum X^T X per 16 input channels, Hessian-weighted E4M3 scale
+ *           sweep (fp8_scale_sweep); format line: E2M1, 16-element blocks, E4M3 block
+ *           scale, FP32 second-level scale.
+ *  [FLOW]   "NVFP4 quantization and export flow" (Gemma-2B decoder), sections 3.4-3.6:
+ *           per-tensor scale amax/6/448, dynamic activation quantize, DQ1/DQ2;
+ *           section 5.4: two FP4 values per byte.
+ *  [CAST]   "From MXFP4 to NVFP4: Model Optimizer mixed-precision format conversion",
+ *           section 2: closed-form cast, global_amax = 6*448*2^(k_max-8), window 17.
+ *  [DSPARK] "From calibration to export: the DSpark three-stage NVFP4 recipe", stage 3:
+ *           nibbles reused, scale bytes double.
+ *  [FP4]    "FP4 quantization overview", sections 1.1-1.2: E2M1 values, MXFP4 vs NVFP4.
+ *
+ * Conventions for every entry point
+ *  - The caller owns all memory.  The library allocates nothing: no device memory,
+ *    no host memory that outlives a call.
+ *  - Pointers named d_* and all tensor pointers are DEVICE pointers.  Job arrays
+ *    of the *_batched calls are HOST arrays, read during the call only.
+ *  - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL = legacy
+ *    default stream).  No call synchronizes the host.  Device scalars (amax, s2)
+ *    travel by device pointer, so a chain of calls needs no host round trip.
+ *  - The return status covers argument validation and launch errors.  Data-dependent
+ *    conditions are OR-ed into the caller's flag word *d_flags (device, uint32,
+ *    zeroed by the caller; may be NULL to ignore them).  Kernels never trap.
+ *  - Layouts are row-major.  `ld` is a leading dimension in elements.  A 16-element
+ *    block b of a row covers columns 16b..16b+15.  Packed FP4: byte i of a row holds
+ *    element 2i in bits 0-3 and element 2i+1 in bits 4-7; an E2M1 code is
+ *    sign(bit 3) | exponent(bits 2-1) | mantissa(bit 0).  Block scales are raw E4M3
+ *    (fn) bytes, [rows, cols/16].
+ *  - Alignment: tensor pointers 16-byte aligned and ld*element_size a multiple of
+ *    16 bytes, else NV4_ERR_ALIGN (there is no slower unaligned path).
+ *  - Calls on different streams that write the same buffers race; the library adds
+ *    no ordering of its own.
+ */
+#ifndef NV4_H
+#define NV4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define NV4_API __attribute__((visibility("default")))
+#else
+#define NV4_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    NV4_OK = 0,
+    NV4_ERR_NULL = 1,    /* a required pointer is NULL                               */
+    NV4_ERR_SHAPE = 2,   /* negative size, cols % 16 != 0 (% 32 for MXFP4), ld < cols */
+    NV4_ERR_ALIGN = 3,   /* pointer or ld*element_size not a multiple of 16 bytes    */
+    NV4_ERR_DTYPE = 4,   /* element type not supported by this entry point           */
+    NV4_ERR_CUDA = 5,    /* a CUDA runtime call or kernel launch failed              */
+    NV4_ERR_LIMIT = 6    /* a size exceeds what one call supports (see the call)     */
+} nv4_status;
+
+typedef enum { NV4_BF16 = 0, NV4_FP16 = 1, NV4_FP32 = 2 } nv4_dtype;
+
+/* data-dependent flags OR-ed into *d_flags */
+#define NV4_FLAG_NONFINITE 1u  /* a NaN or Inf was read; affected outputs are unspecified */
+#define NV4_FLAG_E8M0_NAN  2u  /* an E8M0 scale byte 0xFF (NaN) was read                  */
+#define NV4_FLAG_OVERFLOW  4u  /* a second-level scale or global amax is not finite       */
+#define NV4_FLAG_TIMEOUT   8u  /* a bounded wait inside a kernel gave up; outputs of that
+                                  call are incomplete                                     */
+
+/* Human-readable name of a status code (static storage). */
+NV4_API const char* nv4_status_str(nv4_status s);
+
+/* Library ABI version (major*100 + minor). */
+NV4_API int nv4_version(void);
+
+/* ---------------------------------------------------------------------------
+ * nv4_tensor_amax -- per-tensor absolute maximum, as a running maximum.
+ * [CAL] section 2 step 1 (max calibration records the largest |w| and |x| of each
+ * layer over the calibration data, the initial scales); [FLOW] 3.4 (the calibrated
+ * amax gives the per-tensor scale).
+ *
+ *   *d_amax = max(*d_amax, max_i |x[i]|)
+ *
+ * x      : n elements of type dt (NV4_BF16 or NV4_FP32), contiguous, 16-byte aligned.
+ * d_amax : one float on the device, holding +0.0 or a previous amax before the first
+ *          call (a running max over calibration batches needs no reset between them).
+ * NaN elements are skipped; NaN or Inf sets NV4_FLAG_NONFINITE.  n == 0 is a no-op.
+ */
+NV4_API nv4_status nv4_tensor_amax(const void* x, nv4_dtype dt, int64_t n, float* d_amax,
+                           uint32_t* d_flags, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * nv4_act_quant -- dynamic NVFP4 quantization of activations.  [FLOW] 3.4-3.5:
+ * the per-tensor scale comes from a (calibrated or just measured) amax, the block
+ * scales are computed at run time from the data; [CAL] format line; [FLOW] 5.4.
+ *
+ *   s2        = RN32(amax / 2688)                       (2688 = 6 * 448)
+ *   per block : a_b = max|x|, s_b = E4M3 nearest to a_b / (6*s2) (ties to even code,
+ *               saturating at 448), S = RN32(s_b * s2),
+ *               code_i = sign(x_i) | E2M1 magnitude nearest to |x_i| / S (ties to even)
+ *   amax == 0 gives s2 = 0, block scale 0 and sign-only codes.
+ *
+ * x      : bf16 [rows, cols], leading dimension ld (ld % 8 == 0).  cols % 16 == 0.
+ * d_amax : device float (e.g. the output of nv4_tensor_amax), read on the device.
+ * q      : [rows, cols/2] bytes, contiguous.   scales : [rows, cols/16] E4M3 bytes.
+ * d_s2   : device float receiving s2.
+ */
+NV4_API nv4_status nv4_act_quant(const void* x, int64_t rows, int64_t cols, int64_t ld,
+                         const float* d_amax, uint8_t* q, uint8_t* scales, float* d_s2,
+                         uint32_t* d_flags, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * nv4_dequant -- the two-step dequantization of [FLOW] 3.4 / 5.4:
+ *   DQ1: S = RN32(s_b * s2);  DQ2: y = RN32(e2m1(code) * S), then rounded to out_dt
+ *   (NV4_BF16 default, NV4_FP16, or NV4_FP32 as is), ties to even, overflow to inf.
+ * q [rows, cols/2], scales [rows, cols/16], d_s2 device float; out [rows, cols]
+ * contiguous, 16-byte aligned.  cols % 16 == 0.
+ */
+NV4_API nv4_status nv4_dequant(const uint8_t* q, const uint8_t* scales, const float* d_s2,
+                       int64_t rows, int64_t cols, nv4_dtype out_dt, void* out, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * nv4_hessian_accum -- local Hessian per 16-input-channel block, [CAL] section 2
+ * step 2 (full-precision forward, H = sum X^T X accumulated per 16 channels at the
+ * layer input):
+ *
+ *   H[b][i][j] += sum_t x[t][16b+i] * x[t][16b+j]      (FP32 accumulation)
+ *
+ * x : bf16 [tokens, cols], leading dimension ld (ld % 8 == 0), cols % 16 == 0.
+ * H : float [cols/16][16][16] on the device, accumulated (+=); zero it before the
+ *     first calibration batch.  The result is deterministic (fixed reduction order).
+ * A non-finite partial sum sets NV4_FLAG_NONFINITE.
+ */
+NV4_API nv4_status nv4_hessian_accum(const void* x, int64_t tokens, int64_t cols, int64_t ld,
+                             float* H, uint32_t* d_flags, void* stream);
+
+typedef struct {
+    const void* x;      /* bf16 [tokens, cols], leading dimension ld */
+    int64_t tokens, cols, ld;
+    float* H;           /* [cols/16][16][16], +=; distinct jobs need distinct H */
+} nv4_hessian_job;
+
+/* Batched form: all jobs in one launch (e.g. the experts of an MoE layer).
+ * At most 128 jobs and 65535 64-column slabs in total per call (NV4_ERR_LIMIT beyond). */
+NV4_API nv4_status nv4_hessian_accum_batched(const nv4_hessian_job* jobs, int n_jobs,
+                                     uint32_t* d_flags, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * nv4_scale_sweep -- Hessian-weighted E4M3 block-scale search with NVFP4 pack of
+ * the winner, [CAL] section 2 step 3 (fp8_scale_sweep over all E4M3 scale values,
+ * minimising (W - Wq)^T H (W - Wq) per 16-element weight block).
+ *
+ *   s2 = RN32(amax_w / 2688)
+ *   for every block w and code c in 0x00..0x7E (the 127 finite non-negative codes):
+ *     S_c = RN32(e4m3(c) * s2), q = E2M1(w / S_c) as in nv4_act_quant,
+ *     e = w - e2m1(q) * S_c, cost_c = e^T H_b e
+ *   winner = argmin cost_c, ties to the lowest code.
+ *
+ * w        : [rows, cols] of dt (NV4_BF16 or NV4_FP32), leading dimension ld.
+ * H        : float [cols/16][16][16] (symmetric; e.g. from nv4_hessian_accum).
+ * d_amax_w : device float, the weight tensor's amax.
+ * codes    : [rows, cols/16] winning E4M3 codes.
+ * q        : [rows, cols/2] packed E2M1 codes at the winning scale, or NULL.
+ * cost1    : [rows, cols/16] float winning cost, or NULL.
+ * cost2    : [rows, cols/16] float smallest cost above the winner's (+inf if none),
+ *            or NULL -- a near-tie diagnostic.
+ * Costs are evaluated in FP32; blocks whose best and second-best costs differ by
+ * less than ~1e-6 relative may pick a different code than an exact evaluation.
+ */
+NV4_API nv4_status nv4_scale_sweep(const void* w, nv4_dtype dt, int64_t rows, int64_t cols, int64_t ld,
+                           const float* H, const float* d_amax_w, uint8_t* codes, uint8_t* q,
+                           float* cost1, float* cost2, uint32_t* d_flags, void* stream);
+
+typedef struct {
+    const void* w;      /* [rows, cols] of the call's dt, leading dimension ld */
+    int64_t rows, cols, ld;
+    const float* H;     /* [cols/16][16][16] */
+    const float* d_amax_w;
+    uint8_t* codes;     /* [rows, cols/16] */
+    uint8_t* q;         /* [rows, cols/2] or NULL */
+    float* cost1;       /* or NULL */
+    float* cost2;       /* or NULL */
+} nv4_sweep_job;
+
+/* Batched form (e.g. all gate/up/down matrices of an expert stack) in one launch.
+ * At most 192 jobs per call (NV4_ERR_LIMIT beyond). */
+NV4_API nv4_status nv4_scale_sweep_batched(const nv4_sweep_job* jobs, int n_jobs, nv4_dtype dt,
+                                   uint32_t* d_flags, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * nv4_mxfp4_to_nvfp4 -- closed-form MXFP4 -> NVFP4 cast of one matrix, [CAST] section 2,
+ * [DSPARK] stage 3.
+ *
+ *   k_j = e8m0_j - 127, k_max = max_j k_j over the matrix, m = k_max - 8
+ *   *d_s2 = 2^m, *d_global_amax = 6*448*2^m (FP32; NV4_FLAG_OVERFLOW if not finite)
+ *   each 32-element MX block j gives two 16-element NVFP4 blocks:
+ *     k_max - k_j <= 17 : scale code encodes 2^(k_j - m) exactly, nibbles copied
+ *     otherwise         : re-quantized from the exact values e2m1*2^k_j with the
+ *                         nv4_act_quant rules (block amax max|w_block|, s2 = 2^m)
+ *
+ * mx_q [rows, cols/2] nibbles, e8m0 [rows, cols/32]; cols % 32 == 0.
+ * nv_q [rows, cols/2] (may equal mx_q: then only fallback blocks are rewritten),
+ * nv_scales [rows, cols/16].  d_counts: 3 unsigned long long on the device,
+ * accumulated (+=): [0] in-window 16-blocks, [1] fallback 16-blocks, [2] lossless
+ * 16-blocks (NVFP4 dequant equal to the MXFP4 dequant bit for bit).  An E8M0 byte
+ * 0xFF sets NV4_FLAG_E8M0_NAN and is excluded from k_max; its blocks are unspecified.
+ */
+NV4_API nv4_status nv4_mxfp4_to_nvfp4(const uint8_t* mx_q, const uint8_t* e8m0, int64_t rows, int64_t cols,
+                              uint8_t* nv_q, uint8_t* nv_scales, float* d_global_amax, float* d_s2,
+                              unsigned long long* d_counts, uint32_t* d_flags, void* stream);
+
+typedef struct {
+    const uint8_t* mx_q;
+    const uint8_t* e8m0;
+    int64_t rows, cols;
+    uint8_t* nv_q;
+    uint8_t* nv_scales;
+    float* d_global_amax;
+    float* d_s2;
+} nv4_cast_job;
+
+/* Batched form: one launch for many matrices (each with its own k_max).
+ * At most 128 jobs per call (NV4_ERR_LIMIT beyond). */
+NV4_API nv4_status nv4_mxfp4_to_nvfp4_batched(const nv4_cast_job* jobs, int n_jobs,
+                                      unsigned long long* d_counts, uint32_t* d_flags, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * nv4_selftest -- checks, on the current device, the hardware FP4/FP8 conversion
+ * instructions the kernels rely on (lane order, rounding, sign of zero, saturation).
+ * Writes 64 uint32 results to d_out (device); d_out[0] is a bit mask of failed
+ * checks (0 = all passed), the rest are the raw values observed.  Not a paper
+ * operation: a diagnostic of the build on the GPU it runs on.
+ */
+NV4_API nv4_status nv4_selftest(uint32_t* d_out, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif

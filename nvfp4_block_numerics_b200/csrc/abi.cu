@@ -1,0 +1,258 @@
+// abi.cu -- the extern "C" entry points of libnv4.so (declared in include/nv4.h):
+// argument validation, then one stream-ordered kernel launch per call.
+#include <cstdint>
+
+#include "nv4_common.cuh"
+#include "nv4_internal.h"
+
+namespace nv4 {
+
+int num_sms()
+{
+    static int cache[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (cache[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        cache[dev] = n;
+    }
+    return cache[dev];
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0u; }
+
+static nv4_status from_cuda(cudaError_t e) { return e == cudaSuccess ? NV4_OK : NV4_ERR_CUDA; }
+
+// ---------------------------------------------------------------- self-test
+__global__ void selftest_kernel(uint32_t* out)
+{
+    if (threadIdx.x != 0 || blockIdx.x != 0) return;
+    uint32_t fail = 0u;
+    // E2M1 pack: lane order, RNE ties (2.5 -> 2), saturation (7 -> 6), sign of zero
+    const float v[8] = {0.5f, 6.0f, -1.0f, 0.0f, -0.0f, -0.1f, 7.0f, 2.5f};
+    const uint32_t p = cvt_e2m1x8(v);
+    out[1] = p;
+    if (p != 0x47880A71u) fail |= 1u;
+    // E4M3 pair: lane order and saturation
+    const uint32_t a = cvt_e4m3x2(1.0f, 448.0f);
+    out[2] = a;
+    if (a != 0x7E38u) fail |= 2u;
+    const uint32_t b = cvt_e4m3x2(0x1p-10f, 0x1.8p-10f);   // tie to even (0), nearest subnormal (1)
+    out[3] = b;
+    if (b != 0x0100u) fail |= 4u;
+    const uint32_t c = cvt_e4m3x2(500.0f, 1e30f);
+    out[4] = c;
+    if (c != 0x7E7Eu) fail |= 8u;
+    // E2M1 -> FP16 decode: lane order and sign
+    uint32_t h[4];
+    cvt_e2m1x8_to_f16x8(0x47880A71u, h);
+    for (int i = 0; i < 4; ++i) out[5 + i] = h[i];
+    if (h[0] != 0x46003800u || h[1] != 0x0000BC00u || h[2] != 0x80008000u || h[3] != 0x40004600u) fail |= 16u;
+    // BF16 pair packing order and rounding
+    uint32_t bf;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(bf) : "f"(3.0f), "f"(1.0f + 0x1p-9f));
+    out[9] = bf;
+    if (bf != 0x40403F80u) fail |= 32u;
+    // E4M3 values used by the kernels
+    if (e4m3_value(0x7Eu) != 448.0f || e4m3_value(1u) != 0x1p-9f || e4m3_value(0x38u) != 1.0f) fail |= 64u;
+    // exact fallbacks against known answers
+    if (e4m3_code_exact(448.0f * 6.0f, 1.0f) != 0x7Eu || e4m3_code_exact(6.0f * 0x1p-10f, 1.0f) != 0u ||
+        e4m3_code_exact(6.0f * 0x1.8p-10f, 1.0f) != 1u)
+        fail |= 128u;
+    if (e2m1_code_exact(2.5f, 1.0f) != 4u || e2m1_code_exact(-0.25f, 1.0f) != 8u ||
+        e2m1_code_exact(0.75f, 1.0f) != 2u || e2m1_code_exact(100.0f, 1.0f) != 7u)
+        fail |= 256u;
+    FastDiv fd(7u);
+    if (fd.div(48u) != 6u || fd.div(0xFFFFFFFFu) != 0xFFFFFFFFu / 7u) fail |= 512u;
+    out[0] = fail;
+}
+
+cudaError_t launch_selftest(uint32_t* d_out, cudaStream_t s)
+{
+    selftest_kernel<<<1, 32, 0, s>>>(d_out);
+    return cudaGetLastError();
+}
+
+}  // namespace nv4
+
+using namespace nv4;
+
+extern "C" {
+
+const char* nv4_status_str(nv4_status s)
+{
+    switch (s) {
+    case NV4_OK: return "NV4_OK";
+    case NV4_ERR_NULL: return "NV4_ERR_NULL: a required pointer is NULL";
+    case NV4_ERR_SHAPE: return "NV4_ERR_SHAPE: invalid size or shape";
+    case NV4_ERR_ALIGN: return "NV4_ERR_ALIGN: pointer or leading dimension not 16-byte aligned";
+    case NV4_ERR_DTYPE: return "NV4_ERR_DTYPE: unsupported element type";
+    case NV4_ERR_CUDA: return "NV4_ERR_CUDA: CUDA runtime or launch error";
+    case NV4_ERR_LIMIT: return "NV4_ERR_LIMIT: size beyond what one call supports";
+    }
+    return "unknown nv4_status";
+}
+
+int nv4_version(void) { return 100; }
+
+nv4_status nv4_tensor_amax(const void* x, nv4_dtype dt, int64_t n, float* d_amax, uint32_t* d_flags, void* stream)
+{
+    if (n < 0) return NV4_ERR_SHAPE;
+    if (n == 0) return NV4_OK;
+    if (x == nullptr || d_amax == nullptr) return NV4_ERR_NULL;
+    if (dt != NV4_BF16 && dt != NV4_FP32) return NV4_ERR_DTYPE;
+    if (!aligned16(x)) return NV4_ERR_ALIGN;
+    return from_cuda(launch_amax(x, dt == NV4_BF16 ? 0 : 2, n, d_amax, d_flags, (cudaStream_t)stream));
+}
+
+nv4_status nv4_act_quant(const void* x, int64_t rows, int64_t cols, int64_t ld, const float* d_amax, uint8_t* q,
+                         uint8_t* scales, float* d_s2, uint32_t* d_flags, void* stream)
+{
+    if (rows < 0 || cols < 0 || cols % 16 != 0 || ld < cols) return NV4_ERR_SHAPE;
+    if (d_amax == nullptr || d_s2 == nullptr) return NV4_ERR_NULL;
+    if (rows == 0 || cols == 0) return NV4_OK;
+    if (x == nullptr || q == nullptr || scales == nullptr) return NV4_ERR_NULL;
+    if (!aligned16(x) || !aligned16(q) || ld % 8 != 0) return NV4_ERR_ALIGN;
+    if (rows * (cols / 16) >= (int64_t)1 << 32) return NV4_ERR_LIMIT;
+    return from_cuda(launch_act_quant(x, rows, cols, ld, d_amax, q, scales, d_s2, d_flags, (cudaStream_t)stream));
+}
+
+nv4_status nv4_dequant(const uint8_t* q, const uint8_t* scales, const float* d_s2, int64_t rows, int64_t cols,
+                       nv4_dtype out_dt, void* out, void* stream)
+{
+    if (rows < 0 || cols < 0 || cols % 16 != 0) return NV4_ERR_SHAPE;
+    if (out_dt != NV4_BF16 && out_dt != NV4_FP16 && out_dt != NV4_FP32) return NV4_ERR_DTYPE;
+    if (rows == 0 || cols == 0) return NV4_OK;
+    if (q == nullptr || scales == nullptr || d_s2 == nullptr || out == nullptr) return NV4_ERR_NULL;
+    if (!aligned16(q) || !aligned16(out)) return NV4_ERR_ALIGN;
+    if (rows * (cols / 16) >= (int64_t)1 << 32) return NV4_ERR_LIMIT;
+    return from_cuda(launch_dequant(q, scales, d_s2, rows, cols, (int)out_dt, out, (cudaStream_t)stream));
+}
+
+static nv4_status check_hessian_job(const nv4_hessian_job& J)
+{
+    if (J.tokens < 0 || J.cols < 0 || J.cols % 16 != 0 || J.ld < J.cols) return NV4_ERR_SHAPE;
+    if (J.tokens == 0 || J.cols == 0) return NV4_OK;
+    if (J.x == nullptr || J.H == nullptr) return NV4_ERR_NULL;
+    if (!aligned16(J.x) || J.ld % 8 != 0) return NV4_ERR_ALIGN;
+    if (J.tokens >= ((int64_t)1 << 31) || J.cols >= ((int64_t)1 << 31)) return NV4_ERR_LIMIT;
+    return NV4_OK;
+}
+
+nv4_status nv4_hessian_accum_batched(const nv4_hessian_job* jobs, int n_jobs, uint32_t* d_flags, void* stream)
+{
+    if (n_jobs < 0) return NV4_ERR_SHAPE;
+    if (n_jobs == 0) return NV4_OK;
+    if (jobs == nullptr) return NV4_ERR_NULL;
+    if (n_jobs > kMaxHessianJobs) return NV4_ERR_LIMIT;
+    int64_t slabs = 0;
+    for (int i = 0; i < n_jobs; ++i) {
+        const nv4_status st = check_hessian_job(jobs[i]);
+        if (st != NV4_OK) return st;
+        slabs += (jobs[i].cols + 63) / 64;
+    }
+    if (slabs > 65535) return NV4_ERR_LIMIT;
+    int bad = -1;
+    const cudaError_t e = launch_hessian(jobs, n_jobs, d_flags, (cudaStream_t)stream, &bad);
+    if (bad >= 0) return NV4_ERR_ALIGN;   // the TMA descriptor rejected the tensor's layout
+    return from_cuda(e);
+}
+
+nv4_status nv4_hessian_accum(const void* x, int64_t tokens, int64_t cols, int64_t ld, float* H, uint32_t* d_flags,
+                             void* stream)
+{
+    nv4_hessian_job j;
+    j.x = x; j.tokens = tokens; j.cols = cols; j.ld = ld; j.H = H;
+    return nv4_hessian_accum_batched(&j, 1, d_flags, stream);
+}
+
+static nv4_status check_sweep_job(const nv4_sweep_job& J, nv4_dtype dt)
+{
+    if (J.rows < 0 || J.cols < 0 || J.cols % 16 != 0 || J.ld < J.cols) return NV4_ERR_SHAPE;
+    if (J.d_amax_w == nullptr) return NV4_ERR_NULL;
+    if (J.rows == 0 || J.cols == 0) return NV4_OK;
+    if (J.w == nullptr || J.H == nullptr || J.codes == nullptr) return NV4_ERR_NULL;
+    const int64_t esz = dt == NV4_FP32 ? 4 : 2;
+    if (!aligned16(J.w) || (J.ld * esz) % 16 != 0 || (J.q != nullptr && !aligned16(J.q))) return NV4_ERR_ALIGN;
+    if (J.rows >= ((int64_t)1 << 31) || J.cols >= ((int64_t)1 << 31)) return NV4_ERR_LIMIT;
+    return NV4_OK;
+}
+
+nv4_status nv4_scale_sweep_batched(const nv4_sweep_job* jobs, int n_jobs, nv4_dtype dt, uint32_t* d_flags,
+                                   void* stream)
+{
+    if (n_jobs < 0) return NV4_ERR_SHAPE;
+    if (dt != NV4_BF16 && dt != NV4_FP32) return NV4_ERR_DTYPE;
+    if (n_jobs == 0) return NV4_OK;
+    if (jobs == nullptr) return NV4_ERR_NULL;
+    if (n_jobs > kMaxSweepJobs) return NV4_ERR_LIMIT;
+    int64_t ctas = 0;
+    for (int i = 0; i < n_jobs; ++i) {
+        const nv4_status st = check_sweep_job(jobs[i], dt);
+        if (st != NV4_OK) return st;
+        ctas += ((jobs[i].rows + 127) / 128) * (jobs[i].cols / 16);
+    }
+    if (ctas >= ((int64_t)1 << 31)) return NV4_ERR_LIMIT;
+    return from_cuda(launch_sweep(jobs, n_jobs, dt == NV4_BF16 ? 0 : 2, d_flags, (cudaStream_t)stream));
+}
+
+nv4_status nv4_scale_sweep(const void* w, nv4_dtype dt, int64_t rows, int64_t cols, int64_t ld, const float* H,
+                           const float* d_amax_w, uint8_t* codes, uint8_t* q, float* cost1, float* cost2,
+                           uint32_t* d_flags, void* stream)
+{
+    nv4_sweep_job j;
+    j.w = w; j.rows = rows; j.cols = cols; j.ld = ld; j.H = H; j.d_amax_w = d_amax_w;
+    j.codes = codes; j.q = q; j.cost1 = cost1; j.cost2 = cost2;
+    return nv4_scale_sweep_batched(&j, 1, dt, d_flags, stream);
+}
+
+static nv4_status check_cast_job(const nv4_cast_job& J)
+{
+    if (J.rows < 0 || J.cols < 0 || J.cols % 32 != 0) return NV4_ERR_SHAPE;
+    if (J.rows == 0 || J.cols == 0) return NV4_OK;
+    if (J.mx_q == nullptr || J.e8m0 == nullptr || J.nv_q == nullptr || J.nv_scales == nullptr ||
+        J.d_global_amax == nullptr || J.d_s2 == nullptr)
+        return NV4_ERR_NULL;
+    if (!aligned16(J.mx_q) || !aligned16(J.e8m0) || !aligned16(J.nv_q) || !aligned16(J.nv_scales))
+        return NV4_ERR_ALIGN;
+    if (J.rows * (J.cols / 32) >= ((int64_t)1 << 31)) return NV4_ERR_LIMIT;
+    // in-place is allowed only as exact aliasing of the nibble buffers
+    const uint8_t* a = J.mx_q;
+    const uint8_t* b = J.nv_q;
+    const int64_t bytes = J.rows * (J.cols / 2);
+    if (a != b && a < b + bytes && b < a + bytes) return NV4_ERR_SHAPE;
+    return NV4_OK;
+}
+
+nv4_status nv4_mxfp4_to_nvfp4_batched(const nv4_cast_job* jobs, int n_jobs, unsigned long long* d_counts,
+                                      uint32_t* d_flags, void* stream)
+{
+    if (n_jobs < 0) return NV4_ERR_SHAPE;
+    if (n_jobs == 0) return NV4_OK;
+    if (jobs == nullptr) return NV4_ERR_NULL;
+    if (n_jobs > kMaxCastJobs) return NV4_ERR_LIMIT;
+    for (int i = 0; i < n_jobs; ++i) {
+        const nv4_status st = check_cast_job(jobs[i]);
+        if (st != NV4_OK) return st;
+    }
+    return from_cuda(launch_cast(jobs, n_jobs, d_counts, d_flags, (cudaStream_t)stream));
+}
+
+nv4_status nv4_mxfp4_to_nvfp4(const uint8_t* mx_q, const uint8_t* e8m0, int64_t rows, int64_t cols, uint8_t* nv_q,
+                              uint8_t* nv_scales, float* d_global_amax, float* d_s2, unsigned long long* d_counts,
+                              uint32_t* d_flags, void* stream)
+{
+    nv4_cast_job j;
+    j.mx_q = mx_q; j.e8m0 = e8m0; j.rows = rows; j.cols = cols; j.nv_q = nv_q; j.nv_scales = nv_scales;
+    j.d_global_amax = d_global_amax; j.d_s2 = d_s2;
+    return nv4_mxfp4_to_nvfp4_batched(&j, 1, d_counts, d_flags, stream);
+}
+
+nv4_status nv4_selftest(uint32_t* d_out, void* stream)
+{
+    if (d_out == nullptr) return NV4_ERR_NULL;
+    return from_cuda(launch_selftest(d_out, (cudaStream_t)stream));
+}
+
+}  // extern "C"

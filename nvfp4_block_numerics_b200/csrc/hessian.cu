@@ -1,0 +1,373 @@
+// hessian.cu -- local Hessian H_b += X_b^T X_b per 16-channel block (sm_100a).
+//
+// [CAL] section 2 step 2: with full-precision weights, accumulate H = sum X^T X per
+// block of 16 input channels at each layer input (see nv4.h).
+//
+// The useful work is the block diagonal of the Gram matrix X^T X: 2*16 FLOP per
+// byte of BF16 input, so at HBM speed the contraction needs ~100 TFLOP/s, above
+// what the FP32 pipe delivers.  It runs on the tensor cores with the m16n8k16
+// BF16 MMA, whose 16x16 output tile is exactly one H_b, so no FLOP is spent off
+// the diagonal (a 64- or 128-wide tcgen05 tile would compute 4x-8x more than
+// needed).  Products of BF16 values are exact; accumulation is FP32.
+//
+// Data movement:
+//   * a CTA owns a slab of 64 channels (4 blocks) and a range of 64-token tiles;
+//   * one producer warp streams [64 tokens x 64 channels] tiles (8 KB) with 2-D
+//     TMA loads (128-byte swizzle) into a 6-stage shared-memory ring guarded by
+//     mbarriers; ragged token or channel edges are zero-filled by the TMA unit;
+//   * four consumer warps each take 16 tokens of a tile: one ldmatrix.x4.trans
+//     per block yields the MMA A fragment of X_b^T, and the same four registers
+//     are the B fragments of X_b (A[m][k] = X[k][m] and B[k][n] = X[k][n]);
+//   * the token range of a slab is split over the CTAs of a thread-block cluster;
+//     partials are summed in a fixed order (warps, then cluster ranks through
+//     distributed shared memory) and added to H by cluster rank 0, so the result
+//     is bit-reproducible.
+// Every mbarrier wait is bounded (kWaitLimitNs); on expiry the kernel sets
+// NV4_FLAG_TIMEOUT, stops issuing, drains its own copies in flight and finishes.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "nv4_common.cuh"
+#include "nv4_internal.h"
+
+namespace nv4 {
+
+constexpr int kTok = 64;                 // tokens per tile
+constexpr int kSlab = 64;                // channels per CTA
+constexpr int kStages = 6;
+constexpr int kConsumerWarps = 4;
+constexpr int kHThreads = (kConsumerWarps + 1) * 32;
+constexpr uint32_t kTileBytes = kTok * kSlab * 2;
+constexpr int kMaxCluster = 8;
+
+struct HessJobDev {
+    CUtensorMap tmap;                    // X as [tokens][cols] bf16, box 64x64, swizzle 128B
+    float* H;
+    uint32_t ntiles;                     // ceil(tokens / 64)
+    uint32_t nblk;                       // cols / 16
+    uint32_t slab_begin;                 // prefix sum of slabs over jobs
+    uint32_t pad;
+};
+
+struct HessParams {
+    int n;
+    uint32_t* d_flags;
+    HessJobDev jobs[kMaxHessianJobs];
+};
+
+struct HessSmem {
+    alignas(1024) uint8_t tiles[kStages][kTileBytes];
+    alignas(8) uint64_t full[kStages];
+    uint64_t empty[kStages];
+    uint32_t consumed;                   // tiles fully consumed (for draining on timeout)
+    uint32_t timeout;
+};
+
+// ------------------------------------------------------------------ PTX helpers
+__device__ __forceinline__ uint32_t smem_u32(const void* p)
+{
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(ok)
+                 : "r"(smem_u32(bar)), "r"(parity)
+                 : "memory");
+    return ok != 0u;
+}
+
+// Bounded wait: false when the phase did not complete within kWaitLimitNs.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity)
+{
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    while (!mbar_try_wait(bar, parity))
+        if (global_ns() - t0 > kWaitLimitNs) return false;
+    return true;
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+        ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t addr, uint32_t r[4])
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+
+__device__ __forceinline__ void mma_bf16_16816(float d[4], const uint32_t a[4], uint32_t b0, uint32_t b1)
+{
+    asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+                 "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+                 : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+                 : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t cluster_ctarank()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t cluster_nctarank()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+    return r;
+}
+
+__device__ __forceinline__ void cluster_sync()
+{
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ float ld_dsmem_f32(const float* local, uint32_t rank)
+{
+    uint32_t remote;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(local)), "r"(rank));
+    float v;
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
+    return v;
+}
+
+// ------------------------------------------------------------------ kernel
+__global__ void __launch_bounds__(kHThreads)
+hessian_kernel(const __grid_constant__ HessParams p)
+{
+    extern __shared__ uint8_t smem_raw[];
+    HessSmem& sm = *reinterpret_cast<HessSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+
+    // job and slab of this CTA (blockIdx.y = global slab index)
+    int j = 0;
+    {
+        int lo = 0, hi = p.n - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (p.jobs[mid].slab_begin <= blockIdx.y) lo = mid; else hi = mid - 1;
+        }
+        j = lo;
+    }
+    const HessJobDev& job = p.jobs[j];
+    const uint32_t slab = blockIdx.y - job.slab_begin;
+    const uint32_t rank = cluster_ctarank(), nrank = cluster_nctarank();
+    const uint32_t t_begin = (uint32_t)(((uint64_t)job.ntiles * rank) / nrank);
+    const uint32_t t_end = (uint32_t)(((uint64_t)job.ntiles * (rank + 1)) / nrank);
+    const uint32_t ntile = t_end - t_begin;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&sm.full[s], 1);
+            mbar_init(&sm.empty[s], kConsumerWarps);
+        }
+        sm.consumed = 0u;
+        sm.timeout = 0u;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+
+    float acc[4][2][4];
+#pragma unroll
+    for (int bk = 0; bk < 4; ++bk)
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int k = 0; k < 4; ++k) acc[bk][h][k] = 0.0f;
+
+    if (warp == kConsumerWarps) {
+        // ---------------- producer: one lane issues the TMA loads
+        if (lane == 0) {
+            uint32_t issued = 0;
+            for (uint32_t i = 0; i < ntile; ++i) {
+                const int s = (int)(i % kStages);
+                if (i >= (uint32_t)kStages && !mbar_wait(&sm.empty[s], ((i / kStages) + 1u) & 1u)) {
+                    atomicOr(&sm.timeout, 1u);
+                    break;
+                }
+                if (*reinterpret_cast<volatile uint32_t*>(&sm.timeout)) break;
+                mbar_arrive_expect_tx(&sm.full[s], kTileBytes);
+                tma_load_2d(sm.tiles[s], &job.tmap, &sm.full[s], (int)(slab * kSlab), (int)((t_begin + i) * kTok));
+                ++issued;
+            }
+            // drain: every issued copy must have landed before shared memory is reused
+            const uint32_t done = *reinterpret_cast<volatile uint32_t*>(&sm.consumed);
+            for (uint32_t i = done; i < issued; ++i)
+                if (!mbar_wait(&sm.full[i % kStages], (i / kStages) & 1u)) atomicOr(&sm.timeout, 1u);
+        }
+    } else {
+        // ---------------- consumers
+        const uint32_t row_in = (uint32_t)(lane & 7), mat = (uint32_t)(lane >> 3);
+        const uint32_t tok = (uint32_t)warp * 16u + (mat >> 1) * 8u + row_in;   // token row of this lane's address
+        for (uint32_t i = 0; i < ntile; ++i) {
+            const int s = (int)(i % kStages);
+            if (!mbar_wait(&sm.full[s], (i / kStages) & 1u)) {
+                atomicOr(&sm.timeout, 1u);
+                break;
+            }
+            const uint32_t base = smem_u32(sm.tiles[s]) + tok * 128u;
+#pragma unroll
+            for (int bk = 0; bk < 4; ++bk) {
+                const uint32_t chunk = (uint32_t)(2 * bk) + (mat & 1u);
+                uint32_t a[4];
+                ldmatrix_x4_trans(base + ((chunk ^ (tok & 7u)) << 4), a);
+                mma_bf16_16816(acc[bk][0], a, a[0], a[2]);
+                mma_bf16_16816(acc[bk][1], a, a[1], a[3]);
+            }
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&sm.empty[s]);
+                if (warp == 0) atomicMax(&sm.consumed, i + 1u);
+            }
+            if (*reinterpret_cast<volatile uint32_t*>(&sm.timeout)) break;
+        }
+    }
+    __syncthreads();
+
+    // ---------------- reduce: warps (fixed order) -> CTA partial in shared memory
+    float* part = reinterpret_cast<float*>(sm.tiles[0]);        // [4 warps][4 blocks][256]
+    if (warp < kConsumerWarps) {
+        const int g = lane >> 2, c = lane & 3;
+#pragma unroll
+        for (int bk = 0; bk < 4; ++bk)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                float* P = part + (warp * 4 + bk) * 256;
+                const int n0 = 8 * h + 2 * c;
+                P[g * 16 + n0] = acc[bk][h][0];
+                P[g * 16 + n0 + 1] = acc[bk][h][1];
+                P[(g + 8) * 16 + n0] = acc[bk][h][2];
+                P[(g + 8) * 16 + n0 + 1] = acc[bk][h][3];
+            }
+    }
+    __syncthreads();
+    float* cta_part = reinterpret_cast<float*>(sm.tiles[2]);    // [4 blocks][256]
+    for (int e = threadIdx.x; e < 1024; e += kHThreads)
+        cta_part[e] = ((part[e] + part[1024 + e]) + part[2048 + e]) + part[3072 + e];
+    cluster_sync();
+
+    // ---------------- cluster rank 0 sums the ranks in order and adds into H
+    uint32_t flags = 0u;
+    if (rank == 0) {
+        for (int e = threadIdx.x; e < 1024; e += kHThreads) {
+            const uint32_t bk = slab * 4u + (uint32_t)(e >> 8);
+            if (bk >= job.nblk) continue;
+            float sum = cta_part[e];
+            for (uint32_t r = 1; r < nrank; ++r) sum += ld_dsmem_f32(cta_part + e, r);
+            float* dst = job.H + (int64_t)bk * 256 + (e & 255);
+            const float v = *dst + sum;
+            *dst = v;
+            if (!isfinite(v)) flags |= kFlagNonFinite;
+        }
+    }
+    if (sm.timeout) flags |= kFlagTimeout;
+    cluster_sync();                                              // keep shared memory alive for readers
+    flags = __reduce_or_sync(0xFFFFFFFFu, flags);
+    if (lane == 0) flag_or(p.d_flags, flags);
+}
+
+// ------------------------------------------------------------------ host side
+static PFN_cuTensorMapEncodeTiled_v12000 get_encoder()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (fn == nullptr) {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+    return fn;
+}
+
+static size_t hess_smem_bytes() { return sizeof(HessSmem) + 1024; }
+
+cudaError_t launch_hessian(const nv4_hessian_job* jobs, int n, uint32_t* d_flags, cudaStream_t s, int* bad_job)
+{
+    *bad_job = -1;
+    auto encode = get_encoder();
+    if (encode == nullptr) return cudaErrorNotSupported;
+
+    HessParams p;          // ~25 KB, copied into the launch's parameter buffer
+    p.d_flags = d_flags;
+    int m = 0;
+    uint32_t slabs = 0, max_tiles = 0;
+    for (int i = 0; i < n; ++i) {
+        const nv4_hessian_job& J = jobs[i];
+        if (J.tokens == 0 || J.cols == 0) continue;
+        HessJobDev& d = p.jobs[m];
+        const cuuint64_t dims[2] = {(cuuint64_t)J.cols, (cuuint64_t)J.tokens};
+        const cuuint64_t strides[1] = {(cuuint64_t)J.ld * 2u};
+        const cuuint32_t box[2] = {(cuuint32_t)kSlab, (cuuint32_t)kTok};
+        const cuuint32_t estr[2] = {1u, 1u};
+        const CUresult r = encode(&d.tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(J.x), dims,
+                                  strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) {
+            *bad_job = i;
+            return cudaErrorInvalidValue;
+        }
+        d.H = J.H;
+        d.ntiles = (uint32_t)((J.tokens + kTok - 1) / kTok);
+        d.nblk = (uint32_t)(J.cols / 16);
+        d.slab_begin = slabs;
+        slabs += (uint32_t)((J.cols + kSlab - 1) / kSlab);
+        if (d.ntiles > max_tiles) max_tiles = d.ntiles;
+        ++m;
+    }
+    p.n = m;
+    if (m == 0) return cudaSuccess;
+
+    // cluster size: enough CTAs to fill the GPU (~3 per SM), each with >= 8 tiles
+    const uint32_t target = (uint32_t)num_sms() * 3u;
+    uint32_t z = 1;
+    while (z < (uint32_t)kMaxCluster && slabs * z < target && max_tiles / (2u * z) >= 8u) z *= 2u;
+
+    const size_t smem = hess_smem_bytes();
+    cudaError_t e = cudaFuncSetAttribute(hessian_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(z, slabs, 1);
+    cfg.blockDim = dim3(kHThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = z;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, hessian_kernel, p);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
+}  // namespace nv4

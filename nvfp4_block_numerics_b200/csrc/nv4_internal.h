@@ -1,0 +1,48 @@
+// nv4_internal.h -- declarations shared by the kernel files and the C-ABI layer.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/nv4.h"
+
+namespace nv4 {
+
+// Division of 32-bit unsigned integers by a fixed divisor d >= 1 with one
+// multiply-high, one add and one shift (T. Granlund and P. L. Montgomery,
+// "Division by invariant integers using multiplication", PLDI 1994, round-up
+// method): with s = ceil(log2 d) and m = floor(2^32 (2^s - d) / d) + 1,
+// n / d = (mulhi(n, m) + n) >> s for every n < 2^32.
+struct FastDiv {
+    uint32_t d = 1, m = 1, s = 0;
+    __host__ __device__ FastDiv() {}
+    __host__ __device__ explicit FastDiv(uint32_t div) : d(div)
+    {
+        s = 0;
+        while ((1ull << s) < div) ++s;
+        m = (uint32_t)((((1ull << 32) * ((1ull << s) - div)) / div) + 1ull);
+    }
+    __device__ __forceinline__ uint32_t div(uint32_t n) const
+    {
+        return (uint32_t)(((uint64_t)__umulhi(n, m) + n) >> s);
+    }
+};
+
+int num_sms();
+
+constexpr int kMaxHessianJobs = 128;
+constexpr int kMaxSweepJobs = 192;
+constexpr int kMaxCastJobs = 128;
+
+cudaError_t launch_amax(const void* x, int dt, int64_t n, float* d_amax, uint32_t* d_flags, cudaStream_t s);
+cudaError_t launch_act_quant(const void* x, int64_t rows, int64_t cols, int64_t ld, const float* d_amax,
+                             uint8_t* q, uint8_t* scales, float* d_s2, uint32_t* d_flags, cudaStream_t s);
+cudaError_t launch_dequant(const uint8_t* q, const uint8_t* scales, const float* d_s2, int64_t rows, int64_t cols,
+                           int out_dt, void* out, cudaStream_t s);
+cudaError_t launch_hessian(const nv4_hessian_job* jobs, int n, uint32_t* d_flags, cudaStream_t s, int* bad_job);
+cudaError_t launch_sweep(const nv4_sweep_job* jobs, int n, int dt, uint32_t* d_flags, cudaStream_t s);
+cudaError_t launch_cast(const nv4_cast_job* jobs, int n, unsigned long long* d_counts, uint32_t* d_flags,
+                        cudaStream_t s);
+cudaError_t launch_selftest(uint32_t* d_out, cudaStream_t s);
+
+}  // namespace nv4

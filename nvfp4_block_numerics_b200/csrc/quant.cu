@@ -1,0 +1,328 @@
+// quant.cu -- per-tensor amax, dynamic NVFP4 activation quantization and the
+// two-step dequantization (sm_100a).
+//
+// Operations and their sources are documented at the entry points in
+// include/nv4.h ([CAL] section 2 step 1; [FLOW] sections 3.4-3.6 and 5.4).
+//
+// All three kernels are HBM-bound streams: one pass over the input, 128-bit
+// loads and stores, a grid of a few CTAs per SM striding over the data.
+#include "nv4_common.cuh"
+#include "nv4_internal.h"
+
+namespace nv4 {
+
+// ============================================================== amax
+// Running maximum of |x|.  The maximum of BF16 (or FP32) magnitudes is taken on
+// their bit patterns: for non-negative IEEE values the unsigned order of the bit
+// patterns is the numeric order, and NaN patterns sort above +Inf.  A thread whose
+// data holds a NaN re-scans its own elements without the NaN entries (rare path).
+template <int kThreads>
+__device__ __forceinline__ uint32_t block_max_u32(uint32_t v, uint32_t* red)
+{
+    v = __reduce_max_sync(0xFFFFFFFFu, v);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (lane == 0) red[warp] = v;
+    __syncthreads();
+    if (warp == 0) {
+        v = lane < kThreads / 32 ? red[lane] : 0u;
+        v = __reduce_max_sync(0xFFFFFFFFu, v);
+    }
+    return v;
+}
+
+__device__ __forceinline__ uint32_t absmax_bf16x8(const uint4& v)
+{
+    const uint32_t a = __vmaxu2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu);
+    const uint32_t b = __vmaxu2(v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu);
+    return __vmaxu2(a, b);
+}
+
+__device__ __forceinline__ uint32_t absmax_bf16x8_no_nan(const uint4& v)
+{
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t m = 0u;
+    for (int j = 0; j < 4; ++j) {
+        const uint32_t lo = w[j] & 0x7FFFu, hi = (w[j] >> 16) & 0x7FFFu;
+        if (lo <= 0x7F80u) m = max(m, lo);
+        if (hi <= 0x7F80u) m = max(m, hi);
+    }
+    return m;
+}
+
+template <int kThreads>
+__global__ void __launch_bounds__(kThreads)
+amax_bf16_kernel(const uint4* __restrict__ x, int64_t nvec, const uint16_t* __restrict__ tail, int ntail,
+                 float* __restrict__ d_amax, uint32_t* __restrict__ d_flags)
+{
+    __shared__ uint32_t red[kThreads / 32];
+    const int64_t stride = (int64_t)gridDim.x * kThreads;
+    const int64_t i0 = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+    uint32_t m = 0u;                                   // two packed 16-bit maxima
+    int64_t i = i0;
+    for (; i + 3 * stride < nvec; i += 4 * stride) {   // four independent loads in flight
+        const uint4 v0 = __ldcs(x + i), v1 = __ldcs(x + i + stride);
+        const uint4 v2 = __ldcs(x + i + 2 * stride), v3 = __ldcs(x + i + 3 * stride);
+        m = __vmaxu2(m, __vmaxu2(__vmaxu2(absmax_bf16x8(v0), absmax_bf16x8(v1)),
+                                 __vmaxu2(absmax_bf16x8(v2), absmax_bf16x8(v3))));
+    }
+    for (; i < nvec; i += stride) m = __vmaxu2(m, absmax_bf16x8(__ldcs(x + i)));
+    uint32_t amax = max(m & 0xFFFFu, m >> 16);
+    if (blockIdx.x == 0)
+        for (int t = threadIdx.x; t < ntail; t += kThreads) amax = max(amax, (uint32_t)(tail[t] & 0x7FFFu));
+    uint32_t flags = amax >= 0x7F80u ? kFlagNonFinite : 0u;
+    if (amax > 0x7F80u) {                              // a NaN: recompute without NaN entries
+        amax = 0u;
+        for (int64_t k = i0; k < nvec; k += stride) amax = max(amax, absmax_bf16x8_no_nan(x[k]));
+        if (blockIdx.x == 0)
+            for (int t = threadIdx.x; t < ntail; t += kThreads) {
+                const uint32_t a = tail[t] & 0x7FFFu;
+                if (a <= 0x7F80u) amax = max(amax, a);
+            }
+    }
+    flags = __reduce_or_sync(0xFFFFFFFFu, flags);
+    if ((threadIdx.x & 31) == 0) flag_or(d_flags, flags);
+    amax = block_max_u32<kThreads>(amax << 16, red);   // BF16 bits -> FP32 bits
+    if (threadIdx.x == 0 && amax != 0u) atomicMax(reinterpret_cast<unsigned int*>(d_amax), amax);
+}
+
+template <int kThreads>
+__global__ void __launch_bounds__(kThreads)
+amax_f32_kernel(const uint4* __restrict__ x, int64_t nvec, const uint32_t* __restrict__ tail, int ntail,
+                float* __restrict__ d_amax, uint32_t* __restrict__ d_flags)
+{
+    __shared__ uint32_t red[kThreads / 32];
+    const int64_t stride = (int64_t)gridDim.x * kThreads;
+    const int64_t i0 = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+    uint32_t m = 0u;
+    int64_t i = i0;
+    for (; i + 1 * stride < nvec; i += 2 * stride) {
+        const uint4 v0 = __ldcs(x + i), v1 = __ldcs(x + i + stride);
+        m = max(m, max(max(v0.x & 0x7FFFFFFFu, v0.y & 0x7FFFFFFFu), max(v0.z & 0x7FFFFFFFu, v0.w & 0x7FFFFFFFu)));
+        m = max(m, max(max(v1.x & 0x7FFFFFFFu, v1.y & 0x7FFFFFFFu), max(v1.z & 0x7FFFFFFFu, v1.w & 0x7FFFFFFFu)));
+    }
+    for (; i < nvec; i += stride) {
+        const uint4 v = __ldcs(x + i);
+        m = max(m, max(max(v.x & 0x7FFFFFFFu, v.y & 0x7FFFFFFFu), max(v.z & 0x7FFFFFFFu, v.w & 0x7FFFFFFFu)));
+    }
+    if (blockIdx.x == 0)
+        for (int t = threadIdx.x; t < ntail; t += kThreads) m = max(m, tail[t] & 0x7FFFFFFFu);
+    uint32_t flags = m >= 0x7F800000u ? kFlagNonFinite : 0u;
+    if (m > 0x7F800000u) {
+        m = 0u;
+        for (int64_t k = i0; k < nvec; k += stride) {
+            const uint4 v = x[k];
+            const uint32_t w[4] = {v.x & 0x7FFFFFFFu, v.y & 0x7FFFFFFFu, v.z & 0x7FFFFFFFu, v.w & 0x7FFFFFFFu};
+            for (int j = 0; j < 4; ++j)
+                if (w[j] <= 0x7F800000u) m = max(m, w[j]);
+        }
+        if (blockIdx.x == 0)
+            for (int t = threadIdx.x; t < ntail; t += kThreads) {
+                const uint32_t a = tail[t] & 0x7FFFFFFFu;
+                if (a <= 0x7F800000u) m = max(m, a);
+            }
+    }
+    flags = __reduce_or_sync(0xFFFFFFFFu, flags);
+    if ((threadIdx.x & 31) == 0) flag_or(d_flags, flags);
+    m = block_max_u32<kThreads>(m, red);
+    if (threadIdx.x == 0 && m != 0u) atomicMax(reinterpret_cast<unsigned int*>(d_amax), m);
+}
+
+// ============================================================== act quant
+// Tables of E4M3 values and their FP32 reciprocals, built per CTA in shared memory.
+struct E4M3Tables {
+    float dec[128];
+    float rcp[128];
+};
+
+__device__ __forceinline__ void fill_e4m3_tables(E4M3Tables& t)
+{
+    for (int c = threadIdx.x; c < 128; c += blockDim.x) {
+        const float v = c < 127 ? e4m3_value((uint32_t)c) : 0.0f;
+        t.dec[c] = v;
+        t.rcp[c] = c > 0 && c < 127 ? __frcp_rn(v) : 0.0f;
+    }
+}
+
+// Quantizes 16 values x[] with block scale S into two words of packed E2M1 codes.
+// r_lo / r_hi bracket 1/S (see nv4_common.cuh); exact == true forces the FP64 path.
+__device__ __forceinline__ void quantize16(const float x[16], float S, float r_lo, float r_hi, bool exact,
+                                           uint32_t& w0, uint32_t& w1)
+{
+    if (!exact) {
+        float lo[16], hi[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            lo[i] = __fmul_rn(x[i], r_lo);
+            hi[i] = __fmul_rn(x[i], r_hi);
+        }
+        w0 = cvt_e2m1x8(lo);
+        w1 = cvt_e2m1x8(lo + 8);
+        const uint32_t h0 = cvt_e2m1x8(hi), h1 = cvt_e2m1x8(hi + 8);
+        if (w0 == h0 && w1 == h1) return;
+    }
+    w0 = w1 = 0u;
+    for (int i = 0; i < 8; ++i) w0 |= e2m1_code_exact(x[i], S) << (4 * i);
+    for (int i = 0; i < 8; ++i) w1 |= e2m1_code_exact(x[8 + i], S) << (4 * i);
+}
+
+constexpr int kActThreads = 256;
+
+__global__ void __launch_bounds__(kActThreads)
+act_quant_kernel(const uint16_t* __restrict__ x, uint32_t rows, uint32_t bpr, int64_t ld, FastDiv div_bpr,
+                 const float* __restrict__ d_amax, uint8_t* __restrict__ q, uint8_t* __restrict__ scales,
+                 float* __restrict__ d_s2, uint32_t* __restrict__ d_flags)
+{
+    __shared__ E4M3Tables tab;
+    fill_e4m3_tables(tab);
+    __syncthreads();
+
+    const float amax = *d_amax;
+    const float s2 = __fdiv_rn(amax, 2688.0f);                  // RN32(amax / (6*448))
+    if (blockIdx.x == 0 && threadIdx.x == 0) *d_s2 = s2;
+    const bool fast_scale = s2 >= kTinyScale && s2 <= 0x1p100f;
+    const float k = __frcp_rn(__fmul_rn(6.0f, s2));             // ~ 1/(6*s2)
+    const float k_lo = __fmul_rn(k, kLoMargin), k_hi = __fmul_rn(k, kHiMargin);
+    const float rs2 = __frcp_rn(s2);                            // ~ 1/s2
+    uint32_t flags = isfinite(s2) ? 0u : kFlagOverflow;
+
+    const uint32_t total = rows * bpr;
+    for (uint32_t u = blockIdx.x * kActThreads + threadIdx.x; u < total; u += gridDim.x * kActThreads) {
+        const uint32_t r = div_bpr.div(u), b = u - r * bpr;
+        const uint4* src = reinterpret_cast<const uint4*>(x + (int64_t)r * ld + 16u * b);
+        const uint4 v0 = __ldcs(src), v1 = __ldcs(src + 1);
+        const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+
+        uint32_t m = 0u;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) m = __vmaxu2(m, w[j] & 0x7FFF7FFFu);
+        const uint32_t ab = max(m & 0xFFFFu, m >> 16);
+        if (ab >= 0x7F80u) flags |= kFlagNonFinite;
+        const float a_b = __uint_as_float(ab << 16);
+
+        // block scale: nearest E4M3 to a_b / (6*s2)
+        uint32_t code;
+        if (fast_scale) {
+            const uint32_t cc = cvt_e4m3x2(__fmul_rn(a_b, k_lo), __fmul_rn(a_b, k_hi));
+            code = (cc & 0xFFu) == (cc >> 8) ? (cc & 0xFFu) : e4m3_code_exact(a_b, s2);
+        } else {
+            code = e4m3_code_exact(a_b, s2);
+        }
+        code &= 0x7Fu;                                            // non-negative inputs only
+        const float S = __fmul_rn(tab.dec[code], s2);            // DQ1: RN32(s_b * s2)
+
+        float xv[16];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            xv[2 * j] = bf16_lo(w[j]);
+            xv[2 * j + 1] = bf16_hi(w[j]);
+        }
+        const bool exact = !(S >= kTinyScale && S <= 0x1p100f);
+        const float rr = __fmul_rn(tab.rcp[code], rs2);          // ~ 1/S
+        uint32_t q0, q1;
+        quantize16(xv, S, __fmul_rn(rr, kLoMargin), __fmul_rn(rr, kHiMargin), exact, q0, q1);
+
+        *reinterpret_cast<uint2*>(q + (int64_t)u * 8) = make_uint2(q0, q1);
+        scales[u] = (uint8_t)code;
+    }
+    flags = __reduce_or_sync(__activemask(), flags);
+    if ((threadIdx.x & 31) == 0) flag_or(d_flags, flags);
+}
+
+// ============================================================== dequant
+__device__ __forceinline__ float e4m3_value_signed(uint32_t c)
+{
+    if ((c & 0x7Fu) == 0x7Fu) return __uint_as_float(0x7FC00000u);
+    const float v = e4m3_value(c & 0x7Fu);
+    return (c & 0x80u) ? -v : v;
+}
+
+template <int kOut>   // 0 bf16, 1 fp16, 2 fp32
+__global__ void __launch_bounds__(kActThreads)
+dequant_kernel(const uint8_t* __restrict__ q, const uint8_t* __restrict__ scales, const float* __restrict__ d_s2,
+               uint32_t total, void* __restrict__ out)
+{
+    const float s2 = *d_s2;
+    for (uint32_t u = blockIdx.x * kActThreads + threadIdx.x; u < total; u += gridDim.x * kActThreads) {
+        const uint2 qv = __ldcs(reinterpret_cast<const uint2*>(q) + u);
+        const float S = __fmul_rn(e4m3_value_signed(scales[u]), s2);   // DQ1
+        uint32_t h[8];
+        cvt_e2m1x8_to_f16x8(qv.x, h);
+        cvt_e2m1x8_to_f16x8(qv.y, h + 4);
+        float y[16];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            float a, b;
+            f16x2_to_f32(h[j], a, b);
+            y[2 * j] = __fmul_rn(a, S);                                  // DQ2: RN32(v * S)
+            y[2 * j + 1] = __fmul_rn(b, S);
+        }
+        if constexpr (kOut == 2) {
+            float4* o = reinterpret_cast<float4*>(out) + (int64_t)u * 4;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) __stcs(o + j, make_float4(y[4 * j], y[4 * j + 1], y[4 * j + 2], y[4 * j + 3]));
+        } else {
+            uint32_t p[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                if constexpr (kOut == 0) {
+                    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(p[j]) : "f"(y[2 * j + 1]), "f"(y[2 * j]));
+                } else {
+                    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(p[j]) : "f"(y[2 * j + 1]), "f"(y[2 * j]));
+                }
+            }
+            uint4* o = reinterpret_cast<uint4*>(out) + (int64_t)u * 2;
+            __stcs(o, make_uint4(p[0], p[1], p[2], p[3]));
+            __stcs(o + 1, make_uint4(p[4], p[5], p[6], p[7]));
+        }
+    }
+}
+
+// ============================================================== launchers
+static int grid_for(int64_t work, int threads, int per_sm)
+{
+    const int64_t need = (work + threads - 1) / threads;
+    const int64_t cap = (int64_t)num_sms() * per_sm;
+    return (int)(need < cap ? (need > 0 ? need : 1) : cap);
+}
+
+cudaError_t launch_amax(const void* x, int dt, int64_t n, float* d_amax, uint32_t* d_flags, cudaStream_t s)
+{
+    constexpr int T = 512;
+    if (dt == 0) {
+        const int64_t nvec = n / 8;
+        const int ntail = (int)(n - nvec * 8);
+        const uint16_t* tail = static_cast<const uint16_t*>(x) + nvec * 8;
+        amax_bf16_kernel<T><<<grid_for(nvec, T, 4), T, 0, s>>>(static_cast<const uint4*>(x), nvec, tail, ntail,
+                                                                 d_amax, d_flags);
+    } else {
+        const int64_t nvec = n / 4;
+        const int ntail = (int)(n - nvec * 4);
+        const uint32_t* tail = static_cast<const uint32_t*>(x) + nvec * 4;
+        amax_f32_kernel<T><<<grid_for(nvec, T, 4), T, 0, s>>>(static_cast<const uint4*>(x), nvec, tail, ntail,
+                                                                d_amax, d_flags);
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_act_quant(const void* x, int64_t rows, int64_t cols, int64_t ld, const float* d_amax,
+                             uint8_t* q, uint8_t* scales, float* d_s2, uint32_t* d_flags, cudaStream_t s)
+{
+    const uint32_t bpr = (uint32_t)(cols / 16);
+    const uint32_t total = (uint32_t)rows * bpr;
+    act_quant_kernel<<<grid_for(total, kActThreads, 8), kActThreads, 0, s>>>(
+        static_cast<const uint16_t*>(x), (uint32_t)rows, bpr, ld, FastDiv(bpr), d_amax, q, scales, d_s2, d_flags);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_dequant(const uint8_t* q, const uint8_t* scales, const float* d_s2, int64_t rows, int64_t cols,
+                           int out_dt, void* out, cudaStream_t s)
+{
+    const uint32_t total = (uint32_t)(rows * (cols / 16));
+    const int g = grid_for(total, kActThreads, 8);
+    if (out_dt == 0) dequant_kernel<0><<<g, kActThreads, 0, s>>>(q, scales, d_s2, total, out);
+    else if (out_dt == 1) dequant_kernel<1><<<g, kActThreads, 0, s>>>(q, scales, d_s2, total, out);
+    else dequant_kernel<2><<<g, kActThreads, 0, s>>>(q, scales, d_s2, total, out);
+    return cudaGetLastError();
+}
+
+}  // namespace nv4

@@ -1,0 +1,95 @@
+"""CPU-only checks of the C-ABI library: it loads, exports every entry point that
+include/nv4.h declares, and rejects bad arguments before touching the GPU."""
+import ctypes as C
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def nv4lib():
+    from nvfp4_block_numerics_b200.build import build_library
+    from nvfp4_block_numerics_b200 import binding
+
+    build_library()
+    return binding.lib()
+
+
+def declared_symbols():
+    txt = open(os.path.join(ROOT, "include", "nv4.h")).read()
+    return sorted(set(re.findall(r"^NV4_API\s+[\w\s\*]+?\b(nv4_\w+)\(", txt, flags=re.M)))
+
+
+def test_header_declares_the_hot_path():
+    names = declared_symbols()
+    for n in ("nv4_tensor_amax", "nv4_act_quant", "nv4_dequant", "nv4_hessian_accum", "nv4_scale_sweep",
+              "nv4_mxfp4_to_nvfp4"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(nv4lib):
+    from nvfp4_block_numerics_b200.build import LIB_PATH
+
+    out = subprocess.run(["nm", "-D", "--defined-only", LIB_PATH], capture_output=True, text=True, check=True).stdout
+    exported = set(re.findall(r"\sT\s+(\w+)$", out, flags=re.M))
+    for n in declared_symbols():
+        assert n in exported, n
+        assert getattr(nv4lib, n) is not None
+    # nothing else leaks out of the library
+    assert {e for e in exported if not e.startswith("nv4_")} <= {"_init", "_fini"}
+
+
+def test_status_strings_and_version(nv4lib):
+    assert nv4lib.nv4_version() == 100
+    for s in range(7):
+        assert nv4lib.nv4_status_str(s).startswith(b"NV4_")
+
+
+def test_validation_rejects_before_any_launch(nv4lib):
+    L = nv4lib
+    fake = 0x1000  # never dereferenced: every call below fails validation first
+    assert L.nv4_act_quant(fake, 4, 24, 24, fake, fake, fake, fake, None, None) == 2      # cols % 16
+    assert L.nv4_act_quant(fake, 4, 32, 16, fake, fake, fake, fake, None, None) == 2      # ld < cols
+    assert L.nv4_act_quant(fake + 2, 4, 32, 32, fake, fake, fake, fake, None, None) == 3  # misaligned x
+    assert L.nv4_act_quant(fake, 4, 32, 36, fake, fake, fake, fake, None, None) == 3      # ld*2 % 16
+    assert L.nv4_act_quant(None, 4, 32, 32, fake, fake, fake, fake, None, None) == 1
+    assert L.nv4_tensor_amax(fake, 1, 16, fake, None, None) == 4                           # fp16 unsupported
+    assert L.nv4_tensor_amax(fake, 0, -1, fake, None, None) == 2
+    assert L.nv4_tensor_amax(fake, 0, 0, fake, None, None) == 0                            # no-op
+    assert L.nv4_dequant(fake, fake, fake, 2, 32, 7, fake, None) == 4
+    assert L.nv4_hessian_accum(fake, 10, 40, 40, fake, None, None) == 2
+    assert L.nv4_hessian_accum(fake, 10, 32, 36, fake, None, None) == 3
+    assert L.nv4_scale_sweep(fake, 2, 4, 32, 34, fake, fake, fake, None, None, None, None, None) == 3  # fp32 ld*4
+    assert L.nv4_scale_sweep(fake, 1, 4, 32, 32, fake, fake, fake, None, None, None, None, None) == 4  # fp16 w
+    assert L.nv4_mxfp4_to_nvfp4(fake, fake, 4, 48, fake, fake, fake, fake, None, None, None) == 2     # cols % 32
+    # overlapping but not identical nibble buffers are rejected
+    assert L.nv4_mxfp4_to_nvfp4(fake, fake, 4, 64, fake + 16, fake, fake, fake, None, None, None) == 2
+    from nvfp4_block_numerics_b200 import binding as b
+
+    jobs = (b.HessianJob * 129)()
+    assert L.nv4_hessian_accum_batched(jobs, 129, None, None) == 6                         # > 128 jobs
+
+
+def fastdiv_params(d):
+    s = 0
+    while (1 << s) < d:
+        s += 1
+    m = ((1 << 32) * ((1 << s) - d)) // d + 1
+    return m & 0xFFFFFFFF, s
+
+
+@pytest.mark.parametrize("d", [1, 2, 3, 7, 16, 90, 128, 256, 448, 1000, 4097, 65535, 123457, 2 ** 31 - 1])
+def test_fastdiv_formula(d):
+    """The device's n / d = (mulhi(n, m) + n) >> s (Granlund-Montgomery), mirrored here."""
+    m, s = fastdiv_params(d)
+    rng = np.random.default_rng(d)
+    ns = np.concatenate([rng.integers(0, 2 ** 32, 20000, dtype=np.uint64),
+                         np.array([0, 1, d - 1, d, d + 1, 2 ** 32 - 1, (2 ** 32 - 1) // d * d], dtype=np.uint64)])
+    for n in ns.tolist():
+        q = (((n * m) >> 32) + n) >> s
+        assert q == n // d, (n, d)

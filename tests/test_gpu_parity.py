@@ -1,0 +1,330 @@
+"""GPU parity of every libnv4 entry point against the CPU oracle.
+
+Small, ragged cases are compared element by element; the workloads' full sizes
+run in the same launch configuration as the benchmark and are compared on
+sampled rows (or in full where the oracle is fast enough).  Rules: integer and
+byte outputs bit-exact; H within 1e-5 relative Frobenius of the FP64 oracle;
+sweep codes bit-exact outside near ties (< 0.1% of blocks may differ).
+"""
+import numpy as np
+import pytest
+import torch
+
+import gpu_util as G
+from nvfp4_block_numerics_b200 import binding as nv4
+from nvfp4_block_numerics_b200 import inputs
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    nv4.lib()
+
+
+# ------------------------------------------------------------------ self-test
+def test_selftest_conversions():
+    out = torch.zeros(64, dtype=torch.int32, device=G.DEV)
+    nv4.nv4_selftest(out)
+    v = out.cpu().numpy().view(np.uint32)
+    print("selftest:", [hex(int(x)) for x in v[:10]])
+    assert v[0] == 0, [hex(int(x)) for x in v[:10]]
+
+
+# ------------------------------------------------------------------ amax
+@pytest.mark.parametrize("n", [1, 7, 8, 9, 1000, 4096 + 5, 1 << 20])
+def test_amax_bf16_sizes(orc, n):
+    x = inputs.laplace_bf16(inputs.rng_for(n, "gpu", "amax"), 1, n, outlier_channels=(n // 2,), outlier_scale=70)
+    a = nv4.tensor_amax(G.bf16_dev(x.reshape(-1)))
+    assert a.item() == orc.tensor_amax(x)[0]
+
+
+def test_amax_f32_running_max_and_flags(orc):
+    w = (np.random.default_rng(1).standard_normal(12345) * 0.02).astype(np.float32)
+    d = torch.zeros(1, dtype=torch.float32, device=G.DEV)
+    f = G.flags_dev()
+    nv4.nv4_tensor_amax(G.f32_dev(w[:5000]), d, f)
+    nv4.nv4_tensor_amax(G.f32_dev(w[5000:]), d, f)          # running max across batches
+    assert d.item() == orc.tensor_amax(w)[0] and f.item() == 0
+    wn = w.copy()
+    wn[77] = np.nan
+    d2 = torch.zeros(1, dtype=torch.float32, device=G.DEV)
+    nv4.nv4_tensor_amax(G.f32_dev(wn), d2, f)
+    assert d2.item() == orc.tensor_amax(wn)[0] and f.item() & nv4.FLAG_NONFINITE
+    xb = inputs.f32_to_bf16_bits(w)
+    xb[3] = 0x7FC0
+    f3 = G.flags_dev()
+    d3 = nv4.tensor_amax(G.bf16_dev(xb), d_flags=f3)
+    assert d3.item() == orc.tensor_amax(xb)[0] and f3.item() & nv4.FLAG_NONFINITE
+
+
+# ------------------------------------------------------------------ act quant / dequant
+def _act_check(orc, x_bits, amax=None, rows_sample=None, ld_pad=0):
+    rows, cols = x_bits.shape
+    xs = x_bits
+    if ld_pad:
+        xs = np.zeros((rows, cols + ld_pad), np.uint16)
+        xs[:, :cols] = x_bits
+    xd = G.bf16_dev(xs)[:, :cols]
+    f = G.flags_dev()
+    if amax is None:
+        d_amax = nv4.tensor_amax(G.bf16_dev(x_bits))
+        amax = orc.tensor_amax(x_bits)[0]
+        assert d_amax.item() == amax
+    else:
+        d_amax = torch.tensor([amax], dtype=torch.float32, device=G.DEV)
+    q, sc, s2 = nv4.act_quant(xd, d_amax, d_flags=f)
+    outs = {dt: nv4.dequant(q, sc, s2, dt) for dt in (torch.bfloat16, torch.float16, torch.float32)}
+    torch.cuda.synchronize()
+    idx = np.arange(rows) if rows_sample is None else rows_sample
+    xr = np.ascontiguousarray(x_bits[idx])
+    oq, osc, os2, of = orc.act_quant(xr, amax)
+    assert s2.item() == os2 and f.item() == of
+    qg, scg = G.host(q)[idx], G.host(sc)[idx]
+    assert np.array_equal(scg, osc), np.argwhere(scg != osc)[:5]
+    assert np.array_equal(qg, oq), np.argwhere(qg != oq)[:5]
+    for dt, name in ((torch.bfloat16, "bf16"), (torch.float16, "fp16"), (torch.float32, "fp32")):
+        ref = orc.dequant(oq, osc, os2, name)
+        got = G.host(outs[dt])[idx]
+        if name == "fp32":
+            got, ref = got.view(np.uint32), ref.view(np.uint32)
+        assert np.array_equal(got, ref), name
+
+
+@pytest.mark.parametrize("rows,cols,pad", [(1, 16, 0), (3, 48, 8), (37, 96, 0), (130, 272, 16), (5, 2048, 0)])
+def test_act_quant_small_ragged(orc, rows, cols, pad):
+    x = inputs.laplace_bf16(inputs.rng_for(rows * cols, "gpu", "act"), rows, cols, outlier_channels=(1,),
+                            outlier_scale=50, zero_block_frac=0.05)
+    _act_check(orc, x, ld_pad=pad)
+
+
+def test_act_quant_tiny_config(orc):
+    _act_check(orc, inputs.c1_tiny_linear(0)["X"])
+
+
+def test_act_quant_edge_values(orc):
+    S = 1.0  # amax 2688 -> s2 = 1
+    g = [0.0, 0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 6.0, 7.0, -0.0, -0.25, -0.75, -5.0, 1e-30, -1e-30]
+    rows = [g, [v * 0.5 for v in g], [448.0 * 6] + [0.0] * 15, [-0.0] * 16, [3.0] * 16]
+    x = inputs.f32_to_bf16_bits(np.array(rows, np.float32))
+    _act_check(orc, x, amax=2688.0 * S)
+    _act_check(orc, x, amax=0.0)            # s2 = 0: sign-only codes
+    _act_check(orc, x, amax=1.0)            # calibrated amax below the data: saturation
+
+
+@pytest.mark.parametrize("T,C", inputs.C2_SHAPES)
+def test_act_quant_config_shapes(orc, T, C):
+    x = inputs.c2_shape(T, C)
+    sample = None if T <= 4096 else np.sort(np.random.default_rng(T + C).choice(T, 512, replace=False))
+    _act_check(orc, x, rows_sample=sample)
+
+
+def test_dequant_random_codes(orc):
+    rng = np.random.default_rng(3)
+    q = rng.integers(0, 256, (33, 40), dtype=np.uint8)
+    sc = rng.integers(0, 127, (33, 5), dtype=np.uint8)
+    for s2 in (0.0123, 1.0, 3.3e-3, 2.0 ** -130, 1e30):
+        s2 = float(np.float32(s2))
+        d_s2 = torch.tensor([s2], dtype=torch.float32, device=G.DEV)
+        for dt, name in ((torch.bfloat16, "bf16"), (torch.float16, "fp16"), (torch.float32, "fp32")):
+            got = G.host(nv4.dequant(G.u8_dev(q), G.u8_dev(sc), d_s2, dt))
+            ref = orc.dequant(q, sc, s2, name)
+            if name == "fp32":
+                got, ref = got.view(np.uint32), ref.view(np.uint32)
+            assert np.array_equal(got, ref), (s2, name)
+
+
+# ------------------------------------------------------------------ Hessian
+def _hess_check(orc, x_bits, ld_pad=0, tol=1e-5):
+    T, K = x_bits.shape
+    xs = x_bits
+    if ld_pad:
+        xs = np.zeros((T, K + ld_pad), np.uint16)
+        xs[:, :K] = x_bits
+    xd = G.bf16_dev(xs)[:, :K]
+    f = G.flags_dev()
+    H = nv4.hessian_accum(xd, d_flags=f)
+    ref = orc.hessian_accum(x_bits)
+    Hg = G.host(H).reshape(ref.shape)
+    assert f.item() == 0
+    rel = G.hessian_rel_err(Hg, ref)
+    blk = max(G.hessian_rel_err(Hg[b], ref[b]) for b in range(ref.shape[0]))
+    print(f"H {T}x{K}: rel Frobenius {rel:.2e}, worst block {blk:.2e}")
+    assert rel <= tol
+    return H, ref
+
+
+@pytest.mark.parametrize("T,K,pad", [(1, 16, 0), (63, 48, 8), (64, 64, 0), (1000, 80, 0), (4097, 272, 8)])
+def test_hessian_small_ragged(orc, T, K, pad):
+    x = inputs.laplace_bf16(inputs.rng_for(T * K, "gpu", "H"), T, K, outlier_channels=(2,), outlier_scale=30)
+    _hess_check(orc, x, ld_pad=pad)
+
+
+def test_hessian_accumulates_and_is_deterministic(orc):
+    x = inputs.c1_tiny_linear(0)["X"]
+    xd = G.bf16_dev(x)
+    H1 = nv4.hessian_accum(xd)
+    H2 = nv4.hessian_accum(xd)
+    assert torch.equal(H1, H2)                      # bit-reproducible
+    nv4.hessian_accum(xd, H1)                       # += semantics
+    ref = orc.hessian_accum(x)
+    assert G.hessian_rel_err(G.host(H1).reshape(ref.shape), 2 * ref) <= 1e-5
+
+
+def test_hessian_gemma_layer_full(orc):
+    d = inputs.c3_layer(0, which=("X",))
+    _hess_check(orc, d["X"])
+
+
+def test_hessian_gemma_down_full(orc):
+    d = inputs.c3_layer(0, which=("X_down",))
+    _hess_check(orc, d["X_down"])
+
+
+def test_hessian_moe_batched(orc):
+    xs, Hs, refs = [], [], []
+    for e in range(64):
+        d = inputs.c4_expert(e, which=("X", "X_down"))
+        for name in ("X", "X_down"):
+            xs.append(G.bf16_dev(d[name]))
+            Hs.append(torch.zeros((d[name].shape[1] // 16, 16, 16), dtype=torch.float32, device=G.DEV))
+            if e in (0, 31, 63):
+                refs.append((len(xs) - 1, d[name]))
+    f = G.flags_dev()
+    nv4.nv4_hessian_accum_batched(xs, Hs, f)
+    torch.cuda.synchronize()
+    assert f.item() == 0
+    for i, xb in refs:
+        ref = orc.hessian_accum(xb)
+        assert G.hessian_rel_err(G.host(Hs[i]).reshape(ref.shape), ref) <= 1e-5
+
+
+# ------------------------------------------------------------------ sweep
+def _sweep_check(orc, w, H64, rows_sample=None):
+    """w: float32 or uint16 (bf16 bits) host array; H64: float64 oracle Hessian."""
+    H32 = H64.astype(np.float32)
+    Hin = H32.astype(np.float64)                    # both sides consume the same FP32 H
+    wd = G.f32_dev(w) if w.dtype == np.float32 else G.bf16_dev(w)
+    d_amax = nv4.tensor_amax(wd)
+    amax = orc.tensor_amax(w)[0]
+    assert d_amax.item() == amax
+    f = G.flags_dev()
+    codes, q, c1, c2 = nv4.scale_sweep(wd, G.f32_dev(H32), d_amax, d_flags=f)
+    torch.cuda.synchronize()
+    assert f.item() == 0
+    ref = orc.scale_sweep(w, Hin, amax, rows=rows_sample)
+    idx = ref["rows"]
+    stats = G.sweep_parity(G.host(codes)[idx], G.host(q)[idx], G.host(c1)[idx], ref)
+    print("sweep", w.shape, stats)
+    assert stats["mismatch_frac"] < 1e-3
+    return stats
+
+
+def test_sweep_tiny_config(orc):
+    d = inputs.c1_tiny_linear(0)
+    _sweep_check(orc, d["W"], orc.hessian_accum(d["X"]))
+
+
+@pytest.mark.parametrize("rows,cols", [(1, 16), (3, 48), (129, 80), (300, 256)])
+def test_sweep_small_ragged(orc, rows, cols):
+    r = np.random.default_rng(rows * cols)
+    w = (r.standard_normal((rows, cols)) * 0.02).astype(np.float32)
+    x = inputs.laplace_bf16(inputs.rng_for(cols, "gpu", "sweepX"), 200, cols, outlier_channels=(1,), outlier_scale=20)
+    H = orc.hessian_accum(x)
+    _sweep_check(orc, w, H)
+    _sweep_check(orc, inputs.f32_to_bf16_bits(w), H)
+
+
+def test_sweep_degenerate_blocks(orc):
+    w = np.zeros((4, 32), np.float32)
+    w[1, :16] = 0.5
+    w[2, 16:] = np.array([0, .5, 1, 1.5, 2, 3, 4, 6] * 2, np.float32) * np.float32(0.25)
+    w[3, 16:] = -0.0
+    H = np.stack([np.eye(16), np.zeros((16, 16))])
+    _sweep_check(orc, w, H)
+
+
+def test_sweep_gemma_layer_sampled(orc):
+    d = inputs.c3_layer(0)
+    H = orc.hessian_accum(d["X"])
+    Hd = orc.hessian_accum(d["X_down"])
+    rng = np.random.default_rng(5)
+    for name, HH in (("W_q", H), ("W_gate", H), ("W_up", H), ("W_down", Hd)):
+        w = d[name]
+        rows = np.sort(rng.choice(w.shape[0], 48, replace=False))
+        _sweep_check(orc, w, HH, rows_sample=rows)
+
+
+def test_sweep_moe_batched_sampled(orc):
+    jobs, checks = [], []
+    rng = np.random.default_rng(6)
+    for e in range(64):
+        d = inputs.c4_expert(e)
+        Hx = orc.hessian_accum(d["X"]) if e in (0, 40) else None
+        Hxd = orc.hessian_accum(d["X_down"]) if e in (0, 40) else None
+        for name, HX in (("W_gate", Hx), ("W_up", Hx), ("W_down", Hxd)):
+            w = d[name]
+            H32 = (HX if HX is not None else np.broadcast_to(np.eye(16), (w.shape[1] // 16, 16, 16))).astype(np.float32)
+            wd = G.bf16_dev(w)
+            amax = nv4.tensor_amax(wd)
+            rows, cols = w.shape
+            job = dict(w=wd, H=G.f32_dev(H32), d_amax_w=amax,
+                       codes=torch.empty((rows, cols // 16), dtype=torch.uint8, device=G.DEV),
+                       q=torch.empty((rows, cols // 2), dtype=torch.uint8, device=G.DEV),
+                       cost1=torch.empty((rows, cols // 16), dtype=torch.float32, device=G.DEV),
+                       cost2=torch.empty((rows, cols // 16), dtype=torch.float32, device=G.DEV))
+            jobs.append(job)
+            if HX is not None:
+                checks.append((job, w, H32.astype(np.float64)))
+    f = G.flags_dev()
+    nv4.nv4_scale_sweep_batched(jobs, f)
+    torch.cuda.synchronize()
+    assert f.item() == 0
+    for job, w, Hin in checks:
+        rows = np.sort(rng.choice(w.shape[0], 24, replace=False))
+        ref = orc.scale_sweep(w, Hin, orc.tensor_amax(w)[0], rows=rows)
+        st = G.sweep_parity(G.host(job["codes"])[rows], G.host(job["q"])[rows], G.host(job["cost1"])[rows], ref)
+        assert st["mismatch_frac"] < 1e-3
+
+
+# ------------------------------------------------------------------ cast
+def _cast_check(orc, mats, in_place=False):
+    jobs, refs = [], []
+    counts = torch.zeros(3, dtype=torch.int64, device=G.DEV)
+    f = G.flags_dev()
+    for mxq, e8 in mats:
+        mq = G.u8_dev(mxq)
+        rows, half = mxq.shape
+        jobs.append(dict(mx_q=mq, e8m0=G.u8_dev(e8), nv_q=mq if in_place else torch.empty_like(mq),
+                         nv_scales=torch.empty((rows, half // 8), dtype=torch.uint8, device=G.DEV),
+                         d_global_amax=torch.empty(1, dtype=torch.float32, device=G.DEV),
+                         d_s2=torch.empty(1, dtype=torch.float32, device=G.DEV)))
+        refs.append(orc.mxfp4_to_nvfp4(mxq, e8))
+    nv4.nv4_mxfp4_to_nvfp4_batched(jobs, counts, f)
+    torch.cuda.synchronize()
+    assert f.item() == 0
+    tot = np.zeros(3, np.int64)
+    for j, r in zip(jobs, refs):
+        assert np.array_equal(G.host(j["nv_q"]), r["nv_q"])
+        assert np.array_equal(G.host(j["nv_scales"]), r["nv_scales"])
+        assert j["d_global_amax"].item() == r["global_amax"] and j["d_s2"].item() == r["s2"]
+        tot += r["counts"]
+    assert np.array_equal(counts.cpu().numpy(), tot)
+    return tot
+
+
+def test_cast_small_and_edges(orc):
+    mats = [inputs.mxfp4_matrix(inputs.rng_for(i, "gpu", "cast"), r, c, fallback_frac=0.05)
+            for i, (r, c) in enumerate([(1, 32), (3, 64), (17, 96), (64, 256)])]
+    e = np.array([[127, 127 - 17, 127 - 18, 124]], np.uint8)
+    mats.append((np.full((1, 64), 0x77, np.uint8), e))
+    _cast_check(orc, mats)
+    _cast_check(orc, mats, in_place=True)
+
+
+def test_cast_expert_checkpoint_full(orc):
+    mats = [inputs.c5_cast(i) for i in range(32)]
+    tot = _cast_check(orc, mats)
+    print("cast counts (in-window, fallback, lossless):", tot.tolist(), "lossless fraction", tot[2] / (tot[0] + tot[1]))
+    _cast_check(orc, mats, in_place=True)

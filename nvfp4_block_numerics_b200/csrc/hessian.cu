@@ -351,8 +351,16 @@ cudaError_t launch_hessian(const nv4_hessian_job* jobs, int n, uint32_t* d_flags
     while (z < (uint32_t)kMaxCluster && slabs * z < target && max_tiles / (2u * z) >= 8u) z *= 2u;
 
     const size_t smem = hess_smem_bytes();
-    cudaError_t e = cudaFuncSetAttribute(hessian_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    // once per device (outside any stream capture in practice: the first call sets it)
+    static bool attr_set[64] = {false};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+        e = cudaFuncSetAttribute(hessian_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        if (dev >= 0 && dev < 64) attr_set[dev] = true;
+    }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(z, slabs, 1);
     cfg.blockDim = dim3(kHThreads, 1, 1);

@@ -19,7 +19,9 @@ Distributions (stand-ins for data that is not available here):
 """
 from __future__ import annotations
 
+import os
 import zlib
+from concurrent.futures import ThreadPoolExecutor
 
 import numpy as np
 
@@ -34,6 +36,30 @@ def rng_for(seed: int, workload: str, name: str) -> np.random.Generator:
     """Independent generator per (seed, workload, tensor name)."""
     key = zlib.crc32(f"{workload}/{name}".encode())
     return np.random.default_rng(np.random.SeedSequence([seed, key]))
+
+
+_CHUNK = 1 << 22          # elements per independently seeded chunk
+_THREADS = max(1, min(32, (os.cpu_count() or 1)))
+
+
+def _chunked(rng: np.random.Generator, rows: int, cols: int, fill, out: np.ndarray):
+    """Fill out[rows, cols] chunk by chunk; chunk k draws from its own child generator
+    (spawned from rng), so the result does not depend on the number of threads."""
+    rows_per = max(1, _CHUNK // max(cols, 1))
+    bounds = [(r, min(rows, r + rows_per)) for r in range(0, rows, rows_per)]
+    children = rng.spawn(len(bounds)) if bounds else []
+
+    def run(k):
+        r0, r1 = bounds[k]
+        out[r0:r1] = fill(children[k], r1 - r0, r0)
+
+    if len(bounds) > 1 and _THREADS > 1:
+        with ThreadPoolExecutor(_THREADS) as ex:
+            list(ex.map(run, range(len(bounds))))
+    else:
+        for k in range(len(bounds)):
+            run(k)
+    return out
 
 
 def f32_to_bf16_bits(a: np.ndarray) -> np.ndarray:
@@ -56,32 +82,41 @@ def _laplace_f32(rng: np.random.Generator, shape, b: float) -> np.ndarray:
 
 def laplace_bf16(rng: np.random.Generator, rows: int, cols: int, b: float = 1.0,
                  outlier_channels=(), outlier_scale: float = 1.0,
-                 zero_block_frac: float = 0.0, chunk_rows: int = 4096) -> np.ndarray:
+                 zero_block_frac: float = 0.0) -> np.ndarray:
     """BF16 bits [rows, cols]: Laplace(b) rows, listed channels scaled, and a fraction of
-    (row, 16-element block) pairs set to +0.0.  Generated in row chunks to bound memory."""
-    out = np.empty((rows, cols), np.uint16)
+    (row, 16-element block) pairs set to +0.0."""
     oc = np.asarray(list(outlier_channels), dtype=np.int64)
-    for r0 in range(0, rows, chunk_rows):
-        r1 = min(rows, r0 + chunk_rows)
-        v = _laplace_f32(rng, (r1 - r0, cols), b)
+
+    def fill(r, n, _r0):
+        v = _laplace_f32(r, (n, cols), b)
         if oc.size:
             v[:, oc] *= np.float32(outlier_scale)
         if zero_block_frac > 0.0:
             nb = cols // 16
-            z = rng.random((r1 - r0, nb)) < zero_block_frac
-            v.reshape(r1 - r0, nb, 16)[z] = 0.0
-        out[r0:r1] = f32_to_bf16_bits(v)
-    return out
+            z = r.random((n, nb)) < zero_block_frac
+            v.reshape(n, nb, 16)[z] = 0.0
+        return f32_to_bf16_bits(v)
+
+    return _chunked(rng, rows, cols, fill, np.empty((rows, cols), np.uint16))
 
 
 def normal_weights(rng: np.random.Generator, rows: int, cols: int, std: float) -> np.ndarray:
-    return (rng.standard_normal((rows, cols), dtype=np.float32) * np.float32(std))
+    def fill(r, n, _r0):
+        return r.standard_normal((n, cols), dtype=np.float32) * np.float32(std)
+
+    return _chunked(rng, rows, cols, fill, np.empty((rows, cols), np.float32))
 
 
-def student_t_weights(rng: np.random.Generator, rows: int, cols: int, std: float, nu: float = 4.0):
-    """Student-t(nu) scaled to the given standard deviation (t_nu has variance nu/(nu-2))."""
-    t = rng.standard_t(nu, size=(rows, cols)).astype(np.float32)
-    return t * np.float32(std / np.sqrt(nu / (nu - 2.0)))
+def student_t_weights(rng: np.random.Generator, rows: int, cols: int, std: float) -> np.ndarray:
+    """Student-t with 4 degrees of freedom scaled to the given standard deviation.
+    t_4 = Z / sqrt(V/4) with V ~ chi-square(4) = 2*(E1 + E2), E exponential(1); Var(t_4) = 2."""
+    def fill(r, n, _r0):
+        z = r.standard_normal((n, cols), dtype=np.float32)
+        e = r.standard_exponential((n, cols), dtype=np.float32)
+        e += r.standard_exponential((n, cols), dtype=np.float32)
+        return z * np.sqrt(np.float32(2.0) / e) * np.float32(std / np.sqrt(2.0))
+
+    return _chunked(rng, rows, cols, fill, np.empty((rows, cols), np.float32))
 
 
 def mxfp4_matrix(rng: np.random.Generator, rows: int, cols: int, mean_exp: float = -8.0,

@@ -252,7 +252,7 @@ def kernel_rooflines(W, hbm_peak):
         out["dequant"] = {"bound": "hbm", "bytes": ACT_BYTES["dequant"] * n, "s": t}
         for k in ("tensor_amax", "act_quant", "dequant"):
             out[k]["launch"] = f"[{big['T']}, {big['C']}] bf16"
-    if "calib" in W:
+    if "weights" in W:
         Xd = W["Xd"]
         t = time_launch(lambda: nv4.nv4_hessian_accum(Xd, W["Hd"], W["flags"]), reps=10, flush=flush)
         out["hessian_accum"] = {"bound": "hbm", "bytes": 2.0 * Xd.numel(), "s": t,

@@ -39,6 +39,7 @@ constexpr int kConsumerWarps = 4;
 constexpr int kHThreads = (kConsumerWarps + 1) * 32;
 constexpr uint32_t kTileBytes = kTok * kSlab * 2;
 constexpr int kMaxCluster = 8;
+constexpr uint32_t kChunkTiles = 8;     // tiles per FP32 accumulation chunk
 
 struct HessJobDev {
     CUtensorMap tmap;                    // X as [tokens][cols] bf16, box 64x64, swizzle 128B
@@ -194,13 +195,15 @@ hessian_kernel(const __grid_constant__ HessParams p)
     }
     __syncthreads();
 
-    float acc[4][2][4];
+    // acc: the MMA accumulators of the current chunk of kChunkTiles tiles; tot: the sum
+    // of the chunks.  Each FP32 chain thus adds at most 16*kChunkTiles token products.
+    float acc[4][2][4], tot[4][2][4];
 #pragma unroll
     for (int bk = 0; bk < 4; ++bk)
 #pragma unroll
         for (int h = 0; h < 2; ++h)
 #pragma unroll
-            for (int k = 0; k < 4; ++k) acc[bk][h][k] = 0.0f;
+            for (int k = 0; k < 4; ++k) acc[bk][h][k] = tot[bk][h][k] = 0.0f;
 
     if (warp == kConsumerWarps) {
         // ---------------- producer: one lane issues the TMA loads
@@ -246,8 +249,25 @@ hessian_kernel(const __grid_constant__ HessParams p)
                 mbar_arrive(&sm.empty[s]);
                 if (warp == 0) atomicMax(&sm.consumed, i + 1u);
             }
+            if ((i + 1u) % kChunkTiles == 0u) {
+#pragma unroll
+                for (int bk = 0; bk < 4; ++bk)
+#pragma unroll
+                    for (int h = 0; h < 2; ++h)
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            tot[bk][h][k] += acc[bk][h][k];
+                            acc[bk][h][k] = 0.0f;
+                        }
+            }
             if (*reinterpret_cast<volatile uint32_t*>(&sm.timeout)) break;
         }
+#pragma unroll
+        for (int bk = 0; bk < 4; ++bk)
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+                for (int k = 0; k < 4; ++k) tot[bk][h][k] += acc[bk][h][k];
     }
     __syncthreads();
 
@@ -261,10 +281,10 @@ hessian_kernel(const __grid_constant__ HessParams p)
             for (int h = 0; h < 2; ++h) {
                 float* P = part + (warp * 4 + bk) * 256;
                 const int n0 = 8 * h + 2 * c;
-                P[g * 16 + n0] = acc[bk][h][0];
-                P[g * 16 + n0 + 1] = acc[bk][h][1];
-                P[(g + 8) * 16 + n0] = acc[bk][h][2];
-                P[(g + 8) * 16 + n0 + 1] = acc[bk][h][3];
+                P[g * 16 + n0] = tot[bk][h][0];
+                P[g * 16 + n0 + 1] = tot[bk][h][1];
+                P[(g + 8) * 16 + n0] = tot[bk][h][2];
+                P[(g + 8) * 16 + n0 + 1] = tot[bk][h][3];
             }
     }
     __syncthreads();

@@ -284,40 +284,63 @@ def kernel_rooflines(W, hbm_peak):
 
 def e2e_act(W, steps):
     """The act part end to end through the public API: pinned host inputs copied in,
-    amax -> quantize -> dequantize, packed codes, scales and BF16 output copied back."""
+    amax -> quantize -> dequantize, packed codes, scales and BF16 output copied back.
+    Copy-in, compute and copy-out run on three streams, ordered per shape by events,
+    so the transfers of one shape overlap the kernels of its neighbours."""
     import torch
 
     from nvfp4_block_numerics_b200 import binding as nv4
 
-    dev = W["flags"].device
     hx = [torch.from_numpy(s["host"].view(np.int16)).view(torch.bfloat16).pin_memory() for s in W["act"]]
     hq = [torch.empty(tuple(s["q"].shape), dtype=torch.uint8).pin_memory() for s in W["act"]]
     hs = [torch.empty(tuple(s["sc"].shape), dtype=torch.uint8).pin_memory() for s in W["act"]]
     ho = [torch.empty(tuple(s["out"].shape), dtype=torch.bfloat16).pin_memory() for s in W["act"]]
     h2d = sum(t.numel() * 2 for t in hx)
     d2h = sum(t.numel() for t in hq) + sum(t.numel() for t in hs) + sum(t.numel() * 2 for t in ho)
+    s_in, s_cmp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    n = len(W["act"])
+    done = [None] * n      # compute finished (x may be overwritten)
+    drained = [None] * n   # copy-out finished (q, sc, out may be overwritten)
 
     def one():
-        W["amax_act"].zero_()
         for i, s in enumerate(W["act"]):
-            s["x"].copy_(hx[i], non_blocking=True)
-            a, s2 = W["amax_act"][i:i + 1], W["s2_act"][i:i + 1]
-            nv4.nv4_tensor_amax(s["x"], a, W["flags"])
-            nv4.nv4_act_quant(s["x"], a, s["q"], s["sc"], s2, W["flags"])
-            nv4.nv4_dequant(s["q"], s["sc"], s2, s["out"])
-            hq[i].copy_(s["q"], non_blocking=True)
-            hs[i].copy_(s["sc"], non_blocking=True)
-            ho[i].copy_(s["out"], non_blocking=True)
+            with torch.cuda.stream(s_in):
+                if done[i] is not None:
+                    s_in.wait_event(done[i])
+                s["x"].copy_(hx[i], non_blocking=True)
+                ready = torch.cuda.Event()
+                ready.record(s_in)
+            with torch.cuda.stream(s_cmp):
+                s_cmp.wait_event(ready)
+                if drained[i] is not None:
+                    s_cmp.wait_event(drained[i])
+                a, s2 = W["amax_act"][i:i + 1], W["s2_act"][i:i + 1]
+                a.zero_()
+                nv4.nv4_tensor_amax(s["x"], a, W["flags"], s_cmp)
+                nv4.nv4_act_quant(s["x"], a, s["q"], s["sc"], s2, W["flags"], s_cmp)
+                nv4.nv4_dequant(s["q"], s["sc"], s2, s["out"], s_cmp)
+                done[i] = torch.cuda.Event()
+                done[i].record(s_cmp)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(done[i])
+                hq[i].copy_(s["q"], non_blocking=True)
+                hs[i].copy_(s["sc"], non_blocking=True)
+                ho[i].copy_(s["out"], non_blocking=True)
+                drained[i] = torch.cuda.Event()
+                drained[i].record(s_out)
 
     one()
-    torch.cuda.synchronize(dev)
+    torch.cuda.synchronize()
     a = torch.cuda.Event(enable_timing=True)
     b = torch.cuda.Event(enable_timing=True)
-    a.record()
+    a.record(s_in)
     for _ in range(steps):
         one()
-    b.record()
+    for ev in drained:
+        s_out.wait_event(ev)
+    b.record(s_out)
     b.synchronize()
+    torch.cuda.synchronize()
     return a.elapsed_time(b) / 1e3 / steps, h2d, d2h
 
 

@@ -112,6 +112,7 @@ NV4_API nv4_status nv4_tensor_amax(const void* x, nv4_dtype dt, int64_t n, float
  * d_amax : device float (e.g. the output of nv4_tensor_amax), read on the device.
  * q      : [rows, cols/2] bytes, contiguous.   scales : [rows, cols/16] E4M3 bytes.
  * d_s2   : device float receiving s2.
+ * Limit: rows * cols/16 < 2^30 blocks per call (NV4_ERR_LIMIT beyond).
  */
 NV4_API nv4_status nv4_act_quant(const void* x, int64_t rows, int64_t cols, int64_t ld,
                          const float* d_amax, uint8_t* q, uint8_t* scales, float* d_s2,
@@ -121,8 +122,9 @@ NV4_API nv4_status nv4_act_quant(const void* x, int64_t rows, int64_t cols, int6
  * nv4_dequant -- the two-step dequantization of [FLOW] 3.4 / 5.4:
  *   DQ1: S = RN32(s_b * s2);  DQ2: y = RN32(e2m1(code) * S), then rounded to out_dt
  *   (NV4_BF16 default, NV4_FP16, or NV4_FP32 as is), ties to even, overflow to inf.
- * q [rows, cols/2], scales [rows, cols/16], d_s2 device float; out [rows, cols]
- * contiguous, 16-byte aligned.  cols % 16 == 0.
+ * q [rows, cols/2], scales [rows, cols/16] (both 16-byte aligned), d_s2 device float; out [rows, cols]
+ * contiguous, 16-byte aligned.  cols % 16 == 0.  Limit: rows * cols/16 < 2^30 blocks
+ * per call (NV4_ERR_LIMIT beyond).
  */
 NV4_API nv4_status nv4_dequant(const uint8_t* q, const uint8_t* scales, const float* d_s2,
                        int64_t rows, int64_t cols, nv4_dtype out_dt, void* out, void* stream);

@@ -114,7 +114,7 @@ nv4_status nv4_act_quant(const void* x, int64_t rows, int64_t cols, int64_t ld, 
     if (rows == 0 || cols == 0) return NV4_OK;
     if (x == nullptr || q == nullptr || scales == nullptr) return NV4_ERR_NULL;
     if (!aligned16(x) || !aligned16(q) || ld % 8 != 0) return NV4_ERR_ALIGN;
-    if (rows * (cols / 16) >= (int64_t)1 << 32) return NV4_ERR_LIMIT;
+    if (rows * (cols / 16) >= (int64_t)1 << 30) return NV4_ERR_LIMIT;
     return from_cuda(launch_act_quant(x, rows, cols, ld, d_amax, q, scales, d_s2, d_flags, (cudaStream_t)stream));
 }
 
@@ -125,8 +125,8 @@ nv4_status nv4_dequant(const uint8_t* q, const uint8_t* scales, const float* d_s
     if (out_dt != NV4_BF16 && out_dt != NV4_FP16 && out_dt != NV4_FP32) return NV4_ERR_DTYPE;
     if (rows == 0 || cols == 0) return NV4_OK;
     if (q == nullptr || scales == nullptr || d_s2 == nullptr || out == nullptr) return NV4_ERR_NULL;
-    if (!aligned16(q) || !aligned16(out)) return NV4_ERR_ALIGN;
-    if (rows * (cols / 16) >= (int64_t)1 << 32) return NV4_ERR_LIMIT;
+    if (!aligned16(q) || !aligned16(scales) || !aligned16(out)) return NV4_ERR_ALIGN;
+    if (rows * (cols / 16) >= (int64_t)1 << 30) return NV4_ERR_LIMIT;
     return from_cuda(launch_dequant(q, scales, d_s2, rows, cols, (int)out_dt, out, (cudaStream_t)stream));
 }
 

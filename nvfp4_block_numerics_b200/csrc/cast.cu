@@ -10,15 +10,16 @@
 // CTA reduces the largest E8M0 code of its share of the matrix (and keeps that share
 // in shared memory); the cluster exchanges the partial maxima through distributed
 // shared memory, so k_max needs no second launch and no scratch memory.  Phase 2:
-// one thread per MX block writes the two E4M3 scale bytes and, out of place, copies
-// the 16 nibble bytes with 128-bit loads and stores.
+// each thread takes eight consecutive MX blocks per step, writes their sixteen E4M3
+// scale bytes with one 128-bit store and, out of place, copies the 128 nibble bytes
+// with 128-bit streaming loads and stores (all eight loads in flight together).
 #include "nv4_common.cuh"
 #include "nv4_internal.h"
 
 namespace nv4 {
 
-constexpr int kCastThreads = 512;
-constexpr int kCastCluster = 8;
+constexpr int kCastThreads = 256;
+constexpr int kCastCluster = 16;                 // non-portable cluster size (opted in at launch)
 constexpr uint32_t kCastSmemCodes = 32768;       // cached E8M0 bytes per CTA
 
 struct CastJobDev {
@@ -29,7 +30,6 @@ struct CastJobDev {
     float* d_ga;
     float* d_s2;
     uint32_t rows, nmx;                           // nmx = cols / 32
-    FastDiv div_nmx;
 };
 
 struct CastParams {
@@ -111,7 +111,30 @@ __device__ __noinline__ uint32_t cast_fallback16(const uint32_t nib_words[2], in
     return code;
 }
 
-__global__ void __launch_bounds__(kCastThreads)
+// A block whose E8M0 code is NaN (nibbles copied, scales 0; flagged in phase 1) or lies
+// outside the window (re-quantized).  Returns the two scale bytes; adds to the fallback
+// and lossless counters.
+__device__ __noinline__ uint32_t cast_rare_block(const uint8_t* __restrict__ mx_q, uint8_t* __restrict__ nv_q,
+                                                 uint32_t g, uint32_t c, int k_max, float s2, bool copy,
+                                                 uint32_t* n_fb, uint32_t* n_ll)
+{
+    const uint4 qv = *reinterpret_cast<const uint4*>(mx_q + (int64_t)g * 16);
+    if (c == 0xFFu) {
+        if (copy) *reinterpret_cast<uint4*>(nv_q + (int64_t)g * 16) = qv;
+        return 0u;
+    }
+    const int k = (int)c - 127;
+    const uint32_t lo_words[2] = {qv.x, qv.y}, hi_words[2] = {qv.z, qv.w};
+    uint32_t out_lo[2], out_hi[2], ll0, ll1;
+    const uint32_t s_lo = cast_fallback16(lo_words, k, s2, out_lo, &ll0);
+    const uint32_t s_hi = cast_fallback16(hi_words, k, s2, out_hi, &ll1);
+    *reinterpret_cast<uint4*>(nv_q + (int64_t)g * 16) = make_uint4(out_lo[0], out_lo[1], out_hi[0], out_hi[1]);
+    *n_fb += 2u;
+    *n_ll += ll0 + ll1;
+    return s_lo | (s_hi << 8);
+}
+
+__global__ void __launch_bounds__(kCastThreads, 3)
 cast_kernel(const __grid_constant__ CastParams p)
 {
     __shared__ alignas(16) uint8_t codes[kCastSmemCodes];
@@ -134,19 +157,34 @@ cast_kernel(const __grid_constant__ CastParams p)
     {
         const uint32_t nvec = (g1 - g0) / 16u;
         const uint4* src = reinterpret_cast<const uint4*>(job.e8m0 + g0);
-        for (uint32_t v = threadIdx.x; v < nvec; v += kCastThreads) {
-            const uint4 w = __ldcs(src + v);
-            if (cached) reinterpret_cast<uint4*>(codes)[v] = w;
+        auto scan = [&](const uint4& w) {
             const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
+                // bytes equal to 0xFF are NaN codes: flag them and keep them out of the max
+                const uint32_t nan = __vcmpeq4(ws[k], 0xFFFFFFFFu);
+                if (nan) flags |= kFlagE8M0Nan;
+                mx = max(mx, __vmaxu4(ws[k] & ~nan, 0u) );
+            }
+        };
+        uint32_t v = threadIdx.x;
+        for (; v + 3u * kCastThreads < nvec; v += 4u * kCastThreads) {   // four loads in flight
+            uint4 w[4];
 #pragma unroll
-                for (int b = 0; b < 4; ++b) {
-                    const uint32_t c = (ws[k] >> (8 * b)) & 0xFFu;
-                    if (c == 0xFFu) flags |= kFlagE8M0Nan; else mx = max(mx, c);
-                }
+            for (int k = 0; k < 4; ++k) w[k] = __ldcs(src + v + k * kCastThreads);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                if (cached) reinterpret_cast<uint4*>(codes)[v + k * kCastThreads] = w[k];
+                scan(w[k]);
             }
         }
+        for (; v < nvec; v += kCastThreads) {
+            const uint4 w = __ldcs(src + v);
+            if (cached) reinterpret_cast<uint4*>(codes)[v] = w;
+            scan(w);
+        }
+        // the four byte maxima of mx -> one
+        mx = max(max(mx & 0xFFu, (mx >> 8) & 0xFFu), max((mx >> 16) & 0xFFu, mx >> 24));
         for (uint32_t g = g0 + nvec * 16u + threadIdx.x; g < g1; g += kCastThreads) {
             const uint32_t c = job.e8m0[g];
             if (cached) codes[g - g0] = (uint8_t)c;
@@ -162,9 +200,13 @@ cast_kernel(const __grid_constant__ CastParams p)
         cta_max = m;
     }
     cluster_sync_c();
-    uint32_t kcode = 0u;
-    for (uint32_t r = 0; r < kCastCluster; ++r) kcode = max(kcode, ld_dsmem_u32(&cta_max, r));
+    if (threadIdx.x < 32) {                                         // one warp gathers the partial maxima
+        uint32_t v = threadIdx.x < kCastCluster ? ld_dsmem_u32(&cta_max, threadIdx.x) : 0u;
+        v = __reduce_max_sync(0xFFFFFFFFu, v);
+        if (threadIdx.x == 0) red[0] = v;
+    }
     cluster_sync_c();                                               // all remote reads done
+    const uint32_t kcode = red[0];
 
     const int k_max = (int)kcode - 127, m = k_max - 8;
     const float s2 = exp2_exact(m);                                 // m in [-135, 119]
@@ -175,40 +217,63 @@ cast_kernel(const __grid_constant__ CastParams p)
         if (!isfinite(ga)) flags |= kFlagOverflow;
     }
 
-    // ---------------- phase 2: one thread per MX block
+    // ---------------- phase 2: MX block g covers nibble bytes [16g, 16g+16) and scale
+    // bytes [2g, 2g+2) of the matrix (both arrays are row-major and contiguous), so the
+    // share is walked linearly, eight blocks per thread per step.  In-window blocks are
+    // the common case; NaN-coded and fallback blocks go through cast_rare_block.
     const bool copy = job.nv_q != job.mx_q;
     uint32_t n_in = 0u, n_fb = 0u, n_ll = 0u;
-    for (uint32_t g = g0 + threadIdx.x; g < g1; g += kCastThreads) {
-        const uint32_t c = cached ? codes[g - g0] : job.e8m0[g];
-        const uint32_t r = job.div_nmx.div(g), jb = g - r * job.nmx;
-        const int64_t qoff = ((int64_t)r * job.nmx + jb) * 16;      // 16 nibble bytes per MX block
-        uint16_t sc2;
-        if (c == 0xFFu) {
-            sc2 = 0;                                                // flagged in phase 1
-            if (copy) *reinterpret_cast<uint4*>(job.nv_q + qoff) = *reinterpret_cast<const uint4*>(job.mx_q + qoff);
-        } else {
-            const int k = (int)c - 127, d = k_max - k;
-            if (d <= 17) {
-                const uint32_t sc = e4m3_code_pow2(8 - d);
-                sc2 = (uint16_t)(sc | (sc << 8));
-                if (copy)
-                    __stcs(reinterpret_cast<uint4*>(job.nv_q + qoff), __ldcs(reinterpret_cast<const uint4*>(job.mx_q + qoff)));
+    const uint32_t n8 = (g1 - g0) / 8u;                             // g0 is a multiple of 16
+    for (uint32_t t = threadIdx.x; t < n8; t += kCastThreads) {
+        const uint32_t g = g0 + 8u * t;
+        const uint2 cw = cached ? reinterpret_cast<const uint2*>(codes)[t]
+                                : *reinterpret_cast<const uint2*>(job.e8m0 + g);
+        uint4 qv[8];
+        if (copy) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) qv[i] = __ldcs(reinterpret_cast<const uint4*>(job.mx_q + (int64_t)(g + i) * 16));
+        }
+        uint32_t sw[4] = {0u, 0u, 0u, 0u}, rare = 0u;                // scale bytes, 4 per word
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const uint32_t c = ((i < 4 ? cw.x : cw.y) >> (8 * (i & 3))) & 0xFFu;
+            const int d = k_max - ((int)c - 127);
+            if (c != 0xFFu && d <= 17) {
+                const uint32_t e = e4m3_code_pow2(8 - d);
+                sw[i >> 1] |= (e | (e << 8)) << (16 * (i & 1));
+                if (copy) __stcs(reinterpret_cast<uint4*>(job.nv_q + (int64_t)(g + i) * 16), qv[i]);
                 n_in += 2u;
-                n_ll += 2u;
             } else {
-                const uint4 qv = *reinterpret_cast<const uint4*>(job.mx_q + qoff);
-                const uint32_t lo_words[2] = {qv.x, qv.y}, hi_words[2] = {qv.z, qv.w};
-                uint32_t out_lo[2], out_hi[2], ll0, ll1;
-                const uint32_t s_lo = cast_fallback16(lo_words, k, s2, out_lo, &ll0);
-                const uint32_t s_hi = cast_fallback16(hi_words, k, s2, out_hi, &ll1);
-                *reinterpret_cast<uint4*>(job.nv_q + qoff) = make_uint4(out_lo[0], out_lo[1], out_hi[0], out_hi[1]);
-                sc2 = (uint16_t)(s_lo | (s_hi << 8));
-                n_fb += 2u;
-                n_ll += ll0 + ll1;
+                rare |= 1u << i;
             }
         }
-        *reinterpret_cast<uint16_t*>(job.nv_scales + ((int64_t)r * job.nmx + jb) * 2) = sc2;
+        if (rare) {                                                 // after the copies: nothing else live
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                if (rare & (1u << i)) {
+                    const uint32_t c = ((i < 4 ? cw.x : cw.y) >> (8 * (i & 3))) & 0xFFu;
+                    const uint32_t v = cast_rare_block(job.mx_q, job.nv_q, g + i, c, k_max, s2, copy, &n_fb, &n_ll);
+                    sw[i >> 1] |= v << (16 * (i & 1));
+                }
+        }
+        __stcs(reinterpret_cast<uint4*>(job.nv_scales + (int64_t)g * 2), make_uint4(sw[0], sw[1], sw[2], sw[3]));
     }
+    for (uint32_t g = g0 + 8u * n8 + threadIdx.x; g < g1; g += kCastThreads) {
+        const uint32_t c = cached ? codes[g - g0] : job.e8m0[g];
+        const int d = k_max - ((int)c - 127);
+        uint32_t sc;
+        if (c != 0xFFu && d <= 17) {
+            const uint32_t e = e4m3_code_pow2(8 - d);
+            sc = e | (e << 8);
+            if (copy)
+                *reinterpret_cast<uint4*>(job.nv_q + (int64_t)g * 16) = *reinterpret_cast<const uint4*>(job.mx_q + (int64_t)g * 16);
+            n_in += 2u;
+        } else {
+            sc = cast_rare_block(job.mx_q, job.nv_q, g, c, k_max, s2, copy, &n_fb, &n_ll);
+        }
+        *reinterpret_cast<uint16_t*>(job.nv_scales + (int64_t)g * 2) = (uint16_t)sc;
+    }
+    n_ll += n_in;                                                   // in-window blocks are lossless
 
     // ---------------- counters and flags
     n_in = __reduce_add_sync(0xFFFFFFFFu, n_in);
@@ -241,10 +306,18 @@ cudaError_t launch_cast(const nv4_cast_job* jobs, int n, unsigned long long* d_c
         d.d_ga = J.d_global_amax; d.d_s2 = J.d_s2;
         d.rows = (uint32_t)J.rows;
         d.nmx = (uint32_t)(J.cols / 32);
-        d.div_nmx = FastDiv(d.nmx);
     }
     p.n = m;
     if (m == 0) return cudaSuccess;
+    static bool attr_set[64] = {false};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+        e = cudaFuncSetAttribute(cast_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        if (e != cudaSuccess) return e;
+        if (dev >= 0 && dev < 64) attr_set[dev] = true;
+    }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(m * kCastCluster), 1, 1);
     cfg.blockDim = dim3(kCastThreads, 1, 1);
@@ -257,7 +330,7 @@ cudaError_t launch_cast(const nv4_cast_job* jobs, int n, unsigned long long* d_c
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, cast_kernel, p);
+    e = cudaLaunchKernelEx(&cfg, cast_kernel, p);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }

@@ -145,6 +145,46 @@ static __device__ __noinline__ uint32_t e2m1_code_exact(float x, float S)
     return sign | k;
 }
 
+// ---------------------------------------------------------------- exact fix-ups (FP32)
+// When the two ends of a bracket convert to different codes, the quotient lies
+// within ~2^-19 of exactly one rounding boundary, so the two codes are adjacent and
+// one comparison decides.  fma(b, D, -a) rounds the exact b*D - a once, so its sign
+// is exact, and it is zero only on an exact tie (no underflow: D >= 2^-100 on these
+// paths and the operands agree to ~19 bits).
+
+// Boundary between E2M1 magnitudes k and k+1: 0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.
+__device__ __forceinline__ float e2m1_boundary(uint32_t k)
+{
+    const uint64_t quarters = 0x00140E0A07050301ull;    // 4 x boundary, one byte per k
+    return (float)((uint32_t)(quarters >> (8u * k)) & 0xFFu) * 0.25f;
+}
+
+// Corrects the packed codes lo (8 elements x[0..7], element i in bits 4i..4i+3) at
+// every nibble where the bracket's other end hi disagrees; S is the block scale.
+__device__ __forceinline__ uint32_t e2m1_fix8(const float x[8], float S, uint32_t lo, uint32_t hi)
+{
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const uint32_t cl = (lo >> (4 * i)) & 15u, ch = (hi >> (4 * i)) & 15u;
+        if (cl != ch) {
+            const uint32_t kl = cl & 7u;
+            const float d = fmaf(e2m1_boundary(kl), S, -fabsf(x[i]));
+            const uint32_t k = d < 0.0f ? kl + 1u : (d > 0.0f ? kl : kl + (kl & 1u));
+            lo = (lo & ~(15u << (4 * i))) | ((k | (cl & 8u)) << (4 * i));
+        }
+    }
+    return lo;
+}
+
+// E4M3 block-scale code when the bracket gave codes c and c+1 for a / (6*s2):
+// compares a with the midpoint times 6*s2 ((v_c + v_c+1) * 3 has <= 7 bits: exact).
+__device__ __forceinline__ uint32_t e4m3_fix(uint32_t c, float a, float s2)
+{
+    const float mid6 = (e4m3_value(c) + e4m3_value(c + 1u)) * 3.0f;
+    const float d = fmaf(mid6, s2, -a);
+    return d < 0.0f ? c + 1u : (d > 0.0f ? c : c + (c & 1u));
+}
+
 // ---------------------------------------------------------------- time / waits
 __device__ __forceinline__ uint64_t global_ns()
 {

@@ -4,7 +4,7 @@
 #include <cstdint>
 #include <cuda_runtime.h>
 
-#include "../../include/nv4.h"
+#include "nv4.h"
 
 namespace nv4 {
 

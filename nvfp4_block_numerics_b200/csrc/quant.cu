@@ -144,21 +144,28 @@ __device__ __forceinline__ void fill_e4m3_tables(E4M3Tables& t)
 }
 
 // Quantizes 16 values x[] with block scale S into two words of packed E2M1 codes.
-// r_lo / r_hi bracket 1/S (see nv4_common.cuh); exact == true forces the FP64 path.
+// r_lo / r_hi bracket 1/S (see nv4_common.cuh); exact == true forces the FP64 path
+// (only for a block scale outside [2^-100, 2^100]).  S == 0 passes r_lo = r_hi = 0:
+// the products keep the sign of x and convert to sign-only codes.
 __device__ __forceinline__ void quantize16(const float x[16], float S, float r_lo, float r_hi, bool exact,
                                            uint32_t& w0, uint32_t& w1)
 {
     if (!exact) {
         float lo[16], hi[16];
+        const float2 rl = make_float2(r_lo, r_lo), rh = make_float2(r_hi, r_hi);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            lo[i] = __fmul_rn(x[i], r_lo);
-            hi[i] = __fmul_rn(x[i], r_hi);
+        for (int i = 0; i < 16; i += 2) {
+            const float2 xv = make_float2(x[i], x[i + 1]);
+            const float2 a = __fmul2_rn(xv, rl), b = __fmul2_rn(xv, rh);
+            lo[i] = a.x; lo[i + 1] = a.y;
+            hi[i] = b.x; hi[i + 1] = b.y;
         }
         w0 = cvt_e2m1x8(lo);
         w1 = cvt_e2m1x8(lo + 8);
         const uint32_t h0 = cvt_e2m1x8(hi), h1 = cvt_e2m1x8(hi + 8);
-        if (w0 == h0 && w1 == h1) return;
+        if (w0 != h0) w0 = e2m1_fix8(x, S, w0, h0);
+        if (w1 != h1) w1 = e2m1_fix8(x + 8, S, w1, h1);
+        return;
     }
     w0 = w1 = 0u;
     for (int i = 0; i < 8; ++i) w0 |= e2m1_code_exact(x[i], S) << (4 * i);
@@ -186,10 +193,21 @@ act_quant_kernel(const uint16_t* __restrict__ x, uint32_t rows, uint32_t bpr, in
     uint32_t flags = isfinite(s2) ? 0u : kFlagOverflow;
 
     const uint32_t total = rows * bpr;
-    for (uint32_t u = blockIdx.x * kActThreads + threadIdx.x; u < total; u += gridDim.x * kActThreads) {
-        const uint32_t r = div_bpr.div(u), b = u - r * bpr;
-        const uint4* src = reinterpret_cast<const uint4*>(x + (int64_t)r * ld + 16u * b);
-        const uint4 v0 = __ldcs(src), v1 = __ldcs(src + 1);
+    const uint32_t stride = gridDim.x * kActThreads;
+    // software pipeline: the next block's two 128-bit loads are in flight while this
+    // block is quantized
+    auto load = [&](uint32_t u, uint4& a, uint4& b) {
+        const uint32_t r = div_bpr.div(u), bb = u - r * bpr;
+        const uint4* src = reinterpret_cast<const uint4*>(x + (int64_t)r * ld + 16u * bb);
+        a = __ldcs(src);
+        b = __ldcs(src + 1);
+    };
+    uint32_t u = blockIdx.x * kActThreads + threadIdx.x;
+    uint4 n0 = make_uint4(0u, 0u, 0u, 0u), n1 = n0;
+    if (u < total) load(u, n0, n1);
+    for (; u < total; u += stride) {
+        const uint4 v0 = n0, v1 = n1;
+        if (u + stride < total) load(u + stride, n0, n1);
         const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
 
         uint32_t m = 0u;
@@ -203,7 +221,8 @@ act_quant_kernel(const uint16_t* __restrict__ x, uint32_t rows, uint32_t bpr, in
         uint32_t code;
         if (fast_scale) {
             const uint32_t cc = cvt_e4m3x2(__fmul_rn(a_b, k_lo), __fmul_rn(a_b, k_hi));
-            code = (cc & 0xFFu) == (cc >> 8) ? (cc & 0xFFu) : e4m3_code_exact(a_b, s2);
+            code = cc & 0xFFu;
+            if (code != (cc >> 8)) code = e4m3_fix(code, a_b, s2);
         } else {
             code = e4m3_code_exact(a_b, s2);
         }
@@ -216,8 +235,8 @@ act_quant_kernel(const uint16_t* __restrict__ x, uint32_t rows, uint32_t bpr, in
             xv[2 * j] = bf16_lo(w[j]);
             xv[2 * j + 1] = bf16_hi(w[j]);
         }
-        const bool exact = !(S >= kTinyScale && S <= 0x1p100f);
-        const float rr = __fmul_rn(tab.rcp[code], rs2);          // ~ 1/S
+        const bool exact = S != 0.0f && !(S >= kTinyScale && S <= 0x1p100f);
+        const float rr = S == 0.0f ? 0.0f : __fmul_rn(tab.rcp[code], rs2);   // ~ 1/S
         uint32_t q0, q1;
         quantize16(xv, S, __fmul_rn(rr, kLoMargin), __fmul_rn(rr, kHiMargin), exact, q0, q1);
 
@@ -236,45 +255,63 @@ __device__ __forceinline__ float e4m3_value_signed(uint32_t c)
     return (c & 0x80u) ? -v : v;
 }
 
+// One thread handles eight outputs (half a 16-block): 4 code bytes and the block's
+// scale byte in, 16 (BF16/FP16) or 32 (FP32) bytes out, so a warp reads 128
+// contiguous code bytes and writes 512 or 1024 contiguous output bytes per step.
+template <int kOut>
+__device__ __forceinline__ void dequant8(uint32_t qw, uint32_t sc, float s2, void* __restrict__ out, int64_t h)
+{
+    const float S = __fmul_rn(e4m3_value_signed(sc), s2);      // DQ1: RN32(s_b * s2)
+    uint32_t hv[4];
+    cvt_e2m1x8_to_f16x8(qw, hv);
+    float y[8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        float a, b;
+        f16x2_to_f32(hv[j], a, b);
+        const float2 r = __fmul2_rn(make_float2(a, b), make_float2(S, S));   // DQ2: RN32(v * S)
+        y[2 * j] = r.x;
+        y[2 * j + 1] = r.y;
+    }
+    if constexpr (kOut == 2) {
+        float4* o = reinterpret_cast<float4*>(out) + h * 2;
+        __stcs(o, make_float4(y[0], y[1], y[2], y[3]));
+        __stcs(o + 1, make_float4(y[4], y[5], y[6], y[7]));
+    } else {
+        uint32_t p[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            if constexpr (kOut == 0) {
+                asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(p[j]) : "f"(y[2 * j + 1]), "f"(y[2 * j]));
+            } else {
+                asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(p[j]) : "f"(y[2 * j + 1]), "f"(y[2 * j]));
+            }
+        }
+        __stcs(reinterpret_cast<uint4*>(out) + h, make_uint4(p[0], p[1], p[2], p[3]));
+    }
+}
+
 template <int kOut>   // 0 bf16, 1 fp16, 2 fp32
 __global__ void __launch_bounds__(kActThreads)
 dequant_kernel(const uint8_t* __restrict__ q, const uint8_t* __restrict__ scales, const float* __restrict__ d_s2,
                uint32_t total, void* __restrict__ out)
 {
     const float s2 = *d_s2;
-    for (uint32_t u = blockIdx.x * kActThreads + threadIdx.x; u < total; u += gridDim.x * kActThreads) {
-        const uint2 qv = __ldcs(reinterpret_cast<const uint2*>(q) + u);
-        const float S = __fmul_rn(e4m3_value_signed(scales[u]), s2);   // DQ1
-        uint32_t h[8];
-        cvt_e2m1x8_to_f16x8(qv.x, h);
-        cvt_e2m1x8_to_f16x8(qv.y, h + 4);
-        float y[16];
+    const uint32_t halves = 2u * total;
+    const uint32_t stride = gridDim.x * kActThreads;
+    const uint32_t* qw = reinterpret_cast<const uint32_t*>(q);
+    uint32_t h = blockIdx.x * kActThreads + threadIdx.x;
+    for (; h + 3u * stride < halves; h += 4u * stride) {          // four independent steps in flight
+        uint32_t a[4], c[4];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            float a, b;
-            f16x2_to_f32(h[j], a, b);
-            y[2 * j] = __fmul_rn(a, S);                                  // DQ2: RN32(v * S)
-            y[2 * j + 1] = __fmul_rn(b, S);
+        for (int k = 0; k < 4; ++k) {
+            a[k] = __ldcs(qw + h + k * stride);
+            c[k] = scales[(h + k * stride) >> 1];
         }
-        if constexpr (kOut == 2) {
-            float4* o = reinterpret_cast<float4*>(out) + (int64_t)u * 4;
 #pragma unroll
-            for (int j = 0; j < 4; ++j) __stcs(o + j, make_float4(y[4 * j], y[4 * j + 1], y[4 * j + 2], y[4 * j + 3]));
-        } else {
-            uint32_t p[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                if constexpr (kOut == 0) {
-                    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(p[j]) : "f"(y[2 * j + 1]), "f"(y[2 * j]));
-                } else {
-                    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(p[j]) : "f"(y[2 * j + 1]), "f"(y[2 * j]));
-                }
-            }
-            uint4* o = reinterpret_cast<uint4*>(out) + (int64_t)u * 2;
-            __stcs(o, make_uint4(p[0], p[1], p[2], p[3]));
-            __stcs(o + 1, make_uint4(p[4], p[5], p[6], p[7]));
-        }
+        for (int k = 0; k < 4; ++k) dequant8<kOut>(a[k], c[k], s2, out, h + k * stride);
     }
+    for (; h < halves; h += stride) dequant8<kOut>(__ldcs(qw + h), scales[h >> 1], s2, out, h);
 }
 
 // ============================================================== launchers
@@ -318,7 +355,7 @@ cudaError_t launch_dequant(const uint8_t* q, const uint8_t* scales, const float*
                            int out_dt, void* out, cudaStream_t s)
 {
     const uint32_t total = (uint32_t)(rows * (cols / 16));
-    const int g = grid_for(total, kActThreads, 8);
+    const int g = grid_for((int64_t)total * 2, kActThreads, 8);
     if (out_dt == 0) dequant_kernel<0><<<g, kActThreads, 0, s>>>(q, scales, d_s2, total, out);
     else if (out_dt == 1) dequant_kernel<1><<<g, kActThreads, 0, s>>>(q, scales, d_s2, total, out);
     else dequant_kernel<2><<<g, kActThreads, 0, s>>>(q, scales, d_s2, total, out);

@@ -6,21 +6,23 @@
 //   exactly in E4M3 and the 16 nibble bytes are reused; otherwise the block is
 //   re-quantized from its exact values e2m1 * 2^k_j (rare fallback path).
 //
-// One thread-block cluster of kCastCluster CTAs handles one matrix.  Phase 1: each
-// CTA reduces the largest E8M0 code of its share of the matrix (and keeps that share
-// in shared memory); the cluster exchanges the partial maxima through distributed
-// shared memory, so k_max needs no second launch and no scratch memory.  Phase 2:
-// each thread takes eight consecutive MX blocks per step, writes their sixteen E4M3
-// scale bytes with one 128-bit store and, out of place, copies the 128 nibble bytes
-// with 128-bit streaming loads and stores (all eight loads in flight together).
+// Two stream-ordered kernels, no scratch memory:
+//  1. cast_kmax_kernel: one thread-block cluster of kKmaxCluster CTAs per matrix reads
+//     only the E8M0 bytes, reduces the largest valid code through distributed shared
+//     memory and writes the matrix's outputs s2 = 2^m and global_amax = 6*448*2^m;
+//  2. cast_rewrite_kernel: a flat grid over the MX blocks of every matrix (a warp takes
+//     256 consecutive blocks per step, lane-interleaved so each instruction moves
+//     contiguous bytes) recovers k_max = m + 8 exactly from the s2 it reads back, writes
+//     the two E4M3 scale bytes per block and, out of place, copies the 16 nibble bytes
+//     with 128-bit streaming loads and stores; rare blocks (NaN code, outside the
+//     window) take a separate exact path.
 #include "nv4_common.cuh"
 #include "nv4_internal.h"
 
 namespace nv4 {
 
 constexpr int kCastThreads = 256;
-constexpr int kCastCluster = 16;                 // non-portable cluster size (opted in at launch)
-constexpr uint32_t kCastSmemCodes = 32768;       // cached E8M0 bytes per CTA
+constexpr int kKmaxCluster = 8;                  // CTAs reducing one matrix's largest E8M0 code
 
 struct CastJobDev {
     const uint8_t* mx_q;
@@ -29,11 +31,13 @@ struct CastJobDev {
     uint8_t* nv_scales;
     float* d_ga;
     float* d_s2;
-    uint32_t rows, nmx;                           // nmx = cols / 32
+    uint32_t nb;                                  // MX blocks in the matrix (rows * cols / 32)
+    uint32_t group_begin;                         // prefix sum of 256-block tiles over jobs
 };
 
 struct CastParams {
     int n;
+    uint32_t groups;                              // total 256-block tiles
     unsigned long long* d_counts;
     uint32_t* d_flags;
     CastJobDev jobs[kMaxCastJobs];
@@ -134,62 +138,44 @@ __device__ __noinline__ uint32_t cast_rare_block(const uint8_t* __restrict__ mx_
     return s_lo | (s_hi << 8);
 }
 
-__global__ void __launch_bounds__(kCastThreads, 3)
-cast_kernel(const __grid_constant__ CastParams p)
+// ------------------------------------------------------------------ kernel 1: k_max
+__global__ void __launch_bounds__(kCastThreads)
+cast_kmax_kernel(const __grid_constant__ CastParams p)
 {
-    __shared__ alignas(16) uint8_t codes[kCastSmemCodes];
     __shared__ uint32_t red[kCastThreads / 32];
     __shared__ uint32_t cta_max;
-    __shared__ unsigned long long cnt[3];
-
     const uint32_t rank = cluster_rank_c();
-    const CastJobDev& job = p.jobs[blockIdx.x / kCastCluster];
-    const uint32_t nb = job.rows * job.nmx;                       // MX blocks in the matrix
-    // share of this CTA, 16-aligned so the bulk can move in 16-byte words
-    const uint32_t per = ((nb + kCastCluster - 1) / kCastCluster + 15u) & ~15u;
-    const uint32_t g0 = min(nb, rank * per), g1 = min(nb, g0 + per);
-    const bool cached = (g1 - g0) <= kCastSmemCodes;
+    const CastJobDev& job = p.jobs[blockIdx.x / kKmaxCluster];
+    // share of this CTA, 16-aligned so it moves in 16-byte words
+    const uint32_t per = ((job.nb + kKmaxCluster - 1) / kKmaxCluster + 15u) & ~15u;
+    const uint32_t g0 = min(job.nb, rank * per), g1 = min(job.nb, g0 + per);
 
-    if (threadIdx.x < 3) cnt[threadIdx.x] = 0ull;
-
-    // ---------------- phase 1: largest valid E8M0 code of the share
-    uint32_t mx = 0u, flags = 0u;
-    {
-        const uint32_t nvec = (g1 - g0) / 16u;
-        const uint4* src = reinterpret_cast<const uint4*>(job.e8m0 + g0);
-        auto scan = [&](const uint4& w) {
-            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+    uint32_t mx = 0u, flags = 0u;                                   // four per-byte maxima
+    const uint32_t nvec = (g1 - g0) / 16u;
+    const uint4* src = reinterpret_cast<const uint4*>(job.e8m0 + g0);
+    auto scan = [&](const uint4& w) {
+        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                // bytes equal to 0xFF are NaN codes: flag them and keep them out of the max
-                const uint32_t nan = __vcmpeq4(ws[k], 0xFFFFFFFFu);
-                if (nan) flags |= kFlagE8M0Nan;
-                mx = max(mx, __vmaxu4(ws[k] & ~nan, 0u) );
-            }
-        };
-        uint32_t v = threadIdx.x;
-        for (; v + 3u * kCastThreads < nvec; v += 4u * kCastThreads) {   // four loads in flight
-            uint4 w[4];
+        for (int k = 0; k < 4; ++k) {
+            // bytes equal to 0xFF are NaN codes: flag them and keep them out of the max
+            const uint32_t nan = __vcmpeq4(ws[k], 0xFFFFFFFFu);
+            if (nan) flags |= kFlagE8M0Nan;
+            mx = __vmaxu4(mx, ws[k] & ~nan);
+        }
+    };
+    uint32_t v = threadIdx.x;
+    for (; v + 3u * kCastThreads < nvec; v += 4u * kCastThreads) {  // four loads in flight
+        uint4 w[4];
 #pragma unroll
-            for (int k = 0; k < 4; ++k) w[k] = __ldcs(src + v + k * kCastThreads);
+        for (int k = 0; k < 4; ++k) w[k] = __ldcs(src + v + k * kCastThreads);
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                if (cached) reinterpret_cast<uint4*>(codes)[v + k * kCastThreads] = w[k];
-                scan(w[k]);
-            }
-        }
-        for (; v < nvec; v += kCastThreads) {
-            const uint4 w = __ldcs(src + v);
-            if (cached) reinterpret_cast<uint4*>(codes)[v] = w;
-            scan(w);
-        }
-        // the four byte maxima of mx -> one
-        mx = max(max(mx & 0xFFu, (mx >> 8) & 0xFFu), max((mx >> 16) & 0xFFu, mx >> 24));
-        for (uint32_t g = g0 + nvec * 16u + threadIdx.x; g < g1; g += kCastThreads) {
-            const uint32_t c = job.e8m0[g];
-            if (cached) codes[g - g0] = (uint8_t)c;
-            if (c == 0xFFu) flags |= kFlagE8M0Nan; else mx = max(mx, c);
-        }
+        for (int k = 0; k < 4; ++k) scan(w[k]);
+    }
+    for (; v < nvec; v += kCastThreads) scan(__ldcs(src + v));
+    mx = max(max(mx & 0xFFu, (mx >> 8) & 0xFFu), max((mx >> 16) & 0xFFu, mx >> 24));
+    for (uint32_t g = g0 + nvec * 16u + threadIdx.x; g < g1; g += kCastThreads) {
+        const uint32_t c = job.e8m0[g];
+        if (c == 0xFFu) flags |= kFlagE8M0Nan; else mx = max(mx, c);
     }
     mx = __reduce_max_sync(0xFFFFFFFFu, mx);
     if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mx;
@@ -200,95 +186,107 @@ cast_kernel(const __grid_constant__ CastParams p)
         cta_max = m;
     }
     cluster_sync_c();
-    if (threadIdx.x < 32) {                                         // one warp gathers the partial maxima
-        uint32_t v = threadIdx.x < kCastCluster ? ld_dsmem_u32(&cta_max, threadIdx.x) : 0u;
-        v = __reduce_max_sync(0xFFFFFFFFu, v);
-        if (threadIdx.x == 0) red[0] = v;
+    if (rank == 0 && threadIdx.x < 32) {                           // one warp gathers the partial maxima
+        uint32_t c = threadIdx.x < kKmaxCluster ? ld_dsmem_u32(&cta_max, threadIdx.x) : 0u;
+        c = __reduce_max_sync(0xFFFFFFFFu, c);
+        if (threadIdx.x == 0) {
+            const float s2 = exp2_exact((int)c - 127 - 8);           // m = k_max - 8 in [-135, 119]
+            const float ga = __fmul_rn(2688.0f, s2);                 // 6*448*2^m
+            *job.d_s2 = s2;
+            *job.d_ga = ga;
+            if (!isfinite(ga)) flags |= kFlagOverflow;
+        }
     }
     cluster_sync_c();                                               // all remote reads done
-    const uint32_t kcode = red[0];
+    flags = __reduce_or_sync(0xFFFFFFFFu, flags);
+    if ((threadIdx.x & 31) == 0) flag_or(p.d_flags, flags);
+}
 
-    const int k_max = (int)kcode - 127, m = k_max - 8;
-    const float s2 = exp2_exact(m);                                 // m in [-135, 119]
-    if (rank == 0 && threadIdx.x == 0 && nb > 0) {
-        const float ga = __fmul_rn(2688.0f, s2);                    // 6*448*2^m
-        *job.d_s2 = s2;
-        *job.d_ga = ga;
-        if (!isfinite(ga)) flags |= kFlagOverflow;
-    }
+// m with s2 = 2^m exactly (s2 a power of two, normal or subnormal).
+__device__ __forceinline__ int exact_log2(float s2)
+{
+    const uint32_t b = __float_as_uint(s2);
+    const int e = (int)((b >> 23) & 0xFFu);
+    return e != 0 ? e - 127 : -149 + (31 - __clz(b));
+}
 
-    // ---------------- phase 2: MX block g covers nibble bytes [16g, 16g+16) and scale
-    // bytes [2g, 2g+2) of the matrix (both arrays are row-major and contiguous), so the
-    // share is walked linearly, eight blocks per thread per step.  In-window blocks are
-    // the common case; NaN-coded and fallback blocks go through cast_rare_block.
-    const bool copy = job.nv_q != job.mx_q;
+// ------------------------------------------------------------------ kernel 2: rewrite
+// A warp step covers a tile of 256 consecutive MX blocks of one matrix: lane t takes
+// blocks tile + 32i + t (i = 0..7), so every load and store instruction of the warp
+// moves contiguous bytes (32 code bytes, 512 nibble bytes, 64 scale bytes).
+constexpr uint32_t kTile = 256;
+
+__global__ void __launch_bounds__(kCastThreads)
+cast_rewrite_kernel(const __grid_constant__ CastParams p)
+{
+    const uint32_t lane = threadIdx.x & 31u;
+    const uint32_t warp_id = (blockIdx.x * kCastThreads + threadIdx.x) >> 5;
+    const uint32_t nwarps = (gridDim.x * kCastThreads) >> 5;
     uint32_t n_in = 0u, n_fb = 0u, n_ll = 0u;
-    const uint32_t n8 = (g1 - g0) / 8u;                             // g0 is a multiple of 16
-    for (uint32_t t = threadIdx.x; t < n8; t += kCastThreads) {
-        const uint32_t g = g0 + 8u * t;
-        const uint2 cw = cached ? reinterpret_cast<const uint2*>(codes)[t]
-                                : *reinterpret_cast<const uint2*>(job.e8m0 + g);
-        uint4 qv[8];
-        if (copy) {
-#pragma unroll
-            for (int i = 0; i < 8; ++i) qv[i] = __ldcs(reinterpret_cast<const uint4*>(job.mx_q + (int64_t)(g + i) * 16));
+    for (uint32_t ti = warp_id; ti < p.groups; ti += nwarps) {      // p.groups counts 256-block tiles here
+        int j = 0;
+        {
+            int lo = 0, hi = p.n - 1;
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (p.jobs[mid].group_begin <= ti) lo = mid; else hi = mid - 1;
+            }
+            j = lo;
         }
-        uint32_t sw[4] = {0u, 0u, 0u, 0u}, rare = 0u;                // scale bytes, 4 per word
+        const CastJobDev& job = p.jobs[j];
+        const float s2 = *job.d_s2;
+        const int k_max = exact_log2(s2) + 8;
+        const bool copy = job.nv_q != job.mx_q;
+        const uint32_t base = kTile * (ti - job.group_begin);
+        uint32_t c[8];
+        uint4 qv[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-            const uint32_t c = ((i < 4 ? cw.x : cw.y) >> (8 * (i & 3))) & 0xFFu;
-            const int d = k_max - ((int)c - 127);
-            if (c != 0xFFu && d <= 17) {
+            const uint32_t g = base + 32u * i + lane;
+            c[i] = g < job.nb ? (uint32_t)__ldcs(job.e8m0 + g) : 0u;
+        }
+        if (copy) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const uint32_t g = base + 32u * i + lane;
+                if (g < job.nb) qv[i] = __ldcs(reinterpret_cast<const uint4*>(job.mx_q + (int64_t)g * 16));
+            }
+        }
+        uint32_t rare = 0u;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const uint32_t g = base + 32u * i + lane;
+            if (g >= job.nb) continue;
+            const int d = k_max - ((int)c[i] - 127);
+            if (c[i] != 0xFFu && d <= 17) {
                 const uint32_t e = e4m3_code_pow2(8 - d);
-                sw[i >> 1] |= (e | (e << 8)) << (16 * (i & 1));
-                if (copy) __stcs(reinterpret_cast<uint4*>(job.nv_q + (int64_t)(g + i) * 16), qv[i]);
+                __stcs(reinterpret_cast<unsigned short*>(job.nv_scales + (int64_t)g * 2), (unsigned short)(e | (e << 8)));
+                if (copy) __stcs(reinterpret_cast<uint4*>(job.nv_q + (int64_t)g * 16), qv[i]);
                 n_in += 2u;
             } else {
                 rare |= 1u << i;
             }
         }
-        if (rare) {                                                 // after the copies: nothing else live
+        if (rare) {                                                  // after the copies: nothing else live
 #pragma unroll
             for (int i = 0; i < 8; ++i)
                 if (rare & (1u << i)) {
-                    const uint32_t c = ((i < 4 ? cw.x : cw.y) >> (8 * (i & 3))) & 0xFFu;
-                    const uint32_t v = cast_rare_block(job.mx_q, job.nv_q, g + i, c, k_max, s2, copy, &n_fb, &n_ll);
-                    sw[i >> 1] |= v << (16 * (i & 1));
+                    const uint32_t g = base + 32u * i + lane;
+                    const uint32_t v = cast_rare_block(job.mx_q, job.nv_q, g, c[i], k_max, s2, copy, &n_fb, &n_ll);
+                    *reinterpret_cast<uint16_t*>(job.nv_scales + (int64_t)g * 2) = (uint16_t)v;
                 }
         }
-        __stcs(reinterpret_cast<uint4*>(job.nv_scales + (int64_t)g * 2), make_uint4(sw[0], sw[1], sw[2], sw[3]));
     }
-    for (uint32_t g = g0 + 8u * n8 + threadIdx.x; g < g1; g += kCastThreads) {
-        const uint32_t c = cached ? codes[g - g0] : job.e8m0[g];
-        const int d = k_max - ((int)c - 127);
-        uint32_t sc;
-        if (c != 0xFFu && d <= 17) {
-            const uint32_t e = e4m3_code_pow2(8 - d);
-            sc = e | (e << 8);
-            if (copy)
-                *reinterpret_cast<uint4*>(job.nv_q + (int64_t)g * 16) = *reinterpret_cast<const uint4*>(job.mx_q + (int64_t)g * 16);
-            n_in += 2u;
-        } else {
-            sc = cast_rare_block(job.mx_q, job.nv_q, g, c, k_max, s2, copy, &n_fb, &n_ll);
-        }
-        *reinterpret_cast<uint16_t*>(job.nv_scales + (int64_t)g * 2) = (uint16_t)sc;
-    }
-    n_ll += n_in;                                                   // in-window blocks are lossless
-
-    // ---------------- counters and flags
+    // counters: one set of atomics per warp, no CTA barrier (warps retire independently)
+    n_ll += n_in;                                                    // in-window blocks are lossless
     n_in = __reduce_add_sync(0xFFFFFFFFu, n_in);
     n_fb = __reduce_add_sync(0xFFFFFFFFu, n_fb);
     n_ll = __reduce_add_sync(0xFFFFFFFFu, n_ll);
-    flags = __reduce_or_sync(0xFFFFFFFFu, flags);
-    if ((threadIdx.x & 31) == 0) {
-        if (n_in) atomicAdd(&cnt[0], (unsigned long long)n_in);
-        if (n_fb) atomicAdd(&cnt[1], (unsigned long long)n_fb);
-        if (n_ll) atomicAdd(&cnt[2], (unsigned long long)n_ll);
-        flag_or(p.d_flags, flags);
+    if (lane == 0 && p.d_counts != nullptr) {
+        if (n_in) atomicAdd(p.d_counts + 0, (unsigned long long)n_in);
+        if (n_fb) atomicAdd(p.d_counts + 1, (unsigned long long)n_fb);
+        if (n_ll) atomicAdd(p.d_counts + 2, (unsigned long long)n_ll);
     }
-    __syncthreads();
-    if (threadIdx.x < 3 && p.d_counts != nullptr && cnt[threadIdx.x] != 0ull)
-        atomicAdd(p.d_counts + threadIdx.x, cnt[threadIdx.x]);
 }
 
 cudaError_t launch_cast(const nv4_cast_job* jobs, int n, unsigned long long* d_counts, uint32_t* d_flags,
@@ -298,40 +296,42 @@ cudaError_t launch_cast(const nv4_cast_job* jobs, int n, unsigned long long* d_c
     p.d_counts = d_counts;
     p.d_flags = d_flags;
     int m = 0;
+    uint32_t groups = 0;
     for (int i = 0; i < n; ++i) {
         const nv4_cast_job& J = jobs[i];
         if (J.rows == 0 || J.cols == 0) continue;
         CastJobDev& d = p.jobs[m++];
         d.mx_q = J.mx_q; d.e8m0 = J.e8m0; d.nv_q = J.nv_q; d.nv_scales = J.nv_scales;
         d.d_ga = J.d_global_amax; d.d_s2 = J.d_s2;
-        d.rows = (uint32_t)J.rows;
-        d.nmx = (uint32_t)(J.cols / 32);
+        d.nb = (uint32_t)(J.rows * (J.cols / 32));
+        d.group_begin = groups;
+        groups += (d.nb + kTile - 1u) / kTile;
     }
     p.n = m;
+    p.groups = groups;
     if (m == 0) return cudaSuccess;
-    static bool attr_set[64] = {false};
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= 64 || !attr_set[dev]) {
-        e = cudaFuncSetAttribute(cast_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-        if (e != cudaSuccess) return e;
-        if (dev >= 0 && dev < 64) attr_set[dev] = true;
-    }
+
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(m * kCastCluster), 1, 1);
+    cfg.gridDim = dim3((unsigned)(m * kKmaxCluster), 1, 1);
     cfg.blockDim = dim3(kCastThreads, 1, 1);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = kCastCluster;
+    attr[0].val.clusterDim.x = kKmaxCluster;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, cast_kernel, p);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, cast_kmax_kernel, p);
     if (e != cudaSuccess) return e;
+
+    // a single resident wave (two CTAs per SM at this kernel's register count); warps
+    // stride over the tiles
+    const int64_t need = ((int64_t)groups + kCastThreads / 32 - 1) / (kCastThreads / 32);   // one warp per tile
+    const int64_t cap = (int64_t)num_sms() * 2;
+    const int grid = (int)(need < cap ? (need > 0 ? need : 1) : cap);
+    cast_rewrite_kernel<<<grid, kCastThreads, 0, s>>>(p);
     return cudaGetLastError();
 }
 

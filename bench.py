@@ -212,6 +212,31 @@ PARTS = {"act": part_act, "calib": part_calib, "cast": part_cast}
 LAUNCHES = {"act": 45, "calib": 6, "cast": 1}
 
 
+def traffic_table():
+    """DRAM bytes per launch from profiles/dram_traffic.json, for kernels whose sources
+    still hash to the values recorded with the capture (else the entry is dropped)."""
+    import hashlib
+
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    try:
+        with open(path) as f:
+            doc = json.load(f)
+    except Exception:
+        return {}
+    out = {}
+    for k, e in doc.get("kernels", {}).items():
+        h = hashlib.sha256()
+        try:
+            for fn in e["files"]:
+                with open(os.path.join(ROOT, fn), "rb") as f:
+                    h.update(f.read())
+        except OSError:
+            continue
+        if h.hexdigest() == e.get("sources_sha256"):
+            out[k] = e["dram_read_bytes"] + e["dram_write_bytes"]
+    return out
+
+
 def time_launch(fn, reps=20, flush=None):
     """Average device duration of one launch, events around the launch only."""
     import torch
@@ -253,10 +278,12 @@ def kernel_rooflines(W, hbm_peak):
         for k in ("tensor_amax", "act_quant", "dequant"):
             out[k]["launch"] = f"[{big['T']}, {big['C']}] bf16"
     if "weights" in W:
-        Xd = W["Xd"]
-        t = time_launch(lambda: nv4.nv4_hessian_accum(Xd, W["Hd"], W["flags"]), reps=10, flush=flush)
-        out["hessian_accum"] = {"bound": "hbm", "bytes": 2.0 * Xd.numel(), "s": t,
-                                "launch": f"X [{Xd.shape[0]}, {Xd.shape[1]}] bf16"}
+        X, Xd = W["X"], W["Xd"]
+        t = time_launch(lambda: nv4.nv4_hessian_accum_batched([X, Xd], [W["H"], W["Hd"]], W["flags"]), reps=10,
+                        flush=flush)
+        out["hessian_accum"] = {"bound": "hbm", "bytes": 2.0 * (X.numel() + Xd.numel()), "s": t,
+                                "launch": f"X [{X.shape[0]}, {X.shape[1]}] + X_down [{Xd.shape[0]}, {Xd.shape[1]}] bf16, "
+                                          "one batched launch"}
         jobs = [{k: j[k] for k in ("w", "H", "d_amax_w", "codes", "q", "cost1", "cost2")} for j in W["weights"]]
         blocks = sum(j["codes"].numel() for j in W["weights"])
         t = time_launch(lambda: nv4.nv4_scale_sweep_batched(jobs, W["flags"]), reps=5)
@@ -279,6 +306,9 @@ def kernel_rooflines(W, hbm_peak):
             v["blocks_per_s"] = v["blocks"] / v["s"]
         v["frac"] = v["achieved"] / v["peak"]
         v["ms"] = v["s"] * 1e3
+    traffic = traffic_table()
+    for k, v in out.items():
+        v["traffic"] = traffic.get(k)
     return out
 
 
@@ -560,9 +590,9 @@ def run_ours(args):
     if dom is not None:
         r = roof[dom]
         line["roofline"] = {"kernel": dom, "bound": r["bound"], "achieved": r["achieved"], "peak": r["peak"],
-                            "unit": r["unit"], "frac": r["frac"], "traffic": None,
+                            "unit": r["unit"], "frac": r["frac"], "traffic": r["traffic"],
                             "peak_kind": peak_kind if r["bound"] == "hbm" else "nominal (unit counts x max clock)"}
-    line["rows"] = {k: {kk: v[kk] for kk in ("bound", "achieved", "peak", "unit", "frac", "ms", "launch")}
+    line["rows"] = {k: {kk: v[kk] for kk in ("bound", "achieved", "peak", "unit", "frac", "ms", "launch", "traffic")}
                     for k, v in roof.items()}
     if sweep is not None:
         line["sweep"] = sweep

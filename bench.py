@@ -44,7 +44,9 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "NVFP4 quant GB/s (% HBM peak); scale-sweep blocks/s (% FP32 peak)"
-SWEEP_FLOP_PER_BLOCK = 127 * 300          # 127 candidates x (136-FMA quadratic form + dequant/subtract)
+SWEEP_FLOP_PER_BLOCK = 127 * 300          # exhaustive count: 127 x (136-FMA quadratic form + dequant/subtract)
+SWEEP_FLOP_PER_VISIT = 80                 # per visited candidate: e = w - v*S (16 FMA) + bound sum rd*e^2 (16 x 3)
+SWEEP_FLOP_PER_COST = 272                 # per evaluated cost: the 136-entry symmetric quadratic form
 ACT_BYTES = {"amax": 2.0, "act_quant": 2.5625, "dequant": 2.5625}
 CAST_BYTES_PER_MX_BLOCK = 1 + 16 + 16 + 2  # read E8M0 + nibbles, write nibbles + 2 E4M3 scales
 FP32_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12   # SMs x FP32 lanes x FMA x max clock
@@ -286,8 +288,16 @@ def kernel_rooflines(W, hbm_peak):
                                           "one batched launch"}
         jobs = [{k: j[k] for k in ("w", "H", "d_amax_w", "codes", "q", "cost1", "cost2")} for j in W["weights"]]
         blocks = sum(j["codes"].numel() for j in W["weights"])
+        # executed work, counted on the device in one extra launch
+        work = torch.zeros(2, dtype=torch.int64, device=W["flags"].device)
+        nv4.nv4_scale_sweep_batched([dict(j, d_work=work) for j in jobs], W["flags"])
+        torch.cuda.synchronize()
+        visits, costs = (int(x) for x in work.tolist())
         t = time_launch(lambda: nv4.nv4_scale_sweep_batched(jobs, W["flags"]), reps=5)
-        out["scale_sweep"] = {"bound": "alu", "flops": SWEEP_FLOP_PER_BLOCK * blocks, "blocks": blocks, "s": t,
+        out["scale_sweep"] = {"bound": "alu", "flops": SWEEP_FLOP_PER_VISIT * visits + SWEEP_FLOP_PER_COST * costs,
+                              "blocks": blocks, "s": t, "visits_per_block": visits / blocks,
+                              "costs_per_block": costs / blocks,
+                              "exhaustive_equiv_tflops": SWEEP_FLOP_PER_BLOCK * blocks / t / 1e12,
                               "launch": "q_proj + gate + up + down, one batched launch"}
     if "cast" in W:
         nmx = sum(j["e8m0"].numel() for j in W["cast"])
@@ -560,8 +570,13 @@ def run_ours(args):
         sw = roof["scale_sweep"]
         sweep = {"value": ws * blocks * args.steps / part_s["calib"], "unit": "blocks/s",
                  "note": "blocks over the whole calib part (Hessians + amax + sweep)",
-                 "kernel_blocks_per_s": sw["blocks_per_s"], "kernel_tflops": sw["achieved"],
-                 "frac_fp32": sw["frac"], "fp32_peak_tflops": FP32_PEAK_TFLOPS}
+                 "kernel_blocks_per_s": sw["blocks_per_s"], "kernel_tflops_executed": sw["achieved"],
+                 "frac_fp32": sw["frac"], "fp32_peak_tflops": FP32_PEAK_TFLOPS,
+                 "visits_per_block": sw["visits_per_block"], "costs_per_block": sw["costs_per_block"],
+                 "exhaustive_equiv_tflops": sw["exhaustive_equiv_tflops"],
+                 "note_work": "exact branch and bound over the 127 codes: achieved counts the FLOPs of the "
+                              "candidates visited and costs evaluated (device counters); exhaustive_equiv "
+                              "counts 127 x 300 FLOP per block"}
     # dominant kernel: largest estimated device time per step (largest launch scaled to all launches)
     scale = {}
     if "act" in parts:

@@ -176,6 +176,9 @@ NV4_API nv4_status nv4_hessian_accum_batched(const nv4_hessian_job* jobs, int n_
  *            or NULL -- a near-tie diagnostic.
  * Costs are evaluated in FP32; blocks whose best and second-best costs differ by
  * less than ~1e-6 relative may pick a different code than an exact evaluation.
+ * The search is exact over all 127 codes but skips the cost of candidates that a
+ * lower bound proves cannot be the winner or the runner-up (sweep.cu states the
+ * bounds); the optional per-job work counter reports how many were evaluated.
  */
 NV4_API nv4_status nv4_scale_sweep(const void* w, nv4_dtype dt, int64_t rows, int64_t cols, int64_t ld,
                            const float* H, const float* d_amax_w, uint8_t* codes, uint8_t* q,
@@ -190,6 +193,7 @@ typedef struct {
     uint8_t* q;         /* [rows, cols/2] or NULL */
     float* cost1;       /* or NULL */
     float* cost2;       /* or NULL */
+    unsigned long long* d_work;  /* or NULL: [0] += candidates visited, [1] += costs evaluated */
 } nv4_sweep_job;
 
 /* Batched form (e.g. all gate/up/down matrices of an expert stack) in one launch.

@@ -39,7 +39,7 @@ class HessianJob(C.Structure):
 
 class SweepJob(C.Structure):
     _fields_ = [("w", _vp), ("rows", _i64), ("cols", _i64), ("ld", _i64), ("H", _vp), ("d_amax_w", _vp),
-                ("codes", _vp), ("q", _vp), ("cost1", _vp), ("cost2", _vp)]
+                ("codes", _vp), ("q", _vp), ("cost1", _vp), ("cost2", _vp), ("d_work", _vp)]
 
 
 class CastJob(C.Structure):
@@ -174,7 +174,7 @@ def nv4_hessian_accum_batched(xs, Hs, d_flags: torch.Tensor | None = None, strea
            "nv4_hessian_accum_batched")
 
 
-def _sjob(w, H, d_amax_w, codes, q=None, cost1=None, cost2=None) -> SweepJob:
+def _sjob(w, H, d_amax_w, codes, q=None, cost1=None, cost2=None, d_work=None) -> SweepJob:
     rows, cols, ld = _rowmajor(w, "w")
     nblk = cols // 16
     if H.dtype != torch.float32 or not H.is_contiguous() or H.numel() != nblk * 256:
@@ -186,8 +186,10 @@ def _sjob(w, H, d_amax_w, codes, q=None, cost1=None, cost2=None) -> SweepJob:
     for c in (cost1, cost2):
         if c is not None and (c.dtype != torch.float32 or tuple(c.shape) != (rows, nblk) or not c.is_contiguous()):
             raise NV4Error("cost1/cost2 must be contiguous float32 tensors [rows, cols/16]")
+    if d_work is not None and (d_work.dtype != torch.int64 or d_work.numel() < 2 or not d_work.is_contiguous()):
+        raise NV4Error("d_work must be a contiguous int64 tensor of at least 2 elements")
     return SweepJob(_ptr(w), rows, cols, ld, _ptr(H), _scalar_f32(d_amax_w, "d_amax_w"), _ptr(codes), _ptr(q),
-                    _ptr(cost1), _ptr(cost2))
+                    _ptr(cost1), _ptr(cost2), _ptr(d_work))
 
 
 def nv4_scale_sweep(w, H, d_amax_w, codes, q=None, cost1=None, cost2=None, d_flags=None, stream=None):
@@ -199,7 +201,7 @@ def nv4_scale_sweep(w, H, d_amax_w, codes, q=None, cost1=None, cost2=None, d_fla
 
 
 def nv4_scale_sweep_batched(jobs: list[dict], d_flags=None, stream=None):
-    """jobs: dicts with keys w, H, d_amax_w, codes and optional q, cost1, cost2 (one dtype)."""
+    """jobs: dicts with keys w, H, d_amax_w, codes and optional q, cost1, cost2, d_work (one dtype)."""
     dts = {j["w"].dtype for j in jobs}
     if len(dts) != 1 or next(iter(dts)) not in (torch.bfloat16, torch.float32):
         raise NV4Error("all w must share one dtype, bf16 or float32")

@@ -203,7 +203,7 @@ nv4_status nv4_scale_sweep(const void* w, nv4_dtype dt, int64_t rows, int64_t co
 {
     nv4_sweep_job j;
     j.w = w; j.rows = rows; j.cols = cols; j.ld = ld; j.H = H; j.d_amax_w = d_amax_w;
-    j.codes = codes; j.q = q; j.cost1 = cost1; j.cost2 = cost2;
+    j.codes = codes; j.q = q; j.cost1 = cost1; j.cost2 = cost2; j.d_work = nullptr;
     return nv4_scale_sweep_batched(&j, 1, dt, d_flags, stream);
 }
 

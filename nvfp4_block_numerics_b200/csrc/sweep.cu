@@ -9,21 +9,40 @@
 // scales S_c (and the reciprocal brackets used to round w/S_c) depend only on the
 // matrix's s2; they sit in a shared-memory table.
 //
-// Per candidate, per thread (all FP32; pairs use the packed FP32 instructions):
+// Per visited candidate, per thread (all FP32; pairs use the packed FP32 instructions):
 //   E2M1 codes of w/S_c : bracketed hardware conversion; near a rounding boundary
 //                         one exact FMA comparison fixes the code (nv4_common.cuh)
 //   e_i = w_i - v_i*S_c   (one rounding of the exact difference)
 //   cost = sum_i e_i (H_ii e_i + sum_{j>i} (H_ij + H_ji) e_j), evaluated two rows at
 //          a time: 136 + 16 multiply-adds in 80 packed instructions
-// The loop runs over codes in increasing order and keeps a strictly smaller cost,
-// so ties go to the lowest code.  Identical dequantized blocks produce identical e
-// and therefore identical costs, so such ties are resolved exactly as well.
+//
+// Exact search order (branch and bound).  The result is the argmin over all 127
+// codes, but most candidates are ruled out by lower bounds instead of evaluated:
+//   (1) Scaled diagonal dominance.  With D = diag(H_b) > 0 and H' = D^-1/2 Hs D^-1/2
+//       (Hs the symmetric part), Gershgorin's theorem gives lambda_min(H') >= rho =
+//       1 - max_i sum_{j != i} |H'_ij|, so for every e:  e^T H_b e >= rho sum_i H_ii e_i^2.
+//   (2) Every grid point of scale S is at most 6S in magnitude, so |e_i| >= |w_i| - 6S,
+//       and the same holds at every smaller scale.
+// The winner and the runner-up cost depend only on candidates whose cost is at most
+// the running runner-up cost.  A thread starts at the max-calibrated code (nearest
+// E4M3 to amax_b / (6 s2)) and walks outwards, alternating down and up: a candidate
+// whose bound (1) exceeds the runner-up skips the quadratic form, and once bound (2)
+// over the two largest |w_i| exceeds it, the downward walk ends.  Both comparisons
+// keep a relative margin of 2^-10, far above the FP32 evaluation error, so skipped
+// candidates could not have changed the FP32 result either.  When rho <= 0, or H_b
+// has a zero diagonal entry with a nonzero row, or non-finite entries, the bounds are
+// off and all 127 candidates are evaluated.
+//
+// Ties: the lowest code wins among equal costs, and the runner-up is the smallest
+// cost strictly above the winner's, independent of the visiting order.  Identical
+// dequantized blocks produce identical e and therefore identical costs.
 #include "nv4_common.cuh"
 #include "nv4_internal.h"
 
 namespace nv4 {
 
 constexpr int kSweepThreads = 128;
+constexpr float kPruneScale = 1.0f - 0x1p-10f;   // bound * this must exceed the runner-up
 
 struct SweepJobDev {
     const void* w;
@@ -33,6 +52,7 @@ struct SweepJobDev {
     uint8_t* q;
     float* cost1;
     float* cost2;
+    unsigned long long* d_work;
     int64_t ld;
     uint32_t rows, nblk, row_tiles, cta_begin;
 };
@@ -130,6 +150,47 @@ __device__ __forceinline__ float quad_form(const float2 e[8], const float4* __re
     return acc.x + acc.y;
 }
 
+// rho * H_ii for the lower bound (1), or all zero with *ok = false when the bound
+// is not valid for this H_b.  Run by one warp; FP64 with a 2^-20 safety margin on rho.
+__device__ void block_bound(const float* __restrict__ hs, float* rd, int* ok)
+{
+    const int lane = threadIdx.x & 31;
+    double r = 0.0, di = 0.0;
+    bool bad = false;
+    if (lane < 16) {
+        di = hs[17 * lane];
+        bad = !(di >= 0.0) || !isfinite(di);
+        for (int j = 0; j < 16; ++j) {
+            if (j == lane) continue;
+            const double hij = 0.5 * ((double)hs[16 * lane + j] + (double)hs[16 * j + lane]);
+            if (!isfinite(hij)) { bad = true; continue; }
+            if (hij == 0.0) continue;
+            const double dj = hs[17 * j];
+            if (di > 0.0 && dj > 0.0) r += fabs(hij) / sqrt(di * dj);
+            else bad = true;     // zero diagonal with a nonzero off-diagonal entry
+        }
+    }
+    for (int o = 8; o > 0; o >>= 1) r = fmax(r, __shfl_xor_sync(0xffffffffu, r, o));
+    bad = __any_sync(0xffffffffu, bad || !isfinite(r));
+    const double rho = 1.0 - r - 0x1p-20;
+    const bool good = !bad && rho > 0.0;
+    if (lane < 16) rd[lane] = good ? __double2float_rd(__dmul_rd(rho, di)) : 0.0f;
+    if (lane == 0) *ok = good ? 1 : 0;
+}
+
+// Lower bound (1) for the error vector e: sum_i rd_i e_i^2.
+__device__ __forceinline__ float bound_diag(const float2 e[8], const float4* __restrict__ rd4)
+{
+    float2 acc = make_float2(0.0f, 0.0f);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const float4 d = rd4[k];
+        acc = __ffma2_rn(__fmul2_rn(e[2 * k], make_float2(d.x, d.y)), e[2 * k], acc);
+        acc = __ffma2_rn(__fmul2_rn(e[2 * k + 1], make_float2(d.z, d.w)), e[2 * k + 1], acc);
+    }
+    return acc.x + acc.y;
+}
+
 template <int kDt>   // 0 bf16, 2 fp32
 __global__ void __launch_bounds__(kSweepThreads, 4)
 sweep_kernel(const __grid_constant__ SweepParams p)
@@ -137,6 +198,8 @@ sweep_kernel(const __grid_constant__ SweepParams p)
     __shared__ float4 tab[128];
     __shared__ float4 hp[kHPairs];
     __shared__ float hs[256];
+    __shared__ float4 rd4[4];
+    __shared__ int bound_ok;
 
     // locate job and tile
     int j = 0;
@@ -175,65 +238,111 @@ sweep_kernel(const __grid_constant__ SweepParams p)
     for (int k = threadIdx.x; k < 256; k += kSweepThreads) hs[k] = job.H[(int64_t)b * 256 + k];
     __syncthreads();
     build_hpairs(hs, hp);
+    if (threadIdx.x >= 96) block_bound(hs, reinterpret_cast<float*>(rd4), &bound_ok);
     __syncthreads();
 
     const uint32_t row = tile * kSweepThreads + threadIdx.x;
-    if (row >= job.rows) return;
-
-    float2 w[8];
-    if constexpr (kDt == 0) {
-        const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(job.w) + (int64_t)row * job.ld + 16 * b);
-        const uint4 v0 = __ldg(src), v1 = __ldg(src + 1);
-        const uint32_t u[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+    const bool live = row < job.rows;
+    uint32_t nvisit = 0u, nfull = 0u;
+    if (live) {
+        float2 w[8];
+        if constexpr (kDt == 0) {
+            const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(job.w) + (int64_t)row * job.ld + 16 * b);
+            const uint4 v0 = __ldg(src), v1 = __ldg(src + 1);
+            const uint32_t u[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
 #pragma unroll
-        for (int k = 0; k < 8; ++k) w[k] = make_float2(bf16_lo(u[k]), bf16_hi(u[k]));
-    } else {
-        const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(job.w) + (int64_t)row * job.ld + 16 * b);
+            for (int k = 0; k < 8; ++k) w[k] = make_float2(bf16_lo(u[k]), bf16_hi(u[k]));
+        } else {
+            const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(job.w) + (int64_t)row * job.ld + 16 * b);
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const float4 v = __ldg(src + k);
-            w[2 * k] = make_float2(v.x, v.y);
-            w[2 * k + 1] = make_float2(v.z, v.w);
+            for (int k = 0; k < 4; ++k) {
+                const float4 v = __ldg(src + k);
+                w[2 * k] = make_float2(v.x, v.y);
+                w[2 * k + 1] = make_float2(v.z, v.w);
+            }
         }
-    }
-    uint32_t flags = isfinite(s2) ? 0u : kFlagOverflow;
+        uint32_t flags = isfinite(s2) ? 0u : kFlagOverflow;
+        // the two largest magnitudes with their bound weights (for bound (2))
+        const float* rd = reinterpret_cast<const float*>(rd4);
+        float a1 = 0.0f, a2 = 0.0f, d1 = 0.0f, d2 = 0.0f;
 #pragma unroll
-    for (int k = 0; k < 8; ++k)
-        if (!isfinite(w[k].x) || !isfinite(w[k].y)) flags |= kFlagNonFinite;
+        for (int k = 0; k < 16; ++k) {
+            const float x = k & 1 ? w[k >> 1].y : w[k >> 1].x;
+            if (!isfinite(x)) flags |= kFlagNonFinite;
+            const float a = fabsf(x), d = rd[k];
+            if (a > a1) { a2 = a1; d2 = d1; a1 = a; d1 = d; }
+            else if (a > a2) { a2 = a; d2 = d; }
+        }
+        const bool pr = bound_ok != 0;
 
-    float best = __int_as_float(0x7F800000), second = best;
-    uint32_t best_c = 0u;
+        float best = __int_as_float(0x7F800000), second = best;
+        uint32_t best_c = 0u;
+        if (a1 == 0.0f) {
+            best = 0.0f;                  // all-zero block: every candidate has e = w = 0
+        } else {
+            // first candidate: the max-calibrated code (any start gives the same result)
+            const float t0 = __fmul_rn(a1, __frcp_rn(__fmul_rn(6.0f, s2)));
+            int c = (int)min(cvt_e4m3x2(t0, t0) & 0x7Fu, 126u);
+            int dn = c - 1, up = c + 1;
+            bool go_dn = true;
 #pragma unroll 1
-    for (uint32_t c = 0; c < 127; ++c) {
-        const float4 t = tab[c];
-        uint32_t c0, c1;
-        codes16(w, t, c0, c1);
-        float2 v[8], e[8];
-        decode16(c0, c1, v);
-        const float2 nS = make_float2(-t.x, -t.x);
+            while (c >= 0) {
+                const float4 t = tab[c];
+                uint32_t c0, c1;
+                codes16(w, t, c0, c1);
+                float2 v[8], e[8];
+                decode16(c0, c1, v);
+                const float2 nS = make_float2(-t.x, -t.x);
 #pragma unroll
-        for (int k = 0; k < 8; ++k) e[k] = __ffma2_rn(v[k], nS, w[k]);     // w - v*S, one rounding
-        const float cost = quad_form(e, hp);
-        if (cost < best) {
-            second = best;
-            best = cost;
-            best_c = c;
-        } else if (cost > best && cost < second) {
-            second = cost;
+                for (int k = 0; k < 8; ++k) e[k] = __ffma2_rn(v[k], nS, w[k]);     // w - v*S, one rounding
+                ++nvisit;
+                if (!pr || !(bound_diag(e, rd4) * kPruneScale > second)) {
+                    ++nfull;
+                    const float cost = quad_form(e, hp);
+                    if (cost < best || (cost == best && (uint32_t)c < best_c)) {
+                        if (cost < best) second = best;
+                        best = cost;
+                        best_c = (uint32_t)c;
+                    } else if (cost > best && cost < second) {
+                        second = cost;
+                    }
+                }
+                // next candidate: alternate down / up; bound (2) closes the downward walk
+                bool take_dn = dn >= 0 && (go_dn || up > 126);
+                if (take_dn && pr) {
+                    const float S = tab[dn].x;
+                    const float u1 = fmaxf(fmaf(-6.0f, S, a1), 0.0f), u2 = fmaxf(fmaf(-6.0f, S, a2), 0.0f);
+                    if (fmaf(d1 * u1, u1, d2 * u2 * u2) * kPruneScale > second) {
+                        dn = -1;
+                        take_dn = false;
+                    }
+                }
+                if (take_dn) { c = dn--; go_dn = false; }
+                else if (up <= 126) { c = up++; go_dn = true; }
+                else c = -1;
+            }
+        }
+        if (!isfinite(best)) flags |= kFlagNonFinite;
+
+        const int64_t blk = (int64_t)row * job.nblk + b;
+        job.codes[blk] = (uint8_t)best_c;
+        if (job.q != nullptr) {
+            uint32_t c0, c1;
+            codes16(w, tab[best_c], c0, c1);
+            *reinterpret_cast<uint2*>(job.q + blk * 8) = make_uint2(c0, c1);
+        }
+        if (job.cost1 != nullptr) job.cost1[blk] = best;
+        if (job.cost2 != nullptr) job.cost2[blk] = second;
+        flag_or(p.d_flags, flags);
+    }
+    if (job.d_work != nullptr) {
+        __syncwarp();
+        const uint32_t sv = __reduce_add_sync(0xffffffffu, nvisit), sf = __reduce_add_sync(0xffffffffu, nfull);
+        if ((threadIdx.x & 31) == 0 && sv != 0u) {
+            atomicAdd(job.d_work, (unsigned long long)sv);
+            atomicAdd(job.d_work + 1, (unsigned long long)sf);
         }
     }
-    if (!isfinite(best)) flags |= kFlagNonFinite;
-
-    const int64_t blk = (int64_t)row * job.nblk + b;
-    job.codes[blk] = (uint8_t)best_c;
-    if (job.q != nullptr) {
-        uint32_t c0, c1;
-        codes16(w, tab[best_c], c0, c1);
-        *reinterpret_cast<uint2*>(job.q + blk * 8) = make_uint2(c0, c1);
-    }
-    if (job.cost1 != nullptr) job.cost1[blk] = best;
-    if (job.cost2 != nullptr) job.cost2[blk] = second;
-    flag_or(p.d_flags, flags);
 }
 
 cudaError_t launch_sweep(const nv4_sweep_job* jobs, int n, int dt, uint32_t* d_flags, cudaStream_t s)
@@ -248,7 +357,7 @@ cudaError_t launch_sweep(const nv4_sweep_job* jobs, int n, int dt, uint32_t* d_f
         if (J.rows == 0 || J.cols == 0) continue;
         SweepJobDev& d = p.jobs[m++];
         d.w = J.w; d.H = J.H; d.d_amax = J.d_amax_w; d.codes = J.codes; d.q = J.q;
-        d.cost1 = J.cost1; d.cost2 = J.cost2; d.ld = J.ld;
+        d.cost1 = J.cost1; d.cost2 = J.cost2; d.d_work = J.d_work; d.ld = J.ld;
         d.rows = (uint32_t)J.rows;
         d.nblk = (uint32_t)(J.cols / 16);
         d.row_tiles = (d.rows + kSweepThreads - 1) / kSweepThreads;

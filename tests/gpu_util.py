@@ -36,7 +36,7 @@ def hessian_rel_err(H_gpu: np.ndarray, H_ref: np.ndarray) -> float:
     return float(np.linalg.norm(H_gpu.astype(np.float64) - H_ref) / max(np.linalg.norm(H_ref), 1e-300))
 
 
-def sweep_parity(codes_gpu, q_gpu, c1_gpu, ref, rel_tie=1e-5):
+def sweep_parity(codes_gpu, q_gpu, c1_gpu, ref, rel_tie=1e-5, c2_gpu=None):
     """Apply the sweep parity rule; returns a dict of counts, asserts the hard parts.
 
     Codes must match wherever the oracle's best and second-best costs differ by more
@@ -64,5 +64,13 @@ def sweep_parity(codes_gpu, q_gpu, c1_gpu, ref, rel_tie=1e-5):
     if ok.any():
         rel = np.abs(c1_gpu[ok].astype(np.float64) - c1[ok]) / c1[ok]
         assert rel.max() < 2e-5, rel.max()
+    if c2_gpu is not None:
+        # runner-up: the smallest cost above the winner's; on blocks with a clear winner
+        # it is the oracle's best cost among different dequantized blocks
+        fin = same & clear & np.isfinite(c2)
+        if fin.any():
+            rel2 = np.abs(c2_gpu[fin].astype(np.float64) - c2[fin]) / c2[fin]
+            assert rel2.max() < 2e-5, rel2.max()
+        assert np.all(np.isinf(c2_gpu[same & unique])), "runner-up cost must be +inf when no other block exists"
     return {"blocks": n, "near_ties": int(near.sum()), "near_tie_mismatches": int((mism & near).sum()),
             "mismatch_frac": float((mism & near).sum()) / max(n, 1)}

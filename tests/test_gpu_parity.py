@@ -215,7 +215,7 @@ def _sweep_check(orc, w, H64, rows_sample=None):
     assert f.item() == 0
     ref = orc.scale_sweep(w, Hin, amax, rows=rows_sample)
     idx = ref["rows"]
-    stats = G.sweep_parity(G.host(codes)[idx], G.host(q)[idx], G.host(c1)[idx], ref)
+    stats = G.sweep_parity(G.host(codes)[idx], G.host(q)[idx], G.host(c1)[idx], ref, c2_gpu=G.host(c2)[idx])
     print("sweep", w.shape, stats)
     assert stats["mismatch_frac"] < 1e-3
     return stats
@@ -243,6 +243,114 @@ def test_sweep_degenerate_blocks(orc):
     w[3, 16:] = -0.0
     H = np.stack([np.eye(16), np.zeros((16, 16))])
     _sweep_check(orc, w, H)
+
+
+def _bound_regime_hessians(rng, tokens=4096, corr_noise=1.0):
+    """Six block columns that exercise every branch of the sweep's lower bounds."""
+    cols = 96
+    x = rng.laplace(size=(tokens, cols))
+    x[:, 16:32] = x[:, 16:17] + corr_noise * rng.standard_normal((tokens, 16))   # correlated: bound off
+    x[:, 32:48:3] = 0.0                                                     # dead channels: zero rows
+    x[:, 80] *= 1000.0                                                      # one huge channel
+    xb = inputs.f32_to_bf16_bits(x.astype(np.float32))
+    H = np.asarray(inputs.bf16_bits_to_f32(xb), np.float64)
+    H = np.einsum("tbi,tbj->bij", H.reshape(tokens, 6, 16), H.reshape(tokens, 6, 16))
+    A = rng.standard_normal((16, 16))
+    H[3] = (A + A.T) * tokens / 4.0                                         # indefinite: costs can be negative
+    H[4] = H[0] + np.triu(rng.standard_normal((16, 16)), 1) * tokens / 50.0  # not symmetric
+    return H
+
+
+def _bound_regime_weights(rng, rows=300, cols=96):
+    w = (rng.standard_normal((rows, cols)) * 0.02).astype(np.float32)
+    w[::7, 5] *= 60.0                                 # one outlier per block: clipping can win
+    w[1::11, 48:64] = 0.0                             # all-zero blocks
+    w[2::11, 48:64] = -0.0
+    grid = np.array([0, .5, 1, 1.5, 2, 3, 4, 6, -6, -4, -3, -2, -1.5, -1, -.5, -0.0], np.float32)
+    w[3::13, 64:80] = grid * np.float32(0.01)         # blocks exact at some scale: cost 0
+    w[4::13, 0:16] = np.float32(1e-12)                # far below the smallest candidate scale
+    return w
+
+
+def test_sweep_bound_regimes(orc):
+    rng = np.random.default_rng(77)
+    H = _bound_regime_hessians(rng)
+    w = _bound_regime_weights(rng)
+    _sweep_check(orc, w, H)
+    _sweep_check(orc, inputs.f32_to_bf16_bits(w), H)
+
+
+def _exact_cost(orc, x, Hb, code, s2):
+    S = float(np.float32(orc.e4m3_value(code)) * np.float32(s2))
+    v = np.array([orc.e2m1_value(orc.e2m1_encode(float(t), S)) for t in x])
+    e = x.astype(np.float64) - v * S
+    return float(e @ Hb @ e)
+
+
+def test_sweep_ill_conditioned_hessian(orc):
+    """A near rank-one H_b (channels equal up to 1e-3 noise): costs evaluated in FP32
+    carry errors of ~1e-3 relative here, so near-equal candidates may be ranked
+    differently than in exact arithmetic.  What holds: the chosen code's exact cost is
+    within 1e-3 of the exact minimum, and the other block columns keep strict parity."""
+    rng = np.random.default_rng(79)
+    H = _bound_regime_hessians(rng, corr_noise=1e-3)
+    w = _bound_regime_weights(rng)
+    H32 = H.astype(np.float32)
+    wd = G.f32_dev(w)
+    d_amax = nv4.tensor_amax(wd)
+    codes, q, c1, c2 = nv4.scale_sweep(wd, G.f32_dev(H32), d_amax)
+    amax = orc.tensor_amax(w)[0]
+    ref = orc.scale_sweep(w, H32.astype(np.float64), amax)
+    got = G.host(codes)
+    s2 = orc.s2_from_amax(amax)
+    worst = 0.0
+    for r in np.nonzero(got[:, 1] != ref["codes"][:, 1])[0]:
+        x = w[r, 16:32]
+        worst = max(worst, _exact_cost(orc, x, H32[1].astype(np.float64), int(got[r, 1]), s2) / ref["cost1"][r, 1] - 1)
+    print("ill-conditioned column: mismatches", int((got[:, 1] != ref["codes"][:, 1]).sum()), "worst excess", worst)
+    assert worst < 1e-3
+    keep = [0, 2, 3, 4, 5]
+    sub = {k: ref[k][:, keep] for k in ("codes", "cost1", "cost2")}
+    sub["q"] = ref["q"].reshape(-1, 6, 8)[:, keep].reshape(len(w), -1)
+    st = G.sweep_parity(got[:, keep], G.host(q).reshape(-1, 6, 8)[:, keep].reshape(len(w), -1),
+                        G.host(c1)[:, keep], sub, c2_gpu=G.host(c2)[:, keep])
+    assert st["mismatch_frac"] < 1e-3
+
+
+def test_sweep_work_counter(orc):
+    """Bounds on: far fewer than 127 costs per block; bounds off (correlated channels):
+    every candidate visited and evaluated; the winners match the oracle either way."""
+    rng = np.random.default_rng(78)
+    x = rng.laplace(size=(2048, 32))
+    x[:, 16:] = x[:, 16:17] + rng.standard_normal((2048, 16))       # correlated channels: rho < 0
+    xb = inputs.f32_to_bf16_bits(x.astype(np.float32))
+    H = orc.hessian_accum(xb)
+    w = (rng.standard_normal((256, 32)) * 0.02).astype(np.float32)
+    wd = G.f32_dev(w)
+    rows, cols = w.shape
+    work = []
+    jobs = []
+    for b in range(2):
+        wb = wd[:, 16 * b:16 * b + 16].contiguous()
+        Hb = G.f32_dev(H[b:b + 1].astype(np.float32))
+        work.append(torch.zeros(2, dtype=torch.int64, device=G.DEV))
+        jobs.append(dict(w=wb, H=Hb, d_amax_w=nv4.tensor_amax(wd),
+                         codes=torch.empty((rows, 1), dtype=torch.uint8, device=G.DEV),
+                         q=torch.empty((rows, 8), dtype=torch.uint8, device=G.DEV),
+                         cost1=torch.empty((rows, 1), dtype=torch.float32, device=G.DEV),
+                         cost2=torch.empty((rows, 1), dtype=torch.float32, device=G.DEV), d_work=work[-1]))
+    f = G.flags_dev()
+    nv4.nv4_scale_sweep_batched(jobs, f)
+    torch.cuda.synchronize()
+    assert f.item() == 0
+    on, off = work[0].cpu().numpy(), work[1].cpu().numpy()
+    print("work with bounds", on, "without", off)
+    assert off[0] == 127 * rows and off[1] == 127 * rows
+    assert on[1] <= on[0] <= 127 * rows and on[1] < 0.25 * 127 * rows
+    ref = orc.scale_sweep(w, H.astype(np.float32).astype(np.float64), orc.tensor_amax(w)[0])
+    cat = lambda k: np.concatenate([G.host(j[k]) for j in jobs], axis=1)
+    st = G.sweep_parity(cat("codes"), cat("q"), cat("cost1"), ref, c2_gpu=cat("cost2"))
+    assert st["mismatch_frac"] < 1e-3
 
 
 def test_sweep_gemma_layer_sampled(orc):
@@ -284,7 +392,8 @@ def test_sweep_moe_batched_sampled(orc):
     for job, w, Hin in checks:
         rows = np.sort(rng.choice(w.shape[0], 24, replace=False))
         ref = orc.scale_sweep(w, Hin, orc.tensor_amax(w)[0], rows=rows)
-        st = G.sweep_parity(G.host(job["codes"])[rows], G.host(job["q"])[rows], G.host(job["cost1"])[rows], ref)
+        st = G.sweep_parity(G.host(job["codes"])[rows], G.host(job["q"])[rows], G.host(job["cost1"])[rows], ref,
+                            c2_gpu=G.host(job["cost2"])[rows])
         assert st["mismatch_frac"] < 1e-3
 
 

@@ -59,6 +59,7 @@ struct SweepJobDev {
 
 struct SweepParams {
     int n, dt;
+    uint32_t tiles_per_cta;
     uint32_t* d_flags;
     SweepJobDev jobs[kMaxSweepJobs];
 };
@@ -151,30 +152,32 @@ __device__ __forceinline__ float quad_form(const float2 e[8], const float4* __re
 }
 
 // rho * H_ii for the lower bound (1), or all zero with *ok = false when the bound
-// is not valid for this H_b.  Run by one warp; FP64 with a 2^-20 safety margin on rho.
+// is not valid for this H_b.  Run by one full warp, lane i < 16 owning channel i.
+// FP32 with explicit safety margins: rsqrtf is within 2 ulp and the 15-term sum of
+// positive products within 2^-19 relative, so r * (1 + 2^-16) + 2^-16 bounds the
+// exact Gershgorin radius from above.
 __device__ void block_bound(const float* __restrict__ hs, float* rd, int* ok)
 {
     const int lane = threadIdx.x & 31;
-    double r = 0.0, di = 0.0;
-    bool bad = false;
-    if (lane < 16) {
-        di = hs[17 * lane];
-        bad = !(di >= 0.0) || !isfinite(di);
-        for (int j = 0; j < 16; ++j) {
-            if (j == lane) continue;
-            const double hij = 0.5 * ((double)hs[16 * lane + j] + (double)hs[16 * j + lane]);
-            if (!isfinite(hij)) { bad = true; continue; }
-            if (hij == 0.0) continue;
-            const double dj = hs[17 * j];
-            if (di > 0.0 && dj > 0.0) r += fabs(hij) / sqrt(di * dj);
-            else bad = true;     // zero diagonal with a nonzero off-diagonal entry
-        }
+    const int i = lane & 15;
+    const float di = hs[17 * i];
+    bool bad = lane < 16 && !(di >= 0.0f && di <= 3.0e38f);
+    const float inv = di > 0.0f ? rsqrtf(di) : 0.0f;
+    float r = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+        const float inv_j = __shfl_sync(0xffffffffu, inv, j);
+        if (j == i) continue;
+        const float hij = 0.5f * (hs[16 * i + j] + hs[16 * j + i]);
+        if (!(fabsf(hij) <= 3.0e38f)) bad = true;
+        else if (hij != 0.0f && (inv == 0.0f || inv_j == 0.0f)) bad = true;   // zero diagonal, nonzero row
+        r = fmaf(fabsf(hij) * inv, inv_j, r);
     }
-    for (int o = 8; o > 0; o >>= 1) r = fmax(r, __shfl_xor_sync(0xffffffffu, r, o));
-    bad = __any_sync(0xffffffffu, bad || !isfinite(r));
-    const double rho = 1.0 - r - 0x1p-20;
-    const bool good = !bad && rho > 0.0;
-    if (lane < 16) rd[lane] = good ? __double2float_rd(__dmul_rd(rho, di)) : 0.0f;
+    for (int o = 8; o > 0; o >>= 1) r = fmaxf(r, __shfl_xor_sync(0xffffffffu, r, o));
+    bad = __any_sync(0xffffffffu, bad || !(r <= 3.0e38f));
+    const float rho = 1.0f - fmaf(r, 1.0f + 0x1p-16f, 0x1p-16f);
+    const bool good = !bad && rho > 0.0f;
+    if (lane < 16) rd[lane] = good ? __fmul_rd(rho, di) : 0.0f;
     if (lane == 0) *ok = good ? 1 : 0;
 }
 
@@ -191,6 +194,31 @@ __device__ __forceinline__ float bound_diag(const float2 e[8], const float4* __r
     return acc.x + acc.y;
 }
 
+template <int kDt>
+__device__ __forceinline__ void load_block(const SweepJobDev& job, uint32_t row, uint32_t b, float2 w[8])
+{
+    if constexpr (kDt == 0) {
+        const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(job.w) + (int64_t)row * job.ld + 16 * b);
+        const uint4 v0 = __ldg(src), v1 = __ldg(src + 1);
+        const uint32_t u[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+        for (int k = 0; k < 8; ++k) w[k] = make_float2(bf16_lo(u[k]), bf16_hi(u[k]));
+    } else {
+        const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(job.w) + (int64_t)row * job.ld + 16 * b);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float4 v = __ldg(src + k);
+            w[2 * k] = make_float2(v.x, v.y);
+            w[2 * k + 1] = make_float2(v.z, v.w);
+        }
+    }
+}
+
+constexpr uint32_t kNoRow = 0xFFFFFFFFu;
+
+// One CTA = one block column b of one job and up to p.tiles_per_cta tiles of 128 rows.
+// Per tile the rows are counting-sorted by their starting code, so the lanes of a warp
+// walk similar candidate sequences in lockstep.
 template <int kDt>   // 0 bf16, 2 fp32
 __global__ void __launch_bounds__(kSweepThreads, 4)
 sweep_kernel(const __grid_constant__ SweepParams p)
@@ -200,8 +228,11 @@ sweep_kernel(const __grid_constant__ SweepParams p)
     __shared__ float hs[256];
     __shared__ float4 rd4[4];
     __shared__ int bound_ok;
+    __shared__ uint32_t hist[128], base[128];
+    __shared__ float4 sw[kSweepThreads][4];
+    __shared__ uint32_t srow[kSweepThreads];
 
-    // locate job and tile
+    // locate job and tile group
     int j = 0;
     {
         int lo = 0, hi = p.n - 1;
@@ -213,11 +244,11 @@ sweep_kernel(const __grid_constant__ SweepParams p)
     }
     const SweepJobDev& job = p.jobs[j];
     const uint32_t local = blockIdx.x - job.cta_begin;
-    const uint32_t b = local % job.nblk, tile = local / job.nblk;
+    const uint32_t b = local % job.nblk, group = local / job.nblk;
 
     // candidate table: S_c = RN32(e4m3(c) * s2) and a bracket of 1/S_c
     const float s2 = __fdiv_rn(*job.d_amax, 2688.0f);
-    if (threadIdx.x < 128) {
+    {
         const uint32_t c = threadIdx.x;
         float4 t = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
         if (c < 127) {
@@ -234,37 +265,78 @@ sweep_kernel(const __grid_constant__ SweepParams p)
             }
         }
         tab[c] = t;
+        hist[c] = 0u;
     }
     for (int k = threadIdx.x; k < 256; k += kSweepThreads) hs[k] = job.H[(int64_t)b * 256 + k];
     __syncthreads();
     build_hpairs(hs, hp);
     if (threadIdx.x >= 96) block_bound(hs, reinterpret_cast<float*>(rd4), &bound_ok);
     __syncthreads();
+    const bool pr = bound_ok != 0;
+    const float k6 = __frcp_rn(__fmul_rn(6.0f, s2));            // ~ 1/(6 s2), for the starting code
+    const float* rd = reinterpret_cast<const float*>(rd4);
+    const uint32_t s2flag = isfinite(s2) ? 0u : kFlagOverflow;
 
-    const uint32_t row = tile * kSweepThreads + threadIdx.x;
-    const bool live = row < job.rows;
     uint32_t nvisit = 0u, nfull = 0u;
-    if (live) {
+    const uint32_t tile_end = min(job.row_tiles, (group + 1) * p.tiles_per_cta);
+#pragma unroll 1
+    for (uint32_t tile = group * p.tiles_per_cta; tile < tile_end; ++tile) {
+        // ---- load, starting code, counting sort by starting code
+        uint32_t row = tile * kSweepThreads + threadIdx.x;
         float2 w[8];
-        if constexpr (kDt == 0) {
-            const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(job.w) + (int64_t)row * job.ld + 16 * b);
-            const uint4 v0 = __ldg(src), v1 = __ldg(src + 1);
-            const uint32_t u[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+        uint32_t key = 127u;
+        if (row < job.rows) {
+            load_block<kDt>(job, row, b, w);
+            float a1 = 0.0f;
 #pragma unroll
-            for (int k = 0; k < 8; ++k) w[k] = make_float2(bf16_lo(u[k]), bf16_hi(u[k]));
-        } else {
-            const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(job.w) + (int64_t)row * job.ld + 16 * b);
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const float4 v = __ldg(src + k);
-                w[2 * k] = make_float2(v.x, v.y);
-                w[2 * k + 1] = make_float2(v.z, v.w);
+            for (int k = 0; k < 8; ++k) a1 = fmaxf(a1, fmaxf(fabsf(w[k].x), fabsf(w[k].y)));
+            if (a1 > 0.0f) {
+                const float t0 = __fmul_rn(a1, k6);
+                key = min(cvt_e4m3x2(t0, t0) & 0x7Fu, 126u);
             }
+        } else {
+            row = kNoRow;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) w[k] = make_float2(0.0f, 0.0f);
         }
-        uint32_t flags = isfinite(s2) ? 0u : kFlagOverflow;
-        // the two largest magnitudes with their bound weights (for bound (2))
-        const float* rd = reinterpret_cast<const float*>(rd4);
-        float a1 = 0.0f, a2 = 0.0f, d1 = 0.0f, d2 = 0.0f;
+        const uint32_t rank = atomicAdd(&hist[key], 1u);
+        __syncthreads();
+        if (threadIdx.x < 32) {                 // exclusive scan of the 128 bucket counts
+            const uint32_t l = threadIdx.x;
+            const uint32_t h0 = hist[4 * l], h1 = hist[4 * l + 1], h2 = hist[4 * l + 2], h3 = hist[4 * l + 3];
+            uint32_t sum = h0 + h1 + h2 + h3, incl = sum;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+                if (l >= (uint32_t)o) incl += t;
+            }
+            const uint32_t ex = incl - sum;
+            base[4 * l] = ex;
+            base[4 * l + 1] = ex + h0;
+            base[4 * l + 2] = ex + h0 + h1;
+            base[4 * l + 3] = ex + h0 + h1 + h2;
+            hist[4 * l] = hist[4 * l + 1] = hist[4 * l + 2] = hist[4 * l + 3] = 0u;
+        }
+        __syncthreads();
+        {
+            const uint32_t pos = base[key] + rank;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) sw[pos][k] = make_float4(w[2 * k].x, w[2 * k].y, w[2 * k + 1].x, w[2 * k + 1].y);
+            srow[pos] = row;
+        }
+        __syncthreads();
+        row = srow[threadIdx.x];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float4 v = sw[threadIdx.x][k];
+            w[2 * k] = make_float2(v.x, v.y);
+            w[2 * k + 1] = make_float2(v.z, v.w);
+        }
+        if (row == kNoRow) continue;            // no barrier follows inside this tile
+
+        // ---- the search for this thread's (row, b)
+        uint32_t flags = s2flag;
+        float a1 = 0.0f, a2 = 0.0f, d1 = 0.0f, d2 = 0.0f;   // two largest |w_i|, their bound weights
 #pragma unroll
         for (int k = 0; k < 16; ++k) {
             const float x = k & 1 ? w[k >> 1].y : w[k >> 1].x;
@@ -273,15 +345,12 @@ sweep_kernel(const __grid_constant__ SweepParams p)
             if (a > a1) { a2 = a1; d2 = d1; a1 = a; d1 = d; }
             else if (a > a2) { a2 = a; d2 = d; }
         }
-        const bool pr = bound_ok != 0;
-
         float best = __int_as_float(0x7F800000), second = best;
         uint32_t best_c = 0u;
         if (a1 == 0.0f) {
             best = 0.0f;                  // all-zero block: every candidate has e = w = 0
         } else {
-            // first candidate: the max-calibrated code (any start gives the same result)
-            const float t0 = __fmul_rn(a1, __frcp_rn(__fmul_rn(6.0f, s2)));
+            const float t0 = __fmul_rn(a1, k6);
             int c = (int)min(cvt_e4m3x2(t0, t0) & 0x7Fu, 126u);
             int dn = c - 1, up = c + 1;
             bool go_dn = true;
@@ -361,8 +430,16 @@ cudaError_t launch_sweep(const nv4_sweep_job* jobs, int n, int dt, uint32_t* d_f
         d.rows = (uint32_t)J.rows;
         d.nblk = (uint32_t)(J.cols / 16);
         d.row_tiles = (d.rows + kSweepThreads - 1) / kSweepThreads;
+    }
+    // tiles per CTA: amortize the per-column setup while keeping >= ~16 CTAs per SM
+    uint64_t tiles = 0;
+    for (int i = 0; i < m; ++i) tiles += (uint64_t)p.jobs[i].row_tiles * p.jobs[i].nblk;
+    const uint64_t per = tiles / ((uint64_t)num_sms() * 16u);
+    p.tiles_per_cta = (uint32_t)(per < 1 ? 1 : (per > 4 ? 4 : per));
+    for (int i = 0; i < m; ++i) {
+        SweepJobDev& d = p.jobs[i];
         d.cta_begin = ctas;
-        ctas += d.row_tiles * d.nblk;
+        ctas += ((d.row_tiles + p.tiles_per_cta - 1) / p.tiles_per_cta) * d.nblk;
     }
     p.n = m;
     if (m == 0) return cudaSuccess;

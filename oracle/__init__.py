@@ -65,6 +65,7 @@ def _L():
                 "orc_f32_to_f16": (C.c_uint16, [C.c_float]),
                 "orc_tensor_amax": (C.c_float, [vp, C.c_int, i64, u32p]),
                 "orc_act_quant": (C.c_float, [vp, i64, i64, i64, C.c_float, i64, i64, vp, vp, u32p]),
+                "orc_block_quant": (C.c_float, [vp, C.c_int, i64, i64, i64, C.c_float, i64, i64, vp, vp, u32p]),
                 "orc_dequant": (None, [vp, vp, C.c_float, i64, i64, C.c_int, i64, i64, vp]),
                 "orc_hessian_accum": (None, [vp, i64, i64, i64, i64, i64, vp]),
                 "orc_scale_sweep": (None, [vp, C.c_int, i64, i64, i64, vp, C.c_float, i64, i64,
@@ -194,6 +195,45 @@ def act_quant(x: np.ndarray, amax: float, cols: int | None = None, threads: int 
     else:
         _fanout(run, rows, threads)
     return q, sc, float(np.float32(s2[0])), flags[0]
+
+
+def rtn_quant(w: np.ndarray, amax: float, cols: int | None = None, threads: int | None = None):
+    """Round-to-nearest weight quantization with max-calibrated block scales.
+
+    w: float32 or uint16 (bf16 bits) [rows, ld].  The activation quantizer's
+    arithmetic ([FLOW] 3.4-3.5) applied to a weight tensor with its own amax.
+    Returns (q [rows, cols/2], scales [rows, cols/16], s2, flags)."""
+    assert w.ndim == 2 and w.flags.c_contiguous and w.dtype in (np.float32, np.uint16)
+    dt = F32 if w.dtype == np.float32 else BF16
+    rows, ld = w.shape
+    cols = ld if cols is None else cols
+    assert cols % 16 == 0
+    q = np.zeros((rows, cols // 2), np.uint8)
+    sc = np.zeros((rows, cols // 16), np.uint8)
+    flags = [0]
+    s2 = [float(np.float32(_L().orc_s2_from_amax(amax)))]
+    lk = threading.Lock()
+
+    def run(r0, r1):
+        f = C.c_uint32(0)
+        _L().orc_block_quant(_p(w), dt, rows, cols, ld, amax, r0, r1, _p(q), _p(sc), C.byref(f))
+        with lk:
+            flags[0] |= f.value
+
+    if rows:
+        _fanout(run, rows, threads)
+    else:
+        f = C.c_uint32(0)
+        _L().orc_block_quant(_p(w), dt, 0, cols, ld, amax, 0, 0, _p(q), _p(sc), C.byref(f))
+        flags[0] |= f.value
+    return q, sc, s2[0], flags[0]
+
+
+def fake_qdq(x: np.ndarray, amax: float, out_dtype: str = "bf16", threads: int | None = None):
+    """Quantize then dequantize ([FLOW] 3.4: quantizer followed by DQ1/DQ2), the
+    plain composition of act_quant and dequant.  Returns (out, s2, flags)."""
+    q, sc, s2, flags = act_quant(x, amax, threads=threads)
+    return dequant(q, sc, s2, out_dtype, threads=threads), s2, flags
 
 
 def dequant(q: np.ndarray, scales: np.ndarray, s2: float, out_dtype: str = "bf16",

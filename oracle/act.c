@@ -10,6 +10,10 @@
  *            relative to s2; elements become E2M1 codes of x / (s_b*s2); [FLOW] 5.4: two
  *            FP4 codes per byte.  [CAL] format line: 16-element blocks, E4M3 scale, FP32
  *            second-level scale.
+ *  RTN weight quant [FLOW] 3.5 (static weight quantization) and [CAL] section 2 step 1
+ *            (max calibration gives the initial block scale): the same block arithmetic as
+ *            the activation quantizer, applied once to a BF16 or FP32 weight tensor with its
+ *            own amax.
  *  dequant   [FLOW] 3.4: DQ1 turns (E4M3 scale, FP32 s2) into the FP32 block scale
  *            S = s_b*s2; DQ2 multiplies each FP4 value by S and emits the high-precision
  *            type (BF16 by default, FP16 optional, [FLOW] 3.6).
@@ -49,17 +53,22 @@ float orc_tensor_amax(const void* x, int dtype, int64_t n, uint32_t* flags)
 float orc_act_quant(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, float amax,
                     int64_t row0, int64_t row1, uint8_t* q, uint8_t* scales, uint32_t* flags)
 {
+    return orc_block_quant(x, ORC_BF16, rows, cols, ld, amax, row0, row1, q, scales, flags);
+}
+
+float orc_block_quant(const void* x, int dtype, int64_t rows, int64_t cols, int64_t ld, float amax,
+                      int64_t row0, int64_t row1, uint8_t* q, uint8_t* scales, uint32_t* flags)
+{
     (void)rows;
     float s2 = orc_s2_from_amax(amax);
     if (!isfinite(s2)) *flags |= ORC_FLAG_OVERFLOW;
     const int64_t nblk = cols / 16;
     for (int64_t r = row0; r < row1; ++r) {
-        const uint16_t* xr = x + r * ld;
         for (int64_t b = 0; b < nblk; ++b) {
             double v[16];
             double a_b = 0.0;
             for (int i = 0; i < 16; ++i) {
-                v[i] = orc_bf16_value(xr[16 * b + i]);
+                v[i] = elem_value(x, dtype, r * ld + 16 * b + i);
                 if (!isfinite(v[i])) *flags |= ORC_FLAG_NONFINITE;
                 if (fabs(v[i]) > a_b) a_b = fabs(v[i]);
             }

@@ -70,6 +70,12 @@ float orc_tensor_amax(const void* x, int dtype, int64_t n, uint32_t* flags);
 float orc_act_quant(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, float amax,
                     int64_t row0, int64_t row1, uint8_t* q, uint8_t* scales, uint32_t* flags);
 
+/* ---- round-to-nearest block quantization of a BF16 or FP32 tensor (act.c) --
+ * The activation quantizer's arithmetic for dtype ORC_BF16 or ORC_F32 input (RTN
+ * weight quantization with max-calibrated block scales). */
+float orc_block_quant(const void* x, int dtype, int64_t rows, int64_t cols, int64_t ld, float amax,
+                      int64_t row0, int64_t row1, uint8_t* q, uint8_t* scales, uint32_t* flags);
+
 /* ---- two-step dequantization (act.c) ------------------------------------
  * out_dtype: 0 = bf16 bits (uint16), 1 = fp16 bits (uint16), 2 = fp32. */
 void orc_dequant(const uint8_t* q, const uint8_t* scales, float s2, int64_t rows, int64_t cols,

@@ -115,3 +115,65 @@ def test_dequant_matches_torch_two_step(orc):
         assert np.array_equal(outb, y.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16))
         outh = orc.dequant(q, sc, s2, "fp16")
         assert np.array_equal(outh, y.to(torch.float16).view(torch.int16).numpy().view(np.uint16))
+
+
+# ------------------------------------------------------------ RTN weight quantization
+def test_rtn_quant_fp32_brute_force(orc):
+    """FP32 weights (with exact rounding midpoints planted) decided again in exact rationals."""
+    r = np.random.default_rng(21)
+    w = (r.standard_normal((5, 64)) * 0.02).astype(np.float32)
+    w[1, 3] = 0.9                                      # an outlier sets amax
+    amax, _ = orc.tensor_amax(w)
+    s2r = X.rn32(Fr(amax) / 2688)
+    # plant elements exactly on E2M1 decision boundaries of their block's scale
+    for b in range(4):
+        blk = [float(v) for v in w[2, 16 * b:16 * b + 16]]
+        code, S, _ = X.act_quant_block(blk, s2r)
+        w[2, 16 * b + 5] = X.f32(Fr(5, 4) * S) if b % 2 else X.f32(-Fr(3, 4) * S)
+    q, sc, s2, flags = orc.rtn_quant(w, amax)
+    assert flags == 0 and Fr(s2) == s2r
+    for i in range(w.shape[0]):
+        for b in range(w.shape[1] // 16):
+            code, S, nibs = X.act_quant_block([float(v) for v in w[i, 16 * b:16 * b + 16]], s2r)
+            assert sc[i, b] == code
+            assert q[i, 8 * b:8 * b + 8].tolist() == [nibs[2 * k] | (nibs[2 * k + 1] << 4) for k in range(8)]
+
+
+def test_rtn_quant_bf16_matches_activation_quantizer(orc):
+    x = inputs.laplace_bf16(inputs.rng_for(22, "pin", "rtn"), 9, 80, outlier_channels=(2,), outlier_scale=40)
+    amax, _ = orc.tensor_amax(x)
+    a = orc.act_quant(x, amax)
+    b = orc.rtn_quant(x, amax)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1]) and a[2] == b[2]
+    # the same values as FP32 give the same codes
+    c = orc.rtn_quant(inputs.bf16_bits_to_f32(x).copy(), amax)
+    assert np.array_equal(a[0], c[0]) and np.array_equal(a[1], c[1])
+
+
+# ------------------------------------------------------------ fake quantize-dequantize
+def test_fake_qdq_grid_block_roundtrips_exactly(orc):
+    """amax = 2688 gives s2 = 1; a block of grid values times a power-of-two S whose
+    largest magnitude is 6S gets block scale S and comes back bit-exact."""
+    rows = []
+    for k, S in enumerate((0.25, 1.0, 4.0, 32.0)):
+        v = np.array([6, -0.5, 1, -1.5, 2, 3, -4, 0, 0.5, -6, 4, 1.5, -2, -3, 1, -1], np.float32)
+        rows.append(np.roll(v, k) * np.float32(S))
+    x = inputs.f32_to_bf16_bits(np.stack(rows).reshape(1, -1).astype(np.float32))
+    out, s2, flags = orc.fake_qdq(x, 2688.0)
+    assert s2 == 1.0 and flags == 0
+    assert np.array_equal(out, x)
+
+
+def test_fake_qdq_error_within_half_grid_step(orc):
+    x = inputs.laplace_bf16(inputs.rng_for(23, "pin", "qdq"), 7, 96, outlier_channels=(11,), outlier_scale=25)
+    amax, _ = orc.tensor_amax(x)
+    y32, s2, _ = orc.fake_qdq(x, amax, "fp32")
+    ybf, _, _ = orc.fake_qdq(x, amax, "bf16")
+    q, sc, _, _ = orc.act_quant(x, amax)
+    xf = inputs.bf16_bits_to_f32(x).astype(np.float64)
+    S = np.repeat(np.array([[orc.e4m3_value(int(c)) for c in row] for row in sc]) * s2, 16, axis=1)
+    a = np.abs(xf) / S
+    half = np.where(a <= 2, 0.25, np.where(a <= 4, 0.5, 1.0)) * S
+    assert np.all(np.abs(xf - y32) <= half * (1 + 1e-6) + (a - 6).clip(0) * S)
+    # the BF16 output is the FP32 dequantized value rounded to BF16
+    assert np.array_equal(ybf, inputs.f32_to_bf16_bits(y32.astype(np.float32)))

@@ -277,9 +277,24 @@ def kernel_rooflines(W, hbm_peak):
         out["act_quant"] = {"bound": "hbm", "bytes": ACT_BYTES["act_quant"] * n, "s": t}
         t = time_launch(lambda: nv4.nv4_dequant(big["q"], big["sc"], s2, big["out"]), flush=flush)
         out["dequant"] = {"bound": "hbm", "bytes": ACT_BYTES["dequant"] * n, "s": t}
-        for k in ("tensor_amax", "act_quant", "dequant"):
+        # fused fake quantize-dequantize (a widening of the path; not part of the step)
+        qdq = torch.empty_like(big["x"])
+        t = time_launch(lambda: nv4.nv4_fake_qdq(big["x"], a, qdq, s2, W["flags"]), flush=flush)
+        out["fake_qdq"] = {"bound": "hbm", "bytes": 4.0 * n, "s": t, "in_step": False}
+        del qdq
+        for k in ("tensor_amax", "act_quant", "dequant", "fake_qdq"):
             out[k]["launch"] = f"[{big['T']}, {big['C']}] bf16"
     if "weights" in W:
+        # RTN weight quantization of the gate projection (a widening of the path; not in the step)
+        j = W["weights"][1]
+        rq = torch.empty_like(j["q"])
+        rs = torch.empty((j["w"].shape[0], j["w"].shape[1] // 16), dtype=torch.uint8, device=j["w"].device)
+        rs2 = torch.empty(1, dtype=torch.float32, device=j["w"].device)
+        t = time_launch(lambda: nv4.nv4_weight_quant_rtn(j["w"], j["d_amax_w"], rq, rs, rs2, W["flags"]),
+                        flush=flush)
+        out["weight_quant_rtn"] = {"bound": "hbm", "bytes": ACT_BYTES["act_quant"] * j["w"].numel(), "s": t,
+                                   "in_step": False, "launch": f"{j['name']} {list(j['w'].shape)} bf16"}
+        del rq, rs
         X, Xd = W["X"], W["Xd"]
         t = time_launch(lambda: nv4.nv4_hessian_accum_batched([X, Xd], [W["H"], W["Hd"]], W["flags"]), reps=10,
                         flush=flush)
@@ -585,7 +600,8 @@ def run_ours(args):
         scale.update({k: n_tot / n_big for k in ("tensor_amax", "act_quant", "dequant")})
     if "calib" in parts:
         scale["hessian_accum"] = (W["X"].numel() + W["Xd"].numel()) / W["Xd"].numel()
-    dom = max(roof, key=lambda k: roof[k]["s"] * scale.get(k, 1.0)) if roof else None
+    in_step = [k for k in roof if roof[k].get("in_step", True)]
+    dom = max(in_step, key=lambda k: roof[k]["s"] * scale.get(k, 1.0)) if in_step else None
     shares = {p: part_s[p] / total_s for p in parts}
     line = {
         "metric": METRIC, "value": value, "unit": unit, "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
@@ -607,7 +623,8 @@ def run_ours(args):
         line["roofline"] = {"kernel": dom, "bound": r["bound"], "achieved": r["achieved"], "peak": r["peak"],
                             "unit": r["unit"], "frac": r["frac"], "traffic": r["traffic"],
                             "peak_kind": peak_kind if r["bound"] == "hbm" else "nominal (unit counts x max clock)"}
-    line["rows"] = {k: {kk: v[kk] for kk in ("bound", "achieved", "peak", "unit", "frac", "ms", "launch", "traffic")}
+    line["rows"] = {k: {kk: v.get(kk) for kk in ("bound", "achieved", "peak", "unit", "frac", "ms", "launch", "traffic",
+                                                  "in_step")}
                     for k, v in roof.items()}
     if sweep is not None:
         line["sweep"] = sweep

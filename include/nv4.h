@@ -119,6 +119,37 @@ NV4_API nv4_status nv4_act_quant(const void* x, int64_t rows, int64_t cols, int6
                          uint32_t* d_flags, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * nv4_weight_quant_rtn -- static round-to-nearest NVFP4 quantization of a weight
+ * tensor with max-calibrated block scales: [FLOW] 3.5 (weights quantized once, ahead
+ * of time) with the block arithmetic of nv4_act_quant; [CAL] section 2 step 1 (max
+ * calibration gives the initial scale that the sweep of nv4_scale_sweep improves on).
+ *
+ * w      : [rows, cols] of dt (NV4_BF16 or NV4_FP32), leading dimension ld (16-byte
+ *          multiple), 16-byte aligned.  cols % 16 == 0.
+ * d_amax : device float, the weight tensor's amax.  Other arguments as nv4_act_quant.
+ * Limit: rows * cols/16 < 2^30 blocks per call (NV4_ERR_LIMIT beyond).
+ */
+NV4_API nv4_status nv4_weight_quant_rtn(const void* w, nv4_dtype dt, int64_t rows, int64_t cols, int64_t ld,
+                                const float* d_amax, uint8_t* q, uint8_t* scales, float* d_s2,
+                                uint32_t* d_flags, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * nv4_fake_qdq -- fused fake quantization: nv4_act_quant followed by nv4_dequant in
+ * one pass, without materializing codes or scales ([FLOW] 3.4: quantizer, then DQ1
+ * and DQ2; the quantize-dequantize a calibration forward pass runs on activations).
+ * out = RN_out(RN32(e2m1(code) * S)) with code, S exactly as nv4_act_quant.
+ *
+ * x      : bf16 [rows, cols], leading dimension ld (ld % 8 == 0), 16-byte aligned.
+ * out    : [rows, cols] of out_dt (NV4_BF16, NV4_FP16 or NV4_FP32), leading dimension
+ *          ld_out (a 16-byte multiple), 16-byte aligned; may equal x when out_dt is
+ *          NV4_BF16 and ld_out == ld (in place).
+ * d_amax, d_s2, d_flags as nv4_act_quant.  Limit: rows * cols/16 < 2^30 blocks.
+ */
+NV4_API nv4_status nv4_fake_qdq(const void* x, int64_t rows, int64_t cols, int64_t ld, const float* d_amax,
+                        nv4_dtype out_dt, void* out, int64_t ld_out, float* d_s2, uint32_t* d_flags,
+                        void* stream);
+
+/* ---------------------------------------------------------------------------
  * nv4_dequant -- the two-step dequantization of [FLOW] 3.4 / 5.4:
  *   DQ1: S = RN32(s_b * s2);  DQ2: y = RN32(e2m1(code) * S), then rounded to out_dt
  *   (NV4_BF16 default, NV4_FP16, or NV4_FP32 as is), ties to even, overflow to inf.

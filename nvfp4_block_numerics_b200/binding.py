@@ -19,7 +19,8 @@ import torch
 from .build import LIB_PATH
 
 __all__ = [
-    "NV4Error", "lib", "nv4_tensor_amax", "nv4_act_quant", "nv4_dequant", "nv4_hessian_accum",
+    "NV4Error", "lib", "nv4_tensor_amax", "nv4_act_quant", "nv4_weight_quant_rtn", "nv4_fake_qdq",
+    "nv4_dequant", "nv4_hessian_accum", "weight_quant_rtn", "fake_qdq",
     "nv4_hessian_accum_batched", "nv4_scale_sweep", "nv4_scale_sweep_batched", "nv4_mxfp4_to_nvfp4",
     "nv4_mxfp4_to_nvfp4_batched", "nv4_selftest", "nv4_version", "FLAG_NONFINITE", "FLAG_E8M0_NAN",
     "FLAG_OVERFLOW", "FLAG_TIMEOUT", "tensor_amax", "act_quant", "dequant", "hessian_accum",
@@ -59,6 +60,8 @@ _SIGS = {
     "nv4_version": (C.c_int, []),
     "nv4_tensor_amax": (C.c_int, [_vp, C.c_int, _i64, _vp, _vp, _vp]),
     "nv4_act_quant": (C.c_int, [_vp, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "nv4_weight_quant_rtn": (C.c_int, [_vp, C.c_int, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "nv4_fake_qdq": (C.c_int, [_vp, _i64, _i64, _i64, _vp, C.c_int, _vp, _i64, _vp, _vp, _vp]),
     "nv4_dequant": (C.c_int, [_vp, _vp, _vp, _i64, _i64, C.c_int, _vp, _vp]),
     "nv4_hessian_accum": (C.c_int, [_vp, _i64, _i64, _i64, _vp, _vp, _vp]),
     "nv4_hessian_accum_batched": (C.c_int, [C.POINTER(HessianJob), C.c_int, _vp, _vp]),
@@ -139,6 +142,34 @@ def nv4_act_quant(x: torch.Tensor, d_amax: torch.Tensor, q: torch.Tensor, scales
         raise NV4Error("scales must be a contiguous uint8 tensor [rows, cols/16]")
     _check(lib().nv4_act_quant(_ptr(x), rows, cols, ld, _scalar_f32(d_amax, "d_amax"), _ptr(q), _ptr(scales),
                                _scalar_f32(d_s2, "d_s2"), _ptr(d_flags), _stream(stream)), "nv4_act_quant")
+
+
+def nv4_weight_quant_rtn(w: torch.Tensor, d_amax: torch.Tensor, q: torch.Tensor, scales: torch.Tensor,
+                         d_s2: torch.Tensor, d_flags: torch.Tensor | None = None, stream=None):
+    if w.dtype not in (torch.bfloat16, torch.float32):
+        raise NV4Error("w must be bf16 or float32")
+    rows, cols, ld = _rowmajor(w, "w")
+    if q.dtype != torch.uint8 or tuple(q.shape) != (rows, cols // 2) or not q.is_contiguous():
+        raise NV4Error("q must be a contiguous uint8 tensor [rows, cols/2]")
+    if scales.dtype != torch.uint8 or tuple(scales.shape) != (rows, cols // 16) or not scales.is_contiguous():
+        raise NV4Error("scales must be a contiguous uint8 tensor [rows, cols/16]")
+    _check(lib().nv4_weight_quant_rtn(_ptr(w), _DT[w.dtype], rows, cols, ld, _scalar_f32(d_amax, "d_amax"), _ptr(q),
+                                      _ptr(scales), _scalar_f32(d_s2, "d_s2"), _ptr(d_flags), _stream(stream)),
+           "nv4_weight_quant_rtn")
+
+
+def nv4_fake_qdq(x: torch.Tensor, d_amax: torch.Tensor, out: torch.Tensor, d_s2: torch.Tensor,
+                 d_flags: torch.Tensor | None = None, stream=None):
+    if x.dtype != torch.bfloat16:
+        raise NV4Error("x must be bf16")
+    if out.dtype not in _DT:
+        raise NV4Error("out must be bf16, float16 or float32")
+    rows, cols, ld = _rowmajor(x, "x")
+    orows, ocols, ld_out = _rowmajor(out, "out")
+    if (orows, ocols) != (rows, cols):
+        raise NV4Error("out must have the shape of x")
+    _check(lib().nv4_fake_qdq(_ptr(x), rows, cols, ld, _scalar_f32(d_amax, "d_amax"), _DT[out.dtype], _ptr(out),
+                              ld_out, _scalar_f32(d_s2, "d_s2"), _ptr(d_flags), _stream(stream)), "nv4_fake_qdq")
 
 
 def nv4_dequant(q: torch.Tensor, scales: torch.Tensor, d_s2: torch.Tensor, out: torch.Tensor, stream=None):
@@ -258,6 +289,22 @@ def act_quant(x: torch.Tensor, d_amax: torch.Tensor, d_flags=None, stream=None):
     s2 = torch.empty((1,), dtype=torch.float32, device=x.device)
     nv4_act_quant(x, d_amax, q, sc, s2, d_flags, stream)
     return q, sc, s2
+
+
+def weight_quant_rtn(w: torch.Tensor, d_amax: torch.Tensor, d_flags=None, stream=None):
+    rows, cols = w.shape
+    q = torch.empty((rows, cols // 2), dtype=torch.uint8, device=w.device)
+    sc = torch.empty((rows, cols // 16), dtype=torch.uint8, device=w.device)
+    s2 = torch.empty((1,), dtype=torch.float32, device=w.device)
+    nv4_weight_quant_rtn(w, d_amax, q, sc, s2, d_flags, stream)
+    return q, sc, s2
+
+
+def fake_qdq(x: torch.Tensor, d_amax: torch.Tensor, dtype=torch.bfloat16, d_flags=None, stream=None):
+    out = torch.empty(tuple(x.shape), dtype=dtype, device=x.device)
+    s2 = torch.empty((1,), dtype=torch.float32, device=x.device)
+    nv4_fake_qdq(x, d_amax, out, s2, d_flags, stream)
+    return out, s2
 
 
 def dequant(q, scales, d_s2, dtype=torch.bfloat16, stream=None):

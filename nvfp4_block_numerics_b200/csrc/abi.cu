@@ -118,6 +118,36 @@ nv4_status nv4_act_quant(const void* x, int64_t rows, int64_t cols, int64_t ld, 
     return from_cuda(launch_act_quant(x, rows, cols, ld, d_amax, q, scales, d_s2, d_flags, (cudaStream_t)stream));
 }
 
+nv4_status nv4_weight_quant_rtn(const void* w, nv4_dtype dt, int64_t rows, int64_t cols, int64_t ld,
+                                const float* d_amax, uint8_t* q, uint8_t* scales, float* d_s2, uint32_t* d_flags,
+                                void* stream)
+{
+    if (dt != NV4_BF16 && dt != NV4_FP32) return NV4_ERR_DTYPE;
+    if (rows < 0 || cols < 0 || cols % 16 != 0 || ld < cols) return NV4_ERR_SHAPE;
+    if (d_amax == nullptr || d_s2 == nullptr) return NV4_ERR_NULL;
+    if (rows == 0 || cols == 0) return NV4_OK;
+    if (w == nullptr || q == nullptr || scales == nullptr) return NV4_ERR_NULL;
+    if (!aligned16(w) || !aligned16(q) || ld % (dt == NV4_BF16 ? 8 : 4) != 0) return NV4_ERR_ALIGN;
+    if (rows * (cols / 16) >= (int64_t)1 << 30) return NV4_ERR_LIMIT;
+    return from_cuda(launch_block_quant(w, dt == NV4_BF16 ? 0 : 2, rows, cols, ld, d_amax, q, scales, -1, nullptr, 0,
+                                        d_s2, d_flags, (cudaStream_t)stream));
+}
+
+nv4_status nv4_fake_qdq(const void* x, int64_t rows, int64_t cols, int64_t ld, const float* d_amax,
+                        nv4_dtype out_dt, void* out, int64_t ld_out, float* d_s2, uint32_t* d_flags, void* stream)
+{
+    if (out_dt != NV4_BF16 && out_dt != NV4_FP16 && out_dt != NV4_FP32) return NV4_ERR_DTYPE;
+    if (rows < 0 || cols < 0 || cols % 16 != 0 || ld < cols || ld_out < cols) return NV4_ERR_SHAPE;
+    if (d_amax == nullptr || d_s2 == nullptr) return NV4_ERR_NULL;
+    if (rows == 0 || cols == 0) return NV4_OK;
+    if (x == nullptr || out == nullptr) return NV4_ERR_NULL;
+    if (!aligned16(x) || !aligned16(out) || ld % 8 != 0 || ld_out % (out_dt == NV4_FP32 ? 4 : 8) != 0)
+        return NV4_ERR_ALIGN;
+    if (rows * (cols / 16) >= (int64_t)1 << 30) return NV4_ERR_LIMIT;
+    return from_cuda(launch_block_quant(x, 0, rows, cols, ld, d_amax, nullptr, nullptr, (int)out_dt, out, ld_out,
+                                        d_s2, d_flags, (cudaStream_t)stream));
+}
+
 nv4_status nv4_dequant(const uint8_t* q, const uint8_t* scales, const float* d_s2, int64_t rows, int64_t cols,
                        nv4_dtype out_dt, void* out, void* stream)
 {

@@ -37,6 +37,9 @@ constexpr int kMaxCastJobs = 128;
 cudaError_t launch_amax(const void* x, int dt, int64_t n, float* d_amax, uint32_t* d_flags, cudaStream_t s);
 cudaError_t launch_act_quant(const void* x, int64_t rows, int64_t cols, int64_t ld, const float* d_amax,
                              uint8_t* q, uint8_t* scales, float* d_s2, uint32_t* d_flags, cudaStream_t s);
+cudaError_t launch_block_quant(const void* x, int in_dt, int64_t rows, int64_t cols, int64_t ld,
+                               const float* d_amax, uint8_t* q, uint8_t* scales, int out_dt, void* out,
+                               int64_t ld_out, float* d_s2, uint32_t* d_flags, cudaStream_t s);
 cudaError_t launch_dequant(const uint8_t* q, const uint8_t* scales, const float* d_s2, int64_t rows, int64_t cols,
                            int out_dt, void* out, cudaStream_t s);
 cudaError_t launch_hessian(const nv4_hessian_job* jobs, int n, uint32_t* d_flags, cudaStream_t s, int* bad_job);

@@ -174,10 +174,96 @@ __device__ __forceinline__ void quantize16(const float x[16], float S, float r_l
 
 constexpr int kActThreads = 256;
 
+// One 16-element block of the input: BF16 (two 128-bit words) or FP32 (four).
+template <int kIn>
+struct BlockIn {
+    uint4 v[kIn == 0 ? 2 : 4];
+};
+
+template <int kIn>
+__device__ __forceinline__ void load_block_in(const void* x, int64_t off, BlockIn<kIn>& blk)
+{
+    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const char*>(x) + off * (kIn == 0 ? 2 : 4));
+#pragma unroll
+    for (int k = 0; k < (kIn == 0 ? 2 : 4); ++k) blk.v[k] = __ldcs(src + k);
+}
+
+// Block max magnitude bits (as an FP32 bit pattern) and the 16 values as floats.
+template <int kIn>
+__device__ __forceinline__ uint32_t unpack_block(const BlockIn<kIn>& blk, float xv[16])
+{
+    if constexpr (kIn == 0) {
+        const uint32_t w[8] = {blk.v[0].x, blk.v[0].y, blk.v[0].z, blk.v[0].w,
+                               blk.v[1].x, blk.v[1].y, blk.v[1].z, blk.v[1].w};
+        uint32_t m = 0u;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            m = __vmaxu2(m, w[j] & 0x7FFF7FFFu);
+            xv[2 * j] = bf16_lo(w[j]);
+            xv[2 * j + 1] = bf16_hi(w[j]);
+        }
+        return max(m & 0xFFFFu, m >> 16) << 16;
+    } else {
+        uint32_t m = 0u;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const uint32_t w[4] = {blk.v[k].x, blk.v[k].y, blk.v[k].z, blk.v[k].w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                m = max(m, w[j] & 0x7FFFFFFFu);
+                xv[4 * k + j] = __uint_as_float(w[j]);
+            }
+        }
+        return m;
+    }
+}
+
+// Fake quantize-dequantize output of one block: DQ2 RN32(v * S), then the output type.
+template <int kOut>
+__device__ __forceinline__ void store_qdq(uint32_t q0, uint32_t q1, float S, void* out, int64_t off)
+{
+    uint32_t h[8];
+    cvt_e2m1x8_to_f16x8(q0, h);
+    cvt_e2m1x8_to_f16x8(q1, h + 4);
+    float y[16];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        float a, c;
+        f16x2_to_f32(h[j], a, c);
+        const float2 r = __fmul2_rn(make_float2(a, c), make_float2(S, S));
+        y[2 * j] = r.x;
+        y[2 * j + 1] = r.y;
+    }
+    if constexpr (kOut == 2) {
+        float4* o = reinterpret_cast<float4*>(static_cast<float*>(out) + off);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) __stcs(o + k, make_float4(y[4 * k], y[4 * k + 1], y[4 * k + 2], y[4 * k + 3]));
+    } else {
+        uint32_t p[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            if constexpr (kOut == 0) {
+                asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(p[j]) : "f"(y[2 * j + 1]), "f"(y[2 * j]));
+            } else {
+                asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(p[j]) : "f"(y[2 * j + 1]), "f"(y[2 * j]));
+            }
+        }
+        uint4* o = reinterpret_cast<uint4*>(static_cast<uint16_t*>(out) + off);
+        __stcs(o, make_uint4(p[0], p[1], p[2], p[3]));
+        __stcs(o + 1, make_uint4(p[4], p[5], p[6], p[7]));
+    }
+}
+
+// Block quantizer over a [rows, cols] tensor: one thread per 16-block, grid-stride,
+// with the next block's loads in flight while the current one is quantized.
+// kIn: 0 BF16, 2 FP32 input.  kOut: -1 writes packed codes + E4M3 scales; 0/1/2 writes
+// the fake quantize-dequantize values as BF16/FP16/FP32 (leading dimension ld_out).
+// Every block is read and written by the same thread, read first, so out may alias x.
+template <int kIn, int kOut>
 __global__ void __launch_bounds__(kActThreads)
-act_quant_kernel(const uint16_t* __restrict__ x, uint32_t rows, uint32_t bpr, int64_t ld, FastDiv div_bpr,
+act_quant_kernel(const void* x, uint32_t rows, uint32_t bpr, int64_t ld, FastDiv div_bpr,
                  const float* __restrict__ d_amax, uint8_t* __restrict__ q, uint8_t* __restrict__ scales,
-                 float* __restrict__ d_s2, uint32_t* __restrict__ d_flags)
+                 void* out, int64_t ld_out, float* __restrict__ d_s2, uint32_t* __restrict__ d_flags)
 {
     __shared__ E4M3Tables tab;
     fill_e4m3_tables(tab);
@@ -194,28 +280,20 @@ act_quant_kernel(const uint16_t* __restrict__ x, uint32_t rows, uint32_t bpr, in
 
     const uint32_t total = rows * bpr;
     const uint32_t stride = gridDim.x * kActThreads;
-    // software pipeline: the next block's two 128-bit loads are in flight while this
-    // block is quantized
-    auto load = [&](uint32_t u, uint4& a, uint4& b) {
+    auto offset = [&](uint32_t u, int64_t l) {
         const uint32_t r = div_bpr.div(u), bb = u - r * bpr;
-        const uint4* src = reinterpret_cast<const uint4*>(x + (int64_t)r * ld + 16u * bb);
-        a = __ldcs(src);
-        b = __ldcs(src + 1);
+        return (int64_t)r * l + 16 * (int64_t)bb;
     };
     uint32_t u = blockIdx.x * kActThreads + threadIdx.x;
-    uint4 n0 = make_uint4(0u, 0u, 0u, 0u), n1 = n0;
-    if (u < total) load(u, n0, n1);
+    BlockIn<kIn> nxt;
+    if (u < total) load_block_in<kIn>(x, offset(u, ld), nxt);
     for (; u < total; u += stride) {
-        const uint4 v0 = n0, v1 = n1;
-        if (u + stride < total) load(u + stride, n0, n1);
-        const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-
-        uint32_t m = 0u;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) m = __vmaxu2(m, w[j] & 0x7FFF7FFFu);
-        const uint32_t ab = max(m & 0xFFFFu, m >> 16);
-        if (ab >= 0x7F80u) flags |= kFlagNonFinite;
-        const float a_b = __uint_as_float(ab << 16);
+        const BlockIn<kIn> cur = nxt;
+        if (u + stride < total) load_block_in<kIn>(x, offset(u + stride, ld), nxt);
+        float xv[16];
+        const uint32_t ab = unpack_block<kIn>(cur, xv);
+        if (ab >= 0x7F800000u) flags |= kFlagNonFinite;
+        const float a_b = __uint_as_float(ab);
 
         // block scale: nearest E4M3 to a_b / (6*s2)
         uint32_t code;
@@ -229,19 +307,17 @@ act_quant_kernel(const uint16_t* __restrict__ x, uint32_t rows, uint32_t bpr, in
         code &= 0x7Fu;                                            // non-negative inputs only
         const float S = __fmul_rn(tab.dec[code], s2);            // DQ1: RN32(s_b * s2)
 
-        float xv[16];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            xv[2 * j] = bf16_lo(w[j]);
-            xv[2 * j + 1] = bf16_hi(w[j]);
-        }
         const bool exact = S != 0.0f && !(S >= kTinyScale && S <= 0x1p100f);
         const float rr = S == 0.0f ? 0.0f : __fmul_rn(tab.rcp[code], rs2);   // ~ 1/S
         uint32_t q0, q1;
         quantize16(xv, S, __fmul_rn(rr, kLoMargin), __fmul_rn(rr, kHiMargin), exact, q0, q1);
 
-        *reinterpret_cast<uint2*>(q + (int64_t)u * 8) = make_uint2(q0, q1);
-        scales[u] = (uint8_t)code;
+        if constexpr (kOut < 0) {
+            *reinterpret_cast<uint2*>(q + (int64_t)u * 8) = make_uint2(q0, q1);
+            scales[u] = (uint8_t)code;
+        } else {
+            store_qdq<kOut>(q0, q1, S, out, offset(u, ld_out));
+        }
     }
     flags = __reduce_or_sync(__activemask(), flags);
     if ((threadIdx.x & 31) == 0) flag_or(d_flags, flags);
@@ -344,10 +420,24 @@ cudaError_t launch_amax(const void* x, int dt, int64_t n, float* d_amax, uint32_
 cudaError_t launch_act_quant(const void* x, int64_t rows, int64_t cols, int64_t ld, const float* d_amax,
                              uint8_t* q, uint8_t* scales, float* d_s2, uint32_t* d_flags, cudaStream_t s)
 {
+    return launch_block_quant(x, 0, rows, cols, ld, d_amax, q, scales, -1, nullptr, 0, d_s2, d_flags, s);
+}
+
+cudaError_t launch_block_quant(const void* x, int in_dt, int64_t rows, int64_t cols, int64_t ld,
+                               const float* d_amax, uint8_t* q, uint8_t* scales, int out_dt, void* out,
+                               int64_t ld_out, float* d_s2, uint32_t* d_flags, cudaStream_t s)
+{
     const uint32_t bpr = (uint32_t)(cols / 16);
     const uint32_t total = (uint32_t)rows * bpr;
-    act_quant_kernel<<<grid_for(total, kActThreads, 8), kActThreads, 0, s>>>(
-        static_cast<const uint16_t*>(x), (uint32_t)rows, bpr, ld, FastDiv(bpr), d_amax, q, scales, d_s2, d_flags);
+    const int g = grid_for(total, kActThreads, 8);
+#define NV4_BQ(I, O) act_quant_kernel<I, O><<<g, kActThreads, 0, s>>>(x, (uint32_t)rows, bpr, ld, FastDiv(bpr), \
+        d_amax, q, scales, out, ld_out, d_s2, d_flags)
+    if (in_dt == 0) {
+        if (out_dt < 0) NV4_BQ(0, -1); else if (out_dt == 0) NV4_BQ(0, 0); else if (out_dt == 1) NV4_BQ(0, 1); else NV4_BQ(0, 2);
+    } else {
+        if (out_dt < 0) NV4_BQ(2, -1); else if (out_dt == 0) NV4_BQ(2, 0); else if (out_dt == 1) NV4_BQ(2, 1); else NV4_BQ(2, 2);
+    }
+#undef NV4_BQ
     return cudaGetLastError();
 }
 

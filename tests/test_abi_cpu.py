@@ -28,7 +28,7 @@ def declared_symbols():
 def test_header_declares_the_hot_path():
     names = declared_symbols()
     for n in ("nv4_tensor_amax", "nv4_act_quant", "nv4_dequant", "nv4_hessian_accum", "nv4_scale_sweep",
-              "nv4_mxfp4_to_nvfp4"):
+              "nv4_mxfp4_to_nvfp4", "nv4_weight_quant_rtn", "nv4_fake_qdq"):
         assert n in names
 
 
@@ -62,6 +62,19 @@ def test_validation_rejects_before_any_launch(nv4lib):
     assert L.nv4_tensor_amax(fake, 0, -1, fake, None, None) == 2
     assert L.nv4_tensor_amax(fake, 0, 0, fake, None, None) == 0                            # no-op
     assert L.nv4_dequant(fake, fake, fake, 2, 32, 7, fake, None) == 4
+    # RTN weight quantization: dtype, shape, alignment (FP32 rows need ld % 4), nulls
+    assert L.nv4_weight_quant_rtn(fake, 1, 4, 32, 32, fake, fake, fake, fake, None, None) == 4    # fp16 w
+    assert L.nv4_weight_quant_rtn(fake, 2, 4, 40, 40, fake, fake, fake, fake, None, None) == 2    # cols % 16
+    assert L.nv4_weight_quant_rtn(fake, 2, 4, 32, 34, fake, fake, fake, fake, None, None) == 3    # ld*4 % 16
+    assert L.nv4_weight_quant_rtn(fake, 0, 4, 32, 36, fake, fake, fake, fake, None, None) == 3    # ld*2 % 16
+    assert L.nv4_weight_quant_rtn(fake, 2, 4, 32, 32, fake, None, fake, fake, None, None) == 1
+    assert L.nv4_weight_quant_rtn(fake, 2, 0, 32, 32, fake, None, None, fake, None, None) == 0    # empty
+    # fused fake quantize-dequantize
+    assert L.nv4_fake_qdq(fake, 4, 32, 32, fake, 5, fake, 32, fake, None, None) == 4              # out dtype
+    assert L.nv4_fake_qdq(fake, 4, 32, 32, fake, 0, fake, 16, fake, None, None) == 2              # ld_out < cols
+    assert L.nv4_fake_qdq(fake, 4, 32, 32, fake, 2, fake, 34, fake, None, None) == 3              # fp32 ld_out
+    assert L.nv4_fake_qdq(fake, 4, 32, 32, fake, 0, fake + 8, 32, fake, None, None) == 3          # misaligned out
+    assert L.nv4_fake_qdq(fake, 4, 32, 32, None, 0, fake, 32, fake, None, None) == 1
     assert L.nv4_hessian_accum(fake, 10, 40, 40, fake, None, None) == 2
     assert L.nv4_hessian_accum(fake, 10, 32, 36, fake, None, None) == 3
     assert L.nv4_scale_sweep(fake, 2, 4, 32, 34, fake, fake, fake, None, None, None, None, None) == 3  # fp32 ld*4

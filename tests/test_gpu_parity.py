@@ -135,6 +135,115 @@ def test_dequant_random_codes(orc):
             assert np.array_equal(got, ref), (s2, name)
 
 
+# ------------------------------------------------------------------ RTN weight quantization
+def _rtn_check(orc, w, amax=None, ld_pad=0):
+    rows, cols = w.shape
+    wd_full = G.f32_dev(np.pad(w, ((0, 0), (0, ld_pad)))) if w.dtype == np.float32 else \
+        G.bf16_dev(np.pad(w, ((0, 0), (0, ld_pad))))
+    wd = wd_full[:, :cols]
+    if amax is None:
+        amax = orc.tensor_amax(w)[0]
+    d_amax = torch.tensor([amax], dtype=torch.float32, device=G.DEV)
+    f = G.flags_dev()
+    q, sc, s2 = nv4.weight_quant_rtn(wd, d_amax, d_flags=f)
+    rq, rsc, rs2, rf = orc.rtn_quant(w, amax)
+    torch.cuda.synchronize()
+    assert s2.item() == rs2 and f.item() == rf
+    assert np.array_equal(G.host(sc), rsc)
+    assert np.array_equal(G.host(q), rq)
+
+
+@pytest.mark.parametrize("rows,cols,pad", [(1, 16, 0), (3, 48, 8), (129, 80, 0), (300, 256, 16)])
+def test_weight_quant_rtn_small_ragged(orc, rows, cols, pad):
+    r = np.random.default_rng(rows + cols)
+    w = (r.standard_normal((rows, cols)) * 0.02).astype(np.float32)
+    w[:, 1] *= 40.0
+    w[::5, :16] = 0.0
+    w[1::7, 16:32] = -0.0
+    _rtn_check(orc, w, ld_pad=pad)
+    _rtn_check(orc, inputs.f32_to_bf16_bits(w), ld_pad=pad)
+
+
+def test_weight_quant_rtn_edge_values(orc):
+    g = [0.0, 0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 6.0, 7.0, -0.0, -0.25, -0.75, -5.0, 1e-30, -1e-30]
+    w = np.array([g, [v * 0.5 for v in g], [448.0 * 6] + [0.0] * 15, [3.0] * 16], np.float32)
+    w = np.concatenate([w, np.nextafter(w, np.float32(np.inf))], axis=1)     # one ulp above each boundary
+    for amax in (2688.0, 0.0, 1.0, float(np.float32(2688.0 * 1.37))):
+        _rtn_check(orc, w, amax=amax)
+
+
+def test_weight_quant_rtn_layer_weights(orc):
+    d = inputs.c3_layer(0, which=("W_q", "W_gate"))
+    _rtn_check(orc, d["W_q"])
+    _rtn_check(orc, d["W_gate"])
+    _rtn_check(orc, inputs.c1_tiny_linear(0)["W"])
+
+
+# ------------------------------------------------------------------ fused fake quantize-dequantize
+def _qdq_check(orc, x, amax=None, ld_pad=0, out_pad=0):
+    rows, cols = x.shape
+    xd = G.bf16_dev(np.pad(x, ((0, 0), (0, ld_pad))))[:, :cols]
+    if amax is None:
+        amax = orc.tensor_amax(x)[0]
+    d_amax = torch.tensor([amax], dtype=torch.float32, device=G.DEV)
+    for dt, name in ((torch.bfloat16, "bf16"), (torch.float16, "fp16"), (torch.float32, "fp32")):
+        out = torch.full((rows, cols + out_pad), 7.0, dtype=dt, device=G.DEV)[:, :cols]
+        s2 = torch.empty(1, dtype=torch.float32, device=G.DEV)
+        f = G.flags_dev()
+        nv4.nv4_fake_qdq(xd, d_amax, out, s2, f)
+        ref, rs2, rf = orc.fake_qdq(x, amax, name)
+        torch.cuda.synchronize()
+        got = G.host(out.contiguous())
+        if name == "fp32":
+            got, ref = got.view(np.uint32), ref.view(np.uint32)
+        assert s2.item() == rs2 and f.item() == rf
+        assert np.array_equal(got, ref), name
+        if out_pad:                                   # the padding columns are untouched
+            assert (G.host(out.as_strided((rows, out_pad), (cols + out_pad, 1), cols).float()) == 7.0).all()
+
+
+@pytest.mark.parametrize("rows,cols,pad", [(1, 16, 0), (3, 48, 8), (129, 80, 0), (300, 256, 16)])
+def test_fake_qdq_small_ragged(orc, rows, cols, pad):
+    x = inputs.laplace_bf16(inputs.rng_for(rows * cols, "gpu", "qdq"), rows, cols, outlier_channels=(1,),
+                            outlier_scale=50, zero_block_frac=0.05)
+    _qdq_check(orc, x, ld_pad=pad, out_pad=pad)
+
+
+def test_fake_qdq_edge_values_and_in_place(orc):
+    g = [0.0, 0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 6.0, 7.0, -0.0, -0.25, -0.75, -5.0, 1e-30, -1e-30]
+    x = inputs.f32_to_bf16_bits(np.array([g, [v * 0.5 for v in g], [448.0 * 6] + [0.0] * 15, [-0.0] * 16],
+                                         np.float32))
+    for amax in (2688.0, 0.0, 1.0):
+        _qdq_check(orc, x, amax=amax)
+    # in place, BF16 over the input
+    y = inputs.c2_shape(256, 2048)
+    yd = G.bf16_dev(y)
+    d_amax = nv4.tensor_amax(yd)
+    s2 = torch.empty(1, dtype=torch.float32, device=G.DEV)
+    nv4.nv4_fake_qdq(yd, d_amax, yd, s2)
+    ref, _, _ = orc.fake_qdq(y, orc.tensor_amax(y)[0], "bf16")
+    assert np.array_equal(G.host(yd), ref)
+
+
+@pytest.mark.parametrize("T,C", [(16, 2048), (4096, 4096), (65536, 7168)])
+def test_fake_qdq_config_shapes(orc, T, C):
+    """Against the oracle (sampled rows at the largest size) and against the separate
+    act-quant + dequant kernels (whole tensor, bit for bit)."""
+    x = inputs.c2_shape(T, C)
+    xd = G.bf16_dev(x)
+    d_amax = nv4.tensor_amax(xd)
+    out, s2 = nv4.fake_qdq(xd, d_amax)
+    q, sc, s2b = nv4.act_quant(xd, d_amax)
+    two = nv4.dequant(q, sc, s2b)
+    torch.cuda.synchronize()
+    assert torch.equal(out.view(torch.int16), two.view(torch.int16))
+    rows = np.arange(T) if T <= 4096 else np.sort(np.random.default_rng(T).choice(T, 256, replace=False))
+    xs = np.ascontiguousarray(x[rows])
+    q_r, sc_r, s2_r, _ = orc.act_quant(xs, orc.tensor_amax(x)[0])
+    ref = orc.dequant(q_r, sc_r, s2_r, "bf16")
+    assert np.array_equal(G.host(out)[rows], ref)
+
+
 # ------------------------------------------------------------------ Hessian
 def _hess_check(orc, x_bits, ld_pad=0, tol=1e-5):
     T, K = x_bits.shape

@@ -308,21 +308,35 @@ def scale_sweep(w: np.ndarray, H: np.ndarray, amax_w: float, rows=None, cols: in
 
 
 # ---------------------------------------------------------------- MXFP4 -> NVFP4
-def mxfp4_to_nvfp4(mx_q: np.ndarray, e8m0: np.ndarray, threads: int | None = None):
-    """One matrix: mx_q uint8 [rows, cols/2], e8m0 uint8 [rows, cols/32].
-
-    Raises ValueError on an E8M0 NaN code.  Returns a dict with nv_q, nv_scales, s2,
-    global_amax, k_max, counts (in-window, fallback, lossless 16-blocks) and flags.
-    """
+def _mx_check(mx_q, e8m0):
     mx_q = np.ascontiguousarray(mx_q)
     e8m0 = np.ascontiguousarray(e8m0)
     rows, half = mx_q.shape
-    cols = 2 * half
-    assert cols % 32 == 0 and e8m0.shape == (rows, cols // 32)
+    assert (2 * half) % 32 == 0 and e8m0.shape == (rows, 2 * half // 32)
+    return mx_q, e8m0
+
+
+def _mx_kmax(e8m0):
     f = C.c_uint32(0)
     kmax = _L().orc_mx_kmax(_p(e8m0), e8m0.size, C.byref(f))
     if f.value & FLAG_E8M0_NAN:
         raise ValueError("E8M0 NaN code 0xFF in the input")
+    return kmax
+
+
+def mxfp4_to_nvfp4(mx_q: np.ndarray, e8m0: np.ndarray, threads: int | None = None, k_max: int | None = None):
+    """One matrix: mx_q uint8 [rows, cols/2], e8m0 uint8 [rows, cols/32].
+
+    k_max: None for the matrix's own largest exponent ([CAST] section 2, per layer),
+    or a shared one (a group of matrices with one scale_2, see mxfp4_to_nvfp4_group).
+    Raises ValueError on an E8M0 NaN code.  Returns a dict with nv_q, nv_scales, s2,
+    global_amax, k_max, counts (in-window, fallback, lossless 16-blocks) and flags.
+    """
+    mx_q, e8m0 = _mx_check(mx_q, e8m0)
+    rows, half = mx_q.shape
+    cols = 2 * half
+    kmax = _mx_kmax(e8m0) if k_max is None else int(k_max)
+    f = C.c_uint32(0)
     s2 = C.c_float(0)
     ga = C.c_float(0)
     _L().orc_mx_global(kmax, C.byref(s2), C.byref(ga), C.byref(f))
@@ -341,3 +355,13 @@ def mxfp4_to_nvfp4(mx_q: np.ndarray, e8m0: np.ndarray, threads: int | None = Non
     counts = np.sum(parts, axis=0) if parts else np.zeros(3, np.int64)
     return {"nv_q": nv_q, "nv_scales": nv_s, "s2": s2.value, "global_amax": ga.value,
             "k_max": kmax, "counts": counts, "flags": f.value}
+
+
+def mxfp4_to_nvfp4_group(mats, threads: int | None = None):
+    """Matrices that share one scale_2 ([CAST] section 3: DeepSeek V4 routed experts,
+    w1 and w3 with one scale_2).  Reading: k_max is the largest exponent over the
+    union of the group's E8M0 codes, and every member is cast against it (window and
+    fallback relative to the shared k_max).  mats: list of (mx_q, e8m0)."""
+    mats = [_mx_check(q, e) for q, e in mats]
+    kmax = max(_mx_kmax(e) for _, e in mats)
+    return [mxfp4_to_nvfp4(q, e, threads, k_max=kmax) for q, e in mats]

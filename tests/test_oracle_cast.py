@@ -115,3 +115,31 @@ def test_storage_cost_table(orc):
     for fmt in ("MXFP4", "NVFP4"):
         g, sbits, bpp = int(rows[fmt][0]), int(rows[fmt][1]), float(rows[fmt][2])
         assert 4 + sbits / g == bpp
+
+
+def test_grouped_scale2_window_follows_the_group_max(orc):
+    """Two matrices sharing one scale_2 (the conversion guide's w1/w3 of routed experts):
+    the one holding the group's largest exponent casts as it does alone; the other uses
+    the shared s2, so its blocks exactly 17 below the GROUP maximum stay lossless and
+    those 18 below fall back, although alone they would all be in window."""
+    a_q = np.full((1, 64), 0x77, np.uint8)                    # every element 6.0
+    a_e = np.array([[127, 120, 127, 110]], np.uint8)          # k_max(A) = 0
+    b_q = np.full((1, 64), 0x35, np.uint8)                    # elements 3.0 and 1.5 (codes 5, 3)
+    b_e = np.array([[127 - WINDOW, 127 - WINDOW - 1, 127 - WINDOW - 1, 127 - 14]], np.uint8)
+    alone_a, alone_b = orc.mxfp4_to_nvfp4(a_q, a_e), orc.mxfp4_to_nvfp4(b_q, b_e)
+    ga, gb = orc.mxfp4_to_nvfp4_group([(a_q, a_e), (b_q, b_e)])
+    assert alone_b["counts"].tolist()[:2] == [8, 0]             # alone: k_max(B) = -14, all in window
+    for k in ("nv_q", "nv_scales"):
+        assert np.array_equal(ga[k], alone_a[k])
+    assert ga["s2"] == gb["s2"] == alone_a["s2"] and ga["global_amax"] == gb["global_amax"]
+    assert gb["k_max"] == 0
+    assert gb["counts"].tolist() == [4, 4, 4]                   # blocks 0 and 3 in window, 1 and 2 fall back
+    mx = _dequant_mx(b_q, b_e).numpy().reshape(-1, 16).view(np.uint32)
+    nv = _dequant_nv(gb["nv_q"], gb["nv_scales"], gb["s2"]).numpy().reshape(-1, 16).view(np.uint32)
+    assert np.all(mx[[0, 1, 6, 7]] == nv[[0, 1, 6, 7]])
+    # fallback blocks: 3.0 * 2^-18 and 1.5 * 2^-18 against s2 = 2^-8 are far below the
+    # smallest E4M3 block scale (2^-9 * 2^-8), so they become zero blocks (scale code 0)
+    assert (gb["nv_scales"][0, 2:6] == 0).all()
+    # a group of one is the plain cast
+    (solo,) = orc.mxfp4_to_nvfp4_group([(b_q, b_e)])
+    assert np.array_equal(solo["nv_q"], alone_b["nv_q"]) and solo["s2"] == alone_b["s2"]

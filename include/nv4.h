@@ -262,9 +262,15 @@ typedef struct {
     uint8_t* nv_scales;
     float* d_global_amax;
     float* d_s2;
+    int32_t group;      /* < 0: the matrix has its own scale_2.  Jobs of one call with the
+                           same group id >= 0 share one scale_2 ([CAST] section 3: routed
+                           experts' w1 and w3 with one scale_2): k_max is the largest
+                           exponent over all of their E8M0 codes, each member's window and
+                           fallback are taken against it, and every member's d_s2 and
+                           d_global_amax receive the shared values. */
 } nv4_cast_job;
 
-/* Batched form: one launch for many matrices (each with its own k_max).
+/* Batched form: one launch for many matrices (each with its own k_max unless grouped).
  * At most 128 jobs per call (NV4_ERR_LIMIT beyond). */
 NV4_API nv4_status nv4_mxfp4_to_nvfp4_batched(const nv4_cast_job* jobs, int n_jobs,
                                       unsigned long long* d_counts, uint32_t* d_flags, void* stream);

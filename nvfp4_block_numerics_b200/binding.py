@@ -45,7 +45,7 @@ class SweepJob(C.Structure):
 
 class CastJob(C.Structure):
     _fields_ = [("mx_q", _vp), ("e8m0", _vp), ("rows", _i64), ("cols", _i64), ("nv_q", _vp),
-                ("nv_scales", _vp), ("d_global_amax", _vp), ("d_s2", _vp)]
+                ("nv_scales", _vp), ("d_global_amax", _vp), ("d_s2", _vp), ("group", C.c_int32)]
 
 
 class NV4Error(RuntimeError):
@@ -241,7 +241,7 @@ def nv4_scale_sweep_batched(jobs: list[dict], d_flags=None, stream=None):
            "nv4_scale_sweep_batched")
 
 
-def _cjob(mx_q, e8m0, nv_q, nv_scales, d_global_amax, d_s2) -> CastJob:
+def _cjob(mx_q, e8m0, nv_q, nv_scales, d_global_amax, d_s2, group: int = -1) -> CastJob:
     rows, half = mx_q.shape
     cols = 2 * half
     for t, shape, name in ((mx_q, (rows, half), "mx_q"), (e8m0, (rows, cols // 32), "e8m0"),
@@ -249,7 +249,7 @@ def _cjob(mx_q, e8m0, nv_q, nv_scales, d_global_amax, d_s2) -> CastJob:
         if t.dtype != torch.uint8 or tuple(t.shape) != shape or not t.is_contiguous():
             raise NV4Error(f"{name} must be a contiguous uint8 tensor {shape}")
     return CastJob(_ptr(mx_q), _ptr(e8m0), rows, cols, _ptr(nv_q), _ptr(nv_scales),
-                   _scalar_f32(d_global_amax, "d_global_amax"), _scalar_f32(d_s2, "d_s2"))
+                   _scalar_f32(d_global_amax, "d_global_amax"), _scalar_f32(d_s2, "d_s2"), int(group))
 
 
 def nv4_mxfp4_to_nvfp4(mx_q, e8m0, nv_q, nv_scales, d_global_amax, d_s2, d_counts=None, d_flags=None, stream=None):
@@ -259,7 +259,8 @@ def nv4_mxfp4_to_nvfp4(mx_q, e8m0, nv_q, nv_scales, d_global_amax, d_s2, d_count
 
 
 def nv4_mxfp4_to_nvfp4_batched(jobs: list[dict], d_counts=None, d_flags=None, stream=None):
-    """jobs: dicts with keys mx_q, e8m0, nv_q, nv_scales, d_global_amax, d_s2."""
+    """jobs: dicts with keys mx_q, e8m0, nv_q, nv_scales, d_global_amax, d_s2 and optional group
+    (jobs with the same group id >= 0 share one scale_2)."""
     arr = (CastJob * len(jobs))(*[_cjob(**j) for j in jobs])
     _check(lib().nv4_mxfp4_to_nvfp4_batched(arr, len(jobs), _ptr(d_counts), _ptr(d_flags), _stream(stream)),
            "nv4_mxfp4_to_nvfp4_batched")

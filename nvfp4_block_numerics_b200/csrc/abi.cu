@@ -275,7 +275,7 @@ nv4_status nv4_mxfp4_to_nvfp4(const uint8_t* mx_q, const uint8_t* e8m0, int64_t 
 {
     nv4_cast_job j;
     j.mx_q = mx_q; j.e8m0 = e8m0; j.rows = rows; j.cols = cols; j.nv_q = nv_q; j.nv_scales = nv_scales;
-    j.d_global_amax = d_global_amax; j.d_s2 = d_s2;
+    j.d_global_amax = d_global_amax; j.d_s2 = d_s2; j.group = -1;
     return nv4_mxfp4_to_nvfp4_batched(&j, 1, d_counts, d_flags, stream);
 }
 

@@ -7,9 +7,10 @@
 //   re-quantized from its exact values e2m1 * 2^k_j (rare fallback path).
 //
 // Two stream-ordered kernels, no scratch memory:
-//  1. cast_kmax_kernel: one thread-block cluster of kKmaxCluster CTAs per matrix reads
-//     only the E8M0 bytes, reduces the largest valid code through distributed shared
-//     memory and writes the matrix's outputs s2 = 2^m and global_amax = 6*448*2^m;
+//  1. cast_kmax_kernel: one thread-block cluster of kKmaxCluster CTAs per scale_2 set (a
+//     matrix, or a group of matrices sharing one scale_2, [CAST] section 3) reads only
+//     the E8M0 bytes, reduces the largest valid code through distributed shared memory
+//     and writes every member's outputs s2 = 2^m and global_amax = 6*448*2^m;
 //  2. cast_rewrite_kernel: a flat grid over the MX blocks of every matrix (a warp takes
 //     256 consecutive blocks per step, lane-interleaved so each instruction moves
 //     contiguous bytes) recovers k_max = m + 8 exactly from the s2 it reads back, writes
@@ -37,6 +38,9 @@ struct CastJobDev {
 
 struct CastParams {
     int n;
+    int n_sets;                                   // scale_2 groups (sets of jobs sharing k_max)
+    uint16_t set_begin[kMaxCastJobs + 1];         // members of set g: set_jobs[set_begin[g] .. set_begin[g+1])
+    uint16_t set_jobs[kMaxCastJobs];
     uint32_t groups;                              // total 256-block tiles
     unsigned long long* d_counts;
     uint32_t* d_flags;
@@ -145,14 +149,10 @@ cast_kmax_kernel(const __grid_constant__ CastParams p)
     __shared__ uint32_t red[kCastThreads / 32];
     __shared__ uint32_t cta_max;
     const uint32_t rank = cluster_rank_c();
-    const CastJobDev& job = p.jobs[blockIdx.x / kKmaxCluster];
-    // share of this CTA, 16-aligned so it moves in 16-byte words
-    const uint32_t per = ((job.nb + kKmaxCluster - 1) / kKmaxCluster + 15u) & ~15u;
-    const uint32_t g0 = min(job.nb, rank * per), g1 = min(job.nb, g0 + per);
+    const int set = blockIdx.x / kKmaxCluster;
+    const int m0 = p.set_begin[set], m1 = p.set_begin[set + 1];
 
     uint32_t mx = 0u, flags = 0u;                                   // four per-byte maxima
-    const uint32_t nvec = (g1 - g0) / 16u;
-    const uint4* src = reinterpret_cast<const uint4*>(job.e8m0 + g0);
     auto scan = [&](const uint4& w) {
         const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
@@ -163,20 +163,29 @@ cast_kmax_kernel(const __grid_constant__ CastParams p)
             mx = __vmaxu4(mx, ws[k] & ~nan);
         }
     };
-    uint32_t v = threadIdx.x;
-    for (; v + 3u * kCastThreads < nvec; v += 4u * kCastThreads) {  // four loads in flight
-        uint4 w[4];
+    uint32_t mtail = 0u;                                            // scalar maximum of the tails
+    for (int mi = m0; mi < m1; ++mi) {                              // every matrix of the set
+        const CastJobDev& job = p.jobs[p.set_jobs[mi]];
+        // share of this CTA, 16-aligned so it moves in 16-byte words
+        const uint32_t per = ((job.nb + kKmaxCluster - 1) / kKmaxCluster + 15u) & ~15u;
+        const uint32_t g0 = min(job.nb, rank * per), g1 = min(job.nb, g0 + per);
+        const uint32_t nvec = (g1 - g0) / 16u;
+        const uint4* src = reinterpret_cast<const uint4*>(job.e8m0 + g0);
+        uint32_t v = threadIdx.x;
+        for (; v + 3u * kCastThreads < nvec; v += 4u * kCastThreads) {  // four loads in flight
+            uint4 w[4];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) w[k] = __ldcs(src + v + k * kCastThreads);
+            for (int k = 0; k < 4; ++k) w[k] = __ldcs(src + v + k * kCastThreads);
 #pragma unroll
-        for (int k = 0; k < 4; ++k) scan(w[k]);
+            for (int k = 0; k < 4; ++k) scan(w[k]);
+        }
+        for (; v < nvec; v += kCastThreads) scan(__ldcs(src + v));
+        for (uint32_t g = g0 + nvec * 16u + threadIdx.x; g < g1; g += kCastThreads) {
+            const uint32_t c = job.e8m0[g];
+            if (c == 0xFFu) flags |= kFlagE8M0Nan; else mtail = max(mtail, c);
+        }
     }
-    for (; v < nvec; v += kCastThreads) scan(__ldcs(src + v));
-    mx = max(max(mx & 0xFFu, (mx >> 8) & 0xFFu), max((mx >> 16) & 0xFFu, mx >> 24));
-    for (uint32_t g = g0 + nvec * 16u + threadIdx.x; g < g1; g += kCastThreads) {
-        const uint32_t c = job.e8m0[g];
-        if (c == 0xFFu) flags |= kFlagE8M0Nan; else mx = max(mx, c);
-    }
+    mx = max(max(max(mx & 0xFFu, (mx >> 8) & 0xFFu), max((mx >> 16) & 0xFFu, mx >> 24)), mtail);
     mx = __reduce_max_sync(0xFFFFFFFFu, mx);
     if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mx;
     __syncthreads();
@@ -189,13 +198,14 @@ cast_kmax_kernel(const __grid_constant__ CastParams p)
     if (rank == 0 && threadIdx.x < 32) {                           // one warp gathers the partial maxima
         uint32_t c = threadIdx.x < kKmaxCluster ? ld_dsmem_u32(&cta_max, threadIdx.x) : 0u;
         c = __reduce_max_sync(0xFFFFFFFFu, c);
-        if (threadIdx.x == 0) {
-            const float s2 = exp2_exact((int)c - 127 - 8);           // m = k_max - 8 in [-135, 119]
-            const float ga = __fmul_rn(2688.0f, s2);                 // 6*448*2^m
+        const float s2 = exp2_exact((int)c - 127 - 8);               // m = k_max - 8 in [-135, 119]
+        const float ga = __fmul_rn(2688.0f, s2);                     // 6*448*2^m
+        for (int mi = m0 + (int)threadIdx.x; mi < m1; mi += 32) {    // every member gets the set's scale_2
+            const CastJobDev& job = p.jobs[p.set_jobs[mi]];
             *job.d_s2 = s2;
             *job.d_ga = ga;
-            if (!isfinite(ga)) flags |= kFlagOverflow;
         }
+        if (threadIdx.x == 0 && !isfinite(ga)) flags |= kFlagOverflow;
     }
     cluster_sync_c();                                               // all remote reads done
     flags = __reduce_or_sync(0xFFFFFFFFu, flags);
@@ -310,9 +320,31 @@ cudaError_t launch_cast(const nv4_cast_job* jobs, int n, unsigned long long* d_c
     p.n = m;
     p.groups = groups;
     if (m == 0) return cudaSuccess;
+    // scale_2 sets: jobs with the same non-negative group id share one k_max
+    {
+        int order[kMaxCastJobs];
+        int32_t gid[kMaxCastJobs];
+        int mm = 0;
+        for (int i = 0; i < n; ++i)
+            if (jobs[i].rows != 0 && jobs[i].cols != 0) gid[mm++] = jobs[i].group;
+        bool taken[kMaxCastJobs] = {};
+        int k = 0, sets = 0;
+        for (int i = 0; i < m; ++i) {
+            if (taken[i]) continue;
+            p.set_begin[sets++] = (uint16_t)k;
+            order[k++] = i;
+            taken[i] = true;
+            if (gid[i] < 0) continue;
+            for (int j = i + 1; j < m; ++j)
+                if (!taken[j] && gid[j] == gid[i]) { order[k++] = j; taken[j] = true; }
+        }
+        p.set_begin[sets] = (uint16_t)k;
+        p.n_sets = sets;
+        for (int i = 0; i < m; ++i) p.set_jobs[i] = (uint16_t)order[i];
+    }
 
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(m * kKmaxCluster), 1, 1);
+    cfg.gridDim = dim3((unsigned)(p.n_sets * kKmaxCluster), 1, 1);
     cfg.blockDim = dim3(kCastThreads, 1, 1);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = s;

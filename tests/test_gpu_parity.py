@@ -426,6 +426,35 @@ def test_sweep_ill_conditioned_hessian(orc):
     assert st["mismatch_frac"] < 1e-3
 
 
+def test_sweep_grouped_scale2(orc):
+    """Two matrices sharing one scale_2 (w1/w3 style): both amaxes accumulate into one
+    device float (the running-max contract of nv4_tensor_amax), so both sweeps use
+    s2 = RN32(max(amax1, amax3) / 2688); the oracle gets that group amax."""
+    rng = np.random.default_rng(80)
+    x = inputs.laplace_bf16(inputs.rng_for(80, "gpu", "sweepg"), 512, 64)
+    H = orc.hessian_accum(x).astype(np.float32)
+    w1 = (rng.standard_normal((96, 64)) * 0.02).astype(np.float32)
+    w3 = (rng.standard_normal((96, 64)) * 0.05).astype(np.float32)
+    d_amax = torch.zeros(1, dtype=torch.float32, device=G.DEV)
+    jobs = []
+    for w in (w1, w3):
+        wd = G.f32_dev(w)
+        nv4.nv4_tensor_amax(wd, d_amax)
+        jobs.append(dict(w=wd, H=G.f32_dev(H), d_amax_w=d_amax,
+                         codes=torch.empty((96, 4), dtype=torch.uint8, device=G.DEV),
+                         q=torch.empty((96, 32), dtype=torch.uint8, device=G.DEV),
+                         cost1=torch.empty((96, 4), dtype=torch.float32, device=G.DEV),
+                         cost2=torch.empty((96, 4), dtype=torch.float32, device=G.DEV)))
+    nv4.nv4_scale_sweep_batched(jobs)
+    torch.cuda.synchronize()
+    amax = max(orc.tensor_amax(w1)[0], orc.tensor_amax(w3)[0])
+    assert d_amax.item() == amax
+    for w, j in zip((w1, w3), jobs):
+        ref = orc.scale_sweep(w, H.astype(np.float64), amax)
+        st = G.sweep_parity(G.host(j["codes"]), G.host(j["q"]), G.host(j["cost1"]), ref, c2_gpu=G.host(j["cost2"]))
+        assert st["mismatch_frac"] < 1e-3
+
+
 def test_sweep_work_counter(orc):
     """Bounds on: far fewer than 127 costs per block; bounds off (correlated channels):
     every candidate visited and evaluated; the winners match the oracle either way."""
@@ -507,18 +536,24 @@ def test_sweep_moe_batched_sampled(orc):
 
 
 # ------------------------------------------------------------------ cast
-def _cast_check(orc, mats, in_place=False):
+def _cast_check(orc, mats, in_place=False, groups=None):
     jobs, refs = [], []
     counts = torch.zeros(3, dtype=torch.int64, device=G.DEV)
     f = G.flags_dev()
-    for mxq, e8 in mats:
+    groups = [-1] * len(mats) if groups is None else groups
+    for (mxq, e8), g in zip(mats, groups):
         mq = G.u8_dev(mxq)
         rows, half = mxq.shape
         jobs.append(dict(mx_q=mq, e8m0=G.u8_dev(e8), nv_q=mq if in_place else torch.empty_like(mq),
                          nv_scales=torch.empty((rows, half // 8), dtype=torch.uint8, device=G.DEV),
                          d_global_amax=torch.empty(1, dtype=torch.float32, device=G.DEV),
-                         d_s2=torch.empty(1, dtype=torch.float32, device=G.DEV)))
-        refs.append(orc.mxfp4_to_nvfp4(mxq, e8))
+                         d_s2=torch.empty(1, dtype=torch.float32, device=G.DEV), group=g))
+        if g < 0:
+            refs.append(orc.mxfp4_to_nvfp4(mxq, e8))
+        else:
+            members = [i for i, h in enumerate(groups) if h == g]
+            res = orc.mxfp4_to_nvfp4_group([mats[i] for i in members])
+            refs.append(res[members.index(len(refs))])
     nv4.nv4_mxfp4_to_nvfp4_batched(jobs, counts, f)
     torch.cuda.synchronize()
     assert f.item() == 0
@@ -539,6 +574,26 @@ def test_cast_small_and_edges(orc):
     mats.append((np.full((1, 64), 0x77, np.uint8), e))
     _cast_check(orc, mats)
     _cast_check(orc, mats, in_place=True)
+
+
+def test_cast_grouped_scale2(orc):
+    """Matrices sharing one scale_2: the window-edge example, random pairs whose members
+    sit apart in the job list, singletons and one-member groups in the same call."""
+    win = 17
+    a = (np.full((1, 64), 0x77, np.uint8), np.array([[127, 120, 127, 110]], np.uint8))
+    b = (np.full((1, 64), 0x35, np.uint8), np.array([[127 - win, 126 - win, 126 - win, 113]], np.uint8))
+    rnd = [inputs.mxfp4_matrix(inputs.rng_for(i, "gpu", "castg"), r, c, fallback_frac=0.02, mean_exp=-8.0 - 3 * (i % 2))
+           for i, (r, c) in enumerate([(3, 64), (17, 96), (64, 256), (64, 256), (5, 32)])]
+    mats = [a, rnd[0], b, rnd[1], rnd[2], rnd[3], rnd[4]]
+    groups = [7, 3, 7, -1, 3, 9, 11]
+    tot = _cast_check(orc, mats, groups=groups)
+    assert tot[1] > 0
+    _cast_check(orc, mats, in_place=True, groups=groups)
+
+
+def test_cast_expert_checkpoint_grouped_pairs(orc):
+    mats = [inputs.c5_cast(i) for i in range(32)]
+    _cast_check(orc, mats, groups=[i // 2 for i in range(32)])
 
 
 def test_cast_expert_checkpoint_full(orc):

@@ -492,16 +492,11 @@ def run_reference(args):
 def run_ours(args):
     import torch
 
-    ws, rank, local = dist_setup(args)
+    from nvfp4_block_numerics_b200 import dist
+
+    ws, rank, local = dist.init(backend="nccl", timeout_s=300)
     parts = [p for p in args.parts.split(",") if p]
-    if ws > 1:
-        import datetime
-
-        import torch.distributed as dist
-
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
-    else:
+    if ws == 1:
         torch.cuda.set_device(0)
     dev = torch.device("cuda", torch.cuda.current_device())
     from nvfp4_block_numerics_b200 import binding as nv4
@@ -526,8 +521,7 @@ def run_ours(args):
     torch.cuda.synchronize()
 
     clocks = ClockSampler(dev.index)
-    if ws > 1:
-        torch.distributed.barrier()
+    dist.barrier()
     torch.cuda.synchronize()
     clocks.start()
     time.sleep(0.3)
@@ -546,22 +540,20 @@ def run_ours(args):
             ev[p].append((a, b))
     end.record(stream)
     torch.cuda.synchronize()
-    if ws > 1:
-        torch.distributed.barrier()
+    dist.barrier()
     clk = clocks.stop()
     total_s = start.elapsed_time(end) / 1e3
     part_s = {p: sum(a.elapsed_time(b) for a, b in ev[p]) / 1e3 for p in parts}
-    if ws > 1:
-        t = torch.tensor([total_s] + [part_s[p] for p in parts], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_s = float(t[0])
-        part_s = {p: float(t[i + 1]) for i, p in enumerate(parts)}
+    t = dist.max_over_ranks([total_s] + [part_s[p] for p in parts])      # device times, max over ranks
+    total_s = t[0]
+    part_s = {p: t[i + 1] for i, p in enumerate(parts)}
     flags = int(W["flags"].item())
 
     roof = kernel_rooflines(W, hbm_peak)
     e2e = None
     if "act" in parts and not args.no_e2e:
         e2e_s, h2d, d2h = e2e_act(W, max(1, min(args.steps, 3)))
+        e2e_s = dist.max_over_ranks([e2e_s])[0]
         bytes_act, _ = act_bytes(W)
         e2e = {"value": ws * bytes_act / e2e_s / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_s * 1e3}
@@ -569,9 +561,7 @@ def run_ours(args):
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(args.seed)
 
-    if ws > 1:
-        torch.distributed.barrier()
-        torch.distributed.destroy_process_group()
+    dist.finalize()
     if rank != 0:
         return
 

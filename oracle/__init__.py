@@ -365,3 +365,45 @@ def mxfp4_to_nvfp4_group(mats, threads: int | None = None):
     mats = [_mx_check(q, e) for q, e in mats]
     kmax = max(_mx_kmax(e) for _, e in mats)
     return [mxfp4_to_nvfp4(q, e, threads, k_max=kmax) for q, e in mats]
+
+
+# ---------------------------------------------------------------- W4A4 GEMM (NVFP4 x NVFP4)
+def _dequant_exact(q: np.ndarray, sc: np.ndarray, s2: float) -> np.ndarray:
+    """Exact dequantized values e2m1(code) * e4m3(s_b) * s2 in FP64 (each factor has at
+    most 24 significant bits and the product at most 31, so FP64 holds it exactly)."""
+    e2m1 = np.array([e2m1_value(c) for c in range(16)], np.float64)
+    e4m3 = np.array([e4m3_value(c) for c in range(256)], np.float64)
+    q = np.ascontiguousarray(q)
+    nib = np.stack([q & 15, q >> 4], axis=-1).reshape(q.shape[0], -1)
+    s = np.repeat(e4m3[np.ascontiguousarray(sc)], 16, axis=1)
+    return e2m1[nib] * s * float(s2)
+
+
+def gemm_nvfp4(qa, sa, s2a: float, qb, sb, s2b: float):
+    """NVFP4 x NVFP4 GEMM, D[m, n] = sum_k A[m, k] * B[n, k] with A and B the exact
+    dequantized values of packed codes q [rows, K/2], E4M3 scales [rows, K/16] and FP32
+    second-level scales ([FP4] section 4.1: block-scaled FP4 matrix multiply on tcgen05;
+    [CAST] section 4: W4A4, activations and weights both NVFP4).
+
+    Returns (D, Dabs): D in FP64 (the product of the exactly dequantized matrices, one
+    library matmul), and Dabs = |A| |B|^T, the scale of the accumulation error bound."""
+    A = _dequant_exact(qa, sa, s2a)
+    B = _dequant_exact(qb, sb, s2b)
+    return A @ B.T, np.abs(A) @ np.abs(B).T
+
+
+def scales_to_mma_layout(sc: np.ndarray) -> np.ndarray:
+    """Block-scale bytes [rows, kb] (kb = K/16) rearranged into the layout that the
+    Blackwell block-scaled MMA reads ([FP4] section 4.1: scale factors reorganized for
+    tcgen05.mma): 512-byte atoms of 128 rows x 4 scales, atom (r // 128, j // 4) at
+    ((r // 128) * ceil(kb / 4) + j // 4) * 512, and inside an atom row r, scale j at
+    (r % 32) * 16 + ((r % 128) // 32) * 4 + j % 4.  Rows and scale columns are padded
+    with zeros to multiples of 128 and 4."""
+    rows, kb = sc.shape
+    rt, kt = -(-rows // 128), -(-kb // 4)
+    out = np.zeros(rt * kt * 512, np.uint8)
+    r = np.arange(rows)[:, None]
+    j = np.arange(kb)[None, :]
+    off = ((r // 128) * kt + j // 4) * 512 + (r % 32) * 16 + ((r % 128) // 32) * 4 + j % 4
+    out[off] = sc
+    return out

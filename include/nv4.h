@@ -276,6 +276,34 @@ NV4_API nv4_status nv4_mxfp4_to_nvfp4_batched(const nv4_cast_job* jobs, int n_jo
                                       unsigned long long* d_counts, uint32_t* d_flags, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * W4A4 GEMM on the Blackwell block-scaled tensor cores ([FP4] section 4.1: tcgen05.mma
+ * with reorganized scale factors; [CAST] section 4: activations and weights NVFP4).
+ *
+ * nv4_mma_scale_bytes / nv4_scales_to_mma_layout -- the block scales [rows, cols/16]
+ * written by nv4_act_quant, nv4_weight_quant_rtn or nv4_scale_sweep, rearranged into
+ * the layout the MMA reads: 512-byte atoms of 128 rows x 4 scales; atom (r/128, j/4)
+ * starts at ((r/128) * ceil(cols/64) + j/4) * 512 and holds scale (r, j) at byte
+ * (r%32)*16 + ((r%128)/32)*4 + j%4.  Rows pad to 128 and scale columns to 4, with
+ * zeros.  out: nv4_mma_scale_bytes(rows, cols) bytes, 16-byte aligned.  The size
+ * function returns 0 for invalid shapes.
+ *
+ * nv4_gemm_nvfp4 -- D[m, n] = s2_A * s2_B * sum_k A[m, k] * B[n, k] for NVFP4 operands
+ * given as packed codes qa [M, K/2], qb [N, K/2] (contiguous, 16-byte aligned), their
+ * scales in the MMA layout, and device FP32 second-level scales d_s2a, d_s2b.  Products
+ * of E2M1 values and E4M3 scales are exact; accumulation is FP32 on the tensor cores;
+ * out (NV4_BF16 or NV4_FP32, [M, N] with leading dimension ldd) is RN of the FP32
+ * accumulator times RN32(s2_A * s2_B).  Shapes: M % 128 == 0, N % 128 == 0,
+ * K % 256 == 0 (NV4_ERR_SHAPE otherwise).
+ */
+NV4_API size_t nv4_mma_scale_bytes(int64_t rows, int64_t cols);
+NV4_API nv4_status nv4_scales_to_mma_layout(const uint8_t* scales, int64_t rows, int64_t cols, uint8_t* out,
+                                    void* stream);
+NV4_API nv4_status nv4_gemm_nvfp4(const uint8_t* qa, const uint8_t* sfa_mma, const float* d_s2a,
+                          const uint8_t* qb, const uint8_t* sfb_mma, const float* d_s2b,
+                          int64_t M, int64_t N, int64_t K, nv4_dtype out_dt, void* out, int64_t ldd,
+                          uint32_t* d_flags, void* stream);
+
+/* ---------------------------------------------------------------------------
  * nv4_selftest -- checks, on the current device, the hardware FP4/FP8 conversion
  * instructions the kernels rely on (lane order, rounding, sign of zero, saturation).
  * Writes 64 uint32 results to d_out (device); d_out[0] is a bit mask of failed

@@ -20,7 +20,8 @@ from .build import LIB_PATH
 
 __all__ = [
     "NV4Error", "lib", "nv4_tensor_amax", "nv4_act_quant", "nv4_weight_quant_rtn", "nv4_fake_qdq",
-    "nv4_dequant", "nv4_hessian_accum", "weight_quant_rtn", "fake_qdq",
+    "nv4_dequant", "nv4_hessian_accum", "weight_quant_rtn", "fake_qdq", "nv4_mma_scale_bytes",
+    "nv4_scales_to_mma_layout", "nv4_gemm_nvfp4", "mma_scales", "gemm_nvfp4",
     "nv4_hessian_accum_batched", "nv4_scale_sweep", "nv4_scale_sweep_batched", "nv4_mxfp4_to_nvfp4",
     "nv4_mxfp4_to_nvfp4_batched", "nv4_selftest", "nv4_version", "FLAG_NONFINITE", "FLAG_E8M0_NAN",
     "FLAG_OVERFLOW", "FLAG_TIMEOUT", "tensor_amax", "act_quant", "dequant", "hessian_accum",
@@ -63,6 +64,9 @@ _SIGS = {
     "nv4_weight_quant_rtn": (C.c_int, [_vp, C.c_int, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp]),
     "nv4_fake_qdq": (C.c_int, [_vp, _i64, _i64, _i64, _vp, C.c_int, _vp, _i64, _vp, _vp, _vp]),
     "nv4_dequant": (C.c_int, [_vp, _vp, _vp, _i64, _i64, C.c_int, _vp, _vp]),
+    "nv4_mma_scale_bytes": (C.c_size_t, [_i64, _i64]),
+    "nv4_scales_to_mma_layout": (C.c_int, [_vp, _i64, _i64, _vp, _vp]),
+    "nv4_gemm_nvfp4": (C.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, C.c_int, _vp, _i64, _vp, _vp]),
     "nv4_hessian_accum": (C.c_int, [_vp, _i64, _i64, _i64, _vp, _vp, _vp]),
     "nv4_hessian_accum_batched": (C.c_int, [C.POINTER(HessianJob), C.c_int, _vp, _vp]),
     "nv4_scale_sweep": (C.c_int, [_vp, C.c_int, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
@@ -306,6 +310,56 @@ def fake_qdq(x: torch.Tensor, d_amax: torch.Tensor, dtype=torch.bfloat16, d_flag
     s2 = torch.empty((1,), dtype=torch.float32, device=x.device)
     nv4_fake_qdq(x, d_amax, out, s2, d_flags, stream)
     return out, s2
+
+
+def nv4_mma_scale_bytes(rows: int, cols: int) -> int:
+    return int(lib().nv4_mma_scale_bytes(rows, cols))
+
+
+def nv4_scales_to_mma_layout(scales: torch.Tensor, out: torch.Tensor, stream=None):
+    """scales: contiguous uint8 [rows, cols/16]; out: uint8, nv4_mma_scale_bytes(rows, cols) bytes."""
+    if scales.dtype != torch.uint8 or scales.dim() != 2 or not scales.is_contiguous():
+        raise NV4Error("scales must be a contiguous uint8 tensor [rows, cols/16]")
+    rows, kb = scales.shape
+    need = nv4_mma_scale_bytes(rows, 16 * kb)
+    if out.dtype != torch.uint8 or out.numel() < need or not out.is_contiguous():
+        raise NV4Error(f"out must be a contiguous uint8 tensor of at least {need} bytes")
+    _check(lib().nv4_scales_to_mma_layout(_ptr(scales), rows, 16 * kb, _ptr(out), _stream(stream)),
+           "nv4_scales_to_mma_layout")
+
+
+def nv4_gemm_nvfp4(qa, sfa_mma, d_s2a, qb, sfb_mma, d_s2b, out, d_flags=None, stream=None):
+    """out[M, N] = s2a * s2b * A @ B^T for NVFP4 operands (codes [rows, K/2], MMA-layout scales)."""
+    M, half = qa.shape
+    N = qb.shape[0]
+    K = 2 * half
+    for t, shape, name in ((qa, (M, half), "qa"), (qb, (N, half), "qb")):
+        if t.dtype != torch.uint8 or tuple(t.shape) != shape or not t.is_contiguous():
+            raise NV4Error(f"{name} must be a contiguous uint8 tensor {shape}")
+    for t, rows, name in ((sfa_mma, M, "sfa_mma"), (sfb_mma, N, "sfb_mma")):
+        if t.dtype != torch.uint8 or t.numel() < nv4_mma_scale_bytes(rows, K):
+            raise NV4Error(f"{name} must hold nv4_mma_scale_bytes({rows}, {K}) bytes")
+    if out.dtype not in (torch.bfloat16, torch.float32):
+        raise NV4Error("out must be bf16 or float32")
+    orows, ocols, ldd = _rowmajor(out, "out")
+    if (orows, ocols) != (M, N):
+        raise NV4Error("out must be [M, N]")
+    _check(lib().nv4_gemm_nvfp4(_ptr(qa), _ptr(sfa_mma), _scalar_f32(d_s2a, "d_s2a"), _ptr(qb), _ptr(sfb_mma),
+                                _scalar_f32(d_s2b, "d_s2b"), M, N, K, _DT[out.dtype], _ptr(out), ldd, _ptr(d_flags),
+                                _stream(stream)), "nv4_gemm_nvfp4")
+
+
+def mma_scales(scales: torch.Tensor, stream=None) -> torch.Tensor:
+    rows, kb = scales.shape
+    out = torch.empty(nv4_mma_scale_bytes(rows, 16 * kb), dtype=torch.uint8, device=scales.device)
+    nv4_scales_to_mma_layout(scales, out, stream)
+    return out
+
+
+def gemm_nvfp4(qa, sa, d_s2a, qb, sb, d_s2b, dtype=torch.bfloat16, d_flags=None, stream=None):
+    out = torch.empty((qa.shape[0], qb.shape[0]), dtype=dtype, device=qa.device)
+    nv4_gemm_nvfp4(qa, mma_scales(sa, stream), d_s2a, qb, mma_scales(sb, stream), d_s2b, out, d_flags, stream)
+    return out
 
 
 def dequant(q, scales, d_s2, dtype=torch.bfloat16, stream=None):

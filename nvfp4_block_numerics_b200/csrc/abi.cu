@@ -286,3 +286,39 @@ nv4_status nv4_selftest(uint32_t* d_out, void* stream)
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------ W4A4 GEMM
+size_t nv4_mma_scale_bytes(int64_t rows, int64_t cols)
+{
+    if (rows <= 0 || cols <= 0 || cols % 16 != 0) return 0;
+    return mma_scale_bytes(rows, cols / 16);
+}
+
+nv4_status nv4_scales_to_mma_layout(const uint8_t* scales, int64_t rows, int64_t cols, uint8_t* out, void* stream)
+{
+    if (rows < 0 || cols < 0 || cols % 16 != 0) return NV4_ERR_SHAPE;
+    if (rows == 0 || cols == 0) return NV4_OK;
+    if (scales == nullptr || out == nullptr) return NV4_ERR_NULL;
+    if (!aligned16(out)) return NV4_ERR_ALIGN;
+    if (mma_scale_bytes(rows, cols / 16) >= ((size_t)1 << 34)) return NV4_ERR_LIMIT;
+    return from_cuda(launch_mma_scale_layout(scales, rows, cols / 16, out, (cudaStream_t)stream));
+}
+
+nv4_status nv4_gemm_nvfp4(const uint8_t* qa, const uint8_t* sfa_mma, const float* d_s2a, const uint8_t* qb,
+                          const uint8_t* sfb_mma, const float* d_s2b, int64_t M, int64_t N, int64_t K,
+                          nv4_dtype out_dt, void* out, int64_t ldd, uint32_t* d_flags, void* stream)
+{
+    if (out_dt != NV4_BF16 && out_dt != NV4_FP32) return NV4_ERR_DTYPE;
+    if (M < 0 || N < 0 || K < 0 || M % 128 != 0 || N % 128 != 0 || K % 256 != 0 || ldd < N) return NV4_ERR_SHAPE;
+    if (M == 0 || N == 0) return NV4_OK;
+    if (K == 0) return NV4_ERR_SHAPE;
+    if (qa == nullptr || sfa_mma == nullptr || d_s2a == nullptr || qb == nullptr || sfb_mma == nullptr ||
+        d_s2b == nullptr || out == nullptr)
+        return NV4_ERR_NULL;
+    if (!aligned16(qa) || !aligned16(qb) || !aligned16(sfa_mma) || !aligned16(sfb_mma) || !aligned16(out) ||
+        ldd % (out_dt == NV4_FP32 ? 4 : 8) != 0)
+        return NV4_ERR_ALIGN;
+    if (M / 128 * (N / 128) >= ((int64_t)1 << 31) || K / 2 >= ((int64_t)1 << 32)) return NV4_ERR_LIMIT;
+    return from_cuda(launch_gemm_nvfp4(qa, sfa_mma, d_s2a, qb, sfb_mma, d_s2b, M, N, K, (int)out_dt, out, ldd,
+                                       d_flags, (cudaStream_t)stream));
+}

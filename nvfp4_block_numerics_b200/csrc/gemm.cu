@@ -1,0 +1,426 @@
+// gemm.cu -- NVFP4 x NVFP4 block-scaled GEMM on the 5th-generation tensor cores (sm_100a).
+//
+// [FP4] section 4.1 (block-scaled FP4 matrix multiply with tcgen05.mma and scale
+// factors reorganized for it), [CAST] section 4 (W4A4: activations and weights both
+// NVFP4).  D[m, n] = s2_A * s2_B * sum_k (e2m1(a_mk) * sA[m, k/16]) * (e2m1(b_nk) * sB[n, k/16]),
+// i.e. the product of the two dequantized matrices, accumulated in FP32 and written
+// as BF16 or FP32.
+//
+// Kernel structure (one CTA = one 128 x 128 output tile, 128 threads):
+//   * warp 0, one lane: producer.  Per stage of 256 K-elements it loads the A and B code
+//     tiles (128 rows x 128 bytes each) with 2-D TMA into 128-byte-swizzled shared
+//     memory, and the stage's scale-factor atoms (4 x 512 bytes per operand, already in
+//     the MMA layout, see nv4_scales_to_mma_layout) with 1-D bulk copies, all completing
+//     on the stage's mbarrier.  A 4-stage ring; a stage is reused once the MMAs that
+//     read it have completed (tcgen05.commit on the stage's "empty" mbarrier).
+//   * warp 1: allocates 256 tensor-memory columns (the 128 x 128 FP32 accumulator and
+//     two scale-factor buffers); one lane issues, per stage, tcgen05.cp of the scale
+//     atoms into tensor memory and four tcgen05.mma kind::mxf4nvf4 block16 (K = 64
+//     each) with both operands read from shared memory through matrix descriptors.
+//   * all four warps: epilogue.  Warp w reads accumulator lanes 32w..32w+31 with
+//     tcgen05.ld (one output row per thread), multiplies by s2_A * s2_B, and stores.
+// Every mbarrier wait is bounded (kWaitLimitNs); on expiry the kernel sets
+// NV4_FLAG_TIMEOUT, stops issuing, skips its stores, drains its copies in flight and
+// releases its tensor memory.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "nv4_common.cuh"
+#include "nv4_internal.h"
+
+namespace nv4 {
+
+namespace gemm {
+
+constexpr int kBM = 128, kBN = 128;
+constexpr int kBK = 256;                          // FP4 elements per stage (128 bytes per row)
+constexpr int kStages = 4;
+constexpr int kThreads = 128;
+constexpr uint32_t kTileBytes = 128 * 128;        // one operand's codes per stage
+constexpr uint32_t kSfBytes = 4 * 512;            // one operand's scale atoms per stage
+constexpr uint32_t kStageTx = 2 * kTileBytes + 2 * kSfBytes;
+constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kColSfA = 128, kColSfB = 160;  // two 16-column buffers each
+
+struct Smem {
+    uint8_t a[kStages][kTileBytes];               // 1024-byte aligned (128-byte swizzle atoms)
+    uint8_t b[kStages][kTileBytes];
+    uint8_t sfa[kStages][kSfBytes];
+    uint8_t sfb[kStages][kSfBytes];
+    uint64_t full[kStages], empty[kStages], acc_full;
+    uint32_t tmem_base;
+    uint32_t abort;                               // set by a wait that gave up
+    uint32_t issued, consumed;                    // stages loaded / stages handed to the MMA
+};
+
+struct Params {
+    CUtensorMap map_a, map_b;                     // codes [rows, K/2] bytes, 128 x 128-byte boxes
+    const uint8_t* sfa;                           // scale atoms in the MMA layout
+    const uint8_t* sfb;
+    const float* d_s2a;
+    const float* d_s2b;
+    void* out;
+    int64_t ldd;
+    uint32_t n_tiles, k_stages, kt4;              // kt4 = K / 64: scale atoms per 128-row tile
+    uint32_t* d_flags;
+};
+
+// ---------------------------------------------------------------- PTX helpers
+__device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(ok)
+                 : "r"(smem_u32(bar)), "r"(parity)
+                 : "memory");
+    return ok != 0u;
+}
+
+// Bounded wait: false when the phase did not complete within kWaitLimitNs.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity)
+{
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    while (!mbar_try_wait(bar, parity))
+        if (global_ns() - t0 > kWaitLimitNs) return false;
+    return true;
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+        ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar)
+{
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// Shared-memory matrix descriptor (Blackwell format): start address, leading and
+// stride byte offsets in 16-byte units, descriptor version 1 (bits 46-47) and the
+// layout/swizzle mode in bits 61-63 (0 none, 2 = 128-byte swizzle).
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo, uint32_t layout)
+{
+    return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)(lbo & 0x3FFFu) << 16) |
+           ((uint64_t)(sbo & 0x3FFFu) << 32) | (1ull << 46) | ((uint64_t)layout << 61);
+}
+
+// Instruction descriptor of kind::mxf4nvf4: A and B E2M1 (format 1), K-major, scale
+// factors UE4M3 (bit 23 = 0), N >> 3 in bits 17-22, M >> 4 in bits 24-28, dense K = 64.
+constexpr uint32_t kIdesc = (1u << 7) | (1u << 10) | ((uint32_t)(kBN >> 3) << 17) | ((uint32_t)(kBM >> 4) << 24);
+
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols)
+{
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+                 "r"(ncols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols)
+{
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+// Copies one 512-byte scale atom (32 rows x 16 bytes) into 4 tensor-memory columns,
+// replicated over the four 32-lane sub-partitions.
+__device__ __forceinline__ void tmem_cp_sf(uint32_t taddr, uint64_t desc)
+{
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(desc) : "memory");
+}
+
+__device__ __forceinline__ void mma_fp4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t sfa, uint32_t sfb,
+                                        uint32_t accumulate)
+{
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "setp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t"
+                 "}"
+                 ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+                 : "memory");
+}
+
+// Arrives on mbar once every tcgen05 operation issued so far by this thread completes.
+__device__ __forceinline__ void tc_commit(uint64_t* bar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+
+// 32 consecutive FP32 accumulator columns of this warp's 32 lanes (one row per thread).
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float v[32])
+{
+    uint32_t r[32];
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+                 "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+                 "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+                   "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+                   "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]),
+                   "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]),
+                   "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+                 : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+}  // namespace gemm
+
+namespace gemm {
+
+template <int kOut>   // 0 bf16, 2 fp32
+__global__ void __launch_bounds__(kThreads, 1)
+gemm_nvfp4_kernel(const __grid_constant__ Params p)
+{
+    extern __shared__ uint8_t smem_raw[];
+    Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t n_tile = blockIdx.x % p.n_tiles, m_tile = blockIdx.x / p.n_tiles;
+    const uint32_t KS = p.k_stages;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&sm.full[s], 1);
+            mbar_init(&sm.empty[s], 1);
+        }
+        mbar_init(&sm.acc_full, 1);
+        sm.abort = 0u;
+        sm.issued = sm.consumed = 0u;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&p.map_a)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&p.map_b)) : "memory");
+    }
+    if (warp == 1) tmem_alloc(&sm.tmem_base, kTmemCols);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+    uint32_t flags = 0u;
+
+    if (warp == 0) {
+        if (lane == 0) {                                           // producer
+            uint32_t ks = 0;
+            for (; ks < KS; ++ks) {
+                const uint32_t s = ks % kStages;
+                if (ks >= (uint32_t)kStages && !mbar_wait(&sm.empty[s], ((ks / kStages) - 1u) & 1u)) {
+                    flags |= kFlagTimeout;
+                    atomicOr(&sm.abort, 1u);
+                    break;
+                }
+                if (*reinterpret_cast<volatile uint32_t*>(&sm.abort) != 0u) break;
+                mbar_arrive_expect_tx(&sm.full[s], kStageTx);
+                tma_load_2d(sm.a[s], &p.map_a, &sm.full[s], (int)(ks * 128u), (int)(m_tile * kBM));
+                tma_load_2d(sm.b[s], &p.map_b, &sm.full[s], (int)(ks * 128u), (int)(n_tile * kBN));
+                bulk_load(sm.sfa[s], p.sfa + ((size_t)m_tile * p.kt4 + 4u * ks) * 512u, kSfBytes, &sm.full[s]);
+                bulk_load(sm.sfb[s], p.sfb + ((size_t)n_tile * p.kt4 + 4u * ks) * 512u, kSfBytes, &sm.full[s]);
+            }
+            sm.issued = ks;
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        if (lane == 0) {                                           // MMA issuer
+            uint32_t ks = 0;
+            for (; ks < KS; ++ks) {
+                const uint32_t s = ks % kStages;
+                if (!mbar_wait(&sm.full[s], (ks / kStages) & 1u)) {
+                    flags |= kFlagTimeout;
+                    atomicOr(&sm.abort, 1u);
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t buf = ks & 1u;
+                const uint32_t ta = tmem + kColSfA + 16u * buf, tb = tmem + kColSfB + 16u * buf;
+#pragma unroll
+                for (uint32_t j = 0; j < 4; ++j) {
+                    tmem_cp_sf(ta + 4u * j, smem_desc(smem_u32(sm.sfa[s] + 512u * j), 0u, 8u, 0u));
+                    tmem_cp_sf(tb + 4u * j, smem_desc(smem_u32(sm.sfb[s] + 512u * j), 0u, 8u, 0u));
+                }
+                const uint32_t a0 = smem_u32(sm.a[s]), b0 = smem_u32(sm.b[s]);
+#pragma unroll
+                for (uint32_t j = 0; j < 4; ++j)
+                    mma_fp4(tmem, smem_desc(a0 + 32u * j, 1u, 64u, 2u), smem_desc(b0 + 32u * j, 1u, 64u, 2u),
+                            ta + 4u * j, tb + 4u * j, (ks | j) != 0u ? 1u : 0u);
+                tc_commit(&sm.empty[s]);                           // frees the stage when these MMAs finish
+            }
+            sm.consumed = ks;
+            tc_commit(&sm.acc_full);                               // the accumulator is complete
+        }
+        __syncwarp();
+    }
+
+    // ---- epilogue: every warp, one accumulator row per thread
+    const bool acc_ok = mbar_wait(&sm.acc_full, 0u);
+    if (!acc_ok) flags |= kFlagTimeout;
+    tc_fence_after();
+    __syncwarp();
+    const bool store = acc_ok && *reinterpret_cast<volatile uint32_t*>(&sm.abort) == 0u && KS > 0u;
+    const float alpha = __fmul_rn(*p.d_s2a, *p.d_s2b);
+    const int64_t row = (int64_t)m_tile * kBM + 32 * warp + lane;
+#pragma unroll 1
+    for (int cb = 0; cb < kBN / 32; ++cb) {
+        float v[32];
+        tmem_ld32(tmem + ((uint32_t)(32 * warp) << 16) + (uint32_t)(32 * cb), v);
+        if (!store) continue;
+        const int64_t col = (int64_t)n_tile * kBN + 32 * cb;
+        if constexpr (kOut == 2) {
+            float4* o = reinterpret_cast<float4*>(static_cast<float*>(p.out) + row * p.ldd + col);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                o[i] = make_float4(__fmul_rn(v[4 * i], alpha), __fmul_rn(v[4 * i + 1], alpha),
+                                   __fmul_rn(v[4 * i + 2], alpha), __fmul_rn(v[4 * i + 3], alpha));
+        } else {
+            uint32_t w[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                asm("cvt.rn.bf16x2.f32 %0, %1, %2;"
+                    : "=r"(w[i])
+                    : "f"(__fmul_rn(v[2 * i + 1], alpha)), "f"(__fmul_rn(v[2 * i], alpha)));
+            uint4* o = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + row * p.ldd + col);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) o[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+        }
+    }
+
+    // ---- teardown: drain copies that were loaded but never consumed, free tensor memory
+    tc_fence_before();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        for (uint32_t ks = sm.consumed; ks < sm.issued; ++ks)
+            if (!mbar_wait(&sm.full[ks % kStages], (ks / kStages) & 1u)) flags |= kFlagTimeout;
+    }
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+    flags = __reduce_or_sync(0xFFFFFFFFu, flags);
+    if (lane == 0) flag_or(p.d_flags, flags);
+}
+
+// Block scales [rows, kb] (row-major, kb = K/16) -> the MMA atom layout, one thread per
+// 32-bit word (one row's 4 consecutive scales); padding rows and columns are zero.
+__global__ void __launch_bounds__(256)
+mma_scale_layout_kernel(const uint8_t* __restrict__ sc, uint32_t rows, uint32_t kb, uint32_t kt,
+                        uint32_t total_words, uint32_t* __restrict__ out)
+{
+    for (uint32_t w = blockIdx.x * 256u + threadIdx.x; w < total_words; w += gridDim.x * 256u) {
+        // word w = ((rt * kt) + g) * 128 + (r % 32) * 4 + (r % 128) / 32
+        const uint32_t atom = w >> 7, in = w & 127u;
+        const uint32_t rt = atom / kt, g = atom - rt * kt;
+        const uint32_t r = rt * 128u + (in >> 2) + 32u * (in & 3u);
+        uint32_t v = 0u;
+        if (r < rows) {
+            const uint8_t* src = sc + (size_t)r * kb + 4u * g;
+#pragma unroll
+            for (uint32_t j = 0; j < 4; ++j)
+                if (4u * g + j < kb) v |= (uint32_t)src[j] << (8u * j);
+        }
+        out[w] = v;
+    }
+}
+
+static PFN_cuTensorMapEncodeTiled_v12000 encoder()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (fn == nullptr) {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+    return fn;
+}
+
+static bool code_map(CUtensorMap* map, const uint8_t* q, int64_t rows, int64_t K)
+{
+    auto enc = encoder();
+    if (enc == nullptr) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)(K / 2), (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)(K / 2)};
+    const cuuint32_t box[2] = {128u, 128u};
+    const cuuint32_t es[2] = {1u, 1u};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(q), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace gemm
+
+size_t mma_scale_bytes(int64_t rows, int64_t kb)
+{
+    return (size_t)((rows + 127) / 128) * 128u * (size_t)((kb + 3) / 4) * 4u;
+}
+
+cudaError_t launch_mma_scale_layout(const uint8_t* sc, int64_t rows, int64_t kb, uint8_t* out, cudaStream_t s)
+{
+    const uint32_t kt = (uint32_t)((kb + 3) / 4);
+    const uint32_t words = (uint32_t)(mma_scale_bytes(rows, kb) / 4u);
+    int64_t need = ((int64_t)words + 255) / 256;
+    const int64_t cap = (int64_t)num_sms() * 8;
+    const int grid = (int)(need < cap ? (need > 0 ? need : 1) : cap);
+    gemm::mma_scale_layout_kernel<<<grid, 256, 0, s>>>(sc, (uint32_t)rows, (uint32_t)kb, kt, words,
+                                                       reinterpret_cast<uint32_t*>(out));
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gemm_nvfp4(const uint8_t* qa, const uint8_t* sfa, const float* d_s2a, const uint8_t* qb,
+                              const uint8_t* sfb, const float* d_s2b, int64_t M, int64_t N, int64_t K, int out_dt,
+                              void* out, int64_t ldd, uint32_t* d_flags, cudaStream_t s)
+{
+    using namespace gemm;
+    Params p;
+    if (!code_map(&p.map_a, qa, M, K) || !code_map(&p.map_b, qb, N, K)) return cudaErrorInvalidValue;
+    p.sfa = sfa;
+    p.sfb = sfb;
+    p.d_s2a = d_s2a;
+    p.d_s2b = d_s2b;
+    p.out = out;
+    p.ldd = ldd;
+    p.n_tiles = (uint32_t)(N / kBN);
+    p.k_stages = (uint32_t)(K / kBK);
+    p.kt4 = (uint32_t)(K / 64);
+    p.d_flags = d_flags;
+    const size_t smem = sizeof(Smem) + 1024;
+    static bool attr_set[2][64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const int o = out_dt == 2 ? 1 : 0;
+    if (dev < 0 || dev >= 64 || !attr_set[o][dev]) {
+        e = o ? cudaFuncSetAttribute(gemm_nvfp4_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)
+              : cudaFuncSetAttribute(gemm_nvfp4_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        if (dev >= 0 && dev < 64) attr_set[o][dev] = true;
+    }
+    const unsigned grid = (unsigned)((M / kBM) * (N / kBN));
+    if (o) gemm_nvfp4_kernel<2><<<grid, kThreads, smem, s>>>(p);
+    else gemm_nvfp4_kernel<0><<<grid, kThreads, smem, s>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace nv4

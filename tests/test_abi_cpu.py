@@ -28,7 +28,8 @@ def declared_symbols():
 def test_header_declares_the_hot_path():
     names = declared_symbols()
     for n in ("nv4_tensor_amax", "nv4_act_quant", "nv4_dequant", "nv4_hessian_accum", "nv4_scale_sweep",
-              "nv4_mxfp4_to_nvfp4", "nv4_weight_quant_rtn", "nv4_fake_qdq"):
+              "nv4_mxfp4_to_nvfp4", "nv4_weight_quant_rtn", "nv4_fake_qdq", "nv4_gemm_nvfp4",
+              "nv4_scales_to_mma_layout", "nv4_mma_scale_bytes"):
         assert n in names
 
 
@@ -75,6 +76,20 @@ def test_validation_rejects_before_any_launch(nv4lib):
     assert L.nv4_fake_qdq(fake, 4, 32, 32, fake, 2, fake, 34, fake, None, None) == 3              # fp32 ld_out
     assert L.nv4_fake_qdq(fake, 4, 32, 32, fake, 0, fake + 8, 32, fake, None, None) == 3          # misaligned out
     assert L.nv4_fake_qdq(fake, 4, 32, 32, None, 0, fake, 32, fake, None, None) == 1
+    # W4A4 GEMM: shape multiples (M, N of 128; K of 256), dtype, alignment, nulls
+    g = lambda M, N, K, dt=0, ldd=None, out=fake, qa=fake: L.nv4_gemm_nvfp4(
+        qa, fake, fake, fake, fake, fake, M, N, K, dt, out, N if ldd is None else ldd, None, None)
+    assert g(128, 128, 256, dt=1) == 4                     # fp16 out unsupported
+    assert g(100, 128, 256) == 2 and g(128, 120, 256) == 2 and g(128, 128, 200) == 2
+    assert g(128, 128, 256, ldd=64) == 2                   # ldd < N
+    assert g(128, 128, 256, ldd=132) == 3                  # bf16 row pitch not 16-byte
+    assert g(128, 128, 256, out=fake + 4) == 3
+    assert g(128, 128, 256, qa=None) == 1
+    assert g(0, 128, 256) == 0                             # empty
+    assert L.nv4_mma_scale_bytes(200, 144) == 256 * 12 and L.nv4_mma_scale_bytes(1, 16) == 512
+    assert L.nv4_mma_scale_bytes(5, 20) == 0
+    assert L.nv4_scales_to_mma_layout(fake, 4, 20, fake, None) == 2
+    assert L.nv4_scales_to_mma_layout(fake, 4, 32, fake + 8, None) == 3
     assert L.nv4_hessian_accum(fake, 10, 40, 40, fake, None, None) == 2
     assert L.nv4_hessian_accum(fake, 10, 32, 36, fake, None, None) == 3
     assert L.nv4_scale_sweep(fake, 2, 4, 32, 34, fake, fake, fake, None, None, None, None, None) == 3  # fp32 ld*4

@@ -6,7 +6,8 @@
 // i.e. the product of the two dequantized matrices, accumulated in FP32 and written
 // as BF16 or FP32.
 //
-// Kernel structure (one CTA = one 128 x 128 output tile, 128 threads):
+// Kernel structure (one CTA = one 128 x kBN output tile, kBN = 256 when N allows, else 128;
+// 128 threads):
 //   * warp 0, one lane: producer.  Per stage of 256 K-elements it loads the A and B code
 //     tiles (128 rows x 128 bytes each) with 2-D TMA into 128-byte-swizzled shared
 //     memory, and the stage's scale-factor atoms (4 x 512 bytes per operand, already in
@@ -32,21 +33,35 @@ namespace nv4 {
 
 namespace gemm {
 
-constexpr int kBM = 128, kBN = 128;
+constexpr int kBM = 128;
 constexpr int kBK = 256;                          // FP4 elements per stage (128 bytes per row)
 constexpr int kStages = 4;
 constexpr int kThreads = 128;
-constexpr uint32_t kTileBytes = 128 * 128;        // one operand's codes per stage
-constexpr uint32_t kSfBytes = 4 * 512;            // one operand's scale atoms per stage
-constexpr uint32_t kStageTx = 2 * kTileBytes + 2 * kSfBytes;
-constexpr uint32_t kTmemCols = 256;
-constexpr uint32_t kColSfA = 128, kColSfB = 160;  // two 16-column buffers each
 
+// Tile width kBN = 128 or 256 (one MMA of 128 x kBN x 64 per K-step).
+template <int kBN>
+struct Cfg {
+    static constexpr uint32_t kATile = 128 * 128;                    // A codes per stage
+    static constexpr uint32_t kBTile = kBN * 128;                    // B codes per stage
+    static constexpr uint32_t kSfA = 4 * 512;                        // 4 K-steps x one 128-row atom
+    static constexpr uint32_t kSfB = (kBN / 128) * 4 * 512;
+    static constexpr uint32_t kStageTx = kATile + kBTile + kSfA + kSfB;
+    static constexpr uint32_t kTmemCols = kBN == 128 ? 256 : 512;   // power of two >= accumulator + scales
+    static constexpr uint32_t kColSfA = kBN;                         // two 16-column buffers
+    static constexpr uint32_t kSfBCols = 16 * (kBN / 128);           // per buffer
+    static constexpr uint32_t kColSfB = kBN + 32;                    // two buffers
+    // Instruction descriptor of kind::mxf4nvf4: A and B E2M1 (format 1), K-major, scale
+    // factors UE4M3 (bit 23 = 0), N >> 3 in bits 17-22, M >> 4 in bits 24-28, dense K = 64.
+    static constexpr uint32_t kIdesc =
+        (1u << 7) | (1u << 10) | ((uint32_t)(kBN >> 3) << 17) | ((uint32_t)(kBM >> 4) << 24);
+};
+
+template <int kBN>
 struct Smem {
-    uint8_t a[kStages][kTileBytes];               // 1024-byte aligned (128-byte swizzle atoms)
-    uint8_t b[kStages][kTileBytes];
-    uint8_t sfa[kStages][kSfBytes];
-    uint8_t sfb[kStages][kSfBytes];
+    uint8_t a[kStages][Cfg<kBN>::kATile];         // 1024-byte aligned (128-byte swizzle atoms)
+    uint8_t b[kStages][Cfg<kBN>::kBTile];
+    uint8_t sfa[kStages][Cfg<kBN>::kSfA];
+    uint8_t sfb[kStages][Cfg<kBN>::kSfB];
     uint64_t full[kStages], empty[kStages], acc_full;
     uint32_t tmem_base;
     uint32_t abort;                               // set by a wait that gave up
@@ -126,10 +141,6 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint3
            ((uint64_t)(sbo & 0x3FFFu) << 32) | (1ull << 46) | ((uint64_t)layout << 61);
 }
 
-// Instruction descriptor of kind::mxf4nvf4: A and B E2M1 (format 1), K-major, scale
-// factors UE4M3 (bit 23 = 0), N >> 3 in bits 17-22, M >> 4 in bits 24-28, dense K = 64.
-constexpr uint32_t kIdesc = (1u << 7) | (1u << 10) | ((uint32_t)(kBN >> 3) << 17) | ((uint32_t)(kBM >> 4) << 24);
-
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 
@@ -153,14 +164,14 @@ __device__ __forceinline__ void tmem_cp_sf(uint32_t taddr, uint64_t desc)
     asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(desc) : "memory");
 }
 
-__device__ __forceinline__ void mma_fp4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t sfa, uint32_t sfb,
-                                        uint32_t accumulate)
+__device__ __forceinline__ void mma_fp4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                        uint32_t sfa, uint32_t sfb, uint32_t accumulate)
 {
     asm volatile("{\n\t.reg .pred p;\n\t"
                  "setp.ne.b32 p, %4, 0;\n\t"
                  "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t"
                  "}"
-                 ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+                 ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
                  : "memory");
 }
 
@@ -193,12 +204,13 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float v[32])
 
 namespace gemm {
 
-template <int kOut>   // 0 bf16, 2 fp32
+template <int kBN, int kOut>   // tile width 128 | 256; output 0 bf16, 2 fp32
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_nvfp4_kernel(const __grid_constant__ Params p)
 {
+    using C = Cfg<kBN>;
     extern __shared__ uint8_t smem_raw[];
-    Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    Smem<kBN>& sm = *reinterpret_cast<Smem<kBN>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t n_tile = blockIdx.x % p.n_tiles, m_tile = blockIdx.x / p.n_tiles;
     const uint32_t KS = p.k_stages;
@@ -215,7 +227,7 @@ gemm_nvfp4_kernel(const __grid_constant__ Params p)
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&p.map_a)) : "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&p.map_b)) : "memory");
     }
-    if (warp == 1) tmem_alloc(&sm.tmem_base, kTmemCols);
+    if (warp == 1) tmem_alloc(&sm.tmem_base, C::kTmemCols);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -233,11 +245,15 @@ gemm_nvfp4_kernel(const __grid_constant__ Params p)
                     break;
                 }
                 if (*reinterpret_cast<volatile uint32_t*>(&sm.abort) != 0u) break;
-                mbar_arrive_expect_tx(&sm.full[s], kStageTx);
+                mbar_arrive_expect_tx(&sm.full[s], C::kStageTx);
                 tma_load_2d(sm.a[s], &p.map_a, &sm.full[s], (int)(ks * 128u), (int)(m_tile * kBM));
                 tma_load_2d(sm.b[s], &p.map_b, &sm.full[s], (int)(ks * 128u), (int)(n_tile * kBN));
-                bulk_load(sm.sfa[s], p.sfa + ((size_t)m_tile * p.kt4 + 4u * ks) * 512u, kSfBytes, &sm.full[s]);
-                bulk_load(sm.sfb[s], p.sfb + ((size_t)n_tile * p.kt4 + 4u * ks) * 512u, kSfBytes, &sm.full[s]);
+                bulk_load(sm.sfa[s], p.sfa + ((size_t)m_tile * p.kt4 + 4u * ks) * 512u, C::kSfA, &sm.full[s]);
+#pragma unroll
+                for (uint32_t h = 0; h < (uint32_t)(kBN / 128); ++h)      // one run of 4 atoms per 128 rows
+                    bulk_load(sm.sfb[s] + 2048u * h,
+                              p.sfb + ((size_t)(n_tile * (kBN / 128) + h) * p.kt4 + 4u * ks) * 512u, 2048u,
+                              &sm.full[s]);
             }
             sm.issued = ks;
         }
@@ -254,17 +270,21 @@ gemm_nvfp4_kernel(const __grid_constant__ Params p)
                 }
                 tc_fence_after();
                 const uint32_t buf = ks & 1u;
-                const uint32_t ta = tmem + kColSfA + 16u * buf, tb = tmem + kColSfB + 16u * buf;
+                // scale columns: A row r of K-step j at column ta + 4j + r/32; B row n at tb + nb*j + n/32
+                constexpr uint32_t nb = 4u * (kBN / 128);
+                const uint32_t ta = tmem + C::kColSfA + 16u * buf, tb = tmem + C::kColSfB + C::kSfBCols * buf;
 #pragma unroll
                 for (uint32_t j = 0; j < 4; ++j) {
                     tmem_cp_sf(ta + 4u * j, smem_desc(smem_u32(sm.sfa[s] + 512u * j), 0u, 8u, 0u));
-                    tmem_cp_sf(tb + 4u * j, smem_desc(smem_u32(sm.sfb[s] + 512u * j), 0u, 8u, 0u));
+#pragma unroll
+                    for (uint32_t h = 0; h < (uint32_t)(kBN / 128); ++h)
+                        tmem_cp_sf(tb + nb * j + 4u * h, smem_desc(smem_u32(sm.sfb[s] + 2048u * h + 512u * j), 0u, 8u, 0u));
                 }
                 const uint32_t a0 = smem_u32(sm.a[s]), b0 = smem_u32(sm.b[s]);
 #pragma unroll
                 for (uint32_t j = 0; j < 4; ++j)
                     mma_fp4(tmem, smem_desc(a0 + 32u * j, 1u, 64u, 2u), smem_desc(b0 + 32u * j, 1u, 64u, 2u),
-                            ta + 4u * j, tb + 4u * j, (ks | j) != 0u ? 1u : 0u);
+                            C::kIdesc, ta + 4u * j, tb + nb * j, (ks | j) != 0u ? 1u : 0u);
                 tc_commit(&sm.empty[s]);                           // frees the stage when these MMAs finish
             }
             sm.consumed = ks;
@@ -315,7 +335,7 @@ gemm_nvfp4_kernel(const __grid_constant__ Params p)
     }
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, kTmemCols);
+        tmem_dealloc(tmem, C::kTmemCols);
     }
     flags = __reduce_or_sync(0xFFFFFFFFu, flags);
     if (lane == 0) flag_or(p.d_flags, flags);
@@ -356,13 +376,13 @@ static PFN_cuTensorMapEncodeTiled_v12000 encoder()
     return fn;
 }
 
-static bool code_map(CUtensorMap* map, const uint8_t* q, int64_t rows, int64_t K)
+static bool code_map(CUtensorMap* map, const uint8_t* q, int64_t rows, int64_t K, uint32_t box_rows)
 {
     auto enc = encoder();
     if (enc == nullptr) return false;
     const cuuint64_t dims[2] = {(cuuint64_t)(K / 2), (cuuint64_t)rows};
     const cuuint64_t strides[1] = {(cuuint64_t)(K / 2)};
-    const cuuint32_t box[2] = {128u, 128u};
+    const cuuint32_t box[2] = {128u, box_rows};
     const cuuint32_t es[2] = {1u, 1u};
     return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(q), dims, strides, box, es,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -394,32 +414,35 @@ cudaError_t launch_gemm_nvfp4(const uint8_t* qa, const uint8_t* sfa, const float
 {
     using namespace gemm;
     Params p;
-    if (!code_map(&p.map_a, qa, M, K) || !code_map(&p.map_b, qb, N, K)) return cudaErrorInvalidValue;
+    const bool wide = N % 256 == 0;
+    const int bn = wide ? 256 : 128;
+    if (!code_map(&p.map_a, qa, M, K, 128u) || !code_map(&p.map_b, qb, N, K, (uint32_t)bn)) return cudaErrorInvalidValue;
     p.sfa = sfa;
     p.sfb = sfb;
     p.d_s2a = d_s2a;
     p.d_s2b = d_s2b;
     p.out = out;
     p.ldd = ldd;
-    p.n_tiles = (uint32_t)(N / kBN);
+    p.n_tiles = (uint32_t)(N / bn);
     p.k_stages = (uint32_t)(K / kBK);
     p.kt4 = (uint32_t)(K / 64);
     p.d_flags = d_flags;
-    const size_t smem = sizeof(Smem) + 1024;
-    static bool attr_set[2][64] = {};
+    const size_t smem = (wide ? sizeof(Smem<256>) : sizeof(Smem<128>)) + 1024;
+    static bool attr_set[4][64] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     const int o = out_dt == 2 ? 1 : 0;
-    if (dev < 0 || dev >= 64 || !attr_set[o][dev]) {
-        e = o ? cudaFuncSetAttribute(gemm_nvfp4_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)
-              : cudaFuncSetAttribute(gemm_nvfp4_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const int v = 2 * (wide ? 1 : 0) + o;
+    auto kern = wide ? (o ? gemm_nvfp4_kernel<256, 2> : gemm_nvfp4_kernel<256, 0>)
+                     : (o ? gemm_nvfp4_kernel<128, 2> : gemm_nvfp4_kernel<128, 0>);
+    if (dev < 0 || dev >= 64 || !attr_set[v][dev]) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        if (dev >= 0 && dev < 64) attr_set[o][dev] = true;
+        if (dev >= 0 && dev < 64) attr_set[v][dev] = true;
     }
-    const unsigned grid = (unsigned)((M / kBM) * (N / kBN));
-    if (o) gemm_nvfp4_kernel<2><<<grid, kThreads, smem, s>>>(p);
-    else gemm_nvfp4_kernel<0><<<grid, kThreads, smem, s>>>(p);
+    const unsigned grid = (unsigned)((M / kBM) * (N / bn));
+    kern<<<grid, kThreads, smem, s>>>(p);
     return cudaGetLastError();
 }
 

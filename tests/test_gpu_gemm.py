@@ -81,6 +81,14 @@ def test_gemm_multi_tile_random(orc):
     _check(orc, qa, sa, float(np.float32(3.1e-3)), qb, sb, float(np.float32(0.021)))
 
 
+def test_gemm_narrow_tiles(orc):
+    """N a multiple of 128 but not of 256: the 128-wide tile variant."""
+    rng = np.random.default_rng(15)
+    qa, sa = _random_operand(rng, 256, 768, lo=0x08, hi=0x7E)
+    qb, sb = _random_operand(rng, 384, 768, lo=0x08, hi=0x7E)
+    _check(orc, qa, sa, 1.0, qb, sb, float(np.float32(1e-3)))
+
+
 def test_gemm_quantized_layer(orc):
     """Activations quantized by the oracle's dynamic quantizer, weights by its RTN
     quantizer: the W4A4 product of a 256-token batch through a 2048 -> 512 projection."""

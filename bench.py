@@ -75,6 +75,17 @@ def peaks():
         return 6650.0, "fallback"
 
 
+def fp4_peak_tflops():
+    """Dense NVFP4 tensor peak: the measured BF16 GEMM peak times the nominal FP4/BF16
+    ratio (9 / 2.25 PFLOP/s), else the recipe's fallback 1.59 PFLOP/s BF16 times 4."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return 4.0 * float(json.load(f)["bf16_tflops"])
+    except Exception:
+        return 4.0 * 1590.0
+
+
 # ---------------------------------------------------------------------- clocks
 class ClockSampler:
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -314,6 +325,24 @@ def kernel_rooflines(W, hbm_peak):
                               "costs_per_block": costs / blocks,
                               "exhaustive_equiv_tflops": SWEEP_FLOP_PER_BLOCK * blocks / t / 1e12,
                               "launch": "q_proj + gate + up + down, one batched launch"}
+    if "calib" in W or "act" in W:
+        # W4A4 GEMM (a widening of the path; not part of the step): a 16384-token batch
+        # through the gate projection 2048 -> 16384 and a square 8192^3 product, random
+        # NVFP4 operands (codes and scales resident in HBM, scales in the MMA layout)
+        dev = W["flags"].device
+        g = torch.Generator(device=dev).manual_seed(1)
+        best = None
+        for (M, N, K) in ((16384, 16384, 2048), (8192, 8192, 8192)):
+            qa = torch.randint(0, 256, (M, K // 2), dtype=torch.uint8, device=dev, generator=g)
+            qb = torch.randint(0, 256, (N, K // 2), dtype=torch.uint8, device=dev, generator=g)
+            fa = nv4.mma_scales(torch.randint(0x30, 0x40, (M, K // 16), dtype=torch.uint8, device=dev, generator=g))
+            fb = nv4.mma_scales(torch.randint(0x30, 0x40, (N, K // 16), dtype=torch.uint8, device=dev, generator=g))
+            one = torch.ones(1, dtype=torch.float32, device=dev)
+            o = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+            t = time_launch(lambda: nv4.nv4_gemm_nvfp4(qa, fa, one, qb, fb, one, o, W["flags"]), reps=10)
+            out[f"gemm_nvfp4_{M}x{N}x{K}"] = {"bound": "tensor", "flops": 2.0 * M * N * K, "s": t, "in_step": False,
+                                              "launch": f"A [{M}, {K}] x B [{N}, {K}] NVFP4 -> BF16"}
+            del qa, qb, fa, fb, o
     if "cast" in W:
         nmx = sum(j["e8m0"].numel() for j in W["cast"])
         t = time_launch(lambda: nv4.nv4_mxfp4_to_nvfp4_batched(W["cast"], W["counts"], W["flags"]), flush=flush)
@@ -324,6 +353,10 @@ def kernel_rooflines(W, hbm_peak):
             v["achieved"] = v["bytes"] / v["s"] / 1e9
             v["peak"] = hbm_peak
             v["unit"] = "GB/s"
+        elif v["bound"] == "tensor":
+            v["achieved"] = v["flops"] / v["s"] / 1e12
+            v["peak"] = fp4_peak_tflops()
+            v["unit"] = "TFLOP/s"
         else:
             v["achieved"] = v["flops"] / v["s"] / 1e12
             v["peak"] = FP32_PEAK_TFLOPS

@@ -21,7 +21,7 @@ from concurrent.futures import ThreadPoolExecutor
 import numpy as np
 
 _DIR = os.path.dirname(os.path.abspath(__file__))
-_SOURCES = ["formats.c", "act.c", "hessian.c", "sweep.c", "cast.c"]
+_SOURCES = ["formats.c", "act.c", "hessian.c", "sweep.c", "cast.c", "variants.c"]
 _LIB_PATH = os.path.join(_DIR, "liboracle.so")
 _lock = threading.Lock()
 _lib = None
@@ -67,6 +67,9 @@ def _L():
                 "orc_act_quant": (C.c_float, [vp, i64, i64, i64, C.c_float, i64, i64, vp, vp, u32p]),
                 "orc_block_quant": (C.c_float, [vp, C.c_int, i64, i64, i64, C.c_float, i64, i64, vp, vp, u32p]),
                 "orc_dequant": (None, [vp, vp, C.c_float, i64, i64, C.c_int, i64, i64, vp]),
+                "orc_mxfp4_quant": (None, [vp, C.c_int, i64, i64, i64, i64, vp, vp, u32p]),
+                "orc_mxfp4_dequant": (None, [vp, vp, i64, i64, i64, C.c_int, vp]),
+                "orc_fp8_quant": (C.c_float, [vp, C.c_int, i64, i64, C.c_float, i64, i64, vp, u32p]),
                 "orc_hessian_accum": (None, [vp, i64, i64, i64, i64, i64, vp]),
                 "orc_scale_sweep": (None, [vp, C.c_int, i64, i64, i64, vp, C.c_float, i64, i64,
                                            vp, vp, vp, vp, u32p]),
@@ -407,3 +410,68 @@ def scales_to_mma_layout(sc: np.ndarray) -> np.ndarray:
     off = ((r // 128) * kt + j // 4) * 512 + (r % 32) * 16 + ((r % 128) // 32) * 4 + j % 4
     out[off] = sc
     return out
+
+
+# ---------------------------------------------------------------- format variants
+def mxfp4_quant(x: np.ndarray, cols: int | None = None, threads: int | None = None):
+    """MXFP4 round-to-nearest quantization ([FP4] sections 1.2 and 3.2): 32-element blocks,
+    E8M0 shared exponent floor(log2 amax) - 2, E2M1 elements.  x: float32 or uint16
+    (bf16 bits) [rows, ld].  Returns (q [rows, cols/2], e8m0 [rows, cols/32], flags)."""
+    assert x.ndim == 2 and x.flags.c_contiguous and x.dtype in (np.float32, np.uint16)
+    dt = F32 if x.dtype == np.float32 else BF16
+    rows, ld = x.shape
+    cols = ld if cols is None else cols
+    assert cols % 32 == 0
+    q = np.zeros((rows, cols // 2), np.uint8)
+    e = np.zeros((rows, cols // 32), np.uint8)
+    flags = [0]
+    lk = threading.Lock()
+
+    def run(r0, r1):
+        f = C.c_uint32(0)
+        _L().orc_mxfp4_quant(_p(x), dt, cols, ld, r0, r1, _p(q), _p(e), C.byref(f))
+        with lk:
+            flags[0] |= f.value
+
+    if rows:
+        _fanout(run, rows, threads)
+    return q, e, flags[0]
+
+
+def mxfp4_dequant(q: np.ndarray, e8m0: np.ndarray, out_dtype: str = "bf16", threads: int | None = None):
+    """e2m1(code) * 2^(e8m0 - 127), rounded once to the output type."""
+    rows, cols = q.shape[0], 2 * q.shape[1]
+    code = {"bf16": 0, "fp16": 1, "fp32": 2}[out_dtype]
+    out = np.zeros((rows, cols), np.float32 if code == 2 else np.uint16)
+    q, e8m0 = np.ascontiguousarray(q), np.ascontiguousarray(e8m0)
+    _fanout(lambda r0, r1: _L().orc_mxfp4_dequant(_p(q), _p(e8m0), cols, r0, r1, code, _p(out)), rows, threads)
+    return out
+
+
+def fp8_quant(x: np.ndarray, amax: float, cols: int | None = None, threads: int | None = None):
+    """FP8 E4M3 with one static per-tensor scale ([CAL] layer table: W8A8 layers):
+    s = RN32(amax / 448), code = sign | nearest E4M3 to |x| / s.  Returns (q, s, flags)."""
+    assert x.ndim == 2 and x.flags.c_contiguous and x.dtype in (np.float32, np.uint16)
+    dt = F32 if x.dtype == np.float32 else BF16
+    rows, ld = x.shape
+    cols = ld if cols is None else cols
+    q = np.zeros((rows, cols), np.uint8)
+    flags = [0]
+    s = [float(np.float32(amax / 448.0))]
+    lk = threading.Lock()
+
+    def run(r0, r1):
+        f = C.c_uint32(0)
+        s[0] = _L().orc_fp8_quant(_p(x), dt, cols, ld, amax, r0, r1, _p(q), C.byref(f))
+        with lk:
+            flags[0] |= f.value
+
+    if rows:
+        _fanout(run, rows, threads)
+    return q, float(np.float32(s[0])), flags[0]
+
+
+def fp8_dequant(q: np.ndarray, s: float) -> np.ndarray:
+    """Exact values e4m3(code) * s (FP64); the caller rounds to its output type."""
+    tab = np.array([e4m3_value(c) for c in range(256)], np.float64)
+    return tab[np.ascontiguousarray(q)] * float(s)

@@ -76,6 +76,17 @@ float orc_act_quant(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, f
 float orc_block_quant(const void* x, int dtype, int64_t rows, int64_t cols, int64_t ld, float amax,
                       int64_t row0, int64_t row1, uint8_t* q, uint8_t* scales, uint32_t* flags);
 
+/* ---- format variants (variants.c) ----------------------------------------
+ * MXFP4: 32-element blocks, E8M0 shared power-of-two scale (q [rows, cols/2], e8m0
+ * [rows, cols/32]).  FP8: E4M3 codes with one static per-tensor scale s = amax/448
+ * (returned).  x: dtype ORC_BF16 or ORC_F32, leading dimension ld; rows [row0, row1). */
+void orc_mxfp4_quant(const void* x, int dtype, int64_t cols, int64_t ld, int64_t row0, int64_t row1,
+                     uint8_t* q, uint8_t* e8m0, uint32_t* flags);
+void orc_mxfp4_dequant(const uint8_t* q, const uint8_t* e8m0, int64_t cols, int64_t row0, int64_t row1,
+                       int out_dtype, void* out);
+float orc_fp8_quant(const void* x, int dtype, int64_t cols, int64_t ld, float amax, int64_t row0, int64_t row1,
+                    uint8_t* q, uint32_t* flags);
+
 /* ---- two-step dequantization (act.c) ------------------------------------
  * out_dtype: 0 = bf16 bits (uint16), 1 = fp16 bits (uint16), 2 = fp32. */
 void orc_dequant(const uint8_t* q, const uint8_t* scales, float s2, int64_t rows, int64_t cols,

@@ -304,6 +304,36 @@ NV4_API nv4_status nv4_gemm_nvfp4(const uint8_t* qa, const uint8_t* sfa_mma, con
                           uint32_t* d_flags, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * Format variants ([FP4] sections 1.2 and 3.2; [CAL] layer table and the note under it).
+ *
+ * nv4_mxfp4_quant -- MXFP4 round-to-nearest quantization: 32-element blocks along a row,
+ * one E8M0 scale 2^e per block with e = floor(log2 amax_block) - 2 clamped to [-127, 127]
+ * (code e + 127; an all-zero block gets code 0), elements E2M1 nearest to x / 2^e (ties to
+ * even, saturating at 6, sign kept).  A block holding NaN or Inf gets code 0xFF and sets
+ * NV4_FLAG_NONFINITE.  x: [rows, cols] of dt (NV4_BF16 or NV4_FP32), leading dimension ld
+ * (16-byte multiple), cols % 32 == 0.  q [rows, cols/2] (two codes per byte, low nibble =
+ * even element) and e8m0 [rows, cols/32], contiguous.  The output feeds
+ * nv4_mxfp4_to_nvfp4 directly.
+ * nv4_mxfp4_dequant -- out = RN_out(RN32(e2m1(code) * 2^(e8m0 - 127))) as NV4_BF16/FP16/FP32
+ * (NaN for code 0xFF).  out [rows, cols] contiguous, 16-byte aligned.
+ *
+ * nv4_fp8_quant -- FP8 E4M3 with one static per-tensor scale (W8A8 layers with calibrated
+ * scales): s = RN32(amax / 448) written to *d_scale, code = sign | E4M3 nearest to |x| / s
+ * (ties to even, saturating at 448); s = 0 gives signed zeros.  x as above with
+ * cols % 16 == 0; q [rows, cols] contiguous.
+ * nv4_fp8_dequant -- out = RN_out(RN32(e4m3(code) * s)), as nv4_dequant's DQ2.
+ * Limits: fewer than 2^31 16-element groups per call (NV4_ERR_LIMIT beyond).
+ */
+NV4_API nv4_status nv4_mxfp4_quant(const void* x, nv4_dtype dt, int64_t rows, int64_t cols, int64_t ld,
+                           uint8_t* q, uint8_t* e8m0, uint32_t* d_flags, void* stream);
+NV4_API nv4_status nv4_mxfp4_dequant(const uint8_t* q, const uint8_t* e8m0, int64_t rows, int64_t cols,
+                             nv4_dtype out_dt, void* out, void* stream);
+NV4_API nv4_status nv4_fp8_quant(const void* x, nv4_dtype dt, int64_t rows, int64_t cols, int64_t ld,
+                         const float* d_amax, uint8_t* q, float* d_scale, uint32_t* d_flags, void* stream);
+NV4_API nv4_status nv4_fp8_dequant(const uint8_t* q, const float* d_scale, int64_t rows, int64_t cols,
+                           nv4_dtype out_dt, void* out, void* stream);
+
+/* ---------------------------------------------------------------------------
  * nv4_selftest -- checks, on the current device, the hardware FP4/FP8 conversion
  * instructions the kernels rely on (lane order, rounding, sign of zero, saturation).
  * Writes 64 uint32 results to d_out (device); d_out[0] is a bit mask of failed

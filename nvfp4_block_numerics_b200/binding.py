@@ -21,7 +21,8 @@ from .build import LIB_PATH
 __all__ = [
     "NV4Error", "lib", "nv4_tensor_amax", "nv4_act_quant", "nv4_weight_quant_rtn", "nv4_fake_qdq",
     "nv4_dequant", "nv4_hessian_accum", "weight_quant_rtn", "fake_qdq", "nv4_mma_scale_bytes",
-    "nv4_scales_to_mma_layout", "nv4_gemm_nvfp4", "mma_scales", "gemm_nvfp4",
+    "nv4_scales_to_mma_layout", "nv4_gemm_nvfp4", "mma_scales", "gemm_nvfp4", "nv4_mxfp4_quant",
+    "nv4_mxfp4_dequant", "nv4_fp8_quant", "nv4_fp8_dequant", "mxfp4_quant", "fp8_quant",
     "nv4_hessian_accum_batched", "nv4_scale_sweep", "nv4_scale_sweep_batched", "nv4_mxfp4_to_nvfp4",
     "nv4_mxfp4_to_nvfp4_batched", "nv4_selftest", "nv4_version", "FLAG_NONFINITE", "FLAG_E8M0_NAN",
     "FLAG_OVERFLOW", "FLAG_TIMEOUT", "tensor_amax", "act_quant", "dequant", "hessian_accum",
@@ -65,6 +66,10 @@ _SIGS = {
     "nv4_fake_qdq": (C.c_int, [_vp, _i64, _i64, _i64, _vp, C.c_int, _vp, _i64, _vp, _vp, _vp]),
     "nv4_dequant": (C.c_int, [_vp, _vp, _vp, _i64, _i64, C.c_int, _vp, _vp]),
     "nv4_mma_scale_bytes": (C.c_size_t, [_i64, _i64]),
+    "nv4_mxfp4_quant": (C.c_int, [_vp, C.c_int, _i64, _i64, _i64, _vp, _vp, _vp, _vp]),
+    "nv4_mxfp4_dequant": (C.c_int, [_vp, _vp, _i64, _i64, C.c_int, _vp, _vp]),
+    "nv4_fp8_quant": (C.c_int, [_vp, C.c_int, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp]),
+    "nv4_fp8_dequant": (C.c_int, [_vp, _vp, _i64, _i64, C.c_int, _vp, _vp]),
     "nv4_scales_to_mma_layout": (C.c_int, [_vp, _i64, _i64, _vp, _vp]),
     "nv4_gemm_nvfp4": (C.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, C.c_int, _vp, _i64, _vp, _vp]),
     "nv4_hessian_accum": (C.c_int, [_vp, _i64, _i64, _i64, _vp, _vp, _vp]),
@@ -310,6 +315,65 @@ def fake_qdq(x: torch.Tensor, d_amax: torch.Tensor, dtype=torch.bfloat16, d_flag
     s2 = torch.empty((1,), dtype=torch.float32, device=x.device)
     nv4_fake_qdq(x, d_amax, out, s2, d_flags, stream)
     return out, s2
+
+
+def _u8(t, shape, name):
+    if t.dtype != torch.uint8 or tuple(t.shape) != tuple(shape) or not t.is_contiguous():
+        raise NV4Error(f"{name} must be a contiguous uint8 tensor {tuple(shape)}")
+
+
+def nv4_mxfp4_quant(x: torch.Tensor, q: torch.Tensor, e8m0: torch.Tensor, d_flags=None, stream=None):
+    if x.dtype not in (torch.bfloat16, torch.float32):
+        raise NV4Error("x must be bf16 or float32")
+    rows, cols, ld = _rowmajor(x, "x")
+    _u8(q, (rows, cols // 2), "q")
+    _u8(e8m0, (rows, cols // 32), "e8m0")
+    _check(lib().nv4_mxfp4_quant(_ptr(x), _DT[x.dtype], rows, cols, ld, _ptr(q), _ptr(e8m0), _ptr(d_flags),
+                                 _stream(stream)), "nv4_mxfp4_quant")
+
+
+def nv4_mxfp4_dequant(q: torch.Tensor, e8m0: torch.Tensor, out: torch.Tensor, stream=None):
+    rows, cols = out.shape
+    _u8(q, (rows, cols // 2), "q")
+    _u8(e8m0, (rows, cols // 32), "e8m0")
+    if out.dtype not in _DT or not out.is_contiguous():
+        raise NV4Error("out must be a contiguous bf16, float16 or float32 tensor")
+    _check(lib().nv4_mxfp4_dequant(_ptr(q), _ptr(e8m0), rows, cols, _DT[out.dtype], _ptr(out), _stream(stream)),
+           "nv4_mxfp4_dequant")
+
+
+def nv4_fp8_quant(x: torch.Tensor, d_amax: torch.Tensor, q: torch.Tensor, d_scale: torch.Tensor, d_flags=None,
+                  stream=None):
+    if x.dtype not in (torch.bfloat16, torch.float32):
+        raise NV4Error("x must be bf16 or float32")
+    rows, cols, ld = _rowmajor(x, "x")
+    _u8(q, (rows, cols), "q")
+    _check(lib().nv4_fp8_quant(_ptr(x), _DT[x.dtype], rows, cols, ld, _scalar_f32(d_amax, "d_amax"), _ptr(q),
+                               _scalar_f32(d_scale, "d_scale"), _ptr(d_flags), _stream(stream)), "nv4_fp8_quant")
+
+
+def nv4_fp8_dequant(q: torch.Tensor, d_scale: torch.Tensor, out: torch.Tensor, stream=None):
+    rows, cols = out.shape
+    _u8(q, (rows, cols), "q")
+    if out.dtype not in _DT or not out.is_contiguous():
+        raise NV4Error("out must be a contiguous bf16, float16 or float32 tensor")
+    _check(lib().nv4_fp8_dequant(_ptr(q), _scalar_f32(d_scale, "d_scale"), rows, cols, _DT[out.dtype], _ptr(out),
+                                 _stream(stream)), "nv4_fp8_dequant")
+
+
+def mxfp4_quant(x: torch.Tensor, d_flags=None, stream=None):
+    rows, cols = x.shape
+    q = torch.empty((rows, cols // 2), dtype=torch.uint8, device=x.device)
+    e8 = torch.empty((rows, cols // 32), dtype=torch.uint8, device=x.device)
+    nv4_mxfp4_quant(x, q, e8, d_flags, stream)
+    return q, e8
+
+
+def fp8_quant(x: torch.Tensor, d_amax: torch.Tensor, d_flags=None, stream=None):
+    q = torch.empty(tuple(x.shape), dtype=torch.uint8, device=x.device)
+    sc = torch.empty(1, dtype=torch.float32, device=x.device)
+    nv4_fp8_quant(x, d_amax, q, sc, d_flags, stream)
+    return q, sc
 
 
 def nv4_mma_scale_bytes(rows: int, cols: int) -> int:

@@ -322,3 +322,55 @@ nv4_status nv4_gemm_nvfp4(const uint8_t* qa, const uint8_t* sfa_mma, const float
     return from_cuda(launch_gemm_nvfp4(qa, sfa_mma, d_s2a, qb, sfb_mma, d_s2b, M, N, K, (int)out_dt, out, ldd,
                                        d_flags, (cudaStream_t)stream));
 }
+
+// ------------------------------------------------------------------ format variants
+nv4_status nv4_mxfp4_quant(const void* x, nv4_dtype dt, int64_t rows, int64_t cols, int64_t ld, uint8_t* q,
+                           uint8_t* e8m0, uint32_t* d_flags, void* stream)
+{
+    if (dt != NV4_BF16 && dt != NV4_FP32) return NV4_ERR_DTYPE;
+    if (rows < 0 || cols < 0 || cols % 32 != 0 || ld < cols) return NV4_ERR_SHAPE;
+    if (rows == 0 || cols == 0) return NV4_OK;
+    if (x == nullptr || q == nullptr || e8m0 == nullptr) return NV4_ERR_NULL;
+    if (!aligned16(x) || !aligned16(q) || ld % (dt == NV4_BF16 ? 8 : 4) != 0) return NV4_ERR_ALIGN;
+    if (rows * (cols / 16) >= (int64_t)1 << 31) return NV4_ERR_LIMIT;
+    return from_cuda(launch_mxfp4_quant(x, dt == NV4_BF16 ? 0 : 2, rows, cols, ld, q, e8m0, d_flags,
+                                        (cudaStream_t)stream));
+}
+
+nv4_status nv4_mxfp4_dequant(const uint8_t* q, const uint8_t* e8m0, int64_t rows, int64_t cols, nv4_dtype out_dt,
+                             void* out, void* stream)
+{
+    if (out_dt != NV4_BF16 && out_dt != NV4_FP16 && out_dt != NV4_FP32) return NV4_ERR_DTYPE;
+    if (rows < 0 || cols < 0 || cols % 32 != 0) return NV4_ERR_SHAPE;
+    if (rows == 0 || cols == 0) return NV4_OK;
+    if (q == nullptr || e8m0 == nullptr || out == nullptr) return NV4_ERR_NULL;
+    if (!aligned16(q) || !aligned16(out)) return NV4_ERR_ALIGN;
+    if (rows * (cols / 8) >= (int64_t)1 << 31) return NV4_ERR_LIMIT;
+    return from_cuda(launch_mxfp4_dequant(q, e8m0, rows, cols, (int)out_dt, out, (cudaStream_t)stream));
+}
+
+nv4_status nv4_fp8_quant(const void* x, nv4_dtype dt, int64_t rows, int64_t cols, int64_t ld, const float* d_amax,
+                         uint8_t* q, float* d_scale, uint32_t* d_flags, void* stream)
+{
+    if (dt != NV4_BF16 && dt != NV4_FP32) return NV4_ERR_DTYPE;
+    if (rows < 0 || cols < 0 || cols % 16 != 0 || ld < cols) return NV4_ERR_SHAPE;
+    if (d_amax == nullptr || d_scale == nullptr) return NV4_ERR_NULL;
+    if (rows == 0 || cols == 0) return NV4_OK;
+    if (x == nullptr || q == nullptr) return NV4_ERR_NULL;
+    if (!aligned16(x) || !aligned16(q) || ld % (dt == NV4_BF16 ? 8 : 4) != 0) return NV4_ERR_ALIGN;
+    if (rows * (cols / 16) >= (int64_t)1 << 31) return NV4_ERR_LIMIT;
+    return from_cuda(launch_fp8_quant(x, dt == NV4_BF16 ? 0 : 2, rows, cols, ld, d_amax, q, d_scale, d_flags,
+                                      (cudaStream_t)stream));
+}
+
+nv4_status nv4_fp8_dequant(const uint8_t* q, const float* d_scale, int64_t rows, int64_t cols, nv4_dtype out_dt,
+                           void* out, void* stream)
+{
+    if (out_dt != NV4_BF16 && out_dt != NV4_FP16 && out_dt != NV4_FP32) return NV4_ERR_DTYPE;
+    if (rows < 0 || cols < 0 || cols % 16 != 0) return NV4_ERR_SHAPE;
+    if (rows == 0 || cols == 0) return NV4_OK;
+    if (q == nullptr || d_scale == nullptr || out == nullptr) return NV4_ERR_NULL;
+    if (!aligned16(q) || !aligned16(out)) return NV4_ERR_ALIGN;
+    if (rows * (cols / 16) >= (int64_t)1 << 31) return NV4_ERR_LIMIT;
+    return from_cuda(launch_fp8_dequant(q, d_scale, rows, cols, (int)out_dt, out, (cudaStream_t)stream));
+}

@@ -1,0 +1,330 @@
+// variants.cu -- format variants of the block quantizer (sm_100a): MXFP4 (32-element
+// blocks, E8M0 power-of-two scale) and FP8 E4M3 with one static per-tensor scale.
+//
+// MXFP4 ([FP4] sections 1.2, 3.2): shared exponent e = floor(log2 amax) - 2, clamped to
+// [-127, 127]; elements = E2M1 nearest to x / 2^e.  Dividing by a power of two is exact
+// in FP32 here (|x| / 2^e < 8 and 2^-e is a normal number for every finite amax), so one
+// hardware round-to-nearest-even conversion gives the exact code: no bracket is needed.
+// One thread handles half a block (16 elements); the two lanes of a block exchange their
+// maxima with one shuffle.
+//
+// FP8 ([CAL] layer table, W8A8 with static per-tensor scales): s = RN32(amax / 448),
+// code = sign | E4M3 nearest to |x| / s.  The quotient is bracketed between two FP32
+// products by 1/s with a 2^-20 margin and both ends converted with the hardware's RNE
+// E4M3 conversion; when they differ, one exact FMA comparison with the midpoint decides.
+#include "nv4_common.cuh"
+#include "nv4_internal.h"
+
+namespace nv4 {
+
+constexpr int kVarThreads = 256;
+
+template <int kIn>
+__device__ __forceinline__ void load16(const void* x, int64_t off, float v[16], uint32_t& amax_bits)
+{
+    amax_bits = 0u;
+    if constexpr (kIn == 0) {
+        const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(x) + off);
+        const uint4 a = __ldcs(src), b = __ldcs(src + 1);
+        const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+        uint32_t m = 0u;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            m = __vmaxu2(m, w[j] & 0x7FFF7FFFu);
+            v[2 * j] = bf16_lo(w[j]);
+            v[2 * j + 1] = bf16_hi(w[j]);
+        }
+        amax_bits = max(m & 0xFFFFu, m >> 16) << 16;
+    } else {
+        const uint4* src = reinterpret_cast<const uint4*>(static_cast<const float*>(x) + off);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const uint4 t = __ldcs(src + k);
+            const uint32_t w[4] = {t.x, t.y, t.z, t.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                amax_bits = max(amax_bits, w[j] & 0x7FFFFFFFu);
+                v[4 * k + j] = __uint_as_float(w[j]);
+            }
+        }
+    }
+}
+
+// floor(log2(a)) for a finite positive FP32 bit pattern (normal or subnormal).
+__device__ __forceinline__ int floor_log2_bits(uint32_t b)
+{
+    const int e = (int)(b >> 23);
+    return e != 0 ? e - 127 : -149 + (31 - __clz(b));
+}
+
+// 2^k as FP32 for k in [-149, 127] (exact).
+__device__ __forceinline__ float pow2f(int k)
+{
+    return k >= -126 ? __uint_as_float((uint32_t)(k + 127) << 23) : __uint_as_float(1u << (k + 149));
+}
+
+// ------------------------------------------------------------------ MXFP4
+template <int kIn>
+__global__ void __launch_bounds__(kVarThreads)
+mxfp4_quant_kernel(const void* x, uint32_t rows, uint32_t halves_per_row, int64_t ld, FastDiv div_hpr,
+                   uint8_t* __restrict__ q, uint8_t* __restrict__ e8m0, uint32_t* __restrict__ d_flags)
+{
+    const uint32_t total = rows * halves_per_row;                 // even: two halves per block
+    const uint32_t stride = gridDim.x * kVarThreads;
+    const uint32_t lane = threadIdx.x & 31u;
+    uint32_t flags = 0u;
+    // warp-uniform trip count, so the pair shuffle always has both lanes present
+    for (uint32_t h0 = blockIdx.x * kVarThreads + (threadIdx.x & ~31u); h0 < total; h0 += stride) {
+        const uint32_t h = h0 + lane;
+        const bool live = h < total;                               // partners are both live or both not
+        float v[16];
+        uint32_t ab = 0u;
+        if (live) {
+            const uint32_t r = div_hpr.div(h), hh = h - r * halves_per_row;
+            load16<kIn>(x, (int64_t)r * ld + 16 * (int64_t)hh, v, ab);
+        }
+        ab = max(ab, __shfl_xor_sync(0xFFFFFFFFu, ab, 1));         // the partner half of the block
+        if (!live) continue;
+        uint32_t code, c0 = 0u, c1 = 0u;
+        if (ab >= 0x7F800000u) {                                   // NaN or Inf in the block
+            flags |= kFlagNonFinite;
+            code = 0xFFu;
+        } else {
+            const int e = ab == 0u ? -127 : max(floor_log2_bits(ab) - 2, -127);
+            code = (uint32_t)(e + 127);
+            const float inv = pow2f(-e);                           // normal: -e in [-125, 127]
+            float y[16];
+#pragma unroll
+            for (int i = 0; i < 16; i += 2) {
+                const float2 t = __fmul2_rn(make_float2(v[i], v[i + 1]), make_float2(inv, inv));
+                y[i] = t.x;
+                y[i + 1] = t.y;
+            }
+            c0 = cvt_e2m1x8(y);
+            c1 = cvt_e2m1x8(y + 8);
+        }
+        *reinterpret_cast<uint2*>(q + (int64_t)h * 8) = make_uint2(c0, c1);
+        if ((h & 1u) == 0u) e8m0[h >> 1] = (uint8_t)code;
+    }
+    flags = __reduce_or_sync(__activemask(), flags);
+    if ((threadIdx.x & 31) == 0) flag_or(d_flags, flags);
+}
+
+// One thread per 8 outputs: 4 code bytes, the block's E8M0 byte, 8 outputs.
+template <int kOut>
+__global__ void __launch_bounds__(kVarThreads)
+mxfp4_dequant_kernel(const uint8_t* __restrict__ q, const uint8_t* __restrict__ e8m0, uint32_t total8, void* out)
+{
+    const uint32_t* qw = reinterpret_cast<const uint32_t*>(q);
+    for (uint32_t h = blockIdx.x * kVarThreads + threadIdx.x; h < total8; h += gridDim.x * kVarThreads) {
+        const uint32_t c = e8m0[h >> 2];
+        const float S = c == 0xFFu ? __uint_as_float(0x7FC00000u) : pow2f((int)c - 127);
+        uint32_t hv[4];
+        cvt_e2m1x8_to_f16x8(__ldcs(qw + h), hv);
+        float y[8];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            float a, b;
+            f16x2_to_f32(hv[j], a, b);
+            y[2 * j] = __fmul_rn(a, S);
+            y[2 * j + 1] = __fmul_rn(b, S);
+        }
+        if constexpr (kOut == 2) {
+            float4* o = reinterpret_cast<float4*>(out) + 2 * (int64_t)h;
+            __stcs(o, make_float4(y[0], y[1], y[2], y[3]));
+            __stcs(o + 1, make_float4(y[4], y[5], y[6], y[7]));
+        } else {
+            uint32_t p[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                if constexpr (kOut == 0)
+                    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(p[j]) : "f"(y[2 * j + 1]), "f"(y[2 * j]));
+                else
+                    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(p[j]) : "f"(y[2 * j + 1]), "f"(y[2 * j]));
+            }
+            __stcs(reinterpret_cast<uint4*>(out) + h, make_uint4(p[0], p[1], p[2], p[3]));
+        }
+    }
+}
+
+// ------------------------------------------------------------------ FP8 E4M3, static per-tensor scale
+// Nearest E4M3 code (0..126) to a / s, a >= 0, s > 0, ties to the even code, saturating;
+// exact FP64 comparisons (value * s has at most 28 significant bits).
+static __device__ __noinline__ uint32_t e4m3_div_exact(float a, float s)
+{
+    const double den = (double)s, num = (double)a;
+    uint32_t lo = 0u, hi = 126u;                                 // largest code with value * den <= num
+    while (lo < hi) {
+        const uint32_t mid = (lo + hi + 1u) >> 1;
+        if ((double)e4m3_value(mid) * den <= num) lo = mid; else hi = mid - 1u;
+    }
+    if (lo == 126u) return 126u;
+    const double t = 0.5 * ((double)e4m3_value(lo) + (double)e4m3_value(lo + 1u)) * den;
+    if (num > t) return lo + 1u;
+    if (num == t) return (lo & 1u) ? lo + 1u : lo;
+    return lo;
+}
+
+// Codes of 16 elements against s (bracket r_lo <= 1/s <= r_hi); exact when the two ends agree.
+__device__ __forceinline__ void fp8_codes16(const float v[16], float s, float r_lo, float r_hi, int mode,
+                                            uint32_t out[4])
+{
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+        uint32_t word = 0u;
+#pragma unroll
+        for (int i = 0; i < 4; i += 2) {
+            const float a0 = fabsf(v[4 * w + i]), a1 = fabsf(v[4 * w + i + 1]);
+            uint32_t c0, c1;
+            if (mode == 0) {                                       // s == 0: sign only
+                c0 = c1 = 0u;
+            } else if (mode == 1) {
+                const uint32_t lo = cvt_e4m3x2(a0 * r_lo, a1 * r_lo), hi = cvt_e4m3x2(a0 * r_hi, a1 * r_hi);
+                c0 = lo & 0xFFu;
+                c1 = lo >> 8;
+                if (c0 != (hi & 0xFFu)) {                          // one exact comparison with the midpoint
+                    const float mid = 0.5f * (e4m3_value(c0) + e4m3_value(c0 + 1u));
+                    const float d = fmaf(mid, s, -a0);
+                    c0 = d < 0.0f ? c0 + 1u : (d > 0.0f ? c0 : c0 + (c0 & 1u));
+                }
+                if (c1 != (hi >> 8)) {
+                    const float mid = 0.5f * (e4m3_value(c1) + e4m3_value(c1 + 1u));
+                    const float d = fmaf(mid, s, -a1);
+                    c1 = d < 0.0f ? c1 + 1u : (d > 0.0f ? c1 : c1 + (c1 & 1u));
+                }
+            } else {
+                c0 = e4m3_div_exact(a0, s);
+                c1 = e4m3_div_exact(a1, s);
+            }
+            c0 |= (__float_as_uint(v[4 * w + i]) >> 24) & 0x80u;
+            c1 |= (__float_as_uint(v[4 * w + i + 1]) >> 24) & 0x80u;
+            word |= (c0 | (c1 << 8)) << (8 * i);
+        }
+        out[w] = word;
+    }
+}
+
+template <int kIn>
+__global__ void __launch_bounds__(kVarThreads)
+fp8_quant_kernel(const void* x, uint32_t rows, uint32_t groups_per_row, int64_t ld, FastDiv div_gpr,
+                 const float* __restrict__ d_amax, uint8_t* __restrict__ q, int64_t ldq, float* __restrict__ d_scale,
+                 uint32_t* __restrict__ d_flags)
+{
+    const float s = __fdiv_rn(*d_amax, 448.0f);                   // RN32(amax / 448)
+    if (blockIdx.x == 0 && threadIdx.x == 0) *d_scale = s;
+    const int mode = s == 0.0f ? 0 : (s >= 0x1p-100f && s <= 0x1p100f ? 1 : 2);
+    const float r = mode == 1 ? __frcp_rn(s) : 0.0f;
+    const float r_lo = __fmul_rn(r, kLoMargin), r_hi = __fmul_rn(r, kHiMargin);
+    uint32_t flags = isfinite(s) ? 0u : kFlagOverflow;
+    const uint32_t total = rows * groups_per_row;
+    for (uint32_t g = blockIdx.x * kVarThreads + threadIdx.x; g < total; g += gridDim.x * kVarThreads) {
+        const uint32_t row = div_gpr.div(g), gg = g - row * groups_per_row;
+        float v[16];
+        uint32_t ab;
+        load16<kIn>(x, (int64_t)row * ld + 16 * (int64_t)gg, v, ab);
+        if (ab >= 0x7F800000u) flags |= kFlagNonFinite;
+        uint32_t w[4];
+        fp8_codes16(v, s, r_lo, r_hi, mode, w);
+        __stcs(reinterpret_cast<uint4*>(q + (int64_t)row * ldq + 16 * (int64_t)gg), make_uint4(w[0], w[1], w[2], w[3]));
+    }
+    flags = __reduce_or_sync(__activemask(), flags);
+    if ((threadIdx.x & 31) == 0) flag_or(d_flags, flags);
+}
+
+// One thread per 16 outputs: out = RN(e4m3(code) * s).
+template <int kOut>
+__global__ void __launch_bounds__(kVarThreads)
+fp8_dequant_kernel(const uint8_t* __restrict__ q, const float* __restrict__ d_scale, uint32_t total16, void* out)
+{
+    const float s = *d_scale;
+    for (uint32_t g = blockIdx.x * kVarThreads + threadIdx.x; g < total16; g += gridDim.x * kVarThreads) {
+        const uint4 c = __ldcs(reinterpret_cast<const uint4*>(q) + g);
+        const uint32_t cw[4] = {c.x, c.y, c.z, c.w};
+        float y[16];
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const uint32_t b = (cw[w] >> (8 * i)) & 0xFFu;
+                const float v = (b & 0x7Fu) == 0x7Fu ? __uint_as_float(0x7FC00000u) : e4m3_value(b & 0x7Fu);
+                y[4 * w + i] = __fmul_rn(b & 0x80u ? -v : v, s);
+            }
+        }
+        if constexpr (kOut == 2) {
+            float4* o = reinterpret_cast<float4*>(out) + 4 * (int64_t)g;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) __stcs(o + k, make_float4(y[4 * k], y[4 * k + 1], y[4 * k + 2], y[4 * k + 3]));
+        } else {
+            uint32_t p[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                if constexpr (kOut == 0)
+                    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(p[j]) : "f"(y[2 * j + 1]), "f"(y[2 * j]));
+                else
+                    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(p[j]) : "f"(y[2 * j + 1]), "f"(y[2 * j]));
+            }
+            uint4* o = reinterpret_cast<uint4*>(out) + 2 * (int64_t)g;
+            __stcs(o, make_uint4(p[0], p[1], p[2], p[3]));
+            __stcs(o + 1, make_uint4(p[4], p[5], p[6], p[7]));
+        }
+    }
+}
+
+// ------------------------------------------------------------------ launchers
+static int var_grid(int64_t work)
+{
+    const int64_t need = (work + kVarThreads - 1) / kVarThreads;
+    const int64_t cap = (int64_t)num_sms() * 8;
+    return (int)(need < cap ? (need > 0 ? need : 1) : cap);
+}
+
+cudaError_t launch_mxfp4_quant(const void* x, int in_dt, int64_t rows, int64_t cols, int64_t ld, uint8_t* q,
+                               uint8_t* e8m0, uint32_t* d_flags, cudaStream_t s)
+{
+    const uint32_t hpr = (uint32_t)(cols / 16);
+    const int64_t total = rows * (int64_t)hpr;
+    const int g = var_grid(total);
+    if (in_dt == 0)
+        mxfp4_quant_kernel<0><<<g, kVarThreads, 0, s>>>(x, (uint32_t)rows, hpr, ld, FastDiv(hpr), q, e8m0, d_flags);
+    else
+        mxfp4_quant_kernel<2><<<g, kVarThreads, 0, s>>>(x, (uint32_t)rows, hpr, ld, FastDiv(hpr), q, e8m0, d_flags);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_mxfp4_dequant(const uint8_t* q, const uint8_t* e8m0, int64_t rows, int64_t cols, int out_dt,
+                                 void* out, cudaStream_t s)
+{
+    const uint32_t total8 = (uint32_t)(rows * (cols / 8));
+    const int g = var_grid(total8);
+    if (out_dt == 0) mxfp4_dequant_kernel<0><<<g, kVarThreads, 0, s>>>(q, e8m0, total8, out);
+    else if (out_dt == 1) mxfp4_dequant_kernel<1><<<g, kVarThreads, 0, s>>>(q, e8m0, total8, out);
+    else mxfp4_dequant_kernel<2><<<g, kVarThreads, 0, s>>>(q, e8m0, total8, out);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_fp8_quant(const void* x, int in_dt, int64_t rows, int64_t cols, int64_t ld, const float* d_amax,
+                             uint8_t* q, float* d_scale, uint32_t* d_flags, cudaStream_t s)
+{
+    const uint32_t gpr = (uint32_t)(cols / 16);
+    const int g = var_grid(rows * (int64_t)gpr);
+    if (in_dt == 0)
+        fp8_quant_kernel<0><<<g, kVarThreads, 0, s>>>(x, (uint32_t)rows, gpr, ld, FastDiv(gpr), d_amax, q, cols,
+                                                       d_scale, d_flags);
+    else
+        fp8_quant_kernel<2><<<g, kVarThreads, 0, s>>>(x, (uint32_t)rows, gpr, ld, FastDiv(gpr), d_amax, q, cols,
+                                                       d_scale, d_flags);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_fp8_dequant(const uint8_t* q, const float* d_scale, int64_t rows, int64_t cols, int out_dt,
+                               void* out, cudaStream_t s)
+{
+    const uint32_t total16 = (uint32_t)(rows * (cols / 16));
+    const int g = var_grid(total16);
+    if (out_dt == 0) fp8_dequant_kernel<0><<<g, kVarThreads, 0, s>>>(q, d_scale, total16, out);
+    else if (out_dt == 1) fp8_dequant_kernel<1><<<g, kVarThreads, 0, s>>>(q, d_scale, total16, out);
+    else fp8_dequant_kernel<2><<<g, kVarThreads, 0, s>>>(q, d_scale, total16, out);
+    return cudaGetLastError();
+}
+
+}  // namespace nv4

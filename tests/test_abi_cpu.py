@@ -29,7 +29,8 @@ def test_header_declares_the_hot_path():
     names = declared_symbols()
     for n in ("nv4_tensor_amax", "nv4_act_quant", "nv4_dequant", "nv4_hessian_accum", "nv4_scale_sweep",
               "nv4_mxfp4_to_nvfp4", "nv4_weight_quant_rtn", "nv4_fake_qdq", "nv4_gemm_nvfp4",
-              "nv4_scales_to_mma_layout", "nv4_mma_scale_bytes"):
+              "nv4_scales_to_mma_layout", "nv4_mma_scale_bytes", "nv4_mxfp4_quant", "nv4_mxfp4_dequant",
+              "nv4_fp8_quant", "nv4_fp8_dequant"):
         assert n in names
 
 
@@ -90,6 +91,16 @@ def test_validation_rejects_before_any_launch(nv4lib):
     assert L.nv4_mma_scale_bytes(5, 20) == 0
     assert L.nv4_scales_to_mma_layout(fake, 4, 20, fake, None) == 2
     assert L.nv4_scales_to_mma_layout(fake, 4, 32, fake + 8, None) == 3
+    # format variants
+    assert L.nv4_mxfp4_quant(fake, 1, 4, 32, 32, fake, fake, None, None) == 4        # fp16 input
+    assert L.nv4_mxfp4_quant(fake, 0, 4, 48, 48, fake, fake, None, None) == 2        # cols % 32
+    assert L.nv4_mxfp4_quant(fake, 2, 4, 32, 34, fake, fake, None, None) == 3        # fp32 row pitch
+    assert L.nv4_mxfp4_quant(None, 0, 4, 32, 32, fake, fake, None, None) == 1
+    assert L.nv4_mxfp4_dequant(fake, fake, 4, 48, 0, fake, None) == 2
+    assert L.nv4_fp8_quant(fake, 0, 4, 24, 24, fake, fake, fake, None, None) == 2    # cols % 16
+    assert L.nv4_fp8_quant(fake, 0, 4, 32, 32, None, fake, fake, None, None) == 1    # amax
+    assert L.nv4_fp8_quant(fake, 0, 4, 32, 32, fake, fake + 4, fake, None, None) == 3
+    assert L.nv4_fp8_dequant(fake, fake, 4, 32, 9, fake, None) == 4
     assert L.nv4_hessian_accum(fake, 10, 40, 40, fake, None, None) == 2
     assert L.nv4_hessian_accum(fake, 10, 32, 36, fake, None, None) == 3
     assert L.nv4_scale_sweep(fake, 2, 4, 32, 34, fake, fake, fake, None, None, None, None, None) == 3  # fp32 ld*4

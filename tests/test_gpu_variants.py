@@ -1,0 +1,112 @@
+"""GPU parity of the format variants against the oracle: MXFP4 quantization and
+dequantization (bit-exact), FP8 E4M3 static per-tensor quantization and dequantization
+(bit-exact), and the MXFP4 -> NVFP4 chain through the cast kernel."""
+import numpy as np
+import pytest
+import torch
+
+import gpu_util as G
+from nvfp4_block_numerics_b200 import binding as nv4
+from nvfp4_block_numerics_b200 import inputs
+
+pytestmark = pytest.mark.gpu
+
+
+def _dev(x):
+    return G.f32_dev(x) if x.dtype == np.float32 else G.bf16_dev(x)
+
+
+def _mx_check(orc, x):
+    xd = _dev(x)
+    f = G.flags_dev()
+    q, e8 = nv4.mxfp4_quant(xd, d_flags=f)
+    rq, re8, rf = orc.mxfp4_quant(np.ascontiguousarray(x))
+    torch.cuda.synchronize()
+    assert f.item() == rf
+    assert np.array_equal(G.host(e8), re8)
+    assert np.array_equal(G.host(q), rq)
+    for dt, name in ((torch.bfloat16, "bf16"), (torch.float16, "fp16"), (torch.float32, "fp32")):
+        out = torch.empty(tuple(x.shape), dtype=dt, device=G.DEV)
+        nv4.nv4_mxfp4_dequant(q, e8, out)
+        ref = orc.mxfp4_dequant(rq, re8, name)
+        got = G.host(out)
+        if name == "fp32":
+            got, ref = got.view(np.uint32), ref.view(np.uint32)
+        assert np.array_equal(got, ref), name
+
+
+@pytest.mark.parametrize("rows,cols", [(1, 32), (3, 96), (129, 160), (300, 1024)])
+def test_mxfp4_small_ragged(orc, rows, cols):
+    r = np.random.default_rng(rows * cols)
+    w = (r.laplace(size=(rows, cols)) * 0.03).astype(np.float32)
+    w[:, 1] *= 80.0
+    w[::4, :32] = 0.0
+    w[1::5, 32:64] = -0.0
+    w[2::7, :32] *= np.float32(1e-35)                     # subnormal block maxima
+    _mx_check(orc, w)
+    _mx_check(orc, inputs.f32_to_bf16_bits(w))
+
+
+def test_mxfp4_edge_values(orc):
+    k = 3
+    g = np.array([0, 0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5, 6, 7.9, -0.25, -5, -6, 1e-30, -0.0, 4] * 2, np.float32)
+    x = np.stack([g * np.float32(2.0 ** k), g * np.float32(2.0 ** -130), g * np.float32(2.0 ** 120),
+                  np.full(32, np.float32(3.4e38))])
+    _mx_check(orc, x)
+
+
+def test_mxfp4_layer_shapes(orc):
+    _mx_check(orc, inputs.c2_shape(4096, 7168))
+    _mx_check(orc, inputs.c3_layer(0, which=("W_q",))["W_q"])
+
+
+def test_mxfp4_quant_then_cast(orc):
+    """The GPU MXFP4 quantizer feeding the GPU cast: in-window blocks dequantize to the
+    MXFP4 values exactly; the whole chain matches the oracle chain."""
+    x = inputs.c2_shape(256, 4096)
+    xd = G.bf16_dev(x)
+    q, e8 = nv4.mxfp4_quant(xd)
+    nvq, nvs, ga, s2 = nv4.mxfp4_to_nvfp4(q, e8)
+    rq, re8, _ = orc.mxfp4_quant(x)
+    ref = orc.mxfp4_to_nvfp4(rq, re8)
+    torch.cuda.synchronize()
+    assert np.array_equal(G.host(nvq), ref["nv_q"]) and np.array_equal(G.host(nvs), ref["nv_scales"])
+    assert s2.item() == ref["s2"]
+
+
+def _fp8_check(orc, x, amax=None):
+    xd = _dev(x)
+    if amax is None:
+        amax = orc.tensor_amax(x)[0]
+    d_amax = torch.tensor([amax], dtype=torch.float32, device=G.DEV)
+    f = G.flags_dev()
+    q, sc = nv4.fp8_quant(xd, d_amax, d_flags=f)
+    rq, rs, rf = orc.fp8_quant(np.ascontiguousarray(x), amax)
+    torch.cuda.synchronize()
+    assert sc.item() == rs and f.item() == rf
+    assert np.array_equal(G.host(q), rq)
+    for dt in (torch.bfloat16, torch.float16, torch.float32):
+        out = torch.empty(tuple(x.shape), dtype=dt, device=G.DEV)
+        nv4.nv4_fp8_dequant(q, sc, out)
+        exact = orc.fp8_dequant(rq, rs)
+        ref = torch.from_numpy(exact.astype(np.float32)).to(dt)            # RN32, then RN to the output type
+        assert torch.equal(out.cpu().view(torch.int16 if dt != torch.float32 else torch.int32),
+                           ref.view(torch.int16 if dt != torch.float32 else torch.int32)), dt
+
+
+@pytest.mark.parametrize("rows,cols", [(1, 16), (3, 48), (129, 80), (300, 1024)])
+def test_fp8_small_ragged(orc, rows, cols):
+    r = np.random.default_rng(rows + 7 * cols)
+    x = (r.laplace(size=(rows, cols)) * 2).astype(np.float32)
+    x[0, 0] = -0.0
+    _fp8_check(orc, x)
+    _fp8_check(orc, inputs.f32_to_bf16_bits(x))
+    _fp8_check(orc, x, amax=float(np.abs(x).max()) / 4)                    # values beyond the static amax
+    _fp8_check(orc, x, amax=0.0)
+
+
+def test_fp8_degenerate_scales_and_layer(orc):
+    r = np.random.default_rng(9)
+    x = (r.standard_normal((4, 64)) * 1e-35).astype(np.float32)
+    _fp8_check(orc, x)                                                      # s far below 2^-100: exact path
+    _fp8_check(orc, inputs.c2_shape(4096, 4096))

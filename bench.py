@@ -293,7 +293,18 @@ def kernel_rooflines(W, hbm_peak):
         t = time_launch(lambda: nv4.nv4_fake_qdq(big["x"], a, qdq, s2, W["flags"]), flush=flush)
         out["fake_qdq"] = {"bound": "hbm", "bytes": 4.0 * n, "s": t, "in_step": False}
         del qdq
-        for k in ("tensor_amax", "act_quant", "dequant", "fake_qdq"):
+        # format variants (widenings; not part of the step)
+        mq = torch.empty((big["T"], big["C"] // 2), dtype=torch.uint8, device=big["x"].device)
+        me = torch.empty((big["T"], big["C"] // 32), dtype=torch.uint8, device=big["x"].device)
+        t = time_launch(lambda: nv4.nv4_mxfp4_quant(big["x"], mq, me, W["flags"]), flush=flush)
+        out["mxfp4_quant"] = {"bound": "hbm", "bytes": (2 + 0.5 + 1 / 32) * n, "s": t, "in_step": False}
+        del mq, me
+        fq = torch.empty((big["T"], big["C"]), dtype=torch.uint8, device=big["x"].device)
+        fs = torch.empty(1, dtype=torch.float32, device=big["x"].device)
+        t = time_launch(lambda: nv4.nv4_fp8_quant(big["x"], a, fq, fs, W["flags"]), flush=flush)
+        out["fp8_quant"] = {"bound": "hbm", "bytes": 3.0 * n, "s": t, "in_step": False}
+        del fq
+        for k in ("tensor_amax", "act_quant", "dequant", "fake_qdq", "mxfp4_quant", "fp8_quant"):
             out[k]["launch"] = f"[{big['T']}, {big['C']}] bf16"
     if "weights" in W:
         # RTN weight quantization of the gate projection (a widening of the path; not in the step)

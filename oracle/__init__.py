@@ -475,3 +475,26 @@ def fp8_dequant(q: np.ndarray, s: float) -> np.ndarray:
     """Exact values e4m3(code) * s (FP64); the caller rounds to its output type."""
     tab = np.array([e4m3_value(c) for c in range(256)], np.float64)
     return tab[np.ascontiguousarray(q)] * float(s)
+
+
+# ---------------------------------------------------------------- block Hadamard rotation
+def _sylvester(n: int) -> np.ndarray:
+    """H_1 = [1], H_2m = [[H_m, H_m], [H_m, -H_m]] (the natural-order Hadamard matrix)."""
+    H = np.ones((1, 1), np.float64)
+    while H.shape[0] < n:
+        H = np.block([[H, H], [H, -H]])
+    return H
+
+
+def hadamard_rotate(x: np.ndarray, n: int) -> np.ndarray:
+    """Block Hadamard rotation along each row ([FP4] section 3.1: blocks of 16..128 values
+    rotated by H / sqrt(n) before FP4 quantization; section 4.1: block sizes 16/32/64/128).
+    Reading: y = RN32(RN64(x_block @ H_n) * RN64(1 / sqrt(n))), the Hadamard sums in FP64
+    (exact for BF16 inputs whose values in a block span fewer than ~38 binades).
+    x: float32 or uint16 (bf16 bits) [rows, cols], cols % n == 0.  Returns float32."""
+    assert n in (16, 32, 64, 128) and x.ndim == 2 and x.shape[1] % n == 0
+    xf = (x.astype(np.uint32) << 16).view(np.float32) if x.dtype == np.uint16 else x
+    rows, cols = xf.shape
+    z = xf.astype(np.float64).reshape(rows, cols // n, n) @ _sylvester(n)     # H_n is symmetric
+    c = float(np.float64(1.0) / np.sqrt(np.float64(n)))
+    return (z * c).astype(np.float32).reshape(rows, cols)

@@ -334,6 +334,29 @@ NV4_API nv4_status nv4_fp8_dequant(const uint8_t* q, const float* d_scale, int64
                            nv4_dtype out_dt, void* out, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * Block Hadamard rotation fused with FP4 quantization ([FP4] section 3.1: blocks rotated
+ * by H / sqrt(n) so that outliers spread before quantization; section 4.1: transform
+ * kernels for block sizes 16, 32, 64 and 128).  Along each row of x (bf16 [rows, cols],
+ * leading dimension ld, ld % 8 == 0, 16-byte aligned, cols % 128 == 0), blocks of n in
+ * {16, 32, 64, 128} consecutive values become y = RN32(RN64(x_block H_n) * RN64(1/sqrt(n)))
+ * with H_n the natural-order (Sylvester) Hadamard matrix; the sums are exact in FP64 for
+ * BF16 inputs whose values in a block span fewer than ~38 binades.
+ *
+ * nv4_hadamard_amax        -- *d_amax = max(*d_amax, max |y|) (running max, as nv4_tensor_amax).
+ * nv4_hadamard_mxfp4_quant -- MXFP4 codes and E8M0 scales of y, as nv4_mxfp4_quant.
+ * nv4_hadamard_nvfp4_quant -- NVFP4 codes and E4M3 scales of y with s2 = RN32(amax / 2688)
+ *                             from *d_amax (e.g. from nv4_hadamard_amax), as nv4_act_quant.
+ * Limits: fewer than 2^31 128-element row segments per call.
+ */
+NV4_API nv4_status nv4_hadamard_amax(const void* x, int64_t rows, int64_t cols, int64_t ld, int n,
+                             float* d_amax, uint32_t* d_flags, void* stream);
+NV4_API nv4_status nv4_hadamard_mxfp4_quant(const void* x, int64_t rows, int64_t cols, int64_t ld, int n,
+                                    uint8_t* q, uint8_t* e8m0, uint32_t* d_flags, void* stream);
+NV4_API nv4_status nv4_hadamard_nvfp4_quant(const void* x, int64_t rows, int64_t cols, int64_t ld, int n,
+                                    const float* d_amax, uint8_t* q, uint8_t* scales, float* d_s2,
+                                    uint32_t* d_flags, void* stream);
+
+/* ---------------------------------------------------------------------------
  * nv4_selftest -- checks, on the current device, the hardware FP4/FP8 conversion
  * instructions the kernels rely on (lane order, rounding, sign of zero, saturation).
  * Writes 64 uint32 results to d_out (device); d_out[0] is a bit mask of failed

@@ -22,7 +22,8 @@ __all__ = [
     "NV4Error", "lib", "nv4_tensor_amax", "nv4_act_quant", "nv4_weight_quant_rtn", "nv4_fake_qdq",
     "nv4_dequant", "nv4_hessian_accum", "weight_quant_rtn", "fake_qdq", "nv4_mma_scale_bytes",
     "nv4_scales_to_mma_layout", "nv4_gemm_nvfp4", "mma_scales", "gemm_nvfp4", "nv4_mxfp4_quant",
-    "nv4_mxfp4_dequant", "nv4_fp8_quant", "nv4_fp8_dequant", "mxfp4_quant", "fp8_quant",
+    "nv4_mxfp4_dequant", "nv4_fp8_quant", "nv4_fp8_dequant", "mxfp4_quant", "fp8_quant", "nv4_hadamard_amax",
+    "nv4_hadamard_mxfp4_quant", "nv4_hadamard_nvfp4_quant", "hadamard_mxfp4_quant", "hadamard_nvfp4_quant",
     "nv4_hessian_accum_batched", "nv4_scale_sweep", "nv4_scale_sweep_batched", "nv4_mxfp4_to_nvfp4",
     "nv4_mxfp4_to_nvfp4_batched", "nv4_selftest", "nv4_version", "FLAG_NONFINITE", "FLAG_E8M0_NAN",
     "FLAG_OVERFLOW", "FLAG_TIMEOUT", "tensor_amax", "act_quant", "dequant", "hessian_accum",
@@ -70,6 +71,9 @@ _SIGS = {
     "nv4_mxfp4_dequant": (C.c_int, [_vp, _vp, _i64, _i64, C.c_int, _vp, _vp]),
     "nv4_fp8_quant": (C.c_int, [_vp, C.c_int, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp]),
     "nv4_fp8_dequant": (C.c_int, [_vp, _vp, _i64, _i64, C.c_int, _vp, _vp]),
+    "nv4_hadamard_amax": (C.c_int, [_vp, _i64, _i64, _i64, C.c_int, _vp, _vp, _vp]),
+    "nv4_hadamard_mxfp4_quant": (C.c_int, [_vp, _i64, _i64, _i64, C.c_int, _vp, _vp, _vp, _vp]),
+    "nv4_hadamard_nvfp4_quant": (C.c_int, [_vp, _i64, _i64, _i64, C.c_int, _vp, _vp, _vp, _vp, _vp, _vp]),
     "nv4_scales_to_mma_layout": (C.c_int, [_vp, _i64, _i64, _vp, _vp]),
     "nv4_gemm_nvfp4": (C.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, C.c_int, _vp, _i64, _vp, _vp]),
     "nv4_hessian_accum": (C.c_int, [_vp, _i64, _i64, _i64, _vp, _vp, _vp]),
@@ -359,6 +363,57 @@ def nv4_fp8_dequant(q: torch.Tensor, d_scale: torch.Tensor, out: torch.Tensor, s
         raise NV4Error("out must be a contiguous bf16, float16 or float32 tensor")
     _check(lib().nv4_fp8_dequant(_ptr(q), _scalar_f32(d_scale, "d_scale"), rows, cols, _DT[out.dtype], _ptr(out),
                                  _stream(stream)), "nv4_fp8_dequant")
+
+
+def _bf16_rows(x, name="x"):
+    if x.dtype != torch.bfloat16:
+        raise NV4Error(f"{name} must be bf16")
+    return _rowmajor(x, name)
+
+
+def nv4_hadamard_amax(x: torch.Tensor, n: int, d_amax: torch.Tensor, d_flags=None, stream=None):
+    rows, cols, ld = _bf16_rows(x)
+    _check(lib().nv4_hadamard_amax(_ptr(x), rows, cols, ld, n, _scalar_f32(d_amax, "d_amax"), _ptr(d_flags),
+                                   _stream(stream)), "nv4_hadamard_amax")
+
+
+def nv4_hadamard_mxfp4_quant(x: torch.Tensor, n: int, q: torch.Tensor, e8m0: torch.Tensor, d_flags=None,
+                             stream=None):
+    rows, cols, ld = _bf16_rows(x)
+    _u8(q, (rows, cols // 2), "q")
+    _u8(e8m0, (rows, cols // 32), "e8m0")
+    _check(lib().nv4_hadamard_mxfp4_quant(_ptr(x), rows, cols, ld, n, _ptr(q), _ptr(e8m0), _ptr(d_flags),
+                                          _stream(stream)), "nv4_hadamard_mxfp4_quant")
+
+
+def nv4_hadamard_nvfp4_quant(x: torch.Tensor, n: int, d_amax: torch.Tensor, q: torch.Tensor, scales: torch.Tensor,
+                             d_s2: torch.Tensor, d_flags=None, stream=None):
+    rows, cols, ld = _bf16_rows(x)
+    _u8(q, (rows, cols // 2), "q")
+    _u8(scales, (rows, cols // 16), "scales")
+    _check(lib().nv4_hadamard_nvfp4_quant(_ptr(x), rows, cols, ld, n, _scalar_f32(d_amax, "d_amax"), _ptr(q),
+                                          _ptr(scales), _scalar_f32(d_s2, "d_s2"), _ptr(d_flags), _stream(stream)),
+           "nv4_hadamard_nvfp4_quant")
+
+
+def hadamard_mxfp4_quant(x: torch.Tensor, n: int, d_flags=None, stream=None):
+    rows, cols = x.shape
+    q = torch.empty((rows, cols // 2), dtype=torch.uint8, device=x.device)
+    e8 = torch.empty((rows, cols // 32), dtype=torch.uint8, device=x.device)
+    nv4_hadamard_mxfp4_quant(x, n, q, e8, d_flags, stream)
+    return q, e8
+
+
+def hadamard_nvfp4_quant(x: torch.Tensor, n: int, d_flags=None, stream=None):
+    """Two passes: the amax of the rotated tensor, then the NVFP4 quantization."""
+    rows, cols = x.shape
+    amax = torch.zeros(1, dtype=torch.float32, device=x.device)
+    nv4_hadamard_amax(x, n, amax, d_flags, stream)
+    q = torch.empty((rows, cols // 2), dtype=torch.uint8, device=x.device)
+    sc = torch.empty((rows, cols // 16), dtype=torch.uint8, device=x.device)
+    s2 = torch.empty(1, dtype=torch.float32, device=x.device)
+    nv4_hadamard_nvfp4_quant(x, n, amax, q, sc, s2, d_flags, stream)
+    return q, sc, s2, amax
 
 
 def mxfp4_quant(x: torch.Tensor, d_flags=None, stream=None):

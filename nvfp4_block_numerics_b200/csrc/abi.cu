@@ -374,3 +374,52 @@ nv4_status nv4_fp8_dequant(const uint8_t* q, const float* d_scale, int64_t rows,
     if (rows * (cols / 16) >= (int64_t)1 << 31) return NV4_ERR_LIMIT;
     return from_cuda(launch_fp8_dequant(q, d_scale, rows, cols, (int)out_dt, out, (cudaStream_t)stream));
 }
+
+// ------------------------------------------------------------------ block Hadamard + FP4
+static nv4_status check_hadamard(const void* x, int64_t rows, int64_t cols, int64_t ld, int n)
+{
+    if (n != 16 && n != 32 && n != 64 && n != 128) return NV4_ERR_SHAPE;
+    if (rows < 0 || cols < 0 || cols % 128 != 0 || ld < cols) return NV4_ERR_SHAPE;
+    if (rows == 0 || cols == 0) return NV4_OK;
+    if (x == nullptr) return NV4_ERR_NULL;
+    if (!aligned16(x) || ld % 8 != 0) return NV4_ERR_ALIGN;
+    if (rows * (cols / 128) >= (int64_t)1 << 31) return NV4_ERR_LIMIT;
+    return NV4_OK;
+}
+
+nv4_status nv4_hadamard_amax(const void* x, int64_t rows, int64_t cols, int64_t ld, int n, float* d_amax,
+                             uint32_t* d_flags, void* stream)
+{
+    nv4_status st = check_hadamard(x, rows, cols, ld, n);
+    if (st != NV4_OK) return st;
+    if (d_amax == nullptr) return NV4_ERR_NULL;
+    if (rows == 0 || cols == 0) return NV4_OK;
+    return from_cuda(launch_hadamard_quant(0, x, rows, cols, ld, n, d_amax, nullptr, nullptr, nullptr, d_flags,
+                                           (cudaStream_t)stream));
+}
+
+nv4_status nv4_hadamard_mxfp4_quant(const void* x, int64_t rows, int64_t cols, int64_t ld, int n, uint8_t* q,
+                                    uint8_t* e8m0, uint32_t* d_flags, void* stream)
+{
+    nv4_status st = check_hadamard(x, rows, cols, ld, n);
+    if (st != NV4_OK) return st;
+    if (rows == 0 || cols == 0) return NV4_OK;
+    if (q == nullptr || e8m0 == nullptr) return NV4_ERR_NULL;
+    if (!aligned16(q)) return NV4_ERR_ALIGN;
+    return from_cuda(launch_hadamard_quant(1, x, rows, cols, ld, n, nullptr, q, e8m0, nullptr, d_flags,
+                                           (cudaStream_t)stream));
+}
+
+nv4_status nv4_hadamard_nvfp4_quant(const void* x, int64_t rows, int64_t cols, int64_t ld, int n,
+                                    const float* d_amax, uint8_t* q, uint8_t* scales, float* d_s2, uint32_t* d_flags,
+                                    void* stream)
+{
+    nv4_status st = check_hadamard(x, rows, cols, ld, n);
+    if (st != NV4_OK) return st;
+    if (d_amax == nullptr || d_s2 == nullptr) return NV4_ERR_NULL;
+    if (rows == 0 || cols == 0) return NV4_OK;
+    if (q == nullptr || scales == nullptr) return NV4_ERR_NULL;
+    if (!aligned16(q)) return NV4_ERR_ALIGN;
+    return from_cuda(launch_hadamard_quant(2, x, rows, cols, ld, n, const_cast<float*>(d_amax), q, scales, d_s2,
+                                           d_flags, (cudaStream_t)stream));
+}

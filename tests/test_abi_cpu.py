@@ -30,7 +30,8 @@ def test_header_declares_the_hot_path():
     for n in ("nv4_tensor_amax", "nv4_act_quant", "nv4_dequant", "nv4_hessian_accum", "nv4_scale_sweep",
               "nv4_mxfp4_to_nvfp4", "nv4_weight_quant_rtn", "nv4_fake_qdq", "nv4_gemm_nvfp4",
               "nv4_scales_to_mma_layout", "nv4_mma_scale_bytes", "nv4_mxfp4_quant", "nv4_mxfp4_dequant",
-              "nv4_fp8_quant", "nv4_fp8_dequant"):
+              "nv4_fp8_quant", "nv4_fp8_dequant", "nv4_hadamard_amax", "nv4_hadamard_mxfp4_quant",
+              "nv4_hadamard_nvfp4_quant"):
         assert n in names
 
 
@@ -101,6 +102,12 @@ def test_validation_rejects_before_any_launch(nv4lib):
     assert L.nv4_fp8_quant(fake, 0, 4, 32, 32, None, fake, fake, None, None) == 1    # amax
     assert L.nv4_fp8_quant(fake, 0, 4, 32, 32, fake, fake + 4, fake, None, None) == 3
     assert L.nv4_fp8_dequant(fake, fake, 4, 32, 9, fake, None) == 4
+    # block Hadamard + FP4
+    assert L.nv4_hadamard_mxfp4_quant(fake, 4, 128, 128, 8, fake, fake, None, None) == 2    # n not in 16..128
+    assert L.nv4_hadamard_mxfp4_quant(fake, 4, 96, 96, 32, fake, fake, None, None) == 2     # cols % 128
+    assert L.nv4_hadamard_mxfp4_quant(fake, 4, 128, 132, 32, fake, fake, None, None) == 3   # ld % 8
+    assert L.nv4_hadamard_amax(fake, 4, 128, 128, 64, None, None, None) == 1
+    assert L.nv4_hadamard_nvfp4_quant(fake, 4, 128, 128, 128, fake, None, fake, fake, None, None) == 1
     assert L.nv4_hessian_accum(fake, 10, 40, 40, fake, None, None) == 2
     assert L.nv4_hessian_accum(fake, 10, 32, 36, fake, None, None) == 3
     assert L.nv4_scale_sweep(fake, 2, 4, 32, 34, fake, fake, fake, None, None, None, None, None) == 3  # fp32 ld*4

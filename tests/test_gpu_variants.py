@@ -110,3 +110,34 @@ def test_fp8_degenerate_scales_and_layer(orc):
     x = (r.standard_normal((4, 64)) * 1e-35).astype(np.float32)
     _fp8_check(orc, x)                                                      # s far below 2^-100: exact path
     _fp8_check(orc, inputs.c2_shape(4096, 4096))
+
+
+# ------------------------------------------------------------------ block Hadamard + FP4
+@pytest.mark.parametrize("n", [16, 32, 64, 128])
+def test_hadamard_quant_matches_oracle(orc, n):
+    x = inputs.laplace_bf16(inputs.rng_for(n, "gpu", "had"), 129, 512, outlier_channels=(3, 200), outlier_scale=50,
+                            zero_block_frac=0.02)
+    xd = G.bf16_dev(x)
+    y = orc.hadamard_rotate(x, n)
+    # amax of the rotated tensor
+    amax = torch.zeros(1, dtype=torch.float32, device=G.DEV)
+    nv4.nv4_hadamard_amax(xd, n, amax)
+    assert amax.item() == float(np.abs(y).max())
+    # MXFP4 of the rotated values
+    q, e8 = nv4.hadamard_mxfp4_quant(xd, n)
+    rq, re8, _ = orc.mxfp4_quant(y)
+    assert np.array_equal(G.host(e8), re8) and np.array_equal(G.host(q), rq)
+    # NVFP4 of the rotated values (two passes)
+    q, sc, s2, _ = nv4.hadamard_nvfp4_quant(xd, n)
+    nq, nsc, ns2, _ = orc.rtn_quant(y, float(np.abs(y).max()))
+    assert s2.item() == ns2
+    assert np.array_equal(G.host(sc), nsc) and np.array_equal(G.host(q), nq)
+
+
+def test_hadamard_quant_layer_shape(orc):
+    x = inputs.c2_shape(4096, 7168)
+    rows = np.sort(np.random.default_rng(1).choice(4096, 64, replace=False))
+    xd = G.bf16_dev(x)
+    q, e8 = nv4.hadamard_mxfp4_quant(xd, 128)
+    rq, re8, _ = orc.mxfp4_quant(orc.hadamard_rotate(np.ascontiguousarray(x[rows]), 128))
+    assert np.array_equal(G.host(e8)[rows], re8) and np.array_equal(G.host(q)[rows], rq)

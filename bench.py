@@ -304,7 +304,14 @@ def kernel_rooflines(W, hbm_peak):
         t = time_launch(lambda: nv4.nv4_fp8_quant(big["x"], a, fq, fs, W["flags"]), flush=flush)
         out["fp8_quant"] = {"bound": "hbm", "bytes": 3.0 * n, "s": t, "in_step": False}
         del fq
-        for k in ("tensor_amax", "act_quant", "dequant", "fake_qdq", "mxfp4_quant", "fp8_quant"):
+        # block Hadamard (n = 128) fused with MXFP4 quantization: one pass, 2 B in, 0.53 B out
+        hq = torch.empty((big["T"], big["C"] // 2), dtype=torch.uint8, device=big["x"].device)
+        he = torch.empty((big["T"], big["C"] // 32), dtype=torch.uint8, device=big["x"].device)
+        t = time_launch(lambda: nv4.nv4_hadamard_mxfp4_quant(big["x"], 128, hq, he, W["flags"]), flush=flush)
+        out["hadamard128_mxfp4_quant"] = {"bound": "hbm", "bytes": (2 + 0.5 + 1 / 32) * n, "s": t, "in_step": False}
+        del hq, he
+        for k in ("tensor_amax", "act_quant", "dequant", "fake_qdq", "mxfp4_quant", "fp8_quant",
+                  "hadamard128_mxfp4_quant"):
             out[k]["launch"] = f"[{big['T']}, {big['C']}] bf16"
     if "weights" in W:
         # RTN weight quantization of the gate projection (a widening of the path; not in the step)

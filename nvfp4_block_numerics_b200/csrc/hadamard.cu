@@ -7,12 +7,12 @@
 //   mode 1: MXFP4 quantization of y (32-element blocks, E8M0 scales);
 //   mode 2: NVFP4 quantization of y with s2 = RN32(amax / 2688).
 //
-// Mapping: a half-warp owns a 128-element row segment, 8 consecutive elements per lane
-// (one 16-byte load).  The fast Walsh-Hadamard transform runs in FP64: three butterfly
-// stages inside a lane, then log2(n / 8) stages across lanes with shuffles, so every
-// sum is exact for BF16 inputs spanning fewer than ~38 binades in a block.  The
-// quantizers then work on FP32 y exactly as nv4_mxfp4_quant / nv4_act_quant do: MXFP4
-// blocks are 4 lanes (maxima combined with two shuffles), NVFP4 blocks 2 lanes.
+// Mapping: a lane owns 32 consecutive elements of a row (four 16-byte loads); four lanes
+// cover a 128-element segment.  The fast Walsh-Hadamard transform runs in FP64: up to
+// five butterfly stages inside a lane, then log2(n / 32) stages across lanes with
+// shuffles (n = 64, 128), so every sum is exact for BF16 inputs spanning fewer than ~38
+// binades in a block.  The quantizers then work on FP32 y exactly as nv4_mxfp4_quant /
+// nv4_act_quant do; an MXFP4 block is one lane's 32 values, an NVFP4 block half of them.
 #include <cmath>
 
 #include "nv4_common.cuh"
@@ -20,25 +20,27 @@
 
 namespace nv4 {
 
-constexpr int kHadThreads = 256;
+constexpr int kHadThreads = 128;
 
-// FWHT of 128 / n independent blocks of n values spread over a half-warp, 8 per lane.
-__device__ __forceinline__ void fwht(double v[8], int n, uint32_t lane)
+// FWHT of blocks of n values, 32 consecutive values per lane: five butterfly stages
+// inside the lane, then log2(n / 32) stages across neighbouring lanes (n = 64, 128).
+__device__ __forceinline__ void fwht32(double v[32], int n, uint32_t lane)
 {
 #pragma unroll
-    for (int h = 1; h < 8; h <<= 1) {                 // in-lane stages (bits 0..2 of the index)
+    for (int h = 1; h < 32; h <<= 1) {
+        if (h >= n) break;                            // blocks of 16: only four in-lane stages
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
+        for (int i = 0; i < 32; ++i) {
             if (i & h) continue;
             const double a = v[i], b = v[i + h];
             v[i] = a + b;
             v[i + h] = a - b;
         }
     }
-    for (int d = 1; d < n / 8; d <<= 1) {             // across lanes (bits 3.. of the index)
+    for (int d = 1; d < n / 32; d <<= 1) {
         const bool upper = (lane & (uint32_t)d) != 0u;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
+        for (int i = 0; i < 32; ++i) {
             const double o = __shfl_xor_sync(0xFFFFFFFFu, v[i], d);
             v[i] = upper ? o - v[i] : v[i] + o;
         }
@@ -59,13 +61,14 @@ __device__ __forceinline__ float had_pow2(int k)
 
 template <int kMode>
 __global__ void __launch_bounds__(kHadThreads)
-hadamard_quant_kernel(const uint16_t* x, uint32_t rows, uint32_t segs_per_row, int64_t ld, FastDiv div_spr, int n,
+hadamard_quant_kernel(const uint16_t* x, uint32_t rows, uint32_t chunks_per_row, int64_t ld, FastDiv div_cpr, int n,
                       double c, float* __restrict__ d_amax, uint8_t* __restrict__ q, uint8_t* __restrict__ sc,
                       float* __restrict__ d_s2, uint32_t* __restrict__ d_flags)
 {
-    const uint32_t lane = threadIdx.x & 31u, sub = lane & 15u, half = lane >> 4;
-    const uint32_t total = rows * segs_per_row;
-    const uint32_t warps = gridDim.x * (kHadThreads / 32);
+    // one lane = one 32-element chunk of a row (4 lanes = one 128-element segment)
+    const uint32_t lane = threadIdx.x & 31u;
+    const uint32_t total = rows * chunks_per_row;                 // multiple of 4
+    const uint32_t stride = gridDim.x * kHadThreads;
     uint32_t flags = 0u, mx_bits = 0u;
 
     float s2 = 0.0f, k_lo = 0.0f, k_hi = 0.0f;
@@ -79,100 +82,126 @@ hadamard_quant_kernel(const uint16_t* x, uint32_t rows, uint32_t segs_per_row, i
         k_hi = __fmul_rn(k, kHiMargin);
         if (!isfinite(s2)) flags |= kFlagOverflow;
     }
+    const int64_t cols = (int64_t)chunks_per_row * 32;
 
-    for (uint32_t w = blockIdx.x * (kHadThreads / 32) + (threadIdx.x >> 5); 2u * w < total; w += warps) {
-        const uint32_t seg = 2u * w + half;
-        const bool live = seg < total;
-        uint32_t r = 0u, s = 0u;
-        double v[8];
-        if (live) {
-            r = div_spr.div(seg);
-            s = seg - r * segs_per_row;
-            const uint4 raw = __ldcs(reinterpret_cast<const uint4*>(x + (int64_t)r * ld + 128 * (int64_t)s + 8 * sub));
-            const uint32_t wv[4] = {raw.x, raw.y, raw.z, raw.w};
+    // warp-uniform trip count (lanes of one 128-element segment exchange values); the
+    // next chunk's four loads are issued before the current chunk is transformed
+    auto load = [&](uint32_t ch, uint4 raw[4]) {
+        const uint32_t rr = div_cpr.div(ch), c2 = ch - rr * chunks_per_row;
+        const uint4* src = reinterpret_cast<const uint4*>(x + (int64_t)rr * ld + 32 * (int64_t)c2);
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                v[2 * j] = (double)bf16_lo(wv[j]);
-                v[2 * j + 1] = (double)bf16_hi(wv[j]);
+        for (int k = 0; k < 4; ++k) raw[k] = __ldcs(src + k);
+    };
+    uint4 nxt[4];
+    {
+        const uint32_t ch0 = blockIdx.x * kHadThreads + (threadIdx.x & ~31u) + lane;
+        if (ch0 < total) load(ch0, nxt);
+    }
+    for (uint32_t c0 = blockIdx.x * kHadThreads + (threadIdx.x & ~31u); c0 < total; c0 += stride) {
+        const uint32_t ch = c0 + lane;
+        const bool live = ch < total;                              // segments are all-live or all-dead
+        uint32_t r = 0u, cc = 0u;
+        double v[32];
+        if (live) {
+            r = div_cpr.div(ch);
+            cc = ch - r * chunks_per_row;
+            uint4 raw[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) raw[k] = nxt[k];
+            if (ch + stride < total) load(ch + stride, nxt);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const uint32_t wv[4] = {raw[k].x, raw[k].y, raw[k].z, raw[k].w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    v[8 * k + 2 * j] = (double)bf16_lo(wv[j]);
+                    v[8 * k + 2 * j + 1] = (double)bf16_hi(wv[j]);
+                }
             }
         } else {
 #pragma unroll
-            for (int j = 0; j < 8; ++j) v[j] = 0.0;
+            for (int j = 0; j < 32; ++j) v[j] = 0.0;
         }
-        fwht(v, n, lane);
-        float y[8];
+        fwht32(v, n, lane);
+        if (!live) continue;
+
+        float y[32];
         uint32_t ab = 0u;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            y[j] = (float)(v[j] * c);                    // RN32(RN64(z * c))
+        for (int j = 0; j < 32; ++j) {
+            y[j] = (float)(v[j] * c);                              // RN32(RN64(z * c))
             ab = max(ab, __float_as_uint(y[j]) & 0x7FFFFFFFu);
         }
-        if (ab >= 0x7F800000u && live) flags |= kFlagNonFinite;
+        if (ab >= 0x7F800000u) flags |= kFlagNonFinite;
+        const int64_t col = 32 * (int64_t)cc;
 
         if constexpr (kMode == 0) {
-            if (live && ab <= 0x7F800000u) mx_bits = max(mx_bits, ab);
+            if (ab <= 0x7F800000u) mx_bits = max(mx_bits, ab);
         } else if constexpr (kMode == 1) {
-            // MXFP4 block = 4 lanes (32 elements)
-            uint32_t bm = max(ab, __shfl_xor_sync(0xFFFFFFFFu, ab, 1));
-            bm = max(bm, __shfl_xor_sync(0xFFFFFFFFu, bm, 2));
-            if (live) {
-                uint32_t code, c0 = 0u;
-                if (bm >= 0x7F800000u) {
-                    code = 0xFFu;
-                } else {
-                    const int e = bm == 0u ? -127 : max(had_floor_log2(bm) - 2, -127);
-                    code = (uint32_t)(e + 127);
-                    const float inv = had_pow2(-e);
+            uint32_t code, w[4] = {0u, 0u, 0u, 0u};
+            if (ab >= 0x7F800000u) {
+                code = 0xFFu;
+            } else {
+                const int e = ab == 0u ? -127 : max(had_floor_log2(ab) - 2, -127);
+                code = (uint32_t)(e + 127);
+                const float inv = had_pow2(-e);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
                     float t[8];
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) t[j] = __fmul_rn(y[j], inv);   // exact
-                    c0 = cvt_e2m1x8(t);
+                    for (int j = 0; j < 8; ++j) t[j] = __fmul_rn(y[8 * k + j], inv);   // exact
+                    w[k] = cvt_e2m1x8(t);
                 }
-                const int64_t col = 128 * (int64_t)s + 8 * sub;              // first element of this lane
-                const int64_t cols = (int64_t)segs_per_row * 128;
-                *reinterpret_cast<uint32_t*>(q + (int64_t)r * (cols / 2) + col / 2) = c0;
-                if ((sub & 3u) == 0u) sc[(int64_t)r * (cols / 32) + col / 32] = (uint8_t)code;
             }
+            __stcs(reinterpret_cast<uint4*>(q + (int64_t)r * (cols / 2) + col / 2), make_uint4(w[0], w[1], w[2], w[3]));
+            sc[(int64_t)r * (cols / 32) + col / 32] = (uint8_t)code;
         } else {
-            // NVFP4 block = 2 lanes (16 elements)
-            const uint32_t bm = max(ab, __shfl_xor_sync(0xFFFFFFFFu, ab, 1));
-            if (live) {
+            uint32_t w[4], codes2 = 0u;
+#pragma unroll
+            for (int hb = 0; hb < 2; ++hb) {                       // two NVFP4 blocks of 16
+                uint32_t bm = 0u;
+#pragma unroll
+                for (int j = 0; j < 16; ++j) bm = max(bm, __float_as_uint(y[16 * hb + j]) & 0x7FFFFFFFu);
                 const float a_b = __uint_as_float(bm);
                 uint32_t code;
                 if (fast_scale) {
-                    const uint32_t cc = cvt_e4m3x2(__fmul_rn(a_b, k_lo), __fmul_rn(a_b, k_hi));
-                    code = cc & 0xFFu;
-                    if (code != (cc >> 8)) code = e4m3_fix(code, a_b, s2);
+                    const uint32_t cv = cvt_e4m3x2(__fmul_rn(a_b, k_lo), __fmul_rn(a_b, k_hi));
+                    code = cv & 0xFFu;
+                    if (code != (cv >> 8)) code = e4m3_fix(code, a_b, s2);
                 } else {
                     code = e4m3_code_exact(a_b, s2);
                 }
                 code &= 0x7Fu;
-                const float S = __fmul_rn(e4m3_value(code), s2);           // DQ1: RN32(s_b * s2)
-                uint32_t c0 = 0u;
-                if (S == 0.0f) {
+                codes2 |= code << (8 * hb);
+                const float S = __fmul_rn(e4m3_value(code), s2);   // DQ1: RN32(s_b * s2)
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) c0 |= ((__float_as_uint(y[j]) >> 28) & 8u) << (4 * j);
-                } else if (S >= kTinyScale && S <= 0x1p100f) {
-                    const float rr = __frcp_rn(S);
-                    const float rl = __fmul_rn(rr, kLoMargin), rh = __fmul_rn(rr, kHiMargin);
-                    float lo[8], hi[8];
+                for (int k = 0; k < 2; ++k) {
+                    const float* yy = y + 16 * hb + 8 * k;
+                    uint32_t c8 = 0u;
+                    if (S == 0.0f) {
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        lo[j] = __fmul_rn(y[j], rl);
-                        hi[j] = __fmul_rn(y[j], rh);
+                        for (int j = 0; j < 8; ++j) c8 |= ((__float_as_uint(yy[j]) >> 28) & 8u) << (4 * j);
+                    } else if (S >= kTinyScale && S <= 0x1p100f) {
+                        const float rr = __frcp_rn(S);
+                        const float rl = __fmul_rn(rr, kLoMargin), rh = __fmul_rn(rr, kHiMargin);
+                        float lo[8], hi[8];
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            lo[j] = __fmul_rn(yy[j], rl);
+                            hi[j] = __fmul_rn(yy[j], rh);
+                        }
+                        c8 = cvt_e2m1x8(lo);
+                        const uint32_t h8 = cvt_e2m1x8(hi);
+                        if (c8 != h8) c8 = e2m1_fix8(yy, S, c8, h8);
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) c8 |= e2m1_code_exact(yy[j], S) << (4 * j);
                     }
-                    c0 = cvt_e2m1x8(lo);
-                    const uint32_t h0 = cvt_e2m1x8(hi);
-                    if (c0 != h0) c0 = e2m1_fix8(y, S, c0, h0);
-                } else {
-#pragma unroll 1
-                    for (int j = 0; j < 8; ++j) c0 |= e2m1_code_exact(y[j], S) << (4 * j);
+                    w[2 * hb + k] = c8;
                 }
-                const int64_t col = 128 * (int64_t)s + 8 * sub;
-                const int64_t cols = (int64_t)segs_per_row * 128;
-                *reinterpret_cast<uint32_t*>(q + (int64_t)r * (cols / 2) + col / 2) = c0;
-                if ((sub & 1u) == 0u) sc[(int64_t)r * (cols / 16) + col / 16] = (uint8_t)code;
             }
+            __stcs(reinterpret_cast<uint4*>(q + (int64_t)r * (cols / 2) + col / 2), make_uint4(w[0], w[1], w[2], w[3]));
+            *reinterpret_cast<uint16_t*>(sc + (int64_t)r * (cols / 16) + col / 16) = (uint16_t)codes2;
         }
     }
     if constexpr (kMode == 0) {
@@ -187,10 +216,9 @@ cudaError_t launch_hadamard_quant(int mode, const void* x, int64_t rows, int64_t
                                   float* d_amax, uint8_t* q, uint8_t* sc, float* d_s2, uint32_t* d_flags,
                                   cudaStream_t s)
 {
-    const uint32_t spr = (uint32_t)(cols / 128);
-    const int64_t segs = rows * (int64_t)spr;
-    const int64_t warps_needed = (segs + 1) / 2;
-    const int64_t need = (warps_needed + kHadThreads / 32 - 1) / (kHadThreads / 32);
+    const uint32_t spr = (uint32_t)(cols / 32);                  // 32-element chunks per row
+    const int64_t chunks = rows * (int64_t)spr;
+    const int64_t need = (chunks + kHadThreads - 1) / kHadThreads;
     const int64_t cap = (int64_t)num_sms() * 8;
     const int grid = (int)(need < cap ? (need > 0 ? need : 1) : cap);
     const double c = 1.0 / std::sqrt((double)n);

@@ -62,6 +62,8 @@ def parse_args():
     p.add_argument("--seed", type=int, default=0)
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-rooflines", action="store_true",
+                   help="skip the per-kernel micro-timings (for launch-list profiling of the step alone)")
     return p.parse_args()
 
 
@@ -600,7 +602,7 @@ def run_ours(args):
     part_s = {p: t[i + 1] for i, p in enumerate(parts)}
     flags = int(W["flags"].item())
 
-    roof = kernel_rooflines(W, hbm_peak)
+    roof = {} if args.no_rooflines else kernel_rooflines(W, hbm_peak)
     e2e = None
     if "act" in parts and not args.no_e2e:
         e2e_s, h2d, d2h = e2e_act(W, max(1, min(args.steps, 3)))
@@ -621,7 +623,7 @@ def run_ours(args):
         bytes_act, n_act = act_bytes(W)
         value = ws * bytes_act * args.steps / part_s["act"] / 1e9
     sweep = None
-    if "calib" in parts:
+    if "calib" in parts and "scale_sweep" in roof:
         blocks = sum(j["codes"].numel() for j in W["weights"])
         sw = roof["scale_sweep"]
         sweep = {"value": ws * blocks * args.steps / part_s["calib"], "unit": "blocks/s",

@@ -42,6 +42,8 @@
 namespace nv4 {
 
 constexpr int kSweepThreads = 128;
+constexpr int kMaxTilesPerCta = 4;                     // a CTA sorts and searches up to 512 rows
+constexpr int kMaxRowsPerCta = kMaxTilesPerCta * kSweepThreads;
 constexpr float kPruneScale = 1.0f - 0x1p-10f;   // bound * this must exceed the runner-up
 
 struct SweepJobDev {
@@ -229,8 +231,9 @@ sweep_kernel(const __grid_constant__ SweepParams p)
     __shared__ float4 rd4[4];
     __shared__ int bound_ok;
     __shared__ uint32_t hist[128], base[128];
-    __shared__ float4 sw[kSweepThreads][4];
-    __shared__ uint32_t srow[kSweepThreads];
+    __shared__ float4 sw[kMaxRowsPerCta][4];                 // the group's weight blocks, load order
+    __shared__ uint32_t srow[kMaxRowsPerCta];                 // their rows (kNoRow past the end)
+    __shared__ uint16_t perm[kMaxRowsPerCta];                 // sorted position -> load slot
 
     // locate job and tile group
     int j = 0;
@@ -278,18 +281,22 @@ sweep_kernel(const __grid_constant__ SweepParams p)
     const uint32_t s2flag = isfinite(s2) ? 0u : kFlagOverflow;
 
     uint32_t nvisit = 0u, nfull = 0u;
-    const uint32_t tile_end = min(job.row_tiles, (group + 1) * p.tiles_per_cta);
-#pragma unroll 1
-    for (uint32_t tile = group * p.tiles_per_cta; tile < tile_end; ++tile) {
-        // ---- load, starting code, counting sort by starting code
-        uint32_t row = tile * kSweepThreads + threadIdx.x;
+    // ---- load the group's rows (up to 4 tiles of 128), counting-sort them by starting code
+    const uint32_t tile0 = group * p.tiles_per_cta;
+    const uint32_t ntile = min(job.row_tiles - tile0, p.tiles_per_cta);
+    uint32_t keys[kMaxTilesPerCta], ranks[kMaxTilesPerCta];
+#pragma unroll
+    for (uint32_t k = 0; k < kMaxTilesPerCta; ++k) {
+        if (k >= ntile) break;
+        const uint32_t slot = k * kSweepThreads + threadIdx.x;
+        uint32_t row = (tile0 + k) * kSweepThreads + threadIdx.x;
         float2 w[8];
         uint32_t key = 127u;
         if (row < job.rows) {
             load_block<kDt>(job, row, b, w);
             float a1 = 0.0f;
 #pragma unroll
-            for (int k = 0; k < 8; ++k) a1 = fmaxf(a1, fmaxf(fabsf(w[k].x), fabsf(w[k].y)));
+            for (int j = 0; j < 8; ++j) a1 = fmaxf(a1, fmaxf(fabsf(w[j].x), fabsf(w[j].y)));
             if (a1 > 0.0f) {
                 const float t0 = __fmul_rn(a1, k6);
                 key = min(cvt_e4m3x2(t0, t0) & 0x7Fu, 126u);
@@ -297,42 +304,53 @@ sweep_kernel(const __grid_constant__ SweepParams p)
         } else {
             row = kNoRow;
 #pragma unroll
-            for (int k = 0; k < 8; ++k) w[k] = make_float2(0.0f, 0.0f);
+            for (int j = 0; j < 8; ++j) w[j] = make_float2(0.0f, 0.0f);
         }
-        const uint32_t rank = atomicAdd(&hist[key], 1u);
-        __syncthreads();
-        if (threadIdx.x < 32) {                 // exclusive scan of the 128 bucket counts
-            const uint32_t l = threadIdx.x;
-            const uint32_t h0 = hist[4 * l], h1 = hist[4 * l + 1], h2 = hist[4 * l + 2], h3 = hist[4 * l + 3];
-            uint32_t sum = h0 + h1 + h2 + h3, incl = sum;
 #pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
-                if (l >= (uint32_t)o) incl += t;
-            }
-            const uint32_t ex = incl - sum;
-            base[4 * l] = ex;
-            base[4 * l + 1] = ex + h0;
-            base[4 * l + 2] = ex + h0 + h1;
-            base[4 * l + 3] = ex + h0 + h1 + h2;
-            hist[4 * l] = hist[4 * l + 1] = hist[4 * l + 2] = hist[4 * l + 3] = 0u;
-        }
-        __syncthreads();
-        {
-            const uint32_t pos = base[key] + rank;
+        for (int j = 0; j < 4; ++j) sw[slot][j] = make_float4(w[2 * j].x, w[2 * j].y, w[2 * j + 1].x, w[2 * j + 1].y);
+        srow[slot] = row;
+        keys[k] = key;
+        ranks[k] = atomicAdd(&hist[key], 1u);
+    }
+    __syncthreads();
+    if (threadIdx.x < 32) {                     // exclusive scan of the 128 bucket counts
+        const uint32_t l = threadIdx.x;
+        const uint32_t h0 = hist[4 * l], h1 = hist[4 * l + 1], h2 = hist[4 * l + 2], h3 = hist[4 * l + 3];
+        uint32_t sum = h0 + h1 + h2 + h3, incl = sum;
 #pragma unroll
-            for (int k = 0; k < 4; ++k) sw[pos][k] = make_float4(w[2 * k].x, w[2 * k].y, w[2 * k + 1].x, w[2 * k + 1].y);
-            srow[pos] = row;
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+            if (l >= (uint32_t)o) incl += t;
         }
-        __syncthreads();
-        row = srow[threadIdx.x];
+        const uint32_t ex = incl - sum;
+        base[4 * l] = ex;
+        base[4 * l + 1] = ex + h0;
+        base[4 * l + 2] = ex + h0 + h1;
+        base[4 * l + 3] = ex + h0 + h1 + h2;
+    }
+    __syncthreads();
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const float4 v = sw[threadIdx.x][k];
-            w[2 * k] = make_float2(v.x, v.y);
-            w[2 * k + 1] = make_float2(v.z, v.w);
+    for (uint32_t k = 0; k < kMaxTilesPerCta; ++k) {
+        if (k >= ntile) break;
+        perm[base[keys[k]] + ranks[k]] = (uint16_t)(k * kSweepThreads + threadIdx.x);
+    }
+    __syncthreads();
+
+    // ---- each warp walks interleaved groups of 32 sorted rows, without further barriers
+    const uint32_t nslots = ntile * kSweepThreads;
+    const uint32_t warp = threadIdx.x >> 5, lane = threadIdx.x & 31u;
+#pragma unroll 1
+    for (uint32_t g = warp; 32u * g < nslots; g += kSweepThreads / 32) {
+        const uint32_t slot = perm[32u * g + lane];
+        const uint32_t row = srow[slot];
+        float2 w[8];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float4 v = sw[slot][j];
+            w[2 * j] = make_float2(v.x, v.y);
+            w[2 * j + 1] = make_float2(v.z, v.w);
         }
-        if (row == kNoRow) continue;            // no barrier follows inside this tile
+        if (row == kNoRow) continue;
 
         // ---- the search for this thread's (row, b)
         uint32_t flags = s2flag;
@@ -435,7 +453,7 @@ cudaError_t launch_sweep(const nv4_sweep_job* jobs, int n, int dt, uint32_t* d_f
     uint64_t tiles = 0;
     for (int i = 0; i < m; ++i) tiles += (uint64_t)p.jobs[i].row_tiles * p.jobs[i].nblk;
     const uint64_t per = tiles / ((uint64_t)num_sms() * 16u);
-    p.tiles_per_cta = (uint32_t)(per < 1 ? 1 : (per > 4 ? 4 : per));
+    p.tiles_per_cta = (uint32_t)(per < 1 ? 1 : (per > (uint64_t)kMaxTilesPerCta ? kMaxTilesPerCta : per));
     for (int i = 0; i < m; ++i) {
         SweepJobDev& d = p.jobs[i];
         d.cta_begin = ctas;

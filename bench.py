@@ -500,6 +500,15 @@ def cpu_baseline(seed, budget_s=20.0):
 
 
 # ---------------------------------------------------------------------- arms
+def workload_config(parts, seed, ws):
+    """The workload both arms report (the reference arm times a bounded sample of it)."""
+    return {"workload": "NVFP4 hot path: activation quant sweep (15 [T,C] shapes, amax->quant->dequant) "
+                        "+ Gemma-2B-like layer calibration (Hessians of X 16384x2048 and 16384x16384, "
+                        "sweep of q/gate/up/down) + MXFP4->NVFP4 cast of 32 x 2880x2880",
+            "parts": list(parts), "seed": seed, "parallelism": f"replicas x{ws}",
+            "l2": "no flush: every step touches ~5 GB, above the 126 MB L2"}
+
+
 def dist_setup(args):
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -508,6 +517,10 @@ def dist_setup(args):
 
 
 def run_reference(args):
+    """The oracle (plain CPU code, FP64) as the reference arm: each step runs a bounded sample
+    of the same workload on the host cores -- the activation path on <= 64 rows of every
+    shape (the metric's GB/s half) and the Hessian-weighted sweep on 64 rows x 128 blocks of
+    q_proj (its blocks/s half)."""
     ws, rank, _ = dist_setup(args)
     if rank != 0:
         return
@@ -517,26 +530,41 @@ def run_reference(args):
     threads = oracle.default_threads()
     xs = [inputs.c2_shape(min(T, 64), C, args.seed) for (T, C) in inputs.C2_SHAPES]
     nelem = sum(x.size for x in xs)
+    d = inputs.c3_layer(args.seed, which=("X", "W_q"))
+    H = oracle.hessian_accum(d["X"][:2048], threads=threads)
+    wq = np.ascontiguousarray(d["W_q"][:64])
+    amax_w = oracle.tensor_amax(d["W_q"], threads)[0]
+    n_blocks = wq.size // 16
+    t_act, t_sweep = [0.0], [0.0]
 
     def step():
+        t0 = time.perf_counter()
         for x in xs:
             a, _ = oracle.tensor_amax(x, threads)
             q, sc, s2, _ = oracle.act_quant(x, a, threads=threads)
             oracle.dequant(q, sc, s2, "bf16", threads)
+        t1 = time.perf_counter()
+        oracle.scale_sweep(wq, H, amax_w, threads=threads)
+        t2 = time.perf_counter()
+        t_act[0] += t1 - t0
+        t_sweep[0] += t2 - t1
 
     for _ in range(args.warmup):
         step()
+    t_act[0] = t_sweep[0] = 0.0
     t = time.perf_counter()
     for _ in range(args.steps):
         step()
     el = (time.perf_counter() - t) / args.steps
-    v = nelem * sum(ACT_BYTES.values()) / el / 1e9
-    sample = f"act path on min(T,64) rows of each of the 15 [T, C] shapes ({nelem} elements per step)"
+    v = nelem * sum(ACT_BYTES.values()) / (t_act[0] / args.steps) / 1e9
+    sweep_bps = n_blocks / (t_sweep[0] / args.steps)
+    sample = (f"act path on min(T,64) rows of each of the 15 [T, C] shapes ({nelem} elements per step); "
+              f"sweep on 64 rows x 128 blocks of q_proj ({n_blocks} blocks per step, H from 2048 tokens)")
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "GB/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": el * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": "dynamic activation quant sweep (15 shapes), bounded row sample",
-                       "parallelism": "host threads"},
+            "config": workload_config(args.parts.split(","), args.seed, 1),
+            "sweep": {"value": sweep_bps, "unit": "blocks/s"},
             "cpu_baseline": {"value": v, "unit": "GB/s", "cores": threads, "kind": "oracle", "sample": sample},
             "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -650,11 +678,7 @@ def run_ours(args):
         "metric": METRIC, "value": value, "unit": unit, "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": total_s / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": "NVFP4 hot path: activation quant sweep (15 [T,C] shapes, amax->quant->dequant) "
-                               "+ Gemma-2B-like layer calibration (Hessians of X 16384x2048 and 16384x16384, "
-                               "sweep of q/gate/up/down) + MXFP4->NVFP4 cast of 32 x 2880x2880",
-                   "parts": parts, "seed": args.seed, "parallelism": f"replicas x{ws}",
-                   "l2": "no flush: every step touches ~5 GB, above the 126 MB L2"},
+        "config": workload_config(parts, args.seed, ws),
         "parts_ms_per_step": {p: part_s[p] / args.steps * 1e3 for p in parts},
         "parts_share": shares,
         "gpu_launches": args.steps * sum(LAUNCHES[p] for p in parts),

@@ -365,6 +365,16 @@ NV4_API nv4_status nv4_hadamard_nvfp4_quant(const void* x, int64_t rows, int64_t
  */
 NV4_API nv4_status nv4_selftest(uint32_t* d_out, void* stream);
 
+/* ---------------------------------------------------------------------------
+ * nv4_selftest_wait -- exercises the bounded wait that every pipeline kernel uses (no
+ * kernel of this library waits without a time limit): one thread polls the device word
+ * *d_flag until it is non-zero or limit_ns (<= 2 s, the kernels' own limit; NV4_ERR_LIMIT
+ * beyond) of GPU time has passed.  d_status[0] = 0 if the flag was seen, NV4_FLAG_TIMEOUT
+ * if the wait gave up; d_status[1] = microseconds waited.  The kernel always returns.
+ * Not a paper operation: the failure-detection path, testable without any fault.
+ */
+NV4_API nv4_status nv4_selftest_wait(const uint32_t* d_flag, uint64_t limit_ns, uint32_t* d_status, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

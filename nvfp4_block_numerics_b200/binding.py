@@ -19,7 +19,7 @@ import torch
 from .build import LIB_PATH
 
 __all__ = [
-    "NV4Error", "lib", "nv4_tensor_amax", "nv4_act_quant", "nv4_weight_quant_rtn", "nv4_fake_qdq",
+    "NV4Error", "lib", "nv4_selftest_wait", "nv4_tensor_amax", "nv4_act_quant", "nv4_weight_quant_rtn", "nv4_fake_qdq",
     "nv4_dequant", "nv4_hessian_accum", "weight_quant_rtn", "fake_qdq", "nv4_mma_scale_bytes",
     "nv4_scales_to_mma_layout", "nv4_gemm_nvfp4", "mma_scales", "gemm_nvfp4", "nv4_mxfp4_quant",
     "nv4_mxfp4_dequant", "nv4_fp8_quant", "nv4_fp8_dequant", "mxfp4_quant", "fp8_quant", "nv4_hadamard_amax",
@@ -67,6 +67,7 @@ _SIGS = {
     "nv4_fake_qdq": (C.c_int, [_vp, _i64, _i64, _i64, _vp, C.c_int, _vp, _i64, _vp, _vp, _vp]),
     "nv4_dequant": (C.c_int, [_vp, _vp, _vp, _i64, _i64, C.c_int, _vp, _vp]),
     "nv4_mma_scale_bytes": (C.c_size_t, [_i64, _i64]),
+    "nv4_selftest_wait": (C.c_int, [_vp, C.c_uint64, _vp, _vp]),
     "nv4_mxfp4_quant": (C.c_int, [_vp, C.c_int, _i64, _i64, _i64, _vp, _vp, _vp, _vp]),
     "nv4_mxfp4_dequant": (C.c_int, [_vp, _vp, _i64, _i64, C.c_int, _vp, _vp]),
     "nv4_fp8_quant": (C.c_int, [_vp, C.c_int, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp]),
@@ -277,6 +278,12 @@ def nv4_mxfp4_to_nvfp4_batched(jobs: list[dict], d_counts=None, d_flags=None, st
     arr = (CastJob * len(jobs))(*[_cjob(**j) for j in jobs])
     _check(lib().nv4_mxfp4_to_nvfp4_batched(arr, len(jobs), _ptr(d_counts), _ptr(d_flags), _stream(stream)),
            "nv4_mxfp4_to_nvfp4_batched")
+
+
+def nv4_selftest_wait(flag: torch.Tensor, limit_ns: int, status: torch.Tensor, stream=None):
+    if flag.dtype != torch.int32 or status.dtype != torch.int32 or status.numel() < 2:
+        raise NV4Error("flag and status must be int32 CUDA tensors (status of at least 2 elements)")
+    _check(lib().nv4_selftest_wait(_ptr(flag), int(limit_ns), _ptr(status), _stream(stream)), "nv4_selftest_wait")
 
 
 def nv4_selftest(out: torch.Tensor, stream=None):

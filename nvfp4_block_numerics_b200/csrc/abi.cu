@@ -74,6 +74,30 @@ cudaError_t launch_selftest(uint32_t* d_out, cudaStream_t s)
     return cudaGetLastError();
 }
 
+// The bounded wait every pipeline kernel uses, exercised alone: thread 0 polls *flag
+// until it is non-zero or limit_ns of %globaltimer time has passed, then reports which.
+__global__ void wait_selftest_kernel(const volatile uint32_t* flag, uint64_t limit_ns, uint32_t* status)
+{
+    if (threadIdx.x != 0) return;
+    const uint64_t t0 = global_ns();
+    uint32_t st = kFlagTimeout;
+    while (global_ns() - t0 <= limit_ns) {
+        if (*flag != 0u) {
+            st = 0u;
+            break;
+        }
+        __nanosleep(1000);
+    }
+    status[0] = st;
+    status[1] = (uint32_t)((global_ns() - t0) / 1000u);   // microseconds waited
+}
+
+cudaError_t launch_wait_selftest(const uint32_t* flag, uint64_t limit_ns, uint32_t* status, cudaStream_t s)
+{
+    wait_selftest_kernel<<<1, 32, 0, s>>>(flag, limit_ns, status);
+    return cudaGetLastError();
+}
+
 }  // namespace nv4
 
 using namespace nv4;
@@ -283,6 +307,13 @@ nv4_status nv4_selftest(uint32_t* d_out, void* stream)
 {
     if (d_out == nullptr) return NV4_ERR_NULL;
     return from_cuda(launch_selftest(d_out, (cudaStream_t)stream));
+}
+
+nv4_status nv4_selftest_wait(const uint32_t* d_flag, uint64_t limit_ns, uint32_t* d_status, void* stream)
+{
+    if (d_flag == nullptr || d_status == nullptr) return NV4_ERR_NULL;
+    if (limit_ns > kWaitLimitNs) return NV4_ERR_LIMIT;
+    return from_cuda(launch_wait_selftest(d_flag, limit_ns, d_status, (cudaStream_t)stream));
 }
 
 }  // extern "C"

@@ -11,8 +11,9 @@
 // the hardware's round-to-nearest-even FP4/FP8 conversion.  Rounding to a grid is
 // monotone, so when both ends give the same code that code is the exact answer.
 // When they differ (the quotient sits within ~2^-20 relative of a rounding
-// boundary) the code is decided again by exact FP64 comparisons of the numerator
-// with boundary*divisor, products that are exact in FP64 for these operand widths.
+// boundary) one exact FP32 comparison decides: fma(boundary, divisor, -numerator)
+// rounds the exact difference once, so its sign is exact (see the fix-ups below).
+// Divisors outside [2^-100, 2^100] take exact FP64 comparisons instead.
 #pragma once
 
 #include <cstdint>

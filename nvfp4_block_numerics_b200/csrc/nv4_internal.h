@@ -51,6 +51,7 @@ cudaError_t launch_fp8_dequant(const uint8_t* q, const float* d_scale, int64_t r
 cudaError_t launch_hadamard_quant(int mode, const void* x, int64_t rows, int64_t cols, int64_t ld, int n,
                                   float* d_amax, uint8_t* q, uint8_t* sc, float* d_s2, uint32_t* d_flags,
                                   cudaStream_t s);
+cudaError_t launch_wait_selftest(const uint32_t* flag, uint64_t limit_ns, uint32_t* status, cudaStream_t s);
 size_t mma_scale_bytes(int64_t rows, int64_t kb);
 cudaError_t launch_mma_scale_layout(const uint8_t* sc, int64_t rows, int64_t kb, uint8_t* out, cudaStream_t s);
 cudaError_t launch_gemm_nvfp4(const uint8_t* qa, const uint8_t* sfa, const float* d_s2a, const uint8_t* qb,

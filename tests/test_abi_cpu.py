@@ -31,7 +31,7 @@ def test_header_declares_the_hot_path():
               "nv4_mxfp4_to_nvfp4", "nv4_weight_quant_rtn", "nv4_fake_qdq", "nv4_gemm_nvfp4",
               "nv4_scales_to_mma_layout", "nv4_mma_scale_bytes", "nv4_mxfp4_quant", "nv4_mxfp4_dequant",
               "nv4_fp8_quant", "nv4_fp8_dequant", "nv4_hadamard_amax", "nv4_hadamard_mxfp4_quant",
-              "nv4_hadamard_nvfp4_quant"):
+              "nv4_hadamard_nvfp4_quant", "nv4_selftest_wait"):
         assert n in names
 
 
@@ -102,6 +102,8 @@ def test_validation_rejects_before_any_launch(nv4lib):
     assert L.nv4_fp8_quant(fake, 0, 4, 32, 32, None, fake, fake, None, None) == 1    # amax
     assert L.nv4_fp8_quant(fake, 0, 4, 32, 32, fake, fake + 4, fake, None, None) == 3
     assert L.nv4_fp8_dequant(fake, fake, 4, 32, 9, fake, None) == 4
+    assert L.nv4_selftest_wait(fake, 3_000_000_000, fake, None) == 6                 # above the kernels' 2 s limit
+    assert L.nv4_selftest_wait(None, 1000, fake, None) == 1
     # block Hadamard + FP4
     assert L.nv4_hadamard_mxfp4_quant(fake, 4, 128, 128, 8, fake, fake, None, None) == 2    # n not in 16..128
     assert L.nv4_hadamard_mxfp4_quant(fake, 4, 96, 96, 32, fake, fake, None, None) == 2     # cols % 128

@@ -601,3 +601,24 @@ def test_cast_expert_checkpoint_full(orc):
     tot = _cast_check(orc, mats)
     print("cast counts (in-window, fallback, lossless):", tot.tolist(), "lossless fraction", tot[2] / (tot[0] + tot[1]))
     _cast_check(orc, mats, in_place=True)
+
+
+# ------------------------------------------------------------------ failure detection
+def test_bounded_wait_gives_up_and_reports():
+    """The bounded-wait path, without any fault: a flag nothing sets makes the wait run
+    out (status NV4_FLAG_TIMEOUT after about the limit) and the device stays usable; a
+    set flag ends the wait at once."""
+    flag = torch.zeros(1, dtype=torch.int32, device=G.DEV)
+    status = torch.full((2,), -1, dtype=torch.int32, device=G.DEV)
+    nv4.nv4_selftest_wait(flag, 20_000_000, status)            # 20 ms
+    torch.cuda.synchronize()
+    st = status.cpu().tolist()
+    assert st[0] == nv4.FLAG_TIMEOUT and 19_000 <= st[1] <= 2_000_000, st
+    flag.fill_(1)
+    nv4.nv4_selftest_wait(flag, 20_000_000, status)
+    torch.cuda.synchronize()
+    st = status.cpu().tolist()
+    assert st[0] == 0 and st[1] < 10_000, st
+    # the context still works afterwards
+    x = torch.ones(4, 16, dtype=torch.bfloat16, device=G.DEV)
+    assert nv4.tensor_amax(x).item() == 1.0

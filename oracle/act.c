@@ -18,7 +18,7 @@
  *            S = s_b*s2; DQ2 multiplies each FP4 value by S and emits the high-precision
  *            type (BF16 by default, FP16 optional, [FLOW] 3.6).
  *
- * Readings where the pages are silent (listed in the design doc):
+ * Readings where the pages are silent:
  *  - s2 is amax/2688 rounded once to FP32; a zero amax gives s2 = 0 and all-zero blocks.
  *  - the block scale is the nearest E4M3 value to the exact block_amax/(6*s2), ties to
  *    the even code, saturating at 448 (a calibrated amax below the live data saturates).

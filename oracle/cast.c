@@ -11,7 +11,7 @@
  * [DSPARK] stage 3: the E2M1 nibbles are reused unchanged and the scale bytes double
  * (32-element E8M0 -> 16-element E4M3).
  *
- * Readings:
+ * Readings where the pages are silent:
  *  - k_j is the unbiased exponent code-127; k_max is the maximum over one matrix.
  *  - an E8M0 code 0xFF (NaN) is rejected (flag) and never reaches the cast.
  *  - "w_block" in the fallback is the 16-element NVFP4 block of dequantized values

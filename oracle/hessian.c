@@ -5,7 +5,7 @@
  * again and, at every layer input, accumulate H = sum X^T X per block of 16 channels.
  * Block b covers channels 16b..16b+15, so H_b[i][j] = sum_t x[t][16b+i] * x[t][16b+j].
  *
- * Readings: a plain sum over tokens (not a mean; the sweep's argmin does
+ * Reading where the page is silent: a plain sum over tokens (not a mean; the sweep's argmin does
  * not change under a positive scale), no damping term, and X is whatever the caller
  * passes.  Accumulation (+=) lets calibration run over many token batches.
  *

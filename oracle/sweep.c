@@ -14,9 +14,9 @@
  *     cost = sum_i sum_j e_i H[i][j] e_j
  * The winner is the smallest cost, ties to the lowest code.
  *
- * Readings:
- *  - candidates are the 127 finite non-negative codes 0x00..0x7E; the page's "all 128
- *    values" counts the 7-bit code space whose last point 0x7F is NaN;
+ * Readings where the pages are silent:
+ *  - candidates are the 127 finite non-negative codes 0x00..0x7E; the page's count of
+ *    128 values is the 7-bit code space, whose last point 0x7F is NaN;
  *  - code 0 (S = 0, an all-zero block) is a candidate; nothing is clipped;
  *  - e uses the exact product e2m1*S_c (FP64); it is exact whenever w_i and the product
  *    lie within 2^26 of each other in magnitude, and otherwise off by at most 2^-53

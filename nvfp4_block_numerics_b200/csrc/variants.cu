@@ -165,42 +165,46 @@ static __device__ __noinline__ uint32_t e4m3_div_exact(float a, float s)
     return lo;
 }
 
-// Codes of 16 elements against s (bracket r_lo <= 1/s <= r_hi); exact when the two ends agree.
+// Exact E4M3 code (sign kept) of x / s when the bracket ends gave codes lo and hi for |x|.
+__device__ __forceinline__ uint32_t fp8_fix(float x, float s, uint32_t lo, uint32_t hi)
+{
+    const uint32_t sign = lo & 0x80u;
+    uint32_t c = min(lo & 0x7Fu, hi & 0x7Fu);                     // the bracket's lower magnitude code
+    if ((lo & 0x7Fu) != (hi & 0x7Fu)) {                           // adjacent codes: one exact comparison
+        const float mid = 0.5f * (e4m3_value(c) + e4m3_value(c + 1u));
+        const float d = fmaf(mid, s, -fabsf(x));
+        c = d < 0.0f ? c + 1u : (d > 0.0f ? c : c + (c & 1u));
+    }
+    return sign | c;
+}
+
+// Codes of 16 elements against s (bracket r_lo <= 1/s <= r_hi).  The hardware conversion
+// keeps the sign, so signed products convert directly; a pair is exact when both ends of
+// the bracket agree on both codes.
 __device__ __forceinline__ void fp8_codes16(const float v[16], float s, float r_lo, float r_hi, int mode,
                                             uint32_t out[4])
 {
 #pragma unroll
     for (int w = 0; w < 4; ++w) {
-        uint32_t word = 0u;
+        uint32_t half[2];
 #pragma unroll
-        for (int i = 0; i < 4; i += 2) {
-            const float a0 = fabsf(v[4 * w + i]), a1 = fabsf(v[4 * w + i + 1]);
-            uint32_t c0, c1;
-            if (mode == 0) {                                       // s == 0: sign only
-                c0 = c1 = 0u;
-            } else if (mode == 1) {
-                const uint32_t lo = cvt_e4m3x2(a0 * r_lo, a1 * r_lo), hi = cvt_e4m3x2(a0 * r_hi, a1 * r_hi);
-                c0 = lo & 0xFFu;
-                c1 = lo >> 8;
-                if (c0 != (hi & 0xFFu)) {                          // one exact comparison with the midpoint
-                    const float mid = 0.5f * (e4m3_value(c0) + e4m3_value(c0 + 1u));
-                    const float d = fmaf(mid, s, -a0);
-                    c0 = d < 0.0f ? c0 + 1u : (d > 0.0f ? c0 : c0 + (c0 & 1u));
-                }
-                if (c1 != (hi >> 8)) {
-                    const float mid = 0.5f * (e4m3_value(c1) + e4m3_value(c1 + 1u));
-                    const float d = fmaf(mid, s, -a1);
-                    c1 = d < 0.0f ? c1 + 1u : (d > 0.0f ? c1 : c1 + (c1 & 1u));
-                }
+        for (int h = 0; h < 2; ++h) {
+            const float x0 = v[4 * w + 2 * h], x1 = v[4 * w + 2 * h + 1];
+            if (mode == 1) {
+                const float2 pl = __fmul2_rn(make_float2(x0, x1), make_float2(r_lo, r_lo));
+                const float2 ph = __fmul2_rn(make_float2(x0, x1), make_float2(r_hi, r_hi));
+                const uint32_t lo = cvt_e4m3x2(pl.x, pl.y), hi = cvt_e4m3x2(ph.x, ph.y);
+                half[h] = lo;
+                if (lo != hi)
+                    half[h] = fp8_fix(x0, s, lo & 0xFFu, hi & 0xFFu) | (fp8_fix(x1, s, lo >> 8, hi >> 8) << 8);
             } else {
-                c0 = e4m3_div_exact(a0, s);
-                c1 = e4m3_div_exact(a1, s);
+                const uint32_t s0 = (__float_as_uint(x0) >> 24) & 0x80u, s1 = (__float_as_uint(x1) >> 24) & 0x80u;
+                const uint32_t c0 = mode == 0 ? 0u : e4m3_div_exact(fabsf(x0), s);
+                const uint32_t c1 = mode == 0 ? 0u : e4m3_div_exact(fabsf(x1), s);
+                half[h] = (s0 | c0) | ((s1 | c1) << 8);
             }
-            c0 |= (__float_as_uint(v[4 * w + i]) >> 24) & 0x80u;
-            c1 |= (__float_as_uint(v[4 * w + i + 1]) >> 24) & 0x80u;
-            word |= (c0 | (c1 << 8)) << (8 * i);
         }
-        out[w] = word;
+        out[w] = half[0] | (half[1] << 16);
     }
 }
 
@@ -217,11 +221,53 @@ fp8_quant_kernel(const void* x, uint32_t rows, uint32_t groups_per_row, int64_t 
     const float r_lo = __fmul_rn(r, kLoMargin), r_hi = __fmul_rn(r, kHiMargin);
     uint32_t flags = isfinite(s) ? 0u : kFlagOverflow;
     const uint32_t total = rows * groups_per_row;
-    for (uint32_t g = blockIdx.x * kVarThreads + threadIdx.x; g < total; g += gridDim.x * kVarThreads) {
+    const uint32_t stride = gridDim.x * kVarThreads;
+    // the next group's loads are in flight while this one is converted
+    auto offset = [&](uint32_t g) {
+        const uint32_t row = div_gpr.div(g);
+        return (int64_t)row * ld + 16 * (int64_t)(g - row * groups_per_row);
+    };
+    constexpr int kWords = kIn == 0 ? 2 : 4;
+    uint4 nxt[kWords];
+    uint32_t g = blockIdx.x * kVarThreads + threadIdx.x;
+    if (g < total) {
+        const uint4* src = reinterpret_cast<const uint4*>(static_cast<const char*>(x) + offset(g) * (kIn == 0 ? 2 : 4));
+#pragma unroll
+        for (int k = 0; k < kWords; ++k) nxt[k] = __ldcs(src + k);
+    }
+    for (; g < total; g += stride) {
         const uint32_t row = div_gpr.div(g), gg = g - row * groups_per_row;
+        uint4 cur[kWords];
+#pragma unroll
+        for (int k = 0; k < kWords; ++k) cur[k] = nxt[k];
+        if (g + stride < total) {
+            const uint4* src = reinterpret_cast<const uint4*>(static_cast<const char*>(x) + offset(g + stride) * (kIn == 0 ? 2 : 4));
+#pragma unroll
+            for (int k = 0; k < kWords; ++k) nxt[k] = __ldcs(src + k);
+        }
         float v[16];
-        uint32_t ab;
-        load16<kIn>(x, (int64_t)row * ld + 16 * (int64_t)gg, v, ab);
+        uint32_t ab = 0u;
+        if constexpr (kIn == 0) {
+            const uint32_t w[8] = {cur[0].x, cur[0].y, cur[0].z, cur[0].w, cur[1].x, cur[1].y, cur[1].z, cur[1].w};
+            uint32_t m = 0u;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                m = __vmaxu2(m, w[j] & 0x7FFF7FFFu);
+                v[2 * j] = bf16_lo(w[j]);
+                v[2 * j + 1] = bf16_hi(w[j]);
+            }
+            ab = max(m & 0xFFFFu, m >> 16) << 16;
+        } else {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const uint32_t w[4] = {cur[k].x, cur[k].y, cur[k].z, cur[k].w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    ab = max(ab, w[j] & 0x7FFFFFFFu);
+                    v[4 * k + j] = __uint_as_float(w[j]);
+                }
+            }
+        }
         if (ab >= 0x7F800000u) flags |= kFlagNonFinite;
         uint32_t w[4];
         fp8_codes16(v, s, r_lo, r_hi, mode, w);

@@ -11,18 +11,19 @@
 //     matrix, or a group of matrices sharing one scale_2, [CAST] section 3) reads only
 //     the E8M0 bytes, reduces the largest valid code through distributed shared memory
 //     and writes every member's outputs s2 = 2^m and global_amax = 6*448*2^m;
-//  2. cast_rewrite_kernel: a flat grid over the MX blocks of every matrix (a warp takes
-//     256 consecutive blocks per step, lane-interleaved so each instruction moves
-//     contiguous bytes) recovers k_max = m + 8 exactly from the s2 it reads back, writes
-//     the two E4M3 scale bytes per block and, out of place, copies the 16 nibble bytes
-//     with 128-bit streaming loads and stores; rare blocks (NaN code, outside the
-//     window) take a separate exact path.
+//  2. cast_rewrite_kernel: one resident wave of warps striding over 256-block tiles
+//     (lane-interleaved so each instruction moves contiguous bytes).  It recovers k_max
+//     = m + 8 exactly from the s2 it reads back, writes the two E4M3 scale bytes per
+//     block and, out of place, copies the 16 nibble bytes with 128-bit streaming loads
+//     and stores; rare blocks (NaN code, outside the window) take a separate exact
+//     path.  Launched as a programmatic dependent of kernel 1, it copies the nibbles of
+//     each warp's first tiles while kernel 1 runs, then waits for kernel 1.
 #include "nv4_common.cuh"
 #include "nv4_internal.h"
 
 namespace nv4 {
 
-constexpr int kCastThreads = 256;
+constexpr int kKmaxThreads = 512;
 constexpr int kKmaxCluster = 8;                  // CTAs reducing one matrix's largest E8M0 code
 
 struct CastJobDev {
@@ -33,7 +34,7 @@ struct CastJobDev {
     float* d_ga;
     float* d_s2;
     uint32_t nb;                                  // MX blocks in the matrix (rows * cols / 32)
-    uint32_t group_begin;                         // prefix sum of 256-block tiles over jobs
+    uint32_t chunk_begin;                         // prefix sum of kTile-block tiles over jobs
 };
 
 struct CastParams {
@@ -41,7 +42,7 @@ struct CastParams {
     int n_sets;                                   // scale_2 groups (sets of jobs sharing k_max)
     uint16_t set_begin[kMaxCastJobs + 1];         // members of set g: set_jobs[set_begin[g] .. set_begin[g+1])
     uint16_t set_jobs[kMaxCastJobs];
-    uint32_t groups;                              // total 256-block tiles
+    uint32_t chunks;                              // total kTile-block tiles over all jobs
     unsigned long long* d_counts;
     uint32_t* d_flags;
     CastJobDev jobs[kMaxCastJobs];
@@ -91,63 +92,94 @@ __device__ __forceinline__ float e2m1_times_pow2(uint32_t c, int k)
     return (c & 8u) ? -r : r;
 }
 
-// Re-quantizes one 16-element half of an MX block outside the window.  Returns the
-// E4M3 code, writes the packed nibbles to out[2], and sets *lossless.
-__device__ __noinline__ uint32_t cast_fallback16(const uint32_t nib_words[2], int k, float s2,
-                                                 uint32_t out[2], uint32_t* lossless)
+// Packed E2M1 codes of lo (bits 0-3) and hi (bits 4-7): RNE, saturating at 6, sign kept.
+__device__ __forceinline__ uint32_t cvt_e2m1x2(float lo, float hi)
 {
-    float w[16];
-    float a_b = 0.0f;
-    for (int i = 0; i < 16; ++i) {
-        w[i] = e2m1_times_pow2((nib_words[i >> 3] >> (4 * (i & 7))) & 15u, k);
-        a_b = fmaxf(a_b, fabsf(w[i]));
-    }
-    const uint32_t code = e4m3_code_exact(a_b, s2);
-    const float S = __fmul_rn(e4m3_value(code), s2);
-    out[0] = out[1] = 0u;
-    uint32_t same = 1u;
-    for (int i = 0; i < 16; ++i) {
-        const uint32_t c = e2m1_code_exact(w[i], S);
-        out[i >> 3] |= c << (4 * (i & 7));
-        const uint32_t mag = c & 7u;
-        const float v = mag < 2u ? 0.5f * (float)mag
-                                 : __uint_as_float(((126u + (mag >> 1)) << 23) | ((mag & 1u) << 22));
-        const float y = __fmul_rn((c & 8u) ? -v : v, S);
-        if (__float_as_uint(y) != __float_as_uint(w[i])) same = 0u;
-    }
-    *lossless = same;
-    return code;
+    uint32_t r;
+    asm("{\n\t.reg .b8 b;\n\tcvt.rn.satfinite.e2m1x2.f32 b, %2, %1;\n\tcvt.u32.u8 %0, b;\n\t}"
+        : "=r"(r)
+        : "f"(lo), "f"(hi));
+    return r;
 }
 
-// A block whose E8M0 code is NaN (nibbles copied, scales 0; flagged in phase 1) or lies
-// outside the window (re-quantized).  Returns the two scale bytes; adds to the fallback
-// and lossless counters.
-__device__ __noinline__ uint32_t cast_rare_block(const uint8_t* __restrict__ mx_q, uint8_t* __restrict__ nv_q,
-                                                 uint32_t g, uint32_t c, int k_max, float s2, bool copy,
-                                                 uint32_t* n_fb, uint32_t* n_ll)
+// One rare MX block g (E8M0 code c; arguments warp-uniform), handled by the whole warp:
+// lanes 0-15 take the first 16-element half, lanes 16-31 the second, one element per
+// lane.  A NaN code copies the nibbles (out of place) and writes zero scales.  Otherwise
+// each half is re-quantized from its exact values e2m1 * 2^k with the activation-
+// quantizer rules: block amax a_b, scale code = nearest E4M3 to a_b/(6*s2), codes =
+// nearest E2M1 to w/S with S = RN32(s_b * s2).  Both roundings take the FP32 bracket
+// (hardware conversion of both ends, an exact FMA comparison when they disagree);
+// scales outside [2^-100, 2^100] take the exact FP64 encoders.  Every lane reads its
+// source byte before any lane writes, so nv_q may equal mx_q.
+__device__ __noinline__ void cast_rare_warp(const uint8_t* mx_q, uint8_t* nv_q, uint8_t* nv_scales, uint32_t g,
+                                            uint32_t c, float s2, bool copy, uint32_t lane, uint32_t* n_fb,
+                                            uint32_t* n_ll)
 {
-    const uint4 qv = *reinterpret_cast<const uint4*>(mx_q + (int64_t)g * 16);
+    const uint32_t h = lane >> 4, e = lane & 15u;
+    const size_t at = (size_t)16 * g + 8u * h + (e >> 1);
+    const uint32_t byte = mx_q[at];
     if (c == 0xFFu) {
-        if (copy) *reinterpret_cast<uint4*>(nv_q + (int64_t)g * 16) = qv;
-        return 0u;
+        if (copy && (e & 1u) == 0u) nv_q[at] = (uint8_t)byte;
+        if (lane == 0u) reinterpret_cast<uint16_t*>(nv_scales)[g] = 0;
+        return;
     }
-    const int k = (int)c - 127;
-    const uint32_t lo_words[2] = {qv.x, qv.y}, hi_words[2] = {qv.z, qv.w};
-    uint32_t out_lo[2], out_hi[2], ll0, ll1;
-    const uint32_t s_lo = cast_fallback16(lo_words, k, s2, out_lo, &ll0);
-    const uint32_t s_hi = cast_fallback16(hi_words, k, s2, out_hi, &ll1);
-    *reinterpret_cast<uint4*>(nv_q + (int64_t)g * 16) = make_uint4(out_lo[0], out_lo[1], out_hi[0], out_hi[1]);
-    *n_fb += 2u;
-    *n_ll += ll0 + ll1;
-    return s_lo | (s_hi << 8);
+    const float w = e2m1_times_pow2((byte >> (4u * (e & 1u))) & 15u, (int)c - 127);
+    uint32_t ab = __float_as_uint(w) & 0x7FFFFFFFu;
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) ab = max(ab, __shfl_xor_sync(0xFFFFFFFFu, ab, o));   // within the half
+    const float a_b = __uint_as_float(ab);
+
+    uint32_t code;                                              // nearest E4M3 to a_b / (6*s2)
+    if (s2 >= kTinyScale && s2 <= 0x1p100f) {
+        const float kk = __frcp_rn(__fmul_rn(6.0f, s2));
+        const uint32_t cc = cvt_e4m3x2(__fmul_rn(a_b, __fmul_rn(kk, kLoMargin)), __fmul_rn(a_b, __fmul_rn(kk, kHiMargin)));
+        code = cc & 0xFFu;
+        if (code != (cc >> 8)) code = e4m3_fix(code, a_b, s2);
+        code &= 0x7Fu;
+    } else {
+        code = e4m3_code_exact(a_b, s2);
+    }
+    const float S = __fmul_rn(e4m3_value(code), s2);           // DQ1: RN32(s_b * s2)
+
+    uint32_t q;                                                 // nearest E2M1 to w / S
+    if (S == 0.0f) {
+        q = (__float_as_uint(w) >> 28) & 8u;                    // sign only
+    } else if (S >= kTinyScale && S <= 0x1p100f) {
+        const float r = __frcp_rn(S);
+        const uint32_t cc = cvt_e2m1x2(__fmul_rn(w, __fmul_rn(r, kLoMargin)), __fmul_rn(w, __fmul_rn(r, kHiMargin)));
+        q = cc & 15u;
+        if (q != (cc >> 4)) {                                   // near a rounding boundary
+            const uint32_t kl = q & 7u;
+            const float d = fmaf(e2m1_boundary(kl), S, -fabsf(w));
+            const uint32_t k = d < 0.0f ? kl + 1u : (d > 0.0f ? kl : kl + (kl & 1u));
+            q = k | (q & 8u);
+        }
+    } else {
+        q = e2m1_code_exact(w, S);
+    }
+    // lossless: the NVFP4 value of every element equals its MXFP4 value
+    const uint32_t mag = q & 7u;
+    const float v = mag < 2u ? 0.5f * (float)mag : __uint_as_float(((126u + (mag >> 1)) << 23) | ((mag & 1u) << 22));
+    const float y = __fmul_rn((q & 8u) ? -v : v, S);
+    const uint32_t same = __ballot_sync(0xFFFFFFFFu, __float_as_uint(y) == __float_as_uint(w));
+    const uint32_t partner = __shfl_xor_sync(0xFFFFFFFFu, q, 1);
+    if ((e & 1u) == 0u) nv_q[at] = (uint8_t)(q | (partner << 4));
+    if (e == 0u) nv_scales[(size_t)2 * g + h] = (uint8_t)code;
+    if (lane == 0u) {
+        *n_fb += 2u;
+        *n_ll += ((same & 0xFFFFu) == 0xFFFFu ? 1u : 0u) + ((same >> 16) == 0xFFFFu ? 1u : 0u);
+    }
 }
 
 // ------------------------------------------------------------------ kernel 1: k_max
-__global__ void __launch_bounds__(kCastThreads)
+__global__ void __launch_bounds__(kKmaxThreads)
 cast_kmax_kernel(const __grid_constant__ CastParams p)
 {
-    __shared__ uint32_t red[kCastThreads / 32];
+    __shared__ uint32_t red[kKmaxThreads / 32];
     __shared__ uint32_t cta_max;
+    // the rewrite kernel may start its set-up and first loads now; it waits for this
+    // grid to complete before it reads scale_2
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const uint32_t rank = cluster_rank_c();
     const int set = blockIdx.x / kKmaxCluster;
     const int m0 = p.set_begin[set], m1 = p.set_begin[set + 1];
@@ -172,15 +204,15 @@ cast_kmax_kernel(const __grid_constant__ CastParams p)
         const uint32_t nvec = (g1 - g0) / 16u;
         const uint4* src = reinterpret_cast<const uint4*>(job.e8m0 + g0);
         uint32_t v = threadIdx.x;
-        for (; v + 3u * kCastThreads < nvec; v += 4u * kCastThreads) {  // four loads in flight
+        for (; v + 3u * kKmaxThreads < nvec; v += 4u * kKmaxThreads) {  // four loads in flight
             uint4 w[4];
 #pragma unroll
-            for (int k = 0; k < 4; ++k) w[k] = __ldcs(src + v + k * kCastThreads);
+            for (int k = 0; k < 4; ++k) w[k] = __ldcs(src + v + k * kKmaxThreads);
 #pragma unroll
             for (int k = 0; k < 4; ++k) scan(w[k]);
         }
-        for (; v < nvec; v += kCastThreads) scan(__ldcs(src + v));
-        for (uint32_t g = g0 + nvec * 16u + threadIdx.x; g < g1; g += kCastThreads) {
+        for (; v < nvec; v += kKmaxThreads) scan(__ldcs(src + v));
+        for (uint32_t g = g0 + nvec * 16u + threadIdx.x; g < g1; g += kKmaxThreads) {
             const uint32_t c = job.e8m0[g];
             if (c == 0xFFu) flags |= kFlagE8M0Nan; else mtail = max(mtail, c);
         }
@@ -191,7 +223,7 @@ cast_kmax_kernel(const __grid_constant__ CastParams p)
     __syncthreads();
     if (threadIdx.x == 0) {
         uint32_t m = 0u;
-        for (int w = 0; w < kCastThreads / 32; ++w) m = max(m, red[w]);
+        for (int w = 0; w < kKmaxThreads / 32; ++w) m = max(m, red[w]);
         cta_max = m;
     }
     cluster_sync_c();
@@ -221,33 +253,68 @@ __device__ __forceinline__ int exact_log2(float s2)
 }
 
 // ------------------------------------------------------------------ kernel 2: rewrite
-// A warp step covers a tile of 256 consecutive MX blocks of one matrix: lane t takes
-// blocks tile + 32i + t (i = 0..7), so every load and store instruction of the warp
-// moves contiguous bytes (32 code bytes, 512 nibble bytes, 64 scale bytes).
+// A tile is kTile consecutive MX blocks of one matrix; lane t of a warp takes blocks
+// tile + 32i + t (i = 0..7), so every load and store instruction of the warp moves
+// contiguous bytes (32 code bytes, 512 nibble bytes, 64 scale bytes).  Warps stride over
+// the tiles (warp w takes tiles w, w + W, ...), so at any moment the grid sweeps one
+// region of memory.  The nibble copy of a warp's first kPreTiles tiles needs nothing
+// from kernel 1: under programmatic dependent launch it runs while kernel 1 is still
+// reducing k_max, and the main pass then only writes those tiles' scale bytes.
 constexpr uint32_t kTile = 256;
+constexpr int kRwThreads = 256;
+constexpr int kRwCtasPerSm = 2;
+constexpr uint32_t kPreTiles = 3;
 
-__global__ void __launch_bounds__(kCastThreads)
+// The job holding global tile ti (jobs are ordered by their first tile).
+__device__ __forceinline__ int cast_job_of(const CastParams& p, uint32_t ti)
+{
+    int lo = 0, hi = p.n - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (p.jobs[mid].chunk_begin <= ti) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+}
+
+__global__ void __launch_bounds__(kRwThreads, kRwCtasPerSm)
 cast_rewrite_kernel(const __grid_constant__ CastParams p)
 {
     const uint32_t lane = threadIdx.x & 31u;
-    const uint32_t warp_id = (blockIdx.x * kCastThreads + threadIdx.x) >> 5;
-    const uint32_t nwarps = (gridDim.x * kCastThreads) >> 5;
-    uint32_t n_in = 0u, n_fb = 0u, n_ll = 0u;
-    for (uint32_t ti = warp_id; ti < p.groups; ti += nwarps) {      // p.groups counts 256-block tiles here
-        int j = 0;
-        {
-            int lo = 0, hi = p.n - 1;
-            while (lo < hi) {
-                const int mid = (lo + hi + 1) >> 1;
-                if (p.jobs[mid].group_begin <= ti) lo = mid; else hi = mid - 1;
+    const uint32_t warp_id = (blockIdx.x * kRwThreads + threadIdx.x) >> 5;
+    const uint32_t nwarps = (gridDim.x * kRwThreads) >> 5;
+
+    // ---- nibble copy of the first tiles (out of place), before kernel 1 has finished
+    {
+        uint32_t k = 0u;
+        for (uint32_t ti = warp_id; k < kPreTiles && ti < p.chunks; ti += nwarps, ++k) {
+            const CastJobDev& job = p.jobs[cast_job_of(p, ti)];
+            if (job.nv_q == job.mx_q) continue;
+            const uint32_t base = kTile * (ti - job.chunk_begin);
+            uint4 qv[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const uint32_t g = base + 32u * i + lane;
+                if (g < job.nb) qv[i] = __ldcs(reinterpret_cast<const uint4*>(job.mx_q) + g);
             }
-            j = lo;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const uint32_t g = base + 32u * i + lane;
+                if (g < job.nb) __stcs(reinterpret_cast<uint4*>(job.nv_q) + g, qv[i]);
+            }
         }
-        const CastJobDev& job = p.jobs[j];
+    }
+    // kernel 1's scale_2 values are visible from here on (a no-op without programmatic
+    // dependent launch)
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+
+    uint32_t n_in = 0u, n_fb = 0u, n_ll = 0u;
+    uint32_t k = 0u;
+    for (uint32_t ti = warp_id; ti < p.chunks; ti += nwarps, ++k) {
+        const CastJobDev& job = p.jobs[cast_job_of(p, ti)];
         const float s2 = *job.d_s2;
         const int k_max = exact_log2(s2) + 8;
-        const bool copy = job.nv_q != job.mx_q;
-        const uint32_t base = kTile * (ti - job.group_begin);
+        const bool copy = job.nv_q != job.mx_q && k >= kPreTiles;     // nibbles still to copy
+        const uint32_t base = kTile * (ti - job.chunk_begin);
         uint32_t c[8];
         uint4 qv[8];
 #pragma unroll
@@ -259,7 +326,7 @@ cast_rewrite_kernel(const __grid_constant__ CastParams p)
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
                 const uint32_t g = base + 32u * i + lane;
-                if (g < job.nb) qv[i] = __ldcs(reinterpret_cast<const uint4*>(job.mx_q + (int64_t)g * 16));
+                if (g < job.nb) qv[i] = __ldcs(reinterpret_cast<const uint4*>(job.mx_q) + g);
             }
         }
         uint32_t rare = 0u;
@@ -270,21 +337,28 @@ cast_rewrite_kernel(const __grid_constant__ CastParams p)
             const int d = k_max - ((int)c[i] - 127);
             if (c[i] != 0xFFu && d <= 17) {
                 const uint32_t e = e4m3_code_pow2(8 - d);
-                __stcs(reinterpret_cast<unsigned short*>(job.nv_scales + (int64_t)g * 2), (unsigned short)(e | (e << 8)));
-                if (copy) __stcs(reinterpret_cast<uint4*>(job.nv_q + (int64_t)g * 16), qv[i]);
+                __stcs(reinterpret_cast<unsigned short*>(job.nv_scales) + g, (unsigned short)(e | (e << 8)));
+                if (copy) __stcs(reinterpret_cast<uint4*>(job.nv_q) + g, qv[i]);
                 n_in += 2u;
             } else {
                 rare |= 1u << i;
             }
         }
-        if (rare) {                                                  // after the copies: nothing else live
+        // rare blocks, one at a time by the whole warp; the warp barrier orders every
+        // lane's earlier nibble stores (a pre-copied tile) before other lanes rewrite them
+        if (__ballot_sync(0xFFFFFFFFu, rare != 0u)) {
+            __syncwarp();
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-                if (rare & (1u << i)) {
-                    const uint32_t g = base + 32u * i + lane;
-                    const uint32_t v = cast_rare_block(job.mx_q, job.nv_q, g, c[i], k_max, s2, copy, &n_fb, &n_ll);
-                    *reinterpret_cast<uint16_t*>(job.nv_scales + (int64_t)g * 2) = (uint16_t)v;
+            for (int i = 0; i < 8; ++i) {
+                uint32_t m = __ballot_sync(0xFFFFFFFFu, (rare >> i) & 1u);
+                while (m) {
+                    const uint32_t L = __ffs(m) - 1u;
+                    m &= m - 1u;
+                    const uint32_t cL = __shfl_sync(0xFFFFFFFFu, c[i], L);
+                    cast_rare_warp(job.mx_q, job.nv_q, job.nv_scales, base + 32u * i + L, cL, s2, copy, lane, &n_fb,
+                                   &n_ll);
                 }
+            }
         }
     }
     // counters: one set of atomics per warp, no CTA barrier (warps retire independently)
@@ -306,7 +380,7 @@ cudaError_t launch_cast(const nv4_cast_job* jobs, int n, unsigned long long* d_c
     p.d_counts = d_counts;
     p.d_flags = d_flags;
     int m = 0;
-    uint32_t groups = 0;
+    uint32_t chunks = 0;
     for (int i = 0; i < n; ++i) {
         const nv4_cast_job& J = jobs[i];
         if (J.rows == 0 || J.cols == 0) continue;
@@ -314,11 +388,11 @@ cudaError_t launch_cast(const nv4_cast_job* jobs, int n, unsigned long long* d_c
         d.mx_q = J.mx_q; d.e8m0 = J.e8m0; d.nv_q = J.nv_q; d.nv_scales = J.nv_scales;
         d.d_ga = J.d_global_amax; d.d_s2 = J.d_s2;
         d.nb = (uint32_t)(J.rows * (J.cols / 32));
-        d.group_begin = groups;
-        groups += (d.nb + kTile - 1u) / kTile;
+        d.chunk_begin = chunks;
+        chunks += (d.nb + kTile - 1u) / kTile;
     }
     p.n = m;
-    p.groups = groups;
+    p.chunks = chunks;
     if (m == 0) return cudaSuccess;
     // scale_2 sets: jobs with the same non-negative group id share one k_max
     {
@@ -345,7 +419,7 @@ cudaError_t launch_cast(const nv4_cast_job* jobs, int n, unsigned long long* d_c
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(p.n_sets * kKmaxCluster), 1, 1);
-    cfg.blockDim = dim3(kCastThreads, 1, 1);
+    cfg.blockDim = dim3(kKmaxThreads, 1, 1);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
@@ -358,12 +432,25 @@ cudaError_t launch_cast(const nv4_cast_job* jobs, int n, unsigned long long* d_c
     cudaError_t e = cudaLaunchKernelEx(&cfg, cast_kmax_kernel, p);
     if (e != cudaSuccess) return e;
 
-    // a single resident wave (two CTAs per SM at this kernel's register count); warps
-    // stride over the tiles
-    const int64_t need = ((int64_t)groups + kCastThreads / 32 - 1) / (kCastThreads / 32);   // one warp per tile
-    const int64_t cap = (int64_t)num_sms() * 2;
-    const int grid = (int)(need < cap ? (need > 0 ? need : 1) : cap);
-    cast_rewrite_kernel<<<grid, kCastThreads, 0, s>>>(p);
+    // a single resident wave, launched as a programmatic dependent of the k_max kernel
+    // so that its first loads overlap that kernel; it waits for the k_max results
+    // before using them
+    const uint64_t warps_needed = chunks;
+    const uint64_t cap = (uint64_t)num_sms() * kRwCtasPerSm;
+    const uint64_t need = (warps_needed + kRwThreads / 32 - 1) / (kRwThreads / 32);
+    const int grid = (int)(need < cap ? need : cap);
+    cudaLaunchConfig_t cfg2 = {};
+    cfg2.gridDim = dim3((unsigned)grid, 1, 1);
+    cfg2.blockDim = dim3(kRwThreads, 1, 1);
+    cfg2.dynamicSmemBytes = 0;
+    cfg2.stream = s;
+    cudaLaunchAttribute attr2[1];
+    attr2[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr2[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg2.attrs = attr2;
+    cfg2.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg2, cast_rewrite_kernel, p);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

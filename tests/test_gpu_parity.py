@@ -576,6 +576,29 @@ def test_cast_small_and_edges(orc):
     _cast_check(orc, mats, in_place=True)
 
 
+def test_cast_chunk_tails(orc):
+    """Matrices spanning several 2048-block chunks of the streaming kernel, with tails
+    that are not whole 16-byte words of E8M0 codes or of scale bytes, fallback blocks
+    in every chunk, and more jobs than fit one chunk each."""
+    shapes = [(4099, 32), (2049, 64), (1, 2048 * 32), (3, 683 * 32), (129, 160), (2, 4096 * 32 + 32)]
+    mats = [inputs.mxfp4_matrix(inputs.rng_for(i, "gpu", "castc"), r, c, fallback_frac=0.03)
+            for i, (r, c) in enumerate(shapes)]
+    tot = _cast_check(orc, mats)
+    assert tot[1] > 0
+    _cast_check(orc, mats, in_place=True)
+    _cast_check(orc, mats, groups=[0, 1, 0, 1, 0, 1])
+
+
+def test_cast_extreme_exponents(orc):
+    """Fallback blocks under scale_2 values far from 1: tiny exponents (s2 below 2^-100,
+    where the block-scale encoder takes its exact path) and large ones (s2 above
+    2^100, block scales near the top of FP32)."""
+    mats = [inputs.mxfp4_matrix(inputs.rng_for(i, "gpu", "castx"), 64, 256, mean_exp=m, fallback_frac=0.05)
+            for i, m in enumerate((-110.0, -100.0, 100.0, 112.0))]
+    tot = _cast_check(orc, mats)
+    assert tot[1] > 0
+
+
 def test_cast_grouped_scale2(orc):
     """Matrices sharing one scale_2: the window-edge example, random pairs whose members
     sit apart in the job list, singletons and one-member groups in the same call."""

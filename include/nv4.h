@@ -208,8 +208,10 @@ NV4_API nv4_status nv4_hessian_accum_batched(const nv4_hessian_job* jobs, int n_
  * Costs are evaluated in FP32; blocks whose best and second-best costs differ by
  * less than ~1e-6 relative may pick a different code than an exact evaluation.
  * The search is exact over all 127 codes but skips the cost of candidates that a
- * lower bound proves cannot be the winner or the runner-up (sweep.cu states the
- * bounds); the optional per-job work counter reports how many were evaluated.
+ * lower bound proves cannot be the winner or, when cost2 is requested, the runner-up
+ * (sweep.cu states the bounds): codes and q are the same with or without the cost
+ * outputs, and cheapest without cost2.  The optional per-job work counter reports
+ * how many candidates were visited and evaluated.
  */
 NV4_API nv4_status nv4_scale_sweep(const void* w, nv4_dtype dt, int64_t rows, int64_t cols, int64_t ld,
                            const float* H, const float* d_amax_w, uint8_t* codes, uint8_t* q,

@@ -92,16 +92,6 @@ __device__ __forceinline__ float e2m1_times_pow2(uint32_t c, int k)
     return (c & 8u) ? -r : r;
 }
 
-// Packed E2M1 codes of lo (bits 0-3) and hi (bits 4-7): RNE, saturating at 6, sign kept.
-__device__ __forceinline__ uint32_t cvt_e2m1x2(float lo, float hi)
-{
-    uint32_t r;
-    asm("{\n\t.reg .b8 b;\n\tcvt.rn.satfinite.e2m1x2.f32 b, %2, %1;\n\tcvt.u32.u8 %0, b;\n\t}"
-        : "=r"(r)
-        : "f"(lo), "f"(hi));
-    return r;
-}
-
 // One rare MX block g (E8M0 code c; arguments warp-uniform), handled by the whole warp:
 // lanes 0-15 take the first 16-element half, lanes 16-31 the second, one element per
 // lane.  A NaN code copies the nibbles (out of place) and writes zero scales.  Otherwise

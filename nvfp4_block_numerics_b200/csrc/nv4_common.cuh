@@ -78,6 +78,16 @@ __device__ __forceinline__ uint32_t cvt_e2m1x8(const float v[8])
     return r;
 }
 
+// Packed E2M1 codes of lo (bits 0-3) and hi (bits 4-7): RNE, saturating at 6, sign kept.
+__device__ __forceinline__ uint32_t cvt_e2m1x2(float lo, float hi)
+{
+    uint32_t r;
+    asm("{\n\t.reg .b8 b;\n\tcvt.rn.satfinite.e2m1x2.f32 b, %2, %1;\n\tcvt.u32.u8 %0, b;\n\t}"
+        : "=r"(r)
+        : "f"(lo), "f"(hi));
+    return r;
+}
+
 // Hardware decode of the 8 E2M1 codes packed in w (element k in bits 4k..4k+3)
 // to FP16 pairs: h[j] holds elements 2j (low half) and 2j+1 (high half).  E2M1
 // values are exact in FP16.

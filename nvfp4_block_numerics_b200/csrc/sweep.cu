@@ -24,10 +24,12 @@
 //   (2) Every grid point of scale S is at most 6S in magnitude, so |e_i| >= |w_i| - 6S,
 //       and the same holds at every smaller scale.
 // The winner and the runner-up cost depend only on candidates whose cost is at most
-// the running runner-up cost.  A thread starts at the max-calibrated code (nearest
-// E4M3 to amax_b / (6 s2)) and walks outwards, alternating down and up: a candidate
-// whose bound (1) exceeds the runner-up skips the quadratic form, and once bound (2)
-// over the two largest |w_i| exceeds it, the downward walk ends.  Both comparisons
+// the running runner-up cost; when the runner-up is not an output, only the winner
+// (ties to the lowest code) has to be found and the running best cost is the
+// threshold instead.  A thread starts at the max-calibrated code (nearest E4M3 to
+// amax_b / (6 s2)) and walks outwards, alternating down and up: a candidate whose
+// bound (1) exceeds the threshold skips the quadratic form, and once bound (2) over
+// the two largest |w_i| exceeds it, the downward walk ends.  Both comparisons
 // keep a relative margin of 2^-10, far above the FP32 evaluation error, so skipped
 // candidates could not have changed the FP32 result either.  When rho <= 0, or H_b
 // has a zero diagonal entry with a nonzero row, or non-finite entries, the bounds are
@@ -363,7 +365,10 @@ sweep_kernel(const __grid_constant__ SweepParams p)
             if (a > a1) { a2 = a1; d2 = d1; a1 = a; d1 = d; }
             else if (a > a2) { a2 = a; d2 = d; }
         }
-        float best = __int_as_float(0x7F800000), second = best;
+        // the threshold a candidate's lower bound must exceed to be skipped: the
+        // runner-up cost when it is an output, else the best cost
+        const bool need2 = job.cost2 != nullptr;
+        float best = __int_as_float(0x7F800000), second = best, thr = best;
         uint32_t best_c = 0u;
         if (a1 == 0.0f) {
             best = 0.0f;                  // all-zero block: every candidate has e = w = 0
@@ -383,7 +388,7 @@ sweep_kernel(const __grid_constant__ SweepParams p)
 #pragma unroll
                 for (int k = 0; k < 8; ++k) e[k] = __ffma2_rn(v[k], nS, w[k]);     // w - v*S, one rounding
                 ++nvisit;
-                if (!pr || !(bound_diag(e, rd4) * kPruneScale > second)) {
+                if (!pr || !(bound_diag(e, rd4) * kPruneScale > thr)) {
                     ++nfull;
                     const float cost = quad_form(e, hp);
                     if (cost < best || (cost == best && (uint32_t)c < best_c)) {
@@ -393,13 +398,14 @@ sweep_kernel(const __grid_constant__ SweepParams p)
                     } else if (cost > best && cost < second) {
                         second = cost;
                     }
+                    thr = need2 ? second : best;
                 }
                 // next candidate: alternate down / up; bound (2) closes the downward walk
                 bool take_dn = dn >= 0 && (go_dn || up > 126);
                 if (take_dn && pr) {
                     const float S = tab[dn].x;
                     const float u1 = fmaxf(fmaf(-6.0f, S, a1), 0.0f), u2 = fmaxf(fmaf(-6.0f, S, a2), 0.0f);
-                    if (fmaf(d1 * u1, u1, d2 * u2 * u2) * kPruneScale > second) {
+                    if (fmaf(d1 * u1, u1, d2 * u2 * u2) * kPruneScale > thr) {
                         dn = -1;
                         take_dn = false;
                     }

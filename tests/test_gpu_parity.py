@@ -320,8 +320,12 @@ def _sweep_check(orc, w, H64, rows_sample=None):
     assert d_amax.item() == amax
     f = G.flags_dev()
     codes, q, c1, c2 = nv4.scale_sweep(wd, G.f32_dev(H32), d_amax, d_flags=f)
+    # without the runner-up output the bounds prune against the best cost: the same
+    # winners and nibbles, bit for bit
+    codes_only, q_only, _, _ = nv4.scale_sweep(wd, G.f32_dev(H32), d_amax, with_costs=False, d_flags=f)
     torch.cuda.synchronize()
     assert f.item() == 0
+    assert torch.equal(codes_only, codes) and torch.equal(q_only, q)
     ref = orc.scale_sweep(w, Hin, amax, rows=rows_sample)
     idx = ref["rows"]
     stats = G.sweep_parity(G.host(codes)[idx], G.host(q)[idx], G.host(c1)[idx], ref, c2_gpu=G.host(c2)[idx])
@@ -481,8 +485,16 @@ def test_sweep_work_counter(orc):
     nv4.nv4_scale_sweep_batched(jobs, f)
     torch.cuda.synchronize()
     assert f.item() == 0
-    on, off = work[0].cpu().numpy(), work[1].cpu().numpy()
-    print("work with bounds", on, "without", off)
+    # codes only (no runner-up): pruning against the best cost, fewer costs, same winners
+    lean = torch.zeros(2, dtype=torch.int64, device=G.DEV)
+    j0 = dict(jobs[0], cost1=None, cost2=None, d_work=lean,
+              codes=torch.empty_like(jobs[0]["codes"]), q=torch.empty_like(jobs[0]["q"]))
+    nv4.nv4_scale_sweep_batched([j0], f)
+    torch.cuda.synchronize()
+    assert torch.equal(j0["codes"], jobs[0]["codes"]) and torch.equal(j0["q"], jobs[0]["q"])
+    on, off, ln = work[0].cpu().numpy(), work[1].cpu().numpy(), lean.cpu().numpy()
+    print("work with bounds", on, "without", off, "codes only", ln)
+    assert ln[1] <= on[1] and ln[0] <= on[0]
     assert off[0] == 127 * rows and off[1] == 127 * rows
     assert on[1] <= on[0] <= 127 * rows and on[1] < 0.25 * 127 * rows
     ref = orc.scale_sweep(w, H.astype(np.float32).astype(np.float64), orc.tensor_amax(w)[0])

@@ -15,9 +15,10 @@
 //     (lane-interleaved so each instruction moves contiguous bytes).  It recovers k_max
 //     = m + 8 exactly from the s2 it reads back, writes the two E4M3 scale bytes per
 //     block and, out of place, copies the 16 nibble bytes with 128-bit streaming loads
-//     and stores; rare blocks (NaN code, outside the window) take a separate exact
-//     path.  Launched as a programmatic dependent of kernel 1, it copies the nibbles of
-//     each warp's first tiles while kernel 1 runs, then waits for kernel 1.
+//     and stores; rare blocks (NaN code, outside the window) are handled by the whole
+//     warp, one element per lane.  Launched as a programmatic dependent of kernel 1, it
+//     copies the nibbles of each warp's first tiles while kernel 1 runs, then waits for
+//     kernel 1.
 #include "nv4_common.cuh"
 #include "nv4_internal.h"
 
@@ -34,7 +35,7 @@ struct CastJobDev {
     float* d_ga;
     float* d_s2;
     uint32_t nb;                                  // MX blocks in the matrix (rows * cols / 32)
-    uint32_t chunk_begin;                         // prefix sum of kTile-block tiles over jobs
+    uint32_t tile_begin;                         // prefix sum of kTile-block tiles over jobs
 };
 
 struct CastParams {
@@ -42,7 +43,7 @@ struct CastParams {
     int n_sets;                                   // scale_2 groups (sets of jobs sharing k_max)
     uint16_t set_begin[kMaxCastJobs + 1];         // members of set g: set_jobs[set_begin[g] .. set_begin[g+1])
     uint16_t set_jobs[kMaxCastJobs];
-    uint32_t chunks;                              // total kTile-block tiles over all jobs
+    uint32_t tiles;                               // total kTile-block tiles over all jobs
     unsigned long long* d_counts;
     uint32_t* d_flags;
     CastJobDev jobs[kMaxCastJobs];
@@ -261,7 +262,7 @@ __device__ __forceinline__ int cast_job_of(const CastParams& p, uint32_t ti)
     int lo = 0, hi = p.n - 1;
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
-        if (p.jobs[mid].chunk_begin <= ti) lo = mid; else hi = mid - 1;
+        if (p.jobs[mid].tile_begin <= ti) lo = mid; else hi = mid - 1;
     }
     return lo;
 }
@@ -276,10 +277,10 @@ cast_rewrite_kernel(const __grid_constant__ CastParams p)
     // ---- nibble copy of the first tiles (out of place), before kernel 1 has finished
     {
         uint32_t k = 0u;
-        for (uint32_t ti = warp_id; k < kPreTiles && ti < p.chunks; ti += nwarps, ++k) {
+        for (uint32_t ti = warp_id; k < kPreTiles && ti < p.tiles; ti += nwarps, ++k) {
             const CastJobDev& job = p.jobs[cast_job_of(p, ti)];
             if (job.nv_q == job.mx_q) continue;
-            const uint32_t base = kTile * (ti - job.chunk_begin);
+            const uint32_t base = kTile * (ti - job.tile_begin);
             uint4 qv[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
@@ -299,12 +300,12 @@ cast_rewrite_kernel(const __grid_constant__ CastParams p)
 
     uint32_t n_in = 0u, n_fb = 0u, n_ll = 0u;
     uint32_t k = 0u;
-    for (uint32_t ti = warp_id; ti < p.chunks; ti += nwarps, ++k) {
+    for (uint32_t ti = warp_id; ti < p.tiles; ti += nwarps, ++k) {
         const CastJobDev& job = p.jobs[cast_job_of(p, ti)];
         const float s2 = *job.d_s2;
         const int k_max = exact_log2(s2) + 8;
         const bool copy = job.nv_q != job.mx_q && k >= kPreTiles;     // nibbles still to copy
-        const uint32_t base = kTile * (ti - job.chunk_begin);
+        const uint32_t base = kTile * (ti - job.tile_begin);
         uint32_t c[8];
         uint4 qv[8];
 #pragma unroll
@@ -370,7 +371,7 @@ cudaError_t launch_cast(const nv4_cast_job* jobs, int n, unsigned long long* d_c
     p.d_counts = d_counts;
     p.d_flags = d_flags;
     int m = 0;
-    uint32_t chunks = 0;
+    uint32_t tiles = 0;
     for (int i = 0; i < n; ++i) {
         const nv4_cast_job& J = jobs[i];
         if (J.rows == 0 || J.cols == 0) continue;
@@ -378,11 +379,11 @@ cudaError_t launch_cast(const nv4_cast_job* jobs, int n, unsigned long long* d_c
         d.mx_q = J.mx_q; d.e8m0 = J.e8m0; d.nv_q = J.nv_q; d.nv_scales = J.nv_scales;
         d.d_ga = J.d_global_amax; d.d_s2 = J.d_s2;
         d.nb = (uint32_t)(J.rows * (J.cols / 32));
-        d.chunk_begin = chunks;
-        chunks += (d.nb + kTile - 1u) / kTile;
+        d.tile_begin = tiles;
+        tiles += (d.nb + kTile - 1u) / kTile;
     }
     p.n = m;
-    p.chunks = chunks;
+    p.tiles = tiles;
     if (m == 0) return cudaSuccess;
     // scale_2 sets: jobs with the same non-negative group id share one k_max
     {
@@ -425,7 +426,7 @@ cudaError_t launch_cast(const nv4_cast_job* jobs, int n, unsigned long long* d_c
     // a single resident wave, launched as a programmatic dependent of the k_max kernel
     // so that its first loads overlap that kernel; it waits for the k_max results
     // before using them
-    const uint64_t warps_needed = chunks;
+    const uint64_t warps_needed = tiles;            // one warp per tile at most
     const uint64_t cap = (uint64_t)num_sms() * kRwCtasPerSm;
     const uint64_t need = (warps_needed + kRwThreads / 32 - 1) / (kRwThreads / 32);
     const int grid = (int)(need < cap ? need : cap);

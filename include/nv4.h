@@ -97,6 +97,19 @@ NV4_API int nv4_version(void);
 NV4_API nv4_status nv4_tensor_amax(const void* x, nv4_dtype dt, int64_t n, float* d_amax,
                            uint32_t* d_flags, void* stream);
 
+/* Batched form: the amax of several tensors of one dtype in one launch, each into its
+ * own d_amax (e.g. the 15 activation shapes of a quantization sweep).  Per job the
+ * rules of nv4_tensor_amax; n < 2^37 elements per job; at most 128 jobs (NV4_ERR_LIMIT
+ * beyond). */
+typedef struct {
+    const void* x;      /* n elements, contiguous, 16-byte aligned */
+    int64_t n;
+    float* d_amax;
+} nv4_amax_job;
+
+NV4_API nv4_status nv4_tensor_amax_batched(const nv4_amax_job* jobs, int n_jobs, nv4_dtype dt,
+                                   uint32_t* d_flags, void* stream);
+
 /* ---------------------------------------------------------------------------
  * nv4_act_quant -- dynamic NVFP4 quantization of activations.  [FLOW] 3.4-3.5:
  * the per-tensor scale comes from a (calibrated or just measured) amax, the block
@@ -117,6 +130,20 @@ NV4_API nv4_status nv4_tensor_amax(const void* x, nv4_dtype dt, int64_t n, float
 NV4_API nv4_status nv4_act_quant(const void* x, int64_t rows, int64_t cols, int64_t ld,
                          const float* d_amax, uint8_t* q, uint8_t* scales, float* d_s2,
                          uint32_t* d_flags, void* stream);
+
+/* Batched form: several BF16 tensors, each with its own amax and s2, in one launch.
+ * Per job the rules, layouts and limits of nv4_act_quant; at most 128 jobs. */
+typedef struct {
+    const void* x;      /* bf16 [rows, cols], leading dimension ld */
+    int64_t rows, cols, ld;
+    const float* d_amax;
+    uint8_t* q;         /* [rows, cols/2] */
+    uint8_t* scales;    /* [rows, cols/16] */
+    float* d_s2;
+} nv4_act_job;
+
+NV4_API nv4_status nv4_act_quant_batched(const nv4_act_job* jobs, int n_jobs, uint32_t* d_flags,
+                                 void* stream);
 
 /* ---------------------------------------------------------------------------
  * nv4_weight_quant_rtn -- static round-to-nearest NVFP4 quantization of a weight
@@ -159,6 +186,19 @@ NV4_API nv4_status nv4_fake_qdq(const void* x, int64_t rows, int64_t cols, int64
  */
 NV4_API nv4_status nv4_dequant(const uint8_t* q, const uint8_t* scales, const float* d_s2,
                        int64_t rows, int64_t cols, nv4_dtype out_dt, void* out, void* stream);
+
+/* Batched form: several tensors to one out_dt in one launch; per job the rules,
+ * layouts and limits of nv4_dequant; at most 128 jobs. */
+typedef struct {
+    const uint8_t* q;       /* [rows, cols/2] */
+    const uint8_t* scales;  /* [rows, cols/16] */
+    const float* d_s2;
+    int64_t rows, cols;
+    void* out;              /* [rows, cols] of out_dt, contiguous */
+} nv4_dequant_job;
+
+NV4_API nv4_status nv4_dequant_batched(const nv4_dequant_job* jobs, int n_jobs, nv4_dtype out_dt,
+                               void* stream);
 
 /* ---------------------------------------------------------------------------
  * nv4_hessian_accum -- local Hessian per 16-input-channel block, [CAL] section 2

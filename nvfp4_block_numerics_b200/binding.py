@@ -27,7 +27,8 @@ __all__ = [
     "nv4_hessian_accum_batched", "nv4_scale_sweep", "nv4_scale_sweep_batched", "nv4_mxfp4_to_nvfp4",
     "nv4_mxfp4_to_nvfp4_batched", "nv4_selftest", "nv4_version", "FLAG_NONFINITE", "FLAG_E8M0_NAN",
     "FLAG_OVERFLOW", "FLAG_TIMEOUT", "tensor_amax", "act_quant", "dequant", "hessian_accum",
-    "scale_sweep", "mxfp4_to_nvfp4", "HessianJob", "SweepJob", "CastJob",
+    "scale_sweep", "mxfp4_to_nvfp4", "HessianJob", "SweepJob", "CastJob", "AmaxJob", "ActJob", "DequantJob",
+    "nv4_tensor_amax_batched", "nv4_act_quant_batched", "nv4_dequant_batched",
 ]
 
 BF16, FP16, FP32 = 0, 1, 2
@@ -35,6 +36,19 @@ FLAG_NONFINITE, FLAG_E8M0_NAN, FLAG_OVERFLOW, FLAG_TIMEOUT = 1, 2, 4, 8
 _DT = {torch.bfloat16: BF16, torch.float16: FP16, torch.float32: FP32}
 
 _vp, _i64 = C.c_void_p, C.c_int64
+
+
+class AmaxJob(C.Structure):
+    _fields_ = [("x", _vp), ("n", _i64), ("d_amax", _vp)]
+
+
+class ActJob(C.Structure):
+    _fields_ = [("x", _vp), ("rows", _i64), ("cols", _i64), ("ld", _i64), ("d_amax", _vp), ("q", _vp),
+                ("scales", _vp), ("d_s2", _vp)]
+
+
+class DequantJob(C.Structure):
+    _fields_ = [("q", _vp), ("scales", _vp), ("d_s2", _vp), ("rows", _i64), ("cols", _i64), ("out", _vp)]
 
 
 class HessianJob(C.Structure):
@@ -63,6 +77,9 @@ _SIGS = {
     "nv4_version": (C.c_int, []),
     "nv4_tensor_amax": (C.c_int, [_vp, C.c_int, _i64, _vp, _vp, _vp]),
     "nv4_act_quant": (C.c_int, [_vp, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "nv4_tensor_amax_batched": (C.c_int, [C.POINTER(AmaxJob), C.c_int, C.c_int, _vp, _vp]),
+    "nv4_act_quant_batched": (C.c_int, [C.POINTER(ActJob), C.c_int, _vp, _vp]),
+    "nv4_dequant_batched": (C.c_int, [C.POINTER(DequantJob), C.c_int, C.c_int, _vp]),
     "nv4_weight_quant_rtn": (C.c_int, [_vp, C.c_int, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp]),
     "nv4_fake_qdq": (C.c_int, [_vp, _i64, _i64, _i64, _vp, C.c_int, _vp, _i64, _vp, _vp, _vp]),
     "nv4_dequant": (C.c_int, [_vp, _vp, _vp, _i64, _i64, C.c_int, _vp, _vp]),
@@ -156,6 +173,60 @@ def nv4_act_quant(x: torch.Tensor, d_amax: torch.Tensor, q: torch.Tensor, scales
         raise NV4Error("scales must be a contiguous uint8 tensor [rows, cols/16]")
     _check(lib().nv4_act_quant(_ptr(x), rows, cols, ld, _scalar_f32(d_amax, "d_amax"), _ptr(q), _ptr(scales),
                                _scalar_f32(d_s2, "d_s2"), _ptr(d_flags), _stream(stream)), "nv4_act_quant")
+
+
+def nv4_tensor_amax_batched(xs, d_amaxes, d_flags: torch.Tensor | None = None, stream=None):
+    """The amax of every tensor of xs (one dtype, contiguous) into the matching d_amaxes entry,
+    in one launch."""
+    if len(xs) != len(d_amaxes):
+        raise NV4Error("one d_amax per tensor")
+    if not xs:
+        return
+    dt = xs[0].dtype
+    if dt not in (torch.bfloat16, torch.float32) or any(x.dtype != dt or not x.is_contiguous() for x in xs):
+        raise NV4Error("xs must be contiguous tensors of one dtype, bf16 or float32")
+    arr = (AmaxJob * len(xs))(*[AmaxJob(_ptr(x), x.numel(), _scalar_f32(a, "d_amax")) for x, a in zip(xs, d_amaxes)])
+    _check(lib().nv4_tensor_amax_batched(arr, len(xs), _DT[dt], _ptr(d_flags), _stream(stream)),
+           "nv4_tensor_amax_batched")
+
+
+def nv4_act_quant_batched(jobs: list[dict], d_flags: torch.Tensor | None = None, stream=None):
+    """jobs: dicts with keys x (bf16 [rows, cols]), d_amax, q, scales, d_s2 -- nv4_act_quant per
+    tensor, in one launch."""
+    arr = (ActJob * len(jobs))()
+    for i, j in enumerate(jobs):
+        x = j["x"]
+        if x.dtype != torch.bfloat16:
+            raise NV4Error("x must be bf16")
+        rows, cols, ld = _rowmajor(x, "x")
+        q, sc = j["q"], j["scales"]
+        if q.dtype != torch.uint8 or tuple(q.shape) != (rows, cols // 2) or not q.is_contiguous():
+            raise NV4Error("q must be a contiguous uint8 tensor [rows, cols/2]")
+        if sc.dtype != torch.uint8 or tuple(sc.shape) != (rows, cols // 16) or not sc.is_contiguous():
+            raise NV4Error("scales must be a contiguous uint8 tensor [rows, cols/16]")
+        arr[i] = ActJob(_ptr(x), rows, cols, ld, _scalar_f32(j["d_amax"], "d_amax"), _ptr(q), _ptr(sc),
+                        _scalar_f32(j["d_s2"], "d_s2"))
+    _check(lib().nv4_act_quant_batched(arr, len(jobs), _ptr(d_flags), _stream(stream)), "nv4_act_quant_batched")
+
+
+def nv4_dequant_batched(jobs: list[dict], stream=None):
+    """jobs: dicts with keys q, scales, d_s2, out (all outputs of one dtype) -- nv4_dequant per
+    tensor, in one launch."""
+    if not jobs:
+        return
+    dt = jobs[0]["out"].dtype
+    arr = (DequantJob * len(jobs))()
+    for i, j in enumerate(jobs):
+        q, sc, out = j["q"], j["scales"], j["out"]
+        if out.dtype != dt or out.dtype not in _DT or not out.is_contiguous() or out.dim() != 2:
+            raise NV4Error("outs must be contiguous 2-D tensors of one dtype (bf16, fp16 or float32)")
+        rows, cols = out.shape
+        if tuple(q.shape) != (rows, cols // 2) or tuple(sc.shape) != (rows, cols // 16):
+            raise NV4Error("q / scales shapes do not match out")
+        if not (q.is_contiguous() and sc.is_contiguous()):
+            raise NV4Error("q and scales must be contiguous")
+        arr[i] = DequantJob(_ptr(q), _ptr(sc), _scalar_f32(j["d_s2"], "d_s2"), rows, cols, _ptr(out))
+    _check(lib().nv4_dequant_batched(arr, len(jobs), _DT[dt], _stream(stream)), "nv4_dequant_batched")
 
 
 def nv4_weight_quant_rtn(w: torch.Tensor, d_amax: torch.Tensor, q: torch.Tensor, scales: torch.Tensor,

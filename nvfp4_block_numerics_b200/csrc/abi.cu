@@ -120,18 +120,48 @@ const char* nv4_status_str(nv4_status s)
 
 int nv4_version(void) { return 100; }
 
+// ---------------------------------------------------------------- amax, act quant, dequant
+static nv4_status check_amax(const void* x, int64_t n, const float* d_amax)
+{
+    if (n < 0) return NV4_ERR_SHAPE;
+    if (n == 0) return NV4_OK;
+    if (x == nullptr || d_amax == nullptr) return NV4_ERR_NULL;
+    if (!aligned16(x)) return NV4_ERR_ALIGN;
+    if (n >= (int64_t)1 << 37) return NV4_ERR_LIMIT;
+    return NV4_OK;
+}
+
 nv4_status nv4_tensor_amax(const void* x, nv4_dtype dt, int64_t n, float* d_amax, uint32_t* d_flags, void* stream)
 {
     if (n < 0) return NV4_ERR_SHAPE;
     if (n == 0) return NV4_OK;
     if (x == nullptr || d_amax == nullptr) return NV4_ERR_NULL;
     if (dt != NV4_BF16 && dt != NV4_FP32) return NV4_ERR_DTYPE;
-    if (!aligned16(x)) return NV4_ERR_ALIGN;
-    return from_cuda(launch_amax(x, dt == NV4_BF16 ? 0 : 2, n, d_amax, d_flags, (cudaStream_t)stream));
+    const nv4_status st = check_amax(x, n, d_amax);
+    if (st != NV4_OK) return st;
+    const AmaxTask t = {x, n, d_amax};
+    return from_cuda(launch_amax(&t, 1, dt == NV4_BF16 ? 0 : 2, d_flags, (cudaStream_t)stream));
 }
 
-nv4_status nv4_act_quant(const void* x, int64_t rows, int64_t cols, int64_t ld, const float* d_amax, uint8_t* q,
-                         uint8_t* scales, float* d_s2, uint32_t* d_flags, void* stream)
+nv4_status nv4_tensor_amax_batched(const nv4_amax_job* jobs, int n_jobs, nv4_dtype dt, uint32_t* d_flags,
+                                   void* stream)
+{
+    if (n_jobs < 0) return NV4_ERR_SHAPE;
+    if (n_jobs == 0) return NV4_OK;
+    if (jobs == nullptr) return NV4_ERR_NULL;
+    if (n_jobs > kMaxActJobs) return NV4_ERR_LIMIT;
+    if (dt != NV4_BF16 && dt != NV4_FP32) return NV4_ERR_DTYPE;
+    AmaxTask t[kMaxActJobs];
+    for (int i = 0; i < n_jobs; ++i) {
+        const nv4_status st = check_amax(jobs[i].x, jobs[i].n, jobs[i].d_amax);
+        if (st != NV4_OK) return st;
+        t[i] = {jobs[i].x, jobs[i].n, jobs[i].d_amax};
+    }
+    return from_cuda(launch_amax(t, n_jobs, dt == NV4_BF16 ? 0 : 2, d_flags, (cudaStream_t)stream));
+}
+
+static nv4_status check_act(const void* x, int64_t rows, int64_t cols, int64_t ld, const float* d_amax,
+                            const uint8_t* q, const uint8_t* scales, const float* d_s2)
 {
     if (rows < 0 || cols < 0 || cols % 16 != 0 || ld < cols) return NV4_ERR_SHAPE;
     if (d_amax == nullptr || d_s2 == nullptr) return NV4_ERR_NULL;
@@ -139,7 +169,32 @@ nv4_status nv4_act_quant(const void* x, int64_t rows, int64_t cols, int64_t ld, 
     if (x == nullptr || q == nullptr || scales == nullptr) return NV4_ERR_NULL;
     if (!aligned16(x) || !aligned16(q) || ld % 8 != 0) return NV4_ERR_ALIGN;
     if (rows * (cols / 16) >= (int64_t)1 << 30) return NV4_ERR_LIMIT;
-    return from_cuda(launch_act_quant(x, rows, cols, ld, d_amax, q, scales, d_s2, d_flags, (cudaStream_t)stream));
+    return NV4_OK;
+}
+
+nv4_status nv4_act_quant(const void* x, int64_t rows, int64_t cols, int64_t ld, const float* d_amax, uint8_t* q,
+                         uint8_t* scales, float* d_s2, uint32_t* d_flags, void* stream)
+{
+    const nv4_status st = check_act(x, rows, cols, ld, d_amax, q, scales, d_s2);
+    if (st != NV4_OK || rows == 0 || cols == 0) return st;
+    const QuantTask t = {x, rows, cols, ld, d_amax, q, scales, nullptr, 0, d_s2};
+    return from_cuda(launch_block_quant(&t, 1, 0, -1, d_flags, (cudaStream_t)stream));
+}
+
+nv4_status nv4_act_quant_batched(const nv4_act_job* jobs, int n_jobs, uint32_t* d_flags, void* stream)
+{
+    if (n_jobs < 0) return NV4_ERR_SHAPE;
+    if (n_jobs == 0) return NV4_OK;
+    if (jobs == nullptr) return NV4_ERR_NULL;
+    if (n_jobs > kMaxActJobs) return NV4_ERR_LIMIT;
+    QuantTask t[kMaxActJobs];
+    for (int i = 0; i < n_jobs; ++i) {
+        const nv4_act_job& J = jobs[i];
+        const nv4_status st = check_act(J.x, J.rows, J.cols, J.ld, J.d_amax, J.q, J.scales, J.d_s2);
+        if (st != NV4_OK) return st;
+        t[i] = {J.x, J.rows, J.cols, J.ld, J.d_amax, J.q, J.scales, nullptr, 0, J.d_s2};
+    }
+    return from_cuda(launch_block_quant(t, n_jobs, 0, -1, d_flags, (cudaStream_t)stream));
 }
 
 nv4_status nv4_weight_quant_rtn(const void* w, nv4_dtype dt, int64_t rows, int64_t cols, int64_t ld,
@@ -153,8 +208,8 @@ nv4_status nv4_weight_quant_rtn(const void* w, nv4_dtype dt, int64_t rows, int64
     if (w == nullptr || q == nullptr || scales == nullptr) return NV4_ERR_NULL;
     if (!aligned16(w) || !aligned16(q) || ld % (dt == NV4_BF16 ? 8 : 4) != 0) return NV4_ERR_ALIGN;
     if (rows * (cols / 16) >= (int64_t)1 << 30) return NV4_ERR_LIMIT;
-    return from_cuda(launch_block_quant(w, dt == NV4_BF16 ? 0 : 2, rows, cols, ld, d_amax, q, scales, -1, nullptr, 0,
-                                        d_s2, d_flags, (cudaStream_t)stream));
+    const QuantTask t = {w, rows, cols, ld, d_amax, q, scales, nullptr, 0, d_s2};
+    return from_cuda(launch_block_quant(&t, 1, dt == NV4_BF16 ? 0 : 2, -1, d_flags, (cudaStream_t)stream));
 }
 
 nv4_status nv4_fake_qdq(const void* x, int64_t rows, int64_t cols, int64_t ld, const float* d_amax,
@@ -168,8 +223,19 @@ nv4_status nv4_fake_qdq(const void* x, int64_t rows, int64_t cols, int64_t ld, c
     if (!aligned16(x) || !aligned16(out) || ld % 8 != 0 || ld_out % (out_dt == NV4_FP32 ? 4 : 8) != 0)
         return NV4_ERR_ALIGN;
     if (rows * (cols / 16) >= (int64_t)1 << 30) return NV4_ERR_LIMIT;
-    return from_cuda(launch_block_quant(x, 0, rows, cols, ld, d_amax, nullptr, nullptr, (int)out_dt, out, ld_out,
-                                        d_s2, d_flags, (cudaStream_t)stream));
+    const QuantTask t = {x, rows, cols, ld, d_amax, nullptr, nullptr, out, ld_out, d_s2};
+    return from_cuda(launch_block_quant(&t, 1, 0, (int)out_dt, d_flags, (cudaStream_t)stream));
+}
+
+static nv4_status check_dequant(const uint8_t* q, const uint8_t* scales, const float* d_s2, int64_t rows,
+                                int64_t cols, const void* out)
+{
+    if (rows < 0 || cols < 0 || cols % 16 != 0) return NV4_ERR_SHAPE;
+    if (rows == 0 || cols == 0) return NV4_OK;
+    if (q == nullptr || scales == nullptr || d_s2 == nullptr || out == nullptr) return NV4_ERR_NULL;
+    if (!aligned16(q) || !aligned16(scales) || !aligned16(out)) return NV4_ERR_ALIGN;
+    if (rows * (cols / 16) >= (int64_t)1 << 30) return NV4_ERR_LIMIT;
+    return NV4_OK;
 }
 
 nv4_status nv4_dequant(const uint8_t* q, const uint8_t* scales, const float* d_s2, int64_t rows, int64_t cols,
@@ -177,11 +243,27 @@ nv4_status nv4_dequant(const uint8_t* q, const uint8_t* scales, const float* d_s
 {
     if (rows < 0 || cols < 0 || cols % 16 != 0) return NV4_ERR_SHAPE;
     if (out_dt != NV4_BF16 && out_dt != NV4_FP16 && out_dt != NV4_FP32) return NV4_ERR_DTYPE;
-    if (rows == 0 || cols == 0) return NV4_OK;
-    if (q == nullptr || scales == nullptr || d_s2 == nullptr || out == nullptr) return NV4_ERR_NULL;
-    if (!aligned16(q) || !aligned16(scales) || !aligned16(out)) return NV4_ERR_ALIGN;
-    if (rows * (cols / 16) >= (int64_t)1 << 30) return NV4_ERR_LIMIT;
-    return from_cuda(launch_dequant(q, scales, d_s2, rows, cols, (int)out_dt, out, (cudaStream_t)stream));
+    const nv4_status st = check_dequant(q, scales, d_s2, rows, cols, out);
+    if (st != NV4_OK || rows == 0 || cols == 0) return st;
+    const DequantTask t = {q, scales, d_s2, rows, cols, out};
+    return from_cuda(launch_dequant(&t, 1, (int)out_dt, (cudaStream_t)stream));
+}
+
+nv4_status nv4_dequant_batched(const nv4_dequant_job* jobs, int n_jobs, nv4_dtype out_dt, void* stream)
+{
+    if (n_jobs < 0) return NV4_ERR_SHAPE;
+    if (n_jobs == 0) return NV4_OK;
+    if (jobs == nullptr) return NV4_ERR_NULL;
+    if (n_jobs > kMaxActJobs) return NV4_ERR_LIMIT;
+    if (out_dt != NV4_BF16 && out_dt != NV4_FP16 && out_dt != NV4_FP32) return NV4_ERR_DTYPE;
+    DequantTask t[kMaxActJobs];
+    for (int i = 0; i < n_jobs; ++i) {
+        const nv4_dequant_job& J = jobs[i];
+        const nv4_status st = check_dequant(J.q, J.scales, J.d_s2, J.rows, J.cols, J.out);
+        if (st != NV4_OK) return st;
+        t[i] = {J.q, J.scales, J.d_s2, J.rows, J.cols, J.out};
+    }
+    return from_cuda(launch_dequant(t, n_jobs, (int)out_dt, (cudaStream_t)stream));
 }
 
 static nv4_status check_hessian_job(const nv4_hessian_job& J)

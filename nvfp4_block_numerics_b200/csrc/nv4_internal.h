@@ -34,12 +34,34 @@ constexpr int kMaxHessianJobs = 128;
 constexpr int kMaxSweepJobs = 192;
 constexpr int kMaxCastJobs = 128;
 
-cudaError_t launch_amax(const void* x, int dt, int64_t n, float* d_amax, uint32_t* d_flags, cudaStream_t s);
-cudaError_t launch_act_quant(const void* x, int64_t rows, int64_t cols, int64_t ld, const float* d_amax,
-                             uint8_t* q, uint8_t* scales, float* d_s2, uint32_t* d_flags, cudaStream_t s);
-cudaError_t launch_block_quant(const void* x, int in_dt, int64_t rows, int64_t cols, int64_t ld,
-                               const float* d_amax, uint8_t* q, uint8_t* scales, int out_dt, void* out,
-                               int64_t ld_out, float* d_s2, uint32_t* d_flags, cudaStream_t s);
+// One tensor of a (batched) per-tensor amax, block quantization or dequantization call.
+struct AmaxTask {
+    const void* x;
+    int64_t n;
+    float* d_amax;
+};
+struct QuantTask {
+    const void* x;
+    int64_t rows, cols, ld;
+    const float* d_amax;
+    uint8_t* q;           // packed codes (code output) or null
+    uint8_t* scales;
+    void* out;            // fake quantize-dequantize output or null
+    int64_t ld_out;
+    float* d_s2;
+};
+struct DequantTask {
+    const uint8_t* q;
+    const uint8_t* scales;
+    const float* d_s2;
+    int64_t rows, cols;
+    void* out;
+};
+constexpr int kMaxActJobs = 128;
+
+cudaError_t launch_amax(const AmaxTask* tasks, int n, int dt, uint32_t* d_flags, cudaStream_t s);
+cudaError_t launch_block_quant(const QuantTask* tasks, int n, int in_dt, int out_dt, uint32_t* d_flags,
+                               cudaStream_t s);
 cudaError_t launch_mxfp4_quant(const void* x, int in_dt, int64_t rows, int64_t cols, int64_t ld, uint8_t* q,
                                uint8_t* e8m0, uint32_t* d_flags, cudaStream_t s);
 cudaError_t launch_mxfp4_dequant(const uint8_t* q, const uint8_t* e8m0, int64_t rows, int64_t cols, int out_dt,
@@ -57,8 +79,7 @@ cudaError_t launch_mma_scale_layout(const uint8_t* sc, int64_t rows, int64_t kb,
 cudaError_t launch_gemm_nvfp4(const uint8_t* qa, const uint8_t* sfa, const float* d_s2a, const uint8_t* qb,
                               const uint8_t* sfb, const float* d_s2b, int64_t M, int64_t N, int64_t K, int out_dt,
                               void* out, int64_t ldd, uint32_t* d_flags, cudaStream_t s);
-cudaError_t launch_dequant(const uint8_t* q, const uint8_t* scales, const float* d_s2, int64_t rows, int64_t cols,
-                           int out_dt, void* out, cudaStream_t s);
+cudaError_t launch_dequant(const DequantTask* tasks, int n, int out_dt, cudaStream_t s);
 cudaError_t launch_hessian(const nv4_hessian_job* jobs, int n, uint32_t* d_flags, cudaStream_t s, int* bad_job);
 cudaError_t launch_sweep(const nv4_sweep_job* jobs, int n, int dt, uint32_t* d_flags, cudaStream_t s);
 cudaError_t launch_cast(const nv4_cast_job* jobs, int n, unsigned long long* d_counts, uint32_t* d_flags,

@@ -49,82 +49,127 @@ __device__ __forceinline__ uint32_t absmax_bf16x8_no_nan(const uint4& v)
     return m;
 }
 
-template <int kThreads>
-__global__ void __launch_bounds__(kThreads)
-amax_bf16_kernel(const uint4* __restrict__ x, int64_t nvec, const uint16_t* __restrict__ tail, int ntail,
-                 float* __restrict__ d_amax, uint32_t* __restrict__ d_flags)
+// Jobs: one or more tensors, each split into tiles of kAmaxTile 16-byte vectors; a
+// tile belongs to one job, and a CTA strides over the tiles of all jobs (so the grid
+// sweeps one region of memory at a time).  A CTA keeps a running maximum while its
+// tiles stay in one job and folds it into that job's amax when the job changes.
+constexpr int kAmaxThreads = 512;
+constexpr uint32_t kAmaxVec = 4;                                // vectors per thread per tile
+constexpr uint32_t kAmaxTile = kAmaxThreads * kAmaxVec;
+
+struct AmaxJobDev {
+    const uint4* x;
+    const void* tail;                                           // the n % (elements per vector) last ones
+    int64_t nvec;
+    int ntail;
+    float* d_amax;
+    uint32_t tile_begin, tile_end;
+};
+
+struct AmaxParams {
+    int n;
+    uint32_t tiles;
+    uint32_t* d_flags;
+    AmaxJobDev jobs[kMaxActJobs];
+};
+
+// The job holding tile t (jobs are ordered by their first tile and own at least one).
+template <class P>
+__device__ __forceinline__ int job_of_tile(const P& p, uint32_t t)
 {
-    __shared__ uint32_t red[kThreads / 32];
-    const int64_t stride = (int64_t)gridDim.x * kThreads;
-    const int64_t i0 = (int64_t)blockIdx.x * kThreads + threadIdx.x;
-    uint32_t m = 0u;                                   // two packed 16-bit maxima
-    int64_t i = i0;
-    for (; i + 3 * stride < nvec; i += 4 * stride) {   // four independent loads in flight
-        const uint4 v0 = __ldcs(x + i), v1 = __ldcs(x + i + stride);
-        const uint4 v2 = __ldcs(x + i + 2 * stride), v3 = __ldcs(x + i + 3 * stride);
-        m = __vmaxu2(m, __vmaxu2(__vmaxu2(absmax_bf16x8(v0), absmax_bf16x8(v1)),
-                                 __vmaxu2(absmax_bf16x8(v2), absmax_bf16x8(v3))));
+    int lo = 0, hi = p.n - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (p.jobs[mid].tile_begin <= t) lo = mid; else hi = mid - 1;
     }
-    for (; i < nvec; i += stride) m = __vmaxu2(m, absmax_bf16x8(__ldcs(x + i)));
-    uint32_t amax = max(m & 0xFFFFu, m >> 16);
-    if (blockIdx.x == 0)
-        for (int t = threadIdx.x; t < ntail; t += kThreads) amax = max(amax, (uint32_t)(tail[t] & 0x7FFFu));
-    uint32_t flags = amax >= 0x7F80u ? kFlagNonFinite : 0u;
-    if (amax > 0x7F80u) {                              // a NaN: recompute without NaN entries
-        amax = 0u;
-        for (int64_t k = i0; k < nvec; k += stride) amax = max(amax, absmax_bf16x8_no_nan(x[k]));
-        if (blockIdx.x == 0)
-            for (int t = threadIdx.x; t < ntail; t += kThreads) {
-                const uint32_t a = tail[t] & 0x7FFFu;
-                if (a <= 0x7F80u) amax = max(amax, a);
-            }
-    }
-    flags = __reduce_or_sync(0xFFFFFFFFu, flags);
-    if ((threadIdx.x & 31) == 0) flag_or(d_flags, flags);
-    amax = block_max_u32<kThreads>(amax << 16, red);   // BF16 bits -> FP32 bits
-    if (threadIdx.x == 0 && amax != 0u) atomicMax(reinterpret_cast<unsigned int*>(d_amax), amax);
+    return lo;
 }
 
-template <int kThreads>
-__global__ void __launch_bounds__(kThreads)
-amax_f32_kernel(const uint4* __restrict__ x, int64_t nvec, const uint32_t* __restrict__ tail, int ntail,
-                float* __restrict__ d_amax, uint32_t* __restrict__ d_flags)
+// Largest magnitude of a 16-byte vector as an FP32 bit pattern (NaN patterns included:
+// they sort above +Inf); kDt 0: eight BF16, 2: four FP32.
+template <int kDt>
+__device__ __forceinline__ uint32_t vec_absmax(const uint4& v)
 {
-    __shared__ uint32_t red[kThreads / 32];
-    const int64_t stride = (int64_t)gridDim.x * kThreads;
-    const int64_t i0 = (int64_t)blockIdx.x * kThreads + threadIdx.x;
-    uint32_t m = 0u;
-    int64_t i = i0;
-    for (; i + 1 * stride < nvec; i += 2 * stride) {
-        const uint4 v0 = __ldcs(x + i), v1 = __ldcs(x + i + stride);
-        m = max(m, max(max(v0.x & 0x7FFFFFFFu, v0.y & 0x7FFFFFFFu), max(v0.z & 0x7FFFFFFFu, v0.w & 0x7FFFFFFFu)));
-        m = max(m, max(max(v1.x & 0x7FFFFFFFu, v1.y & 0x7FFFFFFFu), max(v1.z & 0x7FFFFFFFu, v1.w & 0x7FFFFFFFu)));
+    if constexpr (kDt == 0) {
+        const uint32_t m = absmax_bf16x8(v);
+        return max(m & 0xFFFFu, m >> 16) << 16;
+    } else {
+        return max(max(v.x & 0x7FFFFFFFu, v.y & 0x7FFFFFFFu), max(v.z & 0x7FFFFFFFu, v.w & 0x7FFFFFFFu));
     }
-    for (; i < nvec; i += stride) {
-        const uint4 v = __ldcs(x + i);
-        m = max(m, max(max(v.x & 0x7FFFFFFFu, v.y & 0x7FFFFFFFu), max(v.z & 0x7FFFFFFFu, v.w & 0x7FFFFFFFu)));
+}
+
+template <int kDt>
+__device__ __forceinline__ uint32_t vec_absmax_no_nan(const uint4& v)
+{
+    if constexpr (kDt == 0) {
+        return absmax_bf16x8_no_nan(v) << 16;
+    } else {
+        const uint32_t w[4] = {v.x & 0x7FFFFFFFu, v.y & 0x7FFFFFFFu, v.z & 0x7FFFFFFFu, v.w & 0x7FFFFFFFu};
+        uint32_t m = 0u;
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            if (w[j] <= 0x7F800000u) m = max(m, w[j]);
+        return m;
     }
-    if (blockIdx.x == 0)
-        for (int t = threadIdx.x; t < ntail; t += kThreads) m = max(m, tail[t] & 0x7FFFFFFFu);
-    uint32_t flags = m >= 0x7F800000u ? kFlagNonFinite : 0u;
-    if (m > 0x7F800000u) {
-        m = 0u;
-        for (int64_t k = i0; k < nvec; k += stride) {
-            const uint4 v = x[k];
-            const uint32_t w[4] = {v.x & 0x7FFFFFFFu, v.y & 0x7FFFFFFFu, v.z & 0x7FFFFFFFu, v.w & 0x7FFFFFFFu};
-            for (int j = 0; j < 4; ++j)
-                if (w[j] <= 0x7F800000u) m = max(m, w[j]);
-        }
-        if (blockIdx.x == 0)
-            for (int t = threadIdx.x; t < ntail; t += kThreads) {
-                const uint32_t a = tail[t] & 0x7FFFFFFFu;
-                if (a <= 0x7F800000u) m = max(m, a);
-            }
-    }
-    flags = __reduce_or_sync(0xFFFFFFFFu, flags);
-    if ((threadIdx.x & 31) == 0) flag_or(d_flags, flags);
-    m = block_max_u32<kThreads>(m, red);
+}
+
+template <int kDt>
+__device__ __forceinline__ uint32_t tail_abs(const void* tail, int i)
+{
+    if constexpr (kDt == 0) return (uint32_t)(static_cast<const uint16_t*>(tail)[i] & 0x7FFFu) << 16;
+    else return static_cast<const uint32_t*>(tail)[i] & 0x7FFFFFFFu;
+}
+
+__device__ __forceinline__ void amax_fold(float* d_amax, uint32_t m, uint32_t* red)
+{
+    m = block_max_u32<kAmaxThreads>(m, red);
     if (threadIdx.x == 0 && m != 0u) atomicMax(reinterpret_cast<unsigned int*>(d_amax), m);
+    __syncthreads();                                            // red is reused by the next fold
+}
+
+template <int kDt>
+__global__ void __launch_bounds__(kAmaxThreads)
+amax_kernel(const __grid_constant__ AmaxParams p)
+{
+    __shared__ uint32_t red[kAmaxThreads / 32];
+    int cur = -1;                                               // job of the running maximum (CTA-uniform)
+    uint32_t m = 0u, flags = 0u;
+    for (uint32_t t = blockIdx.x; t < p.tiles; t += gridDim.x) {
+        const int j = job_of_tile(p, t);
+        if (j != cur) {
+            if (cur >= 0) amax_fold(p.jobs[cur].d_amax, m, red);
+            cur = j;
+            m = 0u;
+        }
+        const AmaxJobDev& job = p.jobs[j];
+        const int64_t base = (int64_t)(t - job.tile_begin) * kAmaxTile + threadIdx.x;
+        uint4 v[kAmaxVec];
+#pragma unroll
+        for (uint32_t k = 0; k < kAmaxVec; ++k) {                 // four independent loads in flight
+            const int64_t i = base + k * kAmaxThreads;
+            v[k] = i < job.nvec ? __ldcs(job.x + i) : make_uint4(0u, 0u, 0u, 0u);
+        }
+        const bool tail = t + 1u == job.tile_end && (int)threadIdx.x < job.ntail;
+        uint32_t tm = tail ? tail_abs<kDt>(job.tail, threadIdx.x) : 0u;
+#pragma unroll
+        for (uint32_t k = 0; k < kAmaxVec; ++k) tm = max(tm, vec_absmax<kDt>(v[k]));
+        if (tm >= 0x7F800000u) {
+            flags |= kFlagNonFinite;
+            if (tm > 0x7F800000u) {                             // a NaN: these elements again without NaN entries
+                tm = 0u;
+                if (tail) {
+                    const uint32_t a = tail_abs<kDt>(job.tail, threadIdx.x);
+                    if (a <= 0x7F800000u) tm = a;
+                }
+#pragma unroll
+                for (uint32_t k = 0; k < kAmaxVec; ++k) tm = max(tm, vec_absmax_no_nan<kDt>(v[k]));
+            }
+        }
+        m = max(m, tm);
+    }
+    if (cur >= 0) amax_fold(p.jobs[cur].d_amax, m, red);
+    flags = __reduce_or_sync(0xFFFFFFFFu, flags);
+    if ((threadIdx.x & 31) == 0 && flags) flag_or(p.d_flags, flags);
 }
 
 // ============================================================== act quant
@@ -254,73 +299,108 @@ __device__ __forceinline__ void store_qdq(uint32_t q0, uint32_t q1, float S, voi
     }
 }
 
-// Block quantizer over a [rows, cols] tensor: one thread per 16-block, grid-stride,
-// with the next block's loads in flight while the current one is quantized.
+// Block quantizer over one or more [rows, cols] tensors (jobs): one thread per 16-block.
+// Tiles of kActThreads blocks belong to one job; a CTA takes every gridDim.x-th tile of
+// the concatenation (job by job, the job's fields and per-tensor constants -- s2 and
+// its brackets -- in registers) with the next block's loads in flight while the
+// current one is quantized.
 // kIn: 0 BF16, 2 FP32 input.  kOut: -1 writes packed codes + E4M3 scales; 0/1/2 writes
 // the fake quantize-dequantize values as BF16/FP16/FP32 (leading dimension ld_out).
 // Every block is read and written by the same thread, read first, so out may alias x.
+struct QuantJobDev {
+    const void* x;
+    void* out;
+    uint8_t* q;
+    uint8_t* scales;
+    const float* d_amax;
+    float* d_s2;
+    int64_t ld, ld_out;
+    FastDiv div_bpr;
+    uint32_t bpr, units, tile_begin;
+};
+
+struct QuantParams {
+    int n;
+    uint32_t tiles;
+    uint32_t* d_flags;
+    QuantJobDev jobs[kMaxActJobs];
+};
+
 template <int kIn, int kOut>
 __global__ void __launch_bounds__(kActThreads)
-act_quant_kernel(const void* x, uint32_t rows, uint32_t bpr, int64_t ld, FastDiv div_bpr,
-                 const float* __restrict__ d_amax, uint8_t* __restrict__ q, uint8_t* __restrict__ scales,
-                 void* out, int64_t ld_out, float* __restrict__ d_s2, uint32_t* __restrict__ d_flags)
+act_quant_kernel(const __grid_constant__ QuantParams p)
 {
     __shared__ E4M3Tables tab;
     fill_e4m3_tables(tab);
     __syncthreads();
 
-    const float amax = *d_amax;
-    const float s2 = __fdiv_rn(amax, 2688.0f);                  // RN32(amax / (6*448))
-    if (blockIdx.x == 0 && threadIdx.x == 0) *d_s2 = s2;
-    const bool fast_scale = s2 >= kTinyScale && s2 <= 0x1p100f;
-    const float k = __frcp_rn(__fmul_rn(6.0f, s2));             // ~ 1/(6*s2)
-    const float k_lo = __fmul_rn(k, kLoMargin), k_hi = __fmul_rn(k, kHiMargin);
-    const float rs2 = __frcp_rn(s2);                            // ~ 1/s2
-    uint32_t flags = isfinite(s2) ? 0u : kFlagOverflow;
+    uint32_t flags = 0u;
+    const uint32_t G = gridDim.x;
+    // jobs in order; within a job the CTA takes the tiles t = blockIdx.x (mod G), with the
+    // job's fields and constants in registers and the next block's loads in flight
+    for (int j = 0; j < p.n; ++j) {
+        const void* x = p.jobs[j].x;
+        const int64_t ld = p.jobs[j].ld;
+        const uint32_t bpr = p.jobs[j].bpr, units = p.jobs[j].units, tb = p.jobs[j].tile_begin;
+        const FastDiv div_bpr = p.jobs[j].div_bpr;
+        uint8_t* const q = p.jobs[j].q;
+        uint8_t* const scales = p.jobs[j].scales;
+        void* const out = p.jobs[j].out;
+        const int64_t ld_out = p.jobs[j].ld_out;
+        const uint32_t t0 = tb + (blockIdx.x + G - tb % G) % G;     // first tile of this CTA in the job
+        uint32_t u = (t0 - tb) * kActThreads + threadIdx.x;
+        if ((t0 - tb) * kActThreads >= units) continue;            // (CTA-uniform)
+        auto offset = [&](uint32_t uu, int64_t l) {
+            const uint32_t r = div_bpr.div(uu), bb = uu - r * bpr;
+            return (int64_t)r * l + 16 * (int64_t)bb;
+        };
 
-    const uint32_t total = rows * bpr;
-    const uint32_t stride = gridDim.x * kActThreads;
-    auto offset = [&](uint32_t u, int64_t l) {
-        const uint32_t r = div_bpr.div(u), bb = u - r * bpr;
-        return (int64_t)r * l + 16 * (int64_t)bb;
-    };
-    uint32_t u = blockIdx.x * kActThreads + threadIdx.x;
-    BlockIn<kIn> nxt;
-    if (u < total) load_block_in<kIn>(x, offset(u, ld), nxt);
-    for (; u < total; u += stride) {
-        const BlockIn<kIn> cur = nxt;
-        if (u + stride < total) load_block_in<kIn>(x, offset(u + stride, ld), nxt);
-        float xv[16];
-        const uint32_t ab = unpack_block<kIn>(cur, xv);
-        if (ab >= 0x7F800000u) flags |= kFlagNonFinite;
-        const float a_b = __uint_as_float(ab);
+        const float s2 = __fdiv_rn(*p.jobs[j].d_amax, 2688.0f);  // RN32(amax / (6*448))
+        if (t0 == tb && threadIdx.x == 0) *p.jobs[j].d_s2 = s2;
+        const bool fast_scale = s2 >= kTinyScale && s2 <= 0x1p100f;
+        const float k = __frcp_rn(__fmul_rn(6.0f, s2));           // ~ 1/(6*s2)
+        const float k_lo = __fmul_rn(k, kLoMargin), k_hi = __fmul_rn(k, kHiMargin);
+        const float rs2 = __frcp_rn(s2);                          // ~ 1/s2
+        if (!isfinite(s2)) flags |= kFlagOverflow;
 
-        // block scale: nearest E4M3 to a_b / (6*s2)
-        uint32_t code;
-        if (fast_scale) {
-            const uint32_t cc = cvt_e4m3x2(__fmul_rn(a_b, k_lo), __fmul_rn(a_b, k_hi));
-            code = cc & 0xFFu;
-            if (code != (cc >> 8)) code = e4m3_fix(code, a_b, s2);
-        } else {
-            code = e4m3_code_exact(a_b, s2);
-        }
-        code &= 0x7Fu;                                            // non-negative inputs only
-        const float S = __fmul_rn(tab.dec[code], s2);            // DQ1: RN32(s_b * s2)
+        const uint32_t stride = G * kActThreads;
+        BlockIn<kIn> nxt;
+        if (u < units) load_block_in<kIn>(x, offset(u, ld), nxt);
+        for (; u < units; u += stride) {
+            const BlockIn<kIn> blk = nxt;
+            if (u + stride < units) load_block_in<kIn>(x, offset(u + stride, ld), nxt);
+            float xv[16];
+            const uint32_t ab = unpack_block<kIn>(blk, xv);
+            if (ab >= 0x7F800000u) flags |= kFlagNonFinite;
+            const float a_b = __uint_as_float(ab);
 
-        const bool exact = S != 0.0f && !(S >= kTinyScale && S <= 0x1p100f);
-        const float rr = S == 0.0f ? 0.0f : __fmul_rn(tab.rcp[code], rs2);   // ~ 1/S
-        uint32_t q0, q1;
-        quantize16(xv, S, __fmul_rn(rr, kLoMargin), __fmul_rn(rr, kHiMargin), exact, q0, q1);
+            // block scale: nearest E4M3 to a_b / (6*s2)
+            uint32_t code;
+            if (fast_scale) {
+                const uint32_t cc = cvt_e4m3x2(__fmul_rn(a_b, k_lo), __fmul_rn(a_b, k_hi));
+                code = cc & 0xFFu;
+                if (code != (cc >> 8)) code = e4m3_fix(code, a_b, s2);
+            } else {
+                code = e4m3_code_exact(a_b, s2);
+            }
+            code &= 0x7Fu;                                        // non-negative inputs only
+            const float S = __fmul_rn(tab.dec[code], s2);        // DQ1: RN32(s_b * s2)
 
-        if constexpr (kOut < 0) {
-            *reinterpret_cast<uint2*>(q + (int64_t)u * 8) = make_uint2(q0, q1);
-            scales[u] = (uint8_t)code;
-        } else {
-            store_qdq<kOut>(q0, q1, S, out, offset(u, ld_out));
+            const bool exact = S != 0.0f && !(S >= kTinyScale && S <= 0x1p100f);
+            const float rr = S == 0.0f ? 0.0f : __fmul_rn(tab.rcp[code], rs2);   // ~ 1/S
+            uint32_t q0, q1;
+            quantize16(xv, S, __fmul_rn(rr, kLoMargin), __fmul_rn(rr, kHiMargin), exact, q0, q1);
+
+            if constexpr (kOut < 0) {
+                *reinterpret_cast<uint2*>(q + (int64_t)u * 8) = make_uint2(q0, q1);
+                scales[u] = (uint8_t)code;
+            } else {
+                store_qdq<kOut>(q0, q1, S, out, offset(u, ld_out));
+            }
         }
     }
-    flags = __reduce_or_sync(__activemask(), flags);
-    if ((threadIdx.x & 31) == 0) flag_or(d_flags, flags);
+    flags = __reduce_or_sync(0xFFFFFFFFu, flags);
+    if ((threadIdx.x & 31) == 0 && flags) flag_or(p.d_flags, flags);
 }
 
 // ============================================================== dequant
@@ -367,71 +447,116 @@ __device__ __forceinline__ void dequant8(uint32_t qw, uint32_t sc, float s2, voi
     }
 }
 
+// Jobs: tiles of kDeqTile half-blocks, each in one job; a CTA strides over the tiles of
+// all jobs, four half-blocks per thread in flight.
+constexpr uint32_t kDeqTile = kActThreads * 4;
+
+struct DeqJobDev {
+    const uint32_t* qw;
+    const uint8_t* scales;
+    const float* d_s2;
+    void* out;
+    uint32_t halves, tile_begin;
+};
+
+struct DeqParams {
+    int n;
+    uint32_t tiles;
+    DeqJobDev jobs[kMaxActJobs];
+};
+
 template <int kOut>   // 0 bf16, 1 fp16, 2 fp32
 __global__ void __launch_bounds__(kActThreads)
-dequant_kernel(const uint8_t* __restrict__ q, const uint8_t* __restrict__ scales, const float* __restrict__ d_s2,
-               uint32_t total, void* __restrict__ out)
+dequant_kernel(const __grid_constant__ DeqParams p)
 {
-    const float s2 = *d_s2;
-    const uint32_t halves = 2u * total;
-    const uint32_t stride = gridDim.x * kActThreads;
-    const uint32_t* qw = reinterpret_cast<const uint32_t*>(q);
-    uint32_t h = blockIdx.x * kActThreads + threadIdx.x;
-    for (; h + 3u * stride < halves; h += 4u * stride) {          // four independent steps in flight
+    int cur = -1;
+    float s2 = 0.0f;
+    for (uint32_t t = blockIdx.x; t < p.tiles; t += gridDim.x) {
+        const int j = job_of_tile(p, t);
+        const DeqJobDev& job = p.jobs[j];
+        if (j != cur) {
+            cur = j;
+            s2 = *job.d_s2;
+        }
+        const uint32_t base = (t - job.tile_begin) * kDeqTile + threadIdx.x;
         uint32_t a[4], c[4];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            a[k] = __ldcs(qw + h + k * stride);
-            c[k] = scales[(h + k * stride) >> 1];
+        for (int k = 0; k < 4; ++k) {                             // four independent steps in flight
+            const uint32_t h = base + k * kActThreads;
+            if (h < job.halves) {
+                a[k] = __ldcs(job.qw + h);
+                c[k] = job.scales[h >> 1];
+            }
         }
 #pragma unroll
-        for (int k = 0; k < 4; ++k) dequant8<kOut>(a[k], c[k], s2, out, h + k * stride);
+        for (int k = 0; k < 4; ++k) {
+            const uint32_t h = base + k * kActThreads;
+            if (h < job.halves) dequant8<kOut>(a[k], c[k], s2, job.out, h);
+        }
     }
-    for (; h < halves; h += stride) dequant8<kOut>(__ldcs(qw + h), scales[h >> 1], s2, out, h);
 }
 
 // ============================================================== launchers
-static int grid_for(int64_t work, int threads, int per_sm)
+static int grid_for(int64_t work, int per_sm)
 {
-    const int64_t need = (work + threads - 1) / threads;
     const int64_t cap = (int64_t)num_sms() * per_sm;
-    return (int)(need < cap ? (need > 0 ? need : 1) : cap);
+    return (int)(work < cap ? (work > 0 ? work : 1) : cap);
 }
 
-cudaError_t launch_amax(const void* x, int dt, int64_t n, float* d_amax, uint32_t* d_flags, cudaStream_t s)
+cudaError_t launch_amax(const AmaxTask* tasks, int n, int dt, uint32_t* d_flags, cudaStream_t s)
 {
-    constexpr int T = 512;
-    if (dt == 0) {
-        const int64_t nvec = n / 8;
-        const int ntail = (int)(n - nvec * 8);
-        const uint16_t* tail = static_cast<const uint16_t*>(x) + nvec * 8;
-        amax_bf16_kernel<T><<<grid_for(nvec, T, 4), T, 0, s>>>(static_cast<const uint4*>(x), nvec, tail, ntail,
-                                                                 d_amax, d_flags);
-    } else {
-        const int64_t nvec = n / 4;
-        const int ntail = (int)(n - nvec * 4);
-        const uint32_t* tail = static_cast<const uint32_t*>(x) + nvec * 4;
-        amax_f32_kernel<T><<<grid_for(nvec, T, 4), T, 0, s>>>(static_cast<const uint4*>(x), nvec, tail, ntail,
-                                                                d_amax, d_flags);
+    AmaxParams p;
+    p.d_flags = d_flags;
+    const int64_t per_vec = dt == 0 ? 8 : 4;                    // elements per 16-byte vector
+    int m = 0;
+    uint32_t tiles = 0;
+    for (int i = 0; i < n; ++i) {
+        const AmaxTask& T = tasks[i];
+        if (T.n == 0) continue;
+        AmaxJobDev& d = p.jobs[m++];
+        d.x = static_cast<const uint4*>(T.x);
+        d.nvec = T.n / per_vec;
+        d.ntail = (int)(T.n - d.nvec * per_vec);
+        d.tail = static_cast<const char*>(T.x) + d.nvec * 16;
+        d.d_amax = T.d_amax;
+        d.tile_begin = tiles;
+        const int64_t nt = (d.nvec + kAmaxTile - 1) / kAmaxTile;
+        tiles += (uint32_t)(nt > 0 ? nt : 1);
+        d.tile_end = tiles;
     }
+    p.n = m;
+    p.tiles = tiles;
+    if (m == 0) return cudaSuccess;
+    const int g = grid_for(tiles, 4);
+    if (dt == 0) amax_kernel<0><<<g, kAmaxThreads, 0, s>>>(p);
+    else amax_kernel<2><<<g, kAmaxThreads, 0, s>>>(p);
     return cudaGetLastError();
 }
 
-cudaError_t launch_act_quant(const void* x, int64_t rows, int64_t cols, int64_t ld, const float* d_amax,
-                             uint8_t* q, uint8_t* scales, float* d_s2, uint32_t* d_flags, cudaStream_t s)
+cudaError_t launch_block_quant(const QuantTask* tasks, int n, int in_dt, int out_dt, uint32_t* d_flags,
+                               cudaStream_t s)
 {
-    return launch_block_quant(x, 0, rows, cols, ld, d_amax, q, scales, -1, nullptr, 0, d_s2, d_flags, s);
-}
-
-cudaError_t launch_block_quant(const void* x, int in_dt, int64_t rows, int64_t cols, int64_t ld,
-                               const float* d_amax, uint8_t* q, uint8_t* scales, int out_dt, void* out,
-                               int64_t ld_out, float* d_s2, uint32_t* d_flags, cudaStream_t s)
-{
-    const uint32_t bpr = (uint32_t)(cols / 16);
-    const uint32_t total = (uint32_t)rows * bpr;
-    const int g = grid_for(total, kActThreads, 8);
-#define NV4_BQ(I, O) act_quant_kernel<I, O><<<g, kActThreads, 0, s>>>(x, (uint32_t)rows, bpr, ld, FastDiv(bpr), \
-        d_amax, q, scales, out, ld_out, d_s2, d_flags)
+    QuantParams p;
+    p.d_flags = d_flags;
+    int m = 0;
+    uint32_t tiles = 0;
+    for (int i = 0; i < n; ++i) {
+        const QuantTask& T = tasks[i];
+        if (T.rows == 0 || T.cols == 0) continue;
+        QuantJobDev& d = p.jobs[m++];
+        d.x = T.x; d.out = T.out; d.q = T.q; d.scales = T.scales; d.d_amax = T.d_amax; d.d_s2 = T.d_s2;
+        d.ld = T.ld; d.ld_out = T.ld_out;
+        d.bpr = (uint32_t)(T.cols / 16);
+        d.div_bpr = FastDiv(d.bpr);
+        d.units = (uint32_t)T.rows * d.bpr;
+        d.tile_begin = tiles;
+        tiles += (d.units + kActThreads - 1) / kActThreads;
+    }
+    p.n = m;
+    p.tiles = tiles;
+    if (m == 0) return cudaSuccess;
+    const int g = grid_for(tiles, 8);
+#define NV4_BQ(I, O) act_quant_kernel<I, O><<<g, kActThreads, 0, s>>>(p)
     if (in_dt == 0) {
         if (out_dt < 0) NV4_BQ(0, -1); else if (out_dt == 0) NV4_BQ(0, 0); else if (out_dt == 1) NV4_BQ(0, 1); else NV4_BQ(0, 2);
     } else {
@@ -441,14 +566,30 @@ cudaError_t launch_block_quant(const void* x, int in_dt, int64_t rows, int64_t c
     return cudaGetLastError();
 }
 
-cudaError_t launch_dequant(const uint8_t* q, const uint8_t* scales, const float* d_s2, int64_t rows, int64_t cols,
-                           int out_dt, void* out, cudaStream_t s)
+cudaError_t launch_dequant(const DequantTask* tasks, int n, int out_dt, cudaStream_t s)
 {
-    const uint32_t total = (uint32_t)(rows * (cols / 16));
-    const int g = grid_for((int64_t)total * 2, kActThreads, 8);
-    if (out_dt == 0) dequant_kernel<0><<<g, kActThreads, 0, s>>>(q, scales, d_s2, total, out);
-    else if (out_dt == 1) dequant_kernel<1><<<g, kActThreads, 0, s>>>(q, scales, d_s2, total, out);
-    else dequant_kernel<2><<<g, kActThreads, 0, s>>>(q, scales, d_s2, total, out);
+    DeqParams p;
+    int m = 0;
+    uint32_t tiles = 0;
+    for (int i = 0; i < n; ++i) {
+        const DequantTask& T = tasks[i];
+        if (T.rows == 0 || T.cols == 0) continue;
+        DeqJobDev& d = p.jobs[m++];
+        d.qw = reinterpret_cast<const uint32_t*>(T.q);
+        d.scales = T.scales;
+        d.d_s2 = T.d_s2;
+        d.out = T.out;
+        d.halves = (uint32_t)(2 * T.rows * (T.cols / 16));
+        d.tile_begin = tiles;
+        tiles += (d.halves + kDeqTile - 1) / kDeqTile;
+    }
+    p.n = m;
+    p.tiles = tiles;
+    if (m == 0) return cudaSuccess;
+    const int g = grid_for(tiles, 8);
+    if (out_dt == 0) dequant_kernel<0><<<g, kActThreads, 0, s>>>(p);
+    else if (out_dt == 1) dequant_kernel<1><<<g, kActThreads, 0, s>>>(p);
+    else dequant_kernel<2><<<g, kActThreads, 0, s>>>(p);
     return cudaGetLastError();
 }
 

@@ -31,7 +31,8 @@ def test_header_declares_the_hot_path():
               "nv4_mxfp4_to_nvfp4", "nv4_weight_quant_rtn", "nv4_fake_qdq", "nv4_gemm_nvfp4",
               "nv4_scales_to_mma_layout", "nv4_mma_scale_bytes", "nv4_mxfp4_quant", "nv4_mxfp4_dequant",
               "nv4_fp8_quant", "nv4_fp8_dequant", "nv4_hadamard_amax", "nv4_hadamard_mxfp4_quant",
-              "nv4_hadamard_nvfp4_quant", "nv4_selftest_wait"):
+              "nv4_hadamard_nvfp4_quant", "nv4_selftest_wait", "nv4_tensor_amax_batched", "nv4_act_quant_batched",
+              "nv4_dequant_batched"):
         assert n in names
 
 
@@ -121,6 +122,36 @@ def test_validation_rejects_before_any_launch(nv4lib):
 
     jobs = (b.HessianJob * 129)()
     assert L.nv4_hessian_accum_batched(jobs, 129, None, None) == 6                         # > 128 jobs
+
+
+def test_batched_act_path_validation(nv4lib):
+    """The batched amax / act quant / dequant entries apply the single-tensor rules to
+    every job and reject the call before any launch."""
+    from nvfp4_block_numerics_b200 import binding as b
+
+    L, fake = nv4lib, 0x1000
+    am = (b.AmaxJob * 2)(b.AmaxJob(fake, 64, fake), b.AmaxJob(fake + 4, 64, fake))
+    assert L.nv4_tensor_amax_batched(am, 2, 0, None, None) == 3          # second x misaligned
+    assert L.nv4_tensor_amax_batched(am, 1, 1, None, None) == 4          # fp16
+    assert L.nv4_tensor_amax_batched(am, -1, 0, None, None) == 2
+    assert L.nv4_tensor_amax_batched(None, 2, 0, None, None) == 1
+    assert L.nv4_tensor_amax_batched(None, 0, 0, None, None) == 0        # no-op
+    big = (b.AmaxJob * 129)()
+    assert L.nv4_tensor_amax_batched(big, 129, 0, None, None) == 6       # > 128 jobs
+    am2 = (b.AmaxJob * 1)(b.AmaxJob(fake, 1 << 37, fake))
+    assert L.nv4_tensor_amax_batched(am2, 1, 0, None, None) == 6         # n >= 2^37
+    aj = (b.ActJob * 2)(b.ActJob(fake, 4, 32, 32, fake, fake, fake, fake), b.ActJob(fake, 4, 24, 24, fake, fake, fake, fake))
+    assert L.nv4_act_quant_batched(aj, 2, None, None) == 2               # second: cols % 16
+    aj[1] = b.ActJob(fake, 4, 32, 36, fake, fake, fake, fake)
+    assert L.nv4_act_quant_batched(aj, 2, None, None) == 3               # second: ld*2 % 16
+    aj[1] = b.ActJob(fake, 4, 32, 32, None, fake, fake, fake)
+    assert L.nv4_act_quant_batched(aj, 2, None, None) == 1               # second: amax
+    assert L.nv4_act_quant_batched((b.ActJob * 129)(), 129, None, None) == 6
+    dj = (b.DequantJob * 2)(b.DequantJob(fake, fake, fake, 4, 32, fake), b.DequantJob(fake, fake, fake, 4, 32, fake + 8))
+    assert L.nv4_dequant_batched(dj, 2, 0, None) == 3                    # second out misaligned
+    assert L.nv4_dequant_batched(dj, 1, 7, None) == 4                    # out dtype
+    dj[1] = b.DequantJob(fake, fake, None, 4, 32, fake)
+    assert L.nv4_dequant_batched(dj, 2, 0, None) == 1
 
 
 def fastdiv_params(d):

@@ -120,6 +120,79 @@ def test_act_quant_config_shapes(orc, T, C):
     _act_check(orc, x, rows_sample=sample)
 
 
+def test_act_path_batched_matches_single_and_oracle(orc):
+    """The batched amax, act quant and dequant entries over the 15 activation shapes
+    (rows capped at 300 so the oracle checks every row), one of them strided and one
+    empty: bit for bit the single-tensor calls and the oracle."""
+    xs = [inputs.c2_shape(min(T, 300), C) for (T, C) in inputs.C2_SHAPES]
+    xs[4] = xs[4].copy()
+    xs[4][7, 100] = 0x7FC0                                   # a NaN: skipped by the amax, flagged
+    dev = []
+    for i, x in enumerate(xs):
+        if i == 7:                                           # rows of a wider buffer (ld > cols)
+            buf = np.zeros((x.shape[0], x.shape[1] + 64), np.uint16)
+            buf[:, :x.shape[1]] = x
+            dev.append(G.bf16_dev(buf)[:, :x.shape[1]])
+        else:
+            dev.append(G.bf16_dev(x))
+    empty = torch.empty((0, 64), dtype=torch.bfloat16, device=G.DEV)
+    n = len(xs)
+
+    def outputs():
+        return ([torch.empty((x.shape[0], x.shape[1] // 2), dtype=torch.uint8, device=G.DEV) for x in xs],
+                [torch.empty((x.shape[0], x.shape[1] // 16), dtype=torch.uint8, device=G.DEV) for x in xs],
+                [torch.empty(tuple(x.shape), dtype=torch.bfloat16, device=G.DEV) for x in xs])
+
+    # batched (the amax needs contiguous tensors: the strided one goes through its copy)
+    fb = G.flags_dev()
+    am_b, s2_b = torch.zeros(n + 1, device=G.DEV), torch.zeros(n + 1, device=G.DEV)
+    qb, scb, ob = outputs()
+    nv4.nv4_tensor_amax_batched([d.contiguous() for d in dev] + [empty], [am_b[i:i + 1] for i in range(n + 1)], fb)
+    nv4.nv4_act_quant_batched([dict(x=dev[i], d_amax=am_b[i:i + 1], q=qb[i], scales=scb[i], d_s2=s2_b[i:i + 1])
+                               for i in range(n)], fb)
+    nv4.nv4_dequant_batched([dict(q=qb[i], scales=scb[i], d_s2=s2_b[i:i + 1], out=ob[i]) for i in range(n)])
+    # one call per tensor
+    fs = G.flags_dev()
+    am_s, s2_s = torch.zeros(n, device=G.DEV), torch.zeros(n, device=G.DEV)
+    qs, scs, os_ = outputs()
+    for i in range(n):
+        nv4.nv4_tensor_amax(dev[i].contiguous(), am_s[i:i + 1], fs)
+        nv4.nv4_act_quant(dev[i], am_s[i:i + 1], qs[i], scs[i], s2_s[i:i + 1], fs)
+        nv4.nv4_dequant(qs[i], scs[i], s2_s[i:i + 1], os_[i])
+    torch.cuda.synchronize()
+    assert fb.item() == fs.item() == nv4.FLAG_NONFINITE
+    assert am_b[n].item() == 0.0                             # the empty job
+    assert torch.equal(am_b[:n], am_s) and torch.equal(s2_b[:n], s2_s)
+    for i, x in enumerate(xs):
+        assert torch.equal(qb[i], qs[i]) and torch.equal(scb[i], scs[i]), i
+        assert torch.equal(ob[i].view(torch.int16), os_[i].view(torch.int16)), i      # bit patterns (NaN blocks)
+        amax, _ = orc.tensor_amax(x)
+        assert am_b[i].item() == amax, i
+        oq, osc, os2, _ = orc.act_quant(x, amax)
+        assert s2_b[i].item() == os2
+        gq, gsc, go, ro = G.host(qb[i]), G.host(scb[i]), G.host(ob[i]), orc.dequant(oq, osc, os2, "bf16")
+        if i == 4:                                           # the NaN block's outputs are unspecified
+            gq[7, 48:56] = oq[7, 48:56]
+            gsc[7, 6] = osc[7, 6]
+            go[7, 96:112] = ro[7, 96:112]
+        assert np.array_equal(gq, oq) and np.array_equal(gsc, osc), i
+        assert np.array_equal(go, ro), i
+
+
+def test_amax_batched_fp32_and_tails(orc):
+    r = np.random.default_rng(12)
+    xs = [(r.laplace(size=n) * 3).astype(np.float32) for n in (1, 3, 4, 5, 4096 * 4 + 3, 70001)]
+    xs[3][2] = np.float32(np.inf)
+    d = [G.f32_dev(x) for x in xs]
+    am = torch.zeros(len(xs), device=G.DEV)
+    f = G.flags_dev()
+    nv4.nv4_tensor_amax_batched(d, [am[i:i + 1] for i in range(len(xs))], f)
+    torch.cuda.synchronize()
+    assert f.item() == nv4.FLAG_NONFINITE
+    for i, x in enumerate(xs):
+        assert am[i].item() == orc.tensor_amax(x)[0], i
+
+
 def test_dequant_random_codes(orc):
     rng = np.random.default_rng(3)
     q = rng.integers(0, 256, (33, 40), dtype=np.uint8)

@@ -212,8 +212,7 @@ def part_calib(W):
     W["Hd"].zero_()
     W["amax_w"].zero_()
     nv4.nv4_hessian_accum_batched([W["X"], W["Xd"]], [W["H"], W["Hd"]], W["flags"])
-    for j in W["weights"]:
-        nv4.nv4_tensor_amax(j["w"], j["d_amax_w"], W["flags"])
+    nv4.nv4_tensor_amax_batched([j["w"] for j in W["weights"]], [j["d_amax_w"] for j in W["weights"]], W["flags"])
     # the production call: winning codes and packed E2M1 nibbles (no cost diagnostics)
     nv4.nv4_scale_sweep_batched([{k: j[k] for k in ("w", "H", "d_amax_w", "codes", "q")}
                                  for j in W["weights"]], W["flags"])
@@ -227,7 +226,7 @@ def part_cast(W):
 
 
 PARTS = {"act": part_act, "calib": part_calib, "cast": part_cast}
-LAUNCHES = {"act": 3, "calib": 6, "cast": 2}
+LAUNCHES = {"act": 3, "calib": 3, "cast": 2}
 
 
 def traffic_table():

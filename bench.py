@@ -44,9 +44,13 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "NVFP4 quant GB/s (% HBM peak); scale-sweep blocks/s (% FP32 peak)"
-SWEEP_FLOP_PER_BLOCK = 127 * 300          # exhaustive count: 127 x (136-FMA quadratic form + dequant/subtract)
-SWEEP_FLOP_PER_VISIT = 80                 # per visited candidate: e = w - v*S (16 FMA) + bound sum rd*e^2 (16 x 3)
-SWEEP_FLOP_PER_COST = 272                 # per evaluated cost: the 136-entry symmetric quadratic form
+# Algorithmic FP32 work of the sweep, per 16-element block and candidate scale S:
+#   w/S for the E2M1 rounding (16), e = w - v*S (16 FMA = 32), bound sum rd*e^2 (16 x 3 = 48)
+#   and the 136-entry symmetric quadratic form (272).  The second end of the rounding
+#   bracket and the conversions are implementation work and not counted.
+SWEEP_FLOP_PER_VISIT = 16 + 32 + 48       # per visited candidate
+SWEEP_FLOP_PER_COST = 272                 # per evaluated cost
+SWEEP_FLOP_PER_BLOCK = 127 * (16 + 32 + 272)   # exhaustive count: every candidate's quotient, e and cost
 ACT_BYTES = {"amax": 2.0, "act_quant": 2.5625, "dequant": 2.5625}
 CAST_BYTES_PER_MX_BLOCK = 1 + 16 + 16 + 2  # read E8M0 + nibbles, write nibbles + 2 E4M3 scales
 FP32_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12   # SMs x FP32 lanes x FMA x max clock
@@ -689,8 +693,8 @@ def run_ours(args):
                  "visits_per_block": sw["visits_per_block"], "costs_per_block": sw["costs_per_block"],
                  "exhaustive_equiv_tflops": sw["exhaustive_equiv_tflops"],
                  "note_work": "exact branch and bound over the 127 codes: achieved counts the FLOPs of the "
-                              "candidates visited and costs evaluated (device counters); exhaustive_equiv "
-                              "counts 127 x 300 FLOP per block"}
+                              "candidates visited (96 each) and costs evaluated (272 each), from device "
+                              "counters; exhaustive_equiv counts 127 x 320 FLOP per block"}
     # dominant kernel: the largest device time per step (every in-step row times the step's
     # own launch, which runs once per step)
     in_step = [k for k in roof if roof[k].get("in_step", True)]

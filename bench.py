@@ -46,9 +46,11 @@ sys.path.insert(0, ROOT)
 METRIC = "NVFP4 quant GB/s (% HBM peak); scale-sweep blocks/s (% FP32 peak)"
 # Algorithmic FP32 work of the sweep, per 16-element block and candidate scale S:
 #   w/S for the E2M1 rounding (16), e = w - v*S (16 FMA = 32), bound sum rd*e^2 (16 x 3 = 48)
-#   and the 136-entry symmetric quadratic form (272).  The second end of the rounding
-#   bracket and the conversions are implementation work and not counted.
-SWEEP_FLOP_PER_VISIT = 16 + 32 + 48       # per visited candidate
+#   and the 136-entry symmetric quadratic form (272).  The kernel visits a candidate in
+#   halves of 8 elements (48 FLOP each; the second half only when the first does not rule
+#   the candidate out).  The second end of the rounding bracket and the conversions are
+#   implementation work and not counted.
+SWEEP_FLOP_PER_HALF = 8 + 16 + 24         # per visited candidate half
 SWEEP_FLOP_PER_COST = 272                 # per evaluated cost
 SWEEP_FLOP_PER_BLOCK = 127 * (16 + 32 + 272)   # exhaustive count: every candidate's quotient, e and cost
 ACT_BYTES = {"amax": 2.0, "act_quant": 2.5625, "dequant": 2.5625}
@@ -368,10 +370,10 @@ def kernel_rooflines(W, hbm_peak):
         work = torch.zeros(2, dtype=torch.int64, device=W["flags"].device)
         nv4.nv4_scale_sweep_batched([dict(j, d_work=work) for j in jobs], W["flags"])
         torch.cuda.synchronize()
-        visits, costs = (int(x) for x in work.tolist())
+        halves, costs = (int(x) for x in work.tolist())
         t = time_launch(lambda: nv4.nv4_scale_sweep_batched(jobs, W["flags"]), reps=5)
-        out["scale_sweep"] = {"bound": "alu", "flops": SWEEP_FLOP_PER_VISIT * visits + SWEEP_FLOP_PER_COST * costs,
-                              "blocks": blocks, "s": t, "visits_per_block": visits / blocks,
+        out["scale_sweep"] = {"bound": "alu", "flops": SWEEP_FLOP_PER_HALF * halves + SWEEP_FLOP_PER_COST * costs,
+                              "blocks": blocks, "s": t, "half_visits_per_block": halves / blocks,
                               "costs_per_block": costs / blocks,
                               "exhaustive_equiv_tflops": SWEEP_FLOP_PER_BLOCK * blocks / t / 1e12,
                               "launch": "q_proj + gate + up + down, one batched launch"}
@@ -690,10 +692,10 @@ def run_ours(args):
                  "note": "blocks over the whole calib part (Hessians + amax + sweep)",
                  "kernel_blocks_per_s": sw["blocks_per_s"], "kernel_tflops_executed": sw["achieved"],
                  "frac_fp32": sw["frac"], "fp32_peak_tflops": FP32_PEAK_TFLOPS,
-                 "visits_per_block": sw["visits_per_block"], "costs_per_block": sw["costs_per_block"],
+                 "half_visits_per_block": sw["half_visits_per_block"], "costs_per_block": sw["costs_per_block"],
                  "exhaustive_equiv_tflops": sw["exhaustive_equiv_tflops"],
                  "note_work": "exact branch and bound over the 127 codes: achieved counts the FLOPs of the "
-                              "candidates visited (96 each) and costs evaluated (272 each), from device "
+                              "candidate halves visited (48 each) and costs evaluated (272 each), from device "
                               "counters; exhaustive_equiv counts 127 x 320 FLOP per block"}
     # dominant kernel: the largest device time per step (every in-step row times the step's
     # own launch, which runs once per step)

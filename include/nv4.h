@@ -251,7 +251,9 @@ NV4_API nv4_status nv4_hessian_accum_batched(const nv4_hessian_job* jobs, int n_
  * lower bound proves cannot be the winner or, when cost2 is requested, the runner-up
  * (sweep.cu states the bounds): codes and q are the same with or without the cost
  * outputs, and cheapest without cost2.  The optional per-job work counter reports
- * how many candidates were visited and evaluated.
+ * how much of the search ran: candidate halves (8 elements each: a candidate is visited
+ * half by half and its second half only when the first does not rule it out) and
+ * quadratic forms evaluated.
  */
 NV4_API nv4_status nv4_scale_sweep(const void* w, nv4_dtype dt, int64_t rows, int64_t cols, int64_t ld,
                            const float* H, const float* d_amax_w, uint8_t* codes, uint8_t* q,
@@ -266,7 +268,8 @@ typedef struct {
     uint8_t* q;         /* [rows, cols/2] or NULL */
     float* cost1;       /* or NULL */
     float* cost2;       /* or NULL */
-    unsigned long long* d_work;  /* or NULL: [0] += candidates visited, [1] += costs evaluated */
+    unsigned long long* d_work;  /* or NULL: [0] += half-candidates visited (8 elements each),
+                                    [1] += costs evaluated */
 } nv4_sweep_job;
 
 /* Batched form (e.g. all gate/up/down matrices of an expert stack) in one launch.

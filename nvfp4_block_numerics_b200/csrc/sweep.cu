@@ -9,7 +9,9 @@
 // scales S_c (and the reciprocal brackets used to round w/S_c) depend only on the
 // matrix's s2; they sit in a shared-memory table.
 //
-// Per visited candidate, per thread (all FP32; pairs use the packed FP32 instructions):
+// Per visited candidate, per thread (all FP32; pairs use the packed FP32 instructions),
+// in two halves of 8 elements -- the second half only when the first half's part of
+// bound (1) below does not already rule the candidate out:
 //   E2M1 codes of w/S_c : bracketed hardware conversion; near a rounding boundary
 //                         one exact FMA comparison fixes the code (nv4_common.cuh)
 //   e_i = w_i - v_i*S_c   (one rounding of the exact difference)
@@ -67,46 +69,6 @@ struct SweepParams {
     uint32_t* d_flags;
     SweepJobDev jobs[kMaxSweepJobs];
 };
-
-// E2M1 codes of the 16 weights w (as 8 pairs) at candidate t = {S, r_lo, r_hi, exact}.
-__device__ __forceinline__ void codes16(const float2 w[8], const float4& t, uint32_t& c0, uint32_t& c1)
-{
-    if (t.w == 0.0f) {
-        const float2 rl = make_float2(t.y, t.y), rh = make_float2(t.z, t.z);
-        float lo[16], hi[16];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const float2 a = __fmul2_rn(w[j], rl), b = __fmul2_rn(w[j], rh);
-            lo[2 * j] = a.x; lo[2 * j + 1] = a.y;
-            hi[2 * j] = b.x; hi[2 * j + 1] = b.y;
-        }
-        c0 = cvt_e2m1x8(lo);
-        c1 = cvt_e2m1x8(lo + 8);
-        const uint32_t h0 = cvt_e2m1x8(hi), h1 = cvt_e2m1x8(hi + 8);
-        if (c0 != h0 || c1 != h1) {          // near a rounding boundary: exact FP32 fix-up
-            float x[16];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) { x[2 * j] = w[j].x; x[2 * j + 1] = w[j].y; }
-            if (c0 != h0) c0 = e2m1_fix8(x, t.x, c0, h0);
-            if (c1 != h1) c1 = e2m1_fix8(x + 8, t.x, c1, h1);
-        }
-        return;
-    }
-    // S outside [2^-100, 2^100] (degenerate second-level scale): exact FP64 decisions
-    c0 = c1 = 0u;
-    for (int i = 0; i < 8; ++i) c0 |= e2m1_code_exact(i & 1 ? w[i >> 1].y : w[i >> 1].x, t.x) << (4 * i);
-    for (int i = 0; i < 8; ++i) c1 |= e2m1_code_exact(i & 1 ? w[4 + (i >> 1)].y : w[4 + (i >> 1)].x, t.x) << (4 * i);
-}
-
-// Signed E2M1 values of the packed codes, as 8 pairs.
-__device__ __forceinline__ void decode16(uint32_t c0, uint32_t c1, float2 v[8])
-{
-    uint32_t h[8];
-    cvt_e2m1x8_to_f16x8(c0, h);
-    cvt_e2m1x8_to_f16x8(c1, h + 4);
-#pragma unroll
-    for (int j = 0; j < 8; ++j) f16x2_to_f32(h[j], v[j].x, v[j].y);
-}
 
 // Shared-memory image of one H_b for the row-pair quadratic form: for rows (2m, 2m+1)
 // one float4 {H_2m,2m, H_2m+1,2m+1, H'_2m,2m+1, 0} then, for k = 2m+2, 2m+4, ..., 14,
@@ -185,12 +147,49 @@ __device__ void block_bound(const float* __restrict__ hs, float* rd, int* ok)
     if (lane == 0) *ok = good ? 1 : 0;
 }
 
-// Lower bound (1) for the error vector e: sum_i rd_i e_i^2.
-__device__ __forceinline__ float bound_diag(const float2 e[8], const float4* __restrict__ rd4)
+// E2M1 codes of 8 weights (4 pairs) at candidate t = {S, r_lo, r_hi, exact}: both ends of
+// the bracket converted, an exact FP32 fix-up where they disagree; S outside
+// [2^-100, 2^100] (a degenerate second-level scale) takes the exact FP64 decisions.
+__device__ __forceinline__ void codes8h(const float2 w[4], const float4& t, uint32_t& c)
+{
+    if (t.w == 0.0f) {
+        const float2 rl = make_float2(t.y, t.y), rh = make_float2(t.z, t.z);
+        float lo[8], hi[8];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float2 a = __fmul2_rn(w[j], rl), b = __fmul2_rn(w[j], rh);
+            lo[2 * j] = a.x; lo[2 * j + 1] = a.y;
+            hi[2 * j] = b.x; hi[2 * j + 1] = b.y;
+        }
+        c = cvt_e2m1x8(lo);
+        const uint32_t h = cvt_e2m1x8(hi);
+        if (c != h) {                        // near a rounding boundary: exact FP32 fix-up
+            float x[8];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) { x[2 * j] = w[j].x; x[2 * j + 1] = w[j].y; }
+            c = e2m1_fix8(x, t.x, c, h);
+        }
+        return;
+    }
+    c = 0u;
+    for (int i = 0; i < 8; ++i) c |= e2m1_code_exact(i & 1 ? w[i >> 1].y : w[i >> 1].x, t.x) << (4 * i);
+}
+
+// Signed E2M1 values of 8 packed codes, as 4 pairs.
+__device__ __forceinline__ void decode8h(uint32_t c, float2 v[4])
+{
+    uint32_t h[4];
+    cvt_e2m1x8_to_f16x8(c, h);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) f16x2_to_f32(h[j], v[j].x, v[j].y);
+}
+
+// Lower bound (1) over 8 elements: sum_i rd_i e_i^2 (rd4: their rho * H_ii).
+__device__ __forceinline__ float bound_half(const float2 e[4], const float4* __restrict__ rd4)
 {
     float2 acc = make_float2(0.0f, 0.0f);
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
+    for (int k = 0; k < 2; ++k) {
         const float4 d = rd4[k];
         acc = __ffma2_rn(__fmul2_rn(e[2 * k], make_float2(d.x, d.y)), e[2 * k], acc);
         acc = __ffma2_rn(__fmul2_rn(e[2 * k + 1], make_float2(d.z, d.w)), e[2 * k + 1], acc);
@@ -282,7 +281,7 @@ sweep_kernel(const __grid_constant__ SweepParams p)
     const float* rd = reinterpret_cast<const float*>(rd4);
     const uint32_t s2flag = isfinite(s2) ? 0u : kFlagOverflow;
 
-    uint32_t nvisit = 0u, nfull = 0u;
+    uint32_t nhalf = 0u, nfull = 0u;                     // half-visits (8 elements), quadratic forms
     // ---- load the group's rows (up to 4 tiles of 128), counting-sort them by starting code
     const uint32_t tile0 = group * p.tiles_per_cta;
     const uint32_t ntile = min(job.row_tiles - tile0, p.tiles_per_cta);
@@ -380,25 +379,41 @@ sweep_kernel(const __grid_constant__ SweepParams p)
 #pragma unroll 1
             while (c >= 0) {
                 const float4 t = tab[c];
-                uint32_t c0, c1;
-                codes16(w, t, c0, c1);
-                float2 v[8], e[8];
-                decode16(c0, c1, v);
                 const float2 nS = make_float2(-t.x, -t.x);
+                float2 e[8];
+                // first half (elements 0..7): codes, e and its part of bound (1)
+                uint32_t c0, c1 = 0u;
+                codes8h(w, t, c0);
+                {
+                    float2 v[4];
+                    decode8h(c0, v);
 #pragma unroll
-                for (int k = 0; k < 8; ++k) e[k] = __ffma2_rn(v[k], nS, w[k]);     // w - v*S, one rounding
-                ++nvisit;
-                if (!pr || !(bound_diag(e, rd4) * kPruneScale > thr)) {
-                    ++nfull;
-                    const float cost = quad_form(e, hp);
-                    if (cost < best || (cost == best && (uint32_t)c < best_c)) {
-                        if (cost < best) second = best;
-                        best = cost;
-                        best_c = (uint32_t)c;
-                    } else if (cost > best && cost < second) {
-                        second = cost;
+                    for (int k = 0; k < 4; ++k) e[k] = __ffma2_rn(v[k], nS, w[k]);
+                }
+                float lb = bound_half(e, rd4);
+                ++nhalf;
+                if (!pr || !(lb * kPruneScale > thr)) {               // the second half is still needed
+                    ++nhalf;
+                    codes8h(w + 4, t, c1);
+                    {
+                        float2 v[4];
+                        decode8h(c1, v);
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) e[4 + k] = __ffma2_rn(v[k], nS, w[4 + k]);
                     }
-                    thr = need2 ? second : best;
+                    lb += bound_half(e + 4, rd4 + 2);
+                    if (!pr || !(lb * kPruneScale > thr)) {
+                        ++nfull;
+                        const float cost = quad_form(e, hp);
+                        if (cost < best || (cost == best && (uint32_t)c < best_c)) {
+                            if (cost < best) second = best;
+                            best = cost;
+                            best_c = (uint32_t)c;
+                        } else if (cost > best && cost < second) {
+                            second = cost;
+                        }
+                        thr = need2 ? second : best;
+                    }
                 }
                 // next candidate: alternate down / up; bound (2) closes the downward walk
                 bool take_dn = dn >= 0 && (go_dn || up > 126);
@@ -421,7 +436,9 @@ sweep_kernel(const __grid_constant__ SweepParams p)
         job.codes[blk] = (uint8_t)best_c;
         if (job.q != nullptr) {
             uint32_t c0, c1;
-            codes16(w, tab[best_c], c0, c1);
+            const float4 tw = tab[best_c];
+            codes8h(w, tw, c0);
+            codes8h(w + 4, tw, c1);
             *reinterpret_cast<uint2*>(job.q + blk * 8) = make_uint2(c0, c1);
         }
         if (job.cost1 != nullptr) job.cost1[blk] = best;
@@ -430,7 +447,7 @@ sweep_kernel(const __grid_constant__ SweepParams p)
     }
     if (job.d_work != nullptr) {
         __syncwarp();
-        const uint32_t sv = __reduce_add_sync(0xffffffffu, nvisit), sf = __reduce_add_sync(0xffffffffu, nfull);
+        const uint32_t sv = __reduce_add_sync(0xffffffffu, nhalf), sf = __reduce_add_sync(0xffffffffu, nfull);
         if ((threadIdx.x & 31) == 0 && sv != 0u) {
             atomicAdd(job.d_work, (unsigned long long)sv);
             atomicAdd(job.d_work + 1, (unsigned long long)sf);

@@ -534,7 +534,8 @@ def test_sweep_grouped_scale2(orc):
 
 def test_sweep_work_counter(orc):
     """Bounds on: far fewer than 127 costs per block; bounds off (correlated channels):
-    every candidate visited and evaluated; the winners match the oracle either way."""
+    every candidate visited (both halves) and evaluated; the winners match the oracle
+    either way."""
     rng = np.random.default_rng(78)
     x = rng.laplace(size=(2048, 32))
     x[:, 16:] = x[:, 16:17] + rng.standard_normal((2048, 16))       # correlated channels: rho < 0
@@ -568,8 +569,10 @@ def test_sweep_work_counter(orc):
     on, off, ln = work[0].cpu().numpy(), work[1].cpu().numpy(), lean.cpu().numpy()
     print("work with bounds", on, "without", off, "codes only", ln)
     assert ln[1] <= on[1] and ln[0] <= on[0]
-    assert off[0] == 127 * rows and off[1] == 127 * rows
-    assert on[1] <= on[0] <= 127 * rows and on[1] < 0.25 * 127 * rows
+    # bounds off: both halves of every candidate and every cost; on: a candidate's second
+    # half only when its first half leaves it open, a cost only when its whole bound does
+    assert off[0] == 2 * 127 * rows and off[1] == 127 * rows
+    assert on[1] <= on[0] / 2 <= on[0] <= 2 * 127 * rows and on[1] < 0.25 * 127 * rows
     ref = orc.scale_sweep(w, H.astype(np.float32).astype(np.float64), orc.tensor_amax(w)[0])
     cat = lambda k: np.concatenate([G.host(j[k]) for j in jobs], axis=1)
     st = G.sweep_parity(cat("codes"), cat("q"), cat("cost1"), ref, c2_gpu=cat("cost2"))

@@ -19,6 +19,7 @@
 //     warp, one element per lane.  Launched as a programmatic dependent of kernel 1, it
 //     copies the nibbles of each warp's first tiles while kernel 1 runs, then waits for
 //     kernel 1.
+#include "nv4_async.cuh"
 #include "nv4_common.cuh"
 #include "nv4_internal.h"
 
@@ -49,27 +50,6 @@ struct CastParams {
     CastJobDev jobs[kMaxCastJobs];
 };
 
-__device__ __forceinline__ uint32_t cluster_rank_c()
-{
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-    return r;
-}
-
-__device__ __forceinline__ void cluster_sync_c()
-{
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-
-__device__ __forceinline__ uint32_t ld_dsmem_u32(const uint32_t* local, uint32_t rank)
-{
-    uint32_t remote, v;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;"
-                 : "=r"(remote)
-                 : "r"((uint32_t)__cvta_generic_to_shared(local)), "r"(rank));
-    asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(remote) : "memory");
-    return v;
-}
 
 // 2^e as FP32 for e in [-149, 127] (exact; subnormal below -126).
 __device__ __forceinline__ float exp2_exact(int e)
@@ -171,7 +151,7 @@ cast_kmax_kernel(const __grid_constant__ CastParams p)
     // the rewrite kernel may start its set-up and first loads now; it waits for this
     // grid to complete before it reads scale_2
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    const uint32_t rank = cluster_rank_c();
+    const uint32_t rank = cluster_ctarank();
     const int set = blockIdx.x / kKmaxCluster;
     const int m0 = p.set_begin[set], m1 = p.set_begin[set + 1];
 
@@ -217,7 +197,7 @@ cast_kmax_kernel(const __grid_constant__ CastParams p)
         for (int w = 0; w < kKmaxThreads / 32; ++w) m = max(m, red[w]);
         cta_max = m;
     }
-    cluster_sync_c();
+    cluster_sync();
     if (rank == 0 && threadIdx.x < 32) {                           // one warp gathers the partial maxima
         uint32_t c = threadIdx.x < kKmaxCluster ? ld_dsmem_u32(&cta_max, threadIdx.x) : 0u;
         c = __reduce_max_sync(0xFFFFFFFFu, c);
@@ -230,7 +210,7 @@ cast_kmax_kernel(const __grid_constant__ CastParams p)
         }
         if (threadIdx.x == 0 && !isfinite(ga)) flags |= kFlagOverflow;
     }
-    cluster_sync_c();                                               // all remote reads done
+    cluster_sync();                                               // all remote reads done
     flags = __reduce_or_sync(0xFFFFFFFFu, flags);
     if ((threadIdx.x & 31) == 0) flag_or(p.d_flags, flags);
 }

@@ -1,5 +1,5 @@
-// nv4_async.cuh -- shared-memory mbarriers and the copy engine's bulk and tensor loads
-// (sm_90+/sm_100a), used by the pipelined kernels.
+// nv4_async.cuh -- shared-memory mbarriers, the copy engine's bulk and tensor loads and
+// thread-block-cluster helpers (sm_90+/sm_100a), used by the pipelined and clustered kernels.
 //
 // Every wait is bounded by kWaitLimitNs: a caller that sees false sets kFlagTimeout
 // and leaves its loop instead of spinning forever.
@@ -74,6 +74,41 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
         "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
         ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
         : "memory");
+}
+
+// ---------------------------------------------------------------- clusters
+__device__ __forceinline__ uint32_t cluster_ctarank()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t cluster_nctarank()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+    return r;
+}
+
+// Barrier over the whole cluster, ordering shared-memory writes before other CTAs' reads.
+__device__ __forceinline__ void cluster_sync()
+{
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// 32-bit word at the same shared-memory offset as `local` in cluster CTA `rank`.
+__device__ __forceinline__ uint32_t ld_dsmem_u32(const void* local, uint32_t rank)
+{
+    uint32_t remote, v;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(local)), "r"(rank));
+    asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(remote) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ float ld_dsmem_f32(const float* local, uint32_t rank)
+{
+    return __uint_as_float(ld_dsmem_u32(local, rank));
 }
 
 }  // namespace nv4

@@ -6,23 +6,28 @@
 // i.e. the product of the two dequantized matrices, accumulated in FP32 and written
 // as BF16 or FP32.
 //
-// Kernel structure (one CTA = one 128 x kBN output tile, kBN = 256 when N allows, else 128;
-// 128 threads):
-//   * warp 0, one lane: producer.  Per stage of 256 K-elements it loads the A and B code
+// Kernel structure: persistent, one CTA per SM walking the 128 x kBN output tiles
+// t = blockIdx.x, + gridDim.x, ... (kBN = 256 when N allows, else 128); 192 threads:
+//   * warp 4, one lane: producer.  Per stage of 256 K-elements it loads the A and B code
 //     tiles (128 rows x 128 bytes each) with 2-D TMA into 128-byte-swizzled shared
 //     memory, and the stage's scale-factor atoms (4 x 512 bytes per operand, already in
 //     the MMA layout, see nv4_scales_to_mma_layout) with 1-D bulk copies, all completing
-//     on the stage's mbarrier.  A 4-stage ring; a stage is reused once the MMAs that
-//     read it have completed (tcgen05.commit on the stage's "empty" mbarrier).
-//   * warp 1: allocates 256 tensor-memory columns (the 128 x 128 FP32 accumulator and
-//     two scale-factor buffers); one lane issues, per stage, tcgen05.cp of the scale
-//     atoms into tensor memory and four tcgen05.mma kind::mxf4nvf4 block16 (K = 64
-//     each) with both operands read from shared memory through matrix descriptors.
-//   * all four warps: epilogue.  Warp w reads accumulator lanes 32w..32w+31 with
-//     tcgen05.ld (one output row per thread), multiplies by s2_A * s2_B, and stores.
+//     on the stage's mbarrier.  A 4-stage ring that runs across tiles: while the epilogue
+//     drains one tile, the first stages of the next are already loading.  A stage is
+//     reused once the MMAs that read it have completed (tcgen05.commit on "empty").
+//   * warp 5: allocates the tensor memory (the 128 x kBN FP32 accumulator and two
+//     scale-factor buffers); one lane waits until the epilogue has read the previous
+//     tile's accumulator ("acc_empty"), then per stage issues tcgen05.cp of the scale
+//     atoms into tensor memory and four tcgen05.mma kind::mxf4nvf4 block16 (K = 64 each)
+//     with both operands read from shared memory through matrix descriptors, and commits
+//     "acc_full" after the tile's last stage.
+//   * warps 0-3: epilogue.  Warp w reads accumulator lanes 32w..32w+31 with tcgen05.ld (one
+//     output row per thread), multiplies by s2_A * s2_B, stores, and arrives on acc_empty.
+// The accumulator is single-buffered (a second 256-column one does not fit the 512 columns
+// next to the scale buffers), so the epilogue still runs between two tiles' MMAs.
 // Every mbarrier wait is bounded (kWaitLimitNs); on expiry the kernel sets
-// NV4_FLAG_TIMEOUT, stops issuing, skips its stores, drains its copies in flight and
-// releases its tensor memory.
+// NV4_FLAG_TIMEOUT, every role stops, the stores are skipped, copies in flight are
+// drained and the tensor memory is released.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -37,7 +42,7 @@ namespace gemm {
 constexpr int kBM = 128;
 constexpr int kBK = 256;                          // FP4 elements per stage (128 bytes per row)
 constexpr int kStages = 4;
-constexpr int kThreads = 128;
+constexpr int kThreads = 192;                     // warps 0-3 epilogue, 4 producer, 5 MMA issuer
 
 // Tile width kBN = 128 or 256 (one MMA of 128 x kBN x 64 per K-step).
 template <int kBN>
@@ -63,7 +68,7 @@ struct Smem {
     uint8_t b[kStages][Cfg<kBN>::kBTile];
     uint8_t sfa[kStages][Cfg<kBN>::kSfA];
     uint8_t sfb[kStages][Cfg<kBN>::kSfB];
-    uint64_t full[kStages], empty[kStages], acc_full;
+    uint64_t full[kStages], empty[kStages], acc_full, acc_empty, drain;
     uint32_t tmem_base;
     uint32_t abort;                               // set by a wait that gave up
     uint32_t issued, consumed;                    // stages loaded / stages handed to the MMA
@@ -78,6 +83,7 @@ struct Params {
     void* out;
     int64_t ldd;
     uint32_t n_tiles, k_stages, kt4;              // kt4 = K / 64: scale atoms per 128-row tile
+    uint32_t tiles;                               // output tiles in all
     uint32_t* d_flags;
 };
 
@@ -162,128 +168,152 @@ gemm_nvfp4_kernel(const __grid_constant__ Params p)
     extern __shared__ uint8_t smem_raw[];
     Smem<kBN>& sm = *reinterpret_cast<Smem<kBN>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const uint32_t n_tile = blockIdx.x % p.n_tiles, m_tile = blockIdx.x / p.n_tiles;
     const uint32_t KS = p.k_stages;
 
-    if (threadIdx.x == 0) {
+    if (threadIdx.x == 128) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&sm.full[s], 1);
             mbar_init(&sm.empty[s], 1);
         }
         mbar_init(&sm.acc_full, 1);
+        mbar_init(&sm.acc_empty, 4);                               // one arrival per epilogue warp
+        mbar_init(&sm.drain, 1);
         sm.abort = 0u;
         sm.issued = sm.consumed = 0u;
         mbar_init_fence();
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&p.map_a)) : "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&p.map_b)) : "memory");
     }
-    if (warp == 1) tmem_alloc(&sm.tmem_base, C::kTmemCols);
+    if (warp == 5) tmem_alloc(&sm.tmem_base, C::kTmemCols);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
     uint32_t flags = 0u;
+    auto aborted = [&]() { return *reinterpret_cast<volatile uint32_t*>(&sm.abort) != 0u; };
 
-    if (warp == 0) {
-        if (lane == 0) {                                           // producer
-            uint32_t ks = 0;
-            for (; ks < KS; ++ks) {
-                const uint32_t s = ks % kStages;
-                if (ks >= (uint32_t)kStages && !mbar_wait(&sm.empty[s], ((ks / kStages) - 1u) & 1u)) {
-                    flags |= kFlagTimeout;
-                    atomicOr(&sm.abort, 1u);
-                    break;
-                }
-                if (*reinterpret_cast<volatile uint32_t*>(&sm.abort) != 0u) break;
-                mbar_arrive_expect_tx(&sm.full[s], C::kStageTx);
-                tma_load_2d(sm.a[s], &p.map_a, &sm.full[s], (int)(ks * 128u), (int)(m_tile * kBM));
-                tma_load_2d(sm.b[s], &p.map_b, &sm.full[s], (int)(ks * 128u), (int)(n_tile * kBN));
-                bulk_load(sm.sfa[s], p.sfa + ((size_t)m_tile * p.kt4 + 4u * ks) * 512u, C::kSfA, &sm.full[s]);
+    if (warp == 4) {
+        if (lane == 0) {                                           // producer, running ahead across tiles
+            uint32_t g = 0;
+            for (uint32_t t = blockIdx.x; t < p.tiles && !aborted(); t += gridDim.x) {
+                const uint32_t n_tile = t % p.n_tiles, m_tile = t / p.n_tiles;
+                for (uint32_t ks = 0; ks < KS; ++ks, ++g) {
+                    const uint32_t s = g % kStages;
+                    if (g >= (uint32_t)kStages && !mbar_wait(&sm.empty[s], ((g / kStages) - 1u) & 1u)) {
+                        flags |= kFlagTimeout;
+                        atomicOr(&sm.abort, 1u);
+                    }
+                    if (aborted()) break;
+                    mbar_arrive_expect_tx(&sm.full[s], C::kStageTx);
+                    tma_load_2d(sm.a[s], &p.map_a, &sm.full[s], (int)(ks * 128u), (int)(m_tile * kBM));
+                    tma_load_2d(sm.b[s], &p.map_b, &sm.full[s], (int)(ks * 128u), (int)(n_tile * kBN));
+                    bulk_load(sm.sfa[s], p.sfa + ((size_t)m_tile * p.kt4 + 4u * ks) * 512u, C::kSfA, &sm.full[s]);
 #pragma unroll
-                for (uint32_t h = 0; h < (uint32_t)(kBN / 128); ++h)      // one run of 4 atoms per 128 rows
-                    bulk_load(sm.sfb[s] + 2048u * h,
-                              p.sfb + ((size_t)(n_tile * (kBN / 128) + h) * p.kt4 + 4u * ks) * 512u, 2048u,
-                              &sm.full[s]);
+                    for (uint32_t h = 0; h < (uint32_t)(kBN / 128); ++h)  // one run of 4 atoms per 128 rows
+                        bulk_load(sm.sfb[s] + 2048u * h,
+                                  p.sfb + ((size_t)(n_tile * (kBN / 128) + h) * p.kt4 + 4u * ks) * 512u, 2048u,
+                                  &sm.full[s]);
+                }
             }
-            sm.issued = ks;
+            sm.issued = g;
         }
         __syncwarp();
-    } else if (warp == 1) {
+    } else if (warp == 5) {
         if (lane == 0) {                                           // MMA issuer
-            uint32_t ks = 0;
-            for (; ks < KS; ++ks) {
-                const uint32_t s = ks % kStages;
-                if (!mbar_wait(&sm.full[s], (ks / kStages) & 1u)) {
+            uint32_t g = 0, i = 0;
+            for (uint32_t t = blockIdx.x; t < p.tiles && !aborted(); t += gridDim.x, ++i) {
+                // the accumulator is free once the epilogue has read the previous tile
+                if (i > 0 && !mbar_wait(&sm.acc_empty, (i - 1u) & 1u)) {
                     flags |= kFlagTimeout;
                     atomicOr(&sm.abort, 1u);
                     break;
                 }
                 tc_fence_after();
-                const uint32_t buf = ks & 1u;
-                // scale columns: A row r of K-step j at column ta + 4j + r/32; B row n at tb + nb*j + n/32
-                constexpr uint32_t nb = 4u * (kBN / 128);
-                const uint32_t ta = tmem + C::kColSfA + 16u * buf, tb = tmem + C::kColSfB + C::kSfBCols * buf;
+                for (uint32_t ks = 0; ks < KS; ++ks, ++g) {
+                    const uint32_t s = g % kStages;
+                    if (!mbar_wait(&sm.full[s], (g / kStages) & 1u)) {
+                        flags |= kFlagTimeout;
+                        atomicOr(&sm.abort, 1u);
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t buf = g & 1u;
+                    // scale columns: A row r of K-step j at column ta + 4j + r/32; B row n at tb + nb*j + n/32
+                    constexpr uint32_t nb = 4u * (kBN / 128);
+                    const uint32_t ta = tmem + C::kColSfA + 16u * buf, tb = tmem + C::kColSfB + C::kSfBCols * buf;
 #pragma unroll
-                for (uint32_t j = 0; j < 4; ++j) {
-                    tmem_cp_sf(ta + 4u * j, smem_desc(smem_u32(sm.sfa[s] + 512u * j), 0u, 8u, 0u));
+                    for (uint32_t j = 0; j < 4; ++j) {
+                        tmem_cp_sf(ta + 4u * j, smem_desc(smem_u32(sm.sfa[s] + 512u * j), 0u, 8u, 0u));
 #pragma unroll
-                    for (uint32_t h = 0; h < (uint32_t)(kBN / 128); ++h)
-                        tmem_cp_sf(tb + nb * j + 4u * h, smem_desc(smem_u32(sm.sfb[s] + 2048u * h + 512u * j), 0u, 8u, 0u));
+                        for (uint32_t h = 0; h < (uint32_t)(kBN / 128); ++h)
+                            tmem_cp_sf(tb + nb * j + 4u * h, smem_desc(smem_u32(sm.sfb[s] + 2048u * h + 512u * j), 0u, 8u, 0u));
+                    }
+                    const uint32_t a0 = smem_u32(sm.a[s]), b0 = smem_u32(sm.b[s]);
+#pragma unroll
+                    for (uint32_t j = 0; j < 4; ++j)
+                        mma_fp4(tmem, smem_desc(a0 + 32u * j, 1u, 64u, 2u), smem_desc(b0 + 32u * j, 1u, 64u, 2u),
+                                C::kIdesc, ta + 4u * j, tb + nb * j, (ks | j) != 0u ? 1u : 0u);
+                    tc_commit(&sm.empty[s]);                       // frees the stage when these MMAs finish
                 }
-                const uint32_t a0 = smem_u32(sm.a[s]), b0 = smem_u32(sm.b[s]);
-#pragma unroll
-                for (uint32_t j = 0; j < 4; ++j)
-                    mma_fp4(tmem, smem_desc(a0 + 32u * j, 1u, 64u, 2u), smem_desc(b0 + 32u * j, 1u, 64u, 2u),
-                            C::kIdesc, ta + 4u * j, tb + nb * j, (ks | j) != 0u ? 1u : 0u);
-                tc_commit(&sm.empty[s]);                           // frees the stage when these MMAs finish
+                if (aborted()) break;
+                tc_commit(&sm.acc_full);                           // this tile's accumulator is complete
             }
-            sm.consumed = ks;
-            tc_commit(&sm.acc_full);                               // the accumulator is complete
+            sm.consumed = g;
+            tc_commit(&sm.drain);                                  // every tensor-core operation issued
+            if (!mbar_wait(&sm.drain, 0u)) flags |= kFlagTimeout;
         }
         __syncwarp();
-    }
-
-    // ---- epilogue: every warp, one accumulator row per thread
-    const bool acc_ok = mbar_wait(&sm.acc_full, 0u);
-    if (!acc_ok) flags |= kFlagTimeout;
-    tc_fence_after();
-    __syncwarp();
-    const bool store = acc_ok && *reinterpret_cast<volatile uint32_t*>(&sm.abort) == 0u && KS > 0u;
-    const float alpha = __fmul_rn(*p.d_s2a, *p.d_s2b);
-    const int64_t row = (int64_t)m_tile * kBM + 32 * warp + lane;
+    } else {
+        // ---- epilogue warps 0-3: accumulator lanes 32w..32w+31, one output row per thread
+        const float alpha = __fmul_rn(*p.d_s2a, *p.d_s2b);
+        uint32_t i = 0;
+        for (uint32_t t = blockIdx.x; t < p.tiles; t += gridDim.x, ++i) {
+            const bool ok = !aborted() && mbar_wait(&sm.acc_full, i & 1u);
+            if (!ok) {
+                if (!aborted()) { flags |= kFlagTimeout; atomicOr(&sm.abort, 1u); }
+                break;
+            }
+            tc_fence_after();
+            __syncwarp();
+            const uint32_t n_tile = t % p.n_tiles, m_tile = t / p.n_tiles;
+            const int64_t row = (int64_t)m_tile * kBM + 32 * warp + lane;
 #pragma unroll 1
-    for (int cb = 0; cb < kBN / 32; ++cb) {
-        float v[32];
-        tmem_ld32(tmem + ((uint32_t)(32 * warp) << 16) + (uint32_t)(32 * cb), v);
-        if (!store) continue;
-        const int64_t col = (int64_t)n_tile * kBN + 32 * cb;
-        if constexpr (kOut == 2) {
-            float4* o = reinterpret_cast<float4*>(static_cast<float*>(p.out) + row * p.ldd + col);
+            for (int cb = 0; cb < kBN / 32; ++cb) {
+                float v[32];
+                tmem_ld32(tmem + ((uint32_t)(32 * warp) << 16) + (uint32_t)(32 * cb), v);
+                const int64_t col = (int64_t)n_tile * kBN + 32 * cb;
+                if constexpr (kOut == 2) {
+                    float4* o = reinterpret_cast<float4*>(static_cast<float*>(p.out) + row * p.ldd + col);
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-                o[i] = make_float4(__fmul_rn(v[4 * i], alpha), __fmul_rn(v[4 * i + 1], alpha),
-                                   __fmul_rn(v[4 * i + 2], alpha), __fmul_rn(v[4 * i + 3], alpha));
-        } else {
-            uint32_t w[16];
+                    for (int k = 0; k < 8; ++k)
+                        o[k] = make_float4(__fmul_rn(v[4 * k], alpha), __fmul_rn(v[4 * k + 1], alpha),
+                                           __fmul_rn(v[4 * k + 2], alpha), __fmul_rn(v[4 * k + 3], alpha));
+                } else {
+                    uint32_t w[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i)
-                asm("cvt.rn.bf16x2.f32 %0, %1, %2;"
-                    : "=r"(w[i])
-                    : "f"(__fmul_rn(v[2 * i + 1], alpha)), "f"(__fmul_rn(v[2 * i], alpha)));
-            uint4* o = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + row * p.ldd + col);
+                    for (int k = 0; k < 16; ++k)
+                        asm("cvt.rn.bf16x2.f32 %0, %1, %2;"
+                            : "=r"(w[k])
+                            : "f"(__fmul_rn(v[2 * k + 1], alpha)), "f"(__fmul_rn(v[2 * k], alpha)));
+                    uint4* o = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + row * p.ldd + col);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) o[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+                    for (int k = 0; k < 4; ++k) o[k] = make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.acc_empty);             // this warp has read the accumulator
         }
     }
 
     // ---- teardown: drain copies that were loaded but never consumed, free tensor memory
     tc_fence_before();
     __syncthreads();
-    if (threadIdx.x == 0) {
-        for (uint32_t ks = sm.consumed; ks < sm.issued; ++ks)
-            if (!mbar_wait(&sm.full[ks % kStages], (ks / kStages) & 1u)) flags |= kFlagTimeout;
+    if (threadIdx.x == 128) {
+        for (uint32_t g = sm.consumed; g < sm.issued; ++g)
+            if (!mbar_wait(&sm.full[g % kStages], (g / kStages) & 1u)) flags |= kFlagTimeout;
     }
-    if (warp == 1) {
+    if (warp == 5) {
         tc_fence_after();
         tmem_dealloc(tmem, C::kTmemCols);
     }
@@ -376,6 +406,7 @@ cudaError_t launch_gemm_nvfp4(const uint8_t* qa, const uint8_t* sfa, const float
     p.n_tiles = (uint32_t)(N / bn);
     p.k_stages = (uint32_t)(K / kBK);
     p.kt4 = (uint32_t)(K / 64);
+    p.tiles = (uint32_t)((M / kBM) * (N / bn));
     p.d_flags = d_flags;
     const size_t smem = (wide ? sizeof(Smem<256>) : sizeof(Smem<128>)) + 1024;
     static bool attr_set[4][64] = {};
@@ -391,7 +422,7 @@ cudaError_t launch_gemm_nvfp4(const uint8_t* qa, const uint8_t* sfa, const float
         if (e != cudaSuccess) return e;
         if (dev >= 0 && dev < 64) attr_set[v][dev] = true;
     }
-    const unsigned grid = (unsigned)((M / kBM) * (N / bn));
+    const unsigned grid = (unsigned)(p.tiles < (uint32_t)num_sms() ? p.tiles : (uint32_t)num_sms());
     kern<<<grid, kThreads, smem, s>>>(p);
     return cudaGetLastError();
 }

@@ -349,16 +349,18 @@ def kernel_rooflines(W, hbm_peak):
         for k in ("fake_qdq", "mxfp4_quant", "fp8_quant", "hadamard128_mxfp4_quant"):
             out[k]["launch"] = f"[{big['T']}, {big['C']}] bf16"
     if "weights" in W:
-        # RTN weight quantization of the gate projection (a widening of the path; not in the step)
-        j = W["weights"][1]
-        rq = torch.empty_like(j["q"])
-        rs = torch.empty((j["w"].shape[0], j["w"].shape[1] // 16), dtype=torch.uint8, device=j["w"].device)
-        rs2 = torch.empty(1, dtype=torch.float32, device=j["w"].device)
-        t = time_launch(lambda: nv4.nv4_weight_quant_rtn(j["w"], j["d_amax_w"], rq, rs, rs2, W["flags"]),
-                        flush=flush)
-        out["weight_quant_rtn"] = {"bound": "hbm", "bytes": ACT_BYTES["act_quant"] * j["w"].numel(), "s": t,
-                                   "in_step": False, "launch": f"{j['name']} {list(j['w'].shape)} bf16"}
-        del rq, rs
+        # RTN weight quantization of the layer's four weights in one batched launch (a widening
+        # of the path; not in the step)
+        rjobs = [dict(w=j["w"], d_amax=j["d_amax_w"], q=torch.empty_like(j["q"]),
+                      scales=torch.empty((j["w"].shape[0], j["w"].shape[1] // 16), dtype=torch.uint8,
+                                         device=j["w"].device),
+                      d_s2=torch.empty(1, dtype=torch.float32, device=j["w"].device)) for j in W["weights"]]
+        t = time_launch(lambda: nv4.nv4_weight_quant_rtn_batched(rjobs, W["flags"]), flush=flush)
+        out["weight_quant_rtn"] = {"bound": "hbm", "s": t, "in_step": False,
+                                   "bytes": ACT_BYTES["act_quant"] * sum(j["w"].numel() for j in rjobs),
+                                   "launch": " + ".join(f"{j['name']} {list(j['w'].shape)}" for j in W["weights"])
+                                             + " bf16, one batched launch"}
+        del rjobs
         X, Xd = W["X"], W["Xd"]
         t = time_launch(lambda: nv4.nv4_hessian_accum_batched([X, Xd], [W["H"], W["Hd"]], W["flags"]), reps=10,
                         flush=flush)

@@ -160,6 +160,13 @@ NV4_API nv4_status nv4_weight_quant_rtn(const void* w, nv4_dtype dt, int64_t row
                                 const float* d_amax, uint8_t* q, uint8_t* scales, float* d_s2,
                                 uint32_t* d_flags, void* stream);
 
+/* Batched form: several weight tensors of one dtype (e.g. a layer's projections), each
+ * with its own amax and s2, in one launch.  Per job the rules, layouts and limits of
+ * nv4_weight_quant_rtn (the job struct is nv4_act_job with w in place of x); at most 128
+ * jobs. */
+NV4_API nv4_status nv4_weight_quant_rtn_batched(const nv4_act_job* jobs, int n_jobs, nv4_dtype dt,
+                                        uint32_t* d_flags, void* stream);
+
 /* ---------------------------------------------------------------------------
  * nv4_fake_qdq -- fused fake quantization: nv4_act_quant followed by nv4_dequant in
  * one pass, without materializing codes or scales ([FLOW] 3.4: quantizer, then DQ1

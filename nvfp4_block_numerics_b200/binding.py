@@ -28,7 +28,7 @@ __all__ = [
     "nv4_mxfp4_to_nvfp4_batched", "nv4_selftest", "nv4_version", "FLAG_NONFINITE", "FLAG_E8M0_NAN",
     "FLAG_OVERFLOW", "FLAG_TIMEOUT", "tensor_amax", "act_quant", "dequant", "hessian_accum",
     "scale_sweep", "mxfp4_to_nvfp4", "HessianJob", "SweepJob", "CastJob", "AmaxJob", "ActJob", "DequantJob",
-    "nv4_tensor_amax_batched", "nv4_act_quant_batched", "nv4_dequant_batched",
+    "nv4_tensor_amax_batched", "nv4_act_quant_batched", "nv4_dequant_batched", "nv4_weight_quant_rtn_batched",
 ]
 
 BF16, FP16, FP32 = 0, 1, 2
@@ -79,6 +79,7 @@ _SIGS = {
     "nv4_act_quant": (C.c_int, [_vp, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp]),
     "nv4_tensor_amax_batched": (C.c_int, [C.POINTER(AmaxJob), C.c_int, C.c_int, _vp, _vp]),
     "nv4_act_quant_batched": (C.c_int, [C.POINTER(ActJob), C.c_int, _vp, _vp]),
+    "nv4_weight_quant_rtn_batched": (C.c_int, [C.POINTER(ActJob), C.c_int, C.c_int, _vp, _vp]),
     "nv4_dequant_batched": (C.c_int, [C.POINTER(DequantJob), C.c_int, C.c_int, _vp]),
     "nv4_weight_quant_rtn": (C.c_int, [_vp, C.c_int, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp]),
     "nv4_fake_qdq": (C.c_int, [_vp, _i64, _i64, _i64, _vp, C.c_int, _vp, _i64, _vp, _vp, _vp]),
@@ -207,6 +208,31 @@ def nv4_act_quant_batched(jobs: list[dict], d_flags: torch.Tensor | None = None,
         arr[i] = ActJob(_ptr(x), rows, cols, ld, _scalar_f32(j["d_amax"], "d_amax"), _ptr(q), _ptr(sc),
                         _scalar_f32(j["d_s2"], "d_s2"))
     _check(lib().nv4_act_quant_batched(arr, len(jobs), _ptr(d_flags), _stream(stream)), "nv4_act_quant_batched")
+
+
+def nv4_weight_quant_rtn_batched(jobs: list[dict], d_flags: torch.Tensor | None = None, stream=None):
+    """jobs: dicts with keys w (bf16 or float32 [rows, cols], one dtype), d_amax, q, scales,
+    d_s2 -- nv4_weight_quant_rtn per tensor, in one launch."""
+    if not jobs:
+        return
+    dt = jobs[0]["w"].dtype
+    if dt not in (torch.bfloat16, torch.float32):
+        raise NV4Error("w must be bf16 or float32")
+    arr = (ActJob * len(jobs))()
+    for i, j in enumerate(jobs):
+        w = j["w"]
+        if w.dtype != dt:
+            raise NV4Error("all weights of one call must share a dtype")
+        rows, cols, ld = _rowmajor(w, "w")
+        q, sc = j["q"], j["scales"]
+        if q.dtype != torch.uint8 or tuple(q.shape) != (rows, cols // 2) or not q.is_contiguous():
+            raise NV4Error("q must be a contiguous uint8 tensor [rows, cols/2]")
+        if sc.dtype != torch.uint8 or tuple(sc.shape) != (rows, cols // 16) or not sc.is_contiguous():
+            raise NV4Error("scales must be a contiguous uint8 tensor [rows, cols/16]")
+        arr[i] = ActJob(_ptr(w), rows, cols, ld, _scalar_f32(j["d_amax"], "d_amax"), _ptr(q), _ptr(sc),
+                        _scalar_f32(j["d_s2"], "d_s2"))
+    _check(lib().nv4_weight_quant_rtn_batched(arr, len(jobs), _DT[dt], _ptr(d_flags), _stream(stream)),
+           "nv4_weight_quant_rtn_batched")
 
 
 def nv4_dequant_batched(jobs: list[dict], stream=None):

@@ -160,14 +160,15 @@ nv4_status nv4_tensor_amax_batched(const nv4_amax_job* jobs, int n_jobs, nv4_dty
     return from_cuda(launch_amax(t, n_jobs, dt == NV4_BF16 ? 0 : 2, d_flags, (cudaStream_t)stream));
 }
 
+// ld_mult: the row pitch that keeps rows 16-byte aligned (8 BF16 or 4 FP32 elements).
 static nv4_status check_act(const void* x, int64_t rows, int64_t cols, int64_t ld, const float* d_amax,
-                            const uint8_t* q, const uint8_t* scales, const float* d_s2)
+                            const uint8_t* q, const uint8_t* scales, const float* d_s2, int64_t ld_mult = 8)
 {
     if (rows < 0 || cols < 0 || cols % 16 != 0 || ld < cols) return NV4_ERR_SHAPE;
     if (d_amax == nullptr || d_s2 == nullptr) return NV4_ERR_NULL;
     if (rows == 0 || cols == 0) return NV4_OK;
     if (x == nullptr || q == nullptr || scales == nullptr) return NV4_ERR_NULL;
-    if (!aligned16(x) || !aligned16(q) || ld % 8 != 0) return NV4_ERR_ALIGN;
+    if (!aligned16(x) || !aligned16(q) || ld % ld_mult != 0) return NV4_ERR_ALIGN;
     if (rows * (cols / 16) >= (int64_t)1 << 30) return NV4_ERR_LIMIT;
     return NV4_OK;
 }
@@ -210,6 +211,25 @@ nv4_status nv4_weight_quant_rtn(const void* w, nv4_dtype dt, int64_t rows, int64
     if (rows * (cols / 16) >= (int64_t)1 << 30) return NV4_ERR_LIMIT;
     const QuantTask t = {w, rows, cols, ld, d_amax, q, scales, nullptr, 0, d_s2};
     return from_cuda(launch_block_quant(&t, 1, dt == NV4_BF16 ? 0 : 2, -1, d_flags, (cudaStream_t)stream));
+}
+
+nv4_status nv4_weight_quant_rtn_batched(const nv4_act_job* jobs, int n_jobs, nv4_dtype dt, uint32_t* d_flags,
+                                        void* stream)
+{
+    if (n_jobs < 0) return NV4_ERR_SHAPE;
+    if (n_jobs == 0) return NV4_OK;
+    if (jobs == nullptr) return NV4_ERR_NULL;
+    if (n_jobs > kMaxActJobs) return NV4_ERR_LIMIT;
+    if (dt != NV4_BF16 && dt != NV4_FP32) return NV4_ERR_DTYPE;
+    QuantTask t[kMaxActJobs];
+    for (int i = 0; i < n_jobs; ++i) {
+        const nv4_act_job& J = jobs[i];
+        const nv4_status st = check_act(J.x, J.rows, J.cols, J.ld, J.d_amax, J.q, J.scales, J.d_s2,
+                                        dt == NV4_BF16 ? 8 : 4);
+        if (st != NV4_OK) return st;
+        t[i] = {J.x, J.rows, J.cols, J.ld, J.d_amax, J.q, J.scales, nullptr, 0, J.d_s2};
+    }
+    return from_cuda(launch_block_quant(t, n_jobs, dt == NV4_BF16 ? 0 : 2, -1, d_flags, (cudaStream_t)stream));
 }
 
 nv4_status nv4_fake_qdq(const void* x, int64_t rows, int64_t cols, int64_t ld, const float* d_amax,

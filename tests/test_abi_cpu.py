@@ -32,7 +32,7 @@ def test_header_declares_the_hot_path():
               "nv4_scales_to_mma_layout", "nv4_mma_scale_bytes", "nv4_mxfp4_quant", "nv4_mxfp4_dequant",
               "nv4_fp8_quant", "nv4_fp8_dequant", "nv4_hadamard_amax", "nv4_hadamard_mxfp4_quant",
               "nv4_hadamard_nvfp4_quant", "nv4_selftest_wait", "nv4_tensor_amax_batched", "nv4_act_quant_batched",
-              "nv4_dequant_batched"):
+              "nv4_dequant_batched", "nv4_weight_quant_rtn_batched"):
         assert n in names
 
 
@@ -147,6 +147,11 @@ def test_batched_act_path_validation(nv4lib):
     aj[1] = b.ActJob(fake, 4, 32, 32, None, fake, fake, fake)
     assert L.nv4_act_quant_batched(aj, 2, None, None) == 1               # second: amax
     assert L.nv4_act_quant_batched((b.ActJob * 129)(), 129, None, None) == 6
+    rj = (b.ActJob * 2)(b.ActJob(fake, 4, 32, 36, fake, fake, fake, fake), b.ActJob(fake, 4, 32, 34, fake, fake, fake, fake))
+    assert L.nv4_weight_quant_rtn_batched((b.ActJob * 129)(), 129, 2, None, None) == 6
+    assert L.nv4_weight_quant_rtn_batched(rj, 2, 2, None, None) == 3     # second: FP32 row pitch 34
+    assert L.nv4_weight_quant_rtn_batched(rj, 2, 0, None, None) == 3     # BF16 needs a pitch of 8
+    assert L.nv4_weight_quant_rtn_batched(rj, 2, 1, None, None) == 4     # fp16 weights
     dj = (b.DequantJob * 2)(b.DequantJob(fake, fake, fake, 4, 32, fake), b.DequantJob(fake, fake, fake, 4, 32, fake + 8))
     assert L.nv4_dequant_batched(dj, 2, 0, None) == 3                    # second out misaligned
     assert L.nv4_dequant_batched(dj, 1, 7, None) == 4                    # out dtype

@@ -252,6 +252,43 @@ def test_weight_quant_rtn_layer_weights(orc):
     _rtn_check(orc, inputs.c1_tiny_linear(0)["W"])
 
 
+@pytest.mark.parametrize("fp32", [False, True])
+def test_weight_quant_rtn_batched(orc, fp32):
+    """One batched launch over ragged weights (row pitch padding, a one-row tensor, zero
+    blocks, a static amax below the data's) equals the oracle's RTN per tensor."""
+    shapes = [(1, 16, 0), (3, 48, 8), (129, 80, 0), (300, 256, 16), (70, 2048, 0), (17, 176, 24)]
+    ws, jobs, amaxes = [], [], []
+    n = len(shapes)
+    am = torch.zeros(n, device=G.DEV)
+    s2 = torch.zeros(n, device=G.DEV)
+    for i, (rows, cols, pad) in enumerate(shapes):
+        r = np.random.default_rng(77 + i)
+        w = (r.standard_normal((rows, cols + pad)) * float(10.0 ** r.uniform(-3, 1))).astype(np.float32)
+        w[:, :cols] *= np.repeat(r.random((rows, cols // 16)) >= 0.1, 16, axis=1)   # zero blocks
+        if not fp32:
+            w = inputs.f32_to_bf16_bits(w)
+        wd = (G.f32_dev(w) if fp32 else G.bf16_dev(w))[:, :cols]
+        w = np.ascontiguousarray(w[:, :cols])
+        a = float(orc.tensor_amax(w)[0]) * (0.5 if i == 4 else 1.0)
+        am[i] = a
+        ws.append(w)
+        amaxes.append(a)
+        jobs.append(dict(w=wd, d_amax=am[i:i + 1], d_s2=s2[i:i + 1],
+                         q=torch.empty((rows, cols // 2), dtype=torch.uint8, device=G.DEV),
+                         scales=torch.empty((rows, cols // 16), dtype=torch.uint8, device=G.DEV)))
+    f = G.flags_dev()
+    nv4.nv4_weight_quant_rtn_batched(jobs, f)
+    torch.cuda.synchronize()
+    rflags = 0
+    for i, (w, a, j) in enumerate(zip(ws, amaxes, jobs)):
+        rq, rsc, rs2, rf = orc.rtn_quant(w, a)
+        rflags |= rf
+        assert s2[i].item() == rs2, i
+        assert np.array_equal(G.host(j["scales"]), rsc), i
+        assert np.array_equal(G.host(j["q"]), rq), i
+    assert f.item() == rflags
+
+
 # ------------------------------------------------------------------ fused fake quantize-dequantize
 def _qdq_check(orc, x, amax=None, ld_pad=0, out_pad=0):
     rows, cols = x.shape

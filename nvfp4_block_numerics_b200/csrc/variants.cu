@@ -12,6 +12,8 @@
 // code = sign | E4M3 nearest to |x| / s.  The quotient is bracketed between two FP32
 // products by 1/s with a 2^-20 margin and both ends converted with the hardware's RNE
 // E4M3 conversion; when they differ, one exact FMA comparison with the midpoint decides.
+#include <cuda_fp16.h>
+
 #include "nv4_common.cuh"
 #include "nv4_internal.h"
 
@@ -178,6 +180,15 @@ __device__ __forceinline__ uint32_t fp8_fix(float x, float s, uint32_t lo, uint3
     return sign | c;
 }
 
+// Two E4M3 codes (bits 0-7 and 8-15) to their values as FP16 (exact), low code in the
+// low half.
+__device__ __forceinline__ __half2 e4m3x2_to_half2(uint32_t codes)
+{
+    uint32_t r;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"((unsigned short)codes));
+    return *reinterpret_cast<const __half2*>(&r);
+}
+
 // Codes of 16 elements against s (bracket r_lo <= 1/s <= r_hi).  The hardware conversion
 // keeps the sign, so signed products convert directly; a pair is exact when both ends of
 // the bracket agree on both codes.
@@ -208,6 +219,32 @@ __device__ __forceinline__ void fp8_codes16(const float v[16], float s, float r_
     }
 }
 
+// Every group this thread owns when s is zero or far from 1 (mode 0 or 2): no bracket,
+// exact FP64 divisions.  Out of line and entered once, so the streaming loop below keeps
+// few registers.
+template <int kIn>
+static __device__ __noinline__ uint32_t fp8_quant_exact_all(const void* x, uint32_t total, uint32_t groups_per_row,
+                                                            int64_t ld, FastDiv div_gpr, uint8_t* q, int64_t ldq,
+                                                            float s, int mode)
+{
+    uint32_t flags = 0u;
+    for (uint32_t g = blockIdx.x * kVarThreads + threadIdx.x; g < total; g += gridDim.x * kVarThreads) {
+        const uint32_t row = div_gpr.div(g), gg = g - row * groups_per_row;
+        float v[16];
+        uint32_t ab;
+        load16<kIn>(x, (int64_t)row * ld + 16 * (int64_t)gg, v, ab);
+        if (ab >= 0x7F800000u) flags |= kFlagNonFinite;
+        uint32_t w[4];
+        fp8_codes16(v, s, 0.0f, 0.0f, mode, w);
+        __stcs(reinterpret_cast<uint4*>(q + (int64_t)row * ldq + 16 * (int64_t)gg), make_uint4(w[0], w[1], w[2], w[3]));
+    }
+    return flags;
+}
+
+// One thread per group of 16 elements, grid-stride, with the next group's loads in flight
+// while this one is converted: two scaled products per element (the bracket
+// r_lo <= 1/s <= r_hi) and two hardware conversions per pair; the rare elements whose
+// bracket ends disagree get one exact FMA comparison each.
 template <int kIn>
 __global__ void __launch_bounds__(kVarThreads)
 fp8_quant_kernel(const void* x, uint32_t rows, uint32_t groups_per_row, int64_t ld, FastDiv div_gpr,
@@ -217,61 +254,98 @@ fp8_quant_kernel(const void* x, uint32_t rows, uint32_t groups_per_row, int64_t 
     const float s = __fdiv_rn(*d_amax, 448.0f);                   // RN32(amax / 448)
     if (blockIdx.x == 0 && threadIdx.x == 0) *d_scale = s;
     const int mode = s == 0.0f ? 0 : (s >= 0x1p-100f && s <= 0x1p100f ? 1 : 2);
-    const float r = mode == 1 ? __frcp_rn(s) : 0.0f;
-    const float r_lo = __fmul_rn(r, kLoMargin), r_hi = __fmul_rn(r, kHiMargin);
     uint32_t flags = isfinite(s) ? 0u : kFlagOverflow;
     const uint32_t total = rows * groups_per_row;
-    const uint32_t stride = gridDim.x * kVarThreads;
-    // the next group's loads are in flight while this one is converted
-    auto offset = [&](uint32_t g) {
-        const uint32_t row = div_gpr.div(g);
-        return (int64_t)row * ld + 16 * (int64_t)(g - row * groups_per_row);
-    };
-    constexpr int kWords = kIn == 0 ? 2 : 4;
-    uint4 nxt[kWords];
-    uint32_t g = blockIdx.x * kVarThreads + threadIdx.x;
-    if (g < total) {
-        const uint4* src = reinterpret_cast<const uint4*>(static_cast<const char*>(x) + offset(g) * (kIn == 0 ? 2 : 4));
-#pragma unroll
-        for (int k = 0; k < kWords; ++k) nxt[k] = __ldcs(src + k);
-    }
-    for (; g < total; g += stride) {
-        const uint32_t row = div_gpr.div(g), gg = g - row * groups_per_row;
-        uint4 cur[kWords];
-#pragma unroll
-        for (int k = 0; k < kWords; ++k) cur[k] = nxt[k];
-        if (g + stride < total) {
-            const uint4* src = reinterpret_cast<const uint4*>(static_cast<const char*>(x) + offset(g + stride) * (kIn == 0 ? 2 : 4));
+    if (mode != 1) {
+        flags |= fp8_quant_exact_all<kIn>(x, total, groups_per_row, ld, div_gpr, q, ldq, s, mode);
+    } else {
+        const float r = __frcp_rn(s);
+        const float r_lo = __fmul_rn(r, kLoMargin), r_hi = __fmul_rn(r, kHiMargin);
+        const uint32_t stride = gridDim.x * kVarThreads;
+        constexpr int kWords = kIn == 0 ? 2 : 4;
+        constexpr int kElem = kIn == 0 ? 2 : 4;
+        auto offset = [&](uint32_t g) {
+            const uint32_t row = div_gpr.div(g);
+            return (int64_t)row * ld + 16 * (int64_t)(g - row * groups_per_row);
+        };
+        uint4 nxt[kWords];
+        uint32_t g = blockIdx.x * kVarThreads + threadIdx.x;
+        if (g < total) {
+            const uint4* src = reinterpret_cast<const uint4*>(static_cast<const char*>(x) + offset(g) * kElem);
 #pragma unroll
             for (int k = 0; k < kWords; ++k) nxt[k] = __ldcs(src + k);
         }
-        float v[16];
-        uint32_t ab = 0u;
-        if constexpr (kIn == 0) {
-            const uint32_t w[8] = {cur[0].x, cur[0].y, cur[0].z, cur[0].w, cur[1].x, cur[1].y, cur[1].z, cur[1].w};
-            uint32_t m = 0u;
+        for (; g < total; g += stride) {
+            const uint32_t row = div_gpr.div(g), gg = g - row * groups_per_row;
+            uint4 cur[kWords];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                m = __vmaxu2(m, w[j] & 0x7FFF7FFFu);
-                v[2 * j] = bf16_lo(w[j]);
-                v[2 * j + 1] = bf16_hi(w[j]);
+            for (int k = 0; k < kWords; ++k) cur[k] = nxt[k];
+            if (g + stride < total) {
+                const uint4* src =
+                    reinterpret_cast<const uint4*>(static_cast<const char*>(x) + offset(g + stride) * kElem);
+#pragma unroll
+                for (int k = 0; k < kWords; ++k) nxt[k] = __ldcs(src + k);
             }
-            ab = max(m & 0xFFFFu, m >> 16) << 16;
-        } else {
+            float v[16];
+            uint32_t ab = 0u;
+            const uint32_t* cw = reinterpret_cast<const uint32_t*>(cur);
+            if constexpr (kIn == 0) {
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const uint32_t w[4] = {cur[k].x, cur[k].y, cur[k].z, cur[k].w};
+                for (int j = 0; j < 8; ++j) {
+                    ab = __vmaxu2(ab, cw[j] & 0x7FFF7FFFu);
+                    v[2 * j] = bf16_lo(cw[j]);
+                    v[2 * j + 1] = bf16_hi(cw[j]);
+                }
+                ab = max(ab & 0xFFFFu, ab >> 16) << 16;
+            } else {
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    ab = max(ab, w[j] & 0x7FFFFFFFu);
-                    v[4 * k + j] = __uint_as_float(w[j]);
+                for (int j = 0; j < 16; ++j) {
+                    ab = max(ab, cw[j] & 0x7FFFFFFFu);
+                    v[j] = __uint_as_float(cw[j]);
                 }
             }
+            if (ab >= 0x7F800000u) flags |= kFlagNonFinite;
+            uint32_t lo[8], straddle = 0u;                        // codes of pairs (2j, 2j+1)
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const float2 p = make_float2(v[2 * j], v[2 * j + 1]);
+                const float2 pl = __fmul2_rn(p, make_float2(r_lo, r_lo));
+                const float2 ph = __fmul2_rn(p, make_float2(r_hi, r_hi));
+                lo[j] = cvt_e4m3x2(pl.x, pl.y);
+                straddle |= (lo[j] != cvt_e4m3x2(ph.x, ph.y) ? 1u : 0u) << j;
+            }
+            uint8_t* dst = q + (int64_t)row * ldq + 16 * (int64_t)gg;
+            __stcs(reinterpret_cast<uint4*>(dst), make_uint4(lo[0] | (lo[1] << 16), lo[2] | (lo[3] << 16),
+                                                            lo[4] | (lo[5] << 16), lo[6] | (lo[7] << 16)));
+            // Pairs whose bracket ends disagree (about one element in a hundred when s is
+            // close to a short rational, as for amax = 752): the pair is re-read (it is
+            // still in L2), both elements decided exactly and its two bytes rewritten; the
+            // loop runs over the set bits so a warp pays for its busiest lane only.
+            const char* src = static_cast<const char*>(x) + ((int64_t)row * ld + 16 * (int64_t)gg) * kElem;
+            while (straddle != 0u) {
+                const int j = __ffs(straddle) - 1;
+                straddle &= straddle - 1u;
+                float2 p;
+                if constexpr (kIn == 0) {
+                    const uint32_t w2 = __ldcs(reinterpret_cast<const uint32_t*>(src) + j);
+                    p = make_float2(bf16_lo(w2), bf16_hi(w2));
+                } else {
+                    p = __ldcs(reinterpret_cast<const float2*>(src) + j);
+                }
+                const float2 pl = __fmul2_rn(p, make_float2(r_lo, r_lo));
+                const float2 ph = __fmul2_rn(p, make_float2(r_hi, r_hi));
+                const uint32_t l2 = cvt_e4m3x2(pl.x, pl.y), h2 = cvt_e4m3x2(ph.x, ph.y);
+                // the midpoint between each element's two candidate codes (exact in FP16:
+                // at most 5 significant bits), then one exact FMA comparison per element
+                const __half2 vl = e4m3x2_to_half2(l2 & 0x7F7Fu), vh = e4m3x2_to_half2(h2 & 0x7F7Fu);
+                const float2 mid = __half22float2(__hmul2(__hadd2(vl, vh), __float2half2_rn(0.5f)));
+                const float2 d = __ffma2_rn(mid, make_float2(s, s), make_float2(-fabsf(p.x), -fabsf(p.y)));
+                const bool up0 = d.x < 0.0f || (d.x == 0.0f && (l2 & 1u));
+                const bool up1 = d.y < 0.0f || (d.y == 0.0f && ((l2 >> 8) & 1u));
+                reinterpret_cast<unsigned short*>(dst)[j] =
+                    (unsigned short)(((up0 ? h2 : l2) & 0xFFu) | ((up1 ? h2 : l2) & 0xFF00u));
+            }
         }
-        if (ab >= 0x7F800000u) flags |= kFlagNonFinite;
-        uint32_t w[4];
-        fp8_codes16(v, s, r_lo, r_hi, mode, w);
-        __stcs(reinterpret_cast<uint4*>(q + (int64_t)row * ldq + 16 * (int64_t)gg), make_uint4(w[0], w[1], w[2], w[3]));
     }
     flags = __reduce_or_sync(__activemask(), flags);
     if ((threadIdx.x & 31) == 0) flag_or(d_flags, flags);

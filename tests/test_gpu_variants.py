@@ -112,6 +112,33 @@ def test_fp8_degenerate_scales_and_layer(orc):
     _fp8_check(orc, inputs.c2_shape(4096, 4096))
 
 
+def _e4m3_values():
+    c = np.arange(127)
+    e, m = c >> 3, c & 7
+    return np.where(e == 0, m * 2.0 ** -9, (1 + m / 8) * 2.0 ** (e - 7.0))
+
+
+@pytest.mark.parametrize("amax", [752.0, 1000.0, 336.0, 3.3e-3, 123456.7])
+def test_fp8_near_midpoints(orc, amax):
+    """Inputs on, just below and just above every E4M3 midpoint times s (both signs), so
+    the exact decision runs in both directions and on ties; amax = 752 and 336 give an s
+    close to or equal to a short rational (336 / 448 = 0.75 exactly: true ties)."""
+    _, s, _ = orc.fp8_quant(np.zeros((1, 16), np.float32), amax)
+    v = _e4m3_values()
+    t = 0.5 * (v[:-1] + v[1:]) * float(s)                                   # exact in FP64
+    x = np.float32(t)
+    x = np.concatenate([x, np.nextafter(x, np.float32(np.inf)), np.nextafter(x, np.float32(0))])
+    x = np.concatenate([x, -x])
+    x = np.pad(x, (0, -len(x) % 16)).astype(np.float32).reshape(-1, 16)
+    _fp8_check(orc, x, amax)
+    _fp8_check(orc, inputs.f32_to_bf16_bits(x), amax)
+    # BF16 Laplace data with outlier channels at a static amax of 752: about one element in
+    # a hundred straddles a midpoint
+    xl = inputs.laplace_bf16(inputs.rng_for(0, "gpu", "fp8ties"), 257, 1024, outlier_channels=(5, 900),
+                             outlier_scale=50.0, zero_block_frac=0.01)
+    _fp8_check(orc, xl, amax)
+
+
 # ------------------------------------------------------------------ block Hadamard + FP4
 @pytest.mark.parametrize("n", [16, 32, 64, 128])
 def test_hadamard_quant_matches_oracle(orc, n):

@@ -171,18 +171,24 @@ __device__ __forceinline__ float e2m1_boundary(uint32_t k)
 }
 
 // Corrects the packed codes lo (8 elements x[0..7], element i in bits 4i..4i+3) at
-// every nibble where the bracket's other end hi disagrees; S is the block scale.
+// every nibble where the bracket's other end hi disagrees; S is the block scale.  The
+// loop runs over the differing nibbles only (usually one), so a warp whose lanes take
+// this path at different elements pays for its busiest lane, not for every position
+// (an unrolled test of all 8 positions measured 4% slower in the sweep, 1% in the
+// activation quantizer).
 __device__ __forceinline__ uint32_t e2m1_fix8(const float x[8], float S, uint32_t lo, uint32_t hi)
 {
+    uint32_t diff = lo ^ hi;
+    while (diff != 0u) {
+        const uint32_t sh = (uint32_t)(__ffs(diff) - 1) & ~3u;   // 4 x the element index
+        diff &= ~(15u << sh);
+        float xi = x[0];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const uint32_t cl = (lo >> (4 * i)) & 15u, ch = (hi >> (4 * i)) & 15u;
-        if (cl != ch) {
-            const uint32_t kl = cl & 7u;
-            const float d = fmaf(e2m1_boundary(kl), S, -fabsf(x[i]));
-            const uint32_t k = d < 0.0f ? kl + 1u : (d > 0.0f ? kl : kl + (kl & 1u));
-            lo = (lo & ~(15u << (4 * i))) | ((k | (cl & 8u)) << (4 * i));
-        }
+        for (int j = 1; j < 8; ++j) xi = sh == 4u * j ? x[j] : xi;
+        const uint32_t cl = (lo >> sh) & 15u, kl = cl & 7u;
+        const float d = fmaf(e2m1_boundary(kl), S, -fabsf(xi));
+        const uint32_t k = d < 0.0f ? kl + 1u : (d > 0.0f ? kl : kl + (kl & 1u));
+        lo = (lo & ~(15u << sh)) | ((k | (cl & 8u)) << sh);
     }
     return lo;
 }

@@ -46,7 +46,7 @@
 namespace nv4 {
 
 constexpr int kSweepThreads = 128;
-constexpr int kMaxTilesPerCta = 4;                     // a CTA sorts and searches up to 512 rows
+constexpr int kMaxTilesPerCta = 3;                     // a CTA sorts and searches up to 384 rows
 constexpr int kMaxRowsPerCta = kMaxTilesPerCta * kSweepThreads;
 constexpr float kPruneScale = 1.0f - 0x1p-10f;   // bound * this must exceed the runner-up
 
@@ -221,9 +221,12 @@ constexpr uint32_t kNoRow = 0xFFFFFFFFu;
 
 // One CTA = one block column b of one job and up to p.tiles_per_cta tiles of 128 rows.
 // Per tile the rows are counting-sorted by their starting code, so the lanes of a warp
-// walk similar candidate sequences in lockstep.
+// walk similar candidate sequences in lockstep.  Occupancy is the lever on this
+// latency-bound search: 7 CTAs per SM (72 registers, 3 row tiles of staged weights,
+// BF16 blocks staged as their 32 bytes) measured 1.34 ms on the Gemma-like layer against
+// 1.73 ms at 4 CTAs (128 registers, 4 tiles as FP32), 1.38 ms at 6 and 1.35 ms at 8.
 template <int kDt>   // 0 bf16, 2 fp32
-__global__ void __launch_bounds__(kSweepThreads, 4)
+__global__ void __launch_bounds__(kSweepThreads, 7)
 sweep_kernel(const __grid_constant__ SweepParams p)
 {
     __shared__ float4 tab[128];
@@ -232,7 +235,7 @@ sweep_kernel(const __grid_constant__ SweepParams p)
     __shared__ float4 rd4[4];
     __shared__ int bound_ok;
     __shared__ uint32_t hist[128], base[128];
-    __shared__ float4 sw[kMaxRowsPerCta][4];                 // the group's weight blocks, load order
+    __shared__ uint4 sw[kMaxRowsPerCta][kDt == 0 ? 2 : 4];  // the group's weight blocks (BF16 or FP32 bits), load order
     __shared__ uint32_t srow[kMaxRowsPerCta];                 // their rows (kNoRow past the end)
     __shared__ uint16_t perm[kMaxRowsPerCta];                 // sorted position -> load slot
 
@@ -308,7 +311,18 @@ sweep_kernel(const __grid_constant__ SweepParams p)
             for (int j = 0; j < 8; ++j) w[j] = make_float2(0.0f, 0.0f);
         }
 #pragma unroll
-        for (int j = 0; j < 4; ++j) sw[slot][j] = make_float4(w[2 * j].x, w[2 * j].y, w[2 * j + 1].x, w[2 * j + 1].y);
+        for (int j = 0; j < (kDt == 0 ? 2 : 4); ++j) {
+            if constexpr (kDt == 0) {          // the BF16 bits back from their exact FP32 values
+                uint32_t u[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    u[k] = (__float_as_uint(w[4 * j + k].y) & 0xFFFF0000u) | (__float_as_uint(w[4 * j + k].x) >> 16);
+                sw[slot][j] = make_uint4(u[0], u[1], u[2], u[3]);
+            } else {
+                sw[slot][j] = make_uint4(__float_as_uint(w[2 * j].x), __float_as_uint(w[2 * j].y),
+                                         __float_as_uint(w[2 * j + 1].x), __float_as_uint(w[2 * j + 1].y));
+            }
+        }
         srow[slot] = row;
         keys[k] = key;
         ranks[k] = atomicAdd(&hist[key], 1u);
@@ -345,11 +359,21 @@ sweep_kernel(const __grid_constant__ SweepParams p)
         const uint32_t slot = perm[32u * g + lane];
         const uint32_t row = srow[slot];
         float2 w[8];
+        if constexpr (kDt == 0) {
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const float4 v = sw[slot][j];
-            w[2 * j] = make_float2(v.x, v.y);
-            w[2 * j + 1] = make_float2(v.z, v.w);
+            for (int j = 0; j < 2; ++j) {
+                const uint4 v = sw[slot][j];
+                const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int k = 0; k < 4; ++k) w[4 * j + k] = make_float2(bf16_lo(u[k]), bf16_hi(u[k]));
+            }
+        } else {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const uint4 v = sw[slot][j];
+                w[2 * j] = make_float2(__uint_as_float(v.x), __uint_as_float(v.y));
+                w[2 * j + 1] = make_float2(__uint_as_float(v.z), __uint_as_float(v.w));
+            }
         }
         if (row == kNoRow) continue;
 
@@ -378,6 +402,10 @@ sweep_kernel(const __grid_constant__ SweepParams p)
             bool go_dn = true;
 #pragma unroll 1
             while (c >= 0) {
+                // scheduling fence: keeps the compiler from pulling the next candidate's
+                // work into this iteration; without it the kernel spills 332 bytes at 72
+                // registers and takes 1.71 ms instead of 1.34 ms on the Gemma-like layer
+                { const uint32_t am = __activemask(); asm volatile("" :: "r"(am)); }
                 const float4 t = tab[c];
                 const float2 nS = make_float2(-t.x, -t.x);
                 float2 e[8];

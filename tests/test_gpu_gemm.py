@@ -104,3 +104,21 @@ def test_gemm_large(orc):
     qa, sa = _random_operand(rng, 1024, 4096)
     qb, sb = _random_operand(rng, 1024, 4096)
     _check(orc, qa, sa, 0.5, qb, sb, 0.25, dtypes=(torch.float32,))
+
+
+# Persistent path: the grid is min(tiles, SMs), so these shapes give every CTA several
+# output tiles.  Stage counts of 1, 2 and 3 per tile (K = 256, 512, 768) move the
+# 4-deep stage ring's phase across tile boundaries in different ways; the accumulator
+# hand-off between the epilogue and the next tile's MMAs and the teardown drain run on
+# every CTA.
+@pytest.mark.parametrize("M,N,K", [
+    (4096, 4096, 512),    # 16 x 32 = 512 tiles 128 x 256, ~3.5 per CTA, 2 stages per tile
+    (4096, 3968, 512),    # 32 x 31 = 992 tiles 128 x 128 (N not a multiple of 256)
+    (4096, 4096, 256),    # 512 tiles, 1 stage per tile: the ring wraps every 4 tiles
+    (2048, 3968, 768),    # 496 tiles 128 x 128, 3 stages per tile
+])
+def test_gemm_persistent_multi_tile(orc, M, N, K):
+    rng = np.random.default_rng(M + N + K)
+    qa, sa = _random_operand(rng, M, K, lo=0x08, hi=0x7E)
+    qb, sb = _random_operand(rng, N, K, lo=0x08, hi=0x7E)
+    _check(orc, qa, sa, float(np.float32(0.37)), qb, sb, float(np.float32(1.9e-2)))

@@ -124,7 +124,9 @@ NV4_API nv4_status nv4_tensor_amax_batched(const nv4_amax_job* jobs, int n_jobs,
  * x      : bf16 [rows, cols], leading dimension ld (ld % 8 == 0).  cols % 16 == 0.
  * d_amax : device float (e.g. the output of nv4_tensor_amax), read on the device.
  * q      : [rows, cols/2] bytes, contiguous.   scales : [rows, cols/16] E4M3 bytes.
- * d_s2   : device float receiving s2.
+ * d_s2   : device float receiving s2, also when rows or cols is 0 (then x, q and scales
+ *          are not read and may be NULL).  The same holds for every entry point below that
+ *          writes a second-level scale (d_s2, d_scale) from d_amax.
  * Limit: rows * cols/16 < 2^30 blocks per call (NV4_ERR_LIMIT beyond).
  */
 NV4_API nv4_status nv4_act_quant(const void* x, int64_t rows, int64_t cols, int64_t ld,
@@ -165,7 +167,8 @@ NV4_API nv4_status nv4_weight_quant_rtn(const void* w, nv4_dtype dt, int64_t row
  * nv4_weight_quant_rtn (the job struct is nv4_act_job with w in place of x).
  * jobs: host array of n_jobs descriptors, read before the call returns (caller-owned).
  * n_jobs == 0 is a no-op; n_jobs < 0 gives NV4_ERR_SHAPE, a null table NV4_ERR_NULL and
- * more than 128 jobs NV4_ERR_LIMIT; jobs with rows or cols == 0 are skipped.  Every job
+ * more than 128 jobs NV4_ERR_LIMIT; jobs with rows or cols == 0 quantize nothing but still
+ * receive their s2 (their x, q and scales may be NULL).  Every job
  * is validated before anything is launched. */
 NV4_API nv4_status nv4_weight_quant_rtn_batched(const nv4_act_job* jobs, int n_jobs, nv4_dtype dt,
                                         uint32_t* d_flags, void* stream);
@@ -255,8 +258,14 @@ NV4_API nv4_status nv4_hessian_accum_batched(const nv4_hessian_job* jobs, int n_
  * cost1    : [rows, cols/16] float winning cost, or NULL.
  * cost2    : [rows, cols/16] float smallest cost above the winner's (+inf if none),
  *            or NULL -- a near-tie diagnostic.
- * Costs are evaluated in FP32; blocks whose best and second-best costs differ by
- * less than ~1e-6 relative may pick a different code than an exact evaluation.
+ * Accuracy: the winner is the exact argmin except where the two best costs lie within
+ * 1e-5 relative of each other.  Costs are evaluated in FP32 where the block column's
+ * Hessian bounds their error well enough for that (Gershgorin ratio rho >= ~0.6: error
+ * <= 29 * 2^-24 * (2 - rho) / rho relative); in the other columns a block whose FP32
+ * runner-up is within three times that error of the winner, every block when cost1 or
+ * cost2 is requested, and every block of a column without a valid bound (rho < 1/32,
+ * indefinite or non-finite H_b) is searched exhaustively with FP64 costs.  cost1 and
+ * cost2 are then the FP64 costs rounded to FP32.
  * The search is exact over all 127 codes but skips the cost of candidates that a
  * lower bound proves cannot be the winner or, when cost2 is requested, the runner-up
  * (sweep.cu states the bounds): codes and q are the same with or without the cost

@@ -177,7 +177,7 @@ nv4_status nv4_act_quant(const void* x, int64_t rows, int64_t cols, int64_t ld, 
                          uint8_t* scales, float* d_s2, uint32_t* d_flags, void* stream)
 {
     const nv4_status st = check_act(x, rows, cols, ld, d_amax, q, scales, d_s2);
-    if (st != NV4_OK || rows == 0 || cols == 0) return st;
+    if (st != NV4_OK) return st;
     const QuantTask t = {x, rows, cols, ld, d_amax, q, scales, nullptr, 0, d_s2};
     return from_cuda(launch_block_quant(&t, 1, 0, -1, d_flags, (cudaStream_t)stream));
 }
@@ -205,10 +205,11 @@ nv4_status nv4_weight_quant_rtn(const void* w, nv4_dtype dt, int64_t rows, int64
     if (dt != NV4_BF16 && dt != NV4_FP32) return NV4_ERR_DTYPE;
     if (rows < 0 || cols < 0 || cols % 16 != 0 || ld < cols) return NV4_ERR_SHAPE;
     if (d_amax == nullptr || d_s2 == nullptr) return NV4_ERR_NULL;
-    if (rows == 0 || cols == 0) return NV4_OK;
-    if (w == nullptr || q == nullptr || scales == nullptr) return NV4_ERR_NULL;
-    if (!aligned16(w) || !aligned16(q) || ld % (dt == NV4_BF16 ? 8 : 4) != 0) return NV4_ERR_ALIGN;
-    if (rows * (cols / 16) >= (int64_t)1 << 30) return NV4_ERR_LIMIT;
+    if (rows != 0 && cols != 0) {
+        if (w == nullptr || q == nullptr || scales == nullptr) return NV4_ERR_NULL;
+        if (!aligned16(w) || !aligned16(q) || ld % (dt == NV4_BF16 ? 8 : 4) != 0) return NV4_ERR_ALIGN;
+        if (rows * (cols / 16) >= (int64_t)1 << 30) return NV4_ERR_LIMIT;
+    }
     const QuantTask t = {w, rows, cols, ld, d_amax, q, scales, nullptr, 0, d_s2};
     return from_cuda(launch_block_quant(&t, 1, dt == NV4_BF16 ? 0 : 2, -1, d_flags, (cudaStream_t)stream));
 }
@@ -238,11 +239,12 @@ nv4_status nv4_fake_qdq(const void* x, int64_t rows, int64_t cols, int64_t ld, c
     if (out_dt != NV4_BF16 && out_dt != NV4_FP16 && out_dt != NV4_FP32) return NV4_ERR_DTYPE;
     if (rows < 0 || cols < 0 || cols % 16 != 0 || ld < cols || ld_out < cols) return NV4_ERR_SHAPE;
     if (d_amax == nullptr || d_s2 == nullptr) return NV4_ERR_NULL;
-    if (rows == 0 || cols == 0) return NV4_OK;
-    if (x == nullptr || out == nullptr) return NV4_ERR_NULL;
-    if (!aligned16(x) || !aligned16(out) || ld % 8 != 0 || ld_out % (out_dt == NV4_FP32 ? 4 : 8) != 0)
-        return NV4_ERR_ALIGN;
-    if (rows * (cols / 16) >= (int64_t)1 << 30) return NV4_ERR_LIMIT;
+    if (rows != 0 && cols != 0) {
+        if (x == nullptr || out == nullptr) return NV4_ERR_NULL;
+        if (!aligned16(x) || !aligned16(out) || ld % 8 != 0 || ld_out % (out_dt == NV4_FP32 ? 4 : 8) != 0)
+            return NV4_ERR_ALIGN;
+        if (rows * (cols / 16) >= (int64_t)1 << 30) return NV4_ERR_LIMIT;
+    }
     const QuantTask t = {x, rows, cols, ld, d_amax, nullptr, nullptr, out, ld_out, d_s2};
     return from_cuda(launch_block_quant(&t, 1, 0, (int)out_dt, d_flags, (cudaStream_t)stream));
 }
@@ -488,7 +490,8 @@ nv4_status nv4_fp8_quant(const void* x, nv4_dtype dt, int64_t rows, int64_t cols
     if (dt != NV4_BF16 && dt != NV4_FP32) return NV4_ERR_DTYPE;
     if (rows < 0 || cols < 0 || cols % 16 != 0 || ld < cols) return NV4_ERR_SHAPE;
     if (d_amax == nullptr || d_scale == nullptr) return NV4_ERR_NULL;
-    if (rows == 0 || cols == 0) return NV4_OK;
+    if (rows == 0 || cols == 0)                  // an empty tensor still receives its scale
+        return from_cuda(launch_scale_only(&d_amax, &d_scale, 1, 448.0f, d_flags, (cudaStream_t)stream));
     if (x == nullptr || q == nullptr) return NV4_ERR_NULL;
     if (!aligned16(x) || !aligned16(q) || ld % (dt == NV4_BF16 ? 8 : 4) != 0) return NV4_ERR_ALIGN;
     if (rows * (cols / 16) >= (int64_t)1 << 31) return NV4_ERR_LIMIT;
@@ -550,7 +553,8 @@ nv4_status nv4_hadamard_nvfp4_quant(const void* x, int64_t rows, int64_t cols, i
     nv4_status st = check_hadamard(x, rows, cols, ld, n);
     if (st != NV4_OK) return st;
     if (d_amax == nullptr || d_s2 == nullptr) return NV4_ERR_NULL;
-    if (rows == 0 || cols == 0) return NV4_OK;
+    if (rows == 0 || cols == 0)                  // an empty tensor still receives its s2
+        return from_cuda(launch_scale_only(&d_amax, &d_s2, 1, 2688.0f, d_flags, (cudaStream_t)stream));
     if (q == nullptr || scales == nullptr) return NV4_ERR_NULL;
     if (!aligned16(q)) return NV4_ERR_ALIGN;
     return from_cuda(launch_hadamard_quant(2, x, rows, cols, ld, n, const_cast<float*>(d_amax), q, scales, d_s2,

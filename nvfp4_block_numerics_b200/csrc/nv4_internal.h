@@ -60,6 +60,10 @@ struct DequantTask {
 constexpr int kMaxActJobs = 128;
 
 cudaError_t launch_amax(const AmaxTask* tasks, int n, int dt, uint32_t* d_flags, cudaStream_t s);
+// Second-level scales of empty tensors: d_out[i] = RN32(*d_amax[i] / divisor) for n pairs,
+// NV4_FLAG_OVERFLOW where that is not finite (one small launch; nothing else is read).
+cudaError_t launch_scale_only(const float* const* d_amax, float* const* d_out, int n, float divisor,
+                              uint32_t* d_flags, cudaStream_t s);
 cudaError_t launch_block_quant(const QuantTask* tasks, int n, int in_dt, int out_dt, uint32_t* d_flags,
                                cudaStream_t s);
 cudaError_t launch_mxfp4_quant(const void* x, int in_dt, int64_t rows, int64_t cols, int64_t ld, uint8_t* q,

@@ -533,9 +533,57 @@ cudaError_t launch_amax(const AmaxTask* tasks, int n, int dt, uint32_t* d_flags,
     return cudaGetLastError();
 }
 
+struct ScaleOnlyParams {
+    int n;
+    float divisor;
+    uint32_t* d_flags;
+    const float* d_amax[kMaxActJobs];
+    float* d_out[kMaxActJobs];
+};
+
+__global__ void __launch_bounds__(kMaxActJobs)
+scale_only_kernel(const __grid_constant__ ScaleOnlyParams p)
+{
+    const int i = threadIdx.x;
+    if (i >= p.n) return;
+    const float s2 = __fdiv_rn(*p.d_amax[i], p.divisor);
+    *p.d_out[i] = s2;
+    if (!isfinite(s2)) flag_or(p.d_flags, kFlagOverflow);
+}
+
+cudaError_t launch_scale_only(const float* const* d_amax, float* const* d_out, int n, float divisor,
+                              uint32_t* d_flags, cudaStream_t s)
+{
+    if (n <= 0) return cudaSuccess;
+    ScaleOnlyParams p;
+    p.n = n < kMaxActJobs ? n : kMaxActJobs;
+    p.divisor = divisor;
+    p.d_flags = d_flags;
+    for (int i = 0; i < p.n; ++i) {
+        p.d_amax[i] = d_amax[i];
+        p.d_out[i] = d_out[i];
+    }
+    scale_only_kernel<<<1, kMaxActJobs, 0, s>>>(p);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_block_quant(const QuantTask* tasks, int n, int in_dt, int out_dt, uint32_t* d_flags,
                                cudaStream_t s)
 {
+    // empty tensors still receive their s2
+    const float* e_amax[kMaxActJobs];
+    float* e_out[kMaxActJobs];
+    int ne = 0;
+    for (int i = 0; i < n; ++i)
+        if (tasks[i].rows == 0 || tasks[i].cols == 0) {
+            e_amax[ne] = tasks[i].d_amax;
+            e_out[ne++] = tasks[i].d_s2;
+        }
+    if (ne > 0) {
+        const cudaError_t e = launch_scale_only(e_amax, e_out, ne, 2688.0f, d_flags, s);
+        if (e != cudaSuccess) return e;
+    }
+
     QuantParams p;
     p.d_flags = d_flags;
     int m = 0;

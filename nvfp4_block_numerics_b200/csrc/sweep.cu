@@ -33,9 +33,21 @@
 // bound (1) exceeds the threshold skips the quadratic form, and once bound (2) over
 // the two largest |w_i| exceeds it, the downward walk ends.  Both comparisons
 // keep a relative margin of 2^-10, far above the FP32 evaluation error, so skipped
-// candidates could not have changed the FP32 result either.  When rho <= 0, or H_b
+// candidates could not have changed the FP32 result either.  When rho < 1/32, or H_b
 // has a zero diagonal entry with a nonzero row, or non-finite entries, the bounds are
-// off and all 127 candidates are evaluated.
+// off and all 127 candidates are evaluated, in FP64 (below).
+//
+// Accuracy.  An FP32 cost differs from the exact eT H_b e by at most
+// gamma * |e|T |H_b| |e| with gamma = 29 * 2^-24 (the longest chain of roundings a term
+// goes through in quad_form, plus the roundings of e and of H_ij + H_ji), and
+// |e|T |H_b| |e| <= (2 - rho) / rho * eT H_b e by the same Gershgorin argument, so every
+// cost of block column b is exact to eta_b = gamma (2 - rho) / rho relative.  When
+// eta_b <= 4e-6 (rho >= ~0.6) the FP32 argmin is within 1e-5 of the exact minimum, the
+// tolerance of a near tie.  Otherwise the block is searched again in FP64 when its
+// FP32 runner-up lies within 3 eta_b of the winner (or the costs are outputs), and
+// without a valid bound it is searched in FP64 from the start: the FP64 costs carry
+// errors ~1e-16 |e|T |H_b| |e|, so the winner is the exact argmin outside ties closer
+// than that.  Pruning keeps its 2^-10 margin, which exceeds 4 eta_b for rho >= 1/32.
 //
 // Ties: the lowest code wins among equal costs, and the runner-up is the smallest
 // cost strictly above the winner's, independent of the visiting order.  Identical
@@ -118,11 +130,14 @@ __device__ __forceinline__ float quad_form(const float2 e[8], const float4* __re
 }
 
 // rho * H_ii for the lower bound (1), or all zero with *ok = false when the bound
-// is not valid for this H_b.  Run by one full warp, lane i < 16 owning channel i.
-// FP32 with explicit safety margins: rsqrtf is within 2 ulp and the 15-term sum of
-// positive products within 2^-19 relative, so r * (1 + 2^-16) + 2^-16 bounds the
-// exact Gershgorin radius from above.
-__device__ void block_bound(const float* __restrict__ hs, float* rd, int* ok)
+// is not valid for this H_b (or rho < 1/32, where it would prune nothing).  Run by one
+// full warp, lane i < 16 owning channel i.  FP32 with explicit safety margins: rsqrtf
+// is within 2 ulp and the 15-term sum of positive products within 2^-19 relative, so
+// r * (1 + 2^-16) + 2^-16 bounds the exact Gershgorin radius from above.  *eta receives
+// the relative error bound of this column's FP32 costs (+inf without a bound).
+constexpr float kCostGamma = 29.0f * 0x1p-24f;     // roundings per term of quad_form, plus e and H_ij + H_ji
+constexpr float kCertifiedEta = 4e-6f;             // FP32 argmin within 1e-5 of the exact minimum
+__device__ void block_bound(const float* __restrict__ hs, float* rd, int* ok, float* eta)
 {
     const int lane = threadIdx.x & 31;
     const int i = lane & 15;
@@ -142,9 +157,12 @@ __device__ void block_bound(const float* __restrict__ hs, float* rd, int* ok)
     for (int o = 8; o > 0; o >>= 1) r = fmaxf(r, __shfl_xor_sync(0xffffffffu, r, o));
     bad = __any_sync(0xffffffffu, bad || !(r <= 3.0e38f));
     const float rho = 1.0f - fmaf(r, 1.0f + 0x1p-16f, 0x1p-16f);
-    const bool good = !bad && rho > 0.0f;
+    const bool good = !bad && rho >= 0x1p-5f;
     if (lane < 16) rd[lane] = good ? __fmul_rd(rho, di) : 0.0f;
-    if (lane == 0) *ok = good ? 1 : 0;
+    if (lane == 0) {
+        *ok = good ? 1 : 0;
+        *eta = good ? __fdiv_ru(__fmul_ru(kCostGamma, 2.0f - rho), rho) : __int_as_float(0x7F800000);
+    }
 }
 
 // E2M1 codes of 8 weights (4 pairs) at candidate t = {S, r_lo, r_hi, exact}: both ends of
@@ -217,6 +235,90 @@ __device__ __forceinline__ void load_block(const SweepJobDev& job, uint32_t row,
     }
 }
 
+// Signed weights of a staged block (BF16 as its 32 bytes, FP32 as its 64).
+template <int kDt>
+__device__ __forceinline__ void unstage_block(const uint4* __restrict__ src, float2 w[8])
+{
+    if constexpr (kDt == 0) {
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            const uint4 v = src[j];
+            const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) w[4 * j + k] = make_float2(bf16_lo(u[k]), bf16_hi(u[k]));
+        }
+    } else {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const uint4 v = src[j];
+            w[2 * j] = make_float2(__uint_as_float(v.x), __uint_as_float(v.y));
+            w[2 * j + 1] = make_float2(__uint_as_float(v.z), __uint_as_float(v.w));
+        }
+    }
+}
+
+struct Search64 {
+    double best, second;
+    uint32_t code;
+};
+
+// The exhaustive search of one block with every cost in FP64, by a whole warp: lane l
+// takes candidates l, l + 32, l + 64, l + 96.  e_i = w_i - v_i S_c is exact in FP64
+// (v_i S_c has at most 27 significant bits) and eT H_b e is summed as in quad_form; the
+// element codes are the same exact decisions as in the FP32 search.  Winner: smallest
+// cost, ties to the lowest code; runner-up: the smallest cost above the winner's.  Used
+// for the blocks whose FP32 costs cannot certify the argmin, after the FP32 walk and
+// out of line, so that it costs the walk no registers.
+template <int kDt>
+__device__ __noinline__ Search64 search_fp64_warp(const uint4* __restrict__ src, const float4* __restrict__ tab,
+                                                  const float* __restrict__ hs)
+{
+    const uint32_t lane = threadIdx.x & 31u;
+    const double inf = __longlong_as_double(0x7FF0000000000000ll);
+    float2 w[8];
+    unstage_block<kDt>(src, w);
+    double b1 = inf, b2 = inf;       // this lane's best and its smallest cost above it
+    uint32_t bc = 0u;
+#pragma unroll 1
+    for (uint32_t c = lane; c < 127u; c += 32u) {
+        const float4 t = tab[c];
+        uint32_t q0, q1;
+        codes8h(w, t, q0);
+        codes8h(w + 4, t, q1);
+        float2 v[8];
+        decode8h(q0, v);
+        decode8h(q1, v + 4);
+        double e[16];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            e[2 * j] = fma(-(double)v[j].x, (double)t.x, (double)w[j].x);
+            e[2 * j + 1] = fma(-(double)v[j].y, (double)t.x, (double)w[j].y);
+        }
+        double cost = 0.0;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            double z = (double)hs[17 * i] * e[i];
+#pragma unroll
+            for (int j = i + 1; j < 16; ++j) z = fma((double)hs[16 * i + j] + (double)hs[16 * j + i], e[j], z);
+            cost = fma(e[i], z, cost);
+        }
+        if (cost < b1) { b2 = b1; b1 = cost; bc = c; }   // ascending c: equal costs keep the lower code
+        else if (cost > b1 && cost < b2) b2 = cost;
+    }
+    double B = b1;
+    uint32_t C = bc;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const double ob = __shfl_xor_sync(0xffffffffu, B, o);
+        const uint32_t oc = __shfl_xor_sync(0xffffffffu, C, o);
+        if (ob < B || (ob == B && oc < C)) { B = ob; C = oc; }
+    }
+    double s2 = b1 > B ? b1 : b2;    // this lane's smallest cost above the winner's
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s2 = fmin(s2, __shfl_xor_sync(0xffffffffu, s2, o));
+    return Search64{B, s2, C};
+}
+
 constexpr uint32_t kNoRow = 0xFFFFFFFFu;
 
 // One CTA = one block column b of one job and up to p.tiles_per_cta tiles of 128 rows.
@@ -234,7 +336,12 @@ sweep_kernel(const __grid_constant__ SweepParams p)
     __shared__ float hs[256];
     __shared__ float4 rd4[4];
     __shared__ int bound_ok;
-    __shared__ uint32_t hist[128], base[128];
+    __shared__ float eta_s;
+    __shared__ uint32_t sortbuf[256];                         // bucket counts and bases of the sort,
+    uint32_t* const hist = sortbuf;                           // then the list of rows left to the
+    uint32_t* const base = sortbuf + 128;                     // FP64 search (384 slots, 768 bytes)
+    uint16_t* const redo_list = reinterpret_cast<uint16_t*>(sortbuf);
+    __shared__ uint32_t n_redo;
     __shared__ uint4 sw[kMaxRowsPerCta][kDt == 0 ? 2 : 4];  // the group's weight blocks (BF16 or FP32 bits), load order
     __shared__ uint32_t srow[kMaxRowsPerCta];                 // their rows (kNoRow past the end)
     __shared__ uint16_t perm[kMaxRowsPerCta];                 // sorted position -> load slot
@@ -277,9 +384,10 @@ sweep_kernel(const __grid_constant__ SweepParams p)
     for (int k = threadIdx.x; k < 256; k += kSweepThreads) hs[k] = job.H[(int64_t)b * 256 + k];
     __syncthreads();
     build_hpairs(hs, hp);
-    if (threadIdx.x >= 96) block_bound(hs, reinterpret_cast<float*>(rd4), &bound_ok);
+    if (threadIdx.x >= 96) block_bound(hs, reinterpret_cast<float*>(rd4), &bound_ok, &eta_s);
     __syncthreads();
     const bool pr = bound_ok != 0;
+    const float eta = eta_s;                                    // relative error bound of the FP32 costs
     const float k6 = __frcp_rn(__fmul_rn(6.0f, s2));            // ~ 1/(6 s2), for the starting code
     const float* rd = reinterpret_cast<const float*>(rd4);
     const uint32_t s2flag = isfinite(s2) ? 0u : kFlagOverflow;
@@ -350,6 +458,8 @@ sweep_kernel(const __grid_constant__ SweepParams p)
         perm[base[keys[k]] + ranks[k]] = (uint16_t)(k * kSweepThreads + threadIdx.x);
     }
     __syncthreads();
+    if (threadIdx.x == 0) n_redo = 0u;                       // base[] has been read by every thread
+    __syncthreads();
 
     // ---- each warp walks interleaved groups of 32 sorted rows, without further barriers
     const uint32_t nslots = ntile * kSweepThreads;
@@ -359,22 +469,7 @@ sweep_kernel(const __grid_constant__ SweepParams p)
         const uint32_t slot = perm[32u * g + lane];
         const uint32_t row = srow[slot];
         float2 w[8];
-        if constexpr (kDt == 0) {
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                const uint4 v = sw[slot][j];
-                const uint32_t u[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                for (int k = 0; k < 4; ++k) w[4 * j + k] = make_float2(bf16_lo(u[k]), bf16_hi(u[k]));
-            }
-        } else {
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const uint4 v = sw[slot][j];
-                w[2 * j] = make_float2(__uint_as_float(v.x), __uint_as_float(v.y));
-                w[2 * j + 1] = make_float2(__uint_as_float(v.z), __uint_as_float(v.w));
-            }
-        }
+        unstage_block<kDt>(sw[slot], w);
         if (row == kNoRow) continue;
 
         // ---- the search for this thread's (row, b)
@@ -391,10 +486,14 @@ sweep_kernel(const __grid_constant__ SweepParams p)
         // the threshold a candidate's lower bound must exceed to be skipped: the
         // runner-up cost when it is an output, else the best cost
         const bool need2 = job.cost2 != nullptr;
+        const bool need_costs = need2 || job.cost1 != nullptr;
         float best = __int_as_float(0x7F800000), second = best, thr = best;
         uint32_t best_c = 0u;
+        bool redo = false;
         if (a1 == 0.0f) {
             best = 0.0f;                  // all-zero block: every candidate has e = w = 0
+        } else if (!pr) {                 // no valid bound: all 127 candidates, in FP64
+            redo = true;
         } else {
             const float t0 = __fmul_rn(a1, k6);
             int c = (int)min(cvt_e4m3x2(t0, t0) & 0x7Fu, 126u);
@@ -457,6 +556,14 @@ sweep_kernel(const __grid_constant__ SweepParams p)
                 else if (up <= 126) { c = up++; go_dn = true; }
                 else c = -1;
             }
+            // FP32 costs exact to eta relative: a runner-up within 3 eta of the winner (or
+            // costs that are outputs) needs the FP64 search unless eta certifies the argmin
+            redo = eta > kCertifiedEta && (need_costs || !(second > fmaf(best, 3.0f * eta, best)));
+        }
+        if (redo) {                       // decided later by the FP64 search of a whole warp
+            flag_or(p.d_flags, flags);
+            redo_list[atomicAdd(&n_redo, 1u)] = (uint16_t)slot;
+            continue;
         }
         if (!isfinite(best)) flags |= kFlagNonFinite;
 
@@ -472,6 +579,33 @@ sweep_kernel(const __grid_constant__ SweepParams p)
         if (job.cost1 != nullptr) job.cost1[blk] = best;
         if (job.cost2 != nullptr) job.cost2[blk] = second;
         flag_or(p.d_flags, flags);
+    }
+
+    // ---- blocks whose FP32 costs do not certify the argmin: exhaustive FP64 search, one warp each
+    __syncthreads();
+    const uint32_t nr = n_redo;
+#pragma unroll 1
+    for (uint32_t i = warp; i < nr; i += kSweepThreads / 32) {
+        const uint32_t slot = redo_list[i];
+        const Search64 r = search_fp64_warp<kDt>(sw[slot], tab, hs);
+        if (lane == 0) {
+            const int64_t blk = (int64_t)srow[slot] * job.nblk + b;
+            job.codes[blk] = (uint8_t)r.code;
+            if (job.q != nullptr) {
+                float2 w[8];
+                unstage_block<kDt>(sw[slot], w);
+                uint32_t c0, c1;
+                const float4 tw = tab[r.code];
+                codes8h(w, tw, c0);
+                codes8h(w + 4, tw, c1);
+                *reinterpret_cast<uint2*>(job.q + blk * 8) = make_uint2(c0, c1);
+            }
+            if (job.cost1 != nullptr) job.cost1[blk] = (float)r.best;
+            if (job.cost2 != nullptr) job.cost2[blk] = (float)r.second;
+            if (!(fabs(r.best) <= 1.7e308)) flag_or(p.d_flags, kFlagNonFinite);
+            nhalf += 2u * 127u;
+            nfull += 127u;
+        }
     }
     if (job.d_work != nullptr) {
         __syncwarp();

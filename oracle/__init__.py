@@ -498,3 +498,64 @@ def hadamard_rotate(x: np.ndarray, n: int) -> np.ndarray:
     z = xf.astype(np.float64).reshape(rows, cols // n, n) @ _sylvester(n)     # H_n is symmetric
     c = float(np.float64(1.0) / np.sqrt(np.float64(n)))
     return (z * c).astype(np.float32).reshape(rows, cols)
+
+
+def _rn32_of_int(N: int, k: int) -> float:
+    """RN32(N * 2^k) for an integer N, ties to even, with FP32 subnormals and overflow to
+    infinity; returned as a Python float (exactly representable)."""
+    if N == 0:
+        return 0.0
+    sign = -1.0 if N < 0 else 1.0
+    N = abs(N)
+    e = N.bit_length() - 1 + k                  # exponent of the leading bit
+    lsb = max(e - 23, -149)                     # exponent of the last bit FP32 keeps
+    shift = lsb - k
+    if shift > 0:
+        q, r = divmod(N, 1 << shift)
+        half = 1 << (shift - 1)
+        if r > half or (r == half and q & 1):
+            q += 1
+    else:
+        q = N << (-shift)
+    v = float(q) * 2.0 ** lsb                   # q <= 2^24: exact
+    return sign * v if v < 2.0 ** 128 else sign * float("inf")
+
+
+def hadamard2_rotate(w: np.ndarray, n: int) -> np.ndarray:
+    """Two-sided block Hadamard rotation of weight tiles ([FP4] section 3.1: the weight
+    matrix is cut into n x n tiles, n = 16 or 32, and each tile B becomes
+    (H / sqrt(n)) B (H / sqrt(n))^T = H B H^T / n, H the natural-order Hadamard matrix).
+    Reading: y = RN32(exact(H B H^T) / n): 1/n is a power of two, so the final rounding to
+    FP32 is the only one.  The tile's sums are formed in FP64 where that is exact (every
+    value an integer multiple of the tile's smallest unit in the last place, and the sums,
+    with their 2 log2(n) bits of growth, inside 53 bits), else in Python integers.
+    w: float32 or uint16 (bf16 bits) [rows, cols], rows and cols multiples of n.
+    Returns float32 [rows, cols]."""
+    assert n in (16, 32) and w.ndim == 2 and w.shape[0] % n == 0 and w.shape[1] % n == 0
+    wf = (w.astype(np.uint32) << 16).view(np.float32) if w.dtype == np.uint16 else w
+    rows, cols = wf.shape
+    H = _sylvester(n)
+    growth = 2 * int(np.log2(n))
+    out = np.empty((rows, cols), np.float32)
+    for r0 in range(0, rows, n):
+        for c0 in range(0, cols, n):
+            B = wf[r0:r0 + n, c0:c0 + n].astype(np.float64)
+            nz = np.abs(B[B != 0.0])
+            if nz.size == 0:
+                out[r0:r0 + n, c0:c0 + n] = 0.0
+                continue
+            hi = int(np.frexp(nz.max())[1])                      # 2^(hi-1) <= max < 2^hi
+            ulp = int(np.frexp(nz)[1].min()) - 24                 # every FP32 value is a multiple of 2^ulp
+            ulp = max(ulp, -149)
+            if hi - ulp + growth <= 53:
+                Y = H @ B @ H.T                                   # exact: integers times 2^ulp below 2^53
+                out[r0:r0 + n, c0:c0 + n] = (Y / n).astype(np.float32)
+            else:
+                Bi = np.array([[int(v) for v in row] for row in np.ldexp(B, -ulp)], dtype=object)
+                Hi = H.astype(np.int64).astype(object)
+                Yi = Hi.dot(Bi).dot(Hi.T)
+                lg = int(np.log2(n))
+                for i in range(n):
+                    for j in range(n):
+                        out[r0 + i, c0 + j] = _rn32_of_int(int(Yi[i, j]), ulp - lg)
+    return out

@@ -12,17 +12,23 @@ One step is one pass of the whole hot path over one batch of synthetic input:
            [16384 x 16384], the four weight amaxes, and the Hessian-weighted
            E4M3 scale sweep with NVFP4 pack of q_proj, gate, up and down (6.55 M
            blocks, one batched launch);
+  moe   -- an MoE layer's expert calibration: local Hessians of the 64 experts'
+           routed inputs X [2048 x 4096] and down-projection inputs [2048 x 1536]
+           (128 Hessians, one batched launch), the 192 weight amaxes, and the
+           Hessian-weighted sweep with pack of all 192 gate/up/down matrices
+           (Student-t weights, 75.5 M blocks, one batched launch);
   cast  -- MXFP4 -> NVFP4 cast of 32 expert matrices 2880 x 2880 (one launch).
 
 `value` is the first half of the metric, NVFP4 quant GB/s: algorithmic bytes of
 the act part (amax 2 B, quantize 2.5625 B, dequantize 2.5625 B per element) over
 its device time.  The second half, scale-sweep blocks/s against the FP32 pipe, is
-reported in `sweep`.  Each part runs as a CUDA graph; timing uses CUDA events on
+reported in `sweep` (the dense layer) and `sweep_moe` (the expert stack); the FP32
+peak is measured in the same run by an FMA microbenchmark (scalar and packed).  Each part runs as a CUDA graph; timing uses CUDA events on
 the launching stream.  Every step touches ~5 GB, more than the 126 MB L2, so no
 extra flush is inserted between steps.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-       [--parts act,calib,cast] (a subset, e.g. for profiling one kernel)
+       [--parts act,calib,moe,cast] (a subset, e.g. for profiling one kernel)
 Under torchrun every rank runs its own replica of the step on its own GPU
 (independent problems, no collective on the data path: weak scaling); times are
 the max over ranks.
@@ -56,7 +62,8 @@ SWEEP_FLOP_PER_HALF = 8 + 16 + 24         # executed: per visited candidate half
 SWEEP_FLOP_PER_COST = 272                 # executed: per evaluated cost
 ACT_BYTES = {"amax": 2.0, "act_quant": 2.5625, "dequant": 2.5625}
 CAST_BYTES_PER_MX_BLOCK = 1 + 16 + 16 + 2  # read E8M0 + nibbles, write nibbles + 2 E4M3 scales
-FP32_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12   # SMs x FP32 lanes x FMA x max clock
+FP32_NOMINAL_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12   # SMs x FP32 lanes x FMA x max clock
+N_EXPERTS = 64
 
 
 def parse_args():
@@ -65,12 +72,16 @@ def parse_args():
     p.add_argument("--steps", type=int, default=10)
     p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    p.add_argument("--parts", default="act,calib,cast")
+    p.add_argument("--parts", default="act,calib,moe,cast")
     p.add_argument("--seed", type=int, default=0)
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-rooflines", action="store_true",
                    help="skip the per-kernel micro-timings (for launch-list profiling of the step alone)")
+    p.add_argument("--profile", default=None, choices=sorted(PROFILE_CASES),
+                   help="run only one kernel, --profile-reps times, on a case sized for an ncu capture "
+                        "(inputs above the L2, a few GB at most); prints nothing but a one-line summary")
+    p.add_argument("--profile-reps", type=int, default=3)
     return p.parse_args()
 
 
@@ -182,6 +193,32 @@ def build_workload(parts, seed, dev):
                 codes=torch.empty((rows, cols // 16), dtype=torch.uint8, device=dev),
                 q=torch.empty((rows, cols // 2), dtype=torch.uint8, device=dev)))
         W["host"]["c3"] = d
+    if "moe" in parts:
+        from concurrent.futures import ThreadPoolExecutor
+
+        def expert(e):
+            d = inputs.c4_expert(e, seed)
+            return {k: bf16(v) for k, v in d.items()}
+
+        with ThreadPoolExecutor(max(1, min(16, os.cpu_count() or 1))) as ex:
+            experts = list(ex.map(expert, range(N_EXPERTS)))
+        W["moe_X"] = [d["X"] for d in experts]
+        W["moe_Xd"] = [d["X_down"] for d in experts]
+        W["moe_H"] = torch.zeros((N_EXPERTS, 4096 // 16, 16, 16), dtype=torch.float32, device=dev)
+        W["moe_Hd"] = torch.zeros((N_EXPERTS, 1536 // 16, 16, 16), dtype=torch.float32, device=dev)
+        W["moe_amax"] = torch.zeros(3 * N_EXPERTS, dtype=torch.float32, device=dev)
+        W["moe_weights"] = []
+        for e, d in enumerate(experts):
+            for k, name in enumerate(("W_gate", "W_up", "W_down")):
+                w = d[name]
+                rows, cols = w.shape
+                i = 3 * e + k
+                W["moe_weights"].append(dict(
+                    name=f"e{e}/{name}", w=w, H=W["moe_Hd"][e] if name == "W_down" else W["moe_H"][e],
+                    d_amax_w=W["moe_amax"][i:i + 1],
+                    codes=torch.empty((rows, cols // 16), dtype=torch.uint8, device=dev),
+                    q=torch.empty((rows, cols // 2), dtype=torch.uint8, device=dev)))
+        del experts
     if "cast" in parts:
         jobs = []
         for i in range(32):
@@ -225,6 +262,22 @@ def part_calib(W):
                                  for j in W["weights"]], W["flags"])
 
 
+def part_moe(W):
+    """The expert stack's calibration: 128 Hessians in one launch, 192 weight amaxes (two
+    launches of at most 128 tensors), one sweep launch over all 192 matrices."""
+    from nvfp4_block_numerics_b200 import binding as nv4
+
+    W["moe_H"].zero_()
+    W["moe_Hd"].zero_()
+    W["moe_amax"].zero_()
+    nv4.nv4_hessian_accum_batched(W["moe_X"] + W["moe_Xd"], list(W["moe_H"]) + list(W["moe_Hd"]), W["flags"])
+    mw = W["moe_weights"]
+    for k in range(0, len(mw), 128):
+        nv4.nv4_tensor_amax_batched([j["w"] for j in mw[k:k + 128]], [j["d_amax_w"] for j in mw[k:k + 128]],
+                                    W["flags"])
+    nv4.nv4_scale_sweep_batched([{k: j[k] for k in ("w", "H", "d_amax_w", "codes", "q")} for j in mw], W["flags"])
+
+
 def part_cast(W):
     from nvfp4_block_numerics_b200 import binding as nv4
 
@@ -232,8 +285,8 @@ def part_cast(W):
     nv4.nv4_mxfp4_to_nvfp4_batched(W["cast"], W["counts"], W["flags"])
 
 
-PARTS = {"act": part_act, "calib": part_calib, "cast": part_cast}
-LAUNCHES = {"act": 3, "calib": 3, "cast": 2}
+PARTS = {"act": part_act, "calib": part_calib, "moe": part_moe, "cast": part_cast}
+LAUNCHES = {"act": 3, "calib": 3, "moe": 4, "cast": 2}   # launches of this library's kernels per part
 
 
 def traffic_table():
@@ -296,7 +349,62 @@ def time_launch(fn, reps=20, flush=None):
     return tot / reps / 1e3
 
 
-def kernel_rooflines(W, hbm_peak):
+def fp32_peak(dev, reps=5):
+    """The FP32 pipe's throughput on this GPU, measured: the library's FMA microbenchmark
+    (16 independent chains per thread, 148 x 8 CTAs of 256 threads), scalar and packed
+    two-lane FMAs, best of `reps` event-timed launches each."""
+    import torch
+
+    from nvfp4_block_numerics_b200 import binding as nv4
+
+    blocks = torch.cuda.get_device_properties(dev).multi_processor_count * 8
+    iters = 4096
+    sink = torch.zeros(blocks, dtype=torch.float32, device=dev)
+    out = {}
+    for packed in (False, True):
+        nv4.nv4_fp32_probe(packed, blocks, iters, sink)
+        torch.cuda.synchronize()
+        best = None
+        s = torch.cuda.current_stream()
+        for _ in range(reps):
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(s)
+            nv4.nv4_fp32_probe(packed, blocks, iters, sink)
+            b.record(s)
+            b.synchronize()
+            t = a.elapsed_time(b) / 1e3
+            best = t if best is None else min(best, t)
+        out["packed" if packed else "scalar"] = blocks * 256.0 * iters * 32 / best / 1e12
+    out["measured"] = max(out["scalar"], out["packed"])
+    out["nominal"] = FP32_NOMINAL_TFLOPS
+    out["how"] = (f"nv4_fp32_probe: {blocks} CTAs x 256 threads x {iters} rounds x 32 FLOP of independent FMAs, "
+                  f"scalar fma.rn.f32 and packed fma.rn.f32x2, best of {reps} event-timed launches each")
+    return out
+
+
+def sweep_row(nv4, jobs, flags, label, fp32):
+    """Roofline row of one batched sweep launch (the production call, codes + nibbles):
+    blocks/s, the algorithmic count against the measured FP32 peak, and the executed work
+    from the kernel's device counters (one extra launch)."""
+    import torch
+
+    blocks = sum(j["codes"].numel() for j in jobs)
+    work = torch.zeros(2, dtype=torch.int64, device=flags.device)
+    nv4.nv4_scale_sweep_batched([dict(j, d_work=work) for j in jobs], flags)
+    torch.cuda.synchronize()
+    halves, costs = (int(x) for x in work.tolist())
+    t = time_launch(lambda: nv4.nv4_scale_sweep_batched(jobs, flags), reps=5)
+    executed = SWEEP_FLOP_PER_HALF * halves + SWEEP_FLOP_PER_COST * costs
+    return {"bound": "alu", "flops": SWEEP_FLOP_PER_BLOCK * blocks, "blocks": blocks, "s": t,
+            "half_visits_per_block": halves / blocks, "costs_per_block": costs / blocks,
+            "executed_tflops": executed / t / 1e12,
+            "executed_frac": executed / t / 1e12 / fp32["measured"],
+            "executed_frac_nominal": executed / t / 1e12 / fp32["nominal"],
+            "launch": label}
+
+
+def kernel_rooflines(W, hbm_peak, fp32):
     """Per-kernel achieved throughput on each kernel's largest launch of the step."""
     import torch
 
@@ -368,20 +476,17 @@ def kernel_rooflines(W, hbm_peak):
                                 "launch": f"X [{X.shape[0]}, {X.shape[1]}] + X_down [{Xd.shape[0]}, {Xd.shape[1]}] bf16, "
                                           "one batched launch"}
         jobs = [{k: j[k] for k in ("w", "H", "d_amax_w", "codes", "q")} for j in W["weights"]]
-        blocks = sum(j["codes"].numel() for j in W["weights"])
-        # executed work, counted on the device in one extra launch
-        work = torch.zeros(2, dtype=torch.int64, device=W["flags"].device)
-        nv4.nv4_scale_sweep_batched([dict(j, d_work=work) for j in jobs], W["flags"])
-        torch.cuda.synchronize()
-        halves, costs = (int(x) for x in work.tolist())
-        t = time_launch(lambda: nv4.nv4_scale_sweep_batched(jobs, W["flags"]), reps=5)
-        executed = SWEEP_FLOP_PER_HALF * halves + SWEEP_FLOP_PER_COST * costs
-        out["scale_sweep"] = {"bound": "alu", "flops": SWEEP_FLOP_PER_BLOCK * blocks,
-                              "blocks": blocks, "s": t, "half_visits_per_block": halves / blocks,
-                              "costs_per_block": costs / blocks,
-                              "executed_tflops": executed / t / 1e12,
-                              "executed_frac": executed / t / 1e12 / FP32_PEAK_TFLOPS,
-                              "launch": "q_proj + gate + up + down, one batched launch"}
+        out["scale_sweep"] = sweep_row(nv4, jobs, W["flags"], "q_proj + gate + up + down, one batched launch", fp32)
+    if "moe_weights" in W:
+        Xs, Hs = W["moe_X"] + W["moe_Xd"], list(W["moe_H"]) + list(W["moe_Hd"])
+        t = time_launch(lambda: nv4.nv4_hessian_accum_batched(Xs, Hs, W["flags"]), reps=10, flush=flush)
+        out["hessian_accum_moe"] = {"bound": "hbm", "bytes": 2.0 * sum(x.numel() for x in Xs), "s": t,
+                                    "launch": f"{len(W['moe_X'])} x [2048, 4096] + {len(W['moe_Xd'])} x [2048, 1536] "
+                                              "bf16, one batched launch"}
+        jobs = [{k: j[k] for k in ("w", "H", "d_amax_w", "codes", "q")} for j in W["moe_weights"]]
+        out["scale_sweep_moe"] = sweep_row(nv4, jobs, W["flags"],
+                                           f"{len(jobs)} expert matrices (gate/up [1536, 4096], down [4096, 1536]), "
+                                           "one batched launch", fp32)
     if "calib" in W or "act" in W:
         # W4A4 GEMM (a widening of the path; not part of the step): a 16384-token batch
         # through the gate projection 2048 -> 16384 and a square 8192^3 product, random
@@ -416,7 +521,7 @@ def kernel_rooflines(W, hbm_peak):
             v["unit"] = "TFLOP/s"
         else:
             v["achieved"] = v["flops"] / v["s"] / 1e12
-            v["peak"] = FP32_PEAK_TFLOPS
+            v["peak"] = fp32["measured"]
             v["unit"] = "TFLOP/s"
             v["blocks_per_s"] = v["blocks"] / v["s"]
         v["frac"] = v["achieved"] / v["peak"]
@@ -530,10 +635,33 @@ def cpu_baseline(seed, budget_s=20.0):
         if el > budget_s / 2:
             break
     sweep_bps = n_blocks / el
+    moe_bps, moe_blocks = _oracle_moe_sweep(seed, threads, budget_s / 4)
     return {"value": act_gbs, "unit": "GB/s", "cores": threads, "kind": "oracle",
             "sample": f"act path on min(T,256) rows of each of the 15 [T, C] shapes ({nelem} elements, "
-                      f"{reps} reps); sweep on {len(rows)} rows x 128 blocks of q_proj, {n_blocks} blocks",
-            "sweep_blocks_per_s": sweep_bps}
+                      f"{reps} reps); sweep on {len(rows)} rows x 128 blocks of q_proj, {n_blocks} blocks; "
+                      f"expert sweep on 32 rows x 256 blocks of expert 0's gate projection, {moe_blocks} blocks",
+            "sweep_blocks_per_s": sweep_bps, "sweep_moe_blocks_per_s": moe_bps}
+
+
+def _oracle_moe_sweep(seed, threads, budget_s):
+    """The oracle's sweep on 32 rows of one expert's gate projection (Student-t weights,
+    its routed input's Hessian): blocks/s on this host."""
+    import oracle
+    from nvfp4_block_numerics_b200 import inputs
+
+    d = inputs.c4_expert(0, seed + 1000, which=("X", "W_gate"))
+    H = oracle.hessian_accum(d["X"], threads=threads)
+    amax, _ = oracle.tensor_amax(d["W_gate"], threads)
+    rows = np.arange(32)
+    n = 0
+    tt = time.perf_counter()
+    while True:
+        oracle.scale_sweep(d["W_gate"], H, amax, rows=rows, threads=threads)
+        n += len(rows) * (d["W_gate"].shape[1] // 16)
+        el = time.perf_counter() - tt
+        if el > budget_s:
+            break
+    return n / el, n
 
 
 # ---------------------------------------------------------------------- arms
@@ -541,8 +669,9 @@ def workload_config(parts, seed, ws):
     """The workload both arms report (the reference arm times a bounded sample of it)."""
     return {"workload": "NVFP4 hot path: activation quant sweep (15 [T,C] shapes, amax->quant->dequant) "
                         "+ Gemma-2B-like layer calibration (Hessians of X 16384x2048 and 16384x16384, "
-                        "sweep of q/gate/up/down -> winning E4M3 codes + packed E2M1) + MXFP4->NVFP4 cast "
-                        "of 32 x 2880x2880",
+                        "sweep of q/gate/up/down -> winning E4M3 codes + packed E2M1) + MoE expert stack "
+                        "calibration (64 experts: 128 Hessians of 2048-token inputs, sweep of 192 gate/up/down "
+                        "matrices, 75.5 M blocks) + MXFP4->NVFP4 cast of 32 x 2880x2880",
             "parts": list(parts), "seed": seed, "parallelism": f"replicas x{ws}",
             "l2": "no flush between steps: every step touches ~5 GB, above the 126 MB L2; per-kernel "
                   "rooflines: graph replay after writing then reading two 256 MB buffers"}
@@ -558,8 +687,8 @@ def dist_setup(args):
 def run_reference(args):
     """The oracle (plain CPU code, FP64) as the reference arm: each step runs a bounded sample
     of the same workload on the host cores -- the activation path on <= 64 rows of every
-    shape (the metric's GB/s half) and the Hessian-weighted sweep on 64 rows x 128 blocks of
-    q_proj (its blocks/s half)."""
+    shape (the metric's GB/s half), and the Hessian-weighted sweep on 64 rows x 128 blocks of
+    q_proj and on 32 rows x 256 blocks of one expert's gate projection (its blocks/s half)."""
     ws, rank, _ = dist_setup(args)
     if rank != 0:
         return
@@ -574,7 +703,12 @@ def run_reference(args):
     wq = np.ascontiguousarray(d["W_q"][:64])
     amax_w = oracle.tensor_amax(d["W_q"], threads)[0]
     n_blocks = wq.size // 16
-    t_act, t_sweep = [0.0], [0.0]
+    e0 = inputs.c4_expert(0, args.seed, which=("X", "W_gate"))
+    He = oracle.hessian_accum(e0["X"], threads=threads)
+    we = np.ascontiguousarray(e0["W_gate"][:32])
+    amax_e = oracle.tensor_amax(e0["W_gate"], threads)[0]
+    n_blocks_e = we.size // 16
+    t_act, t_sweep, t_moe = [0.0], [0.0], [0.0]
 
     def step():
         t0 = time.perf_counter()
@@ -585,25 +719,31 @@ def run_reference(args):
         t1 = time.perf_counter()
         oracle.scale_sweep(wq, H, amax_w, threads=threads)
         t2 = time.perf_counter()
+        oracle.scale_sweep(we, He, amax_e, threads=threads)
+        t3 = time.perf_counter()
         t_act[0] += t1 - t0
         t_sweep[0] += t2 - t1
+        t_moe[0] += t3 - t2
 
     for _ in range(args.warmup):
         step()
-    t_act[0] = t_sweep[0] = 0.0
+    t_act[0] = t_sweep[0] = t_moe[0] = 0.0
     t = time.perf_counter()
     for _ in range(args.steps):
         step()
     el = (time.perf_counter() - t) / args.steps
     v = nelem * sum(ACT_BYTES.values()) / (t_act[0] / args.steps) / 1e9
     sweep_bps = n_blocks / (t_sweep[0] / args.steps)
+    moe_bps = n_blocks_e / (t_moe[0] / args.steps)
     sample = (f"act path on min(T,64) rows of each of the 15 [T, C] shapes ({nelem} elements per step); "
-              f"sweep on 64 rows x 128 blocks of q_proj ({n_blocks} blocks per step, H from 2048 tokens)")
+              f"sweep on 64 rows x 128 blocks of q_proj ({n_blocks} blocks per step, H from 2048 tokens); "
+              f"expert sweep on 32 rows x 256 blocks of expert 0's gate projection ({n_blocks_e} blocks per step)")
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "GB/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": el * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": workload_config(args.parts.split(","), args.seed, 1),
             "sweep": {"value": sweep_bps, "unit": "blocks/s"},
+            "sweep_moe": {"value": moe_bps, "unit": "blocks/s"},
             "cpu_baseline": {"value": v, "unit": "GB/s", "cores": threads, "kind": "oracle", "sample": sample},
             "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -669,7 +809,8 @@ def run_ours(args):
     part_s = {p: t[i + 1] for i, p in enumerate(parts)}
     flags = int(W["flags"].item())
 
-    roof = {} if args.no_rooflines else kernel_rooflines(W, hbm_peak)
+    fp32 = fp32_peak(dev)
+    roof = {} if args.no_rooflines else kernel_rooflines(W, hbm_peak, fp32)
     e2e = None
     if "act" in parts and not args.no_e2e:
         e2e_s, h2d, d2h = e2e_act(W, max(1, min(args.steps, 3)))
@@ -689,20 +830,25 @@ def run_ours(args):
     if "act" in parts:
         bytes_act, n_act = act_bytes(W)
         value = ws * bytes_act * args.steps / part_s["act"] / 1e9
-    sweep = None
-    if "calib" in parts and "scale_sweep" in roof:
-        blocks = sum(j["codes"].numel() for j in W["weights"])
-        sw = roof["scale_sweep"]
-        sweep = {"value": ws * blocks * args.steps / part_s["calib"], "unit": "blocks/s",
-                 "note": "blocks over the whole calib part (Hessians + amax + sweep)",
-                 "kernel_blocks_per_s": sw["blocks_per_s"],
-                 "algorithmic_tflops": sw["achieved"], "frac_fp32": sw["frac"], "fp32_peak_tflops": FP32_PEAK_TFLOPS,
-                 "executed_tflops": sw["executed_tflops"], "executed_frac_fp32": sw["executed_frac"],
-                 "half_visits_per_block": sw["half_visits_per_block"], "costs_per_block": sw["costs_per_block"],
-                 "note_work": "algorithmic = blocks/s x the exhaustive 127 x 304 FLOP per block (above the FP32 "
-                              "peak: an exact branch and bound proves most candidates irrelevant, same codes); "
-                              "executed = the FLOPs actually done, from device counters (48 per candidate half "
-                              "visited, 272 per cost evaluated)"}
+    def sweep_summary(part, row, weights):
+        blocks = sum(j["codes"].numel() for j in weights)
+        sw = roof[row]
+        return {"value": ws * blocks * args.steps / part_s[part], "unit": "blocks/s",
+                "note": f"blocks over the whole {part} part (Hessians + amax + sweep)",
+                "kernel_blocks_per_s": sw["blocks_per_s"],
+                "algorithmic_tflops": sw["achieved"], "frac_fp32": sw["frac"],
+                "fp32_peak_tflops": fp32["measured"], "fp32_nominal_tflops": fp32["nominal"],
+                "executed_tflops": sw["executed_tflops"], "executed_frac_fp32": sw["executed_frac"],
+                "executed_frac_fp32_nominal": sw["executed_frac_nominal"],
+                "half_visits_per_block": sw["half_visits_per_block"], "costs_per_block": sw["costs_per_block"],
+                "note_work": "algorithmic = blocks/s x the exhaustive 127 x 304 FLOP per block (above the FP32 "
+                             "peak: an exact branch and bound proves most candidates irrelevant, same codes); "
+                             "executed = the FLOPs actually done, from device counters (48 per candidate half "
+                             "visited, 272 per cost evaluated); fractions of the measured FP32 peak, nominal beside"}
+
+    sweep = sweep_summary("calib", "scale_sweep", W["weights"]) if "calib" in parts and "scale_sweep" in roof else None
+    sweep_moe = (sweep_summary("moe", "scale_sweep_moe", W["moe_weights"])
+                 if "moe" in parts and "scale_sweep_moe" in roof else None)
     # dominant kernel: the largest device time per step (every in-step row times the step's
     # own launch, which runs once per step)
     in_step = [k for k in roof if roof[k].get("in_step", True)]
@@ -718,15 +864,19 @@ def run_ours(args):
         "gpu_launches": args.steps * sum(LAUNCHES[p] for p in parts),
         "flags": flags,
         "clocks": clk,
+        "fp32_peak": fp32,
     }
     if dom is not None:
         r = roof[dom]
         line["roofline"] = {"kernel": dom, "bound": r["bound"], "achieved": r["achieved"], "peak": r["peak"],
                             "unit": r["unit"], "frac": r["frac"], "traffic": r["traffic"],
-                            "peak_kind": peak_kind if r["bound"] == "hbm" else "nominal (unit counts x max clock)"}
-        if dom == "scale_sweep":
+                            "peak_kind": (peak_kind if r["bound"] == "hbm" else
+                                          "measured (nv4_fp32_probe, this run)" if r["bound"] == "alu" else
+                                          "4 x the measured BF16 GEMM peak")}
+        if dom.startswith("scale_sweep"):
             line["roofline"]["executed"] = r["executed_tflops"]
             line["roofline"]["executed_frac"] = r["executed_frac"]
+            line["roofline"]["executed_frac_nominal"] = r["executed_frac_nominal"]
             line["roofline"]["note"] = ("achieved counts the exhaustive 127-candidate search (38.6 kFLOP per block); "
                                         "the exact branch and bound skips provably irrelevant candidates, so it reads "
                                         "above the peak; executed counts the work done")
@@ -735,6 +885,8 @@ def run_ours(args):
                     for k, v in roof.items()}
     if sweep is not None:
         line["sweep"] = sweep
+    if sweep_moe is not None:
+        line["sweep_moe"] = sweep_moe
     if e2e is not None:
         line["e2e"] = e2e
     if cpu is not None:
@@ -742,9 +894,124 @@ def run_ours(args):
     print(json.dumps(line), flush=True)
 
 
+# ---------------------------------------------------------------------- single-kernel runs for ncu
+def _prof_setup_gemm(dev, seed):
+    import torch
+
+    from nvfp4_block_numerics_b200 import binding as nv4
+
+    M = N = K = 8192
+    g = torch.Generator(device=dev).manual_seed(seed)
+    r = lambda *sh, lo=0, hi=256: torch.randint(lo, hi, sh, dtype=torch.uint8, device=dev, generator=g)
+    qa, qb = r(M, K // 2), r(N, K // 2)
+    fa, fb = nv4.mma_scales(r(M, K // 16, lo=0x30, hi=0x40)), nv4.mma_scales(r(N, K // 16, lo=0x30, hi=0x40))
+    one = torch.ones(1, dtype=torch.float32, device=dev)
+    out = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+    return (lambda: nv4.nv4_gemm_nvfp4(qa, fa, one, qb, fb, one, out)), "gemm_nvfp4_kernel: 8192^3 NVFP4 -> BF16"
+
+
+def _prof_setup_sweep(dev, seed):
+    W = build_workload(["calib"], seed, dev)
+    part_calib(W)
+    from nvfp4_block_numerics_b200 import binding as nv4
+
+    jobs = [{k: j[k] for k in ("w", "H", "d_amax_w", "codes", "q")} for j in W["weights"]]
+    return (lambda: nv4.nv4_scale_sweep_batched(jobs, W["flags"])), "sweep_kernel: Gemma-like layer, 6.55 M blocks"
+
+
+def _prof_setup_sweep_moe(dev, seed, experts=16):
+    import torch
+
+    from nvfp4_block_numerics_b200 import binding as nv4
+    from nvfp4_block_numerics_b200 import inputs
+
+    jobs = []
+    flags = torch.zeros(1, dtype=torch.int32, device=dev)
+    for e in range(experts):
+        d = inputs.c4_expert(e, seed)
+        b = {k: torch.from_numpy(v.view(np.int16)).view(torch.bfloat16).to(dev) for k, v in d.items()}
+        Hx = nv4.hessian_accum(b["X"])
+        Hd = nv4.hessian_accum(b["X_down"])
+        for name in ("W_gate", "W_up", "W_down"):
+            w = b[name]
+            jobs.append(dict(w=w, H=Hd if name == "W_down" else Hx, d_amax_w=nv4.tensor_amax(w),
+                             codes=torch.empty((w.shape[0], w.shape[1] // 16), dtype=torch.uint8, device=dev),
+                             q=torch.empty((w.shape[0], w.shape[1] // 2), dtype=torch.uint8, device=dev)))
+    blocks = sum(j["codes"].numel() for j in jobs)
+    return (lambda: nv4.nv4_scale_sweep_batched(jobs, flags)), \
+        f"sweep_kernel: {experts} MoE experts ({3 * experts} matrices, {blocks / 1e6:.1f} M blocks)"
+
+
+def _prof_setup_hessian(dev, seed):
+    W = build_workload(["calib"], seed, dev)
+    from nvfp4_block_numerics_b200 import binding as nv4
+
+    return (lambda: nv4.nv4_hessian_accum_batched([W["X"], W["Xd"]], [W["H"], W["Hd"]], W["flags"])), \
+        "hessian_kernel: X [16384, 2048] + X_down [16384, 16384] bf16"
+
+
+def _prof_setup_act(kind):
+    def setup(dev, seed):
+        import torch
+
+        from nvfp4_block_numerics_b200 import binding as nv4
+        from nvfp4_block_numerics_b200 import inputs
+
+        xb = inputs.c2_shape(65536, 7168, seed)
+        x = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).to(dev)
+        a = nv4.tensor_amax(x)
+        q, sc, s2 = nv4.act_quant(x, a)
+        fn = {"amax": lambda: nv4.nv4_tensor_amax(x, a),
+              "act_quant": lambda: nv4.nv4_act_quant(x, a, q, sc, s2),
+              "dequant": lambda: nv4.nv4_dequant(q, sc, s2, torch.empty_like(x)),
+              "fake_qdq": lambda: nv4.nv4_fake_qdq(x, a, torch.empty_like(x), s2),
+              "rtn": lambda: nv4.nv4_weight_quant_rtn(x, a, q, sc, s2),
+              "fp8": lambda: nv4.nv4_fp8_quant(x, a, torch.empty(x.shape, dtype=torch.uint8, device=dev), s2),
+              "mxfp4": lambda: nv4.mxfp4_quant(x),
+              "hadamard": lambda: nv4.hadamard_mxfp4_quant(x, 128)}[kind]
+        return fn, f"{kind}: [65536, 7168] bf16"
+    return setup
+
+
+def _prof_setup_cast(dev, seed):
+    W = build_workload(["cast"], seed, dev)
+    from nvfp4_block_numerics_b200 import binding as nv4
+
+    return (lambda: nv4.nv4_mxfp4_to_nvfp4_batched(W["cast"], W["counts"], W["flags"])), \
+        "cast kernels: 32 x [2880, 2880] MXFP4, out of place"
+
+
+PROFILE_CASES = {"gemm": _prof_setup_gemm, "sweep": _prof_setup_sweep, "sweep_moe": _prof_setup_sweep_moe,
+                 "hessian": _prof_setup_hessian, "cast": _prof_setup_cast,
+                 **{k: _prof_setup_act(k) for k in ("amax", "act_quant", "dequant", "fake_qdq", "rtn", "fp8",
+                                                    "mxfp4", "hadamard")}}
+
+
+def run_profile(args):
+    """One kernel's launch, args.profile_reps times in a row, for an ncu capture (-k, -s, -c
+    select among them); the same call the bench times."""
+    import torch
+
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    fn, what = PROFILE_CASES[args.profile](dev, args.seed)
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(args.profile_reps):
+        fn()
+    b.record()
+    torch.cuda.synchronize()
+    print(json.dumps({"profile": args.profile, "case": what, "reps": args.profile_reps,
+                      "ms_per_rep": a.elapsed_time(b) / args.profile_reps}), flush=True)
+
+
 def main():
     args = parse_args()
-    if args.impl == "reference":
+    if args.profile is not None:
+        run_profile(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)

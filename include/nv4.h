@@ -430,6 +430,18 @@ NV4_API nv4_status nv4_hadamard_nvfp4_quant(const void* x, int64_t rows, int64_t
 NV4_API nv4_status nv4_selftest(uint32_t* d_out, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * nv4_fp32_probe -- a microbenchmark of the FP32 pipe, the denominator of the scale
+ * sweep's roofline.  Launches `blocks` CTAs of 256 threads; every thread runs `iters`
+ * rounds of 32 FLOP of independent fused multiply-adds, as scalar FP32 FMAs (packed = 0)
+ * or as packed two-lane FMAs (packed = 1), so one launch does blocks * 256 * iters * 32
+ * FLOP; time it with events.  d_sink: one float per CTA on the device, written only if a
+ * chain went NaN (never, for the built-in operands); it keeps the work from being
+ * optimized away.  blocks <= 2^20 and iters <= 2^24 (NV4_ERR_LIMIT beyond).
+ * Not a paper operation: a measurement of the GPU it runs on.
+ */
+NV4_API nv4_status nv4_fp32_probe(int packed, uint32_t blocks, uint32_t iters, float* d_sink, void* stream);
+
+/* ---------------------------------------------------------------------------
  * nv4_selftest_wait -- exercises the bounded wait that every pipeline kernel uses (no
  * kernel of this library waits without a time limit): one thread polls the device word
  * *d_flag until it is non-zero or limit_ns (<= 2 s, the kernels' own limit; NV4_ERR_LIMIT

@@ -102,6 +102,7 @@ _SIGS = {
     "nv4_mxfp4_to_nvfp4": (C.c_int, [_vp, _vp, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "nv4_mxfp4_to_nvfp4_batched": (C.c_int, [C.POINTER(CastJob), C.c_int, _vp, _vp, _vp]),
     "nv4_selftest": (C.c_int, [_vp, _vp]),
+    "nv4_fp32_probe": (C.c_int, [C.c_int, C.c_uint32, C.c_uint32, _vp, _vp]),
 }
 
 
@@ -381,6 +382,13 @@ def nv4_selftest_wait(flag: torch.Tensor, limit_ns: int, status: torch.Tensor, s
     if flag.dtype != torch.int32 or status.dtype != torch.int32 or status.numel() < 2:
         raise NV4Error("flag and status must be int32 CUDA tensors (status of at least 2 elements)")
     _check(lib().nv4_selftest_wait(_ptr(flag), int(limit_ns), _ptr(status), _stream(stream)), "nv4_selftest_wait")
+
+
+def nv4_fp32_probe(packed: bool, blocks: int, iters: int, sink: torch.Tensor, stream=None):
+    """FP32 pipe microbenchmark: blocks * 256 * iters * 32 FLOP of independent FMAs."""
+    if sink.dtype != torch.float32 or sink.numel() < blocks:
+        raise NV4Error("sink must be a float32 CUDA tensor with one element per block")
+    _check(lib().nv4_fp32_probe(1 if packed else 0, blocks, iters, _ptr(sink), _stream(stream)), "nv4_fp32_probe")
 
 
 def nv4_selftest(out: torch.Tensor, stream=None):

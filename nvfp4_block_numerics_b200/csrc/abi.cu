@@ -98,6 +98,54 @@ cudaError_t launch_wait_selftest(const uint32_t* flag, uint64_t limit_ns, uint32
     return cudaGetLastError();
 }
 
+// FP32 pipe microbenchmark: every thread runs `iters` rounds of 16 independent fused
+// multiply-add chains, as scalar fma.rn.f32 (kPacked = false) or as 8 packed fma.rn.f32x2
+// (true); 32 FLOP per thread and round either way.  The multiplier and addend come from
+// the arguments, so nothing folds; the chains end in one store that no input makes
+// happen (the sum is finite, never NaN), which keeps them live.
+template <bool kPacked>
+__global__ void __launch_bounds__(256) fma_probe_kernel(uint32_t iters, float m, float c, float* sink)
+{
+    const float x0 = __uint2float_rn(threadIdx.x) * 0x1p-20f;
+    float sum = 0.0f;
+    if constexpr (kPacked) {
+        float2 a[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) a[k] = make_float2(x0 + (float)k, x0 - (float)k);
+        const float2 m2 = make_float2(m, m), c2 = make_float2(c, c);
+#pragma unroll 1
+        for (uint32_t it = 0; it < iters; ++it) {
+#pragma unroll
+            for (int r = 0; r < 4; ++r)
+#pragma unroll
+                for (int k = 0; k < 8; ++k) a[k] = __ffma2_rn(a[k], m2, c2);
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k) sum += a[k].x + a[k].y;
+    } else {
+        float a[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) a[k] = x0 + (float)k;
+#pragma unroll 1
+        for (uint32_t it = 0; it < iters; ++it) {
+#pragma unroll
+            for (int r = 0; r < 4; ++r)
+#pragma unroll
+                for (int k = 0; k < 16; ++k) a[k] = fmaf(a[k], m, c);
+        }
+#pragma unroll
+        for (int k = 0; k < 16; ++k) sum += a[k];
+    }
+    if (isnan(sum)) sink[blockIdx.x] = sum;
+}
+
+cudaError_t launch_fma_probe(int packed, uint32_t blocks, uint32_t iters, float* sink, cudaStream_t s)
+{
+    if (packed) fma_probe_kernel<true><<<blocks, 256, 0, s>>>(iters, 0.9999999f, 1e-7f, sink);
+    else fma_probe_kernel<false><<<blocks, 256, 0, s>>>(iters, 0.9999999f, 1e-7f, sink);
+    return cudaGetLastError();
+}
+
 }  // namespace nv4
 
 using namespace nv4;
@@ -411,6 +459,13 @@ nv4_status nv4_selftest(uint32_t* d_out, void* stream)
 {
     if (d_out == nullptr) return NV4_ERR_NULL;
     return from_cuda(launch_selftest(d_out, (cudaStream_t)stream));
+}
+
+nv4_status nv4_fp32_probe(int packed, uint32_t blocks, uint32_t iters, float* d_sink, void* stream)
+{
+    if (d_sink == nullptr) return NV4_ERR_NULL;
+    if (blocks == 0 || blocks > (1u << 20) || iters == 0 || iters > (1u << 24)) return NV4_ERR_LIMIT;
+    return from_cuda(launch_fma_probe(packed, blocks, iters, d_sink, (cudaStream_t)stream));
 }
 
 nv4_status nv4_selftest_wait(const uint32_t* d_flag, uint64_t limit_ns, uint32_t* d_status, void* stream)

@@ -89,5 +89,6 @@ cudaError_t launch_sweep(const nv4_sweep_job* jobs, int n, int dt, uint32_t* d_f
 cudaError_t launch_cast(const nv4_cast_job* jobs, int n, unsigned long long* d_counts, uint32_t* d_flags,
                         cudaStream_t s);
 cudaError_t launch_selftest(uint32_t* d_out, cudaStream_t s);
+cudaError_t launch_fma_probe(int packed, uint32_t blocks, uint32_t iters, float* sink, cudaStream_t s);
 
 }  // namespace nv4

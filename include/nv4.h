@@ -421,6 +421,39 @@ NV4_API nv4_status nv4_hadamard_nvfp4_quant(const void* x, int64_t rows, int64_t
                                     uint32_t* d_flags, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * Two-sided block Hadamard rotation of weight tiles fused with FP4 quantization ([FP4]
+ * section 3.1: the weight matrix is cut into n x n tiles, n = 16 or 32, and each tile B
+ * becomes (H_n / sqrt(n)) B (H_n / sqrt(n))^T = H_n B H_n / n before quantization; H_n is the
+ * natural-order (Sylvester) Hadamard matrix, which is symmetric).  Per tile:
+ *
+ *   y = RN32(exact(H_n B H_n) / n)        (1/n is a power of two: one rounding, to FP32)
+ *
+ * The kernels form the sums in FP64, exact while a tile's values, as multiples of its
+ * smallest unit in the last place, fit 53 bits with 2*log2(n) bits of growth (BF16 tiles
+ * spanning fewer than ~35 binades, FP32 tiles fewer than ~19); beyond that the FP64 sum
+ * carries a relative error below 2^-52 before the final rounding.
+ *
+ * w : [rows, cols] of dt (NV4_BF16 or NV4_FP32), leading dimension ld (a 16-byte multiple),
+ *     16-byte aligned; rows % n == 0 and cols % 32 == 0 (NV4_ERR_SHAPE otherwise).
+ * nv4_hadamard2_rotate       -- out: y as FP32 [rows, cols], contiguous, 16-byte aligned.
+ * nv4_hadamard2_amax         -- *d_amax = max(*d_amax, max |y|) (running max, as nv4_tensor_amax).
+ * nv4_hadamard2_mxfp4_quant  -- MXFP4 of y along rows (32-element blocks), as nv4_mxfp4_quant.
+ * nv4_hadamard2_nvfp4_quant  -- NVFP4 of y along rows with s2 = RN32(amax / 2688) from *d_amax
+ *                               (e.g. from nv4_hadamard2_amax), as nv4_weight_quant_rtn.
+ * Limits: fewer than 2^31 strips of n x 32 per call.  A NaN or Inf in y sets
+ * NV4_FLAG_NONFINITE.
+ */
+NV4_API nv4_status nv4_hadamard2_rotate(const void* w, nv4_dtype dt, int64_t rows, int64_t cols, int64_t ld, int n,
+                                float* out, uint32_t* d_flags, void* stream);
+NV4_API nv4_status nv4_hadamard2_amax(const void* w, nv4_dtype dt, int64_t rows, int64_t cols, int64_t ld, int n,
+                              float* d_amax, uint32_t* d_flags, void* stream);
+NV4_API nv4_status nv4_hadamard2_mxfp4_quant(const void* w, nv4_dtype dt, int64_t rows, int64_t cols, int64_t ld,
+                                     int n, uint8_t* q, uint8_t* e8m0, uint32_t* d_flags, void* stream);
+NV4_API nv4_status nv4_hadamard2_nvfp4_quant(const void* w, nv4_dtype dt, int64_t rows, int64_t cols, int64_t ld,
+                                     int n, const float* d_amax, uint8_t* q, uint8_t* scales, float* d_s2,
+                                     uint32_t* d_flags, void* stream);
+
+/* ---------------------------------------------------------------------------
  * nv4_selftest -- checks, on the current device, the hardware FP4/FP8 conversion
  * instructions the kernels rely on (lane order, rounding, sign of zero, saturation).
  * Writes 64 uint32 results to d_out (device); d_out[0] is a bit mask of failed
@@ -432,9 +465,9 @@ NV4_API nv4_status nv4_selftest(uint32_t* d_out, void* stream);
 /* ---------------------------------------------------------------------------
  * nv4_fp32_probe -- a microbenchmark of the FP32 pipe, the denominator of the scale
  * sweep's roofline.  Launches `blocks` CTAs of 256 threads; every thread runs `iters`
- * rounds of 32 FLOP of independent fused multiply-adds, as scalar FP32 FMAs (packed = 0)
- * or as packed two-lane FMAs (packed = 1), so one launch does blocks * 256 * iters * 32
- * FLOP; time it with events.  d_sink: one float per CTA on the device, written only if a
+ * iterations of 128 FLOP of independent fused multiply-adds (16 chains, 4 steps each), as
+ * scalar FP32 FMAs (packed = 0) or as packed two-lane FMAs (packed = 1), so one launch does
+ * blocks * 256 * iters * 128 FLOP; time it with events.  d_sink: one float per CTA on the device, written only if a
  * chain went NaN (never, for the built-in operands); it keeps the work from being
  * optimized away.  blocks <= 2^20 and iters <= 2^24 (NV4_ERR_LIMIT beyond).
  * Not a paper operation: a measurement of the GPU it runs on.

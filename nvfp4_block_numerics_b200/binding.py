@@ -103,6 +103,10 @@ _SIGS = {
     "nv4_mxfp4_to_nvfp4_batched": (C.c_int, [C.POINTER(CastJob), C.c_int, _vp, _vp, _vp]),
     "nv4_selftest": (C.c_int, [_vp, _vp]),
     "nv4_fp32_probe": (C.c_int, [C.c_int, C.c_uint32, C.c_uint32, _vp, _vp]),
+    "nv4_hadamard2_rotate": (C.c_int, [_vp, C.c_int, _i64, _i64, _i64, C.c_int, _vp, _vp, _vp]),
+    "nv4_hadamard2_amax": (C.c_int, [_vp, C.c_int, _i64, _i64, _i64, C.c_int, _vp, _vp, _vp]),
+    "nv4_hadamard2_mxfp4_quant": (C.c_int, [_vp, C.c_int, _i64, _i64, _i64, C.c_int, _vp, _vp, _vp, _vp]),
+    "nv4_hadamard2_nvfp4_quant": (C.c_int, [_vp, C.c_int, _i64, _i64, _i64, C.c_int, _vp, _vp, _vp, _vp, _vp, _vp]),
 }
 
 
@@ -384,8 +388,73 @@ def nv4_selftest_wait(flag: torch.Tensor, limit_ns: int, status: torch.Tensor, s
     _check(lib().nv4_selftest_wait(_ptr(flag), int(limit_ns), _ptr(status), _stream(stream)), "nv4_selftest_wait")
 
 
+def _w_rows(w, name="w"):
+    if w.dtype not in (torch.bfloat16, torch.float32):
+        raise NV4Error(f"{name} must be bf16 or float32")
+    return _rowmajor(w, name)
+
+
+def nv4_hadamard2_rotate(w: torch.Tensor, n: int, out: torch.Tensor, d_flags=None, stream=None):
+    rows, cols, ld = _w_rows(w)
+    if out.dtype != torch.float32 or tuple(out.shape) != (rows, cols) or not out.is_contiguous():
+        raise NV4Error("out must be a contiguous float32 tensor [rows, cols]")
+    _check(lib().nv4_hadamard2_rotate(_ptr(w), _DT[w.dtype], rows, cols, ld, n, _ptr(out), _ptr(d_flags),
+                                      _stream(stream)), "nv4_hadamard2_rotate")
+
+
+def nv4_hadamard2_amax(w: torch.Tensor, n: int, d_amax: torch.Tensor, d_flags=None, stream=None):
+    rows, cols, ld = _w_rows(w)
+    _check(lib().nv4_hadamard2_amax(_ptr(w), _DT[w.dtype], rows, cols, ld, n, _scalar_f32(d_amax, "d_amax"),
+                                    _ptr(d_flags), _stream(stream)), "nv4_hadamard2_amax")
+
+
+def nv4_hadamard2_mxfp4_quant(w: torch.Tensor, n: int, q: torch.Tensor, e8m0: torch.Tensor, d_flags=None,
+                              stream=None):
+    rows, cols, ld = _w_rows(w)
+    _u8(q, (rows, cols // 2), "q")
+    _u8(e8m0, (rows, cols // 32), "e8m0")
+    _check(lib().nv4_hadamard2_mxfp4_quant(_ptr(w), _DT[w.dtype], rows, cols, ld, n, _ptr(q), _ptr(e8m0),
+                                           _ptr(d_flags), _stream(stream)), "nv4_hadamard2_mxfp4_quant")
+
+
+def nv4_hadamard2_nvfp4_quant(w: torch.Tensor, n: int, d_amax: torch.Tensor, q: torch.Tensor, scales: torch.Tensor,
+                              d_s2: torch.Tensor, d_flags=None, stream=None):
+    rows, cols, ld = _w_rows(w)
+    _u8(q, (rows, cols // 2), "q")
+    _u8(scales, (rows, cols // 16), "scales")
+    _check(lib().nv4_hadamard2_nvfp4_quant(_ptr(w), _DT[w.dtype], rows, cols, ld, n, _scalar_f32(d_amax, "d_amax"),
+                                           _ptr(q), _ptr(scales), _scalar_f32(d_s2, "d_s2"), _ptr(d_flags),
+                                           _stream(stream)), "nv4_hadamard2_nvfp4_quant")
+
+
+def hadamard2_rotate(w: torch.Tensor, n: int, d_flags=None, stream=None) -> torch.Tensor:
+    out = torch.empty(tuple(w.shape), dtype=torch.float32, device=w.device)
+    nv4_hadamard2_rotate(w, n, out, d_flags, stream)
+    return out
+
+
+def hadamard2_mxfp4_quant(w: torch.Tensor, n: int, d_flags=None, stream=None):
+    rows, cols = w.shape
+    q = torch.empty((rows, cols // 2), dtype=torch.uint8, device=w.device)
+    e8 = torch.empty((rows, cols // 32), dtype=torch.uint8, device=w.device)
+    nv4_hadamard2_mxfp4_quant(w, n, q, e8, d_flags, stream)
+    return q, e8
+
+
+def hadamard2_nvfp4_quant(w: torch.Tensor, n: int, d_flags=None, stream=None):
+    """Two passes: the amax of the rotated tensor, then the NVFP4 quantization."""
+    rows, cols = w.shape
+    amax = torch.zeros(1, dtype=torch.float32, device=w.device)
+    nv4_hadamard2_amax(w, n, amax, d_flags, stream)
+    q = torch.empty((rows, cols // 2), dtype=torch.uint8, device=w.device)
+    sc = torch.empty((rows, cols // 16), dtype=torch.uint8, device=w.device)
+    s2 = torch.empty(1, dtype=torch.float32, device=w.device)
+    nv4_hadamard2_nvfp4_quant(w, n, amax, q, sc, s2, d_flags, stream)
+    return q, sc, s2, amax
+
+
 def nv4_fp32_probe(packed: bool, blocks: int, iters: int, sink: torch.Tensor, stream=None):
-    """FP32 pipe microbenchmark: blocks * 256 * iters * 32 FLOP of independent FMAs."""
+    """FP32 pipe microbenchmark: blocks * 256 * iters * 128 FLOP of independent FMAs."""
     if sink.dtype != torch.float32 or sink.numel() < blocks:
         raise NV4Error("sink must be a float32 CUDA tensor with one element per block")
     _check(lib().nv4_fp32_probe(1 if packed else 0, blocks, iters, _ptr(sink), _stream(stream)), "nv4_fp32_probe")

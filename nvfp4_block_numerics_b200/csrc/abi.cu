@@ -98,9 +98,9 @@ cudaError_t launch_wait_selftest(const uint32_t* flag, uint64_t limit_ns, uint32
     return cudaGetLastError();
 }
 
-// FP32 pipe microbenchmark: every thread runs `iters` rounds of 16 independent fused
-// multiply-add chains, as scalar fma.rn.f32 (kPacked = false) or as 8 packed fma.rn.f32x2
-// (true); 32 FLOP per thread and round either way.  The multiplier and addend come from
+// FP32 pipe microbenchmark: every thread runs `iters` iterations of 4 steps of 16
+// independent fused multiply-add chains, as scalar fma.rn.f32 (kPacked = false) or as 8
+// packed fma.rn.f32x2 (true); 128 FLOP per thread and iteration either way.  The multiplier and addend come from
 // the arguments, so nothing folds; the chains end in one store that no input makes
 // happen (the sum is finite, never NaN), which keeps them live.
 template <bool kPacked>
@@ -614,4 +614,65 @@ nv4_status nv4_hadamard_nvfp4_quant(const void* x, int64_t rows, int64_t cols, i
     if (!aligned16(q)) return NV4_ERR_ALIGN;
     return from_cuda(launch_hadamard_quant(2, x, rows, cols, ld, n, const_cast<float*>(d_amax), q, scales, d_s2,
                                            d_flags, (cudaStream_t)stream));
+}
+
+// ------------------------------------------------------------------ two-sided block Hadamard of weight tiles
+static nv4_status check_hadamard2(const void* w, nv4_dtype dt, int64_t rows, int64_t cols, int64_t ld, int n)
+{
+    if (dt != NV4_BF16 && dt != NV4_FP32) return NV4_ERR_DTYPE;
+    if (n != 16 && n != 32) return NV4_ERR_SHAPE;
+    if (rows < 0 || cols < 0 || rows % n != 0 || cols % 32 != 0 || ld < cols) return NV4_ERR_SHAPE;
+    if (rows == 0 || cols == 0) return NV4_OK;
+    if (w == nullptr) return NV4_ERR_NULL;
+    if (!aligned16(w) || ld % (dt == NV4_BF16 ? 8 : 4) != 0) return NV4_ERR_ALIGN;
+    if ((rows / n) * (cols / 32) >= (int64_t)1 << 31) return NV4_ERR_LIMIT;
+    return NV4_OK;
+}
+
+nv4_status nv4_hadamard2_rotate(const void* w, nv4_dtype dt, int64_t rows, int64_t cols, int64_t ld, int n,
+                                float* out, uint32_t* d_flags, void* stream)
+{
+    const nv4_status st = check_hadamard2(w, dt, rows, cols, ld, n);
+    if (st != NV4_OK || rows == 0 || cols == 0) return st;
+    if (out == nullptr) return NV4_ERR_NULL;
+    if (!aligned16(out)) return NV4_ERR_ALIGN;
+    return from_cuda(launch_hadamard2(3, w, dt == NV4_BF16 ? 0 : 2, rows, cols, ld, n, nullptr, nullptr, nullptr,
+                                      nullptr, out, d_flags, (cudaStream_t)stream));
+}
+
+nv4_status nv4_hadamard2_amax(const void* w, nv4_dtype dt, int64_t rows, int64_t cols, int64_t ld, int n,
+                              float* d_amax, uint32_t* d_flags, void* stream)
+{
+    const nv4_status st = check_hadamard2(w, dt, rows, cols, ld, n);
+    if (st != NV4_OK) return st;
+    if (d_amax == nullptr) return NV4_ERR_NULL;
+    if (rows == 0 || cols == 0) return NV4_OK;
+    return from_cuda(launch_hadamard2(0, w, dt == NV4_BF16 ? 0 : 2, rows, cols, ld, n, d_amax, nullptr, nullptr,
+                                      nullptr, nullptr, d_flags, (cudaStream_t)stream));
+}
+
+nv4_status nv4_hadamard2_mxfp4_quant(const void* w, nv4_dtype dt, int64_t rows, int64_t cols, int64_t ld, int n,
+                                     uint8_t* q, uint8_t* e8m0, uint32_t* d_flags, void* stream)
+{
+    const nv4_status st = check_hadamard2(w, dt, rows, cols, ld, n);
+    if (st != NV4_OK || rows == 0 || cols == 0) return st;
+    if (q == nullptr || e8m0 == nullptr) return NV4_ERR_NULL;
+    if (!aligned16(q)) return NV4_ERR_ALIGN;
+    return from_cuda(launch_hadamard2(1, w, dt == NV4_BF16 ? 0 : 2, rows, cols, ld, n, nullptr, q, e8m0, nullptr,
+                                      nullptr, d_flags, (cudaStream_t)stream));
+}
+
+nv4_status nv4_hadamard2_nvfp4_quant(const void* w, nv4_dtype dt, int64_t rows, int64_t cols, int64_t ld, int n,
+                                     const float* d_amax, uint8_t* q, uint8_t* scales, float* d_s2,
+                                     uint32_t* d_flags, void* stream)
+{
+    const nv4_status st = check_hadamard2(w, dt, rows, cols, ld, n);
+    if (st != NV4_OK) return st;
+    if (d_amax == nullptr || d_s2 == nullptr) return NV4_ERR_NULL;
+    if (rows == 0 || cols == 0)                  // an empty tensor still receives its s2
+        return from_cuda(launch_scale_only(&d_amax, &d_s2, 1, 2688.0f, d_flags, (cudaStream_t)stream));
+    if (q == nullptr || scales == nullptr) return NV4_ERR_NULL;
+    if (!aligned16(q)) return NV4_ERR_ALIGN;
+    return from_cuda(launch_hadamard2(2, w, dt == NV4_BF16 ? 0 : 2, rows, cols, ld, n, const_cast<float*>(d_amax),
+                                      q, scales, d_s2, nullptr, d_flags, (cudaStream_t)stream));
 }

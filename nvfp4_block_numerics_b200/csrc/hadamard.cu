@@ -65,6 +65,85 @@ __device__ __forceinline__ float had_pow2(int k)
     return k >= -126 ? __uint_as_float((uint32_t)(k + 127) << 23) : __uint_as_float(1u << (k + 149));
 }
 
+
+// MXFP4 scale code of a block whose largest |y| has the bit pattern ab: the E8M0 code of
+// 2^(floor(log2 amax) - 2) clamped to [-127, 127], 0 for an all-zero block, 0xFF (NaN) for
+// a block holding NaN or Inf.
+__device__ __forceinline__ uint32_t mx_block_code(uint32_t ab)
+{
+    if (ab >= 0x7F800000u) return 0xFFu;
+    const int e = ab == 0u ? -127 : max(had_floor_log2(ab) - 2, -127);
+    return (uint32_t)(e + 127);
+}
+
+// E2M1 codes of kCount values (16 or 32) under the MXFP4 scale `code`: scaling by 2^-e is
+// exact, so one hardware RNE conversion per pair gives the exact codes.  w: kCount / 8 words.
+template <int kCount>
+__device__ __forceinline__ void mx_encode(const float* y, uint32_t code, uint32_t* w)
+{
+    if (code == 0xFFu) {
+#pragma unroll
+        for (int k = 0; k < kCount / 8; ++k) w[k] = 0u;
+        return;
+    }
+    const float inv = had_pow2(127 - (int)code);
+#pragma unroll
+    for (int k = 0; k < kCount / 8; ++k) {
+        float t[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) t[j] = __fmul_rn(y[8 * k + j], inv);   // exact
+        w[k] = cvt_e2m1x8(t);
+    }
+}
+
+// NVFP4 of one 16-element block y under s2 (k_lo, k_hi: the bracket of 1/(6 s2); fast:
+// s2 inside [2^-100, 2^100]): the E4M3 block scale code (returned) and the 16 E2M1 codes
+// in w[0..1], as nv4_act_quant computes them.
+__device__ __forceinline__ uint32_t nv_block16(const float* y, float s2, float k_lo, float k_hi, bool fast,
+                                               uint32_t* w)
+{
+    uint32_t bm = 0u;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) bm = max(bm, __float_as_uint(y[j]) & 0x7FFFFFFFu);
+    const float a_b = __uint_as_float(bm);
+    uint32_t code;
+    if (fast) {
+        const uint32_t cv = cvt_e4m3x2(__fmul_rn(a_b, k_lo), __fmul_rn(a_b, k_hi));
+        code = cv & 0xFFu;
+        if (code != (cv >> 8)) code = e4m3_fix(code, a_b, s2);
+    } else {
+        code = e4m3_code_exact(a_b, s2);
+    }
+    code &= 0x7Fu;
+    const float S = __fmul_rn(e4m3_value(code), s2);   // DQ1: RN32(s_b * s2)
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+        const float* yy = y + 8 * k;
+        uint32_t c8 = 0u;
+        if (S == 0.0f) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) c8 |= ((__float_as_uint(yy[j]) >> 28) & 8u) << (4 * j);
+        } else if (S >= kTinyScale && S <= 0x1p100f) {
+            const float rr = __frcp_rn(S);
+            const float rl = __fmul_rn(rr, kLoMargin), rh = __fmul_rn(rr, kHiMargin);
+            float lo[8], hi[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                lo[j] = __fmul_rn(yy[j], rl);
+                hi[j] = __fmul_rn(yy[j], rh);
+            }
+            c8 = cvt_e2m1x8(lo);
+            const uint32_t h8 = cvt_e2m1x8(hi);
+            if (c8 != h8) c8 = e2m1_fix8(yy, S, c8, h8);
+        } else {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) c8 |= e2m1_code_exact(yy[j], S) << (4 * j);
+        }
+        w[k] = c8;
+    }
+    return code;
+}
+
 template <int kMode, int kN>
 __global__ void __launch_bounds__(kHadThreads)
 hadamard_quant_kernel(const uint16_t* x, uint32_t rows, uint32_t chunks_per_row, int64_t ld, FastDiv div_cpr,
@@ -144,67 +223,17 @@ hadamard_quant_kernel(const uint16_t* x, uint32_t rows, uint32_t chunks_per_row,
         if constexpr (kMode == 0) {
             if (ab <= 0x7F800000u) mx_bits = max(mx_bits, ab);
         } else if constexpr (kMode == 1) {
-            uint32_t code, w[4] = {0u, 0u, 0u, 0u};
-            if (ab >= 0x7F800000u) {
-                code = 0xFFu;
-            } else {
-                const int e = ab == 0u ? -127 : max(had_floor_log2(ab) - 2, -127);
-                code = (uint32_t)(e + 127);
-                const float inv = had_pow2(-e);
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    float t[8];
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) t[j] = __fmul_rn(y[8 * k + j], inv);   // exact
-                    w[k] = cvt_e2m1x8(t);
-                }
-            }
+            uint32_t w[4];
+            const uint32_t code = mx_block_code(ab);
+            mx_encode<32>(y, code, w);
             __stcs(reinterpret_cast<uint4*>(q + (int64_t)r * (cols / 2) + col / 2), make_uint4(w[0], w[1], w[2], w[3]));
             sc[(int64_t)r * (cols / 32) + col / 32] = (uint8_t)code;
         } else {
             uint32_t w[4], codes2 = 0u;
 #pragma unroll
             for (int hb = 0; hb < 2; ++hb) {                       // two NVFP4 blocks of 16
-                uint32_t bm = 0u;
-#pragma unroll
-                for (int j = 0; j < 16; ++j) bm = max(bm, __float_as_uint(y[16 * hb + j]) & 0x7FFFFFFFu);
-                const float a_b = __uint_as_float(bm);
-                uint32_t code;
-                if (fast_scale) {
-                    const uint32_t cv = cvt_e4m3x2(__fmul_rn(a_b, k_lo), __fmul_rn(a_b, k_hi));
-                    code = cv & 0xFFu;
-                    if (code != (cv >> 8)) code = e4m3_fix(code, a_b, s2);
-                } else {
-                    code = e4m3_code_exact(a_b, s2);
-                }
-                code &= 0x7Fu;
+                const uint32_t code = nv_block16(y + 16 * hb, s2, k_lo, k_hi, fast_scale, w + 2 * hb);
                 codes2 |= code << (8 * hb);
-                const float S = __fmul_rn(e4m3_value(code), s2);   // DQ1: RN32(s_b * s2)
-#pragma unroll
-                for (int k = 0; k < 2; ++k) {
-                    const float* yy = y + 16 * hb + 8 * k;
-                    uint32_t c8 = 0u;
-                    if (S == 0.0f) {
-#pragma unroll
-                        for (int j = 0; j < 8; ++j) c8 |= ((__float_as_uint(yy[j]) >> 28) & 8u) << (4 * j);
-                    } else if (S >= kTinyScale && S <= 0x1p100f) {
-                        const float rr = __frcp_rn(S);
-                        const float rl = __fmul_rn(rr, kLoMargin), rh = __fmul_rn(rr, kHiMargin);
-                        float lo[8], hi[8];
-#pragma unroll
-                        for (int j = 0; j < 8; ++j) {
-                            lo[j] = __fmul_rn(yy[j], rl);
-                            hi[j] = __fmul_rn(yy[j], rh);
-                        }
-                        c8 = cvt_e2m1x8(lo);
-                        const uint32_t h8 = cvt_e2m1x8(hi);
-                        if (c8 != h8) c8 = e2m1_fix8(yy, S, c8, h8);
-                    } else {
-#pragma unroll
-                        for (int j = 0; j < 8; ++j) c8 |= e2m1_code_exact(yy[j], S) << (4 * j);
-                    }
-                    w[2 * hb + k] = c8;
-                }
             }
             __stcs(reinterpret_cast<uint4*>(q + (int64_t)r * (cols / 2) + col / 2), make_uint4(w[0], w[1], w[2], w[3]));
             *reinterpret_cast<uint16_t*>(sc + (int64_t)r * (cols / 16) + col / 16) = (uint16_t)codes2;
@@ -238,6 +267,174 @@ cudaError_t launch_hadamard_quant(int mode, const void* x, int64_t rows, int64_t
     else NV4_HAD_N(2);
 #undef NV4_HAD_N
 #undef NV4_HAD
+    return cudaGetLastError();
+}
+
+
+// ---------------------------------------------------------------- two-sided rotation of weight tiles
+// [FP4] section 3.1: the weight matrix is cut into n x n tiles (n = 16 or 32) and each tile
+// B becomes (H / sqrt(n)) B (H / sqrt(n))^T = H B H / n (H_n is symmetric), before FP4
+// quantization.  y = RN32(exact(H B H) / n): 1/n is a power of two, and the FP64 sums are
+// exact while the tile's values, as multiples of its smallest unit in the last place, fit
+// 53 bits with the 2 log2(n) bits of growth (BF16 tiles spanning up to ~35 binades, FP32
+// tiles up to ~19); beyond that the sum carries a relative error below 2^-52 before the
+// one rounding to FP32.
+//
+// One warp per strip of n rows x 32 columns (one 32 x 32 tile, or two 16 x 16 tiles side by
+// side).  Lane l holds one row of its tile (n = 32: row l; n = 16: row l % 16 of tile
+// l / 16) and runs that row's FWHT in FP64 registers; a transpose through shared memory
+// gives lane l column l of the strip for the column FWHTs; the scaled, rounded values go
+// back through shared memory as FP32 so that lane l again holds its row for quantization:
+//   mode 0: running max |y| into *d_amax;  mode 1: MXFP4 (32-element blocks along the row:
+//   one lane's row for n = 32, lanes l and l + 16 together for n = 16);  mode 2: NVFP4
+//   (16-element blocks) with s2 = RN32(amax / 2688);  mode 3: y itself, FP32 [rows, cols].
+constexpr int kHad2Warps = 4;
+
+template <int kN>
+__device__ __forceinline__ void fwht_regs(double* v)
+{
+#pragma unroll
+    for (int h = 1; h < kN; h <<= 1) {
+#pragma unroll
+        for (int i = 0; i < kN; ++i) {
+            if (i & h) continue;
+            const double a = v[i], b = v[i + h];
+            v[i] = a + b;
+            v[i + h] = a - b;
+        }
+    }
+}
+
+template <int kMode, int kN, int kDt>   // kDt 0 BF16, 2 FP32
+__global__ void __launch_bounds__(32 * kHad2Warps)
+hadamard2_kernel(const void* __restrict__ w, uint32_t strips, uint32_t strips_per_band, int64_t ld, int64_t cols,
+                 float* __restrict__ d_amax, uint8_t* __restrict__ q, uint8_t* __restrict__ sc,
+                 float* __restrict__ d_s2, float* __restrict__ out, uint32_t* __restrict__ d_flags)
+{
+    __shared__ double tbuf[kHad2Warps][kN][33];
+    const uint32_t lane = threadIdx.x & 31u, warp = threadIdx.x >> 5;
+    double (*T)[33] = tbuf[warp];
+    float (*Y)[33] = reinterpret_cast<float (*)[33]>(&tbuf[warp][0][0]);   // kN x 33 floats fit
+    uint32_t flags = 0u, mx_bits = 0u;
+
+    float s2 = 0.0f, k_lo = 0.0f, k_hi = 0.0f;
+    bool fast_scale = false;
+    if constexpr (kMode == 2) {
+        s2 = __fdiv_rn(*d_amax, 2688.0f);
+        if (blockIdx.x == 0 && threadIdx.x == 0) *d_s2 = s2;
+        fast_scale = s2 >= kTinyScale && s2 <= 0x1p100f;
+        const float k = __frcp_rn(__fmul_rn(6.0f, s2));
+        k_lo = __fmul_rn(k, kLoMargin);
+        k_hi = __fmul_rn(k, kHiMargin);
+        if (!isfinite(s2)) flags |= kFlagOverflow;
+    }
+    const uint32_t r = kN == 32 ? lane : (lane & 15u);            // this lane's row in the strip
+    const uint32_t cb = kN == 32 ? 0u : 16u * (lane >> 4);         // and its first column
+
+    for (uint32_t st = blockIdx.x * kHad2Warps + warp; st < strips; st += gridDim.x * kHad2Warps) {
+        const uint32_t band = st / strips_per_band, cs = st - band * strips_per_band;
+        const int64_t row = (int64_t)band * kN + r;
+        const int64_t col = 32 * (int64_t)cs + cb;
+        double v[kN];
+        if constexpr (kDt == 0) {
+            const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(w) + row * ld + col);
+#pragma unroll
+            for (int k = 0; k < kN / 8; ++k) {
+                const uint4 raw = __ldcs(src + k);
+                const uint32_t u[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    v[8 * k + 2 * j] = (double)bf16_lo(u[j]);
+                    v[8 * k + 2 * j + 1] = (double)bf16_hi(u[j]);
+                }
+            }
+        } else {
+            const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(w) + row * ld + col);
+#pragma unroll
+            for (int k = 0; k < kN / 4; ++k) {
+                const float4 f = __ldcs(src + k);
+                v[4 * k] = f.x; v[4 * k + 1] = f.y; v[4 * k + 2] = f.z; v[4 * k + 3] = f.w;
+            }
+        }
+        fwht_regs<kN>(v);                                          // row transform: B H
+#pragma unroll
+        for (int j = 0; j < kN; ++j) T[r][cb + j] = v[j];
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < kN; ++i) v[i] = T[i][lane];            // column `lane` of the strip
+        __syncwarp();
+        fwht_regs<kN>(v);                                          // column transform: H (B H)
+#pragma unroll
+        for (int i = 0; i < kN; ++i) Y[i][lane] = (float)(v[i] * (1.0 / kN));   // exact scaling, one rounding
+        __syncwarp();
+        float y[kN];
+        uint32_t ab = 0u;
+#pragma unroll
+        for (int j = 0; j < kN; ++j) {
+            y[j] = Y[r][cb + j];
+            ab = max(ab, __float_as_uint(y[j]) & 0x7FFFFFFFu);
+        }
+        __syncwarp();                                              // before the next strip reuses T
+        if (ab >= 0x7F800000u) flags |= kFlagNonFinite;
+
+        if constexpr (kMode == 0) {
+            if (ab <= 0x7F800000u) mx_bits = max(mx_bits, ab);
+        } else if constexpr (kMode == 3) {
+            float4* dst = reinterpret_cast<float4*>(out + row * cols + col);
+#pragma unroll
+            for (int k = 0; k < kN / 4; ++k) __stcs(dst + k, make_float4(y[4 * k], y[4 * k + 1], y[4 * k + 2], y[4 * k + 3]));
+        } else if constexpr (kMode == 1) {
+            uint32_t bm = ab;
+            if constexpr (kN == 16) bm = max(bm, __shfl_xor_sync(0xFFFFFFFFu, bm, 16));   // the row's other half
+            const uint32_t code = mx_block_code(bm);
+            uint32_t wv[kN / 8];
+            mx_encode<kN>(y, code, wv);
+            uint8_t* qd = q + row * (cols / 2) + col / 2;
+            if constexpr (kN == 32) __stcs(reinterpret_cast<uint4*>(qd), make_uint4(wv[0], wv[1], wv[2], wv[3]));
+            else __stcs(reinterpret_cast<uint2*>(qd), make_uint2(wv[0], wv[1]));
+            if (cb == 0u) sc[row * (cols / 32) + col / 32] = (uint8_t)code;
+        } else {
+            uint32_t wv[kN / 8], codes = 0u;
+#pragma unroll
+            for (int hb = 0; hb < kN / 16; ++hb)
+                codes |= nv_block16(y + 16 * hb, s2, k_lo, k_hi, fast_scale, wv + 2 * hb) << (8 * hb);
+            uint8_t* qd = q + row * (cols / 2) + col / 2;
+            if constexpr (kN == 32) {
+                __stcs(reinterpret_cast<uint4*>(qd), make_uint4(wv[0], wv[1], wv[2], wv[3]));
+                *reinterpret_cast<uint16_t*>(sc + row * (cols / 16) + col / 16) = (uint16_t)codes;
+            } else {
+                __stcs(reinterpret_cast<uint2*>(qd), make_uint2(wv[0], wv[1]));
+                sc[row * (cols / 16) + col / 16] = (uint8_t)codes;
+            }
+        }
+    }
+    if constexpr (kMode == 0) {
+        mx_bits = __reduce_max_sync(0xFFFFFFFFu, mx_bits);
+        if (lane == 0 && mx_bits != 0u) atomicMax(reinterpret_cast<unsigned int*>(d_amax), mx_bits);
+    }
+    flags = __reduce_or_sync(0xFFFFFFFFu, flags);
+    if (lane == 0) flag_or(d_flags, flags);
+}
+
+cudaError_t launch_hadamard2(int mode, const void* w, int dt, int64_t rows, int64_t cols, int64_t ld, int n,
+                             float* d_amax, uint8_t* q, uint8_t* sc, float* d_s2, float* out, uint32_t* d_flags,
+                             cudaStream_t s)
+{
+    const uint32_t spb = (uint32_t)(cols / 32);                 // strips per band of n rows
+    const uint32_t strips = (uint32_t)(rows / n) * spb;
+    const int64_t need = ((int64_t)strips + kHad2Warps - 1) / kHad2Warps;
+    const int64_t cap = (int64_t)num_sms() * 8;
+    const int grid = (int)(need < cap ? (need > 0 ? need : 1) : cap);
+#define NV4_H2(M, N, D) hadamard2_kernel<M, N, D><<<grid, 32 * kHad2Warps, 0, s>>>(w, strips, spb, ld, cols, d_amax, q, \
+                                                                                 sc, d_s2, out, d_flags)
+#define NV4_H2_ND(M) do { if (n == 16) { if (dt == 0) NV4_H2(M, 16, 0); else NV4_H2(M, 16, 2); } \
+                          else { if (dt == 0) NV4_H2(M, 32, 0); else NV4_H2(M, 32, 2); } } while (0)
+    if (mode == 0) NV4_H2_ND(0);
+    else if (mode == 1) NV4_H2_ND(1);
+    else if (mode == 2) NV4_H2_ND(2);
+    else NV4_H2_ND(3);
+#undef NV4_H2_ND
+#undef NV4_H2
     return cudaGetLastError();
 }
 

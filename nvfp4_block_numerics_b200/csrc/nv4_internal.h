@@ -74,6 +74,9 @@ cudaError_t launch_fp8_quant(const void* x, int in_dt, int64_t rows, int64_t col
                              uint8_t* q, float* d_scale, uint32_t* d_flags, cudaStream_t s);
 cudaError_t launch_fp8_dequant(const uint8_t* q, const float* d_scale, int64_t rows, int64_t cols, int out_dt,
                                void* out, cudaStream_t s);
+cudaError_t launch_hadamard2(int mode, const void* w, int dt, int64_t rows, int64_t cols, int64_t ld, int n,
+                             float* d_amax, uint8_t* q, uint8_t* sc, float* d_s2, float* out, uint32_t* d_flags,
+                             cudaStream_t s);
 cudaError_t launch_hadamard_quant(int mode, const void* x, int64_t rows, int64_t cols, int64_t ld, int n,
                                   float* d_amax, uint8_t* q, uint8_t* sc, float* d_s2, uint32_t* d_flags,
                                   cudaStream_t s);

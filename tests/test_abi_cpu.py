@@ -113,6 +113,17 @@ def test_validation_rejects_before_any_launch(nv4lib):
     assert L.nv4_hadamard_mxfp4_quant(fake, 4, 128, 132, 32, fake, fake, None, None) == 3   # ld % 8
     assert L.nv4_hadamard_amax(fake, 4, 128, 128, 64, None, None, None) == 1
     assert L.nv4_hadamard_nvfp4_quant(fake, 4, 128, 128, 128, fake, None, fake, fake, None, None) == 1
+    # two-sided block Hadamard of weight tiles: n, tile and strip shapes, dtype, alignment, nulls
+    assert L.nv4_hadamard2_rotate(fake, 0, 32, 64, 64, 64, fake, None, None) == 2          # n not 16 or 32
+    assert L.nv4_hadamard2_rotate(fake, 0, 40, 64, 64, 32, fake, None, None) == 2          # rows % n
+    assert L.nv4_hadamard2_rotate(fake, 0, 32, 48, 48, 16, fake, None, None) == 2          # cols % 32
+    assert L.nv4_hadamard2_rotate(fake, 1, 32, 64, 64, 32, fake, None, None) == 4          # fp16 w
+    assert L.nv4_hadamard2_rotate(fake, 2, 32, 64, 66, 32, fake, None, None) == 3          # fp32 row pitch
+    assert L.nv4_hadamard2_rotate(fake, 0, 32, 64, 64, 32, fake + 8, None, None) == 3      # misaligned out
+    assert L.nv4_hadamard2_mxfp4_quant(fake, 0, 32, 64, 64, 32, None, fake, None, None) == 1
+    assert L.nv4_hadamard2_nvfp4_quant(fake, 0, 32, 64, 64, 32, None, fake, fake, fake, None, None) == 1
+    assert L.nv4_hadamard2_amax(fake, 0, 0, 64, 64, 32, fake, None, None) == 0             # empty: no-op
+    assert L.nv4_fp32_probe(0, 0, 16, fake, None) == 6 and L.nv4_fp32_probe(0, 8, 16, None, None) == 1
     assert L.nv4_hessian_accum(fake, 10, 40, 40, fake, None, None) == 2
     assert L.nv4_hessian_accum(fake, 10, 32, 36, fake, None, None) == 3
     assert L.nv4_scale_sweep(fake, 2, 4, 32, 34, fake, fake, fake, None, None, None, None, None) == 3  # fp32 ld*4

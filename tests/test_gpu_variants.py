@@ -168,3 +168,65 @@ def test_hadamard_quant_layer_shape(orc):
     q, e8 = nv4.hadamard_mxfp4_quant(xd, 128)
     rq, re8, _ = orc.mxfp4_quant(orc.hadamard_rotate(np.ascontiguousarray(x[rows]), 128))
     assert np.array_equal(G.host(e8)[rows], re8) and np.array_equal(G.host(q)[rows], rq)
+
+
+# ---------------------------------------------------------------- two-sided block Hadamard of weight tiles
+def _w_dev(w):
+    return G.f32_dev(w) if w.dtype == np.float32 else G.bf16_dev(w)
+
+
+def _two_sided_check(orc, w, n, ld_pad=0):
+    """Rotated values bit for bit, then their amax, MXFP4 and NVFP4 codes, against the
+    oracle's rotation followed by its plain quantizers."""
+    y = orc.hadamard2_rotate(w, n)
+    wd = _w_dev(w)
+    if ld_pad:
+        big = torch.zeros((w.shape[0], w.shape[1] + ld_pad), dtype=wd.dtype, device=G.DEV)
+        big[:, :w.shape[1]] = wd
+        wd = big[:, :w.shape[1]]
+    f = G.flags_dev()
+    got = nv4.hadamard2_rotate(wd, n, d_flags=f)
+    torch.cuda.synchronize()
+    assert f.item() == 0
+    assert np.array_equal(G.host(got).view(np.uint32), y.view(np.uint32))
+    amax = torch.zeros(1, dtype=torch.float32, device=G.DEV)
+    nv4.nv4_hadamard2_amax(wd, n, amax)
+    assert amax.item() == float(np.abs(y).max())
+    q, e8 = nv4.hadamard2_mxfp4_quant(wd, n)
+    rq, re8, _ = orc.mxfp4_quant(y)
+    assert np.array_equal(G.host(e8), re8) and np.array_equal(G.host(q), rq)
+    q, sc, s2, _ = nv4.hadamard2_nvfp4_quant(wd, n)
+    nq, nsc, ns2, _ = orc.rtn_quant(y, float(np.abs(y).max()))
+    assert s2.item() == ns2
+    assert np.array_equal(G.host(sc), nsc) and np.array_equal(G.host(q), nq)
+
+
+@pytest.mark.parametrize("n", [16, 32])
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+def test_two_sided_hadamard_matches_oracle(orc, n, dtype):
+    rng = np.random.default_rng(n)
+    w = (rng.standard_normal((160, 224)) * 0.02).astype(np.float32)
+    w[5, 17] = 3.0                                     # an outlier, spread over its tile
+    w[32:64, 32:64] = 0.0                              # an all-zero tile
+    w[96:96 + n, 64:96] = np.float32(1e-3)             # a constant tile: one nonzero per column pair
+    if dtype == "bf16":
+        w = inputs.f32_to_bf16_bits(w)
+    _two_sided_check(orc, w, n)
+    _two_sided_check(orc, w, n, ld_pad=32)
+
+
+def test_two_sided_hadamard_layer_weights(orc):
+    """The Gemma-like layer's q projection [2048, 2048] BF16, 32 x 32 tiles."""
+    w = inputs.c3_layer(0, which=("W_q",))["W_q"]
+    _two_sided_check(orc, w, 32)
+
+
+def test_two_sided_hadamard_nonfinite_and_empty(orc):
+    w = np.zeros((32, 64), np.float32)
+    w[3, 40] = np.inf
+    f = G.flags_dev()
+    nv4.hadamard2_rotate(G.f32_dev(w), 32, d_flags=f)
+    torch.cuda.synchronize()
+    assert f.item() & 1
+    empty = torch.empty((0, 64), dtype=torch.float32, device=G.DEV)
+    assert nv4.hadamard2_rotate(empty, 16).shape == (0, 64)

@@ -31,7 +31,7 @@
 // threshold instead.  A thread starts at the max-calibrated code (nearest E4M3 to
 // amax_b / (6 s2)) and walks outwards, alternating down and up: a candidate whose
 // bound (1) exceeds the threshold skips the quadratic form, and once bound (2) over
-// the two largest |w_i| exceeds it, the downward walk ends.  Both comparisons
+// the two largest |w_i| exceeds it, the downward walk ends.  The comparisons
 // keep a relative margin of 2^-10, far above the FP32 evaluation error, so skipped
 // candidates could not have changed the FP32 result either.  When rho < 1/32, or H_b
 // has a zero diagonal entry with a nonzero row, or non-finite entries, the bounds are
@@ -319,6 +319,41 @@ __device__ __noinline__ Search64 search_fp64_warp(const uint4* __restrict__ src,
     return Search64{B, s2, C};
 }
 
+// The FP64 searches of a CTA's listed rows, one warp per row; lane 0 writes the outputs.
+// Returns the number of rows this lane finished (lane 0 only), for the work counter.
+template <int kDt>
+__device__ __noinline__ uint32_t redo_phase(const SweepJobDev& job, uint32_t b, uint32_t nr,
+                                            const uint16_t* __restrict__ list, const uint4 (*__restrict__ sw)[kDt == 0 ? 2 : 4],
+                                            const uint32_t* __restrict__ srow, const float4* __restrict__ tab,
+                                            const float* __restrict__ hs, uint32_t* d_flags)
+{
+    const uint32_t warp = threadIdx.x >> 5, lane = threadIdx.x & 31u;
+    uint32_t done = 0u;
+#pragma unroll 1
+    for (uint32_t i = warp; i < nr; i += kSweepThreads / 32) {
+        const uint32_t slot = list[i];
+        const Search64 r = search_fp64_warp<kDt>(sw[slot], tab, hs);
+        if (lane == 0) {
+            const int64_t blk = (int64_t)srow[slot] * job.nblk + b;
+            job.codes[blk] = (uint8_t)r.code;
+            if (job.q != nullptr) {
+                float2 w[8];
+                unstage_block<kDt>(sw[slot], w);
+                uint32_t c0, c1;
+                const float4 tw = tab[r.code];
+                codes8h(w, tw, c0);
+                codes8h(w + 4, tw, c1);
+                *reinterpret_cast<uint2*>(job.q + blk * 8) = make_uint2(c0, c1);
+            }
+            if (job.cost1 != nullptr) job.cost1[blk] = (float)r.best;
+            if (job.cost2 != nullptr) job.cost2[blk] = (float)r.second;
+            if (!(fabs(r.best) <= 1.7e308)) flag_or(d_flags, kFlagNonFinite);
+            ++done;
+        }
+    }
+    return done;
+}
+
 constexpr uint32_t kNoRow = 0xFFFFFFFFu;
 
 // One CTA = one block column b of one job and up to p.tiles_per_cta tiles of 128 rows.
@@ -387,7 +422,6 @@ sweep_kernel(const __grid_constant__ SweepParams p)
     if (threadIdx.x >= 96) block_bound(hs, reinterpret_cast<float*>(rd4), &bound_ok, &eta_s);
     __syncthreads();
     const bool pr = bound_ok != 0;
-    const float eta = eta_s;                                    // relative error bound of the FP32 costs
     const float k6 = __frcp_rn(__fmul_rn(6.0f, s2));            // ~ 1/(6 s2), for the starting code
     const float* rd = reinterpret_cast<const float*>(rd4);
     const uint32_t s2flag = isfinite(s2) ? 0u : kFlagOverflow;
@@ -486,7 +520,6 @@ sweep_kernel(const __grid_constant__ SweepParams p)
         // the threshold a candidate's lower bound must exceed to be skipped: the
         // runner-up cost when it is an output, else the best cost
         const bool need2 = job.cost2 != nullptr;
-        const bool need_costs = need2 || job.cost1 != nullptr;
         float best = __int_as_float(0x7F800000), second = best, thr = best;
         uint32_t best_c = 0u;
         bool redo = false;
@@ -558,7 +591,10 @@ sweep_kernel(const __grid_constant__ SweepParams p)
             }
             // FP32 costs exact to eta relative: a runner-up within 3 eta of the winner (or
             // costs that are outputs) needs the FP64 search unless eta certifies the argmin
-            redo = eta > kCertifiedEta && (need_costs || !(second > fmaf(best, 3.0f * eta, best)));
+            // (eta and the cost outputs are read here, not held through the walk)
+            const float eta = *reinterpret_cast<volatile float*>(&eta_s);
+            redo = eta > kCertifiedEta &&
+                   (job.cost1 != nullptr || job.cost2 != nullptr || !(second > fmaf(best, 3.0f * eta, best)));
         }
         if (redo) {                       // decided later by the FP64 search of a whole warp
             flag_or(p.d_flags, flags);
@@ -583,29 +619,10 @@ sweep_kernel(const __grid_constant__ SweepParams p)
 
     // ---- blocks whose FP32 costs do not certify the argmin: exhaustive FP64 search, one warp each
     __syncthreads();
-    const uint32_t nr = n_redo;
-#pragma unroll 1
-    for (uint32_t i = warp; i < nr; i += kSweepThreads / 32) {
-        const uint32_t slot = redo_list[i];
-        const Search64 r = search_fp64_warp<kDt>(sw[slot], tab, hs);
-        if (lane == 0) {
-            const int64_t blk = (int64_t)srow[slot] * job.nblk + b;
-            job.codes[blk] = (uint8_t)r.code;
-            if (job.q != nullptr) {
-                float2 w[8];
-                unstage_block<kDt>(sw[slot], w);
-                uint32_t c0, c1;
-                const float4 tw = tab[r.code];
-                codes8h(w, tw, c0);
-                codes8h(w + 4, tw, c1);
-                *reinterpret_cast<uint2*>(job.q + blk * 8) = make_uint2(c0, c1);
-            }
-            if (job.cost1 != nullptr) job.cost1[blk] = (float)r.best;
-            if (job.cost2 != nullptr) job.cost2[blk] = (float)r.second;
-            if (!(fabs(r.best) <= 1.7e308)) flag_or(p.d_flags, kFlagNonFinite);
-            nhalf += 2u * 127u;
-            nfull += 127u;
-        }
+    if (n_redo != 0u) {
+        const uint32_t done = redo_phase<kDt>(job, b, n_redo, redo_list, sw, srow, tab, hs, p.d_flags);
+        nhalf += 2u * 127u * done;
+        nfull += 127u * done;
     }
     if (job.d_work != nullptr) {
         __syncwarp();

@@ -82,6 +82,8 @@ def parse_args():
                    help="run only one kernel, --profile-reps times, on a case sized for an ncu capture "
                         "(inputs above the L2, a few GB at most); prints nothing but a one-line summary")
     p.add_argument("--profile-reps", type=int, default=3)
+    p.add_argument("--record-traffic", nargs="+", metavar="ROW=CSV", default=None,
+                   help="write profiles/dram_traffic.json from ncu --csv logs of --profile runs")
     return p.parse_args()
 
 
@@ -290,10 +292,9 @@ LAUNCHES = {"act": 3, "calib": 3, "moe": 4, "cast": 2}   # launches of this libr
 
 
 def traffic_table():
-    """DRAM bytes per launch from profiles/dram_traffic.json, for kernels whose sources
-    still hash to the values recorded with the capture (else the entry is dropped)."""
-    import hashlib
-
+    """DRAM bytes per unit for the rows recorded in profiles/dram_traffic.json, for kernels
+    whose sources still hash to the values recorded with the capture (else the entry is
+    dropped): {row: bytes per unit of the row's --profile case}."""
     path = os.path.join(ROOT, "profiles", "dram_traffic.json")
     try:
         with open(path) as f:
@@ -302,15 +303,12 @@ def traffic_table():
         return {}
     out = {}
     for k, e in doc.get("kernels", {}).items():
-        h = hashlib.sha256()
         try:
-            for fn in e["files"]:
-                with open(os.path.join(ROOT, fn), "rb") as f:
-                    h.update(f.read())
+            ok = _sources_sha([os.path.basename(f) for f in e["files"]]) == e.get("sources_sha256")
         except OSError:
             continue
-        if h.hexdigest() == e.get("sources_sha256"):
-            out[k] = e["dram_read_bytes"] + e["dram_write_bytes"]
+        if ok and e.get("units"):
+            out[k] = (e["dram_read_bytes"] + e["dram_write_bytes"]) / e["units"]
     return out
 
 
@@ -375,10 +373,10 @@ def fp32_peak(dev, reps=5):
             b.synchronize()
             t = a.elapsed_time(b) / 1e3
             best = t if best is None else min(best, t)
-        out["packed" if packed else "scalar"] = blocks * 256.0 * iters * 32 / best / 1e12
+        out["packed" if packed else "scalar"] = blocks * 256.0 * iters * 128 / best / 1e12
     out["measured"] = max(out["scalar"], out["packed"])
     out["nominal"] = FP32_NOMINAL_TFLOPS
-    out["how"] = (f"nv4_fp32_probe: {blocks} CTAs x 256 threads x {iters} rounds x 32 FLOP of independent FMAs, "
+    out["how"] = (f"nv4_fp32_probe: {blocks} CTAs x 256 threads x {iters} iterations x 128 FLOP of independent FMAs, "
                   f"scalar fma.rn.f32 and packed fma.rn.f32x2, best of {reps} event-timed launches each")
     return out
 
@@ -396,7 +394,7 @@ def sweep_row(nv4, jobs, flags, label, fp32):
     halves, costs = (int(x) for x in work.tolist())
     t = time_launch(lambda: nv4.nv4_scale_sweep_batched(jobs, flags), reps=5)
     executed = SWEEP_FLOP_PER_HALF * halves + SWEEP_FLOP_PER_COST * costs
-    return {"bound": "alu", "flops": SWEEP_FLOP_PER_BLOCK * blocks, "blocks": blocks, "s": t,
+    return {"bound": "alu", "flops": SWEEP_FLOP_PER_BLOCK * blocks, "blocks": blocks, "units": blocks, "s": t,
             "half_visits_per_block": halves / blocks, "costs_per_block": costs / blocks,
             "executed_tflops": executed / t / 1e12,
             "executed_frac": executed / t / 1e12 / fp32["measured"],
@@ -432,6 +430,7 @@ def kernel_rooflines(W, hbm_peak, fp32):
         out["dequant"] = {"bound": "hbm", "bytes": ACT_BYTES["dequant"] * n_all, "s": t}
         for k in ("tensor_amax", "act_quant", "dequant"):
             out[k]["launch"] = f"15 [T, C] bf16 shapes, {n_all / 1e6:.0f} M elements, one batched launch"
+            out[k]["units"] = n_all
         # fused fake quantize-dequantize (a widening of the path; not part of the step)
         qdq = torch.empty_like(big["x"])
         t = time_launch(lambda: nv4.nv4_fake_qdq(big["x"], a, qdq, s2, W["flags"]), flush=flush)
@@ -473,6 +472,7 @@ def kernel_rooflines(W, hbm_peak, fp32):
         t = time_launch(lambda: nv4.nv4_hessian_accum_batched([X, Xd], [W["H"], W["Hd"]], W["flags"]), reps=10,
                         flush=flush)
         out["hessian_accum"] = {"bound": "hbm", "bytes": 2.0 * (X.numel() + Xd.numel()), "s": t,
+                                "units": X.numel() + Xd.numel(),
                                 "launch": f"X [{X.shape[0]}, {X.shape[1]}] + X_down [{Xd.shape[0]}, {Xd.shape[1]}] bf16, "
                                           "one batched launch"}
         jobs = [{k: j[k] for k in ("w", "H", "d_amax_w", "codes", "q")} for j in W["weights"]]
@@ -508,7 +508,7 @@ def kernel_rooflines(W, hbm_peak, fp32):
     if "cast" in W:
         nmx = sum(j["e8m0"].numel() for j in W["cast"])
         t = time_launch(lambda: nv4.nv4_mxfp4_to_nvfp4_batched(W["cast"], W["counts"], W["flags"]), flush=flush)
-        out["mxfp4_to_nvfp4"] = {"bound": "hbm", "bytes": CAST_BYTES_PER_MX_BLOCK * nmx, "s": t,
+        out["mxfp4_to_nvfp4"] = {"bound": "hbm", "bytes": CAST_BYTES_PER_MX_BLOCK * nmx, "s": t, "units": nmx,
                                  "launch": "32 x [2880, 2880], out of place"}
     for k, v in out.items():
         if v["bound"] == "hbm":
@@ -528,7 +528,7 @@ def kernel_rooflines(W, hbm_peak, fp32):
         v["ms"] = v["s"] * 1e3
     traffic = traffic_table()
     for k, v in out.items():
-        v["traffic"] = traffic.get(k)
+        v["traffic"] = traffic[k] * v["units"] if k in traffic and v.get("units") else None
     return out
 
 
@@ -591,6 +591,50 @@ def e2e_act(W, steps):
     b.record(s_out)
     b.synchronize()
     torch.cuda.synchronize()
+    return a.elapsed_time(b) / 1e3 / steps, h2d, d2h
+
+
+def e2e_part(W, part, steps):
+    """One part of the step end to end through the public API, from pinned host buffers:
+    the part's inputs copied in, its launches, its outputs copied back, on one stream.
+    calib: X, X_down and the four weights in; winning codes and packed nibbles out.
+    moe: the 128 routed inputs and 192 weights in; codes and nibbles out.  cast: MXFP4
+    nibbles and E8M0 scales in; NVFP4 nibbles, E4M3 scales, s2 and counts out."""
+    import torch
+
+    if part == "calib":
+        ins = [W["X"], W["Xd"]] + [j["w"] for j in W["weights"]]
+        outs = [t for j in W["weights"] for t in (j["codes"], j["q"])]
+    elif part == "moe":
+        ins = W["moe_X"] + W["moe_Xd"] + [j["w"] for j in W["moe_weights"]]
+        outs = [t for j in W["moe_weights"] for t in (j["codes"], j["q"])]
+    else:
+        ins = [t for j in W["cast"] for t in (j["mx_q"], j["e8m0"])]
+        outs = [t for j in W["cast"] for t in (j["nv_q"], j["nv_scales"], j["d_s2"])] + [W["counts"]]
+    h_in = [t.cpu().pin_memory() for t in ins]
+    h_out = [torch.empty(tuple(t.shape), dtype=t.dtype).pin_memory() for t in outs]
+    h2d = sum(t.numel() * t.element_size() for t in h_in)
+    d2h = sum(t.numel() * t.element_size() for t in h_out)
+    st = torch.cuda.Stream()
+
+    def one():
+        with torch.cuda.stream(st):
+            for d, h in zip(ins, h_in):
+                d.copy_(h, non_blocking=True)
+            PARTS[part](W)
+            for h, d in zip(h_out, outs):
+                h.copy_(d, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(st)
+    for _ in range(steps):
+        one()
+    b.record(st)
+    b.synchronize()
+    del h_in, h_out
     return a.elapsed_time(b) / 1e3 / steps, h2d, d2h
 
 
@@ -818,6 +862,23 @@ def run_ours(args):
         bytes_act, _ = act_bytes(W)
         e2e = {"value": ws * bytes_act / e2e_s / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_s * 1e3}
+    if not args.no_e2e:
+        # the other parts end to end from host buffers (one stream each, copies inside the
+        # timed region), reported beside the act part's metric
+        e2e_parts = {}
+        for prt in ("calib", "moe", "cast"):
+            if prt in parts:
+                t_s, h2d_p, d2h_p = e2e_part(W, prt, 2)
+                t_s = dist.max_over_ranks([t_s])[0]
+                e2e_parts[prt] = {"ms_per_step": t_s * 1e3, "h2d_bytes_per_step": h2d_p,
+                                  "d2h_bytes_per_step": d2h_p,
+                                  "device_ms_per_step": part_s[prt] / args.steps * 1e3}
+                if prt in ("calib", "moe"):
+                    wts = W["weights"] if prt == "calib" else W["moe_weights"]
+                    e2e_parts[prt]["blocks_per_s"] = ws * sum(j["codes"].numel() for j in wts) / t_s
+        if e2e is None:
+            e2e = {}
+        e2e["parts"] = e2e_parts
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(args.seed)
@@ -973,6 +1034,20 @@ def _prof_setup_act(kind):
     return setup
 
 
+def _prof_setup_hadamard2(dev, seed):
+    import torch
+
+    from nvfp4_block_numerics_b200 import binding as nv4
+    from nvfp4_block_numerics_b200 import inputs
+
+    w = inputs.f32_to_bf16_bits(inputs.normal_weights(inputs.rng_for(seed, "prof", "h2"), 16384, 8192, 0.02))
+    wd = torch.from_numpy(w.view(np.int16)).view(torch.bfloat16).to(dev)
+    q = torch.empty((16384, 4096), dtype=torch.uint8, device=dev)
+    e8 = torch.empty((16384, 256), dtype=torch.uint8, device=dev)
+    return (lambda: nv4.nv4_hadamard2_mxfp4_quant(wd, 32, q, e8)), \
+        "hadamard2_kernel: [16384, 8192] bf16 weights, 32 x 32 tiles, MXFP4"
+
+
 def _prof_setup_cast(dev, seed):
     W = build_workload(["cast"], seed, dev)
     from nvfp4_block_numerics_b200 import binding as nv4
@@ -982,9 +1057,94 @@ def _prof_setup_cast(dev, seed):
 
 
 PROFILE_CASES = {"gemm": _prof_setup_gemm, "sweep": _prof_setup_sweep, "sweep_moe": _prof_setup_sweep_moe,
-                 "hessian": _prof_setup_hessian, "cast": _prof_setup_cast,
+                 "hessian": _prof_setup_hessian, "cast": _prof_setup_cast, "hadamard2": _prof_setup_hadamard2,
                  **{k: _prof_setup_act(k) for k in ("amax", "act_quant", "dequant", "fake_qdq", "rtn", "fp8",
                                                     "mxfp4", "hadamard")}}
+
+
+# Roofline rows whose DRAM traffic comes from an ncu capture of a --profile case: the
+# case, the kernel-name pattern, the sources the figure is valid for, and the units the
+# case processes (the bench scales the per-unit traffic to its own launch of the row).
+TRAFFIC_ROWS = {
+    "tensor_amax": ("amax", "amax_kernel", ["quant.cu", "nv4_common.cuh"], 65536 * 7168),
+    "act_quant": ("act_quant", "act_quant_kernel", ["quant.cu", "nv4_common.cuh"], 65536 * 7168),
+    "dequant": ("dequant", "dequant_kernel", ["quant.cu", "nv4_common.cuh"], 65536 * 7168),
+    "hessian_accum": ("hessian", "hessian_kernel", ["hessian.cu", "nv4_async.cuh", "nv4_common.cuh"],
+                      16384 * 2048 + 16384 * 16384),
+    "scale_sweep": ("sweep", "sweep_kernel", ["sweep.cu", "nv4_common.cuh"], 6553600),
+    "scale_sweep_moe": ("sweep_moe", "sweep_kernel", ["sweep.cu", "nv4_common.cuh"], 16 * 3 * 1536 * 4096 // 16),
+    "mxfp4_to_nvfp4": ("cast", "cast_", ["cast.cu", "nv4_common.cuh"], 32 * 2880 * 90),
+}
+
+
+def _sources_sha(files):
+    import hashlib
+
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "nvfp4_block_numerics_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def record_traffic(pairs):
+    """profiles/dram_traffic.json from ncu CSV logs (ROW=PATH): DRAM bytes per launch of the
+    row's kernels in the row's --profile case (summed over the kernels one call launches,
+    averaged over the captured calls), with the units the case processed and the hash of the
+    sources they are valid for."""
+    import csv
+
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    try:
+        with open(path) as f:
+            doc = json.load(f)
+    except Exception:
+        doc = {}
+    doc["about"] = ("DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of each row's kernels in one call "
+                    "of its bench.py --profile case, from one ncu capture, with the units that case processes; "
+                    "bench.py scales them to the units of its own launch of the row and reports null once the "
+                    "kernel sources no longer hash to sources_sha256.  Written by bench.py --record-traffic.")
+    kern = doc.setdefault("kernels", {})
+    for pair in pairs:
+        row, csv_path = pair.split("=", 1)
+        case, pattern, files, units = TRAFFIC_ROWS[row]
+        per_id = {}
+        scale = {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9, "KB": 1e3, "MB": 1e6, "GB": 1e9}
+        with open(csv_path) as f:
+            lines = [ln for ln in f if ln.startswith('"')]
+        recs = list(csv.reader(lines))
+        hdr = recs[0]
+        if "Metric Name" in hdr:            # ncu --csv --metrics ... (one row per metric)
+            for rec in (dict(zip(hdr, r)) for r in recs[1:]):
+                name = rec.get("Metric Name")
+                if pattern not in rec.get("Kernel Name", "") or name not in ("dram__bytes_read.sum",
+                                                                           "dram__bytes_write.sum"):
+                    continue
+                val = float(rec["Metric Value"].replace(",", "")) * scale.get(rec.get("Metric Unit", "byte"), 1)
+                d = per_id.setdefault(rec["ID"], {"read": 0.0, "write": 0.0})
+                d["read" if name.endswith("read.sum") else "write"] += val
+        else:                               # ncu -i REP --csv --page raw --metrics ... (one row per launch)
+            units_row = dict(zip(hdr, recs[1]))
+            for rec in (dict(zip(hdr, r)) for r in recs[2:]):
+                if pattern not in rec.get("Kernel Name", ""):
+                    continue
+                d = per_id.setdefault(rec["ID"], {"read": 0.0, "write": 0.0})
+                for key, col in (("read", "dram__bytes_read.sum"), ("write", "dram__bytes_write.sum")):
+                    d[key] += float(rec[col].replace(",", "")) * scale.get(units_row.get(col, "byte"), 1)
+        if not per_id:
+            raise SystemExit(f"no {pattern} launches with DRAM counters in {csv_path}")
+        # a call of the case launches one kernel (two for the cast): group captured launches per call
+        per_call = 2 if row == "mxfp4_to_nvfp4" else 1
+        ids = sorted(per_id, key=int)
+        calls = max(1, len(ids) // per_call)
+        rd = sum(per_id[i]["read"] for i in ids[:calls * per_call]) / calls
+        wr = sum(per_id[i]["write"] for i in ids[:calls * per_call]) / calls
+        kern[row] = {"files": [f"nvfp4_block_numerics_b200/csrc/{f}" for f in files], "case": f"--profile {case}",
+                     "units": units, "dram_read_bytes": int(round(rd)), "dram_write_bytes": int(round(wr)),
+                     "sources_sha256": _sources_sha(files)}
+        print(row, kern[row]["dram_read_bytes"], kern[row]["dram_write_bytes"])
+    with open(path, "w") as f:
+        json.dump(doc, f, indent=1)
 
 
 def run_profile(args):
@@ -1009,7 +1169,9 @@ def run_profile(args):
 
 def main():
     args = parse_args()
-    if args.profile is not None:
+    if args.record_traffic is not None:
+        record_traffic(args.record_traffic)
+    elif args.profile is not None:
         run_profile(args)
     elif args.impl == "reference":
         run_reference(args)

@@ -25,13 +25,18 @@
 //       1 - max_i sum_{j != i} |H'_ij|, so for every e:  e^T H_b e >= rho sum_i H_ii e_i^2.
 //   (2) Every grid point of scale S is at most 6S in magnitude, so |e_i| >= |w_i| - 6S,
 //       and the same holds at every smaller scale.
+//   (3) An element with |w_i| <= S/2 is at least min(|w_i|, S/2 - |w_i|) away from every
+//       grid point of every scale >= S (its nearest points there are 0 and S'/2 >= S/2),
+//       so rho * sum_i H_ii min(.)^2 bounds the cost of every candidate from S upwards.
 // The winner and the runner-up cost depend only on candidates whose cost is at most
 // the running runner-up cost; when the runner-up is not an output, only the winner
 // (ties to the lowest code) has to be found and the running best cost is the
 // threshold instead.  A thread starts at the max-calibrated code (nearest E4M3 to
 // amax_b / (6 s2)) and walks outwards, alternating down and up: a candidate whose
 // bound (1) exceeds the threshold skips the quadratic form, and once bound (2) over
-// the two largest |w_i| exceeds it, the downward walk ends.  The comparisons
+// the two largest |w_i| exceeds it, the downward walk ends; once bound (3) exceeds it,
+// the upward walk ends (long upward walks: weights whose block amax is far below the
+// tensor's, such as heavy-tailed expert weights).  The comparisons
 // keep a relative margin of 2^-10, far above the FP32 evaluation error, so skipped
 // candidates could not have changed the FP32 result either.  When rho < 1/32, or H_b
 // has a zero diagonal entry with a nonzero row, or non-finite entries, the bounds are
@@ -575,8 +580,29 @@ sweep_kernel(const __grid_constant__ SweepParams p)
                         thr = need2 ? second : best;
                     }
                 }
-                // next candidate: alternate down / up; bound (2) closes the downward walk
+                // next candidate: alternate down / up; bound (2) closes the downward walk and
+                // bound (3), checked at every fourth upward code up to 110 (long upward walks
+                // only: rows whose starting code is low, such as heavy-tailed expert weights;
+                // on the Gemma-like layer, whose starting codes are ~115, it would save less
+                // than it costs), the upward one
                 bool take_dn = dn >= 0 && (go_dn || up > 126);
+                if (!take_dn && pr && (up & 3) == 0 && up <= 110) {
+                    const float h = 0.5f * tab[up].x;
+                    float2 acc = make_float2(0.0f, 0.0f);
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        const float ax = fabsf(w[k].x), ay = fabsf(w[k].y);
+                        const float gx = ax <= h ? fminf(ax, h - ax) : 0.0f;
+                        const float gy = ay <= h ? fminf(ay, h - ay) : 0.0f;
+                        const float4 d = rd4[k >> 1];
+                        const float2 dk = (k & 1) ? make_float2(d.z, d.w) : make_float2(d.x, d.y);
+                        acc = __ffma2_rn(__fmul2_rn(dk, make_float2(gx, gy)), make_float2(gx, gy), acc);
+                    }
+                    if ((acc.x + acc.y) * kPruneScale > thr) {
+                        up = 127;
+                        take_dn = dn >= 0;
+                    }
+                }
                 if (take_dn && pr) {
                     const float S = tab[dn].x;
                     const float u1 = fmaxf(fmaf(-6.0f, S, a1), 0.0f), u2 = fmaxf(fmaf(-6.0f, S, a2), 0.0f);

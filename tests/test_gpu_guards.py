@@ -165,3 +165,22 @@ def test_guards_gemm_and_scale_layout(M, N, K, ldd):
         assert f.item() == 0 and full.intact()
         assert torch.all(full.t[:, N:] == 0), "the GEMM wrote into the row padding beyond N"
         assert torch.equal(out, nv4.gemm_nvfp4(qa, sa, one, qb, sb, one, dtype=dt))
+
+
+@pytest.mark.parametrize("n,rows", [(16, 16), (32, 96), (16, 208)])
+def test_guards_two_sided_hadamard(n, rows):
+    cols = 96
+    w = _x(rows, cols, seed=5, dtype=torch.float32)
+    out = Guarded((rows, cols), torch.float32)
+    nv4.nv4_hadamard2_rotate(w, n, out.t)
+    assert out.intact() and torch.equal(out.t, nv4.hadamard2_rotate(w, n))
+    q, e = Guarded((rows, cols // 2), torch.uint8), Guarded((rows, cols // 32), torch.uint8)
+    nv4.nv4_hadamard2_mxfp4_quant(w, n, q.t, e.t)
+    assert q.intact() and e.intact()
+    amax = torch.zeros(1, dtype=torch.float32, device=G.DEV)
+    nv4.nv4_hadamard2_amax(w, n, amax)
+    q, sc, s2 = Guarded((rows, cols // 2), torch.uint8), Guarded((rows, cols // 16), torch.uint8), Guarded((1,), torch.float32)
+    nv4.nv4_hadamard2_nvfp4_quant(w, n, amax, q.t, sc.t, s2.t)
+    assert q.intact() and sc.intact() and s2.intact()
+    qr, scr, _, _ = nv4.hadamard2_nvfp4_quant(w, n)
+    assert torch.equal(q.t, qr) and torch.equal(sc.t, scr)

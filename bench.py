@@ -853,7 +853,7 @@ def run_ours(args):
     part_s = {p: t[i + 1] for i, p in enumerate(parts)}
     flags = int(W["flags"].item())
 
-    fp32 = fp32_peak(dev)
+    fp32 = None if args.no_rooflines else fp32_peak(dev)
     roof = {} if args.no_rooflines else kernel_rooflines(W, hbm_peak, fp32)
     e2e = None
     if "act" in parts and not args.no_e2e:

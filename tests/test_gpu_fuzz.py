@@ -194,3 +194,71 @@ def test_fuzz_hadamard(orc, batch):
         torch.cuda.synchronize()
         assert np.array_equal(G.host(e8), re8) and np.array_equal(G.host(q), rq), (k, n)
         assert s2n.item() == ns2 and np.array_equal(G.host(scn), nsc) and np.array_equal(G.host(qn), nq), (k, n)
+
+
+@pytest.mark.parametrize("batch", range(3))
+def test_fuzz_two_sided_hadamard(orc, batch):
+    """Two-sided block Hadamard of weight tiles (n = 16, 32) fused with MXFP4 and NVFP4
+    quantization on random shapes, dtypes, row pitches and binades: rotated values, codes
+    and scales bit for bit."""
+    for k in range(4):
+        r = np.random.default_rng(40000 + 10 * batch + k)
+        n = int(r.choice([16, 32]))
+        rows, cols = n * int(r.integers(1, 8)), 32 * int(r.integers(1, 7))
+        w = (r.standard_normal((rows, cols)) * float(10.0 ** r.uniform(-25, 25))).astype(np.float32)
+        w[np.abs(w) < np.float32(1e-3) * np.abs(w).max()] = 0.0   # keeps every tile inside the FP64-exact span
+        if r.random() < 0.5:
+            w = inputs.f32_to_bf16_bits(w)
+        pad = int(r.choice([0, 32]))
+        dt = torch.float32 if w.dtype == np.float32 else torch.bfloat16
+        full = torch.zeros((rows, cols + pad), dtype=dt, device=G.DEV)
+        full[:, :cols] = G.f32_dev(w) if w.dtype == np.float32 else G.bf16_dev(w)
+        wd = full[:, :cols]
+        y = orc.hadamard2_rotate(w, n)
+        got = nv4.hadamard2_rotate(wd, n)
+        q, e8 = nv4.hadamard2_mxfp4_quant(wd, n)
+        qn, scn, s2n, _ = nv4.hadamard2_nvfp4_quant(wd, n)
+        torch.cuda.synchronize()
+        assert np.array_equal(G.host(got).view(np.uint32), y.view(np.uint32)), (k, n)
+        rq, re8, _ = orc.mxfp4_quant(y)
+        assert np.array_equal(G.host(e8), re8) and np.array_equal(G.host(q), rq), (k, n)
+        nq, nsc, ns2, _ = orc.rtn_quant(y, float(np.abs(y).max()))
+        assert s2n.item() == ns2 and np.array_equal(G.host(scn), nsc) and np.array_equal(G.host(qn), nq), (k, n)
+
+
+@pytest.mark.parametrize("batch", range(4))
+def test_fuzz_sweep_conditioning(orc, batch):
+    """Hessian columns of random conditioning: scaled Gershgorin ratio rho from -0.5 (no
+    bound: FP64 search) through the uncertified 1/32 .. 0.6 range (FP32 walk, FP64
+    re-search near ties) to 0.95, BF16 and FP32 weights; the plain parity rule, and the
+    codes-only call equal to the full call."""
+    r = np.random.default_rng(50000 + batch)
+    rhos = r.uniform(-0.5, 0.95, 6)
+    H = np.stack([_gershgorin_block(r, rho) for rho in rhos])
+    w = (r.standard_normal((int(r.integers(40, 300)), 96)) * 0.02).astype(np.float32)
+    w[:: int(r.integers(3, 9)), int(r.integers(0, 96))] *= 30.0
+    if r.random() < 0.5:
+        w = inputs.f32_to_bf16_bits(w)
+    H32 = H.astype(np.float32)
+    wd = G.f32_dev(w) if w.dtype == np.float32 else G.bf16_dev(w)
+    d_amax = nv4.tensor_amax(wd)
+    fl = G.flags_dev()
+    codes, q, c1, c2 = nv4.scale_sweep(wd, G.f32_dev(H32), d_amax, d_flags=fl)
+    co, qo, _, _ = nv4.scale_sweep(wd, G.f32_dev(H32), d_amax, with_costs=False, d_flags=fl)
+    torch.cuda.synchronize()
+    assert fl.item() == 0
+    assert torch.equal(co, codes) and torch.equal(qo, q)
+    ref = orc.scale_sweep(w, H32.astype(np.float64), orc.tensor_amax(w)[0])
+    st = G.sweep_parity(G.host(codes), G.host(q), G.host(c1), ref, c2_gpu=G.host(c2))
+    assert st["mismatch_frac"] < 1e-3, (rhos, st)
+
+
+def _gershgorin_block(r, rho, tokens=4096):
+    """D^1/2 (I + (1 - rho) S) D^1/2 with S symmetric, zero diagonal, random signs and largest
+    absolute row sum 1: its scaled Gershgorin ratio is rho; positive definite for rho > 0,
+    possibly indefinite below."""
+    S = np.triu(r.standard_normal((16, 16)) * r.uniform(0.2, 1.0, (16, 16)), 1)
+    S = S + S.T
+    S /= np.abs(S).sum(1).max()
+    d = tokens * 4.0 ** r.uniform(-1, 1, 16)
+    return np.sqrt(d)[:, None] * (np.eye(16) + (1.0 - rho) * S) * np.sqrt(d)[None, :]

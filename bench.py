@@ -852,6 +852,7 @@ def run_ours(args):
     total_s = t[0]
     part_s = {p: t[i + 1] for i, p in enumerate(parts)}
     flags = int(W["flags"].item())
+    cast_counts = [int(v) for v in W["counts"].tolist()] if "cast" in parts else None   # the last step's
 
     fp32 = None if args.no_rooflines else fp32_peak(dev)
     roof = {} if args.no_rooflines else kernel_rooflines(W, hbm_peak, fp32)
@@ -948,6 +949,12 @@ def run_ours(args):
         line["sweep"] = sweep
     if sweep_moe is not None:
         line["sweep_moe"] = sweep_moe
+    if cast_counts is not None:
+        n16 = cast_counts[0] + cast_counts[1]
+        line["cast"] = {"in_window_blocks": cast_counts[0], "fallback_blocks": cast_counts[1],
+                        "lossless_blocks": cast_counts[2], "lossless_fraction": cast_counts[2] / max(n16, 1),
+                        "note": "16-element NVFP4 blocks of the 32 matrices; lossless = NVFP4 dequant equal to the "
+                                "MXFP4 dequant bit for bit"}
     if e2e is not None:
         line["e2e"] = e2e
     if cpu is not None:

@@ -281,10 +281,12 @@ cudaError_t launch_hadamard_quant(int mode, const void* x, int64_t rows, int64_t
 // one rounding to FP32.
 //
 // One warp per strip of n rows x 32 columns (one 32 x 32 tile, or two 16 x 16 tiles side by
-// side).  Lane l holds one row of its tile (n = 32: row l; n = 16: row l % 16 of tile
-// l / 16) and runs that row's FWHT in FP64 registers; a transpose through shared memory
-// gives lane l column l of the strip for the column FWHTs; the scaled, rounded values go
-// back through shared memory as FP32 so that lane l again holds its row for quantization:
+// side), with the next strip's loads issued before the current one is transformed.  Lane l
+// holds one row of its tile (n = 32: row l; n = 16: row l % 16 of tile l / 16) and runs that
+// row's FWHT in FP64 registers; a transpose through shared memory (rows written as 16-byte
+// pairs) gives lane l column l of the strip for the column FWHTs; the scaled, rounded values
+// go back through shared memory as FP32 (rows read as 16-byte quads) so that lane l again
+// holds its row for quantization:
 //   mode 0: running max |y| into *d_amax;  mode 1: MXFP4 (32-element blocks along the row:
 //   one lane's row for n = 32, lanes l and l + 16 together for n = 16);  mode 2: NVFP4
 //   (16-element blocks) with s2 = RN32(amax / 2688);  mode 3: y itself, FP32 [rows, cols].
@@ -311,10 +313,10 @@ hadamard2_kernel(const void* __restrict__ w, uint32_t strips, uint32_t strips_pe
                  float* __restrict__ d_amax, uint8_t* __restrict__ q, uint8_t* __restrict__ sc,
                  float* __restrict__ d_s2, float* __restrict__ out, uint32_t* __restrict__ d_flags)
 {
-    __shared__ double tbuf[kHad2Warps][kN][33];
+    __shared__ __align__(16) double tbuf[kHad2Warps][kN][34];
     const uint32_t lane = threadIdx.x & 31u, warp = threadIdx.x >> 5;
-    double (*T)[33] = tbuf[warp];
-    float (*Y)[33] = reinterpret_cast<float (*)[33]>(&tbuf[warp][0][0]);   // kN x 33 floats fit
+    double (*T)[34] = tbuf[warp];                                         // rows 16-byte aligned
+    float (*Y)[36] = reinterpret_cast<float (*)[36]>(&tbuf[warp][0][0]);   // kN x 36 floats fit
     uint32_t flags = 0u, mx_bits = 0u;
 
     float s2 = 0.0f, k_lo = 0.0f, k_hi = 0.0f;
@@ -331,34 +333,46 @@ hadamard2_kernel(const void* __restrict__ w, uint32_t strips, uint32_t strips_pe
     const uint32_t r = kN == 32 ? lane : (lane & 15u);            // this lane's row in the strip
     const uint32_t cb = kN == 32 ? 0u : 16u * (lane >> 4);         // and its first column
 
-    for (uint32_t st = blockIdx.x * kHad2Warps + warp; st < strips; st += gridDim.x * kHad2Warps) {
+    constexpr int kRaw = kN * (kDt == 0 ? 2 : 4) / 16;            // 16-byte loads per lane and strip
+    const uint32_t stride = gridDim.x * kHad2Warps;
+    auto load = [&](uint32_t st, uint4 raw[kRaw]) {
         const uint32_t band = st / strips_per_band, cs = st - band * strips_per_band;
         const int64_t row = (int64_t)band * kN + r;
         const int64_t col = 32 * (int64_t)cs + cb;
-        double v[kN];
-        if constexpr (kDt == 0) {
-            const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(w) + row * ld + col);
+        const uint4* src = reinterpret_cast<const uint4*>(static_cast<const char*>(w) +
+                                                          (row * ld + col) * (kDt == 0 ? 2 : 4));
 #pragma unroll
-            for (int k = 0; k < kN / 8; ++k) {
-                const uint4 raw = __ldcs(src + k);
-                const uint32_t u[4] = {raw.x, raw.y, raw.z, raw.w};
+        for (int k = 0; k < kRaw; ++k) raw[k] = __ldcs(src + k);
+    };
+    uint4 nxt[kRaw];
+    if (blockIdx.x * kHad2Warps + warp < strips) load(blockIdx.x * kHad2Warps + warp, nxt);
+    for (uint32_t st = blockIdx.x * kHad2Warps + warp; st < strips; st += stride) {
+        const uint32_t band = st / strips_per_band, cs = st - band * strips_per_band;
+        const int64_t row = (int64_t)band * kN + r;
+        const int64_t col = 32 * (int64_t)cs + cb;
+        uint4 raw[kRaw];
+#pragma unroll
+        for (int k = 0; k < kRaw; ++k) raw[k] = nxt[k];
+        if (st + stride < strips) load(st + stride, nxt);         // the next strip's loads in flight
+        double v[kN];
+#pragma unroll
+        for (int k = 0; k < kRaw; ++k) {
+            const uint32_t u[4] = {raw[k].x, raw[k].y, raw[k].z, raw[k].w};
+            if constexpr (kDt == 0) {
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                     v[8 * k + 2 * j] = (double)bf16_lo(u[j]);
                     v[8 * k + 2 * j + 1] = (double)bf16_hi(u[j]);
                 }
-            }
-        } else {
-            const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(w) + row * ld + col);
+            } else {
 #pragma unroll
-            for (int k = 0; k < kN / 4; ++k) {
-                const float4 f = __ldcs(src + k);
-                v[4 * k] = f.x; v[4 * k + 1] = f.y; v[4 * k + 2] = f.z; v[4 * k + 3] = f.w;
+                for (int j = 0; j < 4; ++j) v[4 * k + j] = (double)__uint_as_float(u[j]);
             }
         }
         fwht_regs<kN>(v);                                          // row transform: B H
 #pragma unroll
-        for (int j = 0; j < kN; ++j) T[r][cb + j] = v[j];
+        for (int j = 0; j < kN; j += 2)
+            *reinterpret_cast<double2*>(&T[r][cb + j]) = make_double2(v[j], v[j + 1]);
         __syncwarp();
 #pragma unroll
         for (int i = 0; i < kN; ++i) v[i] = T[i][lane];            // column `lane` of the strip
@@ -370,10 +384,12 @@ hadamard2_kernel(const void* __restrict__ w, uint32_t strips, uint32_t strips_pe
         float y[kN];
         uint32_t ab = 0u;
 #pragma unroll
-        for (int j = 0; j < kN; ++j) {
-            y[j] = Y[r][cb + j];
-            ab = max(ab, __float_as_uint(y[j]) & 0x7FFFFFFFu);
+        for (int j = 0; j < kN; j += 4) {
+            const float4 f4 = *reinterpret_cast<const float4*>(&Y[r][cb + j]);
+            y[j] = f4.x; y[j + 1] = f4.y; y[j + 2] = f4.z; y[j + 3] = f4.w;
         }
+#pragma unroll
+        for (int j = 0; j < kN; ++j) ab = max(ab, __float_as_uint(y[j]) & 0x7FFFFFFFu);
         __syncwarp();                                              // before the next strip reuses T
         if (ab >= 0x7F800000u) flags |= kFlagNonFinite;
 

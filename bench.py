@@ -834,14 +834,18 @@ def run_ours(args):
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
     start.record(stream)
-    for _ in range(args.steps):
+    for i in range(args.steps):
+        torch.cuda.nvtx.range_push(f"step {i}")              # NVTX ranges: visible in an nsys/ncu timeline
         for p in parts:
             a = torch.cuda.Event(enable_timing=True)
             b = torch.cuda.Event(enable_timing=True)
+            torch.cuda.nvtx.range_push(p)
             a.record(stream)
             graphs[p].replay()
             b.record(stream)
+            torch.cuda.nvtx.range_pop()
             ev[p].append((a, b))
+        torch.cuda.nvtx.range_pop()
     end.record(stream)
     torch.cuda.synchronize()
     dist.barrier()

@@ -30,7 +30,10 @@
 //     memory through matrix descriptors, commits "empty" and "sf_free", and commits
 //     "acc_full" after the tile's last stage.
 //   * warps 0-3: epilogue.  Warp w reads accumulator lanes 32w..32w+31 with tcgen05.ld (one
-//     output row per thread), multiplies by s2_A * s2_B, stores, and arrives on acc_empty.
+//     output row per thread), multiplies by s2_A * s2_B and, for BF16, transposes each 32 x
+//     32 block through 2 KB of shared memory so that a store instruction writes 8 rows x 64
+//     contiguous bytes instead of 32 rows x 16 (8192^3: +4%, 16384 x 16384 x 2048: +9%);
+//     it arrives on acc_empty once the accumulator has been read.
 // The accumulator is single-buffered (a second 256-column one does not fit the 512 columns
 // next to the scale buffers), so the epilogue still runs between two tiles' MMAs.
 // Every mbarrier wait is bounded (kWaitLimitNs); on expiry the kernel sets
@@ -78,6 +81,7 @@ struct Smem {
     uint8_t b[kStages][Cfg<kBN>::kBTile];
     uint8_t sfa[kStages][Cfg<kBN>::kSfA];
     uint8_t sfb[kStages][Cfg<kBN>::kSfB];
+    uint8_t stg[4][2048];                         // per epilogue warp: 32 rows x 64 bytes, swizzled
     uint64_t full[kStages], empty[kStages], sf_full[kSfBufs], sf_free[kSfBufs], acc_full, acc_empty, drain;
     uint32_t tmem_base;
     uint32_t abort;                               // set by a wait that gave up
@@ -377,9 +381,23 @@ gemm_nvfp4_kernel(const __grid_constant__ Params p)
                         asm("cvt.rn.bf16x2.f32 %0, %1, %2;"
                             : "=r"(w[k])
                             : "f"(__fmul_rn(v[2 * k + 1], alpha)), "f"(__fmul_rn(v[2 * k], alpha)));
-                    uint4* o = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + row * p.ldd + col);
+                    // transpose through the warp's staging rows: written one row per thread,
+                    // read back as 8 rows x 64 bytes per instruction (16-byte piece p of row r
+                    // at r * 64 + 16 * (p ^ (r & 3)): conflict-free both ways)
+                    uint8_t* st = sm.stg[warp];
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) o[k] = make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+                    for (int k = 0; k < 4; ++k)
+                        *reinterpret_cast<uint4*>(st + 64 * lane + 16 * (k ^ (lane & 3))) =
+                            make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+                    __syncwarp();
+                    const int pr = lane >> 2, pc = lane & 3;
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const int rr = pr + 8 * k;
+                        const uint4 x = *reinterpret_cast<const uint4*>(st + 64 * rr + 16 * (pc ^ (rr & 3)));
+                        *reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + (row - lane + rr) * p.ldd + col + 8 * pc) = x;
+                    }
+                    __syncwarp();
                 }
             }
             tc_fence_before();

@@ -7,7 +7,7 @@
 // as BF16 or FP32.
 //
 // Kernel structure: persistent, one CTA per SM walking the 128 x kBN output tiles
-// t = blockIdx.x, + gridDim.x, ... (kBN = 256 when N allows, else 128); 320 threads:
+// t = blockIdx.x, + gridDim.x, ... (kBN = 256 when N allows, else 128); 448 threads:
 //   * warp 8, one lane: producer.  Per stage of 256 K-elements it loads the A and B code
 //     tiles (128 rows x 128 bytes each) with 2-D TMA into 128-byte-swizzled shared
 //     memory, and the stage's scale-factor atoms (4 x 512 bytes per operand, already in
@@ -29,13 +29,15 @@
 //     tcgen05.mma kind::mxf4nvf4 block16 (K = 64 each) with both operands read from shared
 //     memory through matrix descriptors, commits "empty" and "sf_free", and commits
 //     "acc_full" after the tile's last stage.
-//   * warps 0-3: epilogue.  Warp w reads accumulator lanes 32w..32w+31 with tcgen05.ld (one
-//     output row per thread), multiplies by s2_A * s2_B and, for BF16, transposes each 32 x
-//     32 block through 2 KB of shared memory so that a store instruction writes 8 rows x 64
-//     contiguous bytes instead of 32 rows x 16 (8192^3: +4%, 16384 x 16384 x 2048: +9%);
-//     it arrives on acc_empty once the accumulator has been read.
+//   * warps 0-3 and 10-13: epilogue, two warps per 32-lane sub-partition, half the columns
+//     each.  A warp reads its 32 rows x kBN/2 accumulator columns with tcgen05.ld (one row
+//     per thread), multiplies by s2_A * s2_B and arrives on acc_empty; for BF16 the half
+//     row is converted into registers first and stored only after the accumulator has been
+//     released, so the stores overlap the next tile's MMAs, each 32 x 16 block transposed
+//     through 1 KB of shared memory so that a store instruction writes 16 rows x 32
+//     contiguous bytes instead of 32 rows x 16.
 // The accumulator is single-buffered (a second 256-column one does not fit the 512 columns
-// next to the scale buffers), so the epilogue still runs between two tiles' MMAs.
+// next to the scale buffers): the tensor pipe idles while the epilogue reads it.
 // Every mbarrier wait is bounded (kWaitLimitNs); on expiry the kernel sets
 // NV4_FLAG_TIMEOUT, every role stops, the stores are skipped, copies in flight are
 // drained and the tensor memory is released.
@@ -54,7 +56,7 @@ constexpr int kBM = 128;
 constexpr int kBK = 256;                          // FP4 elements per stage (128 bytes per row)
 constexpr int kStages = 4;
 constexpr int kSfBufs = 4;                        // scale-factor buffers in tensor memory
-constexpr int kThreads = 320;                     // warps 0-3 epilogue, 4-7 scale writers, 8 producer, 9 MMA issuer
+constexpr int kThreads = 448;                     // warps 0-3, 10-13 epilogue, 4-7 scale writers, 8 producer, 9 MMA issuer
 constexpr int kProducer = 256, kIssuer = 288;     // the two single-thread roles
 
 // Tile width kBN = 128 or 256 (one MMA of 128 x kBN x 64 per K-step).
@@ -81,7 +83,7 @@ struct Smem {
     uint8_t b[kStages][Cfg<kBN>::kBTile];
     uint8_t sfa[kStages][Cfg<kBN>::kSfA];
     uint8_t sfb[kStages][Cfg<kBN>::kSfB];
-    uint8_t stg[4][2048];                         // per epilogue warp: 32 rows x 64 bytes, swizzled
+    uint8_t stg[8][1024];                         // per epilogue warp: 32 rows x 32 bytes, swizzled
     uint64_t full[kStages], empty[kStages], sf_full[kSfBufs], sf_free[kSfBufs], acc_full, acc_empty, drain;
     uint32_t tmem_base;
     uint32_t abort;                               // set by a wait that gave up
@@ -219,7 +221,7 @@ gemm_nvfp4_kernel(const __grid_constant__ Params p)
             mbar_init(&sm.sf_free[b], 1);
         }
         mbar_init(&sm.acc_full, 1);
-        mbar_init(&sm.acc_empty, 4);                               // one arrival per epilogue warp
+        mbar_init(&sm.acc_empty, 8);                               // one arrival per epilogue warp
         mbar_init(&sm.drain, 1);
         sm.abort = 0u;
         sm.issued = sm.consumed = 0u;
@@ -302,7 +304,7 @@ gemm_nvfp4_kernel(const __grid_constant__ Params p)
             if (!mbar_wait(&sm.drain, 0u)) flags |= kFlagTimeout;
         }
         __syncwarp();
-    } else if (warp >= 4) {
+    } else if (warp >= 4 && warp < 8) {
         // ---- scale writers, warps 4-7 (tensor-memory sub-partition q = warp % 4, lanes
         // 32q..32q+31).  The block-scaled MMA reads the scale factors of a K-step from the
         // lanes of every sub-partition: row r of a 512-byte atom (32 rows x 16 bytes, rows r,
@@ -350,8 +352,16 @@ gemm_nvfp4_kernel(const __grid_constant__ Params p)
         }
         __syncwarp();
     } else {
-        // ---- epilogue warps 0-3: accumulator lanes 32w..32w+31, one output row per thread
+        // ---- epilogue warps 0-3 and 10-13: warp w reads accumulator lanes 32q..32q+31
+        // (q = w % 4, one output row per thread), columns [h * kBN/2, (h + 1) * kBN/2) with
+        // h = (w >= 10).  BF16: the half row is converted into registers, the accumulator is
+        // released, and only then stored (overlapping the next tile's MMAs), each 32 x 16
+        // block transposed through the warp's 1 KB of shared memory so that a store
+        // instruction writes 16 rows x 32 contiguous bytes.  FP32: stored as read.
+        const uint32_t q = (uint32_t)warp & 3u, h = warp >= 10 ? 1u : 0u;
+        uint8_t* st = sm.stg[q + 4u * h];
         const float alpha = __fmul_rn(*p.d_s2a, *p.d_s2b);
+        constexpr int kChunks = kBN / 64;                          // 32-column chunks per warp
         uint32_t i = 0;
         for (uint32_t t = blockIdx.x; t < p.tiles; t += gridDim.x, ++i) {
             const bool ok = !aborted() && mbar_wait(&sm.acc_full, i & 1u);
@@ -362,47 +372,59 @@ gemm_nvfp4_kernel(const __grid_constant__ Params p)
             tc_fence_after();
             __syncwarp();
             const uint32_t n_tile = t % p.n_tiles, m_tile = t / p.n_tiles;
-            const int64_t row = (int64_t)m_tile * kBM + 32 * warp + lane;
+            const int64_t row0 = (int64_t)m_tile * kBM + 32 * q;  // this warp's first row
+            const int64_t col0 = (int64_t)n_tile * kBN + (int64_t)h * (kBN / 2);
+            const uint32_t taddr = tmem + ((32u * q) << 16) + h * (uint32_t)(kBN / 2);
+            if constexpr (kOut == 2) {
 #pragma unroll 1
-            for (int cb = 0; cb < kBN / 32; ++cb) {
-                float v[32];
-                tmem_ld32(tmem + ((uint32_t)(32 * warp) << 16) + (uint32_t)(32 * cb), v);
-                const int64_t col = (int64_t)n_tile * kBN + 32 * cb;
-                if constexpr (kOut == 2) {
-                    float4* o = reinterpret_cast<float4*>(static_cast<float*>(p.out) + row * p.ldd + col);
+                for (int cb = 0; cb < kChunks; ++cb) {
+                    float v[32];
+                    tmem_ld32(taddr + (uint32_t)(32 * cb), v);
+                    float4* o = reinterpret_cast<float4*>(static_cast<float*>(p.out) + (row0 + lane) * p.ldd + col0 + 32 * cb);
 #pragma unroll
                     for (int k = 0; k < 8; ++k)
                         o[k] = make_float4(__fmul_rn(v[4 * k], alpha), __fmul_rn(v[4 * k + 1], alpha),
                                            __fmul_rn(v[4 * k + 2], alpha), __fmul_rn(v[4 * k + 3], alpha));
-                } else {
-                    uint32_t w[16];
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sm.acc_empty);
+            } else {
+                uint32_t w[16 * kChunks];
+#pragma unroll
+                for (int cb = 0; cb < kChunks; ++cb) {
+                    float v[32];
+                    tmem_ld32(taddr + (uint32_t)(32 * cb), v);
 #pragma unroll
                     for (int k = 0; k < 16; ++k)
                         asm("cvt.rn.bf16x2.f32 %0, %1, %2;"
-                            : "=r"(w[k])
+                            : "=r"(w[16 * cb + k])
                             : "f"(__fmul_rn(v[2 * k + 1], alpha)), "f"(__fmul_rn(v[2 * k], alpha)));
-                    // transpose through the warp's staging rows: written one row per thread,
-                    // read back as 8 rows x 64 bytes per instruction (16-byte piece p of row r
-                    // at r * 64 + 16 * (p ^ (r & 3)): conflict-free both ways)
-                    uint8_t* st = sm.stg[warp];
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sm.acc_empty);         // the accumulator is free
+                // 16-byte piece p of staged row r at r * 32 + 16 * (p ^ ((r >> 2) & 1)):
+                // conflict-free for the row-per-thread writes and the 16-rows-per-instruction reads
+                const int pr = lane >> 1, pc = lane & 1;
 #pragma unroll
-                    for (int k = 0; k < 4; ++k)
-                        *reinterpret_cast<uint4*>(st + 64 * lane + 16 * (k ^ (lane & 3))) =
-                            make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+                for (int c16 = 0; c16 < 2 * kChunks; ++c16) {
+#pragma unroll
+                    for (int k = 0; k < 2; ++k)
+                        *reinterpret_cast<uint4*>(st + 32 * lane + 16 * (k ^ ((lane >> 2) & 1))) =
+                            make_uint4(w[8 * c16 + 4 * k], w[8 * c16 + 4 * k + 1], w[8 * c16 + 4 * k + 2],
+                                       w[8 * c16 + 4 * k + 3]);
                     __syncwarp();
-                    const int pr = lane >> 2, pc = lane & 3;
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        const int rr = pr + 8 * k;
-                        const uint4 x = *reinterpret_cast<const uint4*>(st + 64 * rr + 16 * (pc ^ (rr & 3)));
-                        *reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + (row - lane + rr) * p.ldd + col + 8 * pc) = x;
+                    for (int k = 0; k < 2; ++k) {
+                        const int rr = pr + 16 * k;
+                        const uint4 x = *reinterpret_cast<const uint4*>(st + 32 * rr + 16 * (pc ^ ((rr >> 2) & 1)));
+                        *reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + (row0 + rr) * p.ldd + col0 + 16 * c16 +
+                                                  8 * pc) = x;
                     }
                     __syncwarp();
                 }
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.acc_empty);             // this warp has read the accumulator
         }
     }
 

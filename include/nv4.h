@@ -260,12 +260,14 @@ NV4_API nv4_status nv4_hessian_accum_batched(const nv4_hessian_job* jobs, int n_
  *            or NULL -- a near-tie diagnostic.
  * Accuracy: the winner is the exact argmin except where the two best costs lie within
  * 1e-5 relative of each other.  Costs are evaluated in FP32 where the block column's
- * Hessian bounds their error well enough for that (Gershgorin ratio rho >= ~0.6: error
- * <= 29 * 2^-24 * (2 - rho) / rho relative); in the other columns a block whose FP32
- * runner-up is within three times that error of the winner, every block when cost1 or
- * cost2 is requested, and every block of a column without a valid bound (rho < 1/32,
- * indefinite or non-finite H_b) is searched exhaustively with FP64 costs.  cost1 and
- * cost2 are then the FP64 costs rounded to FP32.
+ * Hessian bounds their error well enough for that (error <= 29 * 2^-24 * (2 - rho) / mu
+ * relative, rho the Gershgorin ratio and mu a certified lower bound of the smallest
+ * eigenvalue of the diagonally scaled H_b; certified when <= 4e-6); in the other
+ * columns a block whose FP32 runner-up is within three times that error of the winner
+ * or ties it exactly, every block when cost1 or cost2 is requested, and every block of
+ * a column without a valid bound (mu < 1/32, error bound above 2^-12, indefinite or
+ * non-finite H_b) is searched exhaustively with FP64 costs.  cost1 and cost2 are then
+ * the FP64 costs rounded to FP32.
  * The search is exact over all 127 codes but skips the cost of candidates that a
  * lower bound proves cannot be the winner or, when cost2 is requested, the runner-up
  * (sweep.cu states the bounds): codes and q are the same with or without the cost

@@ -20,14 +20,16 @@
 //
 // Exact search order (branch and bound).  The result is the argmin over all 127
 // codes, but most candidates are ruled out by lower bounds instead of evaluated:
-//   (1) Scaled diagonal dominance.  With D = diag(H_b) > 0 and H' = D^-1/2 Hs D^-1/2
-//       (Hs the symmetric part), Gershgorin's theorem gives lambda_min(H') >= rho =
-//       1 - max_i sum_{j != i} |H'_ij|, so for every e:  e^T H_b e >= rho sum_i H_ii e_i^2.
+//   (1) Scaled eigenvalue bound.  With D = diag(H_b) > 0 and H' = D^-1/2 Hs D^-1/2 (Hs
+//       the symmetric part), every mu <= lambda_min(H') gives, for every e:
+//       e^T H_b e >= mu sum_i H_ii e_i^2.  Per block column, mu is the larger of
+//       Gershgorin's rho = 1 - max_i sum_{j != i} |H'_ij| and a value that a
+//       floating-point Cholesky factorization of H' - mu I certifies (block_bound).
 //   (2) Every grid point of scale S is at most 6S in magnitude, so |e_i| >= |w_i| - 6S,
 //       and the same holds at every smaller scale.
 //   (3) An element with |w_i| <= S/2 is at least min(|w_i|, S/2 - |w_i|) away from every
 //       grid point of every scale >= S (its nearest points there are 0 and S'/2 >= S/2),
-//       so rho * sum_i H_ii min(.)^2 bounds the cost of every candidate from S upwards.
+//       so mu * sum_i H_ii min(.)^2 bounds the cost of every candidate from S upwards.
 // The winner and the runner-up cost depend only on candidates whose cost is at most
 // the running runner-up cost; when the runner-up is not an output, only the winner
 // (ties to the lowest code) has to be found and the running best cost is the
@@ -38,24 +40,26 @@
 // the upward walk ends (long upward walks: weights whose block amax is far below the
 // tensor's, such as heavy-tailed expert weights).  The comparisons
 // keep a relative margin of 2^-10, far above the FP32 evaluation error, so skipped
-// candidates could not have changed the FP32 result either.  When rho < 1/32, or H_b
-// has a zero diagonal entry with a nonzero row, or non-finite entries, the bounds are
-// off and all 127 candidates are evaluated, in FP64 (below).
+// candidates could not have changed the FP32 result either.  When mu < 1/32, or eta_b
+// (below) exceeds 2^-12, or H_b has a zero diagonal entry with a nonzero row, or
+// non-finite entries, the bounds are off and all 127 candidates are evaluated, in FP64.
 //
 // Accuracy.  An FP32 cost differs from the exact eT H_b e by at most
 // gamma * |e|T |H_b| |e| with gamma = 29 * 2^-24 (the longest chain of roundings a term
 // goes through in quad_form, plus the roundings of e and of H_ij + H_ji), and
-// |e|T |H_b| |e| <= (2 - rho) / rho * eT H_b e by the same Gershgorin argument, so every
-// cost of block column b is exact to eta_b = gamma (2 - rho) / rho relative.  When
-// eta_b <= 4e-6 (rho >= ~0.6) the FP32 argmin is within 1e-5 of the exact minimum, the
-// tolerance of a near tie.  Otherwise the block is searched again in FP64 when its
+// |e|T |H_b| |e| <= (2 - rho) sum_i H_ii e_i^2 <= (2 - rho) / mu * eT H_b e (Gershgorin
+// for the absolute values, then bound (1)), so every cost of block column b is exact to
+// eta_b = gamma (2 - rho) / mu relative.  When eta_b <= 4e-6 the FP32 argmin is within
+// 1e-5 of the exact minimum, the tolerance of a near tie.  Otherwise the block is searched again in FP64 when its
 // FP32 runner-up lies within 3 eta_b of the winner (or the costs are outputs), and
 // without a valid bound it is searched in FP64 from the start: the FP64 costs carry
 // errors ~1e-16 |e|T |H_b| |e|, so the winner is the exact argmin outside ties closer
-// than that.  Pruning keeps its 2^-10 margin, which exceeds 4 eta_b for rho >= 1/32.
+// than that.  Pruning keeps its 2^-10 margin, at least 4 eta_b wherever the bounds are on.
 //
 // Ties: the lowest code wins among equal costs, and the runner-up is the smallest
-// cost strictly above the winner's, independent of the visiting order.  Identical
+// cost strictly above the winner's, independent of the visiting order.  In a column whose
+// FP32 costs are not certified, two codes with exactly the same FP32 cost are a near tie
+// like a runner-up within 3 eta_b: the block is searched again in FP64.  Identical
 // dequantized blocks produce identical e and therefore identical costs.
 #include "nv4_common.cuh"
 #include "nv4_internal.h"
@@ -63,8 +67,11 @@
 namespace nv4 {
 
 constexpr int kSweepThreads = 128;
-constexpr int kMaxTilesPerCta = 3;                     // a CTA sorts and searches up to 384 rows
-constexpr int kMaxRowsPerCta = kMaxTilesPerCta * kSweepThreads;
+// Row tiles of 128 per CTA (the bounds' set-up is paid once per CTA): up to 4 for BF16
+// weights (24 KB of shared memory, 7 CTAs per SM), 3 for FP32 (the staged blocks are
+// twice as large)
+template <int kDt> constexpr int kMaxTilesPerCta = kDt == 0 ? 4 : 3;
+template <int kDt> constexpr int kMaxRowsPerCta = kMaxTilesPerCta<kDt> * kSweepThreads;
 constexpr float kPruneScale = 1.0f - 0x1p-10f;   // bound * this must exceed the runner-up
 
 struct SweepJobDev {
@@ -134,12 +141,63 @@ __device__ __forceinline__ float quad_form(const float2 e[8], const float4* __re
     return acc.x + acc.y;
 }
 
-// rho * H_ii for the lower bound (1), or all zero with *ok = false when the bound
-// is not valid for this H_b (or rho < 1/32, where it would prune nothing).  Run by one
-// full warp, lane i < 16 owning channel i.  FP32 with explicit safety margins: rsqrtf
-// is within 2 ulp and the 15-term sum of positive products within 2^-19 relative, so
-// r * (1 + 2^-16) + 2^-16 bounds the exact Gershgorin radius from above.  *eta receives
-// the relative error bound of this column's FP32 costs (+inf without a bound).
+// The scaled symmetric part M = D^-1/2 Hs D^-1/2 of H_b, row lane % 16 (both 16-lane
+// halves of the warp hold the matrix; s_i = RN(1 / sqrt(H_ii)), 0 for a zero diagonal,
+// whose row is then a unit row): m_ij = 0.5 (H_ij + H_ji) s_i s_j in FP32, at most 5
+// roundings (3e-7 relative) from the exact value.
+__device__ __forceinline__ float scaled_entry(const float* __restrict__ hs, float si, int j)
+{
+    const int i = threadIdx.x & 15;
+    const float sj = __shfl_sync(0xffffffffu, si, j, 16);
+    const float h = 0.5f * (hs[16 * i + j] + hs[16 * j + i]);
+    return j == i ? 1.0f : __fmul_rn(__fmul_rn(h, si), sj);
+}
+
+// Whether M - (mu + 2^-13) I is positive definite, each 16-lane half of the warp testing
+// its own mu: an FP32 Cholesky factorization (outer-product form), each column scaled by
+// rsqrtf of its pivot (within 2 ulp).  If it completes with positive pivots,
+// lambda_min(M) >= mu: the factorization's backward error is at most (gamma_17 + 3 *
+// 2^-22) |L||L|^T, whose 2-norm is at most its trace, the trace of the factored matrix
+// (< 16), so below 3e-5 (Rump's criterion for floating-point Cholesky); the rounding of
+// the scaled entries (16 per row, < 1 each) adds less than 5e-6: both far below the
+// 2^-13 (1.2e-4) shift.  Pivots below 2^-60 count as failures.  No early exit: both
+// halves run all 16 steps (a failed half computes on, its result discarded), so every
+// shuffle is executed by the whole warp.
+__device__ __noinline__ bool chol_test(const float* __restrict__ hs, float si, float mu)
+{
+    const int ll = threadIdx.x & 15;
+    const float d = __fadd_rn(mu, 0x1p-13f);
+    float a[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) a[j] = scaled_entry(hs, si, j) - (j == ll ? d : 0.0f);
+    bool ok = true;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+        const float piv = __shfl_sync(0xffffffffu, a[k], k, 16);
+        ok = ok && piv >= 0x1p-60f;                            // smaller pivots count as failures
+        const float l = ll > k ? a[k] * rsqrtf(fmaxf(piv, 0x1p-60f)) : 0.0f;
+#pragma unroll
+        for (int j = k + 1; j < 16; ++j) a[j] = fmaf(-l, __shfl_sync(0xffffffffu, l, j, 16), a[j]);
+    }
+    return ok;
+}
+
+// mu * H_ii for the lower bounds (1)-(3), or all zero with *ok = false when no bound is
+// valid for this H_b.  Run by one full warp, lane i < 16 owning channel i.
+//   Gershgorin: rho = 1 - max_i sum_{j != i} |H'_ij| (H' the scaled symmetric part), in
+//   FP32 with explicit safety margins: rsqrtf is within 2 ulp and the 15-term sum of
+//   positive products within 2^-19 relative, so r * (1 + 2^-16) + 2^-16 bounds the exact
+//   radius from above.  Always a lower bound of lambda_min(H'), often a loose one.
+//   Certified lambda_min: one trisection of [max(rho, 0), 1 - max |m_ij|] (the upper end
+//   is the smaller eigenvalue of a 2 x 2 principal minor), the two halves of the warp
+//   testing the two inner points with chol_test at once; a test that succeeds proves its
+//   mu (on the bench's Hessians lambda_min is 1.2 to 1.35 x rho, and the larger factor
+//   prunes more candidates in all three bounds; a second trisection round, or the
+//   bisection with four sequential tests, cost more in the CTA's prologue than they save).
+// mu = the larger of the two; the bounds are used when mu >= 1/32 and the FP32 cost error
+// bound eta = gamma * (2 - rho) / mu (|e|T |H_b| |e| <= (1 + r) sum_i H_ii e_i^2 <=
+// (2 - rho) / mu * eT H_b e) is at most 2^-12, below the pruning margin 2^-10.  *eta
+// receives that relative error bound of this column's FP32 costs (+inf without a bound).
 constexpr float kCostGamma = 29.0f * 0x1p-24f;     // roundings per term of quad_form, plus e and H_ij + H_ji
 constexpr float kCertifiedEta = 4e-6f;             // FP32 argmin within 1e-5 of the exact minimum
 __device__ void block_bound(const float* __restrict__ hs, float* rd, int* ok, float* eta)
@@ -162,11 +220,36 @@ __device__ void block_bound(const float* __restrict__ hs, float* rd, int* ok, fl
     for (int o = 8; o > 0; o >>= 1) r = fmaxf(r, __shfl_xor_sync(0xffffffffu, r, o));
     bad = __any_sync(0xffffffffu, bad || !(r <= 3.0e38f));
     const float rho = 1.0f - fmaf(r, 1.0f + 0x1p-16f, 0x1p-16f);
-    const bool good = !bad && rho >= 0x1p-5f;
-    if (lane < 16) rd[lane] = good ? __fmul_rd(rho, di) : 0.0f;
+    float mu = rho;
+    if (!bad) {
+        const float si = di > 0.0f ? __frsqrt_rn(di) : 0.0f;
+        float mmax = 0.0f;                                   // max |m_ij|, i != j
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            const float mij = scaled_entry(hs, si, j);       // every lane: it shuffles
+            if (j != i) mmax = fabsf(mij) < 1.0f ? fmaxf(mmax, fabsf(mij)) : 2.0f;   // also NaN
+        }
+        for (int o = 16; o > 0; o >>= 1) mmax = fmaxf(mmax, __shfl_xor_sync(0xffffffffu, mmax, o));
+        if (mmax < 1.0f) {                                   // warp-uniform; else lambda_min <= 0
+            float lo = fmaxf(rho, 0.0f), hi = 1.0f - mmax;
+#pragma unroll 1
+            for (int round = 0; round < 1 && lo < hi; ++round) {
+                const float t1 = fmaf(hi - lo, 1.0f / 3.0f, lo), t2 = fmaf(hi - lo, 2.0f / 3.0f, lo);
+                const bool okh = chol_test(hs, si, lane < 16 ? t1 : t2);
+                const bool ok1 = __shfl_sync(0xffffffffu, okh, 0), ok2 = __shfl_sync(0xffffffffu, okh, 16);
+                if (ok2) lo = t2;
+                else if (ok1) { lo = t1; hi = t2; }
+                else hi = t1;
+            }
+            mu = fmaxf(rho, lo);
+        }
+    }
+    const float gam = __fdiv_ru(__fmul_ru(kCostGamma, 2.0f - rho), mu);
+    const bool good = !bad && mu >= 0x1p-5f && gam <= 0x1p-12f;
+    if (lane < 16) rd[lane] = good ? __fmul_rd(mu, di) : 0.0f;
     if (lane == 0) {
         *ok = good ? 1 : 0;
-        *eta = good ? __fdiv_ru(__fmul_ru(kCostGamma, 2.0f - rho), rho) : __int_as_float(0x7F800000);
+        *eta = good ? gam : __int_as_float(0x7F800000);
     }
 }
 
@@ -207,7 +290,7 @@ __device__ __forceinline__ void decode8h(uint32_t c, float2 v[4])
     for (int j = 0; j < 4; ++j) f16x2_to_f32(h[j], v[j].x, v[j].y);
 }
 
-// Lower bound (1) over 8 elements: sum_i rd_i e_i^2 (rd4: their rho * H_ii).
+// Lower bound (1) over 8 elements: sum_i rd_i e_i^2 (rd4: their mu * H_ii).
 __device__ __forceinline__ float bound_half(const float2 e[4], const float4* __restrict__ rd4)
 {
     float2 acc = make_float2(0.0f, 0.0f);
@@ -377,14 +460,15 @@ sweep_kernel(const __grid_constant__ SweepParams p)
     __shared__ float4 rd4[4];
     __shared__ int bound_ok;
     __shared__ float eta_s;
+    static_assert(kMaxRowsPerCta<kDt> <= 512, "the FP64 search list shares the sort's 1 KB");
     __shared__ uint32_t sortbuf[256];                         // bucket counts and bases of the sort,
     uint32_t* const hist = sortbuf;                           // then the list of rows left to the
-    uint32_t* const base = sortbuf + 128;                     // FP64 search (384 slots, 768 bytes)
+    uint32_t* const base = sortbuf + 128;                     // FP64 search (one 16-bit slot per row)
     uint16_t* const redo_list = reinterpret_cast<uint16_t*>(sortbuf);
     __shared__ uint32_t n_redo;
-    __shared__ uint4 sw[kMaxRowsPerCta][kDt == 0 ? 2 : 4];  // the group's weight blocks (BF16 or FP32 bits), load order
-    __shared__ uint32_t srow[kMaxRowsPerCta];                 // their rows (kNoRow past the end)
-    __shared__ uint16_t perm[kMaxRowsPerCta];                 // sorted position -> load slot
+    __shared__ uint4 sw[kMaxRowsPerCta<kDt>][kDt == 0 ? 2 : 4];  // the group's weight blocks (BF16 or FP32 bits), load order
+    __shared__ uint32_t srow[kMaxRowsPerCta<kDt>];                 // their rows (kNoRow past the end)
+    __shared__ uint16_t perm[kMaxRowsPerCta<kDt>];                 // sorted position -> load slot
 
     // locate job and tile group
     int j = 0;
@@ -424,9 +508,8 @@ sweep_kernel(const __grid_constant__ SweepParams p)
     for (int k = threadIdx.x; k < 256; k += kSweepThreads) hs[k] = job.H[(int64_t)b * 256 + k];
     __syncthreads();
     build_hpairs(hs, hp);
+    // warp 3 computes the bounds while the others load their rows (read after the next barrier)
     if (threadIdx.x >= 96) block_bound(hs, reinterpret_cast<float*>(rd4), &bound_ok, &eta_s);
-    __syncthreads();
-    const bool pr = bound_ok != 0;
     const float k6 = __frcp_rn(__fmul_rn(6.0f, s2));            // ~ 1/(6 s2), for the starting code
     const float* rd = reinterpret_cast<const float*>(rd4);
     const uint32_t s2flag = isfinite(s2) ? 0u : kFlagOverflow;
@@ -435,9 +518,9 @@ sweep_kernel(const __grid_constant__ SweepParams p)
     // ---- load the group's rows (up to 4 tiles of 128), counting-sort them by starting code
     const uint32_t tile0 = group * p.tiles_per_cta;
     const uint32_t ntile = min(job.row_tiles - tile0, p.tiles_per_cta);
-    uint32_t keys[kMaxTilesPerCta], ranks[kMaxTilesPerCta];
+    uint32_t keys[kMaxTilesPerCta<kDt>], ranks[kMaxTilesPerCta<kDt>];
 #pragma unroll
-    for (uint32_t k = 0; k < kMaxTilesPerCta; ++k) {
+    for (uint32_t k = 0; k < kMaxTilesPerCta<kDt>; ++k) {
         if (k >= ntile) break;
         const uint32_t slot = k * kSweepThreads + threadIdx.x;
         uint32_t row = (tile0 + k) * kSweepThreads + threadIdx.x;
@@ -492,7 +575,7 @@ sweep_kernel(const __grid_constant__ SweepParams p)
     }
     __syncthreads();
 #pragma unroll
-    for (uint32_t k = 0; k < kMaxTilesPerCta; ++k) {
+    for (uint32_t k = 0; k < kMaxTilesPerCta<kDt>; ++k) {
         if (k >= ntile) break;
         perm[base[keys[k]] + ranks[k]] = (uint16_t)(k * kSweepThreads + threadIdx.x);
     }
@@ -501,6 +584,7 @@ sweep_kernel(const __grid_constant__ SweepParams p)
     __syncthreads();
 
     // ---- each warp walks interleaved groups of 32 sorted rows, without further barriers
+    const bool pr = bound_ok != 0;                           // written by warp 3 before the barriers above
     const uint32_t nslots = ntile * kSweepThreads;
     const uint32_t warp = threadIdx.x >> 5, lane = threadIdx.x & 31u;
 #pragma unroll 1
@@ -527,12 +611,13 @@ sweep_kernel(const __grid_constant__ SweepParams p)
         const bool need2 = job.cost2 != nullptr;
         float best = __int_as_float(0x7F800000), second = best, thr = best;
         uint32_t best_c = 0u;
-        bool redo = false;
+        bool redo = false, tie = false;   // tie: another code reached exactly the best FP32 cost
         if (a1 == 0.0f) {
             best = 0.0f;                  // all-zero block: every candidate has e = w = 0
-        } else if (!pr) {                 // no valid bound: all 127 candidates, in FP64
-            redo = true;
-        } else {
+        } else if (!pr || ((job.cost1 != nullptr || job.cost2 != nullptr) &&
+                           *reinterpret_cast<volatile float*>(&eta_s) > kCertifiedEta)) {
+            redo = true;                  // no valid bound, or costs that FP32 cannot certify:
+        } else {                          // all 127 candidates, in FP64
             const float t0 = __fmul_rn(a1, k6);
             int c = (int)min(cvt_e4m3x2(t0, t0) & 0x7Fu, 126u);
             int dn = c - 1, up = c + 1;
@@ -571,10 +656,12 @@ sweep_kernel(const __grid_constant__ SweepParams p)
                         ++nfull;
                         const float cost = quad_form(e, hp);
                         if (cost < best || (cost == best && (uint32_t)c < best_c)) {
-                            if (cost < best) second = best;
+                            if (cost < best) { second = best; tie = false; } else tie = true;
                             best = cost;
                             best_c = (uint32_t)c;
-                        } else if (cost > best && cost < second) {
+                        } else if (cost == best) {
+                            tie = true;
+                        } else if (cost < second) {
                             second = cost;
                         }
                         thr = need2 ? second : best;
@@ -619,8 +706,8 @@ sweep_kernel(const __grid_constant__ SweepParams p)
             // costs that are outputs) needs the FP64 search unless eta certifies the argmin
             // (eta and the cost outputs are read here, not held through the walk)
             const float eta = *reinterpret_cast<volatile float*>(&eta_s);
-            redo = eta > kCertifiedEta &&
-                   (job.cost1 != nullptr || job.cost2 != nullptr || !(second > fmaf(best, 3.0f * eta, best)));
+            redo = eta > kCertifiedEta && (job.cost1 != nullptr || job.cost2 != nullptr || tie ||
+                                           !(second > fmaf(best, 3.0f * eta, best)));
         }
         if (redo) {                       // decided later by the FP64 search of a whole warp
             flag_or(p.d_flags, flags);
@@ -681,7 +768,8 @@ cudaError_t launch_sweep(const nv4_sweep_job* jobs, int n, int dt, uint32_t* d_f
     uint64_t tiles = 0;
     for (int i = 0; i < m; ++i) tiles += (uint64_t)p.jobs[i].row_tiles * p.jobs[i].nblk;
     const uint64_t per = tiles / ((uint64_t)num_sms() * 16u);
-    p.tiles_per_cta = (uint32_t)(per < 1 ? 1 : (per > (uint64_t)kMaxTilesPerCta ? kMaxTilesPerCta : per));
+    const uint64_t cap = (uint64_t)(dt == 0 ? kMaxTilesPerCta<0> : kMaxTilesPerCta<2>);
+    p.tiles_per_cta = (uint32_t)(per < 1 ? 1 : (per > cap ? cap : per));
     for (int i = 0; i < m; ++i) {
         SweepJobDev& d = p.jobs[i];
         d.cta_begin = ctas;

@@ -575,7 +575,9 @@ def test_sweep_small_positive_rho(orc):
     below rho ~ 0.6.  Blocks whose FP32 runner-up is that close to the winner (and every
     block when the costs are outputs) are searched again in FP64; the plain parity rule
     holds on every column, in both modes (codes + nibbles alone, and with the costs).
-    At rho = 0.02 (below 1/32) the bounds are off and the column is searched in FP64."""
+    At rho = 0.02 (below 1/32) Gershgorin alone would switch the bounds off; the certified
+    lambda_min keeps them on, with FP32 costs whose error bound is not certified, so near
+    ties and exact FP32 ties between two codes go to the FP64 search."""
     rng = np.random.default_rng(81)
     H = _gershgorin_hessians(rng, [0.02, 0.05, 0.1, 0.3, 0.55, 0.9])
     w = (rng.standard_normal((2048, 96)) * 0.02).astype(np.float32)
@@ -639,20 +641,30 @@ def test_sweep_grouped_scale2(orc):
 
 
 def test_sweep_work_counter(orc):
-    """Bounds on: far fewer than 127 costs per block; bounds off (correlated channels):
-    every candidate visited (both halves) and evaluated; the winners match the oracle
-    either way."""
+    """Bounds on: far fewer than 127 costs per block, both for independent channels and
+    for correlated ones (Gershgorin's rho < 0, but lambda_min of the scaled H_b well above
+    1/32, which the Cholesky certificate proves); bounds off (a duplicated channel: H_b
+    singular): every candidate visited (both halves) and evaluated.  The winners match the
+    oracle either way."""
     rng = np.random.default_rng(78)
-    x = rng.laplace(size=(2048, 32))
-    x[:, 16:] = x[:, 16:17] + rng.standard_normal((2048, 16))       # correlated channels: rho < 0
+    x = rng.laplace(size=(2048, 48))
+    x[:, 16:48] = x[:, 16:17] + rng.standard_normal((2048, 32))     # correlated channels
+    x[:, 33] = x[:, 32]                                              # H_2 singular
     xb = inputs.f32_to_bf16_bits(x.astype(np.float32))
     H = orc.hessian_accum(xb)
-    w = (rng.standard_normal((256, 32)) * 0.02).astype(np.float32)
+    for b in range(3):                                               # what the three columns exercise
+        Hs = H[b].astype(np.float32).astype(np.float64)
+        dm = 1.0 / np.sqrt(np.diag(Hs))
+        M = dm[:, None] * Hs * dm[None, :]
+        rho = 1.0 - (np.abs(M).sum(1) - 1.0).max()
+        lmin = np.linalg.eigvalsh(M)[0]
+        assert (rho > 0.1, rho < 0 and lmin > 0.1, rho < 0 and abs(lmin) < 1e-6)[b], (b, rho, lmin)
+    w = (rng.standard_normal((256, 48)) * 0.02).astype(np.float32)
     wd = G.f32_dev(w)
     rows, cols = w.shape
     work = []
     jobs = []
-    for b in range(2):
+    for b in range(3):
         wb = wd[:, 16 * b:16 * b + 16].contiguous()
         Hb = G.f32_dev(H[b:b + 1].astype(np.float32))
         work.append(torch.zeros(2, dtype=torch.int64, device=G.DEV))
@@ -666,19 +678,26 @@ def test_sweep_work_counter(orc):
     torch.cuda.synchronize()
     assert f.item() == 0
     # codes only (no runner-up): pruning against the best cost, fewer costs, same winners
-    lean = torch.zeros(2, dtype=torch.int64, device=G.DEV)
-    j0 = dict(jobs[0], cost1=None, cost2=None, d_work=lean,
-              codes=torch.empty_like(jobs[0]["codes"]), q=torch.empty_like(jobs[0]["q"]))
-    nv4.nv4_scale_sweep_batched([j0], f)
-    torch.cuda.synchronize()
-    assert torch.equal(j0["codes"], jobs[0]["codes"]) and torch.equal(j0["q"], jobs[0]["q"])
-    on, off, ln = work[0].cpu().numpy(), work[1].cpu().numpy(), lean.cpu().numpy()
-    print("work with bounds", on, "without", off, "codes only", ln)
+    lean = [torch.zeros(2, dtype=torch.int64, device=G.DEV) for _ in range(2)]
+    for b in range(2):
+        jb = dict(jobs[b], cost1=None, cost2=None, d_work=lean[b],
+                  codes=torch.empty_like(jobs[b]["codes"]), q=torch.empty_like(jobs[b]["q"]))
+        nv4.nv4_scale_sweep_batched([jb], f)
+        torch.cuda.synchronize()
+        assert torch.equal(jb["codes"], jobs[b]["codes"]) and torch.equal(jb["q"], jobs[b]["q"])
+    on, corr, off = (w_.cpu().numpy() for w_ in work)
+    ln, ln_corr = (w_.cpu().numpy() for w_ in lean)
+    print("work with bounds", on, "correlated", corr, "without", off, "codes only", ln, ln_corr)
     assert ln[1] <= on[1] and ln[0] <= on[0]
     # bounds off: both halves of every candidate and every cost; on: a candidate's second
-    # half only when its first half leaves it open, a cost only when its whole bound does
+    # half only when its first half leaves it open, a cost only when its whole bound does.
+    # The correlated column's FP32 costs are not certified (eta_b > 4e-6): with the costs
+    # as outputs every block is searched in FP64; for codes alone the walk prunes, and
+    # only near ties go to FP64.
     assert off[0] == 2 * 127 * rows and off[1] == 127 * rows
-    assert on[1] <= on[0] / 2 <= on[0] <= 2 * 127 * rows and on[1] < 0.25 * 127 * rows
+    assert corr[0] == 2 * 127 * rows and corr[1] == 127 * rows
+    for v in (on, ln_corr):
+        assert v[1] <= v[0] / 2 <= v[0] <= 2 * 127 * rows and v[1] < 0.25 * 127 * rows
     ref = orc.scale_sweep(w, H.astype(np.float32).astype(np.float64), orc.tensor_amax(w)[0])
     cat = lambda k: np.concatenate([G.host(j[k]) for j in jobs], axis=1)
     st = G.sweep_parity(cat("codes"), cat("q"), cat("cost1"), ref, c2_gpu=cat("cost2"))

@@ -587,6 +587,45 @@ def test_sweep_small_positive_rho(orc):
     print("small rho", st)
 
 
+def _eigen_hessians(rng, lmins, tokens=8192):
+    """Block columns whose diagonally scaled matrix has about a given smallest eigenvalue:
+    M = Q diag(lambda) Q^T with a random orthogonal Q, lambda_min given and the rest in
+    [lambda_min, 2 - lambda_min], rescaled to a unit diagonal (which keeps M positive
+    definite but moves its eigenvalues, so lambda_min is measured, not assumed), then
+    H_b = S M S with channel scales S over two binades."""
+    blocks, lams = [], []
+    for lm in lmins:
+        q, _ = np.linalg.qr(rng.standard_normal((16, 16)))
+        lam = np.concatenate([[lm], rng.uniform(lm, 2.0 - lm, 15)])
+        m = (q * lam) @ q.T
+        dm = 1.0 / np.sqrt(np.diag(m))
+        m = dm[:, None] * m * dm[None, :]
+        s = np.sqrt(tokens * 4.0 ** rng.uniform(-1, 1, 16))
+        blocks.append(s[:, None] * m * s[None, :])
+        lams.append(np.linalg.eigvalsh(m)[0])
+    return np.stack(blocks), np.array(lams)
+
+
+def test_sweep_certified_lambda_min(orc):
+    """Block columns with lambda_min of the scaled H_b from ~0.03 to ~0.95 and Gershgorin
+    ratios below it (half of them negative): the bounds run on the Cholesky-certified
+    lambda_min.  A certificate above the true lambda_min would let the bounds prune
+    winners; the plain parity rule and the agreement of both modes, on FP32 and BF16
+    weights with outlier elements, show that none was lost."""
+    rng = np.random.default_rng(83)
+    H, lams = _eigen_hessians(rng, [0.03, 0.06, 0.12, 0.25, 0.5, 0.7, 0.85, 0.95])
+    dm = 1.0 / np.sqrt(np.einsum("bii->bi", H))
+    M = dm[:, :, None] * H * dm[:, None, :]
+    rho = 1.0 - (np.abs(M).sum(2) - 1.0).max(1)
+    assert (rho < lams).all() and (rho < 0).sum() >= 4 and lams.min() < 0.05 and lams.max() > 0.9, (rho, lams)
+    w = (rng.standard_normal((1024, 128)) * 0.02).astype(np.float32)
+    w[::7, 3] *= 30.0
+    w[1::11, 77] *= 60.0
+    st = _sweep_check(orc, w, H)
+    st_b = _sweep_check(orc, inputs.f32_to_bf16_bits(w), H)
+    print("certified lambda_min", lams.round(3), "rho", rho.round(2), st, st_b)
+
+
 def test_sweep_c1_chain_on_device(orc):
     """The tiny Linear's calibration chain with every step on the GPU -- weight amax,
     local Hessian of the activations, sweep with pack ([CAL] section 2 steps 1-3) --

@@ -303,26 +303,6 @@ __device__ __forceinline__ float bound_half(const float2 e[4], const float4* __r
     return acc.x + acc.y;
 }
 
-template <int kDt>
-__device__ __forceinline__ void load_block(const SweepJobDev& job, uint32_t row, uint32_t b, float2 w[8])
-{
-    if constexpr (kDt == 0) {
-        const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(job.w) + (int64_t)row * job.ld + 16 * b);
-        const uint4 v0 = __ldg(src), v1 = __ldg(src + 1);
-        const uint32_t u[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-#pragma unroll
-        for (int k = 0; k < 8; ++k) w[k] = make_float2(bf16_lo(u[k]), bf16_hi(u[k]));
-    } else {
-        const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(job.w) + (int64_t)row * job.ld + 16 * b);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const float4 v = __ldg(src + k);
-            w[2 * k] = make_float2(v.x, v.y);
-            w[2 * k + 1] = make_float2(v.z, v.w);
-        }
-    }
-}
-
 // Signed weights of a staged block (BF16 as its 32 bytes, FP32 as its 64).
 template <int kDt>
 __device__ __forceinline__ void unstage_block(const uint4* __restrict__ src, float2 w[8])
@@ -519,15 +499,33 @@ sweep_kernel(const __grid_constant__ SweepParams p)
     const uint32_t tile0 = group * p.tiles_per_cta;
     const uint32_t ntile = min(job.row_tiles - tile0, p.tiles_per_cta);
     uint32_t keys[kMaxTilesPerCta<kDt>], ranks[kMaxTilesPerCta<kDt>];
+    // all of this thread's loads first (one memory latency instead of one per tile), then
+    // the keys; the blocks are staged as their bits
+    constexpr int kVec = kDt == 0 ? 2 : 4;                  // 16-byte pieces per block
+    uint4 raw[kMaxTilesPerCta<kDt>][kVec];
+#pragma unroll
+    for (uint32_t k = 0; k < kMaxTilesPerCta<kDt>; ++k) {
+        const uint32_t row = (tile0 + k) * kSweepThreads + threadIdx.x;
+        const bool live = k < ntile && row < job.rows;
+        const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(job.w) +
+                                                          ((int64_t)row * job.ld + 16 * b) * (kDt == 0 ? 2 : 4));
+        if (live) {
+#pragma unroll
+            for (int j = 0; j < kVec; ++j) raw[k][j] = __ldg(src + j);
+        } else {
+#pragma unroll
+            for (int j = 0; j < kVec; ++j) raw[k][j] = make_uint4(0u, 0u, 0u, 0u);
+        }
+    }
 #pragma unroll
     for (uint32_t k = 0; k < kMaxTilesPerCta<kDt>; ++k) {
         if (k >= ntile) break;
         const uint32_t slot = k * kSweepThreads + threadIdx.x;
         uint32_t row = (tile0 + k) * kSweepThreads + threadIdx.x;
-        float2 w[8];
         uint32_t key = 127u;
         if (row < job.rows) {
-            load_block<kDt>(job, row, b, w);
+            float2 w[8];
+            unstage_block<kDt>(raw[k], w);
             float a1 = 0.0f;
 #pragma unroll
             for (int j = 0; j < 8; ++j) a1 = fmaxf(a1, fmaxf(fabsf(w[j].x), fabsf(w[j].y)));
@@ -537,22 +535,9 @@ sweep_kernel(const __grid_constant__ SweepParams p)
             }
         } else {
             row = kNoRow;
-#pragma unroll
-            for (int j = 0; j < 8; ++j) w[j] = make_float2(0.0f, 0.0f);
         }
 #pragma unroll
-        for (int j = 0; j < (kDt == 0 ? 2 : 4); ++j) {
-            if constexpr (kDt == 0) {          // the BF16 bits back from their exact FP32 values
-                uint32_t u[4];
-#pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    u[k] = (__float_as_uint(w[4 * j + k].y) & 0xFFFF0000u) | (__float_as_uint(w[4 * j + k].x) >> 16);
-                sw[slot][j] = make_uint4(u[0], u[1], u[2], u[3]);
-            } else {
-                sw[slot][j] = make_uint4(__float_as_uint(w[2 * j].x), __float_as_uint(w[2 * j].y),
-                                         __float_as_uint(w[2 * j + 1].x), __float_as_uint(w[2 * j + 1].y));
-            }
-        }
+        for (int j = 0; j < kVec; ++j) sw[slot][j] = raw[k][j];
         srow[slot] = row;
         keys[k] = key;
         ranks[k] = atomicAdd(&hist[key], 1u);

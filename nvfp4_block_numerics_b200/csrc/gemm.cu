@@ -38,6 +38,11 @@
 //     contiguous bytes instead of 32 rows x 16.
 // The accumulator is single-buffered (a second 256-column one does not fit the 512 columns
 // next to the scale buffers): the tensor pipe idles while the epilogue reads it.
+//
+// When M and N are multiples of 256 the product runs on CTA pairs instead (the kernel
+// gemm_nvfp4_pair_kernel below: 256 x 256 tiles, the 2-SM MMA): 8192^3 +2%, 16384 x 16384 x
+// 2048 +7%.  Its cross-CTA hand-offs use plain (CTA-scope) mbarrier waits and remote
+// arrives: with cluster-scope acquire/release on them the same kernel ran 40% slower.
 // Every mbarrier wait is bounded (kWaitLimitNs); on expiry the kernel sets
 // NV4_FLAG_TIMEOUT, every role stops, the stores are skipped, copies in flight are
 // drained and the tensor memory is released.
@@ -443,6 +448,315 @@ gemm_nvfp4_kernel(const __grid_constant__ Params p)
     if (lane == 0) flag_or(p.d_flags, flags);
 }
 
+// ---------------------------------------------------------------- the CTA-pair kernel
+// 256 x 256 output tiles computed by a pair of CTAs (a 2-CTA cluster) with the 2-SM MMA
+// (tcgen05.mma.cta_group::2, M = 256): CTA r of the pair holds rows 128r..128r+127 of the
+// tile's A and of its B in its own shared memory, the full N = 256 of B's scale atoms, and
+// its 128 x 256 FP32 accumulator.  The pair's MMA reads each B half once and shares it, so
+// per SM a stage moves 16 KB less B through shared memory (TMA write and MMA read) than
+// the single-CTA 128 x 256 tile does for the same work.  Roles per CTA as in the kernel
+// above (producer, scale writers, epilogue); warp 9 of rank 0 issues the pair's MMAs and
+// warp 9 of rank 1 forwards "this stage's codes have landed and its scales are written"
+// to it (a cluster-scope mbarrier arrive).  The MMA thread's commits arrive on the
+// barriers of both CTAs (tcgen05.commit ... multicast::cluster, mask 0b11); rank 1's
+// epilogue warps release the accumulator on rank 0's acc_empty.  No load is multicast.
+constexpr int kStages2 = 5;
+constexpr int kSfBufs2 = 5;                       // 256 + 5 x 48 = 496 tensor-memory columns
+
+struct Smem2 {
+    uint8_t a[kStages2][128 * 128];               // this CTA's 128 rows of A (1024-byte aligned)
+    uint8_t b[kStages2][128 * 128];               // this CTA's 128 rows of B
+    uint8_t sfa[kStages2][4 * 512];               // A scale atoms of this CTA's rows
+    uint8_t sfb[kStages2][8 * 512];               // B scale atoms of all 256 rows
+    uint8_t stg[8][1024];                         // epilogue transposes
+    uint64_t full[kStages2], empty[kStages2], peer_ready[kStages2], sf_full[kSfBufs2], sf_free[kSfBufs2];
+    uint64_t acc_full, acc_empty, drain;
+    uint32_t tmem_base;
+    uint32_t abort;
+    uint32_t issued, consumed;
+};
+
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols)
+{
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+                 "r"(ncols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols)
+{
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+__device__ __forceinline__ void mma_fp4_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                             uint32_t sfa, uint32_t sfb, uint32_t accumulate)
+{
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "setp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t"
+                 "}"
+                 ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+                 : "memory");
+}
+
+// Arrives on the barrier at bar's offset in both CTAs of the pair once every tcgen05
+// operation issued so far by this thread completes.
+__device__ __forceinline__ void tc_commit_pair(uint64_t* bar)
+{
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
+                 ::"r"(smem_u32(bar)), "h"((uint16_t)3u)
+                 : "memory");
+}
+
+template <int kOut>
+__global__ void __launch_bounds__(kThreads, 1)
+gemm_nvfp4_pair_kernel(const __grid_constant__ Params p)
+{
+    using C = Cfg<256>;
+    constexpr int kStages = kStages2;
+    constexpr uint32_t kTx = 2u * 128u * 128u + 4u * 512u + 8u * 512u;
+    // instruction descriptor: as Cfg<256>::kIdesc with M = 256 (the pair)
+    constexpr uint32_t kIdesc2 = (1u << 7) | (1u << 10) | ((uint32_t)(256 >> 3) << 17) | ((uint32_t)(256 >> 4) << 24);
+    extern __shared__ uint8_t smem_raw[];
+    Smem2& sm = *reinterpret_cast<Smem2*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t KS = p.k_stages;
+    const uint32_t rank = cluster_ctarank();
+    const uint32_t pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+
+    if (threadIdx.x == kProducer) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&sm.full[s], 1);
+            mbar_init(&sm.empty[s], 1);
+            mbar_init(&sm.peer_ready[s], 1);
+        }
+        for (int b = 0; b < kSfBufs2; ++b) {
+            mbar_init(&sm.sf_full[b], 8);                          // the writers of both CTAs
+            mbar_init(&sm.sf_free[b], 1);
+        }
+        mbar_init(&sm.acc_full, 1);
+        mbar_init(&sm.acc_empty, 16);                              // 8 epilogue warps in each CTA
+        mbar_init(&sm.drain, 1);
+        sm.abort = 0u;
+        sm.issued = sm.consumed = 0u;
+        mbar_init_fence();
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&p.map_a)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&p.map_b)) : "memory");
+    }
+    if (warp == kIssuer / 32) tmem_alloc_pair(&sm.tmem_base, C::kTmemCols);
+    tc_fence_before();
+    cluster_sync();                                                // barriers of both CTAs initialised
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+    uint32_t flags = 0u;
+    auto aborted = [&]() { return *reinterpret_cast<volatile uint32_t*>(&sm.abort) != 0u; };
+    auto give_up = [&]() { flags |= kFlagTimeout; atomicOr(&sm.abort, 1u); };
+
+    if (warp == kProducer / 32) {
+        if (lane == 0) {                                           // producer: this CTA's halves
+            uint32_t g = 0;
+            for (uint32_t t = pair; t < p.tiles && !aborted(); t += npairs) {
+                const uint32_t n_tile = t % p.n_tiles, m_tile = t / p.n_tiles;
+                const uint32_t mrow = 2u * m_tile + rank, nrow = 2u * n_tile + rank;   // 128-row tiles
+                for (uint32_t ks = 0; ks < KS; ++ks, ++g) {
+                    const uint32_t s = g % kStages;
+                    if (g >= (uint32_t)kStages && !mbar_wait(&sm.empty[s], ((g / kStages) - 1u) & 1u)) give_up();
+                    if (aborted()) break;
+                    mbar_arrive_expect_tx(&sm.full[s], kTx);
+                    tma_load_2d(sm.a[s], &p.map_a, &sm.full[s], (int)(ks * 128u), (int)(mrow * 128u));
+                    tma_load_2d(sm.b[s], &p.map_b, &sm.full[s], (int)(ks * 128u), (int)(nrow * 128u));
+                    bulk_load(sm.sfa[s], p.sfa + ((size_t)mrow * p.kt4 + 4u * ks) * 512u, 2048u, &sm.full[s]);
+#pragma unroll
+                    for (uint32_t h = 0; h < 2u; ++h)
+                        bulk_load(sm.sfb[s] + 2048u * h, p.sfb + ((size_t)(2u * n_tile + h) * p.kt4 + 4u * ks) * 512u,
+                                  2048u, &sm.full[s]);
+                }
+            }
+            sm.issued = g;
+        }
+        __syncwarp();
+    } else if (warp == kIssuer / 32) {
+        if (lane == 0 && rank == 0) {                              // the pair's MMA issuer
+            uint32_t g = 0, i = 0;
+            for (uint32_t t = pair; t < p.tiles && !aborted(); t += npairs, ++i) {
+                if (i > 0 && !mbar_wait(&sm.acc_empty, (i - 1u) & 1u)) {
+                    give_up();
+                    break;
+                }
+                tc_fence_after();
+                for (uint32_t ks = 0; ks < KS; ++ks, ++g) {
+                    const uint32_t s = g % kStages, b = g % kSfBufs2, ph = (g / kStages) & 1u;
+                    if (!mbar_wait(&sm.full[s], ph) || !mbar_wait(&sm.sf_full[b], (g / kSfBufs2) & 1u) ||
+                        !mbar_wait(&sm.peer_ready[s], ph)) {
+                        give_up();
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t ta = tmem + 256u + C::kSfCols * b, tb = ta + 16u;
+                    const uint32_t a0 = smem_u32(sm.a[s]), b0 = smem_u32(sm.b[s]);
+#pragma unroll
+                    for (uint32_t j = 0; j < 4; ++j)
+                        mma_fp4_pair(tmem, smem_desc(a0 + 32u * j, 1u, 64u, 2u), smem_desc(b0 + 32u * j, 1u, 64u, 2u),
+                                     kIdesc2, ta + 4u * j, tb + 8u * j, (ks | j) != 0u ? 1u : 0u);
+                    tc_commit_pair(&sm.empty[s]);
+                    tc_commit_pair(&sm.sf_free[b]);
+                }
+                if (aborted()) break;
+                tc_commit_pair(&sm.acc_full);
+            }
+            sm.consumed = g;
+            tc_commit_pair(&sm.drain);
+            if (!mbar_wait(&sm.drain, 0u)) flags |= kFlagTimeout;
+        } else if (lane == 0) {                                    // rank 1: forwards its landed stages
+            uint32_t g = 0;
+            for (uint32_t t = pair; t < p.tiles && !aborted(); t += npairs) {
+                for (uint32_t ks = 0; ks < KS; ++ks, ++g) {
+                    const uint32_t s = g % kStages;
+                    if (!mbar_wait(&sm.full[s], (g / kStages) & 1u)) {
+                        give_up();
+                        break;
+                    }
+                    mbar_arrive_cluster(&sm.peer_ready[s], 0u);
+                }
+            }
+            sm.consumed = g;
+        }
+        __syncwarp();
+    } else if (warp >= 4 && warp < 8) {
+        // ---- scale writers: as in the single-CTA kernel, this CTA's rows of A, all of B
+        const uint32_t lanes = (uint32_t)(32 * (warp & 3)) << 16;
+        uint32_t g = 0;
+        bool quit = false;
+        for (uint32_t t = pair; t < p.tiles && !quit; t += npairs) {
+            for (uint32_t ks = 0; ks < KS; ++ks, ++g) {
+                const uint32_t s = g % kStages, b = g % kSfBufs2;
+                bool ok = mbar_wait(&sm.full[s], (g / kStages) & 1u);
+                if (ok && g >= (uint32_t)kSfBufs2) ok = mbar_wait(&sm.sf_free[b], ((g / kSfBufs2) - 1u) & 1u);
+                const bool timed_out = __any_sync(0xFFFFFFFFu, !ok);
+                quit = timed_out || __any_sync(0xFFFFFFFFu, aborted());
+                if (quit) {
+                    if (timed_out && lane == 0) give_up();
+                    break;
+                }
+                tc_fence_after();
+                uint32_t va[16], vb[32];
+#pragma unroll
+                for (uint32_t j = 0; j < 4; ++j) {
+                    const uint4 x = *reinterpret_cast<const uint4*>(sm.sfa[s] + 512u * j + 16u * lane);
+                    va[4 * j] = x.x; va[4 * j + 1] = x.y; va[4 * j + 2] = x.z; va[4 * j + 3] = x.w;
+#pragma unroll
+                    for (uint32_t h = 0; h < 2u; ++h) {
+                        const uint4 y = *reinterpret_cast<const uint4*>(sm.sfb[s] + 2048u * h + 512u * j + 16u * lane);
+                        const uint32_t c = 8u * j + 4u * h;
+                        vb[c] = y.x; vb[c + 1] = y.y; vb[c + 2] = y.z; vb[c + 3] = y.w;
+                    }
+                }
+                const uint32_t ta = tmem + lanes + 256u + C::kSfCols * b;
+                tmem_st<16>(ta, va);
+                tmem_st<32>(ta + 16u, vb);
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {                                   // on the MMA issuer's CTA
+                    if (rank == 0) mbar_arrive(&sm.sf_full[b]);
+                    else mbar_arrive_cluster(&sm.sf_full[b], 0u);
+                }
+            }
+        }
+        __syncwarp();
+    } else {
+        // ---- epilogue warps 0-3 and 10-13, as in the single-CTA kernel; rows 128 * rank + ...
+        const uint32_t q = (uint32_t)warp & 3u, h = warp >= 10 ? 1u : 0u;
+        uint8_t* st = sm.stg[q + 4u * h];
+        const float alpha = __fmul_rn(*p.d_s2a, *p.d_s2b);
+        auto release = [&]() {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                if (rank == 0) mbar_arrive(&sm.acc_empty);
+                else mbar_arrive_cluster(&sm.acc_empty, 0u);
+            }
+        };
+        uint32_t i = 0;
+        for (uint32_t t = pair; t < p.tiles; t += npairs, ++i) {
+            const bool ok = !aborted() && mbar_wait(&sm.acc_full, i & 1u);
+            if (!ok) {
+                if (!aborted()) give_up();
+                break;
+            }
+            tc_fence_after();
+            __syncwarp();
+            const uint32_t n_tile = t % p.n_tiles, m_tile = t / p.n_tiles;
+            const int64_t row0 = (int64_t)m_tile * 256 + 128 * (int64_t)rank + 32 * q;
+            const int64_t col0 = (int64_t)n_tile * 256 + (int64_t)h * 128;
+            const uint32_t taddr = tmem + ((32u * q) << 16) + h * 128u;
+            if constexpr (kOut == 2) {
+#pragma unroll 1
+                for (int cb = 0; cb < 4; ++cb) {
+                    float v[32];
+                    tmem_ld32(taddr + (uint32_t)(32 * cb), v);
+                    float4* o = reinterpret_cast<float4*>(static_cast<float*>(p.out) + (row0 + lane) * p.ldd + col0 + 32 * cb);
+#pragma unroll
+                    for (int k = 0; k < 8; ++k)
+                        o[k] = make_float4(__fmul_rn(v[4 * k], alpha), __fmul_rn(v[4 * k + 1], alpha),
+                                           __fmul_rn(v[4 * k + 2], alpha), __fmul_rn(v[4 * k + 3], alpha));
+                }
+                release();
+            } else {
+                uint32_t w[64];
+#pragma unroll
+                for (int cb = 0; cb < 4; ++cb) {
+                    float v[32];
+                    tmem_ld32(taddr + (uint32_t)(32 * cb), v);
+#pragma unroll
+                    for (int k = 0; k < 16; ++k)
+                        asm("cvt.rn.bf16x2.f32 %0, %1, %2;"
+                            : "=r"(w[16 * cb + k])
+                            : "f"(__fmul_rn(v[2 * k + 1], alpha)), "f"(__fmul_rn(v[2 * k], alpha)));
+                }
+                release();
+                const int pr = lane >> 1, pc = lane & 1;
+#pragma unroll
+                for (int c16 = 0; c16 < 8; ++c16) {
+#pragma unroll
+                    for (int k = 0; k < 2; ++k)
+                        *reinterpret_cast<uint4*>(st + 32 * lane + 16 * (k ^ ((lane >> 2) & 1))) =
+                            make_uint4(w[8 * c16 + 4 * k], w[8 * c16 + 4 * k + 1], w[8 * c16 + 4 * k + 2],
+                                       w[8 * c16 + 4 * k + 3]);
+                    __syncwarp();
+#pragma unroll
+                    for (int k = 0; k < 2; ++k) {
+                        const int rr = pr + 16 * k;
+                        const uint4 x = *reinterpret_cast<const uint4*>(st + 32 * rr + 16 * (pc ^ ((rr >> 2) & 1)));
+                        *reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + (row0 + rr) * p.ldd + col0 + 16 * c16 +
+                                                  8 * pc) = x;
+                    }
+                    __syncwarp();
+                }
+            }
+        }
+    }
+
+    // ---- teardown: this CTA's loads drained, then the pair's barrier (rank 0 reaches it
+    // only after its MMAs, which read both CTAs' shared memory, have completed), then the
+    // pair's tensor memory is released
+    tc_fence_before();
+    __syncthreads();
+    if (threadIdx.x == kProducer) {
+        for (uint32_t g = sm.consumed; g < sm.issued; ++g)
+            if (!mbar_wait(&sm.full[g % kStages], (g / kStages) & 1u)) flags |= kFlagTimeout;
+    }
+    tc_fence_before();
+    cluster_sync();
+    if (warp == kIssuer / 32) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem, C::kTmemCols);
+    }
+    flags = __reduce_or_sync(0xFFFFFFFFu, flags);
+    if (lane == 0) flag_or(p.d_flags, flags);
+}
+
 // Block scales [rows, kb] (row-major, kb = K/16) -> the MMA atom layout, one thread per
 // 32-bit word (one row's 4 consecutive scales); padding rows and columns are zero.
 __global__ void __launch_bounds__(256)
@@ -516,6 +830,60 @@ cudaError_t launch_gemm_nvfp4(const uint8_t* qa, const uint8_t* sfa, const float
 {
     using namespace gemm;
     Params p;
+    static bool attr_set[6][64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const int o = out_dt == 2 ? 1 : 0;
+    if (M % 256 == 0 && N % 256 == 0) {
+        // 256 x 256 tiles on CTA pairs (2-SM MMA)
+        if (!code_map(&p.map_a, qa, M, K, 128u) || !code_map(&p.map_b, qb, N, K, 128u)) return cudaErrorInvalidValue;
+        p.sfa = sfa;
+        p.sfb = sfb;
+        p.d_s2a = d_s2a;
+        p.d_s2b = d_s2b;
+        p.out = out;
+        p.ldd = ldd;
+        p.n_tiles = (uint32_t)(N / 256);
+        p.k_stages = (uint32_t)(K / kBK);
+        p.kt4 = (uint32_t)(K / 64);
+        p.tiles = (uint32_t)((M / 256) * (N / 256));
+        p.d_flags = d_flags;
+        const size_t smem = sizeof(Smem2) + 1024;
+        auto kern = o ? gemm_nvfp4_pair_kernel<2> : gemm_nvfp4_pair_kernel<0>;
+        if (dev < 0 || dev >= 64 || !attr_set[4 + o][dev]) {
+            e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            if (e != cudaSuccess) return e;
+            if (dev >= 0 && dev < 64) attr_set[4 + o][dev] = true;
+        }
+        cudaLaunchConfig_t cfg = {};
+        cfg.blockDim = dim3(kThreads, 1, 1);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = s;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        // persistent: as many pairs as can be resident at once (once per device and output type)
+        static int resident[2][64] = {};
+        int pairs_cap = dev >= 0 && dev < 64 ? resident[o][dev] : 0;
+        if (pairs_cap <= 0) {
+            cfg.gridDim = dim3(2u * (uint32_t)(num_sms() / 2), 1, 1);
+            if (cudaOccupancyMaxActiveClusters(&pairs_cap, kern, &cfg) != cudaSuccess || pairs_cap <= 0) {
+                (void)cudaGetLastError();
+                pairs_cap = num_sms() / 2;
+            }
+            if (dev >= 0 && dev < 64) resident[o][dev] = pairs_cap;
+        }
+        const uint32_t npairs = p.tiles < (uint32_t)pairs_cap ? p.tiles : (uint32_t)pairs_cap;
+        cfg.gridDim = dim3(2u * npairs, 1, 1);
+        e = cudaLaunchKernelEx(&cfg, kern, p);
+        if (e != cudaSuccess) return e;
+        return cudaGetLastError();
+    }
     const bool wide = N % 256 == 0;
     const int bn = wide ? 256 : 128;
     if (!code_map(&p.map_a, qa, M, K, 128u) || !code_map(&p.map_b, qb, N, K, (uint32_t)bn)) return cudaErrorInvalidValue;
@@ -531,11 +899,6 @@ cudaError_t launch_gemm_nvfp4(const uint8_t* qa, const uint8_t* sfa, const float
     p.tiles = (uint32_t)((M / kBM) * (N / bn));
     p.d_flags = d_flags;
     const size_t smem = (wide ? sizeof(Smem<256>) : sizeof(Smem<128>)) + 1024;
-    static bool attr_set[4][64] = {};
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    const int o = out_dt == 2 ? 1 : 0;
     const int v = 2 * (wide ? 1 : 0) + o;
     auto kern = wide ? (o ? gemm_nvfp4_kernel<256, 2> : gemm_nvfp4_kernel<256, 0>)
                      : (o ? gemm_nvfp4_kernel<128, 2> : gemm_nvfp4_kernel<128, 0>);

@@ -106,16 +106,20 @@ def test_gemm_large(orc):
     _check(orc, qa, sa, 0.5, qb, sb, 0.25, dtypes=(torch.float32,))
 
 
-# Persistent path: the grid is min(tiles, SMs), so these shapes give every CTA several
-# output tiles.  Stage counts of 1, 2 and 3 per tile (K = 256, 512, 768) move the
-# 4-deep stage ring's phase across tile boundaries in different ways; the accumulator
-# hand-off between the epilogue and the next tile's MMAs and the teardown drain run on
-# every CTA.
+# Persistent paths: the grid is min(tiles, resident CTAs or CTA pairs), so these shapes give
+# every CTA (pair) several output tiles.  M and N multiples of 256 run the CTA-pair kernel
+# (256 x 256 tiles, 5-stage ring); other shapes the single-CTA kernel (128 x 256 tiles when
+# N allows, else 128 x 128; 4-stage ring).  Stage counts per tile of 1, 2, 3 and 5 move the
+# rings' phases across tile boundaries in different ways; the accumulator hand-off between
+# the epilogue and the next tile's MMAs and the teardown drain run on every CTA.
 @pytest.mark.parametrize("M,N,K", [
-    (4096, 4096, 512),    # 16 x 32 = 512 tiles 128 x 256, ~3.5 per CTA, 2 stages per tile
-    (4096, 3968, 512),    # 32 x 31 = 992 tiles 128 x 128 (N not a multiple of 256)
-    (4096, 4096, 256),    # 512 tiles, 1 stage per tile: the ring wraps every 4 tiles
-    (2048, 3968, 768),    # 496 tiles 128 x 128, 3 stages per tile
+    (4096, 4096, 512),    # pairs: 16 x 16 = 256 tiles 256 x 256, ~3.5 per pair, 2 stages per tile
+    (4096, 4096, 256),    # pairs: 1 stage per tile, the ring wraps every 5 tiles
+    (4096, 4096, 1280),   # pairs: 5 stages per tile, the ring's period
+    (3968, 4096, 512),    # single CTA: 31 x 16 = 496 tiles 128 x 256 (M not a multiple of 256)
+    (3968, 4096, 256),    # single CTA, 1 stage per tile: the ring wraps every 4 tiles
+    (4096, 3968, 512),    # single CTA: 32 x 31 = 992 tiles 128 x 128 (N not a multiple of 256)
+    (2048, 3968, 768),    # single CTA: 496 tiles 128 x 128, 3 stages per tile
 ])
 def test_gemm_persistent_multi_tile(orc, M, N, K):
     rng = np.random.default_rng(M + N + K)

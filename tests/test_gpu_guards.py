@@ -145,7 +145,8 @@ def test_guards_cast(rows, cols):
     assert torch.equal(nq.t, nqr) and torch.equal(ns.t, nsr)
 
 
-@pytest.mark.parametrize("M,N,K,ldd", [(128, 128, 256, 128), (256, 384, 512, 400), (384, 256, 768, 264)])
+@pytest.mark.parametrize("M,N,K,ldd", [(128, 128, 256, 128), (256, 384, 512, 400), (384, 256, 768, 264),
+                                         (256, 512, 512, 520)])   # the last: the CTA-pair kernel
 def test_guards_gemm_and_scale_layout(M, N, K, ldd):
     g = torch.Generator(device=G.DEV).manual_seed(M + N + K)
     qa = torch.randint(0, 256, (M, K // 2), dtype=torch.uint8, device=G.DEV, generator=g)

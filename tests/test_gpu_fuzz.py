@@ -228,10 +228,11 @@ def test_fuzz_two_sided_hadamard(orc, batch):
 
 @pytest.mark.parametrize("batch", range(4))
 def test_fuzz_sweep_conditioning(orc, batch):
-    """Hessian columns of random conditioning: scaled Gershgorin ratio rho from -0.5 (no
-    bound: FP64 search) through the uncertified 1/32 .. 0.6 range (FP32 walk, FP64
-    re-search near ties) to 0.95, BF16 and FP32 weights; the plain parity rule, and the
-    codes-only call equal to the full call."""
+    """Hessian columns of random conditioning: scaled Gershgorin ratio rho from -0.5 through
+    0.95.  Whether the bounds are on is decided by the certified lambda_min (at least rho):
+    columns without a bound go to the FP64 search, uncertified ones walk in FP32 with FP64
+    re-searches of near and exact ties.  BF16 and FP32 weights; the plain parity rule, and
+    the codes-only call equal to the full call."""
     r = np.random.default_rng(50000 + batch)
     rhos = r.uniform(-0.5, 0.95, 6)
     H = np.stack([_gershgorin_block(r, rho) for rho in rhos])

@@ -120,6 +120,8 @@ def test_gemm_large(orc):
     (3968, 4096, 256),    # single CTA, 1 stage per tile: the ring wraps every 4 tiles
     (4096, 3968, 512),    # single CTA: 32 x 31 = 992 tiles 128 x 128 (N not a multiple of 256)
     (2048, 3968, 768),    # single CTA: 496 tiles 128 x 128, 3 stages per tile
+    (256, 256, 256),      # pairs: a single tile, one pair of CTAs
+    (512, 768, 512),      # pairs: 2 x 3 tiles, fewer tiles than pairs
 ])
 def test_gemm_persistent_multi_tile(orc, M, N, K):
     rng = np.random.default_rng(M + N + K)

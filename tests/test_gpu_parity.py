@@ -497,6 +497,27 @@ def test_sweep_small_ragged(orc, rows, cols):
     _sweep_check(orc, inputs.f32_to_bf16_bits(w), H)
 
 
+@pytest.mark.parametrize("fp32", [False, True])
+def test_sweep_multi_tile_ctas(orc, fp32):
+    """Enough row tiles that each CTA takes several tiles of 128 rows (at most 4 for BF16
+    weights, 3 for FP32), with a ragged last group and a ragged last tile: the rows on every
+    tile boundary and every row of the last 400 (the whole last group) equal the oracle's."""
+    rows, cols = 3900, 4096                           # 31 row tiles, the last of 60 rows
+    tiles = -(-rows // 128) * (cols // 16)
+    per = min(tiles // (torch.cuda.get_device_properties(0).multi_processor_count * 16), 3 if fp32 else 4)
+    assert per >= 3 and -(-rows // 128) % per != 0   # several tiles per CTA, a short last group
+    r = np.random.default_rng(91 + fp32)
+    w = (r.standard_normal((rows, cols)) * 0.02).astype(np.float32)
+    w[:: 37, int(r.integers(0, cols))] *= 25.0
+    if not fp32:
+        w = inputs.f32_to_bf16_bits(w)
+    x = inputs.laplace_bf16(inputs.rng_for(93, "gpu", "sweepmt"), 384, cols, outlier_channels=(5, 700), outlier_scale=20)
+    H = orc.hessian_accum(x)
+    edges = [k * 128 + d for k in range(1, rows // 128 + 1) for d in (-1, 0)]
+    sample = sorted(set(e for e in edges if e < rows) | set(range(rows - 400, rows)) | {0})
+    _sweep_check(orc, w, H, rows_sample=sample)
+
+
 def test_sweep_degenerate_blocks(orc):
     w = np.zeros((4, 32), np.float32)
     w[1, :16] = 0.5

@@ -7,15 +7,19 @@
 //   mode 1: MXFP4 quantization of y (32-element blocks, E8M0 scales);
 //   mode 2: NVFP4 quantization of y with s2 = RN32(amax / 2688).
 //
-// Mapping: a lane owns 32 consecutive elements of a row (four 16-byte loads); four lanes
-// cover a 128-element segment.  The fast Walsh-Hadamard transform runs in FP64: up to
-// five butterfly stages inside a lane, then log2(n / 32) stages across lanes with
-// shuffles (n = 64, 128), so every sum is exact for BF16 inputs spanning fewer than ~38
-// binades in a block.  n is a template parameter: with static stage counts the kernel
-// needs 104 registers instead of 160 (4 CTAs per SM instead of 3), 0.63 ms instead of
-// 0.70 ms for n = 128 on a [65536, 7168] BF16 input and 0.37 ms instead of 0.49 ms for
-// n = 32.  The quantizers then work on FP32 y exactly as nv4_mxfp4_quant /
-// nv4_act_quant do; an MXFP4 block is one lane's 32 values, an NVFP4 block half of them.
+// Mapping: a lane owns 32 consecutive elements of a row (four 16-byte loads); n / 32 lanes
+// cover a segment of n elements.  The fast Walsh-Hadamard transform runs in FP64, so every
+// sum is exact for BF16 inputs spanning fewer than ~38 binades in a block: up to five
+// butterfly stages inside a lane, then log2(n / 32) stages across the segment's lanes.  For
+// n = 64 the one cross-lane stage is a shuffle and one FMA with a factor of +-1; for n = 128
+// the lanes exchange their values through shared memory, each lane takes an eighth of every
+// chunk of its segment and runs both stages in registers, and the rounded FP32 outputs go
+// back through shared memory so that the quantizers again see one chunk per lane (the
+// amax of mode 0 skips that second exchange).  On a [65536, 7168] BF16 input: n = 128
+// MXFP4 in 0.51 ms (0.63 ms with two shuffle stages of 2 shuffles and a select per value),
+// NVFP4 0.58 ms (0.68), the amax pass 0.43 ms (0.54); n = 64 MXFP4 0.43 ms (0.50), n = 32
+// 0.37 ms.  The quantizers then work on FP32 y exactly as nv4_mxfp4_quant / nv4_act_quant
+// do; an MXFP4 block is one lane's 32 values, an NVFP4 block half of them.
 #include <cmath>
 
 #include "nv4_common.cuh"
@@ -25,30 +29,20 @@ namespace nv4 {
 
 constexpr int kHadThreads = 128;
 
-// FWHT of blocks of n values, 32 consecutive values per lane: five butterfly stages
-// inside the lane, then log2(n / 32) stages across neighbouring lanes (n = 64, 128).
+// The in-lane part of the FWHT of blocks of n values, 32 consecutive values per lane: up to
+// five butterfly stages (four for n = 16).
 template <int kN>
-__device__ __forceinline__ void fwht32(double v[32], uint32_t lane)
+__device__ __forceinline__ void fwht_lane(double v[32])
 {
-    constexpr int n = kN;
 #pragma unroll
     for (int h = 1; h < 32; h <<= 1) {
-        if (h >= n) break;                            // blocks of 16: only four in-lane stages
+        if (h >= kN) break;
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
             if (i & h) continue;
             const double a = v[i], b = v[i + h];
             v[i] = a + b;
             v[i + h] = a - b;
-        }
-    }
-#pragma unroll
-    for (int d = 1; d < n / 32; d <<= 1) {
-        const bool upper = (lane & (uint32_t)d) != 0u;
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            const double o = __shfl_xor_sync(0xFFFFFFFFu, v[i], d);
-            v[i] = upper ? o - v[i] : v[i] + o;
         }
     }
 }
@@ -96,15 +90,11 @@ __device__ __forceinline__ void mx_encode(const float* y, uint32_t code, uint32_
     }
 }
 
-// NVFP4 of one 16-element block y under s2 (k_lo, k_hi: the bracket of 1/(6 s2); fast:
-// s2 inside [2^-100, 2^100]): the E4M3 block scale code (returned) and the 16 E2M1 codes
-// in w[0..1], as nv4_act_quant computes them.
-__device__ __forceinline__ uint32_t nv_block16(const float* y, float s2, float k_lo, float k_hi, bool fast,
-                                               uint32_t* w)
+// NVFP4 block scale code (E4M3, 7 bits) of a block whose largest |y| has the bit pattern bm,
+// under s2 (k_lo, k_hi: the bracket of 1/(6 s2); fast: s2 inside [2^-100, 2^100]), as
+// nv4_act_quant computes it.
+__device__ __forceinline__ uint32_t nv_block_code(uint32_t bm, float s2, float k_lo, float k_hi, bool fast)
 {
-    uint32_t bm = 0u;
-#pragma unroll
-    for (int j = 0; j < 16; ++j) bm = max(bm, __float_as_uint(y[j]) & 0x7FFFFFFFu);
     const float a_b = __uint_as_float(bm);
     uint32_t code;
     if (fast) {
@@ -114,33 +104,46 @@ __device__ __forceinline__ uint32_t nv_block16(const float* y, float s2, float k
     } else {
         code = e4m3_code_exact(a_b, s2);
     }
-    code &= 0x7Fu;
-    const float S = __fmul_rn(e4m3_value(code), s2);   // DQ1: RN32(s_b * s2)
+    return code & 0x7Fu;
+}
+
+// E2M1 codes of 8 values of a block whose dequantization scale is S = RN32(s_b * s2).
+__device__ __forceinline__ uint32_t nv_encode8(const float* yy, float S)
+{
+    uint32_t c8 = 0u;
+    if (S == 0.0f) {
 #pragma unroll
-    for (int k = 0; k < 2; ++k) {
-        const float* yy = y + 8 * k;
-        uint32_t c8 = 0u;
-        if (S == 0.0f) {
+        for (int j = 0; j < 8; ++j) c8 |= ((__float_as_uint(yy[j]) >> 28) & 8u) << (4 * j);
+    } else if (S >= kTinyScale && S <= 0x1p100f) {
+        const float rr = __frcp_rn(S);
+        const float rl = __fmul_rn(rr, kLoMargin), rh = __fmul_rn(rr, kHiMargin);
+        float lo[8], hi[8];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) c8 |= ((__float_as_uint(yy[j]) >> 28) & 8u) << (4 * j);
-        } else if (S >= kTinyScale && S <= 0x1p100f) {
-            const float rr = __frcp_rn(S);
-            const float rl = __fmul_rn(rr, kLoMargin), rh = __fmul_rn(rr, kHiMargin);
-            float lo[8], hi[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                lo[j] = __fmul_rn(yy[j], rl);
-                hi[j] = __fmul_rn(yy[j], rh);
-            }
-            c8 = cvt_e2m1x8(lo);
-            const uint32_t h8 = cvt_e2m1x8(hi);
-            if (c8 != h8) c8 = e2m1_fix8(yy, S, c8, h8);
-        } else {
-#pragma unroll
-            for (int j = 0; j < 8; ++j) c8 |= e2m1_code_exact(yy[j], S) << (4 * j);
+        for (int j = 0; j < 8; ++j) {
+            lo[j] = __fmul_rn(yy[j], rl);
+            hi[j] = __fmul_rn(yy[j], rh);
         }
-        w[k] = c8;
+        c8 = cvt_e2m1x8(lo);
+        const uint32_t h8 = cvt_e2m1x8(hi);
+        if (c8 != h8) c8 = e2m1_fix8(yy, S, c8, h8);
+    } else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) c8 |= e2m1_code_exact(yy[j], S) << (4 * j);
     }
+    return c8;
+}
+
+// NVFP4 of one 16-element block y: the scale code (returned) and the 16 E2M1 codes in w[0..1].
+__device__ __forceinline__ uint32_t nv_block16(const float* y, float s2, float k_lo, float k_hi, bool fast,
+                                               uint32_t* w)
+{
+    uint32_t bm = 0u;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) bm = max(bm, __float_as_uint(y[j]) & 0x7FFFFFFFu);
+    const uint32_t code = nv_block_code(bm, s2, k_lo, k_hi, fast);
+    const float S = __fmul_rn(e4m3_value(code), s2);   // DQ1: RN32(s_b * s2)
+    w[0] = nv_encode8(y, S);
+    w[1] = nv_encode8(y + 8, S);
     return code;
 }
 
@@ -150,8 +153,12 @@ hadamard_quant_kernel(const uint16_t* x, uint32_t rows, uint32_t chunks_per_row,
                       double c, float* __restrict__ d_amax, uint8_t* __restrict__ q, uint8_t* __restrict__ sc,
                       float* __restrict__ d_s2, uint32_t* __restrict__ d_flags)
 {
-    // one lane = one 32-element chunk of a row (4 lanes = one 128-element segment)
+    // one lane = one 32-element chunk of a row; kG lanes = one segment of n elements
+    constexpr int kG = kN > 32 ? kN / 32 : 1;
+    constexpr int kPitch = 34;                                     // doubles per lane in the exchange buffer
+    __shared__ __align__(16) double xbuf[kG == 4 ? kHadThreads : 1][kPitch];
     const uint32_t lane = threadIdx.x & 31u;
+    const uint32_t t = lane & (uint32_t)(kG - 1);                  // this lane's place in its segment
     const uint32_t total = rows * chunks_per_row;                 // multiple of 4
     const uint32_t stride = gridDim.x * kHadThreads;
     uint32_t flags = 0u, mx_bits = 0u;
@@ -169,8 +176,8 @@ hadamard_quant_kernel(const uint16_t* x, uint32_t rows, uint32_t chunks_per_row,
     }
     const int64_t cols = (int64_t)chunks_per_row * 32;
 
-    // warp-uniform trip count (lanes of one 128-element segment exchange values); the
-    // next chunk's four loads are issued before the current chunk is transformed
+    // warp-uniform trip count (the lanes of a segment exchange values); the next chunk's
+    // four loads are issued before the current chunk is transformed
     auto load = [&](uint32_t ch, uint4 raw[4]) {
         const uint32_t rr = div_cpr.div(ch), c2 = ch - rr * chunks_per_row;
         const uint4* src = reinterpret_cast<const uint4*>(x + (int64_t)rr * ld + 32 * (int64_t)c2);
@@ -207,16 +214,84 @@ hadamard_quant_kernel(const uint16_t* x, uint32_t rows, uint32_t chunks_per_row,
 #pragma unroll
             for (int j = 0; j < 32; ++j) v[j] = 0.0;
         }
-        fwht32<kN>(v, lane);
+        fwht_lane<kN>(v);
+        if constexpr (kG == 2) {
+            // n = 64: the last stage pairs neighbouring lanes; the upper lane forms lower - upper
+            // as one FMA with a factor of -1 (a single rounding, like the subtraction)
+            const double sg = (lane & 1u) != 0u ? -1.0 : 1.0;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                const double o = __shfl_xor_sync(0xFFFFFFFFu, v[i], 1);
+                v[i] = fma(sg, v[i], o);
+            }
+        } else if constexpr (kG == 4) {
+            // n = 128: the two stages across the 4 lanes of a segment, through shared memory.
+            // Lane a of the segment holds z_a[0..31] (its chunk after the in-lane stages);
+            // afterwards lane t holds, for every a', the outputs a' * 32 + i of the segment for
+            // i = 8 t .. 8 t + 7, out[a'][ii] = sum over a of (-1)^popcount(a' & a) z_a[i], formed
+            // in the butterfly order of one stage per lane bit (lower + upper, lower - upper).
+            // A lane's 16 pairs go to positions (k % 4) * 4 + k / 4 of its row (a 272-byte
+            // pitch), so that the writes and the segment-wise reads each touch 32 distinct banks.
+            double* mine = &xbuf[threadIdx.x][0];
+#pragma unroll
+            for (int k = 0; k < 16; ++k)
+                *reinterpret_cast<double2*>(mine + 2 * ((k % 4) * 4 + k / 4)) = make_double2(v[2 * k], v[2 * k + 1]);
+            __syncwarp();
+            const double* grp = &xbuf[threadIdx.x & ~3u][0] + 2 * t;
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                    const double2 d2 = *reinterpret_cast<const double2*>(grp + a * kPitch + 8 * kk);
+                    v[8 * a + 2 * kk] = d2.x;
+                    v[8 * a + 2 * kk + 1] = d2.y;
+                }
+            __syncwarp();                                          // before the buffer is written again
+#pragma unroll
+            for (int h = 1; h < 4; h <<= 1)
+#pragma unroll
+                for (int a = 0; a < 4; ++a) {
+                    if (a & h) continue;
+#pragma unroll
+                    for (int ii = 0; ii < 8; ++ii) {
+                        const double lo = v[8 * a + ii], hi = v[8 * (a + h) + ii];
+                        v[8 * a + ii] = lo + hi;
+                        v[8 * (a + h) + ii] = lo - hi;
+                    }
+                }
+        }
+        float y[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) y[j] = (float)(v[j] * c);    // RN32(RN64(z * c))
+        if constexpr (kG == 4 && kMode != 0) {
+            // back to one chunk per lane for the quantizers (the maximum of mode 0 takes the
+            // values in any order), through shared memory as FP32: output chunk k (four
+            // values) of lane a' goes to 16-byte slot (k + 2 a') % 8 of a' 's 128-byte row, the
+            // segments 1088 bytes apart plus 16 for odd ones, so that both sides touch 32
+            // distinct banks
+            const uint32_t sw = lane >> 2;                         // the segment's place in its warp
+            float* segbuf = reinterpret_cast<float*>(&xbuf[threadIdx.x & ~31u][0]) + sw * 272u + 4u * (sw & 1u);
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const uint32_t k = 2u * t + (uint32_t)j;       // the chunk's place in row a
+                    *reinterpret_cast<float4*>(segbuf + 32 * a + 4 * ((k + 2u * a) & 7u)) =
+                        make_float4(y[8 * a + 4 * j], y[8 * a + 4 * j + 1], y[8 * a + 4 * j + 2], y[8 * a + 4 * j + 3]);
+                }
+            __syncwarp();
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const float4 f4 = *reinterpret_cast<const float4*>(segbuf + 32 * t + 4 * ((k + 2u * t) & 7u));
+                y[4 * k] = f4.x; y[4 * k + 1] = f4.y; y[4 * k + 2] = f4.z; y[4 * k + 3] = f4.w;
+            }
+            __syncwarp();                                          // before the next chunk's writes
+        }
         if (!live) continue;
 
-        float y[32];
         uint32_t ab = 0u;
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-            y[j] = (float)(v[j] * c);                              // RN32(RN64(z * c))
-            ab = max(ab, __float_as_uint(y[j]) & 0x7FFFFFFFu);
-        }
+        for (int j = 0; j < 32; ++j) ab = max(ab, __float_as_uint(y[j]) & 0x7FFFFFFFu);
         if (ab >= 0x7F800000u) flags |= kFlagNonFinite;
         const int64_t col = 32 * (int64_t)cc;
 
@@ -231,10 +306,8 @@ hadamard_quant_kernel(const uint16_t* x, uint32_t rows, uint32_t chunks_per_row,
         } else {
             uint32_t w[4], codes2 = 0u;
 #pragma unroll
-            for (int hb = 0; hb < 2; ++hb) {                       // two NVFP4 blocks of 16
-                const uint32_t code = nv_block16(y + 16 * hb, s2, k_lo, k_hi, fast_scale, w + 2 * hb);
-                codes2 |= code << (8 * hb);
-            }
+            for (int hb = 0; hb < 2; ++hb)                         // two NVFP4 blocks of 16
+                codes2 |= nv_block16(y + 16 * hb, s2, k_lo, k_hi, fast_scale, w + 2 * hb) << (8 * hb);
             __stcs(reinterpret_cast<uint4*>(q + (int64_t)r * (cols / 2) + col / 2), make_uint4(w[0], w[1], w[2], w[3]));
             *reinterpret_cast<uint16_t*>(sc + (int64_t)r * (cols / 16) + col / 16) = (uint16_t)codes2;
         }

@@ -170,6 +170,32 @@ def test_hadamard_quant_layer_shape(orc):
     assert np.array_equal(G.host(e8)[rows], re8) and np.array_equal(G.host(q)[rows], rq)
 
 
+@pytest.mark.filterwarnings("ignore:overflow encountered in cast")      # the oracle's RN32 of the overflowing sum
+@pytest.mark.parametrize("n", [16, 32, 64, 128])
+def test_hadamard_quant_nonfinite_overflow_tiny(orc, n):
+    """A NaN and an Inf input (every output of their block turns non-finite), a block of
+    BF16 values near the top of the range whose rotated sum overflows FP32, and a row of
+    BF16 subnormals: MXFP4 codes and scales (0xFF for non-finite blocks) and the non-finite
+    flag as the oracle gives them, and the amax pass skipping NaN but keeping Inf."""
+    x = inputs.laplace_bf16(inputs.rng_for(n, "gpu", "had_nf"), 6, 512, outlier_channels=(9,), outlier_scale=30)
+    x[1, 7] = 0x7FC0                                             # NaN
+    x[2, 300] = 0x7F80                                           # +Inf
+    x[3, 0:128] = 0x7F61                                         # ~3.0e38: the block's first sum overflows
+    x[4, :] = inputs.f32_to_bf16_bits((np.arange(512) % 97 - 48).astype(np.float32) * np.float32(2.0 ** -133))
+    x[5, 256:384] = 0                                            # an all-zero block
+    xd = G.bf16_dev(x)
+    y = orc.hadamard_rotate(x, n)
+    f = G.flags_dev()
+    q, e8 = nv4.hadamard_mxfp4_quant(xd, n, d_flags=f)
+    rq, re8, rf = orc.mxfp4_quant(y)
+    torch.cuda.synchronize()
+    assert np.array_equal(G.host(e8), re8) and np.array_equal(G.host(q), rq)
+    assert (re8 == 0xFF).any() and f.item() == rf
+    amax = torch.zeros(1, dtype=torch.float32, device=G.DEV)
+    nv4.nv4_hadamard_amax(xd, n, amax)
+    assert amax.item() == float(np.nanmax(np.abs(y)))
+
+
 # ---------------------------------------------------------------- two-sided block Hadamard of weight tiles
 def _w_dev(w):
     return G.f32_dev(w) if w.dtype == np.float32 else G.bf16_dev(w)

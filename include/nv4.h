@@ -412,7 +412,7 @@ NV4_API nv4_status nv4_fp8_dequant(const uint8_t* q, const float* d_scale, int64
  * nv4_hadamard_mxfp4_quant -- MXFP4 codes and E8M0 scales of y, as nv4_mxfp4_quant.
  * nv4_hadamard_nvfp4_quant -- NVFP4 codes and E4M3 scales of y with s2 = RN32(amax / 2688)
  *                             from *d_amax (e.g. from nv4_hadamard_amax), as nv4_act_quant.
- * Limits: fewer than 2^31 128-element row segments per call.
+ * Limits: fewer than 2^31 32-element row chunks per call (NV4_ERR_LIMIT).
  */
 NV4_API nv4_status nv4_hadamard_amax(const void* x, int64_t rows, int64_t cols, int64_t ld, int n,
                              float* d_amax, uint32_t* d_flags, void* stream);

@@ -574,7 +574,7 @@ static nv4_status check_hadamard(const void* x, int64_t rows, int64_t cols, int6
     if (rows == 0 || cols == 0) return NV4_OK;
     if (x == nullptr) return NV4_ERR_NULL;
     if (!aligned16(x) || ld % 8 != 0) return NV4_ERR_ALIGN;
-    if (rows * (cols / 128) >= (int64_t)1 << 31) return NV4_ERR_LIMIT;
+    if (rows * (cols / 32) >= (int64_t)1 << 31) return NV4_ERR_LIMIT;      // the kernel's 32-element chunk count
     return NV4_OK;
 }
 

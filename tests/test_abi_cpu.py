@@ -113,6 +113,7 @@ def test_validation_rejects_before_any_launch(nv4lib):
     assert L.nv4_hadamard_mxfp4_quant(fake, 4, 128, 132, 32, fake, fake, None, None) == 3   # ld % 8
     assert L.nv4_hadamard_amax(fake, 4, 128, 128, 64, None, None, None) == 1
     assert L.nv4_hadamard_nvfp4_quant(fake, 4, 128, 128, 128, fake, None, fake, fake, None, None) == 1
+    assert L.nv4_hadamard_mxfp4_quant(fake, 1 << 26, 1024, 1024, 128, fake, fake, None, None) == 6  # 2^31 chunks
     # two-sided block Hadamard of weight tiles: n, tile and strip shapes, dtype, alignment, nulls
     assert L.nv4_hadamard2_rotate(fake, 0, 32, 64, 64, 64, fake, None, None) == 2          # n not 16 or 32
     assert L.nv4_hadamard2_rotate(fake, 0, 40, 64, 64, 32, fake, None, None) == 2          # rows % n

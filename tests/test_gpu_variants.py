@@ -161,6 +161,32 @@ def test_hadamard_quant_matches_oracle(orc, n):
     assert np.array_equal(G.host(sc), nsc) and np.array_equal(G.host(q), nq)
 
 
+@pytest.mark.parametrize("n", [16, 32, 64, 128])
+@pytest.mark.parametrize("pad", [8, 64])
+def test_hadamard_quant_strided_rows(orc, n, pad):
+    """Rows inside a wider buffer (row pitch cols + pad), 37 rows so that the last warp of
+    segments is only partly live: amax, MXFP4 and NVFP4 of the rotated rows as the oracle
+    gives them, and the padding columns never read into the result."""
+    rows, cols = 37, 384
+    xc = inputs.laplace_bf16(inputs.rng_for(n + pad, "gpu", "had_ld"), rows, cols, outlier_channels=(5, 300),
+                             outlier_scale=40, zero_block_frac=0.02)
+    x = np.full((rows, cols + pad), 0x7FC0, np.uint16)           # NaN padding: must stay out of every result
+    x[:, :cols] = xc
+    xd = G.bf16_dev(x)[:, :cols]
+    y = orc.hadamard_rotate(xc, n)
+    f = G.flags_dev()
+    amax = torch.zeros(1, dtype=torch.float32, device=G.DEV)
+    nv4.nv4_hadamard_amax(xd, n, amax, f)
+    q, e8 = nv4.hadamard_mxfp4_quant(xd, n, d_flags=f)
+    qn, sc, s2, _ = nv4.hadamard_nvfp4_quant(xd, n, d_flags=f)
+    rq, re8, _ = orc.mxfp4_quant(y)
+    nq, nsc, ns2, _ = orc.rtn_quant(y, float(np.abs(y).max()))
+    torch.cuda.synchronize()
+    assert f.item() == 0 and amax.item() == float(np.abs(y).max())
+    assert np.array_equal(G.host(e8), re8) and np.array_equal(G.host(q), rq)
+    assert s2.item() == ns2 and np.array_equal(G.host(sc), nsc) and np.array_equal(G.host(qn), nq)
+
+
 def test_hadamard_quant_layer_shape(orc):
     x = inputs.c2_shape(4096, 7168)
     rows = np.sort(np.random.default_rng(1).choice(4096, 64, replace=False))

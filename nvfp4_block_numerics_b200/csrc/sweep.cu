@@ -12,8 +12,11 @@
 // Per visited candidate, per thread (all FP32; pairs use the packed FP32 instructions),
 // in two halves of 8 elements -- the second half only when the first half's part of
 // bound (1) below does not already rule the candidate out:
-//   E2M1 codes of w/S_c : bracketed hardware conversion; near a rounding boundary
-//                         one exact FMA comparison fixes the code (nv4_common.cuh)
+//   E2M1 codes of w/S_c : for bound (1), the hardware conversion of the lower end of the
+//                         bracket alone; for a candidate the bound leaves open, the exact
+//                         codes (both ends converted, near a rounding boundary one exact FMA
+//                         comparison fixes the code, nv4_common.cuh) and e again where they
+//                         differ
 //   e_i = w_i - v_i*S_c   (one rounding of the exact difference)
 //   cost = sum_i e_i (H_ii e_i + sum_{j>i} (H_ij + H_ji) e_j), evaluated two rows at
 //          a time: 136 + 16 multiply-adds in 80 packed instructions
@@ -39,8 +42,9 @@
 // the two largest |w_i| exceeds it, the downward walk ends; once bound (3) exceeds it,
 // the upward walk ends (long upward walks: weights whose block amax is far below the
 // tensor's, such as heavy-tailed expert weights).  The comparisons
-// keep a relative margin of 2^-10, far above the FP32 evaluation error, so skipped
-// candidates could not have changed the FP32 result either.  When mu < 1/32, or eta_b
+// keep a relative margin of 2^-10, far above the FP32 evaluation error and the 2^-15 by
+// which bound (1) from the lower-end codes can exceed the bound from the exact codes, so
+// skipped candidates could not have changed the FP32 result either.  When mu < 1/32, or eta_b
 // (below) exceeds 2^-12, or H_b has a zero diagonal entry with a nonzero row, or
 // non-finite entries, the bounds are off and all 127 candidates are evaluated, in FP64.
 //
@@ -279,6 +283,45 @@ __device__ __forceinline__ void codes8h(const float2 w[4], const float4& t, uint
     }
     c = 0u;
     for (int i = 0; i < 8; ++i) c |= e2m1_code_exact(i & 1 ? w[i >> 1].y : w[i >> 1].x, t.x) << (4 * i);
+}
+
+// E2M1 codes of 8 weights from the lower end of the bracket alone.  They differ from the
+// exact codes only where w/S_c lies within the bracket's relative width (2^-20) above a
+// rounding midpoint m, and there the other neighbour is as far from w to within a relative
+// 2 m 2^-20 / (half the grid spacing at m) <= 14 * 2^-20 < 2^-16: bound (1) from these codes
+// exceeds the one from the exact codes by less than 2^-15 relative, far inside the pruning
+// margin.
+__device__ __forceinline__ uint32_t codes8h_lo(const float2 w[4], const float4& t)
+{
+    const float2 rl = make_float2(t.y, t.y);
+    float lo[8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const float2 a = __fmul2_rn(w[j], rl);
+        lo[2 * j] = a.x; lo[2 * j + 1] = a.y;
+    }
+    return cvt_e2m1x8(lo);
+}
+
+// The exact codes given the lower-end codes c (t.w == 0): the upper end converted, the
+// exact FP32 fix-up where the two ends disagree.
+__device__ __forceinline__ uint32_t codes8h_exact_from(const float2 w[4], const float4& t, uint32_t c)
+{
+    const float2 rh = make_float2(t.z, t.z);
+    float hi[8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const float2 b = __fmul2_rn(w[j], rh);
+        hi[2 * j] = b.x; hi[2 * j + 1] = b.y;
+    }
+    const uint32_t h = cvt_e2m1x8(hi);
+    if (c != h) {
+        float x[8];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) { x[2 * j] = w[j].x; x[2 * j + 1] = w[j].y; }
+        c = e2m1_fix8(x, t.x, c, h);
+    }
+    return c;
 }
 
 // Signed E2M1 values of 8 packed codes, as 4 pairs.
@@ -616,9 +659,11 @@ sweep_kernel(const __grid_constant__ SweepParams p)
                 const float4 t = tab[c];
                 const float2 nS = make_float2(-t.x, -t.x);
                 float2 e[8];
-                // first half (elements 0..7): codes, e and its part of bound (1)
+                // first half (elements 0..7): codes, e and its part of bound (1); the bound
+                // takes the lower-end codes, the quadratic form the exact ones
+                const bool exact_t = t.w != 0.0f;
                 uint32_t c0, c1 = 0u;
-                codes8h(w, t, c0);
+                if (exact_t) codes8h(w, t, c0); else c0 = codes8h_lo(w, t);
                 {
                     float2 v[4];
                     decode8h(c0, v);
@@ -629,7 +674,7 @@ sweep_kernel(const __grid_constant__ SweepParams p)
                 ++nhalf;
                 if (!pr || !(lb * kPruneScale > thr)) {               // the second half is still needed
                     ++nhalf;
-                    codes8h(w + 4, t, c1);
+                    if (exact_t) codes8h(w + 4, t, c1); else c1 = codes8h_lo(w + 4, t);
                     {
                         float2 v[4];
                         decode8h(c1, v);
@@ -638,6 +683,22 @@ sweep_kernel(const __grid_constant__ SweepParams p)
                     }
                     lb += bound_half(e + 4, rd4 + 2);
                     if (!pr || !(lb * kPruneScale > thr)) {
+                        if (!exact_t) {                                 // exact codes, e where they differ
+                            const uint32_t x0 = codes8h_exact_from(w, t, c0);
+                            const uint32_t x1 = codes8h_exact_from(w + 4, t, c1);
+                            if (x0 != c0) {
+                                float2 v[4];
+                                decode8h(x0, v);
+#pragma unroll
+                                for (int k = 0; k < 4; ++k) e[k] = __ffma2_rn(v[k], nS, w[k]);
+                            }
+                            if (x1 != c1) {
+                                float2 v[4];
+                                decode8h(x1, v);
+#pragma unroll
+                                for (int k = 0; k < 4; ++k) e[4 + k] = __ffma2_rn(v[k], nS, w[4 + k]);
+                            }
+                        }
                         ++nfull;
                         const float cost = quad_form(e, hp);
                         if (cost < best || (cost == best && (uint32_t)c < best_c)) {
